@@ -1,0 +1,171 @@
+"""fp64 CPU oracle for the batch-invariant forward path (TEST INFRASTRUCTURE).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path never does.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64); this module compiles it
+with gcc (OpenMP over independent rows) and marshals numpy arrays into it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
+    """Compile ``oracle.c`` (or another copy of it) into a shared library
+    with gcc -O2 -fopenmp."""
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + ".tmp%d" % os.getpid()
+        # -ffp-contract=off: no fused multiply-add, so every product and sum
+        # rounds exactly as written in the source.
+        cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+               "-shared", "-fPIC", src, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, out)
+    return out
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, "bfloat16 inputs are passed as uint16 bit patterns"
+    return a
+
+
+class Oracle:
+    """The oracle's entry points, bound to one build of ``oracle.c``."""
+
+    def __init__(self, path: str):
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i64, i32, f64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+        lib.oracle_rmsnorm.argtypes = [P, P, i64, i64, f64, P]
+        lib.oracle_matmul.argtypes = [P, P, i64, i64, i64, P]
+        lib.oracle_kv_write.argtypes = [P, P, i32, i32, P, P, P, i64]
+        lib.oracle_attention.argtypes = [P, i64, i32, P, P, P, i32, P, P, i32, P, i32, f64, P, P]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        self.lib = lib
+
+    def num_threads(self) -> int:
+        return int(self.lib.oracle_num_threads())
+
+    def set_num_threads(self, n: int) -> None:
+        self.lib.oracle_set_num_threads(int(n))
+
+    def rmsnorm(self, x, w, eps: float) -> np.ndarray:
+        """y = x / sqrt(mean(x^2) + eps) * w per row; x [M, H], w [H] (bf16 bits)."""
+        x, w = _u16(x), _u16(w)
+        M, H = x.shape
+        y = np.empty((M, H), dtype=np.float64)
+        self.lib.oracle_rmsnorm(_p(x), _p(w), M, H, float(eps), _p(y))
+        return y
+
+    def matmul(self, a, w) -> np.ndarray:
+        """C = A @ W.T; a [M, K], w [N, K] (bf16 bits) -> C [M, N] float64."""
+        a, w = _u16(a), _u16(w)
+        M, K = a.shape
+        N, K2 = w.shape
+        assert K == K2
+        c = np.empty((M, N), dtype=np.float64)
+        self.lib.oracle_matmul(_p(a), _p(w), M, N, K, _p(c))
+        return c
+
+    def kv_write(self, k_cache, v_cache, k_new, v_new, slots) -> None:
+        """Scatter new tokens into the paged cache in place (bit copy)."""
+        k_cache, v_cache = _u16(k_cache), _u16(v_cache)
+        k_new, v_new = _u16(k_new), _u16(v_new)
+        slots = np.ascontiguousarray(slots, dtype=np.int64)
+        _, Hkv, page, d = k_cache.shape
+        assert page == 16
+        T = k_new.shape[0]
+        self.lib.oracle_kv_write(_p(k_cache), _p(v_cache), Hkv, d, _p(k_new), _p(v_new),
+                                 _p(slots), T)
+
+    def attention(self, q_rows, row_seq, row_head, row_pos, Hq: int, k_cache, v_cache,
+                  block_table, scale: float | None = None, want_lse: bool = False):
+        """Causal softmax attention of query rows over a paged cache.
+
+        ``q_rows`` [R, d] bf16 bits; row r is head ``row_head[r]`` of sequence
+        ``row_seq[r]`` at absolute position ``row_pos[r]`` (it sees keys
+        ``0..row_pos[r]``).  Returns ``o`` [R, d] float64 (and ``lse`` [R]).
+        """
+        q_rows = _u16(q_rows)
+        k_cache, v_cache = _u16(k_cache), _u16(v_cache)
+        R, d = q_rows.shape
+        _, Hkv, page, d2 = k_cache.shape
+        assert page == 16 and d2 == d and Hq % Hkv == 0
+        bt = np.ascontiguousarray(block_table, dtype=np.int32)
+        rs = np.ascontiguousarray(row_seq, dtype=np.int32)
+        rh = np.ascontiguousarray(row_head, dtype=np.int32)
+        rp = np.ascontiguousarray(row_pos, dtype=np.int32)
+        assert rs.shape == rh.shape == rp.shape == (R,)
+        if scale is None:
+            scale = 1.0 / np.sqrt(d)
+        o = np.empty((R, d), dtype=np.float64)
+        lse = np.empty((R,), dtype=np.float64)
+        self.lib.oracle_attention(_p(q_rows), R, d, _p(rs), _p(rh), _p(rp), Hq, _p(k_cache),
+                                  _p(v_cache), Hkv, _p(bt), bt.shape[1], float(scale), _p(o),
+                                  _p(lse))
+        return (o, lse) if want_lse else o
+
+
+def default() -> Oracle:
+    global _lib
+    if _lib is None:
+        _lib = Oracle(build())
+    return _lib
+
+
+def num_threads() -> int:
+    return default().num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    default().set_num_threads(n)
+
+
+def rmsnorm(x, w, eps: float) -> np.ndarray:
+    return default().rmsnorm(x, w, eps)
+
+
+def matmul(a, w) -> np.ndarray:
+    return default().matmul(a, w)
+
+
+def kv_write(k_cache, v_cache, k_new, v_new, slots) -> None:
+    default().kv_write(k_cache, v_cache, k_new, v_new, slots)
+
+
+def attention(q_rows, row_seq, row_head, row_pos, Hq: int, k_cache, v_cache, block_table,
+              scale: float | None = None, want_lse: bool = False):
+    return default().attention(q_rows, row_seq, row_head, row_pos, Hq, k_cache, v_cache,
+                               block_table, scale=scale, want_lse=want_lse)
+
+
+def decode_rows(q, seq_lens, heads=None):
+    """Rows for a decode step: every head of every request at position L-1.
+    ``q`` [B, Hq, d].  Returns (q_rows, row_seq, row_head, row_pos)."""
+    B, Hq, d = q.shape
+    heads = range(Hq) if heads is None else heads
+    heads = list(heads)
+    rs, rh, rp, rows = [], [], [], []
+    for b in range(B):
+        for h in heads:
+            rs.append(b)
+            rh.append(h)
+            rp.append(int(seq_lens[b]) - 1)
+            rows.append(q[b, h])
+    return np.stack(rows), np.array(rs), np.array(rh), np.array(rp)

@@ -1,0 +1,197 @@
+/*
+ * oracle.c -- plain fp64 CPU reference for the batch-invariant forward path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the package smoke check and the
+ * bench's CPU-baseline leg may load this library.  It shares no code, header
+ * or table with the CUDA library; the two meet only through the seeded input
+ * generators.
+ *
+ * The reports on "Defeating Nondeterminism in LLM Inference" name the three
+ * operations whose batch-invariant versions make up the path -- RMSNorm,
+ * matrix multiplication and attention (xitu-tech news, "构建确定性解决方案";
+ * neican.ai insight, "技术原理与创新点解析") -- but print no formula for any of
+ * them.  Each result the invariant kernels reach has a plain mathematical
+ * definition (the kernels only fix the order of the floating-point
+ * operations), so every function below is that definition written out in
+ * double precision, in the most direct loop order, with no blocking, no
+ * splitting of reductions and no reordering.
+ *
+ * Inputs are bfloat16 bit patterns (uint16_t), widened exactly to double.
+ * Outputs are double.
+ *
+ * Readings of points the pages leave open (each listed in the design notes):
+ *   - RMSNorm: y = x / sqrt(mean(x^2) + eps) * w, eps inside the root, plain
+ *     weight (not 1 + w).
+ *   - Matmul: C = A * W^T with W stored [N, K] (output-feature-major).
+ *   - Attention: softmax(q.k * scale) over the keys a query may see,
+ *     key j visible to the query at absolute position t iff j <= t;
+ *     query head h reads kv head floor(h / (Hq / Hkv)); the paged cache is
+ *     [num_pages, Hkv, 16, d] with the page of token j of sequence b being
+ *     block_table[b][j / 16] and its slot j % 16.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_PAGE 16
+
+static double bf16_to_double(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/*
+ * RMSNorm of each row (xitu-tech news, "构建确定性解决方案", RMSNorm item;
+ * neican.ai insight, "技术原理与创新点解析", batch-invariant RMSNorm bullet):
+ *   y[r, j] = x[r, j] / sqrt( (1/H) * sum_i x[r, i]^2 + eps ) * w[j]
+ */
+void oracle_rmsnorm(const uint16_t *x, const uint16_t *w, int64_t M, int64_t H,
+                    double eps, double *y)
+{
+    int64_t r;
+#pragma omp parallel for schedule(static)
+    for (r = 0; r < M; ++r) {
+        const uint16_t *xr = x + r * H;
+        double ss = 0.0;
+        for (int64_t i = 0; i < H; ++i) {
+            double v = bf16_to_double(xr[i]);
+            ss += v * v;
+        }
+        double denom = sqrt(ss / (double)H + eps);
+        for (int64_t j = 0; j < H; ++j)
+            y[r * H + j] = bf16_to_double(xr[j]) / denom * bf16_to_double(w[j]);
+    }
+}
+
+/*
+ * Matrix product (xitu-tech news, "构建确定性解决方案", matmul item;
+ * neican.ai insight, "技术原理与创新点解析", batch-invariant matmul bullet):
+ *   C[m, n] = sum_k A[m, k] * W[n, k]        A: [M, K], W: [N, K], C: [M, N]
+ */
+void oracle_matmul(const uint16_t *a, const uint16_t *w, int64_t M, int64_t N, int64_t K,
+                   double *c)
+{
+    int64_t m;
+#pragma omp parallel for schedule(static)
+    for (m = 0; m < M; ++m) {
+        const uint16_t *am = a + m * K;
+        for (int64_t n = 0; n < N; ++n) {
+            const uint16_t *wn = w + n * K;
+            double s = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                s += bf16_to_double(am[k]) * bf16_to_double(wn[k]);
+            c[m * N + n] = s;
+        }
+    }
+}
+
+/*
+ * Write new tokens' keys and values into the paged cache before attention
+ * runs (neican.ai insight, "技术原理与创新点解析", batch-invariant attention
+ * bullet: the KV-cache page table is updated before the kernel launches).
+ *   cache[slot / 16][g][slot % 16][:] = new[t][g][:]   for slot = slots[t] >= 0
+ * Bit copy; slots < 0 are skipped.
+ */
+void oracle_kv_write(uint16_t *k_cache, uint16_t *v_cache, int32_t Hkv, int32_t d,
+                     const uint16_t *k_new, const uint16_t *v_new, const int64_t *slots,
+                     int64_t T)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        int64_t slot = slots[t];
+        if (slot < 0) continue;
+        int64_t page = slot / ORACLE_PAGE, off = slot % ORACLE_PAGE;
+        for (int32_t g = 0; g < Hkv; ++g) {
+            int64_t dst = ((page * Hkv + g) * ORACLE_PAGE + off) * d;
+            int64_t src = (t * Hkv + g) * (int64_t)d;
+            memcpy(k_cache + dst, k_new + src, (size_t)d * sizeof(uint16_t));
+            memcpy(v_cache + dst, v_new + src, (size_t)d * sizeof(uint16_t));
+        }
+    }
+}
+
+/*
+ * Causal softmax attention of single query rows over a paged KV cache
+ * (neican.ai insight, "技术原理与创新点解析", batch-invariant attention bullet;
+ * liuwei.blog, "破解之道", the attention example: parallel over queries,
+ * reduce over keys and values).
+ *
+ * Row r is query head row_head[r] of sequence row_seq[r] at absolute position
+ * row_pos[r] = t.  With g = floor(h / (Hq / Hkv)):
+ *   s_j   = scale * sum_i q[r, i] * K_b[j, g, i]          j = 0 .. t
+ *   p_j   = exp(s_j - max_j s_j) / sum_j exp(s_j - max_j s_j)
+ *   o[r]  = sum_j p_j * V_b[j, g, :]
+ *   lse[r] = max_j s_j + log(sum_j exp(s_j - max_j s_j))
+ * where K_b[j] is read from page block_table[b][j / 16], slot j % 16.
+ * The sequence is never split: the whole key range is reduced in one pass.
+ * lse may be NULL.
+ */
+void oracle_attention(const uint16_t *q, int64_t R, int32_t d,
+                      const int32_t *row_seq, const int32_t *row_head, const int32_t *row_pos,
+                      int32_t Hq, const uint16_t *k_cache, const uint16_t *v_cache,
+                      int32_t Hkv, const int32_t *block_table, int32_t max_pages,
+                      double scale, double *o, double *lse)
+{
+    int32_t group = Hq / Hkv;
+    int64_t r;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (r = 0; r < R; ++r) {
+        int32_t b = row_seq[r], h = row_head[r], t = row_pos[r];
+        int32_t g = h / group;
+        const uint16_t *qr = q + r * d;
+        int64_t n = (int64_t)t + 1;
+        double mx = -INFINITY;
+        /* first pass: the logits and their maximum */
+        for (int64_t j = 0; j < n; ++j) {
+            int64_t page = block_table[(int64_t)b * max_pages + j / ORACLE_PAGE];
+            const uint16_t *kj = k_cache + ((page * Hkv + g) * ORACLE_PAGE + j % ORACLE_PAGE) * d;
+            double s = 0.0;
+            for (int32_t i = 0; i < d; ++i)
+                s += bf16_to_double(qr[i]) * bf16_to_double(kj[i]);
+            s *= scale;
+            if (s > mx) mx = s;
+        }
+        /* second pass: exponentials, their sum, and the weighted values */
+        double *orow = o + r * d;
+        for (int32_t i = 0; i < d; ++i) orow[i] = 0.0;
+        double l = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+            int64_t page = block_table[(int64_t)b * max_pages + j / ORACLE_PAGE];
+            int64_t base = ((page * Hkv + g) * ORACLE_PAGE + j % ORACLE_PAGE) * d;
+            const uint16_t *kj = k_cache + base;
+            const uint16_t *vj = v_cache + base;
+            double s = 0.0;
+            for (int32_t i = 0; i < d; ++i)
+                s += bf16_to_double(qr[i]) * bf16_to_double(kj[i]);
+            double p = exp(s * scale - mx);
+            l += p;
+            for (int32_t i = 0; i < d; ++i)
+                orow[i] += p * bf16_to_double(vj[i]);
+        }
+        for (int32_t i = 0; i < d; ++i) orow[i] /= l;
+        if (lse) lse[r] = mx + log(l);
+    }
+}

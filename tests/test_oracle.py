@@ -1,0 +1,318 @@
+"""Pins for the fp64 oracle: closed forms, brute force on tiny inputs and
+independent library routines.  No GPU; each pin is chosen so that a plausible
+slip in the oracle (a dropped term, a wrong index, a transposed operand, a
+misplaced eps, a wrong head mapping, a causal off-by-one) fails it."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as _oracle_mod
+from synth import (bf16_bits_to_f32, f32_to_bf16_bits, normal_bf16, page_table, paged_kv, rng,
+                   slot_mapping, uniform_bf16)
+
+
+@pytest.fixture
+def oracle():
+    return _oracle_mod.default()
+
+
+def bf(vals):
+    return f32_to_bf16_bits(np.asarray(vals, dtype=np.float32))
+
+
+def widen(bits):
+    return bf16_bits_to_f32(bits).astype(np.float64)
+
+
+# ---------------------------------------------------------------- RMSNorm
+
+
+@pytest.mark.parametrize("c", [1.0, -2.5, 0.001, 96.0])
+def test_rmsnorm_constant_row_closed_form(oracle, c):
+    # x = c * 1  =>  mean(x^2) = c^2  =>  y = c / sqrt(c^2 + eps) * w
+    H, eps = 64, 1e-6
+    g = rng(11)
+    w = uniform_bf16(g, (H,), 0.5, 1.5)
+    x = np.tile(bf([c] * H), (2, 1))
+    y = oracle.rmsnorm(x, w, eps)
+    cc = float(widen(bf([c]))[0])
+    want = cc / math.sqrt(cc * cc + eps) * widen(w)
+    np.testing.assert_allclose(y[0], want, rtol=1e-14, atol=0)
+    np.testing.assert_allclose(y[1], want, rtol=1e-14, atol=0)
+
+
+def test_rmsnorm_alternating_sign_closed_form(oracle):
+    H, eps, c = 32, 1e-6, 1.5
+    x = bf([c if i % 2 == 0 else -c for i in range(H)])[None, :]
+    w = bf(np.ones(H))
+    y = oracle.rmsnorm(x, w, eps)[0]
+    mag = c / math.sqrt(c * c + eps)
+    want = np.array([mag if i % 2 == 0 else -mag for i in range(H)])
+    np.testing.assert_allclose(y, want, rtol=1e-14)
+
+
+def test_rmsnorm_hand_example(oracle):
+    # x = [1, 2, 3, 4]: mean square (1+4+9+16)/4 = 7.5; eps = 0
+    x = bf([1, 2, 3, 4])[None, :]
+    w = bf([1, 0.5, 2, 1])
+    y = oracle.rmsnorm(x, w, 0.0)[0]
+    r = 1.0 / math.sqrt(7.5)
+    np.testing.assert_allclose(y, [1 * r, 2 * r * 0.5, 3 * r * 2, 4 * r], rtol=1e-15)
+
+
+def test_rmsnorm_eps_inside_the_root(oracle):
+    # c = 1e-3: c^2 = 1e-6 = eps, so y = c / sqrt(2e-6) = 1/sqrt(2) (eps inside)
+    # whereas eps outside the root would give c / (c + eps) ~ 0.999.
+    c = float(widen(bf([1e-3]))[0])
+    x = bf([1e-3] * 8)[None, :]
+    y = oracle.rmsnorm(x, bf(np.ones(8)), 1e-6)[0]
+    np.testing.assert_allclose(y, c / math.sqrt(c * c + 1e-6), rtol=1e-14)
+    assert abs(y[0] - 1 / math.sqrt(2)) < 0.01
+
+
+def test_rmsnorm_matches_torch_fp64(oracle):
+    g = rng(12)
+    x = normal_bf16(g, (5, 96))
+    w = uniform_bf16(g, (96,), 0.5, 1.5)
+    y = oracle.rmsnorm(x, w, 1e-6)
+    xt = torch.from_numpy(widen(x))
+    want = torch.nn.functional.rms_norm(xt, (96,), weight=torch.from_numpy(widen(w)), eps=1e-6)
+    np.testing.assert_allclose(y, want.numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_rmsnorm_scale_invariance_without_eps(oracle):
+    g = rng(13)
+    x = normal_bf16(g, (3, 40))
+    x2 = bf(widen(x) * 4.0)  # exact: scaling by a power of two
+    w = uniform_bf16(g, (40,), 0.5, 1.5)
+    np.testing.assert_allclose(oracle.rmsnorm(x, w, 0.0), oracle.rmsnorm(x2, w, 0.0), rtol=1e-14)
+
+
+def test_rmsnorm_rows_independent(oracle):
+    g = rng(14)
+    x = normal_bf16(g, (6, 24))
+    w = uniform_bf16(g, (24,), 0.5, 1.5)
+    full = oracle.rmsnorm(x, w, 1e-6)
+    for r in range(6):
+        np.testing.assert_array_equal(oracle.rmsnorm(x[r:r + 1], w, 1e-6)[0], full[r])
+
+
+# ---------------------------------------------------------------- matmul
+
+
+def test_matmul_identity_weight(oracle):
+    g = rng(20)
+    a = normal_bf16(g, (7, 16))
+    eye = bf(np.eye(16))
+    np.testing.assert_array_equal(oracle.matmul(a, eye), widen(a))
+
+
+def test_matmul_one_hot_rows_select_columns(oracle):
+    g = rng(21)
+    a = normal_bf16(g, (4, 12))
+    pick = [3, 0, 11, 5, 5]
+    w = np.zeros((5, 12), dtype=np.float32)
+    for n, k in enumerate(pick):
+        w[n, k] = 1.0
+    c = oracle.matmul(a, bf(w))
+    np.testing.assert_array_equal(c, widen(a)[:, pick])
+
+
+def test_matmul_small_integers_brute_force(oracle):
+    # M=3, N=5, K=7: distinct sizes so a transposed operand cannot pass.
+    g = rng(22)
+    A = g.integers(-8, 9, size=(3, 7))
+    W = g.integers(-8, 9, size=(5, 7))
+    c = oracle.matmul(bf(A), bf(W))
+    for m in range(3):
+        for n in range(5):
+            assert c[m, n] == sum(int(A[m, k]) * int(W[n, k]) for k in range(7))
+
+
+def test_matmul_hand_example(oracle):
+    # [[1, 2, 3], [4, 5, 6]] times the transpose of [[1, 0, -1], [2, 1, 0]]
+    c = oracle.matmul(bf([[1, 2, 3], [4, 5, 6]]), bf([[1, 0, -1], [2, 1, 0]]))
+    np.testing.assert_array_equal(c, [[1 - 3, 2 + 2], [4 - 6, 8 + 5]])
+
+
+def test_matmul_matches_torch_fp64(oracle):
+    g = rng(23)
+    a = normal_bf16(g, (9, 130))
+    w = normal_bf16(g, (33, 130), std=0.02)
+    want = torch.from_numpy(widen(a)) @ torch.from_numpy(widen(w)).T
+    np.testing.assert_allclose(oracle.matmul(a, w), want.numpy(), rtol=1e-12, atol=1e-15)
+
+
+# ---------------------------------------------------------------- kv_write
+
+
+def test_kv_write_matches_direct_scatter(oracle):
+    g = rng(30)
+    Hkv, d = 2, 8
+    bt, num_pages = page_table(g, [37, 5], extra_pages=3)
+    kc = normal_bf16(g, (num_pages, Hkv, 16, d))
+    vc = normal_bf16(g, (num_pages, Hkv, 16, d))
+    kn = normal_bf16(g, (6, Hkv, d))
+    vn = normal_bf16(g, (6, Hkv, d))
+    slots = np.concatenate([slot_mapping(bt, 0, [0, 17, 36]), [-1], slot_mapping(bt, 1, [2, 4])])
+    k2, v2 = kc.copy(), vc.copy()
+    oracle.kv_write(k2, v2, kn, vn, slots)
+    kw, vw = kc.copy(), vc.copy()
+    for t, s in enumerate(slots):
+        if s >= 0:
+            kw[s // 16, :, s % 16, :] = kn[t]
+            vw[s // 16, :, s % 16, :] = vn[t]
+    np.testing.assert_array_equal(k2, kw)
+    np.testing.assert_array_equal(v2, vw)
+    assert not np.array_equal(k2, kc)
+
+
+# ---------------------------------------------------------------- attention
+
+
+def _contig_cache(K, V):
+    """Place logical K/V [L, Hkv, d] on pages 0, 1, 2, ... in order."""
+    L, Hkv, d = K.shape
+    n = (L + 15) // 16
+    kc = np.zeros((n, Hkv, 16, d), dtype=np.uint16)
+    vc = np.zeros_like(kc)
+    for j in range(L):
+        kc[j // 16, :, j % 16] = K[j]
+        vc[j // 16, :, j % 16] = V[j]
+    return kc, vc, np.arange(n, dtype=np.int32)[None, :]
+
+
+def test_attention_identical_keys_give_prefix_mean(oracle):
+    # Every key equal => uniform softmax over keys 0..t => o = mean(V[0..t]).
+    g = rng(40)
+    L, Hkv, d = 40, 1, 8
+    k0 = normal_bf16(g, (d,))
+    K = np.tile(k0, (L, Hkv, 1))
+    V = normal_bf16(g, (L, Hkv, d))
+    kc, vc, bt = _contig_cache(K, V)
+    q = normal_bf16(g, (L, d))
+    pos = np.arange(L)
+    o, lse = oracle.attention(q, np.zeros(L), np.zeros(L), pos, 1, kc, vc, bt, want_lse=True)
+    Vw = widen(V)[:, 0, :]
+    for t in range(L):
+        np.testing.assert_allclose(o[t], Vw[: t + 1].mean(axis=0), rtol=1e-12, atol=1e-14)
+        s = float(widen(q[t]) @ widen(k0)) / math.sqrt(d)
+        assert abs(lse[t] - (s + math.log(t + 1))) < 1e-12
+
+
+def test_attention_single_key_returns_value_row(oracle):
+    g = rng(41)
+    kv = paged_kv(g, [1, 1, 1], num_kv_heads=2, head_dim=16)
+    q = normal_bf16(g, (3, 4, 16))
+    rows = _oracle_mod.decode_rows(q, kv.seq_lens)
+    o = oracle.attention(*rows, 4, kv.k_cache, kv.v_cache, kv.block_table)
+    for i, (b, h) in enumerate(zip(rows[1], rows[2])):
+        page = kv.block_table[b, 0]
+        np.testing.assert_array_equal(o[i], widen(kv.v_cache[page, h // 2, 0]))
+
+
+def test_attention_dominant_logit_closed_form(oracle):
+    # keys are scaled basis vectors; q = lam * e_j gives logit Delta on key j
+    # and 0 elsewhere: o = (e^Delta v_j + sum_{i != j} v_i) / (e^Delta + L - 1)
+    g = rng(42)
+    L, d, j, lam = 12, 16, 7, 4.0
+    K = np.zeros((L, 1, d), dtype=np.float32)
+    for i in range(L):
+        K[i, 0, i] = 1.0
+    V = normal_bf16(g, (L, 1, d))
+    kc, vc, bt = _contig_cache(bf(K), V)
+    qv = np.zeros(d, dtype=np.float32)
+    qv[j] = lam
+    o = oracle.attention(bf(qv)[None], [0], [0], [L - 1], 1, kc, vc, bt, scale=1.0)[0]
+    Vw = widen(V)[:, 0, :]
+    e = math.exp(lam)
+    want = (e * Vw[j] + Vw.sum(axis=0) - Vw[j]) / (e + L - 1)
+    np.testing.assert_allclose(o, want, rtol=1e-12, atol=1e-14)
+
+
+def test_attention_gqa_head_mapping(oracle):
+    # V of kv head g is the constant g + 1, so head h must return h // (Hq/Hkv) + 1.
+    g = rng(43)
+    Hq, Hkv, d = 8, 2, 4
+    kv = paged_kv(g, [20, 33], Hkv, d)
+    for gg in range(Hkv):
+        kv.v_cache[:, gg] = bf([gg + 1.0])[0]
+    q = normal_bf16(g, (2, Hq, d))
+    rows = _oracle_mod.decode_rows(q, kv.seq_lens)
+    o = oracle.attention(*rows, Hq, kv.k_cache, kv.v_cache, kv.block_table)
+    for i, h in enumerate(rows[2]):
+        np.testing.assert_allclose(o[i], np.full(d, h // (Hq // Hkv) + 1.0), rtol=1e-14)
+
+
+def test_attention_is_causal(oracle):
+    g = rng(44)
+    L, d = 30, 8
+    K = normal_bf16(g, (L, 1, d))
+    V = normal_bf16(g, (L, 1, d))
+    q = normal_bf16(g, (1, d))
+    t = 17
+    kc, vc, bt = _contig_cache(K, V)
+    base = oracle.attention(q, [0], [0], [t], 1, kc, vc, bt)
+    K2, V2 = K.copy(), V.copy()
+    K2[t + 1:] = normal_bf16(g, (L - t - 1, 1, d))
+    V2[t + 1:] = normal_bf16(g, (L - t - 1, 1, d))
+    kc2, vc2, _ = _contig_cache(K2, V2)
+    np.testing.assert_array_equal(oracle.attention(q, [0], [0], [t], 1, kc2, vc2, bt), base)
+    V3 = V.copy()
+    V3[t] = normal_bf16(g, (1, d))
+    kc3, vc3, _ = _contig_cache(K, V3)
+    assert not np.array_equal(oracle.attention(q, [0], [0], [t], 1, kc3, vc3, bt), base)
+
+
+def test_attention_paging_is_transparent(oracle):
+    # Same logical K/V on shuffled pages vs on contiguous pages: equal in fp64.
+    g = rng(45)
+    lens = [50, 3, 129]
+    Hq, Hkv, d = 4, 2, 16
+    kv = paged_kv(g, lens, Hkv, d, extra_pages=5)
+    q = normal_bf16(g, (3, Hq, d))
+    rows = _oracle_mod.decode_rows(q, kv.seq_lens)
+    got = oracle.attention(*rows, Hq, kv.k_cache, kv.v_cache, kv.block_table)
+    for b, L in enumerate(lens):
+        K = np.stack([kv.k_cache[kv.block_table[b, j // 16], :, j % 16] for j in range(L)])
+        V = np.stack([kv.v_cache[kv.block_table[b, j // 16], :, j % 16] for j in range(L)])
+        kc, vc, bt = _contig_cache(K, V)
+        sel = rows[1] == b
+        o = oracle.attention(rows[0][sel], np.zeros(sel.sum()), rows[2][sel], rows[3][sel], Hq, kc, vc, bt)
+        np.testing.assert_array_equal(o, got[sel])
+
+
+def test_attention_matches_torch_sdpa_fp64(oracle):
+    g = rng(46)
+    S, Hq, Hkv, d = 70, 4, 2, 16
+    Q = normal_bf16(g, (S, Hq, d))
+    K = normal_bf16(g, (S, Hkv, d))
+    V = normal_bf16(g, (S, Hkv, d))
+    kc, vc, bt = _contig_cache(K, V)
+    rs = np.zeros(S * Hq)
+    rh = np.tile(np.arange(Hq), S)
+    rp = np.repeat(np.arange(S), Hq)
+    o = oracle.attention(Q.reshape(S * Hq, d), rs, rh, rp, Hq, kc, vc, bt).reshape(S, Hq, d)
+    qt = torch.from_numpy(widen(Q)).permute(1, 0, 2)
+    kt = torch.from_numpy(widen(K)).permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0)
+    vt = torch.from_numpy(widen(V)).permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0)
+    mask = torch.ones(S, S, dtype=torch.bool).tril()
+    want = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask)
+    np.testing.assert_allclose(o, want.permute(1, 0, 2).numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_attention_brute_force_tiny(oracle):
+    # d = 2, three keys, scale 1: written out by hand.
+    K = bf([[1, 0], [0, 1], [1, 1]])[:, None, :]
+    V = bf([[2, 0], [0, 4], [-2, 2]])[:, None, :]
+    kc, vc, bt = _contig_cache(K, V)
+    q = bf([[0.5, -1.0]])
+    o, lse = oracle.attention(q, [0], [0], [2], 1, kc, vc, bt, scale=1.0, want_lse=True)
+    s = [0.5, -1.0, -0.5]
+    e = [math.exp(x - 0.5) for x in s]
+    Z = sum(e)
+    want = [(2 * e[0] - 2 * e[2]) / Z, (4 * e[1] + 2 * e[2]) / Z]
+    np.testing.assert_allclose(o[0], want, rtol=1e-14)
+    assert abs(lse[0] - (0.5 + math.log(Z))) < 1e-14

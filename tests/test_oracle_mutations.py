@@ -1,0 +1,98 @@
+"""Plants plausible mistakes in copies of the oracle's C source, on the CPU,
+and checks that the oracle's pins catch every one of them.  This shows the
+pins have teeth: an oracle with any of these slips would not pass."""
+import json
+import os
+import shutil
+
+import numpy as np
+import pytest
+
+import oracle
+import test_oracle as pins
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(os.path.dirname(HERE), "oracle", "oracle.c")
+
+# (name, text in oracle.c, replacement, pins that must catch it)
+MUTATIONS = [
+    ("rmsnorm_drops_eps", "sqrt(ss / (double)H + eps)", "sqrt(ss / (double)H)",
+     [pins.test_rmsnorm_eps_inside_the_root]),
+    ("rmsnorm_eps_outside_root", "sqrt(ss / (double)H + eps)", "(sqrt(ss / (double)H) + eps)",
+     [pins.test_rmsnorm_eps_inside_the_root]),
+    ("rmsnorm_wrong_weight_index", "* bf16_to_double(w[j])", "* bf16_to_double(w[H - 1 - j])",
+     [pins.test_rmsnorm_matches_torch_fp64, pins.test_rmsnorm_hand_example]),
+    ("rmsnorm_mean_over_h_minus_1", "ss / (double)H", "ss / (double)(H - 1)",
+     [pins.test_rmsnorm_hand_example, pins.test_rmsnorm_matches_torch_fp64]),
+    ("matmul_transposed_weight", "s += bf16_to_double(am[k]) * bf16_to_double(wn[k]);",
+     "s += bf16_to_double(am[k]) * bf16_to_double(w[k * N + n]);",
+     [pins.test_matmul_small_integers_brute_force, pins.test_matmul_matches_torch_fp64]),
+    ("matmul_drops_last_k", "for (int64_t k = 0; k < K; ++k)", "for (int64_t k = 0; k < K - 1; ++k)",
+     [pins.test_matmul_identity_weight, pins.test_matmul_hand_example]),
+    ("kv_write_wrong_offset", "off = slot % ORACLE_PAGE", "off = (slot + 1) % ORACLE_PAGE",
+     [pins.test_kv_write_matches_direct_scatter]),
+    ("attention_wrong_gqa_map", "int32_t g = h / group;", "int32_t g = h % Hkv;",
+     [pins.test_attention_gqa_head_mapping]),
+    ("attention_causal_off_by_one", "int64_t n = (int64_t)t + 1;", "int64_t n = (int64_t)t;",
+     [pins.test_attention_identical_keys_give_prefix_mean, pins.test_attention_is_causal]),
+    ("attention_drops_scale", "double p = exp(s * scale - mx);", "double p = exp(s - mx);",
+     [pins.test_attention_matches_torch_sdpa_fp64, pins.test_attention_dominant_logit_closed_form]),
+    ("attention_lse_drops_max", "lse[r] = mx + log(l);", "lse[r] = log(l);",
+     [pins.test_attention_identical_keys_give_prefix_mean, pins.test_attention_brute_force_tiny]),
+    ("attention_wrong_slot", "j % ORACLE_PAGE) * d;\n            const uint16_t *kj",
+     "(j + 1) % ORACLE_PAGE) * d;\n            const uint16_t *kj",
+     [pins.test_attention_paging_is_transparent, pins.test_attention_matches_torch_sdpa_fp64]),
+    ("attention_values_not_normalised", "orow[i] /= l;", "orow[i] /= 1.0;",
+     [pins.test_attention_identical_keys_give_prefix_mean]),
+]
+
+
+def _catches(pin, orc):
+    try:
+        if pin is pins.test_rmsnorm_constant_row_closed_form:
+            pin(orc, 0.001)
+        else:
+            pin(orc)
+    except AssertionError:
+        return True
+    return False
+
+
+@pytest.mark.parametrize("name,find,repl,catchers", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_planted_mistake(tmp_path, name, find, repl, catchers):
+    src = open(SRC).read()
+    assert src.count(find) == 1, "mutation anchor must occur exactly once: %r" % find
+    mut = tmp_path / ("oracle_%s.c" % name)
+    mut.write_text(src.replace(find, repl))
+    lib = oracle.build(force=True, src=str(mut), out=str(tmp_path / ("lib_%s.so" % name)))
+    orc = oracle.Oracle(lib)
+    caught = [p.__name__ for p in catchers if _catches(p, orc)]
+    assert caught, "no pin caught the planted mistake %s" % name
+
+
+def test_unmutated_copy_passes_every_listed_pin(tmp_path):
+    dst = tmp_path / "oracle_copy.c"
+    shutil.copy(SRC, dst)
+    orc = oracle.Oracle(oracle.build(force=True, src=str(dst), out=str(tmp_path / "lib.so")))
+    for _, _, _, catchers in MUTATIONS:
+        for p in catchers:
+            assert not _catches(p, orc), p.__name__
+
+
+def test_oracle_matches_its_regression_fixture():
+    """tests/golden/oracle_tiny.json was written by make_oracle_tiny.py from
+    the oracle; any change to the oracle's arithmetic shows up here."""
+    with open(os.path.join(HERE, "golden", "oracle_tiny.json")) as f:
+        g = json.load(f)
+    u16 = lambda a: np.asarray(a, dtype=np.uint16)  # noqa: E731
+    r = g["rmsnorm"]
+    np.testing.assert_array_equal(oracle.rmsnorm(u16(r["x"]), u16(r["w"]), r["eps"]), r["y"])
+    m = g["matmul"]
+    np.testing.assert_array_equal(oracle.matmul(u16(m["a"]), u16(m["w"])), m["c"])
+    a = g["attention"]
+    q = u16(a["q"])
+    rows = oracle.decode_rows(q, a["seq_lens"])
+    o, lse = oracle.attention(*rows, a["Hq"], u16(a["k_cache"]), u16(a["v_cache"]),
+                              np.asarray(a["block_table"], dtype=np.int32), want_lse=True)
+    np.testing.assert_allclose(o, a["o"], rtol=1e-15, atol=0)
+    np.testing.assert_allclose(lse, a["lse"], rtol=1e-15, atol=0)
