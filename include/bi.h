@@ -1,0 +1,235 @@
+/*
+ * bi.h -- C ABI of the batch-invariant forward kernels for B200 (sm_100a).
+ *
+ * Every output row of every call below is bitwise identical whatever else is
+ * in the batch: the batch size, the other rows or requests, their order, the
+ * physical pages of the KV cache, how full the cache pool is, whether a token
+ * is processed by decode, full prefill or chunked prefill, and how the work is
+ * divided among thread blocks.  The reports on "Defeating Nondeterminism in
+ * LLM Inference" trace run-to-run differences of served models to kernels
+ * whose reduction strategy changes with the batch (xitu-tech news, section
+ * "揭露真正元凶"; neican.ai insight, section "技术原理与创新点解析") and name the
+ * three operations that need batch-invariant versions: RMSNorm, matmul and
+ * attention (same sections, and xitu-tech news, section "构建确定性解决方案").
+ *
+ * Conventions for every entry point
+ *   - Pointers marked "device" are CUDA device pointers on the current device;
+ *     pointers marked "host" are host memory.  The caller owns every buffer;
+ *     the library never allocates device memory.
+ *   - bfloat16 tensors are dense and row-major (last index fastest).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call only enqueues work on it and returns without synchronising.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and return BI_ERR_INVALID (or BI_ERR_UNSUPPORTED / BI_ERR_WORKSPACE);
+ *     a failed launch returns BI_ERR_CUDA.  Errors that only the device can
+ *     see (an out-of-range page id or slot, a bounded wait that ran out) are
+ *     recorded in a per-device status word that bi_device_status() reads.
+ *   - No C++ exception crosses this boundary.
+ */
+#ifndef BI_H
+#define BI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BI_OK = 0,
+    BI_ERR_INVALID = 1,      /* bad pointer, size, alignment or layout        */
+    BI_ERR_UNSUPPORTED = 2,  /* valid but not built (e.g. head_dim 96)        */
+    BI_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed             */
+    BI_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out            */
+    BI_ERR_WORKSPACE = 5,    /* workspace missing or smaller than required    */
+    BI_ERR_DEVICE_INDEX = 6  /* the device met an out-of-range page id / slot */
+} bi_status;
+
+typedef enum {
+    BI_BF16 = 0,
+    BI_F32 = 1
+} bi_dtype;
+
+/* Tokens per KV-cache page. */
+#define BI_PAGE_SIZE 16
+/* Keys per attention split: the fixed split SIZE (not split count). */
+#define BI_SPLIT_KEYS 256
+
+/*
+ * Paged KV cache (vLLM-style paging, as the neican.ai insight describes in
+ * section "技术原理与创新点解析", batch-invariant attention bullet).
+ *   k_cache, v_cache : device, bf16 [num_pages, num_kv_heads, 16, head_dim].
+ *                      The 16 x head_dim block of one (page, kv head) is
+ *                      contiguous.  Both start 16-byte aligned.
+ *   block_table      : device, int32 [num_seqs, max_pages_per_seq];
+ *                      block_table[b][i] is the physical page holding tokens
+ *                      16*i .. 16*i+15 of sequence b.  Entries past a
+ *                      sequence's last page are never read.
+ *   page_size        : must be 16.
+ *   head_dim         : 64 or 128.
+ */
+typedef struct bi_paged_kv {
+    void *k_cache;
+    void *v_cache;
+    const int32_t *block_table;
+    int32_t max_pages_per_seq;
+    int32_t num_pages;
+    int32_t page_size;
+    int32_t num_kv_heads;
+    int32_t head_dim;
+} bi_paged_kv;
+
+/*
+ * bi_rmsnorm -- batch-invariant RMSNorm (xitu-tech news, "构建确定性解决方案",
+ * RMSNorm item; neican.ai insight, "技术原理与创新点解析", data-parallel
+ * RMSNorm bullet: one batch row per core, its whole reduction inside that
+ * core, never a split reduction).
+ *
+ *   y[r, j] = round( x[r, j] * rsqrt( sum_i x[r, i]^2 / H + eps ) * w[j] )
+ *
+ *   x : device, bf16 [M, H];  w : device, bf16 [H];
+ *   y : device, [M, H] of out_dtype (BI_BF16: round to nearest even; BI_F32).
+ *   Requirements: H % 8 == 0, 8 <= H <= 65536, x, w, y 16-byte aligned,
+ *   y must not overlap x.  M == 0 is a no-op.
+ *   fp32 arithmetic; each row is reduced by one thread block in an order that
+ *   depends only on H.
+ */
+bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H, float eps,
+                     bi_dtype out_dtype, void *stream);
+
+/*
+ * bi_matmul -- batch-invariant matrix product (xitu-tech news,
+ * "构建确定性解决方案", matmul item: no split-K chosen from the input size, one
+ * fixed kernel configuration with one tile size; neican.ai insight,
+ * "技术原理与创新点解析", data-parallel matmul bullet: 2-D output tiles, each
+ * core computes its whole dot products).
+ *
+ *   C[m, n] = round( sum_k A[m, k] * W[n, k] )        (C = A W^T)
+ *
+ *   a : device, bf16 [M, K];  w : device, bf16 [N, K] (output-feature-major,
+ *   the nn.Linear weight layout);  c : device, [M, N] of out_dtype.
+ *   Requirements: K % 8 == 0, N % 8 == 0, M, N, K >= 1, all three pointers
+ *   16-byte aligned, c not overlapping a or w.  M == 0 is a no-op.
+ *   One fixed 128 x 256 output tile, K consumed in 64-wide slices in
+ *   ascending order with fp32 accumulation on the tensor cores; there is no
+ *   split-K and no choice of kernel by shape.
+ *   ws / ws_bytes: workspace (device); the invariant build needs none
+ *   (bi_matmul_workspace_bytes returns 0, ws may be NULL).  The variant-off
+ *   build uses it for split-K partial sums.
+ */
+bi_status bi_matmul(const void *a, const void *w, void *c, int64_t M, int64_t N, int64_t K,
+                    bi_dtype out_dtype, void *ws, size_t ws_bytes, void *stream);
+size_t bi_matmul_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * bi_kv_write -- write the step's new keys and values into the paged cache
+ * before attention runs, so that the attention kernel sees one consistent
+ * KV layout (neican.ai insight, "技术原理与创新点解析", batch-invariant
+ * attention bullet: the page table is updated before the kernel launches).
+ *
+ *   k_new, v_new : device, bf16 [T, num_kv_heads, head_dim]
+ *   slot_mapping : device, int64 [T]; token t goes to page slot/16, offset
+ *                  slot%16.  slot < 0 skips the token.  A slot at or past
+ *                  num_pages*16 is skipped and flags BI_ERR_DEVICE_INDEX.
+ *   Bit copy.  T == 0 is a no-op.  Two tokens of one call must not share a
+ *   slot.
+ */
+bi_status bi_kv_write(const bi_paged_kv *kv, const void *k_new, const void *v_new,
+                      const int64_t *slot_mapping, int64_t T, void *stream);
+
+/*
+ * bi_attention_decode -- one new query token per sequence against the paged
+ * cache (neican.ai insight, "技术原理与创新点解析", batch-invariant attention
+ * bullet: fix the SIZE of each split rather than the number of splits, so
+ * the reduction order does not depend on how many query tokens are
+ * processed; xitu-tech news, "构建确定性解决方案", attention item).
+ *
+ *   q        : device, bf16 [B, Hq, head_dim] (the token at position L_b - 1)
+ *   o        : device, bf16 [B, Hq, head_dim]
+ *   lse      : device, fp32 [B, Hq] natural-log sum of exp of the scaled
+ *              logits, or NULL
+ *   seq_lens : device, int32 [B]; L_b >= 1 includes the new token, whose K/V
+ *              bi_kv_write has already placed in the cache.
+ *   max_seq_len : host int, >= every L_b (sizes the grid and workspace).
+ *   scale    : softmax scale (usually 1/sqrt(head_dim)).
+ *   splits_per_cta : how many 256-key splits one thread block handles; 0
+ *              picks a value from B, Hq/Hkv and the SM count.  It changes
+ *              only the speed: the output bits do not depend on it.
+ *   ws, ws_bytes : device workspace of at least
+ *              bi_attention_decode_workspace_bytes(...) bytes (fp32 split
+ *              partials; may be 0 bytes, in which case ws may be NULL).
+ *   Query head h reads kv head h / (Hq / num_kv_heads).  Keys are reduced in
+ *   splits of 256 aligned to position 0; each split's partial (max, sum,
+ *   weighted values) is formed on its own and the partials are merged from
+ *   split 0 upwards, in that order, whichever block computed them.
+ *   Requirements: Hq % num_kv_heads == 0, Hq / num_kv_heads <= 128,
+ *   head_dim in {64, 128}, q and o 16-byte aligned.
+ */
+bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, float *lse,
+                              const int32_t *seq_lens, int32_t B, int32_t Hq,
+                              int32_t max_seq_len, float scale, int32_t splits_per_cta,
+                              void *ws, size_t ws_bytes, void *stream);
+size_t bi_attention_decode_workspace_bytes(const bi_paged_kv *kv, int32_t B, int32_t Hq,
+                                           int32_t max_seq_len, int32_t splits_per_cta);
+
+/*
+ * bi_attention_prefill -- causal attention of a batch of prompt chunks
+ * against the paged cache (liuwei.blog, "破解之道": the order in which the
+ * keys of token 1000 are reduced must not depend on whether the cache was
+ * empty (prefill) or full (decode); neican.ai insight, "技术原理与创新点解析").
+ *
+ *   q        : device, bf16 [T_total, Hq, head_dim], sequences packed
+ *   o        : device, bf16 [T_total, Hq, head_dim]
+ *   lse      : device, fp32 [T_total, Hq] or NULL
+ *   cu_q     : device, int32 [B + 1]; sequence b owns rows cu_q[b]..cu_q[b+1]-1
+ *   ctx_lens : device, int32 [B]; tokens of sequence b already in the cache
+ *              before this chunk.  The chunk's own K/V must already be in the
+ *              cache (bi_kv_write), so the cache holds ctx_lens[b] +
+ *              (cu_q[b+1]-cu_q[b]) tokens of sequence b.
+ *   max_q_len : host int, >= every chunk length.
+ *   The row at absolute position t attends keys 0..t with the same 256-key
+ *   splits, the same per-split arithmetic and the same merge order as
+ *   bi_attention_decode, so a token's output is bitwise the same in decode,
+ *   full prefill and chunked prefill of any chunk size.
+ *   ws / ws_bytes: reserved, pass NULL / 0 (bi_attention_prefill_workspace_bytes
+ *   returns 0).
+ */
+bi_status bi_attention_prefill(const bi_paged_kv *kv, const void *q, void *o, float *lse,
+                               const int32_t *cu_q, const int32_t *ctx_lens, int32_t B,
+                               int32_t Hq, int64_t T_total, int32_t max_q_len, float scale,
+                               void *ws, size_t ws_bytes, void *stream);
+size_t bi_attention_prefill_workspace_bytes(const bi_paged_kv *kv, int32_t B, int32_t Hq,
+                                            int32_t max_q_len);
+
+/* Human-readable name of a status code (static string). */
+const char *bi_status_string(bi_status s);
+
+/* 1 for the batch-invariant build, 0 for the variant-off build (split-K
+ * matmul, split count chosen from the load, split-reduction RMSNorm) that
+ * exists to measure what invariance costs. */
+int bi_build_invariant(void);
+
+/*
+ * bi_device_status -- synchronise `stream`, then read and clear the current
+ * device's status word.  Returns BI_OK, BI_ERR_TIMEOUT or
+ * BI_ERR_DEVICE_INDEX (the first error recorded since the last read), or
+ * BI_ERR_CUDA if the synchronisation itself failed.
+ */
+bi_status bi_device_status(void *stream);
+
+/*
+ * bi_debug_bounded_wait -- launches one thread block that waits on a
+ * barrier nothing ever arrives at, using the same bounded wait as every
+ * kernel of the library, with a limit of `timeout_ns` nanoseconds
+ * (1e3 .. 1e9).  The wait gives up, records BI_ERR_TIMEOUT in the status
+ * word and the kernel returns normally: the context stays usable.  It exists
+ * so that a test can check the timeout path without faulting the GPU.
+ */
+bi_status bi_debug_bounded_wait(uint64_t timeout_ns, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BI_H */

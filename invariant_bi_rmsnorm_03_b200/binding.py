@@ -1,0 +1,277 @@
+"""Thin ctypes binding of the C ABI (include/bi.h), taking torch tensors.
+
+Each method marshals its arguments (device pointers, sizes, the current CUDA
+stream) and calls the C entry point of the same name; every step of the
+computation runs in the library's CUDA kernels.  torch provides device
+memory and streams only.  There is no fallback: if the library is missing or
+cannot be loaded, :func:`load` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import enum
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+LIBDIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib")
+PAGE_SIZE = 16
+SPLIT_KEYS = 256
+
+
+class Status(enum.IntEnum):
+    OK = 0
+    INVALID = 1
+    UNSUPPORTED = 2
+    CUDA = 3
+    TIMEOUT = 4
+    WORKSPACE = 5
+    DEVICE_INDEX = 6
+
+
+class BIError(RuntimeError):
+    def __init__(self, fn: str, status: int, text: str):
+        super().__init__("%s failed: %s (%d)" % (fn, text, status))
+        self.status = Status(status)
+
+
+class _PagedKV(ctypes.Structure):
+    _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+                ("block_table", ctypes.c_void_p), ("max_pages_per_seq", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+@dataclass
+class PagedKV:
+    """A paged KV cache on the device: ``k_cache``/``v_cache`` bf16
+    ``[num_pages, Hkv, 16, d]`` and ``block_table`` int32 ``[num_seqs,
+    max_pages]``.  The caller owns the tensors."""
+
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    block_table: torch.Tensor
+
+    def c_struct(self) -> _PagedKV:
+        k, v, bt = self.k_cache, self.v_cache, self.block_table
+        if k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16 or bt.dtype != torch.int32:
+            raise TypeError("k_cache/v_cache must be bfloat16 and block_table int32")
+        if k.shape != v.shape or k.dim() != 4 or k.shape[2] != PAGE_SIZE:
+            raise ValueError("cache tensors must be [num_pages, Hkv, 16, d]")
+        for t in (k, v, bt):
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError("cache tensors must be contiguous CUDA tensors")
+        return _PagedKV(k.data_ptr(), v.data_ptr(), bt.data_ptr(), bt.shape[1], k.shape[0],
+                        PAGE_SIZE, k.shape[1], k.shape[3])
+
+    @property
+    def num_kv_heads(self) -> int:
+        return self.k_cache.shape[1]
+
+    @property
+    def head_dim(self) -> int:
+        return self.k_cache.shape[3]
+
+
+_DT = {torch.bfloat16: 0, torch.float32: 1}
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+class Library:
+    """One loaded build of the library (invariant or variant-off)."""
+
+    SYMBOLS = ("bi_rmsnorm", "bi_matmul", "bi_matmul_workspace_bytes", "bi_kv_write",
+               "bi_attention_decode", "bi_attention_decode_workspace_bytes",
+               "bi_attention_prefill", "bi_attention_prefill_workspace_bytes",
+               "bi_status_string", "bi_build_invariant", "bi_device_status",
+               "bi_debug_bounded_wait")
+
+    def __init__(self, path: str):
+        if not os.path.exists(path):
+            raise ImportError("CUDA library %s is missing: build it with "
+                              "`python -m invariant_bi_rmsnorm_03_b200.build`" % path)
+        self.path = path
+        L = ctypes.CDLL(path)
+        P, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
+        sz, st = ctypes.c_size_t, ctypes.c_int
+        kvp = ctypes.POINTER(_PagedKV)
+        L.bi_rmsnorm.argtypes = [P, P, P, i64, i64, f32, st, P]
+        L.bi_matmul.argtypes = [P, P, P, i64, i64, i64, st, P, sz, P]
+        L.bi_matmul_workspace_bytes.argtypes = [i64, i64, i64]
+        L.bi_matmul_workspace_bytes.restype = sz
+        L.bi_kv_write.argtypes = [kvp, P, P, P, i64, P]
+        L.bi_attention_decode.argtypes = [kvp, P, P, P, P, i32, i32, i32, f32, i32, P, sz, P]
+        L.bi_attention_decode_workspace_bytes.argtypes = [kvp, i32, i32, i32, i32]
+        L.bi_attention_decode_workspace_bytes.restype = sz
+        L.bi_attention_prefill.argtypes = [kvp, P, P, P, P, P, i32, i32, i64, i32, f32, P, sz, P]
+        L.bi_attention_prefill_workspace_bytes.argtypes = [kvp, i32, i32, i32]
+        L.bi_attention_prefill_workspace_bytes.restype = sz
+        L.bi_status_string.argtypes = [st]
+        L.bi_status_string.restype = ctypes.c_char_p
+        L.bi_build_invariant.restype = ctypes.c_int
+        L.bi_device_status.argtypes = [P]
+        L.bi_debug_bounded_wait.argtypes = [ctypes.c_uint64, P]
+        for name in ("bi_rmsnorm", "bi_matmul", "bi_kv_write", "bi_attention_decode",
+                     "bi_attention_prefill", "bi_device_status", "bi_debug_bounded_wait"):
+            getattr(L, name).restype = st
+        self.lib = L
+
+    # ------------------------------------------------------------ helpers
+    def _check(self, fn: str, status: int):
+        if status != 0:
+            raise BIError(fn, status, self.lib.bi_status_string(status).decode())
+
+    def bi_build_invariant(self) -> int:
+        return int(self.lib.bi_build_invariant())
+
+    def bi_status_string(self, status: int) -> str:
+        return self.lib.bi_status_string(int(status)).decode()
+
+    def bi_device_status(self, stream=None) -> Status:
+        return Status(self.lib.bi_device_status(_stream(stream)))
+
+    def bi_debug_bounded_wait(self, timeout_ns: int, stream=None) -> None:
+        self._check("bi_debug_bounded_wait",
+                    self.lib.bi_debug_bounded_wait(int(timeout_ns), _stream(stream)))
+
+    # ------------------------------------------------------------ RMSNorm
+    def bi_rmsnorm(self, x: torch.Tensor, w: torch.Tensor, eps: float = 1e-6, out=None,
+                   out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+        _need(x, "x", torch.bfloat16)
+        M, H = x.shape
+        _need(w, "w", torch.bfloat16, (H,))
+        if out is None:
+            out = torch.empty((M, H), dtype=out_dtype, device=x.device)
+        _need(out, "out", out_dtype, (M, H))
+        self._check("bi_rmsnorm", self.lib.bi_rmsnorm(_ptr(x), _ptr(w), _ptr(out), M, H,
+                                                      float(eps), _DT[out_dtype], _stream(stream)))
+        return out
+
+    # ------------------------------------------------------------ matmul
+    def bi_matmul_workspace_bytes(self, M: int, N: int, K: int) -> int:
+        return int(self.lib.bi_matmul_workspace_bytes(M, N, K))
+
+    def bi_matmul(self, a: torch.Tensor, w: torch.Tensor, out=None, out_dtype=torch.bfloat16,
+                  ws=None, stream=None) -> torch.Tensor:
+        """C = a @ w.T with a [M, K] and w [N, K] (bf16)."""
+        _need(a, "a", torch.bfloat16)
+        M, K = a.shape
+        _need(w, "w", torch.bfloat16)
+        N = w.shape[0]
+        if w.shape[1] != K:
+            raise ValueError("w must be [N, K] with K = %d" % K)
+        if out is None:
+            out = torch.empty((M, N), dtype=out_dtype, device=a.device)
+        _need(out, "out", out_dtype, (M, N))
+        need = self.bi_matmul_workspace_bytes(M, N, K)
+        if need and (ws is None or ws.numel() * ws.element_size() < need):
+            ws = torch.empty(need, dtype=torch.uint8, device=a.device)
+        nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+        self._check("bi_matmul", self.lib.bi_matmul(_ptr(a), _ptr(w), _ptr(out), M, N, K,
+                                                    _DT[out_dtype], _ptr(ws), nbytes,
+                                                    _stream(stream)))
+        return out
+
+    # ------------------------------------------------------------ KV cache
+    def bi_kv_write(self, kv: PagedKV, k_new: torch.Tensor, v_new: torch.Tensor,
+                    slot_mapping: torch.Tensor, stream=None) -> None:
+        T = k_new.shape[0]
+        shape = (T, kv.num_kv_heads, kv.head_dim)
+        _need(k_new, "k_new", torch.bfloat16, shape)
+        _need(v_new, "v_new", torch.bfloat16, shape)
+        _need(slot_mapping, "slot_mapping", torch.int64, (T,))
+        c = kv.c_struct()
+        self._check("bi_kv_write", self.lib.bi_kv_write(ctypes.byref(c), _ptr(k_new), _ptr(v_new),
+                                                        _ptr(slot_mapping), T, _stream(stream)))
+
+    # ------------------------------------------------------------ attention
+    def bi_attention_decode_workspace_bytes(self, kv: PagedKV, B: int, Hq: int, max_seq_len: int,
+                                            splits_per_cta: int = 0) -> int:
+        c = kv.c_struct()
+        return int(self.lib.bi_attention_decode_workspace_bytes(ctypes.byref(c), B, Hq,
+                                                                max_seq_len, splits_per_cta))
+
+    def bi_attention_decode(self, kv: PagedKV, q: torch.Tensor, seq_lens: torch.Tensor,
+                            max_seq_len: int, scale: float | None = None, want_lse: bool = False,
+                            splits_per_cta: int = 0, out=None, lse=None, ws=None, stream=None):
+        """One query token per sequence: q [B, Hq, d] -> o [B, Hq, d] (and lse [B, Hq])."""
+        _need(q, "q", torch.bfloat16)
+        B, Hq, d = q.shape
+        _need(seq_lens, "seq_lens", torch.int32, (B,))
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        if out is None:
+            out = torch.empty_like(q)
+        _need(out, "out", torch.bfloat16, (B, Hq, d))
+        if want_lse and lse is None:
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        if lse is not None:
+            _need(lse, "lse", torch.float32, (B, Hq))
+        c = kv.c_struct()
+        need = int(self.lib.bi_attention_decode_workspace_bytes(ctypes.byref(c), B, Hq,
+                                                                max_seq_len, splits_per_cta))
+        if need and (ws is None or ws.numel() * ws.element_size() < need):
+            ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+        nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+        self._check("bi_attention_decode", self.lib.bi_attention_decode(
+            ctypes.byref(c), _ptr(q), _ptr(out), _ptr(lse), _ptr(seq_lens), B, Hq,
+            int(max_seq_len), float(scale), int(splits_per_cta), _ptr(ws), nbytes,
+            _stream(stream)))
+        return (out, lse) if want_lse else out
+
+    def bi_attention_prefill(self, kv: PagedKV, q: torch.Tensor, cu_q: torch.Tensor,
+                             ctx_lens: torch.Tensor, max_q_len: int, scale: float | None = None,
+                             want_lse: bool = False, out=None, lse=None, stream=None):
+        """Causal prompt chunks: q [T_total, Hq, d] packed by cu_q -> o (and lse [T_total, Hq])."""
+        _need(q, "q", torch.bfloat16)
+        T, Hq, d = q.shape
+        B = ctx_lens.shape[0]
+        _need(cu_q, "cu_q", torch.int32, (B + 1,))
+        _need(ctx_lens, "ctx_lens", torch.int32, (B,))
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        if out is None:
+            out = torch.empty_like(q)
+        _need(out, "out", torch.bfloat16, (T, Hq, d))
+        if want_lse and lse is None:
+            lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+        if lse is not None:
+            _need(lse, "lse", torch.float32, (T, Hq))
+        c = kv.c_struct()
+        self._check("bi_attention_prefill", self.lib.bi_attention_prefill(
+            ctypes.byref(c), _ptr(q), _ptr(out), _ptr(lse), _ptr(cu_q), _ptr(ctx_lens), B, Hq, T,
+            int(max_q_len), float(scale), None, 0, _stream(stream)))
+        return (out, lse) if want_lse else out
+
+
+_LIBS: dict = {}
+
+
+def load(variant: bool = False) -> Library:
+    """The invariant library (default) or the variant-off build."""
+    name = "libbi_variant.so" if variant else "libbi.so"
+    if name not in _LIBS:
+        _LIBS[name] = Library(os.path.join(LIBDIR, name))
+    return _LIBS[name]

@@ -1,0 +1,363 @@
+// api.cu -- the C ABI declared in include/bi.h: argument checks, TMA
+// descriptor encoding, launches and the device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "bi.h"
+#include "bi_common.cuh"
+#include "bi_launch.h"
+
+// The per-device status word: first error recorded by any kernel.
+__device__ unsigned g_bi_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool ready = false;
+    unsigned *status = nullptr;
+    int num_sms = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bi_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BI_OK : BI_ERR_CUDA; }
+
+// Looks up the current device's status-word address and SM count (once).
+bi_status device_state(DeviceState **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BI_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState &d = g_dev[dev];
+    if (!d.ready) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_bi_status) != cudaSuccess) return BI_ERR_CUDA;
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return BI_ERR_CUDA;
+        d.status = static_cast<unsigned *>(p);
+        d.num_sms = sms;
+        d.ready = true;
+    }
+    if (!g_encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                             cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return BI_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    *out = &d;
+    return BI_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// bf16 tensor map, 128-byte swizzle, zero fill out of bounds.  dims[0] is
+// the contiguous dimension; strides are in bytes for dims 1.. .
+bool encode(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
+            const uint64_t *strides, const uint32_t *box)
+{
+    uint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+                                const_cast<void *>(base), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool kv_ok(const bi_paged_kv *kv)
+{
+    if (!kv || !kv->k_cache || !kv->v_cache || !kv->block_table) return false;
+    if (kv->page_size != BI_PAGE_SIZE) return false;
+    if (kv->num_kv_heads < 1 || kv->num_pages < 1 || kv->max_pages_per_seq < 1) return false;
+    if (!aligned16(kv->k_cache) || !aligned16(kv->v_cache)) return false;
+    // TMA row coordinates of the cache are 32-bit
+    if (int64_t(kv->num_pages) * kv->num_kv_heads * BI_PAGE_SIZE >= (int64_t(1) << 31))
+        return false;
+    return true;
+}
+
+bool head_dim_ok(int d) { return d == 64 || d == 128; }
+
+int decode_splits_per_cta(int B, int Hkv, int max_splits, int requested, int num_sms)
+{
+    if (requested > 0) return requested < max_splits ? requested : max_splits;
+    const int units = B * Hkv;
+    int k = (2 * num_sms + units - 1) / units;  // blocks per sequence that fill the GPU
+    if (k < 1) k = 1;
+    int c = (max_splits + k - 1) / k;
+    return c < 1 ? 1 : c;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *bi_status_string(bi_status s)
+{
+    switch (s) {
+    case BI_OK: return "ok";
+    case BI_ERR_INVALID: return "invalid argument";
+    case BI_ERR_UNSUPPORTED: return "unsupported configuration";
+    case BI_ERR_CUDA: return "CUDA error";
+    case BI_ERR_TIMEOUT: return "device-side wait timed out";
+    case BI_ERR_WORKSPACE: return "workspace missing or too small";
+    case BI_ERR_DEVICE_INDEX: return "device met an out-of-range page id or slot";
+    }
+    return "unknown status";
+}
+
+int bi_build_invariant(void) { return BI_INVARIANT ? 1 : 0; }
+
+bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H, float eps,
+                     bi_dtype out_dtype, void *stream)
+{
+    if (M < 0 || H < 8 || H % 8 != 0 || H > 65536) return BI_ERR_INVALID;
+    if (out_dtype != BI_BF16 && out_dtype != BI_F32) return BI_ERR_INVALID;
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return BI_ERR_INVALID;
+    if (M == 0) return BI_OK;
+    if (!x || !w || !y || !aligned16(x) || !aligned16(w) || !aligned16(y)) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_rmsnorm(x, w, y, M, H, eps, out_dtype == BI_F32, d->num_sms,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+size_t bi_matmul_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    DeviceState *d;
+    if (device_state(&d) != BI_OK) return 0;
+    const int ks = bi::gemm_k_splits(M, N, K, d->num_sms);
+    return ks > 1 ? size_t(ks) * M * N * sizeof(float) : 0;
+}
+
+bi_status bi_matmul(const void *a, const void *w, void *c, int64_t M, int64_t N, int64_t K,
+                    bi_dtype out_dtype, void *ws, size_t ws_bytes, void *stream)
+{
+    if (M < 0 || N < 1 || K < 1 || N % 8 != 0 || K % 8 != 0) return BI_ERR_INVALID;
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return BI_ERR_INVALID;
+    if (out_dtype != BI_BF16 && out_dtype != BI_F32) return BI_ERR_INVALID;
+    if (M == 0) return BI_OK;
+    if (!a || !w || !c || !aligned16(a) || !aligned16(w) || !aligned16(c)) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    const int ks = bi::gemm_k_splits(M, N, K, d->num_sms);
+    if (ks > 1) {
+        if (!ws || ws_bytes < size_t(ks) * M * N * sizeof(float) || !aligned16(ws))
+            return BI_ERR_WORKSPACE;
+    }
+    CUtensorMap ta, tw;
+    const uint64_t da[2] = {uint64_t(K), uint64_t(M)}, sa[1] = {uint64_t(K) * 2};
+    const uint64_t dw[2] = {uint64_t(K), uint64_t(N)}, sw[1] = {uint64_t(K) * 2};
+    const uint32_t ba[2] = {uint32_t(bi::kGemmBK), uint32_t(bi::kGemmBM)};
+    const uint32_t bw[2] = {uint32_t(bi::kGemmBK), uint32_t(bi::kGemmBN)};
+    if (!encode(&ta, a, 2, da, sa, ba) || !encode(&tw, w, 2, dw, sw, bw)) return BI_ERR_CUDA;
+    return from_cuda(bi::launch_gemm(ta, tw, c, int(M), int(N), int(K), out_dtype == BI_F32,
+                                     static_cast<float *>(ws), ks, d->num_sms, d->status,
+                                     bi::kDefaultTimeoutNs, static_cast<cudaStream_t>(stream)));
+}
+
+bi_status bi_kv_write(const bi_paged_kv *kv, const void *k_new, const void *v_new,
+                      const int64_t *slot_mapping, int64_t T, void *stream)
+{
+    if (!kv_ok(kv) || !head_dim_ok(kv->head_dim) || T < 0) return BI_ERR_INVALID;
+    if (T == 0) return BI_OK;
+    if (!k_new || !v_new || !slot_mapping || !aligned16(k_new) || !aligned16(v_new))
+        return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_kv_write(kv->k_cache, kv->v_cache, kv->num_pages, kv->num_kv_heads,
+                                         kv->head_dim, k_new, v_new, slot_mapping, T, d->status,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+static bool attn_common_ok(const bi_paged_kv *kv, int32_t Hq)
+{
+    if (!kv_ok(kv)) return false;
+    if (Hq < 1 || Hq % kv->num_kv_heads != 0) return false;
+    if (Hq / kv->num_kv_heads > 128) return false;
+    return true;
+}
+
+size_t bi_attention_decode_workspace_bytes(const bi_paged_kv *kv, int32_t B, int32_t Hq,
+                                           int32_t max_seq_len, int32_t splits_per_cta)
+{
+    if (!kv || B < 1 || Hq < 1 || max_seq_len < 1 || kv->num_kv_heads < 1) return 0;
+    DeviceState *d;
+    if (device_state(&d) != BI_OK) return 0;
+    const int max_splits = (max_seq_len + bi::kSplit - 1) / bi::kSplit;
+    const int c = decode_splits_per_cta(B, kv->num_kv_heads, max_splits, splits_per_cta, d->num_sms);
+    const int chunks = (max_splits + c - 1) / c;
+    return bi::attn_ws_bytes(B, Hq, kv->head_dim, max_splits, chunks);
+}
+
+bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, float *lse,
+                              const int32_t *seq_lens, int32_t B, int32_t Hq,
+                              int32_t max_seq_len, float scale, int32_t splits_per_cta,
+                              void *ws, size_t ws_bytes, void *stream)
+{
+    if (!attn_common_ok(kv, Hq)) return BI_ERR_INVALID;
+    if (!head_dim_ok(kv->head_dim)) return BI_ERR_UNSUPPORTED;
+    if (B < 0 || max_seq_len < 1 || splits_per_cta < 0 || !std::isfinite(scale))
+        return BI_ERR_INVALID;
+    if (int64_t(max_seq_len) > int64_t(kv->max_pages_per_seq) * BI_PAGE_SIZE) return BI_ERR_INVALID;
+    if (B == 0) return BI_OK;
+    if (B > 65535) return BI_ERR_UNSUPPORTED;
+    if (!q || !o || !seq_lens || !aligned16(q) || !aligned16(o)) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+
+    const int D = kv->head_dim, Hkv = kv->num_kv_heads, group = Hq / Hkv;
+    const int max_splits = (max_seq_len + bi::kSplit - 1) / bi::kSplit;
+    const int c = decode_splits_per_cta(B, Hkv, max_splits, splits_per_cta, d->num_sms);
+    const int chunks = (max_splits + c - 1) / c;
+    const size_t need = bi::attn_ws_bytes(B, Hq, D, max_splits, chunks);
+    if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return BI_ERR_WORKSPACE;
+
+    bi::AttnParams p{};
+    p.v_cache = kv->v_cache;
+    p.block_table = kv->block_table;
+    p.max_pages = kv->max_pages_per_seq;
+    p.num_pages = kv->num_pages;
+    p.Hkv = Hkv;
+    p.Hq = Hq;
+    p.group = group;
+    p.rows_per_q = (group + 3) / 4;
+    p.decode = 1;
+    p.B = B;
+    p.seq_lens = seq_lens;
+    p.splits_per_cta = c;
+    p.max_splits = max_splits;
+    p.scale_log2 = float(double(scale) * 1.4426950408889634);
+    p.o = o;
+    p.lse = lse;
+    p.ws = static_cast<float *>(ws);
+    p.status = d->status;
+    p.timeout_ns = bi::kDefaultTimeoutNs;
+
+    CUtensorMap tq, tk, tv;
+    const uint64_t dq[3] = {uint64_t(D), uint64_t(Hq), uint64_t(B)};
+    const uint64_t sq[2] = {uint64_t(D) * 2, uint64_t(Hq) * D * 2};
+    const uint32_t bq[3] = {64, uint32_t(p.rows_per_q), 1};
+    const uint64_t dkv[2] = {uint64_t(D), uint64_t(kv->num_pages) * Hkv * BI_PAGE_SIZE};
+    const uint64_t skv[1] = {uint64_t(D) * 2};
+    const uint32_t bkv[2] = {64, BI_PAGE_SIZE};
+    if (!encode(&tq, q, 3, dq, sq, bq) || !encode(&tk, kv->k_cache, 2, dkv, skv, bkv) ||
+        !encode(&tv, kv->v_cache, 2, dkv, skv, bkv))
+        return BI_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = bi::launch_attention(tq, tk, tv, p, D, s);
+    if (e != cudaSuccess) return BI_ERR_CUDA;
+    if (chunks > 1) e = bi::launch_attn_combine(p, D, s);
+    return from_cuda(e);
+}
+
+size_t bi_attention_prefill_workspace_bytes(const bi_paged_kv *kv, int32_t B, int32_t Hq,
+                                            int32_t max_q_len)
+{
+    (void)kv, (void)B, (void)Hq, (void)max_q_len;
+    return 0;
+}
+
+bi_status bi_attention_prefill(const bi_paged_kv *kv, const void *q, void *o, float *lse,
+                               const int32_t *cu_q, const int32_t *ctx_lens, int32_t B,
+                               int32_t Hq, int64_t T_total, int32_t max_q_len, float scale,
+                               void *ws, size_t ws_bytes, void *stream)
+{
+    (void)ws, (void)ws_bytes;
+    if (!attn_common_ok(kv, Hq)) return BI_ERR_INVALID;
+    if (!head_dim_ok(kv->head_dim)) return BI_ERR_UNSUPPORTED;
+    if (B < 0 || T_total < 0 || max_q_len < 0 || !std::isfinite(scale)) return BI_ERR_INVALID;
+    if (T_total > INT32_MAX) return BI_ERR_UNSUPPORTED;
+    if (B == 0 || T_total == 0 || max_q_len == 0) return BI_OK;
+    if (B > 65535 || Hq > 65535) return BI_ERR_UNSUPPORTED;
+    if (!q || !o || !cu_q || !ctx_lens || !aligned16(q) || !aligned16(o)) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+
+    const int D = kv->head_dim, Hkv = kv->num_kv_heads;
+    bi::AttnParams p{};
+    p.v_cache = kv->v_cache;
+    p.block_table = kv->block_table;
+    p.max_pages = kv->max_pages_per_seq;
+    p.num_pages = kv->num_pages;
+    p.Hkv = Hkv;
+    p.Hq = Hq;
+    p.group = Hq / Hkv;
+    p.rows_per_q = 32;
+    p.decode = 0;
+    p.B = B;
+    p.cu_q = cu_q;
+    p.ctx_lens = ctx_lens;
+    p.num_q_tiles = (max_q_len + 127) / 128;
+    p.scale_log2 = float(double(scale) * 1.4426950408889634);
+    p.o = o;
+    p.lse = lse;
+    p.status = d->status;
+    p.timeout_ns = bi::kDefaultTimeoutNs;
+
+    CUtensorMap tq, tk, tv;
+    const uint64_t dq[3] = {uint64_t(D), uint64_t(Hq), uint64_t(T_total)};
+    const uint64_t sq[2] = {uint64_t(D) * 2, uint64_t(Hq) * D * 2};
+    const uint32_t bq[3] = {64, 1, 128};
+    const uint64_t dkv[2] = {uint64_t(D), uint64_t(kv->num_pages) * Hkv * BI_PAGE_SIZE};
+    const uint64_t skv[1] = {uint64_t(D) * 2};
+    const uint32_t bkv[2] = {64, BI_PAGE_SIZE};
+    if (!encode(&tq, q, 3, dq, sq, bq) || !encode(&tk, kv->k_cache, 2, dkv, skv, bkv) ||
+        !encode(&tv, kv->v_cache, 2, dkv, skv, bkv))
+        return BI_ERR_CUDA;
+    return from_cuda(bi::launch_attention(tq, tk, tv, p, D, static_cast<cudaStream_t>(stream)));
+}
+
+bi_status bi_device_status(void *stream)
+{
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return BI_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpy(&v, d->status, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return BI_ERR_CUDA;
+    if (v != 0) {
+        const unsigned zero = 0;
+        if (cudaMemcpy(d->status, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess)
+            return BI_ERR_CUDA;
+    }
+    switch (v) {
+    case 0: return BI_OK;
+    case bi::BI_DEV_TIMEOUT: return BI_ERR_TIMEOUT;
+    case bi::BI_DEV_BAD_INDEX: return BI_ERR_DEVICE_INDEX;
+    default: return BI_ERR_CUDA;
+    }
+}
+
+bi_status bi_debug_bounded_wait(uint64_t timeout_ns, void *stream)
+{
+    if (timeout_ns < 1000 || timeout_ns > 1000000000ull) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_bounded_wait_probe(d->status, timeout_ns,
+                                                   static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

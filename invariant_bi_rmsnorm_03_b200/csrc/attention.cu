@@ -1,0 +1,622 @@
+// attention.cu -- batch-invariant attention over a paged KV cache.
+//
+// neican.ai insight, "技术原理与创新点解析", batch-invariant attention bullet:
+// the KV-cache page table is updated before the kernel launches, and a
+// split reduction fixes the SIZE of each split rather than the number of
+// splits, so the reduction order is the same however many query tokens are
+// processed.  liuwei.blog, "破解之道": FlashAttention-2 parallelises over
+// queries and reduces over keys/values, and the order in which the keys of a
+// token are reduced must not depend on whether the cache was empty (prefill)
+// or full (decode).  xitu-tech news, "构建确定性解决方案", attention item.
+//
+// The method as built here.  For a query row at absolute position t the keys
+// 0..t are cut into splits of 256 keys aligned to key 0.  For each split s,
+// on its own:
+//   S      = Q K_s^T                    tcgen05, M=128 rows, N=256 keys, fp32
+//   x_j    = S_j * scale * log2(e), masked to -inf where key j > t
+//   m_s    = max_j x_j
+//   p_j    = 2^(x_j - m_s),  l_s = sum_j p_j   (fixed order: 32-key chunks
+//            summed by a pairwise tree, chunk sums added left to right)
+//   O_s    = bf16(p) V_s                tcgen05, P read from tensor memory
+// and the partials are merged from split 0 upwards, always in that order:
+//   m' = max(m, m_s), a = 2^(m - m'), c = 2^(m_s - m')
+//   l' = l a + l_s c,  O' = O a + O_s c          (separately rounded fp32)
+//   out = O / l,  lse = (m + log2 l) ln 2.
+// One kernel body serves decode (rows = the Hq/Hkv query heads of one
+// token) and prefill (rows = 128 tokens of one head); a row's arithmetic is
+// the same instruction sequence in both, so a token's output has the same
+// bits in decode, full prefill and chunked prefill of any chunk size.
+//
+// Decode divides a sequence's splits among blocks (`splits_per_cta`).  A
+// block whose range starts at split 0 merges in registers; every other block
+// writes each split's own partial (m_s, l_s, O_s) to the workspace, and
+// attn_combine continues the merge from where block 0 stopped, split by
+// split, with the same merge function.  The bits therefore do not depend on
+// how many blocks served a sequence.
+//
+// Block of 192 threads, one per SM (224 KB shared memory, 512 TMEM columns):
+//   warp 0     producer: Q by TMA once; per split K then V, 16 pages of
+//              [16 x 64] bf16 boxes each (gathered through the page table),
+//              into a 3-slot ring; the V rows past the sequence end are
+//              zero (TMA out-of-bounds fill for whole pages, explicit stores
+//              for the partial page) so that 0 * stale never reaches O.
+//   warp 1     TMEM allocation and MMA issue (one thread)
+//   warps 2-5  softmax and merge; warp w owns TMEM lanes 32(w%4)..+31.
+//              Decode spreads the query heads over the four lane quarters.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "bi_common.cuh"
+#include "bi_launch.h"
+#include "bi_ptx.cuh"
+
+namespace bi {
+namespace {
+
+constexpr int THREADS = 192;
+constexpr float kLn2 = 0.693147180559945309f;
+
+template <int D>
+struct Cfg {
+    static constexpr int KB = D / 64;                   // 128-byte column blocks of a row
+    static constexpr int Q_KB_BYTES = 128 * 128;        // one column block of the Q tile
+    static constexpr int Q_BYTES = KB * Q_KB_BYTES;
+    static constexpr int KV_KB_BYTES = kSplit * 128;    // one column block of a 256-key tile
+    static constexpr int KV_BYTES = KB * KV_KB_BYTES;
+    static constexpr int PAGE_KB_BYTES = kPage * 128;   // one page of one column block
+    static constexpr int NSLOT = 3;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM = 1024 + Q_BYTES + NSLOT * KV_BYTES + BAR_BYTES;
+    static constexpr uint32_t S_COL = 0, P_COL = 256, O_COL = 384, TMEM_COLS = 512;
+    static constexpr int REC = D + 4;                   // floats per spilled partial
+};
+
+// ---------------------------------------------------------------- merge
+
+__device__ __forceinline__ void merge_scales(float m, float ms, float &mn, float &a, float &c)
+{
+    mn = fmaxf(m, ms);
+    a = ex2(__fsub_rn(m, mn));
+    c = ex2(__fsub_rn(ms, mn));
+}
+
+__device__ __forceinline__ float merge_val(float x, float a, float xs, float c)
+{
+    return __fadd_rn(__fmul_rn(x, a), __fmul_rn(xs, c));
+}
+
+__device__ __forceinline__ float finish_lse(float m, float l)
+{
+    return __fmul_rn(__fadd_rn(m, log2f(l)), kLn2);
+}
+
+template <int D>
+__device__ __forceinline__ void write_out(const float (&O)[D], float l, float m,
+                                          __nv_bfloat16 *orow, float *lse_ptr)
+{
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        uint4 v;
+        v.x = pack_bf16x2(__fdiv_rn(O[8 * c + 0], l), __fdiv_rn(O[8 * c + 1], l));
+        v.y = pack_bf16x2(__fdiv_rn(O[8 * c + 2], l), __fdiv_rn(O[8 * c + 3], l));
+        v.z = pack_bf16x2(__fdiv_rn(O[8 * c + 4], l), __fdiv_rn(O[8 * c + 5], l));
+        v.w = pack_bf16x2(__fdiv_rn(O[8 * c + 6], l), __fdiv_rn(O[8 * c + 7], l));
+        reinterpret_cast<uint4 *>(orow)[c] = v;
+    }
+    if (lse_ptr) *lse_ptr = finish_lse(m, l);
+}
+
+__device__ bool wait_drain(uint64_t *bar, uint32_t parity, uint64_t timeout_ns)
+{
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > timeout_ns) return false;
+    return true;
+}
+
+// ---------------------------------------------------------------- work item
+
+struct Item {
+    int b, g, h;          // sequence, kv head, query head (prefill)
+    int s0, s1, n_splits; // split range of this block; splits of the sequence
+    int kv_len;           // keys in the cache for this sequence
+    int q_row0;           // prefill: first packed token of the tile
+    int rows;             // prefill: valid tokens in the tile
+    int pos0;             // prefill: absolute position of the tile's first row
+};
+
+__device__ __forceinline__ bool make_item(const AttnParams &p, Item &it)
+{
+    if (p.decode) {
+        it.b = blockIdx.z;
+        it.g = blockIdx.y;
+        it.h = 0;
+        it.kv_len = p.seq_lens[it.b];
+        it.n_splits = (it.kv_len + kSplit - 1) / kSplit;
+        it.s0 = blockIdx.x * p.splits_per_cta;
+        if (it.kv_len <= 0 || it.s0 >= it.n_splits) return false;
+        it.s1 = min(it.n_splits, it.s0 + p.splits_per_cta);
+        it.q_row0 = it.rows = it.pos0 = 0;
+    } else {
+        it.b = blockIdx.z;
+        it.h = blockIdx.y;
+        it.g = it.h / p.group;
+        const int tile = p.num_q_tiles - 1 - static_cast<int>(blockIdx.x);  // long tiles first
+        const int q0 = p.cu_q[it.b];
+        const int n = p.cu_q[it.b + 1] - q0;
+        if (tile * 128 >= n) return false;
+        const int ctx = p.ctx_lens[it.b];
+        it.kv_len = ctx + n;
+        it.q_row0 = q0 + tile * 128;
+        it.rows = min(128, n - tile * 128);
+        it.pos0 = ctx + tile * 128;
+        const int t_max = it.pos0 + it.rows - 1;
+        it.s0 = 0;
+        it.s1 = t_max / kSplit + 1;
+        it.n_splits = (it.kv_len + kSplit - 1) / kSplit;
+    }
+    return true;
+}
+
+// Byte offset of 16-byte chunk `c` of row `r` in a 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t swz(int r, int c)
+{
+    return uint32_t(r) * 128u + (uint32_t((c ^ (r & 7))) << 4);
+}
+
+// ---------------------------------------------------------------- kernel
+
+template <int D>
+__global__ void __launch_bounds__(THREADS, 1)
+    attn_split_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                      const __grid_constant__ CUtensorMap tv, const AttnParams p)
+{
+    using C = Cfg<D>;
+    Item it;
+    if (!make_item(p, it)) return;
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
+    uint8_t *sQ = smem;
+    uint8_t *sKV = smem + C::Q_BYTES;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sKV + C::NSLOT * C::KV_BYTES);
+    uint64_t *empty = full + C::NSLOT;
+    uint64_t *barQ = empty + C::NSLOT;
+    uint64_t *barS = barQ + 1;
+    uint64_t *barP = barS + 1;
+    uint64_t *barO = barP + 1;
+    uint64_t *drain = barO + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NSLOT; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(barQ, 1);
+        mbar_init(barS, 1);
+        mbar_init(barP, 128);
+        mbar_init(barO, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
+    const int32_t *bt_row = p.block_table + int64_t(it.b) * p.max_pages;
+
+    if (warp == 0) {
+        // ====================================================== producer
+        bool ok = true;
+        uint32_t armed = 0, armed_parity = 0;
+        if (lane == 0) {
+            if (p.decode) {
+                const int rpq = p.rows_per_q;
+                mbar_arrive_expect_tx(barQ, 4u * C::KB * rpq * 128u);
+                for (int q = 0; q < 4; ++q)
+                    for (int kb = 0; kb < C::KB; ++kb)
+                        tma_load_3d(sQ + kb * C::Q_KB_BYTES + q * 32 * 128, &tq, barQ, kb * 64,
+                                    it.g * p.group + q * rpq, it.b);
+            } else {
+                mbar_arrive_expect_tx(barQ, uint32_t(C::Q_BYTES));
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tma_load_3d(sQ + kb * C::Q_KB_BYTES, &tq, barQ, kb * 64, it.h, it.q_row0);
+            }
+        }
+        int slot = 0;
+        uint32_t phase = 0;
+        for (int s = it.s0; ok && s < it.s1; ++s) {
+            const int nk = min(kSplit, it.kv_len - s * kSplit);  // valid keys, >= 1
+            const int full_pages = nk / kPage;
+            const int npages = (nk + kPage - 1) / kPage;
+            for (int which = 0; which < 2; ++which) {  // 0: K, 1: V
+                int got = 1;
+                if (lane == 0) got = wait(&empty[slot], phase ^ 1u, ctl) ? 1 : 0;
+                got = __shfl_sync(0xffffffffu, got, 0);
+                if (!got) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *dst = sKV + slot * C::KV_BYTES;
+                const CUtensorMap *map = which ? &tv : &tk;
+                // V: the partial last page is copied by the whole warp, with
+                // the rows past the sequence end set to zero.
+                if (which == 1 && full_pages < npages) {
+                    const int pg = full_pages;
+                    const int lp = s * (kSplit / kPage) + pg;  // logical page
+                    const int phys = lp < p.max_pages ? __ldg(bt_row + lp) : -1;
+                    const bool good = phys >= 0 && phys < p.num_pages;
+                    if (!good && lane == 0) record_status(p.status, BI_DEV_BAD_INDEX);
+                    const int valid = nk - pg * kPage;
+                    for (int i = lane; i < kPage * C::KB * 8; i += 32) {
+                        const int r = i / (C::KB * 8);
+                        const int kb = (i / 8) % C::KB;
+                        const int c = i % 8;
+                        uint4 v = make_uint4(0, 0, 0, 0);
+                        if (good && r < valid) {
+                            const int64_t src = ((int64_t(phys) * p.Hkv + it.g) * kPage + r) * D +
+                                                kb * 64 + c * 8;
+                            v = __ldg(reinterpret_cast<const uint4 *>(
+                                static_cast<const __nv_bfloat16 *>(p.v_cache) + src));
+                        }
+                        *reinterpret_cast<uint4 *>(dst + kb * C::KV_KB_BYTES +
+                                                   swz(pg * kPage + r, c)) = v;
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                if (lane == 0) {
+                    // K: pages holding valid keys.  V: whole valid pages, plus
+                    // all-zero (out-of-bounds) boxes for pages past the end.
+                    const int tma_pages = which ? (kSplit / kPage) - (npages - full_pages) : npages;
+                    mbar_arrive_expect_tx(&full[slot], uint32_t(tma_pages) * C::KB * C::PAGE_KB_BYTES);
+                    const int last = which ? (kSplit / kPage) : npages;
+                    for (int pg = 0; pg < last; ++pg) {
+                        if (which && pg == full_pages && full_pages < npages) continue;
+                        int row = -kPage;  // out of bounds: zero fill
+                        if (pg < (which ? full_pages : npages)) {
+                            const int lp = s * (kSplit / kPage) + pg;
+                            const int phys = lp < p.max_pages ? __ldg(bt_row + lp) : -1;
+                            if (phys >= 0 && phys < p.num_pages)
+                                row = (phys * p.Hkv + it.g) * kPage;
+                            else
+                                record_status(p.status, BI_DEV_BAD_INDEX);
+                        }
+                        for (int kb = 0; kb < C::KB; ++kb)
+                            tma_load_2d(dst + kb * C::KV_KB_BYTES + pg * C::PAGE_KB_BYTES, map,
+                                        &full[slot], kb * 64, row);
+                    }
+                    armed |= 1u << slot;
+                    armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
+                }
+                __syncwarp();
+                if (++slot == C::NSLOT) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            for (int s = 0; s < C::NSLOT; ++s)
+                if (armed & (1u << s)) wait_drain(&full[s], (armed_parity >> s) & 1u, p.timeout_ns);
+            wait_drain(barQ, 0, p.timeout_ns);
+        }
+    } else if (warp == 1) {
+        // ====================================================== MMA issue
+        if (lane == 0) {
+            const uint32_t idesc_qk = idesc_bf16_f32(128, kSplit, 0, 0);
+            const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+            const uint32_t q_base = smem_u32(sQ);
+            bool ok = wait(barQ, 0, ctl);
+            int slot = 0;
+            uint32_t phase = 0, p_phase = 0;
+            for (int s = it.s0; ok && s < it.s1; ++s) {
+                // S = Q K^T
+                if (!wait(&full[slot], phase, ctl)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t k_base = smem_u32(sKV + slot * C::KV_BYTES);
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t kb = k >> 2, kk = k & 3;
+                    mma_ss(tmem + C::S_COL,
+                           sdesc_sw128(q_base + kb * C::Q_KB_BYTES + kk * 32, 16, 1024),
+                           sdesc_sw128(k_base + kb * C::KV_KB_BYTES + kk * 32, 16, 1024), idesc_qk,
+                           k > 0 ? 1u : 0u);
+                }
+                mma_commit(barS);
+                mma_commit(&empty[slot]);
+                if (++slot == C::NSLOT) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+                // O_s = P V
+                if (!wait(barP, p_phase, ctl)) {
+                    ok = false;
+                    break;
+                }
+                p_phase ^= 1u;
+                if (!wait(&full[slot], phase, ctl)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t v_base = smem_u32(sKV + slot * C::KV_BYTES);
+#pragma unroll
+                for (int i = 0; i < kSplit / 16; ++i) {
+                    mma_ts(tmem + C::O_COL, tmem + C::P_COL + 8 * i,
+                           sdesc_sw128(v_base + i * 16 * 128, C::KV_KB_BYTES, 1024), idesc_pv,
+                           i > 0 ? 1u : 0u);
+                }
+                mma_commit(barO);
+                mma_commit(&empty[slot]);
+                if (++slot == C::NSLOT) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) {
+                mma_commit(drain);
+                wait_drain(drain, 0, p.timeout_ns);
+            }
+        }
+    } else {
+        // ====================================================== softmax
+        const int q = warp & 3;
+        bool valid;
+        int t, local;
+        int64_t out_row;
+        bool active;
+        if (p.decode) {
+            local = q * p.rows_per_q + lane;
+            valid = lane < p.rows_per_q && local < p.group;
+            t = it.kv_len - 1;
+            const int head = it.g * p.group + local;
+            out_row = int64_t(it.b) * p.Hq + head;
+            active = q * p.rows_per_q < p.group;
+        } else {
+            local = 32 * q + lane;
+            valid = local < it.rows;
+            t = it.pos0 + local;
+            out_row = int64_t(it.q_row0 + local) * p.Hq + it.h;
+            active = 32 * q < it.rows;
+        }
+        const uint32_t lane_base = tmem_addr(tmem, 32 * q, 0);
+        const float cs = p.scale_log2;
+        const bool spill = p.decode && it.s0 > 0;
+        float m = -INFINITY, l = 0.0f;
+        float O[D];
+#pragma unroll
+        for (int j = 0; j < D; ++j) O[j] = 0.0f;
+        uint32_t s_phase = 0, o_phase = 0;
+        bool ok = true;
+
+        for (int s = it.s0; s < it.s1; ++s) {
+            const int k0 = s * kSplit;
+            if (!wait(barS, s_phase, ctl)) {
+                ok = false;
+                break;
+            }
+            s_phase ^= 1u;
+            tc_fence_after();
+            float m_s = -INFINITY, l_s = 0.0f;
+            if (active) {
+                uint32_t r[32];
+                // pass 1: the split's row maximum
+#pragma unroll 1
+                for (int c = 0; c < kSplit / 32; ++c) {
+                    tmem_ld32(lane_base + C::S_COL + 32 * c, r);
+                    tmem_wait_ld(r);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float x = __fmul_rn(__uint_as_float(r[j]), cs);
+                        if (k0 + 32 * c + j <= t) m_s = fmaxf(m_s, x);
+                    }
+                }
+                // pass 2: exponentials, their sum and P (bf16) into TMEM
+#pragma unroll 1
+                for (int c = 0; c < kSplit / 32; ++c) {
+                    tmem_ld32(lane_base + C::S_COL + 32 * c, r);
+                    tmem_wait_ld(r);
+                    float e[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float x = __fmul_rn(__uint_as_float(r[j]), cs);
+                        e[j] = (k0 + 32 * c + j <= t) ? ex2(__fsub_rn(x, m_s)) : 0.0f;
+                    }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(e[2 * j], e[2 * j + 1]);
+                    tmem_st16(lane_base + C::P_COL + 16 * c, pk);
+#pragma unroll
+                    for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+                        for (int j = 0; j < w; ++j) e[j] = __fadd_rn(e[j], e[j + w]);
+                    l_s = __fadd_rn(l_s, e[0]);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(barP);
+
+            if (!wait(barO, o_phase, ctl)) {
+                ok = false;
+                break;
+            }
+            o_phase ^= 1u;
+            tc_fence_after();
+            if (active) {
+                if (spill) {
+                    // not the first block of this sequence: write the
+                    // split's own partial for attn_combine
+                    float *rec = p.ws + ((out_row * p.max_splits) + s) * C::REC;
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t r[32];
+                        tmem_ld32(lane_base + C::O_COL + 32 * c, r);
+                        tmem_wait_ld(r);
+                        if (valid) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                reinterpret_cast<float4 *>(rec + 4 + 32 * c)[j] = make_float4(
+                                    __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                    __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+                        }
+                    }
+                    if (valid) {
+                        rec[0] = m_s;
+                        rec[1] = l_s;
+                    }
+                } else {
+                    const bool first = (s == 0);
+                    const bool take = k0 <= t;  // the row sees at least key k0
+                    float mn, a, cc;
+                    merge_scales(m, m_s, mn, a, cc);
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t r[32];
+                        tmem_ld32(lane_base + C::O_COL + 32 * c, r);
+                        tmem_wait_ld(r);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float os = __uint_as_float(r[j]);
+                            if (first)
+                                O[32 * c + j] = os;
+                            else if (take)
+                                O[32 * c + j] = merge_val(O[32 * c + j], a, os, cc);
+                        }
+                    }
+                    if (first) {
+                        m = m_s;
+                        l = l_s;
+                    } else if (take) {
+                        l = merge_val(l, a, l_s, cc);
+                        m = mn;
+                    }
+                }
+            }
+        }
+
+        if (ok && active && valid && !spill) {
+            if (!p.decode || it.s1 == it.n_splits) {
+                write_out<D>(O, l, m, static_cast<__nv_bfloat16 *>(p.o) + out_row * D,
+                             p.lse ? p.lse + out_row : nullptr);
+            } else {
+                // first block of a sequence served by several: hand the
+                // merged state over split s1-1 to attn_combine
+                float *rec = p.ws + ((out_row * p.max_splits) + (it.s1 - 1)) * C::REC;
+                rec[0] = m;
+                rec[1] = l;
+#pragma unroll
+                for (int j = 0; j < D / 4; ++j)
+                    reinterpret_cast<float4 *>(rec + 4)[j] =
+                        make_float4(O[4 * j], O[4 * j + 1], O[4 * j + 2], O[4 * j + 3]);
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// Continues the merge of a decode row past the first block's range, split by
+// split in ascending order; one warp per (sequence, query head).
+template <int D>
+__global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p)
+{
+    using C = Cfg<D>;
+    constexpr int PER = D / 32;  // columns per lane
+    const int64_t row = int64_t(blockIdx.x) * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= int64_t(p.B) * p.Hq) return;
+    const int b = static_cast<int>(row / p.Hq);
+    const int L = p.seq_lens[b];
+    const int n = (L + kSplit - 1) / kSplit;
+    const int first_end = p.splits_per_cta;  // splits merged by the first block
+    if (L <= 0 || n <= first_end) return;
+    const float *base = p.ws + row * p.max_splits * C::REC;
+    const float *rec = base + int64_t(first_end - 1) * C::REC;
+    float m = rec[0], l = rec[1];
+    float O[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) O[j] = rec[4 + lane * PER + j];
+    for (int s = first_end; s < n; ++s) {
+        rec = base + int64_t(s) * C::REC;
+        const float ms = rec[0], ls = rec[1];
+        float mn, a, cc;
+        merge_scales(m, ms, mn, a, cc);
+#pragma unroll
+        for (int j = 0; j < PER; ++j) O[j] = merge_val(O[j], a, rec[4 + lane * PER + j], cc);
+        l = merge_val(l, a, ls, cc);
+        m = mn;
+    }
+    __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.o) + row * D + lane * PER;
+#pragma unroll
+    for (int j = 0; j < PER; j += 2)
+        *reinterpret_cast<uint32_t *>(orow + j) = pack_bf16x2(__fdiv_rn(O[j], l), __fdiv_rn(O[j + 1], l));
+    if (p.lse && lane == 0) p.lse[row] = finish_lse(m, l);
+}
+
+}  // namespace
+
+size_t attn_smem_bytes(int head_dim) { return head_dim == 64 ? Cfg<64>::SMEM : Cfg<128>::SMEM; }
+
+size_t attn_ws_bytes(int B, int Hq, int head_dim, int max_splits, int max_chunks)
+{
+    if (max_chunks <= 1) return 0;
+    return size_t(B) * Hq * max_splits * (head_dim + 4) * sizeof(float);
+}
+
+cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                             const AttnParams &p, int head_dim, cudaStream_t s)
+{
+    dim3 grid;
+    if (p.decode)
+        grid = dim3((p.max_splits + p.splits_per_cta - 1) / p.splits_per_cta, p.Hkv, p.B);
+    else
+        grid = dim3(p.num_q_tiles, p.Hq, p.B);
+    cudaError_t e;
+    if (head_dim == 128) {
+        e = cudaFuncSetAttribute(attn_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<128>::SMEM);
+        if (e != cudaSuccess) return e;
+        attn_split_kernel<128><<<grid, THREADS, Cfg<128>::SMEM, s>>>(tq, tk, tv, p);
+    } else {
+        e = cudaFuncSetAttribute(attn_split_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<64>::SMEM);
+        if (e != cudaSuccess) return e;
+        attn_split_kernel<64><<<grid, THREADS, Cfg<64>::SMEM, s>>>(tq, tk, tv, p);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn_combine(const AttnParams &p, int head_dim, cudaStream_t s)
+{
+    const int64_t rows = int64_t(p.B) * p.Hq;
+    const unsigned blocks = static_cast<unsigned>((rows + 3) / 4);
+    if (head_dim == 128)
+        attn_combine_kernel<128><<<blocks, 128, 0, s>>>(p);
+    else
+        attn_combine_kernel<64><<<blocks, 128, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace bi

@@ -1,0 +1,71 @@
+// bi_launch.h -- host-side launchers of the kernels (internal to the library;
+// the public boundary is include/bi.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace bi {
+
+// ---------------------------------------------------------------- RMSNorm
+void rmsnorm_shape(int64_t H, int *items, int *threads);
+cudaError_t launch_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H,
+                           float eps, bool out_f32, int num_sms, cudaStream_t s);
+
+// ---------------------------------------------------------------- matmul
+constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64, kGemmStages = 4;
+size_t gemm_smem_bytes();
+// k_splits > 1 only in the variant-off build: fp32 partial sums go to ws
+// ([k_splits, M, N]) and a second kernel adds them.
+int gemm_k_splits(int64_t M, int64_t N, int64_t K, int num_sms);
+cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tw, void *c, int M, int N,
+                        int K, bool out_f32, float *ws, int k_splits, int num_sms,
+                        unsigned *status, uint64_t timeout_ns, cudaStream_t s);
+
+// ---------------------------------------------------------------- KV write
+cudaError_t launch_kv_write(void *k_cache, void *v_cache, int64_t num_pages, int Hkv, int d,
+                            const void *k_new, const void *v_new, const int64_t *slots,
+                            int64_t T, unsigned *status, cudaStream_t s);
+
+// ---------------------------------------------------------------- attention
+struct AttnParams {
+    // cache
+    const void *v_cache;       // read directly for the partial last page of V
+    const int32_t *block_table;
+    int32_t max_pages;
+    int32_t num_pages;
+    int32_t Hkv;
+    int32_t Hq;
+    int32_t group;         // Hq / Hkv
+    int32_t rows_per_q;    // decode: query rows per TMEM lane quarter
+    // mode
+    int32_t decode;        // 1 decode, 0 prefill
+    int32_t B;
+    const int32_t *seq_lens;   // decode
+    const int32_t *cu_q;       // prefill
+    const int32_t *ctx_lens;   // prefill
+    int32_t splits_per_cta;    // decode work division
+    int32_t max_splits;        // decode: splits of the longest sequence
+    int32_t num_q_tiles;       // prefill: tiles of the longest chunk
+    float scale_log2;          // softmax scale * log2(e)
+    // outputs
+    void *o;
+    float *lse;
+    float *ws;                 // decode split partials
+    unsigned *status;
+    uint64_t timeout_ns;
+};
+
+size_t attn_smem_bytes(int head_dim);
+size_t attn_ws_bytes(int B, int Hq, int head_dim, int max_splits, int max_chunks);
+cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                             const AttnParams &p, int head_dim, cudaStream_t s);
+cudaError_t launch_attn_combine(const AttnParams &p, int head_dim, cudaStream_t s);
+
+// ---------------------------------------------------------------- debug
+cudaError_t launch_bounded_wait_probe(unsigned *status, uint64_t timeout_ns, cudaStream_t s);
+
+}  // namespace bi

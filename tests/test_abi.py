@@ -1,0 +1,110 @@
+"""The C-ABI library loads and exports every entry point include/bi.h
+declares, and rejects bad arguments on the host before touching a device.
+CPU only: no call here reaches a kernel launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import invariant_bi_rmsnorm_03_b200 as bi
+from invariant_bi_rmsnorm_03_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bi.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bi_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module", params=[False, True], ids=["invariant", "variant_off"])
+def lib(request):
+    return bi.load(variant=request.param)
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for s in ("bi_rmsnorm", "bi_matmul", "bi_kv_write", "bi_attention_decode",
+              "bi_attention_prefill", "bi_device_status"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for s in declared_symbols():
+        assert hasattr(lib.lib, s), s
+        assert ctypes.cast(getattr(lib.lib, s), ctypes.c_void_p).value
+
+
+def test_build_flavour(lib):
+    want = 0 if lib.path.endswith("libbi_variant.so") else 1
+    assert lib.bi_build_invariant() == want
+
+
+def test_status_strings(lib):
+    for s in binding.Status:
+        assert lib.bi_status_string(int(s))
+    assert lib.bi_status_string(0) == "ok"
+
+
+P = ctypes.c_void_p
+FAKE = P(0x10000)  # a 16-byte aligned non-null value; never dereferenced
+
+
+def test_rmsnorm_rejects_bad_sizes(lib):
+    L = lib.lib
+    assert L.bi_rmsnorm(FAKE, FAKE, FAKE, 4, 12, 1e-6, 0, None) == binding.Status.INVALID   # H % 8
+    assert L.bi_rmsnorm(FAKE, FAKE, FAKE, -1, 64, 1e-6, 0, None) == binding.Status.INVALID
+    assert L.bi_rmsnorm(FAKE, FAKE, FAKE, 4, 64, 1e-6, 7, None) == binding.Status.INVALID   # dtype
+    assert L.bi_rmsnorm(FAKE, FAKE, FAKE, 4, 65544, 1e-6, 0, None) == binding.Status.INVALID
+    assert L.bi_rmsnorm(FAKE, FAKE, FAKE, 4, 64, float("nan"), 0, None) == binding.Status.INVALID
+    assert L.bi_rmsnorm(P(0x10008), FAKE, FAKE, 4, 64, 1e-6, 0, None) == binding.Status.INVALID
+    assert L.bi_rmsnorm(None, FAKE, FAKE, 4, 64, 1e-6, 0, None) == binding.Status.INVALID
+    assert L.bi_rmsnorm(None, None, None, 0, 64, 1e-6, 0, None) == binding.Status.OK  # M == 0
+
+
+def test_matmul_rejects_bad_sizes(lib):
+    L = lib.lib
+    assert L.bi_matmul(FAKE, FAKE, FAKE, 4, 12, 64, 0, None, 0, None) == binding.Status.INVALID
+    assert L.bi_matmul(FAKE, FAKE, FAKE, 4, 64, 12, 0, None, 0, None) == binding.Status.INVALID
+    assert L.bi_matmul(FAKE, FAKE, FAKE, 4, 0, 64, 0, None, 0, None) == binding.Status.INVALID
+    assert L.bi_matmul(None, FAKE, FAKE, 4, 64, 64, 0, None, 0, None) == binding.Status.INVALID
+    assert L.bi_matmul(None, None, None, 0, 64, 64, 0, None, 0, None) == binding.Status.OK
+
+
+def _kv(**over):
+    f = dict(k_cache=0x10000, v_cache=0x20000, block_table=0x30000, max_pages_per_seq=4,
+             num_pages=8, page_size=16, num_kv_heads=2, head_dim=128)
+    f.update(over)
+    return binding._PagedKV(**f)
+
+
+def test_attention_rejects_bad_layouts(lib):
+    L = lib.lib
+    dec = lambda kv, Hq=4, B=1, mx=32: L.bi_attention_decode(  # noqa: E731
+        ctypes.byref(kv), FAKE, FAKE, None, FAKE, B, Hq, mx, 0.1, 0, None, 0, None)
+    assert dec(_kv(page_size=8)) == binding.Status.INVALID
+    assert dec(_kv(), Hq=3) == binding.Status.INVALID               # Hq % Hkv
+    assert dec(_kv(head_dim=96)) == binding.Status.UNSUPPORTED
+    assert dec(_kv(k_cache=0x10004)) == binding.Status.INVALID       # alignment
+    assert dec(_kv(), mx=65) == binding.Status.INVALID               # > max_pages * 16
+    assert dec(_kv(), Hq=2 * 129) == binding.Status.INVALID          # group > 128
+    assert dec(_kv(), B=0) == binding.Status.OK
+    pre = lambda kv, Hq=4: L.bi_attention_prefill(  # noqa: E731
+        ctypes.byref(kv), FAKE, FAKE, None, FAKE, FAKE, 1, Hq, 16, 16, 0.1, None, 0, None)
+    assert pre(_kv(num_kv_heads=0)) == binding.Status.INVALID
+    assert pre(_kv(head_dim=32)) == binding.Status.UNSUPPORTED
+    assert L.bi_kv_write(ctypes.byref(_kv(page_size=32)), FAKE, FAKE, FAKE, 4, None) == \
+        binding.Status.INVALID
+
+
+def test_debug_wait_rejects_out_of_range_limits(lib):
+    assert lib.lib.bi_debug_bounded_wait(10, None) == binding.Status.INVALID
+    assert lib.lib.bi_debug_bounded_wait(10 ** 10, None) == binding.Status.INVALID
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(ImportError):
+        binding.Library(str(tmp_path / "libbi.so"))
