@@ -137,6 +137,10 @@ __device__ __forceinline__ bool make_item(const AttnParams &p, Item &it)
         it.kv_len = p.seq_lens[it.b];
         it.n_splits = (it.kv_len + kSplit - 1) / kSplit;
         it.s0 = blockIdx.x * p.splits_per_cta;
+        if (it.n_splits > p.max_splits) {  // longer than the declared maximum
+            if (threadIdx.x == 0 && blockIdx.x == 0) record_status(p.status, BI_DEV_BAD_INDEX);
+            return false;
+        }
         if (it.kv_len <= 0 || it.s0 >= it.n_splits) return false;
         it.s1 = min(it.n_splits, it.s0 + p.splits_per_cta);
         it.q_row0 = it.rows = it.pos0 = 0;
@@ -551,7 +555,7 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p)
     const int L = p.seq_lens[b];
     const int n = (L + kSplit - 1) / kSplit;
     const int first_end = p.splits_per_cta;  // splits merged by the first block
-    if (L <= 0 || n <= first_end) return;
+    if (L <= 0 || n <= first_end || n > p.max_splits) return;
     const float *base = p.ws + row * p.max_splits * C::REC;
     const float *rec = base + int64_t(first_end - 1) * C::REC;
     float m = rec[0], l = rec[1];

@@ -73,6 +73,8 @@ def test_decode_bits_do_not_depend_on_work_division(L):
     g = rng(23)
     lens = [5, 700, 2049, 4000, 300, 1]
     kv = paged_kv(g, lens, 4, 128)
+    kv.block_table = np.pad(kv.block_table, ((0, 0), (0, 600 - kv.block_table.shape[1])),
+                            constant_values=-1)
     q = dev_bf16(normal_bf16(g, (len(lens), 64, 128)))
     dkv, sl = dev_kv(kv), i32(kv.seq_lens)
     ref_o, ref_l = L.bi_attention_decode(dkv, q, sl, 4000, want_lse=True)
