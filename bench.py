@@ -1,0 +1,656 @@
+"""Benchmark of the batch-invariant forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole hot path over one batch of synthetic input,
+shaped like the serving workloads the reports describe:
+  * bi_kv_write   the step's new tokens into the paged caches (256 decode
+                  tokens; the 8192 prompt tokens of the prefill sequence)
+  * bi_rmsnorm    x[2048, 4096] (hidden 4096)
+  * bi_matmul     x[2048, 4096] @ W[12288, 4096]^T
+  * bi_attention_decode   256 requests, GQA 64/4, d=128, KV lengths
+                          U(1, 32768), shuffled 16-token pages, 256-key splits
+  * bi_attention_prefill  one causal 8192-token prompt, 32/8 heads, d=128
+The L2 cache (126 MB) is flushed between steps with a 512 MB write; each
+step is timed with CUDA events on the launching stream.
+
+``value`` is the batch-invariant GEMM throughput (TFLOP/s, all ranks'
+matmul FLOPs over the slowest rank's matmul time); ``split_kv_attn`` carries
+the decode attention's HBM throughput.  ``roofline`` is for the kernel that
+takes most of the step.  ``e2e`` repeats the measurement through the same
+public calls with the step's activations copied from pinned host memory and
+its results copied back inside the timed region.  ``cpu_baseline`` is the
+fp64 oracle timed on a bounded sample on this host's cores.
+``--impl reference`` times that oracle alone (the only other implementation
+of the method here) and prints its own line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "batch-invariant GEMM TFLOP/s + split-KV attn GB/s (% of peak); bitwise match"
+WORKLOAD = ("hidden-4096 RMSNorm + matmul (M=2048, N=12288) + paged decode attention "
+            "(B=256, GQA 64/4, d=128, KV U(1,32768)) + causal prefill (8192 tokens, 32/8 heads)")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL = {"hbm_gbs": 7700.0, "bf16_tflops": 2250.0}
+
+# Workload sizes.
+H, M_ROWS, N_COLS = 4096, 2048, 12288
+DEC_B, DEC_HQ, DEC_HKV, D = 256, 64, 4, 128
+DEC_MAXLEN = 32768
+PRE_S, PRE_HQ, PRE_HKV = 8192, 32, 8
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- workload
+
+class Workload:
+    """Device-resident inputs of one step (seeded, synthetic)."""
+
+    def __init__(self, torch, bi, dev, seed_base=0):
+        from synth import (decode_lengths, norm_matmul, normal_bf16, page_table, rng,
+                           slot_mapping, torch_normal_bf16)
+
+        self.torch = torch
+        T = torch
+        nm = norm_matmul(seed=1 + seed_base, M=M_ROWS, H=H, N=N_COLS)
+        self.x = T.from_numpy(nm["x"].view(np.int16)).to(dev).view(T.bfloat16)
+        self.w = T.from_numpy(nm["w"].view(np.int16)).to(dev).view(T.bfloat16)
+        self.W = T.from_numpy(nm["W"].view(np.int16)).to(dev).view(T.bfloat16)
+        self.eps = nm["eps"]
+        self.y = T.empty_like(self.x)
+        self.c = T.empty((M_ROWS, N_COLS), dtype=T.bfloat16, device=dev)
+        self.x_np, self.W_np, self.w_np = nm["x"], nm["W"], nm["w"]
+
+        # decode: lengths include the step's new token
+        g = rng(2 + seed_base)
+        lens = decode_lengths(2 + seed_base, DEC_B, DEC_MAXLEN)
+        bt, num_pages = page_table(g, lens, max_pages=DEC_MAXLEN // 16)
+        self.dec_lens_np, self.dec_bt_np = lens, bt
+        shape = (num_pages, DEC_HKV, 16, D)
+        self.dec_kv = bi.PagedKV(torch_normal_bf16(shape, 1000 + seed_base, dev),
+                                 torch_normal_bf16(shape, 2000 + seed_base, dev),
+                                 T.from_numpy(bt).to(dev))
+        self.dec_q = T.from_numpy(normal_bf16(g, (DEC_B, DEC_HQ, D)).view(np.int16)).to(dev).view(T.bfloat16)
+        self.dec_knew = T.from_numpy(normal_bf16(g, (DEC_B, DEC_HKV, D)).view(np.int16)).to(dev).view(T.bfloat16)
+        self.dec_vnew = T.from_numpy(normal_bf16(g, (DEC_B, DEC_HKV, D)).view(np.int16)).to(dev).view(T.bfloat16)
+        slots = np.array([slot_mapping(bt, b, [int(lens[b]) - 1])[0] for b in range(DEC_B)])
+        self.dec_slots = T.from_numpy(slots).to(dev)
+        self.dec_lens = T.from_numpy(lens).to(dev)
+        self.dec_o = T.empty_like(self.dec_q)
+        self.dec_ws_bytes = bi.load().bi_attention_decode_workspace_bytes(
+            self.dec_kv, DEC_B, DEC_HQ, DEC_MAXLEN)
+        self.dec_ws = T.empty(max(self.dec_ws_bytes, 16), dtype=T.uint8, device=dev)
+
+        # prefill: one prompt of PRE_S tokens into an empty (NaN) cache
+        gp = rng(3 + seed_base)
+        self.pre_q_np = normal_bf16(gp, (PRE_S, PRE_HQ, D))
+        self.pre_q = T.from_numpy(self.pre_q_np.view(np.int16)).to(dev).view(T.bfloat16)
+        self.pre_k = T.from_numpy(normal_bf16(gp, (PRE_S, PRE_HKV, D)).view(np.int16)).to(dev).view(T.bfloat16)
+        self.pre_v = T.from_numpy(normal_bf16(gp, (PRE_S, PRE_HKV, D)).view(np.int16)).to(dev).view(T.bfloat16)
+        pbt, pnp = page_table(gp, [PRE_S])
+        self.pre_bt_np = pbt
+        self.pre_kv = bi.PagedKV(T.full((pnp, PRE_HKV, 16, D), float("nan"), dtype=T.bfloat16, device=dev),
+                                 T.full((pnp, PRE_HKV, 16, D), float("nan"), dtype=T.bfloat16, device=dev),
+                                 T.from_numpy(pbt).to(dev))
+        self.pre_slots = T.from_numpy(slot_mapping(pbt, 0, np.arange(PRE_S))).to(dev)
+        self.pre_cu = T.tensor([0, PRE_S], dtype=T.int32, device=dev)
+        self.pre_ctx = T.tensor([0], dtype=T.int32, device=dev)
+        self.pre_o = T.empty_like(self.pre_q)
+
+        self.flush = T.empty(512 * 1024 * 1024, dtype=T.uint8, device=dev)
+
+        # algorithmic work per step
+        self.gemm_flops = 2.0 * M_ROWS * N_COLS * H
+        self.norm_bytes = 2.0 * M_ROWS * H * 2 + 2 * H
+        Lsum = float(lens.astype(np.int64).sum())
+        self.dec_bytes = (Lsum * DEC_HKV * D * 2 * 2            # K and V rows read once
+                          + 2.0 * DEC_B * DEC_HQ * D * 2          # q in, o out
+                          + 4.0 * float(((lens + 15) // 16).sum())  # block-table entries
+                          + 4.0 * DEC_B)                          # lengths
+        self.pre_flops = 4.0 * PRE_HQ * D * (PRE_S * (PRE_S + 1) / 2.0)
+        # new K and V rows read once and written once
+        self.kvw_bytes = 4.0 * D * 2 * (DEC_B * DEC_HKV + PRE_S * PRE_HKV)
+
+    def step(self, L, ev=None):
+        """One pass of the hot path.  ev: 7 CUDA events recorded between kernels."""
+        rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
+        rec(0)
+        L.bi_kv_write(self.dec_kv, self.dec_knew, self.dec_vnew, self.dec_slots)
+        L.bi_kv_write(self.pre_kv, self.pre_k, self.pre_v, self.pre_slots)
+        rec(1)
+        L.bi_rmsnorm(self.x, self.w, self.eps, out=self.y)
+        rec(2)
+        L.bi_matmul(self.y, self.W, out=self.c)
+        rec(3)
+        L.bi_attention_decode(self.dec_kv, self.dec_q, self.dec_lens, DEC_MAXLEN, out=self.dec_o,
+                              ws=self.dec_ws)
+        rec(4)
+        L.bi_attention_prefill(self.pre_kv, self.pre_q, self.pre_cu, self.pre_ctx, PRE_S,
+                               out=self.pre_o)
+        rec(5)
+
+    def launches_per_step(self, L) -> int:
+        ws = L.bi_attention_decode_workspace_bytes(self.dec_kv, DEC_B, DEC_HQ, DEC_MAXLEN)
+        return 2 + 1 + 1 + 1 + (1 if ws > 0 else 0) + 1
+
+
+# ---------------------------------------------------------------- clocks
+
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(index), "--query-gpu=" + self.Q,
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as fh:
+            for line in fh:
+                parts = [s.strip() for s in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        load = [s for s in sm if s > 0.5 * (max(mx) if mx else 1)] or sm
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- ours
+
+def timed_steps(torch, L, wl, steps, warmup, dist=None):
+    for _ in range(warmup):
+        wl.flush.zero_()
+        wl.step(L)
+    torch.cuda.synchronize()
+    per = np.zeros((steps, 5))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(steps):
+        wl.flush.zero_()
+        wl.step(L, evs[i])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    if dist is not None:
+        dist.barrier()
+    for i in range(steps):
+        e = evs[i]
+        per[i] = [e[j].elapsed_time(e[j + 1]) for j in range(5)]
+    return per, wall  # ms: kv_write, rmsnorm, matmul, decode, prefill
+
+
+def e2e_steps(torch, L, wl, steps, warmup):
+    """The same step through the public calls with host buffers: pinned host
+    activations copied in and results copied out inside the timed region."""
+    T = torch
+    hx = wl.x.cpu().pin_memory()
+    hq = wl.dec_q.cpu().pin_memory()
+    hkn, hvn = wl.dec_knew.cpu().pin_memory(), wl.dec_vnew.cpu().pin_memory()
+    hpq = wl.pre_q.cpu().pin_memory()
+    hpk, hpv = wl.pre_k.cpu().pin_memory(), wl.pre_v.cpu().pin_memory()
+    hc = T.empty(wl.c.shape, dtype=wl.c.dtype).pin_memory()
+    ho = T.empty(wl.dec_o.shape, dtype=wl.dec_o.dtype).pin_memory()
+    hpo = T.empty(wl.pre_o.shape, dtype=wl.pre_o.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hq, hkn, hvn, hpq, hpk, hpv))
+    d2h = sum(t.numel() * t.element_size() for t in (hc, ho, hpo))
+
+    def one(ev=None):
+        rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
+        rec(0)
+        wl.x.copy_(hx, non_blocking=True)
+        L.bi_rmsnorm(wl.x, wl.w, wl.eps, out=wl.y)
+        L.bi_matmul(wl.y, wl.W, out=wl.c)
+        hc.copy_(wl.c, non_blocking=True)
+        rec(1)
+        wl.dec_q.copy_(hq, non_blocking=True)
+        wl.dec_knew.copy_(hkn, non_blocking=True)
+        wl.dec_vnew.copy_(hvn, non_blocking=True)
+        L.bi_kv_write(wl.dec_kv, wl.dec_knew, wl.dec_vnew, wl.dec_slots)
+        L.bi_attention_decode(wl.dec_kv, wl.dec_q, wl.dec_lens, DEC_MAXLEN, out=wl.dec_o,
+                              ws=wl.dec_ws)
+        ho.copy_(wl.dec_o, non_blocking=True)
+        rec(2)
+        wl.pre_q.copy_(hpq, non_blocking=True)
+        wl.pre_k.copy_(hpk, non_blocking=True)
+        wl.pre_v.copy_(hpv, non_blocking=True)
+        L.bi_kv_write(wl.pre_kv, wl.pre_k, wl.pre_v, wl.pre_slots)
+        L.bi_attention_prefill(wl.pre_kv, wl.pre_q, wl.pre_cu, wl.pre_ctx, PRE_S, out=wl.pre_o)
+        hpo.copy_(wl.pre_o, non_blocking=True)
+        rec(3)
+
+    for _ in range(warmup):
+        wl.flush.zero_()
+        one()
+    torch.cuda.synchronize()
+    evs = [[T.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        wl.flush.zero_()
+        one(evs[i])
+    torch.cuda.synchronize()
+    per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(3)] for e in evs])
+    return per, h2d, d2h
+
+
+def invariance_checks(torch, L, wl) -> dict:
+    """Bitwise checks on the bench's own data: rows against smaller batches,
+    a request alone against the batch, the last prompt token in decode
+    against prefill."""
+    T = torch
+    eq = lambda a, b: bool(T.equal(a.contiguous().view(T.int16), b.contiguous().view(T.int16)))  # noqa: E731
+    out = {}
+    wl.step(L)
+    T.cuda.synchronize()
+    ok = True
+    for M in (1, 7, 128, 1000):
+        ok &= eq(L.bi_rmsnorm(wl.x[:M], wl.w, wl.eps), wl.y[:M])
+        ok &= eq(L.bi_matmul(wl.y[:M], wl.W), wl.c[:M])
+    out["gemm_rows_vs_batch"] = ok
+    ok = True
+    for b in (0, 17, 255):
+        kv1 = type(wl.dec_kv)(wl.dec_kv.k_cache, wl.dec_kv.v_cache,
+                              wl.dec_kv.block_table[b:b + 1].contiguous())
+        o1 = L.bi_attention_decode(kv1, wl.dec_q[b:b + 1].contiguous(), wl.dec_lens[b:b + 1],
+                                   int(wl.dec_lens_np[b]))
+        ok &= eq(o1[0], wl.dec_o[b])
+    out["decode_request_vs_batch"] = ok
+    t = PRE_S - 1
+    od = L.bi_attention_decode(wl.pre_kv, wl.pre_q[t:t + 1].contiguous(),
+                               T.tensor([PRE_S], dtype=T.int32, device=wl.x.device), PRE_S)
+    out["decode_vs_prefill"] = eq(od[0], wl.pre_o[t])
+    out["all"] = all(out.values())
+    return out
+
+
+def cpu_baseline(wl, budget_s: float = 20.0) -> dict:
+    """The oracle (fp64, OpenMP) on a bounded sample of the same workload."""
+    import oracle
+
+    cores = oracle.num_threads()
+    # matmul: rows of the step's x (after RMSNorm, which the oracle recomputes)
+    t0 = time.perf_counter()
+    rows = 0
+    while time.perf_counter() - t0 < budget_s / 2 and rows < M_ROWS:
+        xs = wl.x_np[rows:rows + 8]
+        oracle.matmul(xs, wl.W_np)
+        rows += xs.shape[0]
+    tg = time.perf_counter() - t0
+    gemm_tflops = 2.0 * rows * N_COLS * H / tg / 1e12
+    # decode attention: whole requests of the batch (device-to-host copies untimed)
+    import torch
+
+    kc, vc = wl.dec_kv.k_cache, wl.dec_kv.v_cache
+    tstart = time.perf_counter()
+    ta, done, nbytes = 0.0, 0, 0.0
+    order = np.argsort(wl.dec_lens_np)
+    while time.perf_counter() - tstart < budget_s / 2 and done < 16:
+        b = int(order[(done * 16) % DEC_B])
+        Lb = int(wl.dec_lens_np[b])
+        pages = wl.dec_bt_np[b, :(Lb + 15) // 16].tolist()
+        k = kc[pages].view(torch.int16).cpu().numpy().view(np.uint16)
+        v = vc[pages].view(torch.int16).cpu().numpy().view(np.uint16)
+        bt = np.arange(len(pages), dtype=np.int32)[None, :]
+        q = wl.dec_q[b].view(torch.int16).cpu().numpy().view(np.uint16)
+        ts = time.perf_counter()
+        oracle.attention(q, np.zeros(DEC_HQ), np.arange(DEC_HQ), np.full(DEC_HQ, Lb - 1), DEC_HQ,
+                         k, v, bt)
+        ta += time.perf_counter() - ts
+        nbytes += Lb * DEC_HKV * D * 4.0 + 2 * DEC_HQ * D * 2
+        done += 1
+    return {"value": gemm_tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": "matmul: %d of %d rows of x[2048,4096] times W[12288,4096]^T; decode: %d "
+                      "whole requests of the batch" % (rows, M_ROWS, done),
+            "split_kv_attn_gbs": nbytes / ta / 1e9 if ta > 0 else None}
+
+
+def traffic_record(kernel_src: str, name: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    rec = d.get(name)
+    if not rec:
+        return None
+    with open(os.path.join(ROOT, "invariant_bi_rmsnorm_03_b200", "csrc", kernel_src), "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    if rec.get("source_sha") != sha:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def run_ours(args):
+    import torch
+
+    import invariant_bi_rmsnorm_03_b200 as bi
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as td
+
+        torch.cuda.set_device(local)
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = td
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    L = bi.load()
+    wl = Workload(torch, bi, dev, seed_base=0)
+    launches = wl.launches_per_step(L)
+
+    clocks = Clocks(local)
+    per, wall = timed_steps(torch, L, wl, args.steps, args.warmup, dist)
+    clk = clocks.stop()
+    mean = per.mean(axis=0)  # ms per kernel group
+    step_ms = float(per.sum(axis=1).mean())
+
+    # whole-job figures: all ranks' work over the slowest rank's time
+    def maxall(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    gemm_ms = maxall(float(mean[2]))
+    dec_ms = maxall(float(mean[3]))
+    pre_ms = maxall(float(mean[4]))
+    norm_ms = maxall(float(mean[1]))
+    kvw_ms = maxall(float(mean[0]))
+    step_ms = maxall(step_ms)
+    gemm_tf = world * wl.gemm_flops / (gemm_ms * 1e-3) / 1e12
+    dec_gbs = world * wl.dec_bytes / (dec_ms * 1e-3) / 1e9
+
+    # e2e through host buffers
+    e2e_per, h2d, d2h = e2e_steps(torch, L, wl, max(2, args.steps // 2), 1)
+    e2e_gemm_ms = maxall(float(e2e_per[:, 0].mean()))
+    e2e_dec_ms = maxall(float(e2e_per[:, 1].mean()))
+
+    # variant-off build on the same step (the cost of invariance)
+    Lv = bi.load(variant=True)
+    wl_v_ws = Lv.bi_attention_decode_workspace_bytes(wl.dec_kv, DEC_B, DEC_HQ, DEC_MAXLEN)
+    if wl_v_ws > wl.dec_ws.numel():
+        wl.dec_ws = torch.empty(wl_v_ws, dtype=torch.uint8, device=dev)
+    per_v, _ = timed_steps(torch, Lv, wl, max(3, args.steps // 2), 2, dist)
+    mean_v = per_v.mean(axis=0)
+    names = ["kv_write", "rmsnorm", "matmul", "attention_decode", "attention_prefill"]
+    overhead = {n: float(mean[i] / mean_v[i] - 1.0) for i, n in enumerate(names)}
+    overhead["step"] = float(per.sum(axis=1).mean() / per_v.sum(axis=1).mean() - 1.0)
+
+    checks = invariance_checks(torch, L, wl)
+
+    if rank != 0:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return None
+
+    pk, src = peaks()
+    dec_traffic = traffic_record("attention.cu", "attn_split_kernel<128>/decode")
+    kernels = {
+        "bi_kv_write": {"ms": float(mean[0]), "GB/s": wl.kvw_bytes / (mean[0] * 1e-3) / 1e9},
+        "bi_rmsnorm": {"ms": float(mean[1]), "GB/s": wl.norm_bytes / (mean[1] * 1e-3) / 1e9,
+                       "frac_hbm": wl.norm_bytes / (mean[1] * 1e-3) / 1e9 / pk["hbm_gbs"]},
+        "bi_matmul": {"ms": float(mean[2]), "TFLOP/s": wl.gemm_flops / (mean[2] * 1e-3) / 1e12,
+                      "frac_bf16": wl.gemm_flops / (mean[2] * 1e-3) / 1e12 / pk["bf16_tflops"]},
+        "bi_attention_decode": {"ms": float(mean[3]), "GB/s": wl.dec_bytes / (mean[3] * 1e-3) / 1e9,
+                                "frac_hbm": wl.dec_bytes / (mean[3] * 1e-3) / 1e9 / pk["hbm_gbs"]},
+        "bi_attention_prefill": {"ms": float(mean[4]),
+                                 "TFLOP/s": wl.pre_flops / (mean[4] * 1e-3) / 1e12,
+                                 "frac_bf16": wl.pre_flops / (mean[4] * 1e-3) / 1e12 / pk["bf16_tflops"]},
+    }
+    # dominant kernel of the step
+    dom = int(np.argmax(mean))
+    if dom == 3:
+        ach = wl.dec_bytes / (mean[3] * 1e-3) / 1e9
+        roof = {"kernel": "bi_attention_decode", "bound": "hbm", "achieved": ach,
+                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
+                "traffic": dec_traffic, "algorithmic_bytes": wl.dec_bytes,
+                "peak_source": src + " (copy bandwidth)"}
+    elif dom == 4:
+        ach = wl.pre_flops / (mean[4] * 1e-3) / 1e12
+        roof = {"kernel": "bi_attention_prefill", "bound": "tensor", "achieved": ach,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
+                "traffic": None, "algorithmic_flops": wl.pre_flops,
+                "peak_source": src + " (cuBLAS bf16, burst)"}
+    else:
+        ach = wl.gemm_flops / (mean[2] * 1e-3) / 1e12
+        roof = {"kernel": "bi_matmul", "bound": "tensor", "achieved": ach,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
+                "traffic": None, "algorithmic_flops": wl.gemm_flops,
+                "peak_source": src + " (cuBLAS bf16, burst)"}
+    cpu = cpu_baseline(wl, budget_s=args.cpu_budget)
+    line = {
+        "metric": METRIC,
+        "value": gemm_tf,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "hidden": H, "M": M_ROWS, "N": N_COLS,
+                   "decode": {"B": DEC_B, "Hq": DEC_HQ, "Hkv": DEC_HKV, "d": D,
+                              "kv_len": "U(1,32768)", "page": 16, "split": 256},
+                   "prefill": {"S": PRE_S, "Hq": PRE_HQ, "Hkv": PRE_HKV, "d": D},
+                   "l2": "flushed between steps (512 MB write)", "parallelism": "replicas"},
+        "split_kv_attn": {"value": dec_gbs, "unit": "GB/s", "frac": dec_gbs / world / pk["hbm_gbs"],
+                          "peak": pk["hbm_gbs"]},
+        "bitwise_match": checks,
+        "roofline": roof,
+        "kernels": kernels,
+        "overhead_vs_variant_off": overhead,
+        "e2e": {"value": world * wl.gemm_flops / (e2e_gemm_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "split_kv_attn_gbs": world * wl.dec_bytes / (e2e_dec_ms * 1e-3) / 1e9},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+        "peaks": {"source": src, **pk, "nominal_hbm_gbs": NOMINAL["hbm_gbs"],
+                  "nominal_bf16_tflops": NOMINAL["bf16_tflops"]},
+        "wall_s_timed_region": wall,
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The fp64 oracle, as it stands, on this host's cores: each step is a
+    bounded sample of the same workload (8 rows of the matmul)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    import oracle
+    from synth import norm_matmul
+
+    nm = norm_matmul(seed=1, M=M_ROWS, H=H, N=N_COLS)
+    x, W = nm["x"], nm["W"]
+    rows_per_step = 8
+
+    def step(i):
+        r0 = (i * rows_per_step) % M_ROWS
+        oracle.matmul(x[r0:r0 + rows_per_step], W)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * rows_per_step * N_COLS * H * args.steps
+    val = flops / dt / 1e12
+    sample = "%d rows of x[2048,4096] times W[12288,4096]^T per step" % rows_per_step
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": val,
+        "unit": "TFLOP/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "hidden": H, "M": M_ROWS, "N": N_COLS},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return line
+
+
+# ---------------------------------------------------------------- profiling cases
+
+def run_profile_case(args):
+    """Runs one kernel alone on a reduced case (inputs above L2, a few GB at
+    most) for ncu captures: --profile {rmsnorm,matmul,decode,prefill}."""
+    import torch
+
+    import invariant_bi_rmsnorm_03_b200 as bi
+    from synth import (decode_lengths, norm_matmul, normal_bf16, page_table, rng,
+                       slot_mapping, torch_normal_bf16)
+
+    dev = torch.device("cuda", 0)
+    L = bi.load(variant=args.variant)
+    T = torch
+    d16 = lambda a: T.from_numpy(a.view(np.int16)).to(dev).view(T.bfloat16)  # noqa: E731
+    if args.profile in ("rmsnorm", "matmul"):
+        nm = norm_matmul(seed=1, M=M_ROWS, H=H, N=N_COLS)
+        x, w, W = d16(nm["x"]), d16(nm["w"]), d16(nm["W"])
+        if args.profile == "rmsnorm":
+            # 16 row-blocks of 2048 x 4096 rotate through 268 MB (> L2)
+            xs = [d16(norm_matmul(seed=10 + i, M=M_ROWS, H=H, N=8)["x"]) for i in range(16)]
+            fn = lambda i: L.bi_rmsnorm(xs[i % 16], w, 1e-6)  # noqa: E731
+        else:
+            fn = lambda i: L.bi_matmul(x, W)  # noqa: E731
+    elif args.profile == "decode":
+        B = args.profile_batch
+        g = rng(2)
+        lens = decode_lengths(2, B, DEC_MAXLEN)
+        bt, num_pages = page_table(g, lens, max_pages=DEC_MAXLEN // 16)
+        shape = (num_pages, DEC_HKV, 16, D)
+        kv = bi.PagedKV(torch_normal_bf16(shape, 1000, dev), torch_normal_bf16(shape, 2000, dev),
+                        T.from_numpy(bt).to(dev))
+        q = d16(normal_bf16(g, (B, DEC_HQ, D)))
+        sl = T.from_numpy(lens).to(dev)
+        fn = lambda i: L.bi_attention_decode(kv, q, sl, DEC_MAXLEN)  # noqa: E731
+    else:
+        gp = rng(3)
+        S = args.profile_seq
+        q = d16(normal_bf16(gp, (S, PRE_HQ, D)))
+        k = d16(normal_bf16(gp, (S, PRE_HKV, D)))
+        v = d16(normal_bf16(gp, (S, PRE_HKV, D)))
+        pbt, pnp = page_table(gp, [S])
+        kv = bi.PagedKV(T.zeros((pnp, PRE_HKV, 16, D), dtype=T.bfloat16, device=dev),
+                        T.zeros((pnp, PRE_HKV, 16, D), dtype=T.bfloat16, device=dev),
+                        T.from_numpy(pbt).to(dev))
+        L.bi_kv_write(kv, k, v, T.from_numpy(slot_mapping(pbt, 0, np.arange(S))).to(dev))
+        cu = T.tensor([0, S], dtype=T.int32, device=dev)
+        ctx = T.tensor([0], dtype=T.int32, device=dev)
+        fn = lambda i: L.bi_attention_prefill(kv, q, cu, ctx, S)  # noqa: E731
+    for i in range(args.warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    ev = [T.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    for i in range(args.steps):
+        ev[i].record()
+        fn(i)
+    ev[-1].record()
+    torch.cuda.synchronize()
+    ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    print(json.dumps({"profile": args.profile, "ms": ms, "status": int(L.bi_device_status())}))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=20.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--profile", choices=["rmsnorm", "matmul", "decode", "prefill"],
+                    help="run one kernel alone on a reduced case (for ncu)")
+    ap.add_argument("--profile-batch", type=int, default=32)
+    ap.add_argument("--profile-seq", type=int, default=4096)
+    ap.add_argument("--variant", action="store_true", help="--profile the variant-off build")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.profile:
+        run_profile_case(args)
+    elif args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -402,7 +402,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         const uint32_t lane_base = tmem_addr(tmem, 32 * q, 0);
         const float cs = p.scale_log2;
+#if BI_INVARIANT
+        // blocks after a sequence's first write every split's own partial
         const bool spill = p.decode && it.s0 > 0;
+#else
+        // variant-off: every block merges its own range (the grouping of the
+        // merge then depends on how many blocks served the sequence)
+        const bool spill = false;
+#endif
         float m = -INFINITY, l = 0.0f;
         float O[D];
 #pragma unroll
@@ -487,7 +494,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         rec[1] = l_s;
                     }
                 } else {
-                    const bool first = (s == 0);
+                    const bool first = (s == it.s0);
                     const bool take = k0 <= t;  // the row sees at least key k0
                     float mn, a, cc;
                     merge_scales(m, m_s, mn, a, cc);
@@ -562,8 +569,14 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p)
     float O[PER];
 #pragma unroll
     for (int j = 0; j < PER; ++j) O[j] = rec[4 + lane * PER + j];
+#if BI_INVARIANT
     for (int s = first_end; s < n; ++s) {
         rec = base + int64_t(s) * C::REC;
+#else
+    // variant-off: one record per block, at the block's last split
+    for (int e = 2 * first_end; e < n + first_end; e += first_end) {
+        rec = base + int64_t(min(e, n) - 1) * C::REC;
+#endif
         const float ms = rec[0], ls = rec[1];
         float mn, a, cc;
         merge_scales(m, ms, mn, a, cc);
