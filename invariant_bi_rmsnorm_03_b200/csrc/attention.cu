@@ -70,7 +70,9 @@ struct Cfg {
     static constexpr int NSLOT = 3;
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM = 1024 + Q_BYTES + NSLOT * KV_BYTES + BAR_BYTES;
-    static constexpr uint32_t S_COL = 0, P_COL = 256, O_COL = 384, TMEM_COLS = 512;
+    // TMEM: two buffers of 256 columns.  In buffer b: S over all 256
+    // columns; P (bf16 pairs) written over its first 128; O_s in the next D.
+    static constexpr uint32_t BUF_COLS = 256, P_OFF = 0, O_OFF = 128, TMEM_COLS = 512;
     static constexpr int REC = D + 4;                   // floats per spilled partial
 };
 
@@ -173,6 +175,82 @@ __device__ __forceinline__ uint32_t swz(int r, int c)
 
 // ---------------------------------------------------------------- kernel
 
+// 32 + 32 columns of one lane quarter into two register arrays, one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r0)[32], uint32_t (&r1)[32])
+{
+    tmem_ld32(taddr, r0);
+    tmem_ld32(taddr + 32, r1);
+    tmem_wait_ld(r0);
+    tmem_wait_ld(r1);
+}
+
+// Softmax of one split for the row owned by this thread.  S is read from
+// TMEM columns sb .. sb+255 in two passes; P (bf16 pairs) is written over
+// columns sb .. sb+127 as the second pass goes (each store lands on columns
+// this thread has already read).  Returns m_s (scaled, log2 units) and l_s.
+__device__ __forceinline__ void split_softmax(uint32_t sb, int k0, int t, float cs, float &m_s,
+                                              float &l_s)
+{
+    // pass 1: maximum of the raw logits over the visible keys.  For c > 0,
+    // x -> round(x * c) is monotonic, so max_j round(S_j c) = round(max_j S_j * c).
+    float mraw = -INFINITY;
+#pragma unroll 1
+    for (int c = 0; c < kSplit / 32; c += 2) {
+        uint32_t r0[32], r1[32];
+        tmem_ld64(sb + 32 * c, r0, r1);
+        const int kc = k0 + 32 * c;
+        if (kc + 63 <= t) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) mraw = fmaxf(mraw, __uint_as_float(r0[j]));
+#pragma unroll
+            for (int j = 0; j < 32; ++j) mraw = fmaxf(mraw, __uint_as_float(r1[j]));
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (kc + j <= t) mraw = fmaxf(mraw, __uint_as_float(r0[j]));
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (kc + 32 + j <= t) mraw = fmaxf(mraw, __uint_as_float(r1[j]));
+        }
+    }
+    m_s = __fmul_rn(mraw, cs);
+    // pass 2: p = 2^(round(S c) - m_s), masked keys 0; 32-key chunk sums by a
+    // pairwise tree, added to l_s chunk by chunk in key order.
+    float l = 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < kSplit / 32; c += 2) {
+        uint32_t r[2][32];
+        tmem_ld64(sb + 32 * c, r[0], r[1]);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int kc = k0 + 32 * (c + h);
+            float e[32];
+            if (kc + 31 <= t) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    e[j] = ex2(__fsub_rn(__fmul_rn(__uint_as_float(r[h][j]), cs), m_s));
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    e[j] = (kc + j <= t)
+                               ? ex2(__fsub_rn(__fmul_rn(__uint_as_float(r[h][j]), cs), m_s))
+                               : 0.0f;
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(e[2 * j], e[2 * j + 1]);
+            tmem_st16(sb + 16 * (c + h), pk);
+#pragma unroll
+            for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+                for (int j = 0; j < w; ++j) e[j] = __fadd_rn(e[j], e[j + w]);
+            l = __fadd_rn(l, e[0]);
+        }
+    }
+    tmem_wait_st();
+    l_s = l;
+}
+
 template <int D>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_split_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -190,10 +268,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint64_t *full = reinterpret_cast<uint64_t *>(sKV + C::NSLOT * C::KV_BYTES);
     uint64_t *empty = full + C::NSLOT;
     uint64_t *barQ = empty + C::NSLOT;
-    uint64_t *barS = barQ + 1;
-    uint64_t *barP = barS + 1;
-    uint64_t *barO = barP + 1;
-    uint64_t *drain = barO + 1;
+    uint64_t *barS = barQ + 1;     // [2] S of buffer b computed
+    uint64_t *barP = barS + 2;     // [2] P of buffer b written (128 arrivals)
+    uint64_t *barO = barP + 2;     // [2] O_s of buffer b computed
+    uint64_t *barF = barO + 2;     // [2] buffer b free again (128 arrivals)
+    uint64_t *drain = barF + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
@@ -204,9 +283,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(barQ, 1);
-        mbar_init(barS, 1);
-        mbar_init(barP, 128);
-        mbar_init(barO, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&barS[b], 1);
+            mbar_init(&barP[b], 128);
+            mbar_init(&barO[b], 1);
+            mbar_init(&barF[b], 128);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -224,6 +306,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp == 0) {
         // ====================================================== producer
+        // Loads in the order K(s0), V(s0), K(s0+1), V(s0+1), ...; load i
+        // goes to ring slot i % NSLOT.
         bool ok = true;
         uint32_t armed = 0, armed_parity = 0;
         if (lane == 0) {
@@ -240,12 +324,29 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tma_load_3d(sQ + kb * C::Q_KB_BYTES, &tq, barQ, kb * 64, it.h, it.q_row0);
             }
         }
+        // Lane i < 16 looks up page i of a split, one split ahead, and
+        // issues that page's boxes itself.
+        auto lookup = [&](int s) -> int {
+            const int lp = s * (kSplit / kPage) + lane;  // logical page
+            if (lane >= kSplit / kPage || lp * kPage >= it.kv_len) return -1;
+            const int phys = lp < p.max_pages ? __ldg(bt_row + lp) : -1;
+            if (phys < 0 || phys >= p.num_pages) {
+                record_status(p.status, BI_DEV_BAD_INDEX);
+                return -1;
+            }
+            return phys;
+        };
         int slot = 0;
         uint32_t phase = 0;
+        int phys_next = it.s0 < it.s1 ? lookup(it.s0) : -1;
         for (int s = it.s0; ok && s < it.s1; ++s) {
+            const int phys = phys_next;
+            if (s + 1 < it.s1) phys_next = lookup(s + 1);
             const int nk = min(kSplit, it.kv_len - s * kSplit);  // valid keys, >= 1
             const int full_pages = nk / kPage;
             const int npages = (nk + kPage - 1) / kPage;
+            // box row of this lane's page; -16 = out of bounds, zero filled
+            const int row = phys >= 0 ? (phys * p.Hkv + it.g) * kPage : -kPage;
             for (int which = 0; which < 2; ++which) {  // 0: K, 1: V
                 int got = 1;
                 if (lane == 0) got = wait(&empty[slot], phase ^ 1u, ctl) ? 1 : 0;
@@ -256,14 +357,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 uint8_t *dst = sKV + slot * C::KV_BYTES;
                 const CUtensorMap *map = which ? &tv : &tk;
+                const int partial_phys = __shfl_sync(0xffffffffu, phys, full_pages & 31);
                 // V: the partial last page is copied by the whole warp, with
                 // the rows past the sequence end set to zero.
                 if (which == 1 && full_pages < npages) {
                     const int pg = full_pages;
-                    const int lp = s * (kSplit / kPage) + pg;  // logical page
-                    const int phys = lp < p.max_pages ? __ldg(bt_row + lp) : -1;
-                    const bool good = phys >= 0 && phys < p.num_pages;
-                    if (!good && lane == 0) record_status(p.status, BI_DEV_BAD_INDEX);
+                    const bool good = partial_phys >= 0;
                     const int valid = nk - pg * kPage;
                     for (int i = lane; i < kPage * C::KB * 8; i += 32) {
                         const int r = i / (C::KB * 8);
@@ -271,8 +370,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                         const int c = i % 8;
                         uint4 v = make_uint4(0, 0, 0, 0);
                         if (good && r < valid) {
-                            const int64_t src = ((int64_t(phys) * p.Hkv + it.g) * kPage + r) * D +
-                                                kb * 64 + c * 8;
+                            const int64_t src =
+                                ((int64_t(partial_phys) * p.Hkv + it.g) * kPage + r) * D + kb * 64 +
+                                c * 8;
                             v = __ldg(reinterpret_cast<const uint4 *>(
                                 static_cast<const __nv_bfloat16 *>(p.v_cache) + src));
                         }
@@ -282,29 +382,28 @@ __global__ void __launch_bounds__(THREADS, 1)
                     fence_proxy_async_smem();
                     __syncwarp();
                 }
+                // K: the pages holding valid keys.  V: whole valid pages plus
+                // all-zero (out-of-bounds) boxes for the pages past the end.
+                const int tma_pages = which ? (kSplit / kPage) - (npages - full_pages) : npages;
                 if (lane == 0) {
-                    // K: pages holding valid keys.  V: whole valid pages, plus
-                    // all-zero (out-of-bounds) boxes for pages past the end.
-                    const int tma_pages = which ? (kSplit / kPage) - (npages - full_pages) : npages;
                     mbar_arrive_expect_tx(&full[slot], uint32_t(tma_pages) * C::KB * C::PAGE_KB_BYTES);
-                    const int last = which ? (kSplit / kPage) : npages;
-                    for (int pg = 0; pg < last; ++pg) {
-                        if (which && pg == full_pages && full_pages < npages) continue;
-                        int row = -kPage;  // out of bounds: zero fill
-                        if (pg < (which ? full_pages : npages)) {
-                            const int lp = s * (kSplit / kPage) + pg;
-                            const int phys = lp < p.max_pages ? __ldg(bt_row + lp) : -1;
-                            if (phys >= 0 && phys < p.num_pages)
-                                row = (phys * p.Hkv + it.g) * kPage;
-                            else
-                                record_status(p.status, BI_DEV_BAD_INDEX);
-                        }
-                        for (int kb = 0; kb < C::KB; ++kb)
-                            tma_load_2d(dst + kb * C::KV_KB_BYTES + pg * C::PAGE_KB_BYTES, map,
-                                        &full[slot], kb * 64, row);
-                    }
                     armed |= 1u << slot;
                     armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
+                }
+                __syncwarp();
+                const int pg = lane;
+                bool issue;
+                int r = row;
+                if (which == 0) {
+                    issue = pg < npages;
+                } else {
+                    issue = pg < kSplit / kPage && !(pg == full_pages && full_pages < npages);
+                    if (pg >= full_pages) r = -kPage;  // past the end: zero box
+                }
+                if (issue) {
+                    for (int kb = 0; kb < C::KB; ++kb)
+                        tma_load_2d(dst + kb * C::KV_KB_BYTES + pg * C::PAGE_KB_BYTES, map,
+                                    &full[slot], kb * 64, r);
                 }
                 __syncwarp();
                 if (++slot == C::NSLOT) {
@@ -320,58 +419,65 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else if (warp == 1) {
         // ====================================================== MMA issue
+        // Tensor-pipe order: QK(s0), QK(s0+1), PV(s0), QK(s0+2), PV(s0+1),
+        // ... so that S of the next split is ready while a split's softmax
+        // runs.  Split s uses TMEM buffer (s - s0) & 1.
         if (lane == 0) {
             const uint32_t idesc_qk = idesc_bf16_f32(128, kSplit, 0, 0);
             const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t q_base = smem_u32(sQ);
             bool ok = wait(barQ, 0, ctl);
-            int slot = 0;
-            uint32_t phase = 0, p_phase = 0;
-            for (int s = it.s0; ok && s < it.s1; ++s) {
-                // S = Q K^T
-                if (!wait(&full[slot], phase, ctl)) {
-                    ok = false;
-                    break;
-                }
+            auto issue_qk = [&](int s) -> bool {
+                const int i = 2 * (s - it.s0);
+                const int slot = i % C::NSLOT;
+                if (!wait(&full[slot], uint32_t(i / C::NSLOT) & 1u, ctl)) return false;
                 tc_fence_after();
+                const uint32_t d = tmem + C::BUF_COLS * uint32_t((s - it.s0) & 1);
                 const uint32_t k_base = smem_u32(sKV + slot * C::KV_BYTES);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t kb = k >> 2, kk = k & 3;
-                    mma_ss(tmem + C::S_COL,
-                           sdesc_sw128(q_base + kb * C::Q_KB_BYTES + kk * 32, 16, 1024),
+                    mma_ss(d, sdesc_sw128(q_base + kb * C::Q_KB_BYTES + kk * 32, 16, 1024),
                            sdesc_sw128(k_base + kb * C::KV_KB_BYTES + kk * 32, 16, 1024), idesc_qk,
                            k > 0 ? 1u : 0u);
                 }
-                mma_commit(barS);
+                mma_commit(&barS[(s - it.s0) & 1]);
                 mma_commit(&empty[slot]);
-                if (++slot == C::NSLOT) {
-                    slot = 0;
-                    phase ^= 1u;
-                }
-                // O_s = P V
-                if (!wait(barP, p_phase, ctl)) {
+                return true;
+            };
+            if (ok) ok = issue_qk(it.s0);
+            if (ok && it.s0 + 1 < it.s1) ok = issue_qk(it.s0 + 1);
+            for (int s = it.s0; ok && s < it.s1; ++s) {
+                const int b = (s - it.s0) & 1;
+                const uint32_t par = uint32_t((s - it.s0) >> 1) & 1u;
+                if (!wait(&barP[b], par, ctl)) {
                     ok = false;
                     break;
                 }
-                p_phase ^= 1u;
-                if (!wait(&full[slot], phase, ctl)) {
+                const int i = 2 * (s - it.s0) + 1;
+                const int slot = i % C::NSLOT;
+                if (!wait(&full[slot], uint32_t(i / C::NSLOT) & 1u, ctl)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t buf = tmem + C::BUF_COLS * uint32_t(b);
                 const uint32_t v_base = smem_u32(sKV + slot * C::KV_BYTES);
 #pragma unroll
-                for (int i = 0; i < kSplit / 16; ++i) {
-                    mma_ts(tmem + C::O_COL, tmem + C::P_COL + 8 * i,
-                           sdesc_sw128(v_base + i * 16 * 128, C::KV_KB_BYTES, 1024), idesc_pv,
-                           i > 0 ? 1u : 0u);
+                for (int j = 0; j < kSplit / 16; ++j) {
+                    mma_ts(buf + C::O_OFF, buf + C::P_OFF + 8 * j,
+                           sdesc_sw128(v_base + j * 16 * 128, C::KV_KB_BYTES, 1024), idesc_pv,
+                           j > 0 ? 1u : 0u);
                 }
-                mma_commit(barO);
+                mma_commit(&barO[b]);
                 mma_commit(&empty[slot]);
-                if (++slot == C::NSLOT) {
-                    slot = 0;
-                    phase ^= 1u;
+                if (s + 2 < it.s1) {
+                    if (!wait(&barF[b], par, ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    ok = issue_qk(s + 2);
                 }
             }
             if (!ok) {
@@ -414,62 +520,27 @@ __global__ void __launch_bounds__(THREADS, 1)
         float O[D];
 #pragma unroll
         for (int j = 0; j < D; ++j) O[j] = 0.0f;
-        uint32_t s_phase = 0, o_phase = 0;
         bool ok = true;
 
         for (int s = it.s0; s < it.s1; ++s) {
+            const int b = (s - it.s0) & 1;
+            const uint32_t par = uint32_t((s - it.s0) >> 1) & 1u;
+            const uint32_t sb = lane_base + C::BUF_COLS * uint32_t(b);
             const int k0 = s * kSplit;
-            if (!wait(barS, s_phase, ctl)) {
+            if (!wait(&barS[b], par, ctl)) {
                 ok = false;
                 break;
             }
-            s_phase ^= 1u;
             tc_fence_after();
             float m_s = -INFINITY, l_s = 0.0f;
-            if (active) {
-                uint32_t r[32];
-                // pass 1: the split's row maximum
-#pragma unroll 1
-                for (int c = 0; c < kSplit / 32; ++c) {
-                    tmem_ld32(lane_base + C::S_COL + 32 * c, r);
-                    tmem_wait_ld(r);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float x = __fmul_rn(__uint_as_float(r[j]), cs);
-                        if (k0 + 32 * c + j <= t) m_s = fmaxf(m_s, x);
-                    }
-                }
-                // pass 2: exponentials, their sum and P (bf16) into TMEM
-#pragma unroll 1
-                for (int c = 0; c < kSplit / 32; ++c) {
-                    tmem_ld32(lane_base + C::S_COL + 32 * c, r);
-                    tmem_wait_ld(r);
-                    float e[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float x = __fmul_rn(__uint_as_float(r[j]), cs);
-                        e[j] = (k0 + 32 * c + j <= t) ? ex2(__fsub_rn(x, m_s)) : 0.0f;
-                    }
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(e[2 * j], e[2 * j + 1]);
-                    tmem_st16(lane_base + C::P_COL + 16 * c, pk);
-#pragma unroll
-                    for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-                        for (int j = 0; j < w; ++j) e[j] = __fadd_rn(e[j], e[j + w]);
-                    l_s = __fadd_rn(l_s, e[0]);
-                }
-                tmem_wait_st();
-            }
+            if (active) split_softmax(sb + C::P_OFF, k0, t, cs, m_s, l_s);
             tc_fence_before();
-            mbar_arrive(barP);
+            mbar_arrive(&barP[b]);
 
-            if (!wait(barO, o_phase, ctl)) {
+            if (!wait(&barO[b], par, ctl)) {
                 ok = false;
                 break;
             }
-            o_phase ^= 1u;
             tc_fence_after();
             if (active) {
                 if (spill) {
@@ -477,16 +548,19 @@ __global__ void __launch_bounds__(THREADS, 1)
                     // split's own partial for attn_combine
                     float *rec = p.ws + ((out_row * p.max_splits) + s) * C::REC;
 #pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t r[32];
-                        tmem_ld32(lane_base + C::O_COL + 32 * c, r);
-                        tmem_wait_ld(r);
+                    for (int c = 0; c < D / 32; c += 2) {
+                        uint32_t r0[32], r1[32];
+                        tmem_ld64(sb + C::O_OFF + 32 * c, r0, r1);
                         if (valid) {
 #pragma unroll
-                            for (int j = 0; j < 8; ++j)
+                            for (int j = 0; j < 8; ++j) {
                                 reinterpret_cast<float4 *>(rec + 4 + 32 * c)[j] = make_float4(
-                                    __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                    __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+                                    __uint_as_float(r0[4 * j]), __uint_as_float(r0[4 * j + 1]),
+                                    __uint_as_float(r0[4 * j + 2]), __uint_as_float(r0[4 * j + 3]));
+                                reinterpret_cast<float4 *>(rec + 4 + 32 * c + 32)[j] = make_float4(
+                                    __uint_as_float(r1[4 * j]), __uint_as_float(r1[4 * j + 1]),
+                                    __uint_as_float(r1[4 * j + 2]), __uint_as_float(r1[4 * j + 3]));
+                            }
                         }
                     }
                     if (valid) {
@@ -499,17 +573,20 @@ __global__ void __launch_bounds__(THREADS, 1)
                     float mn, a, cc;
                     merge_scales(m, m_s, mn, a, cc);
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t r[32];
-                        tmem_ld32(lane_base + C::O_COL + 32 * c, r);
-                        tmem_wait_ld(r);
+                    for (int c = 0; c < D / 32; c += 2) {
+                        uint32_t r0[32], r1[32];
+                        tmem_ld64(sb + C::O_OFF + 32 * c, r0, r1);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
-                            const float os = __uint_as_float(r[j]);
-                            if (first)
-                                O[32 * c + j] = os;
-                            else if (take)
-                                O[32 * c + j] = merge_val(O[32 * c + j], a, os, cc);
+                            const float o0 = __uint_as_float(r0[j]);
+                            const float o1 = __uint_as_float(r1[j]);
+                            if (first) {
+                                O[32 * c + j] = o0;
+                                O[32 * c + 32 + j] = o1;
+                            } else if (take) {
+                                O[32 * c + j] = merge_val(O[32 * c + j], a, o0, cc);
+                                O[32 * c + 32 + j] = merge_val(O[32 * c + 32 + j], a, o1, cc);
+                            }
                         }
                     }
                     if (first) {
@@ -521,6 +598,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(&barF[b]);
         }
 
         if (ok && active && valid && !spill) {
