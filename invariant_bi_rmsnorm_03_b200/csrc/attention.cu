@@ -56,7 +56,9 @@
 namespace bi {
 namespace {
 
-constexpr int THREADS = 192;
+// Warp roles: 0 producer, 1 MMA, 4-7 softmax, 2-3 and 8-9 merge ("fold").
+// Softmax warp w and fold warp w' own TMEM lane quarter w % 4.
+constexpr int THREADS = 320;
 constexpr float kLn2 = 0.693147180559945309f;
 
 template <int D>
@@ -68,8 +70,10 @@ struct Cfg {
     static constexpr int KV_BYTES = KB * KV_KB_BYTES;
     static constexpr int PAGE_KB_BYTES = kPage * 128;   // one page of one column block
     static constexpr int NSLOT = 3;
+    static constexpr int ML_BYTES = 2 * 128 * 2 * 4;   // (m_s, l_s) per row, two buffers
     static constexpr int BAR_BYTES = 256;
-    static constexpr int SMEM = 1024 + Q_BYTES + NSLOT * KV_BYTES + BAR_BYTES;
+    static constexpr int SLACK = 768;                  // alignment slack of the base
+    static constexpr int SMEM = SLACK + ML_BYTES + Q_BYTES + NSLOT * KV_BYTES + BAR_BYTES;
     // TMEM: two buffers of 256 columns.  In buffer b: S over all 256
     // columns; P (bf16 pairs) written over its first 128; O_s in the next D.
     static constexpr uint32_t BUF_COLS = 256, P_OFF = 0, O_OFF = 128, TMEM_COLS = 512;
@@ -188,12 +192,17 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r0)[32], ui
 // TMEM columns sb .. sb+255 in two passes; P (bf16 pairs) is written over
 // columns sb .. sb+127 as the second pass goes (each store lands on columns
 // this thread has already read).  Returns m_s (scaled, log2 units) and l_s.
+// (P V cannot start before the whole pass is done: it writes O_s over the
+// columns that hold the logits of keys 128..255.)
 __device__ __forceinline__ void split_softmax(uint32_t sb, int k0, int t, float cs, float &m_s,
                                               float &l_s)
 {
     // pass 1: maximum of the raw logits over the visible keys.  For c > 0,
     // x -> round(x * c) is monotonic, so max_j round(S_j c) = round(max_j S_j * c).
-    float mraw = -INFINITY;
+    // (A maximum is exact in any order; eight accumulators break the chain.)
+    float mx[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
 #pragma unroll 1
     for (int c = 0; c < kSplit / 32; c += 2) {
         uint32_t r0[32], r1[32];
@@ -201,18 +210,20 @@ __device__ __forceinline__ void split_softmax(uint32_t sb, int k0, int t, float 
         const int kc = k0 + 32 * c;
         if (kc + 63 <= t) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) mraw = fmaxf(mraw, __uint_as_float(r0[j]));
+            for (int j = 0; j < 32; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r0[j]));
 #pragma unroll
-            for (int j = 0; j < 32; ++j) mraw = fmaxf(mraw, __uint_as_float(r1[j]));
+            for (int j = 0; j < 32; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r1[j]));
         } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-                if (kc + j <= t) mraw = fmaxf(mraw, __uint_as_float(r0[j]));
+                if (kc + j <= t) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r0[j]));
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-                if (kc + 32 + j <= t) mraw = fmaxf(mraw, __uint_as_float(r1[j]));
+                if (kc + 32 + j <= t) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r1[j]));
         }
     }
+    const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
     m_s = __fmul_rn(mraw, cs);
     // pass 2: p = 2^(round(S c) - m_s), masked keys 0; 32-key chunk sums by a
     // pairwise tree, added to l_s chunk by chunk in key order.
@@ -262,16 +273,22 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
-    uint8_t *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
-    uint8_t *sQ = smem;
-    uint8_t *sKV = smem + C::Q_BYTES;
+    const uint32_t pad = (1024 - (raw & 1023)) & 1023;
+    if (pad > uint32_t(C::SLACK)) {  // cannot happen with a 1 KB-aligned base
+        if (threadIdx.x == 0) record_status(p.status, BI_DEV_BAD_INDEX);
+        return;
+    }
+    uint8_t *smem = smem_raw + pad;
+    float *sML = reinterpret_cast<float *>(smem);               // [2][128][2]
+    uint8_t *sQ = smem + C::ML_BYTES;
+    uint8_t *sKV = sQ + C::Q_BYTES;
     uint64_t *full = reinterpret_cast<uint64_t *>(sKV + C::NSLOT * C::KV_BYTES);
     uint64_t *empty = full + C::NSLOT;
     uint64_t *barQ = empty + C::NSLOT;
     uint64_t *barS = barQ + 1;     // [2] S of buffer b computed
-    uint64_t *barP = barS + 2;     // [2] P of buffer b written (128 arrivals)
+    uint64_t *barP = barS + 2;     // [2] P and (m_s, l_s) of buffer b written (128 arrivals)
     uint64_t *barO = barP + 2;     // [2] O_s of buffer b computed
-    uint64_t *barF = barO + 2;     // [2] buffer b free again (128 arrivals)
+    uint64_t *barF = barO + 2;     // [2] O_s of buffer b merged, buffer free (128 arrivals)
     uint64_t *drain = barF + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
@@ -420,8 +437,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else if (warp == 1) {
         // ====================================================== MMA issue
         // Tensor-pipe order: QK(s0), QK(s0+1), PV(s0), QK(s0+2), PV(s0+1),
-        // ... so that S of the next split is ready while a split's softmax
-        // runs.  Split s uses TMEM buffer (s - s0) & 1.
+        // ...; split s uses TMEM buffer (s - s0) & 1, which QK(s+2) reuses
+        // once the fold warps have merged O_s(s).
         if (lane == 0) {
             const uint32_t idesc_qk = idesc_bf16_f32(128, kSplit, 0, 0);
             const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
@@ -450,19 +467,19 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int s = it.s0; ok && s < it.s1; ++s) {
                 const int b = (s - it.s0) & 1;
                 const uint32_t par = uint32_t((s - it.s0) >> 1) & 1u;
-                if (!wait(&barP[b], par, ctl)) {
-                    ok = false;
-                    break;
-                }
                 const int i = 2 * (s - it.s0) + 1;
                 const int slot = i % C::NSLOT;
                 if (!wait(&full[slot], uint32_t(i / C::NSLOT) & 1u, ctl)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
                 const uint32_t buf = tmem + C::BUF_COLS * uint32_t(b);
                 const uint32_t v_base = smem_u32(sKV + slot * C::KV_BYTES);
+                if (!wait(&barP[b], par, ctl)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
 #pragma unroll
                 for (int j = 0; j < kSplit / 16; ++j) {
                     mma_ts(buf + C::O_OFF, buf + C::P_OFF + 8 * j,
@@ -486,12 +503,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
     } else {
-        // ====================================================== softmax
+        // ====================================================== rows
+        // Softmax warps (4-7) and fold warps (2, 3, 8, 9) of lane quarter q
+        // serve the same 32 rows.
+        const bool is_softmax = warp >= 4 && warp < 8;
         const int q = warp & 3;
-        bool valid;
+        bool valid, active;
         int t, local;
         int64_t out_row;
-        bool active;
         if (p.decode) {
             local = q * p.rows_per_q + lane;
             valid = lane < p.rows_per_q && local < p.group;
@@ -507,115 +526,122 @@ __global__ void __launch_bounds__(THREADS, 1)
             active = 32 * q < it.rows;
         }
         const uint32_t lane_base = tmem_addr(tmem, 32 * q, 0);
-        const float cs = p.scale_log2;
+        const int row_id = 32 * q + lane;  // TMEM lane of this row
+
+        if (is_softmax) {
+            // -------------------------------------------------- softmax
+            const float cs = p.scale_log2;
+            for (int s = it.s0; s < it.s1; ++s) {
+                const int b = (s - it.s0) & 1;
+                const uint32_t par = uint32_t((s - it.s0) >> 1) & 1u;
+                const uint32_t sb = lane_base + C::BUF_COLS * uint32_t(b);
+                if (!wait(&barS[b], par, ctl)) break;
+                tc_fence_after();
+                float m_s = -INFINITY, l_s = 0.0f;
+                if (active) split_softmax(sb + C::P_OFF, s * kSplit, t, cs, m_s, l_s);
+                sML[(b * 128 + row_id) * 2 + 0] = m_s;
+                sML[(b * 128 + row_id) * 2 + 1] = l_s;
+                tc_fence_before();
+                mbar_arrive(&barP[b]);
+            }
+        } else {
+            // -------------------------------------------------- fold
 #if BI_INVARIANT
-        // blocks after a sequence's first write every split's own partial
-        const bool spill = p.decode && it.s0 > 0;
+            // blocks after a sequence's first write every split's own partial
+            const bool spill = p.decode && it.s0 > 0;
 #else
-        // variant-off: every block merges its own range (the grouping of the
-        // merge then depends on how many blocks served the sequence)
-        const bool spill = false;
+            // variant-off: every block merges its own range (the grouping of
+            // the merge then depends on how many blocks served the sequence)
+            const bool spill = false;
 #endif
-        float m = -INFINITY, l = 0.0f;
-        float O[D];
+            float m = -INFINITY, l = 0.0f;
+            float O[D];
 #pragma unroll
-        for (int j = 0; j < D; ++j) O[j] = 0.0f;
-        bool ok = true;
-
-        for (int s = it.s0; s < it.s1; ++s) {
-            const int b = (s - it.s0) & 1;
-            const uint32_t par = uint32_t((s - it.s0) >> 1) & 1u;
-            const uint32_t sb = lane_base + C::BUF_COLS * uint32_t(b);
-            const int k0 = s * kSplit;
-            if (!wait(&barS[b], par, ctl)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            float m_s = -INFINITY, l_s = 0.0f;
-            if (active) split_softmax(sb + C::P_OFF, k0, t, cs, m_s, l_s);
-            tc_fence_before();
-            mbar_arrive(&barP[b]);
-
-            if (!wait(&barO[b], par, ctl)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            if (active) {
-                if (spill) {
-                    // not the first block of this sequence: write the
-                    // split's own partial for attn_combine
-                    float *rec = p.ws + ((out_row * p.max_splits) + s) * C::REC;
+            for (int j = 0; j < D; ++j) O[j] = 0.0f;
+            bool ok = true;
+            for (int s = it.s0; s < it.s1; ++s) {
+                const int b = (s - it.s0) & 1;
+                const uint32_t par = uint32_t((s - it.s0) >> 1) & 1u;
+                const uint32_t ob = lane_base + C::BUF_COLS * uint32_t(b) + C::O_OFF;
+                const int k0 = s * kSplit;
+                // barP: (m_s, l_s) of this split are in shared memory;
+                // barO: O_s is in TMEM.
+                if (!wait(&barP[b], par, ctl) || !wait(&barO[b], par, ctl)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float m_s = sML[(b * 128 + row_id) * 2 + 0];
+                const float l_s = sML[(b * 128 + row_id) * 2 + 1];
+                if (active) {
+                    if (spill) {
+                        // not the first block of this sequence: write the
+                        // split's own partial for attn_combine
+                        float *rec = p.ws + ((out_row * p.max_splits) + s) * C::REC;
 #pragma unroll 1
-                    for (int c = 0; c < D / 32; c += 2) {
-                        uint32_t r0[32], r1[32];
-                        tmem_ld64(sb + C::O_OFF + 32 * c, r0, r1);
+                        for (int c = 0; c < D / 16; ++c) {
+                            uint32_t r0[16];
+                            tmem_ld16(ob + 16 * c, r0);
+                            tmem_wait_ld(r0);
+                            if (valid) {
+#pragma unroll
+                                for (int j = 0; j < 4; ++j)
+                                    reinterpret_cast<float4 *>(rec + 4 + 16 * c)[j] = make_float4(
+                                        __uint_as_float(r0[4 * j]), __uint_as_float(r0[4 * j + 1]),
+                                        __uint_as_float(r0[4 * j + 2]), __uint_as_float(r0[4 * j + 3]));
+                            }
+                        }
                         if (valid) {
+                            rec[0] = m_s;
+                            rec[1] = l_s;
+                        }
+                    } else {
+                        const bool first = (s == it.s0);
+                        const bool take = k0 <= t;  // the row sees at least key k0
+                        float mn, a, cc;
+                        merge_scales(m, m_s, mn, a, cc);
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                reinterpret_cast<float4 *>(rec + 4 + 32 * c)[j] = make_float4(
-                                    __uint_as_float(r0[4 * j]), __uint_as_float(r0[4 * j + 1]),
-                                    __uint_as_float(r0[4 * j + 2]), __uint_as_float(r0[4 * j + 3]));
-                                reinterpret_cast<float4 *>(rec + 4 + 32 * c + 32)[j] = make_float4(
-                                    __uint_as_float(r1[4 * j]), __uint_as_float(r1[4 * j + 1]),
-                                    __uint_as_float(r1[4 * j + 2]), __uint_as_float(r1[4 * j + 3]));
+                        for (int c = 0; c < D / 16; ++c) {
+                            uint32_t r0[16];
+                            tmem_ld16(ob + 16 * c, r0);
+                            tmem_wait_ld(r0);
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const float o0 = __uint_as_float(r0[j]);
+                                if (first)
+                                    O[16 * c + j] = o0;
+                                else if (take)
+                                    O[16 * c + j] = merge_val(O[16 * c + j], a, o0, cc);
                             }
                         }
-                    }
-                    if (valid) {
-                        rec[0] = m_s;
-                        rec[1] = l_s;
-                    }
-                } else {
-                    const bool first = (s == it.s0);
-                    const bool take = k0 <= t;  // the row sees at least key k0
-                    float mn, a, cc;
-                    merge_scales(m, m_s, mn, a, cc);
-#pragma unroll
-                    for (int c = 0; c < D / 32; c += 2) {
-                        uint32_t r0[32], r1[32];
-                        tmem_ld64(sb + C::O_OFF + 32 * c, r0, r1);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float o0 = __uint_as_float(r0[j]);
-                            const float o1 = __uint_as_float(r1[j]);
-                            if (first) {
-                                O[32 * c + j] = o0;
-                                O[32 * c + 32 + j] = o1;
-                            } else if (take) {
-                                O[32 * c + j] = merge_val(O[32 * c + j], a, o0, cc);
-                                O[32 * c + 32 + j] = merge_val(O[32 * c + 32 + j], a, o1, cc);
-                            }
+                        if (first) {
+                            m = m_s;
+                            l = l_s;
+                        } else if (take) {
+                            l = merge_val(l, a, l_s, cc);
+                            m = mn;
                         }
-                    }
-                    if (first) {
-                        m = m_s;
-                        l = l_s;
-                    } else if (take) {
-                        l = merge_val(l, a, l_s, cc);
-                        m = mn;
                     }
                 }
+                tc_fence_before();
+                mbar_arrive(&barF[b]);
             }
-            tc_fence_before();
-            mbar_arrive(&barF[b]);
-        }
 
-        if (ok && active && valid && !spill) {
-            if (!p.decode || it.s1 == it.n_splits) {
-                write_out<D>(O, l, m, static_cast<__nv_bfloat16 *>(p.o) + out_row * D,
-                             p.lse ? p.lse + out_row : nullptr);
-            } else {
-                // first block of a sequence served by several: hand the
-                // merged state over split s1-1 to attn_combine
-                float *rec = p.ws + ((out_row * p.max_splits) + (it.s1 - 1)) * C::REC;
-                rec[0] = m;
-                rec[1] = l;
+            if (ok && active && valid && !spill) {
+                if (!p.decode || it.s1 == it.n_splits) {
+                    write_out<D>(O, l, m, static_cast<__nv_bfloat16 *>(p.o) + out_row * D,
+                                 p.lse ? p.lse + out_row : nullptr);
+                } else {
+                    // first block of a sequence served by several: hand the
+                    // merged state over split s1-1 to attn_combine
+                    float *rec = p.ws + ((out_row * p.max_splits) + (it.s1 - 1)) * C::REC;
+                    rec[0] = m;
+                    rec[1] = l;
 #pragma unroll
-                for (int j = 0; j < D / 4; ++j)
-                    reinterpret_cast<float4 *>(rec + 4)[j] =
-                        make_float4(O[4 * j], O[4 * j + 1], O[4 * j + 2], O[4 * j + 3]);
+                    for (int j = 0; j < D / 4; ++j)
+                        reinterpret_cast<float4 *>(rec + 4)[j] =
+                            make_float4(O[4 * j], O[4 * j + 1], O[4 * j + 2], O[4 * j + 3]);
+                }
             }
         }
     }

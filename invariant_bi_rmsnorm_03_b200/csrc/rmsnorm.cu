@@ -17,9 +17,10 @@
 // T and ITEMS depend only on H, so a row gets the same bits whatever M is,
 // whichever block handles it and wherever it sits in the batch.
 //
-// Memory: the row is loaded once into registers with 128-bit loads, the
-// output is written with 128-bit stores.  The grid is min(M, cap) blocks
-// striding over rows.
+// Memory: rows are loaded once into registers with 128-bit loads (a block
+// loads all of its R rows before reducing any, to keep more bytes in
+// flight), the output is written with 128-bit stores.  The grid strides
+// over groups of R rows.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -52,89 +53,121 @@ __device__ __forceinline__ float scale1(float x, float rstd, float w)
     return __fmul_rn(__fmul_rn(x, rstd), w);
 }
 
-template <int ITEMS, bool OUT_F32>
+template <bool OUT_F32>
+__device__ __forceinline__ void store8(void *y, int64_t idx, const uint4 &xv, const uint4 &wv,
+                                       float rstd)
+{
+    float o[8];
+    o[0] = scale1(bf_lo(xv.x), rstd, bf_lo(wv.x));
+    o[1] = scale1(bf_hi(xv.x), rstd, bf_hi(wv.x));
+    o[2] = scale1(bf_lo(xv.y), rstd, bf_lo(wv.y));
+    o[3] = scale1(bf_hi(xv.y), rstd, bf_hi(wv.y));
+    o[4] = scale1(bf_lo(xv.z), rstd, bf_lo(wv.z));
+    o[5] = scale1(bf_hi(xv.z), rstd, bf_hi(wv.z));
+    o[6] = scale1(bf_lo(xv.w), rstd, bf_lo(wv.w));
+    o[7] = scale1(bf_hi(xv.w), rstd, bf_hi(wv.w));
+    if constexpr (OUT_F32) {
+        float4 *yr = reinterpret_cast<float4 *>(y) + idx * 2;
+        __stcs(yr, make_float4(o[0], o[1], o[2], o[3]));
+        __stcs(yr + 1, make_float4(o[4], o[5], o[6], o[7]));
+    } else {
+        uint4 ov;
+        __nv_bfloat162 p0 = __floats2bfloat162_rn(o[0], o[1]);
+        __nv_bfloat162 p1 = __floats2bfloat162_rn(o[2], o[3]);
+        __nv_bfloat162 p2 = __floats2bfloat162_rn(o[4], o[5]);
+        __nv_bfloat162 p3 = __floats2bfloat162_rn(o[6], o[7]);
+        ov.x = *reinterpret_cast<uint32_t *>(&p0);
+        ov.y = *reinterpret_cast<uint32_t *>(&p1);
+        ov.z = *reinterpret_cast<uint32_t *>(&p2);
+        ov.w = *reinterpret_cast<uint32_t *>(&p3);
+        __stcs(reinterpret_cast<uint4 *>(y) + idx, ov);
+    }
+}
+
+// A block handles R rows at a time: all R rows are loaded before any is
+// reduced, so that more bytes are in flight.  R changes only how rows are
+// grouped into blocks; each row's arithmetic is the same for every R.
+template <int ITEMS, int R, bool OUT_F32>
 __global__ void __launch_bounds__(1024) rmsnorm_kernel(const uint4 *__restrict__ x,
                                                        const uint4 *__restrict__ w,
                                                        void *__restrict__ y, int64_t M, int H,
                                                        float eps)
 {
-    __shared__ float part[32];
+    __shared__ float part[R][32];
     const int chunks = H >> 3;
     const int T = blockDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const float inv_h_den = static_cast<float>(H);
+    const float h_den = static_cast<float>(H);
 
-    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
-        const uint4 *xr = x + row * chunks;
-        uint4 v[ITEMS];
-        float acc = 0.0f;
+    for (int64_t row0 = int64_t(blockIdx.x) * R; row0 < M; row0 += int64_t(gridDim.x) * R) {
+        uint4 v[R][ITEMS];
+        float acc[R];
 #pragma unroll
-        for (int it = 0; it < ITEMS; ++it) {
-            const int c = threadIdx.x + it * T;
-            if (c < chunks) {
-                v[it] = __ldcs(xr + c);
-                acc = sumsq8(v[it], acc);
+        for (int r = 0; r < R; ++r) {
+            acc[r] = 0.0f;
+            const int64_t row = row0 + r;
+#pragma unroll
+            for (int it = 0; it < ITEMS; ++it) {
+                const int c = threadIdx.x + it * T;
+                if (row < M && c < chunks) v[r][it] = __ldcs(x + row * chunks + c);
             }
         }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
-        if (lane == 0) part[warp] = acc;
+        for (int r = 0; r < R; ++r) {
+#pragma unroll
+            for (int it = 0; it < ITEMS; ++it) {
+                const int c = threadIdx.x + it * T;
+                if (row0 + r < M && c < chunks) acc[r] = sumsq8(v[r][it], acc[r]);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                acc[r] = __fadd_rn(acc[r], __shfl_xor_sync(0xffffffffu, acc[r], off));
+            if (lane == 0) part[r][warp] = acc[r];
+        }
         __syncthreads();
-        float tot = 0.0f;
-        for (int i = 0; i < (T >> 5); ++i) tot = __fadd_rn(tot, part[i]);
-        const float rstd = rsqrtf(__fadd_rn(__fdiv_rn(tot, inv_h_den), eps));
-
 #pragma unroll
-        for (int it = 0; it < ITEMS; ++it) {
-            const int c = threadIdx.x + it * T;
-            if (c < chunks) {
-                const uint4 wv = __ldg(w + c);
-                const uint4 xv = v[it];
-                float o[8];
-                o[0] = scale1(bf_lo(xv.x), rstd, bf_lo(wv.x));
-                o[1] = scale1(bf_hi(xv.x), rstd, bf_hi(wv.x));
-                o[2] = scale1(bf_lo(xv.y), rstd, bf_lo(wv.y));
-                o[3] = scale1(bf_hi(xv.y), rstd, bf_hi(wv.y));
-                o[4] = scale1(bf_lo(xv.z), rstd, bf_lo(wv.z));
-                o[5] = scale1(bf_hi(xv.z), rstd, bf_hi(wv.z));
-                o[6] = scale1(bf_lo(xv.w), rstd, bf_lo(wv.w));
-                o[7] = scale1(bf_hi(xv.w), rstd, bf_hi(wv.w));
-                if constexpr (OUT_F32) {
-                    float4 *yr = reinterpret_cast<float4 *>(y) + (row * chunks + c) * 2;
-                    __stcs(yr, make_float4(o[0], o[1], o[2], o[3]));
-                    __stcs(yr + 1, make_float4(o[4], o[5], o[6], o[7]));
-                } else {
-                    uint4 ov;
-                    __nv_bfloat162 p0 = __floats2bfloat162_rn(o[0], o[1]);
-                    __nv_bfloat162 p1 = __floats2bfloat162_rn(o[2], o[3]);
-                    __nv_bfloat162 p2 = __floats2bfloat162_rn(o[4], o[5]);
-                    __nv_bfloat162 p3 = __floats2bfloat162_rn(o[6], o[7]);
-                    ov.x = *reinterpret_cast<uint32_t *>(&p0);
-                    ov.y = *reinterpret_cast<uint32_t *>(&p1);
-                    ov.z = *reinterpret_cast<uint32_t *>(&p2);
-                    ov.w = *reinterpret_cast<uint32_t *>(&p3);
-                    __stcs(reinterpret_cast<uint4 *>(y) + row * chunks + c, ov);
-                }
+        for (int r = 0; r < R; ++r) {
+            const int64_t row = row0 + r;
+            if (row >= M) break;
+            float tot = 0.0f;
+            for (int i = 0; i < (T >> 5); ++i) tot = __fadd_rn(tot, part[r][i]);
+            const float rstd = rsqrtf(__fadd_rn(__fdiv_rn(tot, h_den), eps));
+#pragma unroll
+            for (int it = 0; it < ITEMS; ++it) {
+                const int c = threadIdx.x + it * T;
+                if (c < chunks) store8<OUT_F32>(y, row * chunks + c, v[r][it], __ldg(w + c), rstd);
             }
         }
-        __syncthreads();  // part[] is reused by the next row
+        __syncthreads();  // part[] is reused by the next group of rows
     }
+}
+
+template <int ITEMS, int R>
+cudaError_t launch_rows(const void *x, const void *w, void *y, int64_t M, int H, float eps,
+                        bool out_f32, int threads, cudaStream_t s)
+{
+    const int64_t cap = int64_t(1) << 20;
+    const int64_t groups = (M + R - 1) / R;
+    const unsigned grid = static_cast<unsigned>(groups < cap ? groups : cap);
+    if (out_f32)
+        rmsnorm_kernel<ITEMS, R, true><<<grid, threads, 0, s>>>(
+            static_cast<const uint4 *>(x), static_cast<const uint4 *>(w), y, M, H, eps);
+    else
+        rmsnorm_kernel<ITEMS, R, false><<<grid, threads, 0, s>>>(
+            static_cast<const uint4 *>(x), static_cast<const uint4 *>(w), y, M, H, eps);
+    return cudaGetLastError();
 }
 
 template <int ITEMS>
 cudaError_t launch_items(const void *x, const void *w, void *y, int64_t M, int H, float eps,
-                         bool out_f32, int threads, cudaStream_t s)
+                         bool out_f32, int threads, int rows_per_block, cudaStream_t s)
 {
-    const int64_t cap = int64_t(1) << 20;
-    const unsigned grid = static_cast<unsigned>(M < cap ? M : cap);
-    if (out_f32)
-        rmsnorm_kernel<ITEMS, true><<<grid, threads, 0, s>>>(
-            static_cast<const uint4 *>(x), static_cast<const uint4 *>(w), y, M, H, eps);
-    else
-        rmsnorm_kernel<ITEMS, false><<<grid, threads, 0, s>>>(
-            static_cast<const uint4 *>(x), static_cast<const uint4 *>(w), y, M, H, eps);
-    return cudaGetLastError();
+    // ITEMS * rows_per_block <= 8 (the host never asks for more)
+    if constexpr (ITEMS <= 2)
+        if (rows_per_block >= 4) return launch_rows<ITEMS, 4>(x, w, y, M, H, eps, out_f32, threads, s);
+    if constexpr (ITEMS <= 4)
+        if (rows_per_block >= 2) return launch_rows<ITEMS, 2>(x, w, y, M, H, eps, out_f32, threads, s);
+    return launch_rows<ITEMS, 1>(x, w, y, M, H, eps, out_f32, threads, s);
 }
 
 }  // namespace
@@ -165,15 +198,17 @@ cudaError_t launch_rmsnorm(const void *x, const void *w, void *y, int64_t M, int
         int64_t t = (H / 8 + items - 1) / items;
         threads = static_cast<int>((t + 31) / 32 * 32);
     }
-#else
-    (void)num_sms;
 #endif
+    // Rows per block: enough that one wave of resident blocks covers M.
+    const int64_t resident = int64_t(num_sms) * (2048 / threads);
+    int rpb = 1;
+    while (rpb < 4 && int64_t(rpb) * resident < M && items * rpb < 8) rpb *= 2;
     const int h = static_cast<int>(H);
     switch (items) {
-    case 1: return launch_items<1>(x, w, y, M, h, eps, out_f32, threads, s);
-    case 2: return launch_items<2>(x, w, y, M, h, eps, out_f32, threads, s);
-    case 4: return launch_items<4>(x, w, y, M, h, eps, out_f32, threads, s);
-    default: return launch_items<8>(x, w, y, M, h, eps, out_f32, threads, s);
+    case 1: return launch_items<1>(x, w, y, M, h, eps, out_f32, threads, rpb, s);
+    case 2: return launch_items<2>(x, w, y, M, h, eps, out_f32, threads, rpb, s);
+    case 4: return launch_items<4>(x, w, y, M, h, eps, out_f32, threads, rpb, s);
+    default: return launch_items<8>(x, w, y, M, h, eps, out_f32, threads, rpb, s);
     }
 }
 
