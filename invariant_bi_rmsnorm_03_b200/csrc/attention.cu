@@ -179,21 +179,25 @@ __device__ __forceinline__ uint32_t swz(int r, int c)
 
 // ---------------------------------------------------------------- kernel
 
-// 32 + 32 columns of one lane quarter into two register arrays, one wait.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r0)[32], uint32_t (&r1)[32])
+// 128 columns of one lane quarter into four register arrays, one wait.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[4][32])
 {
-    tmem_ld32(taddr, r0);
-    tmem_ld32(taddr + 32, r1);
-    tmem_wait_ld(r0);
-    tmem_wait_ld(r1);
+    tmem_ld32(taddr, r[0]);
+    tmem_ld32(taddr + 32, r[1]);
+    tmem_ld32(taddr + 64, r[2]);
+    tmem_ld32(taddr + 96, r[3]);
+    tmem_wait_ld(r[0]);
+    tmem_wait_ld(r[1]);
+    tmem_wait_ld(r[2]);
+    tmem_wait_ld(r[3]);
 }
 
 // Softmax of one split for the row owned by this thread.  S is read from
-// TMEM columns sb .. sb+255 in two passes; P (bf16 pairs) is written over
-// columns sb .. sb+127 as the second pass goes (each store lands on columns
-// this thread has already read).  Returns m_s (scaled, log2 units) and l_s.
-// (P V cannot start before the whole pass is done: it writes O_s over the
-// columns that hold the logits of keys 128..255.)
+// TMEM columns sb .. sb+255 in two passes of two 128-column loads; P (bf16
+// pairs) is written over columns sb .. sb+127 as the second pass goes (each
+// store lands on columns this thread has already read).  Returns m_s
+// (scaled, log2 units) and l_s.  (P V cannot start before the whole pass is
+// done: it writes O_s over the columns of the logits of keys 128..255.)
 __device__ __forceinline__ void split_softmax(uint32_t sb, int k0, int t, float cs, float &m_s,
                                               float &l_s)
 {
@@ -204,22 +208,20 @@ __device__ __forceinline__ void split_softmax(uint32_t sb, int k0, int t, float 
 #pragma unroll
     for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
 #pragma unroll 1
-    for (int c = 0; c < kSplit / 32; c += 2) {
-        uint32_t r0[32], r1[32];
-        tmem_ld64(sb + 32 * c, r0, r1);
-        const int kc = k0 + 32 * c;
-        if (kc + 63 <= t) {
+    for (int c = 0; c < kSplit / 32; c += 4) {
+        uint32_t r[4][32];
+        tmem_ld128(sb + 32 * c, r);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r0[j]));
+        for (int h = 0; h < 4; ++h) {
+            const int kc = k0 + 32 * (c + h);
+            if (kc + 31 <= t) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r1[j]));
-        } else {
+                for (int j = 0; j < 32; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[h][j]));
+            } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (kc + j <= t) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r0[j]));
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (kc + 32 + j <= t) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r1[j]));
+                for (int j = 0; j < 32; ++j)
+                    if (kc + j <= t) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[h][j]));
+            }
         }
     }
     const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
@@ -229,11 +231,11 @@ __device__ __forceinline__ void split_softmax(uint32_t sb, int k0, int t, float 
     // pairwise tree, added to l_s chunk by chunk in key order.
     float l = 0.0f;
 #pragma unroll 1
-    for (int c = 0; c < kSplit / 32; c += 2) {
-        uint32_t r[2][32];
-        tmem_ld64(sb + 32 * c, r[0], r[1]);
+    for (int c = 0; c < kSplit / 32; c += 4) {
+        uint32_t r[4][32];
+        tmem_ld128(sb + 32 * c, r);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < 4; ++h) {
             const int kc = k0 + 32 * (c + h);
             float e[32];
             if (kc + 31 <= t) {
@@ -353,81 +355,91 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             return phys;
         };
+        // Load list (relative split j, n splits): K0, K1, V0, K2, V1, K3,
+        // ..., V(n-2), V(n-1): keys two splits ahead of values, which is the
+        // order in which the MMA warp consumes them.  Load i goes to ring
+        // slot i % NSLOT.  Lane i < 16 keeps the page ids of the splits in
+        // flight in a 4-entry ring (looked up ahead of use).
+        const int n = it.s1 - it.s0;
         int slot = 0;
         uint32_t phase = 0;
-        int phys_next = it.s0 < it.s1 ? lookup(it.s0) : -1;
-        for (int s = it.s0; ok && s < it.s1; ++s) {
-            const int phys = phys_next;
-            if (s + 1 < it.s1) phys_next = lookup(s + 1);
+        int pages[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pages[e] = e < n ? lookup(it.s0 + e) : -1;
+        auto emit = [&](int which, int j) -> bool {
+            const int s = it.s0 + j;
+            const int phys = pages[j & 3];
             const int nk = min(kSplit, it.kv_len - s * kSplit);  // valid keys, >= 1
             const int full_pages = nk / kPage;
             const int npages = (nk + kPage - 1) / kPage;
             // box row of this lane's page; -16 = out of bounds, zero filled
             const int row = phys >= 0 ? (phys * p.Hkv + it.g) * kPage : -kPage;
-            for (int which = 0; which < 2; ++which) {  // 0: K, 1: V
-                int got = 1;
-                if (lane == 0) got = wait(&empty[slot], phase ^ 1u, ctl) ? 1 : 0;
-                got = __shfl_sync(0xffffffffu, got, 0);
-                if (!got) {
-                    ok = false;
-                    break;
-                }
-                uint8_t *dst = sKV + slot * C::KV_BYTES;
-                const CUtensorMap *map = which ? &tv : &tk;
-                const int partial_phys = __shfl_sync(0xffffffffu, phys, full_pages & 31);
-                // V: the partial last page is copied by the whole warp, with
-                // the rows past the sequence end set to zero.
-                if (which == 1 && full_pages < npages) {
-                    const int pg = full_pages;
-                    const bool good = partial_phys >= 0;
-                    const int valid = nk - pg * kPage;
-                    for (int i = lane; i < kPage * C::KB * 8; i += 32) {
-                        const int r = i / (C::KB * 8);
-                        const int kb = (i / 8) % C::KB;
-                        const int c = i % 8;
-                        uint4 v = make_uint4(0, 0, 0, 0);
-                        if (good && r < valid) {
-                            const int64_t src =
-                                ((int64_t(partial_phys) * p.Hkv + it.g) * kPage + r) * D + kb * 64 +
-                                c * 8;
-                            v = __ldg(reinterpret_cast<const uint4 *>(
-                                static_cast<const __nv_bfloat16 *>(p.v_cache) + src));
-                        }
-                        *reinterpret_cast<uint4 *>(dst + kb * C::KV_KB_BYTES +
-                                                   swz(pg * kPage + r, c)) = v;
+            int got = 1;
+            if (lane == 0) got = wait(&empty[slot], phase ^ 1u, ctl) ? 1 : 0;
+            got = __shfl_sync(0xffffffffu, got, 0);
+            if (!got) return false;
+            uint8_t *dst = sKV + slot * C::KV_BYTES;
+            const CUtensorMap *map = which ? &tv : &tk;
+            const int partial_phys = __shfl_sync(0xffffffffu, phys, full_pages & 31);
+            // V: the partial last page is copied by the whole warp, with the
+            // rows past the sequence end set to zero.
+            if (which == 1 && full_pages < npages) {
+                const int pg = full_pages;
+                const bool good = partial_phys >= 0;
+                const int valid = nk - pg * kPage;
+                for (int e = lane; e < kPage * C::KB * 8; e += 32) {
+                    const int r = e / (C::KB * 8);
+                    const int kb = (e / 8) % C::KB;
+                    const int c = e % 8;
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (good && r < valid) {
+                        const int64_t src =
+                            ((int64_t(partial_phys) * p.Hkv + it.g) * kPage + r) * D + kb * 64 + c * 8;
+                        v = __ldg(reinterpret_cast<const uint4 *>(
+                            static_cast<const __nv_bfloat16 *>(p.v_cache) + src));
                     }
-                    fence_proxy_async_smem();
-                    __syncwarp();
+                    *reinterpret_cast<uint4 *>(dst + kb * C::KV_KB_BYTES + swz(pg * kPage + r, c)) = v;
                 }
-                // K: the pages holding valid keys.  V: whole valid pages plus
-                // all-zero (out-of-bounds) boxes for the pages past the end.
-                const int tma_pages = which ? (kSplit / kPage) - (npages - full_pages) : npages;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[slot], uint32_t(tma_pages) * C::KB * C::PAGE_KB_BYTES);
-                    armed |= 1u << slot;
-                    armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
-                }
+                fence_proxy_async_smem();
                 __syncwarp();
-                const int pg = lane;
-                bool issue;
-                int r = row;
-                if (which == 0) {
-                    issue = pg < npages;
-                } else {
-                    issue = pg < kSplit / kPage && !(pg == full_pages && full_pages < npages);
-                    if (pg >= full_pages) r = -kPage;  // past the end: zero box
-                }
-                if (issue) {
-                    for (int kb = 0; kb < C::KB; ++kb)
-                        tma_load_2d(dst + kb * C::KV_KB_BYTES + pg * C::PAGE_KB_BYTES, map,
-                                    &full[slot], kb * 64, r);
-                }
-                __syncwarp();
-                if (++slot == C::NSLOT) {
-                    slot = 0;
-                    phase ^= 1u;
-                }
             }
+            // K: the pages holding valid keys.  V: whole valid pages plus
+            // all-zero (out-of-bounds) boxes for the pages past the end.
+            const int tma_pages = which ? (kSplit / kPage) - (npages - full_pages) : npages;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&full[slot], uint32_t(tma_pages) * C::KB * C::PAGE_KB_BYTES);
+                armed |= 1u << slot;
+                armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
+            }
+            __syncwarp();
+            const int pg = lane;
+            bool issue;
+            int r = row;
+            if (which == 0) {
+                issue = pg < npages;
+            } else {
+                issue = pg < kSplit / kPage && !(pg == full_pages && full_pages < npages);
+                if (pg >= full_pages) r = -kPage;  // past the end: zero box
+            }
+            if (issue) {
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tma_load_2d(dst + kb * C::KV_KB_BYTES + pg * C::PAGE_KB_BYTES, map, &full[slot],
+                                kb * 64, r);
+            }
+            __syncwarp();
+            if (++slot == C::NSLOT) {
+                slot = 0;
+                phase ^= 1u;
+            }
+            return true;
+        };
+        if (n > 0) ok = emit(0, 0);
+        if (ok && n > 1) ok = emit(0, 1);
+        for (int j = 0; ok && j < n; ++j) {
+            ok = emit(1, j);
+            // split j is done with its page ids: look up split j + 4
+            pages[j & 3] = (j + 4 < n) ? lookup(it.s0 + j + 4) : -1;
+            if (ok && j + 2 < n) ok = emit(0, j + 2);
         }
         if (!ok && lane == 0) {
             for (int s = 0; s < C::NSLOT; ++s)
@@ -437,15 +449,20 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else if (warp == 1) {
         // ====================================================== MMA issue
         // Tensor-pipe order: QK(s0), QK(s0+1), PV(s0), QK(s0+2), PV(s0+1),
-        // ...; split s uses TMEM buffer (s - s0) & 1, which QK(s+2) reuses
-        // once the fold warps have merged O_s(s).
+        // ... -- the order of the producer's load list; split s uses TMEM
+        // buffer (s - s0) & 1, which QK(s+2) reuses once the fold warps
+        // have merged O_s(s).
         if (lane == 0) {
             const uint32_t idesc_qk = idesc_bf16_f32(128, kSplit, 0, 0);
             const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t q_base = smem_u32(sQ);
             bool ok = wait(barQ, 0, ctl);
+            // index of each load in the producer's list K0, K1, V0, K2, V1, ...
+            const int n = it.s1 - it.s0;
+            auto k_index = [](int j) { return j < 2 ? j : 2 * j - 1; };
+            auto v_index = [n](int j) { return min(2 + 2 * j, 2 * n - 1); };
             auto issue_qk = [&](int s) -> bool {
-                const int i = 2 * (s - it.s0);
+                const int i = k_index(s - it.s0);
                 const int slot = i % C::NSLOT;
                 if (!wait(&full[slot], uint32_t(i / C::NSLOT) & 1u, ctl)) return false;
                 tc_fence_after();
@@ -467,7 +484,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int s = it.s0; ok && s < it.s1; ++s) {
                 const int b = (s - it.s0) & 1;
                 const uint32_t par = uint32_t((s - it.s0) >> 1) & 1u;
-                const int i = 2 * (s - it.s0) + 1;
+                const int i = v_index(s - it.s0);
                 const int slot = i % C::NSLOT;
                 if (!wait(&full[slot], uint32_t(i / C::NSLOT) & 1u, ctl)) {
                     ok = false;
@@ -601,17 +618,23 @@ __global__ void __launch_bounds__(THREADS, 1)
                         float mn, a, cc;
                         merge_scales(m, m_s, mn, a, cc);
 #pragma unroll
-                        for (int c = 0; c < D / 16; ++c) {
-                            uint32_t r0[16];
+                        for (int c = 0; c < D / 16; c += 2) {
+                            uint32_t r0[16], r1[16];
                             tmem_ld16(ob + 16 * c, r0);
+                            tmem_ld16(ob + 16 * c + 16, r1);
                             tmem_wait_ld(r0);
+                            tmem_wait_ld(r1);
 #pragma unroll
                             for (int j = 0; j < 16; ++j) {
                                 const float o0 = __uint_as_float(r0[j]);
-                                if (first)
+                                const float o1 = __uint_as_float(r1[j]);
+                                if (first) {
                                     O[16 * c + j] = o0;
-                                else if (take)
+                                    O[16 * c + 16 + j] = o1;
+                                } else if (take) {
                                     O[16 * c + j] = merge_val(O[16 * c + j], a, o0, cc);
+                                    O[16 * c + 16 + j] = merge_val(O[16 * c + 16 + j], a, o1, cc);
+                                }
                             }
                         }
                         if (first) {
