@@ -313,6 +313,7 @@ def invariance_checks(torch, L, wl) -> dict:
 def cpu_baseline(wl, budget_s: float = 20.0) -> dict:
     """The oracle (fp64, OpenMP) on a bounded sample of the same workload."""
     import oracle
+    from synth import kv_from_blocks
 
     cores = oracle.num_threads()
     # matmul: rows of the step's x (after RMSNorm, which the oracle recomputes)
@@ -335,8 +336,8 @@ def cpu_baseline(wl, budget_s: float = 20.0) -> dict:
         b = int(order[(done * 16) % DEC_B])
         Lb = int(wl.dec_lens_np[b])
         pages = wl.dec_bt_np[b, :(Lb + 15) // 16].tolist()
-        k = kc[pages].view(torch.int16).cpu().numpy().view(np.uint16)
-        v = vc[pages].view(torch.int16).cpu().numpy().view(np.uint16)
+        k = kv_from_blocks(kc[pages].view(torch.int16).cpu().numpy().view(np.uint16))
+        v = kv_from_blocks(vc[pages].view(torch.int16).cpu().numpy().view(np.uint16))
         bt = np.arange(len(pages), dtype=np.int32)[None, :]
         q = wl.dec_q[b].view(torch.int16).cpu().numpy().view(np.uint16)
         ts = time.perf_counter()

@@ -59,9 +59,16 @@ typedef enum {
 /*
  * Paged KV cache (vLLM-style paging, as the neican.ai insight describes in
  * section "技术原理与创新点解析", batch-invariant attention bullet).
- *   k_cache, v_cache : device, bf16 [num_pages, num_kv_heads, 16, head_dim].
- *                      The 16 x head_dim block of one (page, kv head) is
- *                      contiguous.  Both start 16-byte aligned.
+ *   k_cache, v_cache : device, bf16.  num_pages x num_kv_heads page blocks of
+ *                      16 x head_dim values, each block contiguous
+ *                      (32 * head_dim bytes) and stored in core-matrix order:
+ *                        block[kg][vg][r][c] = X[token 8*kg + r][value 8*vg + c]
+ *                      for kg in 0..1, vg in 0..head_dim/8-1, r, c in 0..7
+ *                      (token = position inside the page).  This is the
+ *                      order the tensor core reads its operands in, so a page
+ *                      block is copied to shared memory unchanged.  Blocks
+ *                      are indexed [page][kv head].  Both caches start
+ *                      16-byte aligned.  bi_kv_write produces this layout.
  *   block_table      : device, int32 [num_seqs, max_pages_per_seq];
  *                      block_table[b][i] is the physical page holding tokens
  *                      16*i .. 16*i+15 of sequence b.  Entries past a

@@ -46,9 +46,11 @@ class _PagedKV(ctypes.Structure):
 
 @dataclass
 class PagedKV:
-    """A paged KV cache on the device: ``k_cache``/``v_cache`` bf16
-    ``[num_pages, Hkv, 16, d]`` and ``block_table`` int32 ``[num_seqs,
-    max_pages]``.  The caller owns the tensors."""
+    """A paged KV cache on the device: ``k_cache``/``v_cache`` bf16 tensors
+    of shape ``[num_pages, Hkv, 16, d]`` holding one 16 x d block per (page,
+    kv head), each block stored in the tensor core's core-matrix order (see
+    ``include/bi.h``; ``bi_kv_write`` produces it), and ``block_table`` int32
+    ``[num_seqs, max_pages]``.  The caller owns the tensors."""
 
     k_cache: torch.Tensor
     v_cache: torch.Tensor

@@ -84,9 +84,8 @@ bool kv_ok(const bi_paged_kv *kv)
     if (kv->page_size != BI_PAGE_SIZE) return false;
     if (kv->num_kv_heads < 1 || kv->num_pages < 1 || kv->max_pages_per_seq < 1) return false;
     if (!aligned16(kv->k_cache) || !aligned16(kv->v_cache)) return false;
-    // TMA row coordinates of the cache are 32-bit
-    if (int64_t(kv->num_pages) * kv->num_kv_heads * BI_PAGE_SIZE >= (int64_t(1) << 31))
-        return false;
+    // page ids and (page, head) block indices are 32-bit
+    if (int64_t(kv->num_pages) * kv->num_kv_heads >= (int64_t(1) << 31)) return false;
     return true;
 }
 
@@ -233,6 +232,7 @@ bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, flo
     if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return BI_ERR_WORKSPACE;
 
     bi::AttnParams p{};
+    p.k_cache = kv->k_cache;
     p.v_cache = kv->v_cache;
     p.block_table = kv->block_table;
     p.max_pages = kv->max_pages_per_seq;
@@ -253,18 +253,13 @@ bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, flo
     p.status = d->status;
     p.timeout_ns = bi::kDefaultTimeoutNs;
 
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq;
     const uint64_t dq[3] = {uint64_t(D), uint64_t(Hq), uint64_t(B)};
     const uint64_t sq[2] = {uint64_t(D) * 2, uint64_t(Hq) * D * 2};
     const uint32_t bq[3] = {64, uint32_t(p.rows_per_q), 1};
-    const uint64_t dkv[2] = {uint64_t(D), uint64_t(kv->num_pages) * Hkv * BI_PAGE_SIZE};
-    const uint64_t skv[1] = {uint64_t(D) * 2};
-    const uint32_t bkv[2] = {64, BI_PAGE_SIZE};
-    if (!encode(&tq, q, 3, dq, sq, bq) || !encode(&tk, kv->k_cache, 2, dkv, skv, bkv) ||
-        !encode(&tv, kv->v_cache, 2, dkv, skv, bkv))
-        return BI_ERR_CUDA;
+    if (!encode(&tq, q, 3, dq, sq, bq)) return BI_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = bi::launch_attention(tq, tk, tv, p, D, s);
+    cudaError_t e = bi::launch_attention(tq, p, D, s);
     if (e != cudaSuccess) return BI_ERR_CUDA;
     if (chunks > 1) e = bi::launch_attn_combine(p, D, s);
     return from_cuda(e);
@@ -296,6 +291,7 @@ bi_status bi_attention_prefill(const bi_paged_kv *kv, const void *q, void *o, fl
 
     const int D = kv->head_dim, Hkv = kv->num_kv_heads;
     bi::AttnParams p{};
+    p.k_cache = kv->k_cache;
     p.v_cache = kv->v_cache;
     p.block_table = kv->block_table;
     p.max_pages = kv->max_pages_per_seq;
@@ -315,17 +311,12 @@ bi_status bi_attention_prefill(const bi_paged_kv *kv, const void *q, void *o, fl
     p.status = d->status;
     p.timeout_ns = bi::kDefaultTimeoutNs;
 
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq;
     const uint64_t dq[3] = {uint64_t(D), uint64_t(Hq), uint64_t(T_total)};
     const uint64_t sq[2] = {uint64_t(D) * 2, uint64_t(Hq) * D * 2};
     const uint32_t bq[3] = {64, 1, 128};
-    const uint64_t dkv[2] = {uint64_t(D), uint64_t(kv->num_pages) * Hkv * BI_PAGE_SIZE};
-    const uint64_t skv[1] = {uint64_t(D) * 2};
-    const uint32_t bkv[2] = {64, BI_PAGE_SIZE};
-    if (!encode(&tq, q, 3, dq, sq, bq) || !encode(&tk, kv->k_cache, 2, dkv, skv, bkv) ||
-        !encode(&tv, kv->v_cache, 2, dkv, skv, bkv))
-        return BI_ERR_CUDA;
-    return from_cuda(bi::launch_attention(tq, tk, tv, p, D, static_cast<cudaStream_t>(stream)));
+    if (!encode(&tq, q, 3, dq, sq, bq)) return BI_ERR_CUDA;
+    return from_cuda(bi::launch_attention(tq, p, D, static_cast<cudaStream_t>(stream)));
 }
 
 bi_status bi_device_status(void *stream)

@@ -35,11 +35,13 @@
 // how many blocks served a sequence.
 //
 // Block of 192 threads, one per SM (224 KB shared memory, 512 TMEM columns):
-//   warp 0     producer: Q by TMA once; per split K then V, 16 pages of
-//              [16 x 64] bf16 boxes each (gathered through the page table),
-//              into a 3-slot ring; the V rows past the sequence end are
-//              zero (TMA out-of-bounds fill for whole pages, explicit stores
-//              for the partial page) so that 0 * stale never reaches O.
+//   warp 0     producer: Q by TMA once; per split the 16 pages of K and of
+//              V, one bulk copy per page block (gathered through the page
+//              table; the cache keeps each page block in the tensor core's
+//              core-matrix order, so it is used in place), into a 3-slot
+//              ring; the V rows past the sequence end are zero (copies of a
+//              zero page, explicit stores for the partial page) so that
+//              0 * stale never reaches O.
 //   warp 1     TMEM allocation and MMA issue (one thread)
 //   warps 2-5  softmax and merge; warp w owns TMEM lanes 32(w%4)..+31.
 //              Decode spreads the query heads over the four lane quarters.
@@ -66,9 +68,11 @@ struct Cfg {
     static constexpr int KB = D / 64;                   // 128-byte column blocks of a row
     static constexpr int Q_KB_BYTES = 128 * 128;        // one column block of the Q tile
     static constexpr int Q_BYTES = KB * Q_KB_BYTES;
-    static constexpr int KV_KB_BYTES = kSplit * 128;    // one column block of a 256-key tile
-    static constexpr int KV_BYTES = KB * KV_KB_BYTES;
-    static constexpr int PAGE_KB_BYTES = kPage * 128;   // one page of one column block
+    // A cache page block (16 keys x D) in core-matrix order: 2 key groups
+    // of D/8 core matrices (8 keys x 8 values, 128 contiguous bytes).
+    static constexpr int PAGE_BYTES = kPage * D * 2;
+    static constexpr int KGROUP_BYTES = PAGE_BYTES / 2;  // stride between 8-key groups
+    static constexpr int KV_BYTES = (kSplit / kPage) * PAGE_BYTES;  // one split of K or V
     static constexpr int NSLOT = 3;
     static constexpr int ML_BYTES = 2 * 128 * 2 * 4;   // (m_s, l_s) per row, two buffers
     static constexpr int BAR_BYTES = 256;
@@ -79,6 +83,9 @@ struct Cfg {
     static constexpr uint32_t BUF_COLS = 256, P_OFF = 0, O_OFF = 128, TMEM_COLS = 512;
     static constexpr int REC = D + 4;                   // floats per spilled partial
 };
+
+// Source of the all-zero value pages past a sequence's end.
+__device__ __align__(128) uint8_t g_zero_page[kPage * 128 * 2];
 
 // ---------------------------------------------------------------- merge
 
@@ -171,10 +178,12 @@ __device__ __forceinline__ bool make_item(const AttnParams &p, Item &it)
     return true;
 }
 
-// Byte offset of 16-byte chunk `c` of row `r` in a 128-byte-swizzled tile.
-__device__ __forceinline__ uint32_t swz(int r, int c)
+// Byte offset, inside a page block in core-matrix order, of the 16 bytes
+// holding values 8c..8c+7 of key r.
+template <int D>
+__device__ __forceinline__ uint32_t page_off(int r, int c)
 {
-    return uint32_t(r) * 128u + (uint32_t((c ^ (r & 7))) << 4);
+    return uint32_t(r >> 3) * (D * 16) + uint32_t(c) * 128u + uint32_t(r & 7) * 16u;
 }
 
 // ---------------------------------------------------------------- kernel
@@ -192,14 +201,34 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[4][32])
     tmem_wait_ld(r[3]);
 }
 
-// Softmax of one split for the row owned by this thread.  S is read from
-// TMEM columns sb .. sb+255 in two passes of two 128-column loads; P (bf16
-// pairs) is written over columns sb .. sb+127 as the second pass goes (each
-// store lands on columns this thread has already read).  Returns m_s
-// (scaled, log2 units) and l_s.  (P V cannot start before the whole pass is
-// done: it writes O_s over the columns of the logits of keys 128..255.)
-__device__ __forceinline__ void split_softmax(uint32_t sb, int k0, int t, float cs, float &m_s,
-                                              float &l_s)
+// The order of the split sum l_s, shared by both softmax paths below.  The
+// 256 keys of a split are cut into 32-key chunks; inside a chunk, key
+// 32c + 8i + 2u + j (i < 4, u < 4, j < 2) belongs to class u.  For each class
+// u, S_u accumulates, chunk by chunk in key order, the chunk's eight class-u
+// values summed as ((a0 + b0) + (a1 + b1)) + ((a2 + b2) + (a3 + b3)) with
+// a_i = p[32c + 8i + 2u], b_i = p[32c + 8i + 2u + 1].  Then
+// l_s = (S_0 + S_1) + (S_2 + S_3).
+__device__ __forceinline__ float tree8(float a0, float b0, float a1, float b1, float a2, float b2,
+                                       float a3, float b3)
+{
+    return __fadd_rn(__fadd_rn(__fadd_rn(a0, b0), __fadd_rn(a1, b1)),
+                     __fadd_rn(__fadd_rn(a2, b2), __fadd_rn(a3, b3)));
+}
+
+__device__ __forceinline__ float logit(uint32_t s, float cs, float m_s)
+{
+    return ex2(__fsub_rn(__fmul_rn(__uint_as_float(s), cs), m_s));
+}
+
+// Softmax of one split, one row per thread (any row layout; used by
+// prefill and by decode with more than 8 query rows per lane quarter).
+// S is read from TMEM columns sb .. sb+255 in two passes of two 128-column
+// loads; P (bf16 pairs) is written over columns sb .. sb+127 as the second
+// pass goes (each store lands on columns this thread has already read).
+// Returns m_s (scaled, log2 units) and l_s.  (P V cannot start before the
+// whole pass is done: it writes O_s over the logits of keys 128..255.)
+__device__ __forceinline__ void softmax_rows(uint32_t sb, int k0, int t, float cs, float &m_s,
+                                             float &l_s)
 {
     // pass 1: maximum of the raw logits over the visible keys.  For c > 0,
     // x -> round(x * c) is monotonic, so max_j round(S_j c) = round(max_j S_j * c).
@@ -227,9 +256,9 @@ __device__ __forceinline__ void split_softmax(uint32_t sb, int k0, int t, float 
     const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
     m_s = __fmul_rn(mraw, cs);
-    // pass 2: p = 2^(round(S c) - m_s), masked keys 0; 32-key chunk sums by a
-    // pairwise tree, added to l_s chunk by chunk in key order.
-    float l = 0.0f;
+    // pass 2: p = 2^(round(S c) - m_s), masked keys 0; P into TMEM; the sum
+    // in the order described above.
+    float S[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll 1
     for (int c = 0; c < kSplit / 32; c += 4) {
         uint32_t r[4][32];
@@ -240,34 +269,95 @@ __device__ __forceinline__ void split_softmax(uint32_t sb, int k0, int t, float 
             float e[32];
             if (kc + 31 <= t) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    e[j] = ex2(__fsub_rn(__fmul_rn(__uint_as_float(r[h][j]), cs), m_s));
+                for (int j = 0; j < 32; ++j) e[j] = logit(r[h][j], cs, m_s);
             } else {
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    e[j] = (kc + j <= t)
-                               ? ex2(__fsub_rn(__fmul_rn(__uint_as_float(r[h][j]), cs), m_s))
-                               : 0.0f;
+                for (int j = 0; j < 32; ++j) e[j] = (kc + j <= t) ? logit(r[h][j], cs, m_s) : 0.0f;
             }
             uint32_t pk[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(e[2 * j], e[2 * j + 1]);
             tmem_st16(sb + 16 * (c + h), pk);
 #pragma unroll
-            for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-                for (int j = 0; j < w; ++j) e[j] = __fadd_rn(e[j], e[j + w]);
-            l = __fadd_rn(l, e[0]);
+            for (int u = 0; u < 4; ++u)
+                S[u] = __fadd_rn(S[u], tree8(e[2 * u], e[2 * u + 1], e[8 + 2 * u], e[9 + 2 * u],
+                                             e[16 + 2 * u], e[17 + 2 * u], e[24 + 2 * u],
+                                             e[25 + 2 * u]));
         }
     }
     tmem_wait_st();
-    l_s = l;
+    l_s = __fadd_rn(__fadd_rn(S[0], S[1]), __fadd_rn(S[2], S[3]));
+}
+
+// Softmax of one split for decode when the query rows of this lane quarter
+// sit in its lanes 0..7: four threads share a row.  Thread t = u + 4 v
+// handles lane v, keys 8m + 2u and 8m + 2u + 1 (m < 32) -- class u of the
+// order above -- read with the 16-lane TMEM shape, and writes the packed P
+// of those keys (P column 4m + u) with the matching 16-lane store.  The
+// arithmetic per row is the same as softmax_rows, so the bits are equal.
+// sb is the TMEM address of lane 0 of the quarter.
+__device__ __forceinline__ void softmax_heads16(uint32_t sb, int k0, int t, float cs, float &m_s,
+                                                float &l_s)
+{
+    const int u = threadIdx.x & 3;
+    float v[64];  // v[2m], v[2m+1]: keys 8m + 2u, 8m + 2u + 1
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t r[64];
+        tmem_ld_16x256b_x16(sb + 128 * h, r);
+        tmem_wait_ld(r);
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            v[2 * (16 * h + m)] = __uint_as_float(r[4 * m]);
+            v[2 * (16 * h + m) + 1] = __uint_as_float(r[4 * m + 1]);
+        }
+    }
+    const bool whole = k0 + kSplit - 1 <= t;  // every key of the split visible
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int m = 0; m < 32; ++m)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+            if (whole || k0 + 8 * m + 2 * u + j <= t) mx[m & 3] = fmaxf(mx[m & 3], v[2 * m + j]);
+    float mraw = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+    mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 1));
+    mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 2));
+    m_s = __fmul_rn(mraw, cs);
+
+    float S = 0.0f;
+    uint32_t pk[2][32];  // 16x128b store operands: [half][2 * m' + lane-half]
+#pragma unroll
+    for (int c = 0; c < kSplit / 32; ++c) {
+        float e[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int m = 4 * c + i;
+                const float x = ex2(__fsub_rn(__fmul_rn(v[2 * m + j], cs), m_s));
+                e[2 * i + j] = (whole || k0 + 8 * m + 2 * u + j <= t) ? x : 0.0f;
+            }
+        S = __fadd_rn(S, tree8(e[0], e[1], e[2], e[3], e[4], e[5], e[6], e[7]));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int m = 4 * c + i;
+            pk[m >> 4][2 * (m & 15)] = pack_bf16x2(e[2 * i], e[2 * i + 1]);
+            pk[m >> 4][2 * (m & 15) + 1] = 0u;  // lanes 8..15 hold no query row
+        }
+    }
+    tmem_st_16x128b_x16(sb, pk[0]);
+    tmem_st_16x128b_x16(sb + 64, pk[1]);
+    tmem_wait_st();
+    // (S_u + S_u^1) + (S_u^2 + S_u^3): commutativity gives every thread the
+    // same bits.
+    S = __fadd_rn(S, __shfl_xor_sync(0xffffffffu, S, 1));
+    S = __fadd_rn(S, __shfl_xor_sync(0xffffffffu, S, 2));
+    l_s = S;
 }
 
 template <int D>
 __global__ void __launch_bounds__(THREADS, 1)
-    attn_split_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                      const __grid_constant__ CUtensorMap tv, const AttnParams p)
+    attn_split_kernel(const __grid_constant__ CUtensorMap tq, const AttnParams p)
 {
     using C = Cfg<D>;
     Item it;
@@ -343,17 +433,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tma_load_3d(sQ + kb * C::Q_KB_BYTES, &tq, barQ, kb * 64, it.h, it.q_row0);
             }
         }
-        // Lane i < 16 looks up page i of a split, one split ahead, and
-        // issues that page's boxes itself.
+        // Lane i < 16 looks up page i of a split ahead of use and issues
+        // that page's boxes itself.  The id is only loaded here; it is
+        // checked where it is used, so the load overlaps other work.
         auto lookup = [&](int s) -> int {
             const int lp = s * (kSplit / kPage) + lane;  // logical page
             if (lane >= kSplit / kPage || lp * kPage >= it.kv_len) return -1;
-            const int phys = lp < p.max_pages ? __ldg(bt_row + lp) : -1;
-            if (phys < 0 || phys >= p.num_pages) {
-                record_status(p.status, BI_DEV_BAD_INDEX);
-                return -1;
-            }
-            return phys;
+            return lp < p.max_pages ? __ldg(bt_row + lp) : -2;
         };
         // Load list (relative split j, n splits): K0, K1, V0, K2, V1, K3,
         // ..., V(n-2), V(n-1): keys two splits ahead of values, which is the
@@ -368,64 +454,60 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int e = 0; e < 4; ++e) pages[e] = e < n ? lookup(it.s0 + e) : -1;
         auto emit = [&](int which, int j) -> bool {
             const int s = it.s0 + j;
-            const int phys = pages[j & 3];
+            int phys = pages[j & 3];
+            if (phys == -2 || phys >= p.num_pages || phys < -1) {  // bad id: zero box, flagged
+                if (which == 0) record_status(p.status, BI_DEV_BAD_INDEX);
+                phys = -1;
+            }
             const int nk = min(kSplit, it.kv_len - s * kSplit);  // valid keys, >= 1
             const int full_pages = nk / kPage;
             const int npages = (nk + kPage - 1) / kPage;
-            // box row of this lane's page; -16 = out of bounds, zero filled
-            const int row = phys >= 0 ? (phys * p.Hkv + it.g) * kPage : -kPage;
             int got = 1;
             if (lane == 0) got = wait(&empty[slot], phase ^ 1u, ctl) ? 1 : 0;
             got = __shfl_sync(0xffffffffu, got, 0);
             if (!got) return false;
             uint8_t *dst = sKV + slot * C::KV_BYTES;
-            const CUtensorMap *map = which ? &tv : &tk;
+            const uint8_t *cache = static_cast<const uint8_t *>(which ? p.v_cache : p.k_cache);
             const int partial_phys = __shfl_sync(0xffffffffu, phys, full_pages & 31);
             // V: the partial last page is copied by the whole warp, with the
-            // rows past the sequence end set to zero.
+            // keys past the sequence end set to zero.
             if (which == 1 && full_pages < npages) {
                 const int pg = full_pages;
                 const bool good = partial_phys >= 0;
                 const int valid = nk - pg * kPage;
-                for (int e = lane; e < kPage * C::KB * 8; e += 32) {
-                    const int r = e / (C::KB * 8);
-                    const int kb = (e / 8) % C::KB;
-                    const int c = e % 8;
+                const uint8_t *blk =
+                    cache + (int64_t(partial_phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
+                for (int e = lane; e < kPage * (D / 8); e += 32) {
+                    const int r = e / (D / 8), c = e % (D / 8);
+                    const uint32_t off = page_off<D>(r, c);
                     uint4 v = make_uint4(0, 0, 0, 0);
-                    if (good && r < valid) {
-                        const int64_t src =
-                            ((int64_t(partial_phys) * p.Hkv + it.g) * kPage + r) * D + kb * 64 + c * 8;
-                        v = __ldg(reinterpret_cast<const uint4 *>(
-                            static_cast<const __nv_bfloat16 *>(p.v_cache) + src));
-                    }
-                    *reinterpret_cast<uint4 *>(dst + kb * C::KV_KB_BYTES + swz(pg * kPage + r, c)) = v;
+                    if (good && r < valid) v = __ldg(reinterpret_cast<const uint4 *>(blk + off));
+                    *reinterpret_cast<uint4 *>(dst + pg * C::PAGE_BYTES + off) = v;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
             }
             // K: the pages holding valid keys.  V: whole valid pages plus
-            // all-zero (out-of-bounds) boxes for the pages past the end.
-            const int tma_pages = which ? (kSplit / kPage) - (npages - full_pages) : npages;
+            // all-zero pages past the end.  One bulk copy per page.
+            const int copies = which ? (kSplit / kPage) - (npages - full_pages) : npages;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&full[slot], uint32_t(tma_pages) * C::KB * C::PAGE_KB_BYTES);
+                mbar_arrive_expect_tx(&full[slot], uint32_t(copies) * C::PAGE_BYTES);
                 armed |= 1u << slot;
                 armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
             }
             __syncwarp();
             const int pg = lane;
             bool issue;
-            int r = row;
+            const uint8_t *src = g_zero_page;
             if (which == 0) {
                 issue = pg < npages;
+                if (phys >= 0) src = cache + (int64_t(phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
             } else {
                 issue = pg < kSplit / kPage && !(pg == full_pages && full_pages < npages);
-                if (pg >= full_pages) r = -kPage;  // past the end: zero box
+                if (pg < full_pages && phys >= 0)
+                    src = cache + (int64_t(phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
             }
-            if (issue) {
-                for (int kb = 0; kb < C::KB; ++kb)
-                    tma_load_2d(dst + kb * C::KV_KB_BYTES + pg * C::PAGE_KB_BYTES, map, &full[slot],
-                                kb * 64, r);
-            }
+            if (issue) bulk_load(dst + pg * C::PAGE_BYTES, src, C::PAGE_BYTES, &full[slot]);
             __syncwarp();
             if (++slot == C::NSLOT) {
                 slot = 0;
@@ -471,8 +553,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t kb = k >> 2, kk = k & 3;
+                    // K: K-major, core matrices; 16 values of the head dim
+                    // are two core matrices 128 bytes apart, 8-key groups
+                    // are KGROUP_BYTES apart (also across pages).
                     mma_ss(d, sdesc_sw128(q_base + kb * C::Q_KB_BYTES + kk * 32, 16, 1024),
-                           sdesc_sw128(k_base + kb * C::KV_KB_BYTES + kk * 32, 16, 1024), idesc_qk,
+                           sdesc_plain(k_base + k * 256, 128, C::KGROUP_BYTES), idesc_qk,
                            k > 0 ? 1u : 0u);
                 }
                 mma_commit(&barS[(s - it.s0) & 1]);
@@ -499,8 +584,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int j = 0; j < kSplit / 16; ++j) {
+                    // V: MN-major, core matrices; step j is page j; its two
+                    // 8-key groups are KGROUP_BYTES apart, 8-value blocks of
+                    // the head dim 128 bytes apart.
                     mma_ts(buf + C::O_OFF, buf + C::P_OFF + 8 * j,
-                           sdesc_sw128(v_base + j * 16 * 128, C::KV_KB_BYTES, 1024), idesc_pv,
+                           sdesc_plain(v_base + j * C::PAGE_BYTES, C::KGROUP_BYTES, 128), idesc_pv,
                            j > 0 ? 1u : 0u);
                 }
                 mma_commit(&barO[b]);
@@ -548,6 +636,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (is_softmax) {
             // -------------------------------------------------- softmax
             const float cs = p.scale_log2;
+            const uint32_t quarter_base = tmem_addr(tmem, 32 * q, 0);
+            // decode with at most 8 query rows per quarter: the 16-lane path
+            const bool heads16 = p.decode && p.rows_per_q <= 8 && active;
             for (int s = it.s0; s < it.s1; ++s) {
                 const int b = (s - it.s0) & 1;
                 const uint32_t par = uint32_t((s - it.s0) >> 1) & 1u;
@@ -555,9 +646,19 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (!wait(&barS[b], par, ctl)) break;
                 tc_fence_after();
                 float m_s = -INFINITY, l_s = 0.0f;
-                if (active) split_softmax(sb + C::P_OFF, s * kSplit, t, cs, m_s, l_s);
-                sML[(b * 128 + row_id) * 2 + 0] = m_s;
-                sML[(b * 128 + row_id) * 2 + 1] = l_s;
+                if (heads16) {
+                    // rows of this quarter in lanes 0..7, four threads a row
+                    softmax_heads16(quarter_base + C::BUF_COLS * uint32_t(b) + C::P_OFF, s * kSplit,
+                                    t, cs, m_s, l_s);
+                    if ((lane & 3) == 0) {
+                        sML[(b * 128 + 32 * q + (lane >> 2)) * 2 + 0] = m_s;
+                        sML[(b * 128 + 32 * q + (lane >> 2)) * 2 + 1] = l_s;
+                    }
+                } else {
+                    if (active) softmax_rows(sb + C::P_OFF, s * kSplit, t, cs, m_s, l_s);
+                    sML[(b * 128 + row_id) * 2 + 0] = m_s;
+                    sML[(b * 128 + row_id) * 2 + 1] = l_s;
+                }
                 tc_fence_before();
                 mbar_arrive(&barP[b]);
             }
@@ -730,8 +831,8 @@ size_t attn_ws_bytes(int B, int Hq, int head_dim, int max_splits, int max_chunks
     return size_t(B) * Hq * max_splits * (head_dim + 4) * sizeof(float);
 }
 
-cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                             const AttnParams &p, int head_dim, cudaStream_t s)
+cudaError_t launch_attention(const CUtensorMap &tq, const AttnParams &p, int head_dim,
+                             cudaStream_t s)
 {
     dim3 grid;
     if (p.decode)
@@ -743,12 +844,12 @@ cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const
         e = cudaFuncSetAttribute(attn_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg<128>::SMEM);
         if (e != cudaSuccess) return e;
-        attn_split_kernel<128><<<grid, THREADS, Cfg<128>::SMEM, s>>>(tq, tk, tv, p);
+        attn_split_kernel<128><<<grid, THREADS, Cfg<128>::SMEM, s>>>(tq, p);
     } else {
         e = cudaFuncSetAttribute(attn_split_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg<64>::SMEM);
         if (e != cudaSuccess) return e;
-        attn_split_kernel<64><<<grid, THREADS, Cfg<64>::SMEM, s>>>(tq, tk, tv, p);
+        attn_split_kernel<64><<<grid, THREADS, Cfg<64>::SMEM, s>>>(tq, p);
     }
     return cudaGetLastError();
 }

@@ -32,8 +32,9 @@ cudaError_t launch_kv_write(void *k_cache, void *v_cache, int64_t num_pages, int
 
 // ---------------------------------------------------------------- attention
 struct AttnParams {
-    // cache
-    const void *v_cache;       // read directly for the partial last page of V
+    // cache (page blocks in core-matrix order, see include/bi.h)
+    const void *k_cache;
+    const void *v_cache;
     const int32_t *block_table;
     int32_t max_pages;
     int32_t num_pages;
@@ -61,8 +62,8 @@ struct AttnParams {
 
 size_t attn_smem_bytes(int head_dim);
 size_t attn_ws_bytes(int B, int Hq, int head_dim, int max_splits, int max_chunks);
-cudaError_t launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                             const AttnParams &p, int head_dim, cudaStream_t s);
+cudaError_t launch_attention(const CUtensorMap &tq, const AttnParams &p, int head_dim,
+                             cudaStream_t s);
 cudaError_t launch_attn_combine(const AttnParams &p, int head_dim, cudaStream_t s);
 
 // ---------------------------------------------------------------- debug

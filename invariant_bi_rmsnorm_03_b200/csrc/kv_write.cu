@@ -4,9 +4,13 @@
 // before the kernel starts, so the kernel always sees one consistent
 // layout).
 //
-// Cache layout [num_pages, Hkv, 16, d] bf16; token t of the step with slot
-// s = slot_mapping[t] lands at page s / 16, offset s % 16 for every kv head.
-// One thread moves one 16-byte piece; a bit copy, so trivially invariant.
+// Cache layout: page blocks [num_pages, Hkv] of 16 x d bf16, each block in
+// core-matrix order [2 key groups][d/8 value groups][8 keys][8 values] (the
+// order the attention kernel's tensor-core operands use, so a block is
+// copied to shared memory as it is).  Token t of the step with slot
+// s = slot_mapping[t] lands at page s / 16, key s % 16 for every kv head.
+// One thread moves one 16-byte piece (8 values of one key); a bit copy, so
+// trivially invariant.
 //
 // Also here: the probe kernel of the bounded-wait path (bi_debug_bounded_wait).
 #include <cuda_runtime.h>
@@ -39,8 +43,11 @@ __global__ void kv_write_kernel(uint4 *__restrict__ kc, uint4 *__restrict__ vc, 
             if (piece == 0 && g == 0) record_status(status, BI_DEV_BAD_INDEX);
             continue;
         }
-        const int64_t page = slot / kPage, off = slot % kPage;
-        const int64_t dst = ((page * Hkv + g) * kPage + off) * pieces + piece;
+        const int64_t page = slot / kPage;
+        const int off = static_cast<int>(slot % kPage);
+        // page block in core-matrix order: [key group][value group][8 keys][8 values]
+        const int64_t dst = (page * Hkv + g) * (kPage * pieces) + (off >> 3) * (8 * pieces) +
+                            piece * 8 + (off & 7);
         kc[dst] = kn[i];
         vc[dst] = vn[i];
     }

@@ -136,6 +136,23 @@ def paged_kv(g: np.random.Generator, seq_lens, num_kv_heads: int, head_dim: int,
     return PagedKV(k, v, bt, np.asarray(seq_lens, dtype=np.int32), num_kv_heads, head_dim)
 
 
+def kv_to_blocks(cache: np.ndarray) -> np.ndarray:
+    """Logical cache [num_pages, Hkv, 16, d] -> the device layout: each
+    (page, head) block of 16 x d values in core-matrix order
+    [key group 2][value group d/8][8 keys][8 values].  A pure permutation."""
+    P, H, T, d = cache.shape
+    assert T == PAGE
+    x = cache.reshape(P, H, 2, 8, d // 8, 8)          # page, head, kg, r, vg, c
+    return np.ascontiguousarray(x.transpose(0, 1, 2, 4, 3, 5)).reshape(P, H, T, d)
+
+
+def kv_from_blocks(blocks: np.ndarray) -> np.ndarray:
+    """Inverse of kv_to_blocks."""
+    P, H, T, d = blocks.shape
+    x = blocks.reshape(P, H, 2, d // 8, 8, 8)         # page, head, kg, vg, r, c
+    return np.ascontiguousarray(x.transpose(0, 1, 2, 4, 3, 5)).reshape(P, H, T, d)
+
+
 def slot_mapping(block_table: np.ndarray, seq: int, positions) -> np.ndarray:
     """Physical slot (page * 16 + offset) of each absolute token position."""
     positions = np.asarray(positions, dtype=np.int64)

@@ -8,7 +8,8 @@ import torch
 import invariant_bi_rmsnorm_03_b200 as bi
 import oracle
 from gpu_util import DEV, TOL_BF16, dev_bf16, host_bits, rowwise_normwise, same_bytes, to_f64
-from synth import PagedKV, normal_bf16, page_table, paged_kv, rng, slot_mapping, tiny_layer
+from synth import (PagedKV, kv_from_blocks, kv_to_blocks, normal_bf16, page_table, paged_kv, rng,
+                   slot_mapping, tiny_layer)
 
 pytestmark = pytest.mark.gpu
 
@@ -21,7 +22,8 @@ def L():
 
 
 def dev_kv(kv: PagedKV) -> bi.PagedKV:
-    return bi.PagedKV(dev_bf16(kv.k_cache), dev_bf16(kv.v_cache),
+    """Upload a logical cache in the device's page-block layout."""
+    return bi.PagedKV(dev_bf16(kv_to_blocks(kv.k_cache)), dev_bf16(kv_to_blocks(kv.v_cache)),
                       torch.from_numpy(np.ascontiguousarray(kv.block_table)).to(DEV))
 
 
@@ -182,7 +184,8 @@ def write_sequence(L, S, Hkv, d, k_bits, v_bits, chunk=None, seed=0, fill="nan")
 
 
 def host_cache(dkv):
-    return host_bits(dkv.k_cache), host_bits(dkv.v_cache)
+    """Download a device cache as logical [num_pages, Hkv, 16, d] arrays."""
+    return kv_from_blocks(host_bits(dkv.k_cache)), kv_from_blocks(host_bits(dkv.v_cache))
 
 
 def test_prefill_parity_with_context(L):
@@ -283,8 +286,9 @@ def test_kv_write_is_a_bit_exact_scatter(L):
     L.bi_kv_write(dkv, dev_bf16(kn), dev_bf16(vn), torch.from_numpy(slots).to(DEV))
     kw, vw = kv.k_cache.copy(), kv.v_cache.copy()
     oracle.kv_write(kw, vw, kn, vn, slots)
-    np.testing.assert_array_equal(host_bits(dkv.k_cache), kw)
-    np.testing.assert_array_equal(host_bits(dkv.v_cache), vw)
+    kd, vd = host_cache(dkv)
+    np.testing.assert_array_equal(kd, kw)
+    np.testing.assert_array_equal(vd, vw)
     assert L.bi_device_status() == bi.Status.OK
 
 
@@ -296,7 +300,7 @@ def test_kv_write_out_of_range_slot_is_flagged(L):
     kn = normal_bf16(g, (1, 1, 64))
     L.bi_kv_write(dkv, dev_bf16(kn), dev_bf16(kn), torch.tensor([kv.num_pages * 16], device=DEV))
     assert L.bi_device_status() == bi.Status.DEVICE_INDEX
-    np.testing.assert_array_equal(host_bits(dkv.k_cache), before)
+    np.testing.assert_array_equal(host_bits(dkv.k_cache), before)  # untouched, any layout
     assert L.bi_device_status() == bi.Status.OK  # read-and-clear
 
 
