@@ -164,8 +164,10 @@ bi_status bi_kv_write(const bi_paged_kv *kv, const void *k_new, const void *v_ne
  *              picks a value from B, Hq/Hkv and the SM count.  It changes
  *              only the speed: the output bits do not depend on it.
  *   ws, ws_bytes : device workspace of at least
- *              bi_attention_decode_workspace_bytes(...) bytes (fp32 split
- *              partials; may be 0 bytes, in which case ws may be NULL).
+ *              bi_attention_decode_workspace_bytes(...) bytes, 16-byte
+ *              aligned: the launch order of the sequences (longest first)
+ *              and, when a sequence spans several blocks, the fp32 split
+ *              partials.
  *   Query head h reads kv head h / (Hq / num_kv_heads).  Keys are reduced in
  *   splits of 256 aligned to position 0; each split's partial (max, sum,
  *   weighted values) is formed on its own and the partials are merged from

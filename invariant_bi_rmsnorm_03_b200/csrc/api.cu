@@ -91,6 +91,10 @@ bool kv_ok(const bi_paged_kv *kv)
 
 bool head_dim_ok(int d) { return d == 64 || d == 128; }
 
+// Decode workspace: the launch order of the sequences (int32 [B], padded to
+// 256 bytes), then the split partials when a sequence spans several blocks.
+size_t order_bytes(int B) { return (size_t(B) * 4 + 255) / 256 * 256; }
+
 int decode_splits_per_cta(int B, int Hkv, int max_splits, int requested, int num_sms)
 {
     if (requested > 0) return requested < max_splits ? requested : max_splits;
@@ -204,7 +208,7 @@ size_t bi_attention_decode_workspace_bytes(const bi_paged_kv *kv, int32_t B, int
     const int max_splits = (max_seq_len + bi::kSplit - 1) / bi::kSplit;
     const int c = decode_splits_per_cta(B, kv->num_kv_heads, max_splits, splits_per_cta, d->num_sms);
     const int chunks = (max_splits + c - 1) / c;
-    return bi::attn_ws_bytes(B, Hq, kv->head_dim, max_splits, chunks);
+    return order_bytes(B) + bi::attn_ws_bytes(B, Hq, kv->head_dim, max_splits, chunks);
 }
 
 bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, float *lse,
@@ -228,8 +232,10 @@ bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, flo
     const int max_splits = (max_seq_len + bi::kSplit - 1) / bi::kSplit;
     const int c = decode_splits_per_cta(B, Hkv, max_splits, splits_per_cta, d->num_sms);
     const int chunks = (max_splits + c - 1) / c;
-    const size_t need = bi::attn_ws_bytes(B, Hq, D, max_splits, chunks);
-    if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return BI_ERR_WORKSPACE;
+    const size_t need = order_bytes(B) + bi::attn_ws_bytes(B, Hq, D, max_splits, chunks);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return BI_ERR_WORKSPACE;
+    int32_t *order = static_cast<int32_t *>(ws);
+    float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + order_bytes(B));
 
     bi::AttnParams p{};
     p.k_cache = kv->k_cache;
@@ -244,12 +250,13 @@ bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, flo
     p.decode = 1;
     p.B = B;
     p.seq_lens = seq_lens;
+    p.order = order;
     p.splits_per_cta = c;
     p.max_splits = max_splits;
     p.scale_log2 = float(double(scale) * 1.4426950408889634);
     p.o = o;
     p.lse = lse;
-    p.ws = static_cast<float *>(ws);
+    p.ws = partials;
     p.status = d->status;
     p.timeout_ns = bi::kDefaultTimeoutNs;
 
@@ -259,7 +266,9 @@ bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, flo
     const uint32_t bq[3] = {64, uint32_t(p.rows_per_q), 1};
     if (!encode(&tq, q, 3, dq, sq, bq)) return BI_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = bi::launch_attention(tq, p, D, s);
+    cudaError_t e = bi::launch_attn_order(seq_lens, B, order, s);
+    if (e != cudaSuccess) return BI_ERR_CUDA;
+    e = bi::launch_attention(tq, p, D, s);
     if (e != cudaSuccess) return BI_ERR_CUDA;
     if (chunks > 1) e = bi::launch_attn_combine(p, D, s);
     return from_cuda(e);

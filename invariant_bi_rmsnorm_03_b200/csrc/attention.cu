@@ -144,7 +144,7 @@ struct Item {
 __device__ __forceinline__ bool make_item(const AttnParams &p, Item &it)
 {
     if (p.decode) {
-        it.b = blockIdx.z;
+        it.b = p.order ? p.order[blockIdx.z] : static_cast<int>(blockIdx.z);
         it.g = blockIdx.y;
         it.h = 0;
         it.kv_len = p.seq_lens[it.b];
@@ -777,6 +777,51 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 }
 
+// Launch order of decode sequences: longest first (by split count), so that
+// the block scheduler, which starts blocks in index order, ends with short
+// ones (a greedy longest-processing-time schedule).  A counting sort over
+// at most 1024 length buckets; the order inside a bucket is whatever the
+// atomics give -- it changes which block runs when, never what a block
+// computes.
+__global__ void __launch_bounds__(1024) attn_order_kernel(const int32_t *__restrict__ seq_lens,
+                                                          int B, int32_t *__restrict__ order)
+{
+    __shared__ int cnt[1024];
+    __shared__ int warp_tot[32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    cnt[tid] = 0;
+    __syncthreads();
+    auto bucket = [](int L) {
+        const int n = L > 0 ? (L + kSplit - 1) / kSplit : 0;
+        return 1023 - (n < 1023 ? n : 1023);  // longest in bucket 0
+    };
+    for (int b = tid; b < B; b += 1024) atomicAdd(&cnt[bucket(seq_lens[b])], 1);
+    __syncthreads();
+    // exclusive prefix sum of cnt over the buckets
+    const int v = cnt[tid];
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = warp_tot[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        warp_tot[lane] = w;
+    }
+    __syncthreads();
+    cnt[tid] = x - v + (warp > 0 ? warp_tot[warp - 1] : 0);
+    __syncthreads();
+    for (int b = tid; b < B; b += 1024) order[atomicAdd(&cnt[bucket(seq_lens[b])], 1)] = b;
+}
+
 // Continues the merge of a decode row past the first block's range, split by
 // split in ascending order; one warp per (sequence, query head).
 template <int D>
@@ -851,6 +896,12 @@ cudaError_t launch_attention(const CUtensorMap &tq, const AttnParams &p, int hea
         if (e != cudaSuccess) return e;
         attn_split_kernel<64><<<grid, THREADS, Cfg<64>::SMEM, s>>>(tq, p);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn_order(const int32_t *seq_lens, int B, int32_t *order, cudaStream_t s)
+{
+    attn_order_kernel<<<1, 1024, 0, s>>>(seq_lens, B, order);
     return cudaGetLastError();
 }
 

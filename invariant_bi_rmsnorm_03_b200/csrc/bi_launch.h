@@ -46,6 +46,7 @@ struct AttnParams {
     int32_t decode;        // 1 decode, 0 prefill
     int32_t B;
     const int32_t *seq_lens;   // decode
+    const int32_t *order;      // decode: launch order of the sequences (or null)
     const int32_t *cu_q;       // prefill
     const int32_t *ctx_lens;   // prefill
     int32_t splits_per_cta;    // decode work division
@@ -65,6 +66,7 @@ size_t attn_ws_bytes(int B, int Hq, int head_dim, int max_splits, int max_chunks
 cudaError_t launch_attention(const CUtensorMap &tq, const AttnParams &p, int head_dim,
                              cudaStream_t s);
 cudaError_t launch_attn_combine(const AttnParams &p, int head_dim, cudaStream_t s);
+cudaError_t launch_attn_order(const int32_t *seq_lens, int B, int32_t *order, cudaStream_t s);
 
 // ---------------------------------------------------------------- debug
 cudaError_t launch_bounded_wait_probe(unsigned *status, uint64_t timeout_ns, cudaStream_t s);
