@@ -183,6 +183,42 @@ size_t bi_attention_decode_workspace_bytes(const bi_paged_kv *kv, int32_t B, int
                                            int32_t max_seq_len, int32_t splits_per_cta);
 
 /*
+ * bi_attention_decode_noalloc -- bi_attention_decode for callers that cannot
+ * allocate device memory.  (The pages have no counterpart of this entry
+ * point; it is an interface convenience of this library.)
+ *
+ * Some callers may not call cudaMalloc or any allocating routine: code that
+ * runs inside a host framework which owns every device allocation through
+ * its own pool, latency-critical serving loops where an allocation could
+ * synchronise the device or fail under fragmentation, and embedders whose
+ * memory budget is fixed when the process starts.  This variant takes no
+ * workspace: its scratch (the launch order of the sequences and the fp32
+ * split partials) lives in one fixed array of BI_NOALLOC_SCRATCH_BYTES
+ * inside the library, which every GPU that loads the library holds until
+ * the process exits.  The caller still passes q, o, lse and seq_lens.
+ *
+ * Arguments, layouts and output bits are exactly those of
+ * bi_attention_decode.  With splits_per_cta == 0 the work division is picked
+ * so that the scratch fits (falling back to one block per sequence, which
+ * changes only the speed); a request that cannot fit -- an explicit
+ * splits_per_cta whose partials exceed the array, or more sequences than
+ * the array can order -- returns BI_ERR_WORKSPACE before any launch.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any
+ * stream capture.  Every call on a device shares the one array and each
+ * call writes all of the scratch it later reads, so nothing has to start at
+ * zero; two calls whose work overlaps on the GPU (different streams without
+ * ordering) race on the array and must not be issued.  No device memory is
+ * allocated or freed.
+ */
+#define BI_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+bi_status bi_attention_decode_noalloc(const bi_paged_kv *kv, const void *q, void *o, float *lse,
+                                      const int32_t *seq_lens, int32_t B, int32_t Hq,
+                                      int32_t max_seq_len, float scale, int32_t splits_per_cta,
+                                      void *stream);
+
+/*
  * bi_attention_prefill -- causal attention of a batch of prompt chunks
  * against the paged cache (liuwei.blog, "破解之道": the order in which the
  * keys of token 1000 are reduced must not depend on whether the cache was

@@ -135,6 +135,8 @@ class Library:
         L.bi_build_invariant.restype = ctypes.c_int
         L.bi_device_status.argtypes = [P]
         L.bi_debug_bounded_wait.argtypes = [ctypes.c_uint64, P]
+        L.bi_attention_decode_noalloc.argtypes = [kvp, P, P, P, P, i32, i32, i32, f32, i32, P]
+        L.bi_attention_decode_noalloc.restype = st
         for name in ("bi_rmsnorm", "bi_matmul", "bi_kv_write", "bi_attention_decode",
                      "bi_attention_prefill", "bi_device_status", "bi_debug_bounded_wait"):
             getattr(L, name).restype = st
@@ -241,6 +243,31 @@ class Library:
             ctypes.byref(c), _ptr(q), _ptr(out), _ptr(lse), _ptr(seq_lens), B, Hq,
             int(max_seq_len), float(scale), int(splits_per_cta), _ptr(ws), nbytes,
             _stream(stream)))
+        return (out, lse) if want_lse else out
+
+    def bi_attention_decode_noalloc(self, kv: PagedKV, q: torch.Tensor, seq_lens: torch.Tensor,
+                                    max_seq_len: int, scale: float | None = None,
+                                    want_lse: bool = False, splits_per_cta: int = 0, out=None,
+                                    lse=None, stream=None):
+        """bi_attention_decode with its scratch in the library's fixed array
+        (no workspace, no device allocation by the library).  `out` and
+        `lse` are the caller's; pass them to avoid any allocation here."""
+        _need(q, "q", torch.bfloat16)
+        B, Hq, d = q.shape
+        _need(seq_lens, "seq_lens", torch.int32, (B,))
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        if out is None:
+            out = torch.empty_like(q)
+        _need(out, "out", torch.bfloat16, (B, Hq, d))
+        if want_lse and lse is None:
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        if lse is not None:
+            _need(lse, "lse", torch.float32, (B, Hq))
+        c = kv.c_struct()
+        self._check("bi_attention_decode_noalloc", self.lib.bi_attention_decode_noalloc(
+            ctypes.byref(c), _ptr(q), _ptr(out), _ptr(lse), _ptr(seq_lens), B, Hq,
+            int(max_seq_len), float(scale), int(splits_per_cta), _stream(stream)))
         return (out, lse) if want_lse else out
 
     def bi_attention_prefill(self, kv: PagedKV, q: torch.Tensor, cu_q: torch.Tensor,

@@ -274,6 +274,109 @@ bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, flo
     return from_cuda(e);
 }
 
+// ---------------------------------------------------------------- no-alloc decode
+//
+// bi_attention_decode_noalloc: the same decode attention for callers that
+// cannot allocate device memory.  Its scratch (the launch order of the
+// sequences and the split partials) is this fixed array, which every GPU
+// that loads the library holds until the process exits.
+static __device__ __align__(256) uint8_t g_decode_scratch[BI_NOALLOC_SCRATCH_BYTES];
+
+static std::mutex g_scratch_mu;
+static void *g_scratch_addr[kMaxDevices];
+
+// Device address of the scratch array on the current device, looked up once
+// per device.  (In host code the array's name is a host-side stand-in, not a
+// device address, so it is never handed to a kernel directly.)
+static bi_status decode_scratch(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BI_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr)
+            return BI_ERR_CUDA;
+        g_scratch_addr[dev] = ptr;
+    }
+    *out = g_scratch_addr[dev];
+    return BI_OK;
+}
+
+bi_status bi_attention_decode_noalloc(const bi_paged_kv *kv, const void *q, void *o, float *lse,
+                                      const int32_t *seq_lens, int32_t B, int32_t Hq,
+                                      int32_t max_seq_len, float scale, int32_t splits_per_cta,
+                                      void *stream)
+{
+    if (!attn_common_ok(kv, Hq)) return BI_ERR_INVALID;
+    if (!head_dim_ok(kv->head_dim)) return BI_ERR_UNSUPPORTED;
+    if (B < 0 || max_seq_len < 1 || splits_per_cta < 0 || !std::isfinite(scale))
+        return BI_ERR_INVALID;
+    if (int64_t(max_seq_len) > int64_t(kv->max_pages_per_seq) * BI_PAGE_SIZE) return BI_ERR_INVALID;
+    if (B == 0) return BI_OK;
+    if (B > 65535) return BI_ERR_UNSUPPORTED;
+    if (!q || !o || !seq_lens || !aligned16(q) || !aligned16(o)) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    void *scratch = nullptr;
+    st = decode_scratch(&scratch);
+    if (st != BI_OK) return st;
+
+    const int D = kv->head_dim, Hkv = kv->num_kv_heads, group = Hq / Hkv;
+    const int max_splits = (max_seq_len + bi::kSplit - 1) / bi::kSplit;
+    int c = decode_splits_per_cta(B, Hkv, max_splits, splits_per_cta, d->num_sms);
+    int chunks = (max_splits + c - 1) / c;
+    size_t need = order_bytes(B) + bi::attn_ws_bytes(B, Hq, D, max_splits, chunks);
+    if (need > BI_NOALLOC_SCRATCH_BYTES && splits_per_cta == 0) {
+        // The work division chosen from the load would need more partials
+        // than the array holds: give each sequence one block instead (the
+        // output bits do not depend on the division).
+        c = max_splits;
+        chunks = 1;
+        need = order_bytes(B);
+    }
+    if (need > BI_NOALLOC_SCRATCH_BYTES) return BI_ERR_WORKSPACE;
+    int32_t *order = static_cast<int32_t *>(scratch);
+    float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(scratch) + order_bytes(B));
+
+    bi::AttnParams p{};
+    p.k_cache = kv->k_cache;
+    p.v_cache = kv->v_cache;
+    p.block_table = kv->block_table;
+    p.max_pages = kv->max_pages_per_seq;
+    p.num_pages = kv->num_pages;
+    p.Hkv = Hkv;
+    p.Hq = Hq;
+    p.group = group;
+    p.rows_per_q = (group + 3) / 4;
+    p.decode = 1;
+    p.B = B;
+    p.seq_lens = seq_lens;
+    p.order = order;
+    p.splits_per_cta = c;
+    p.max_splits = max_splits;
+    p.scale_log2 = float(double(scale) * 1.4426950408889634);
+    p.o = o;
+    p.lse = lse;
+    p.ws = partials;
+    p.status = d->status;
+    p.timeout_ns = bi::kDefaultTimeoutNs;
+
+    CUtensorMap tq;
+    const uint64_t dq[3] = {uint64_t(D), uint64_t(Hq), uint64_t(B)};
+    const uint64_t sq[2] = {uint64_t(D) * 2, uint64_t(Hq) * D * 2};
+    const uint32_t bq[3] = {64, uint32_t(p.rows_per_q), 1};
+    if (!encode(&tq, q, 3, dq, sq, bq)) return BI_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = bi::launch_attn_order(seq_lens, B, order, s);
+    if (e != cudaSuccess) return BI_ERR_CUDA;
+    e = bi::launch_attention(tq, p, D, s);
+    if (e != cudaSuccess) return BI_ERR_CUDA;
+    if (chunks > 1) e = bi::launch_attn_combine(p, D, s);
+    return from_cuda(e);
+}
+
 size_t bi_attention_prefill_workspace_bytes(const bi_paged_kv *kv, int32_t B, int32_t Hq,
                                             int32_t max_q_len)
 {
