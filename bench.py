@@ -582,7 +582,12 @@ def run_profile_case(args):
     L = bi.load(variant=args.variant)
     T = torch
     d16 = lambda a: T.from_numpy(a.view(np.int16)).to(dev).view(T.bfloat16)  # noqa: E731
-    if args.profile in ("rmsnorm", "matmul"):
+    if args.profile == "copy":
+        # size-matched reference for RMSNorm: a device copy of x[2048,4096]
+        xs = [d16(norm_matmul(seed=10 + i, M=M_ROWS, H=H, N=8)["x"]) for i in range(16)]
+        ys = [torch.empty_like(x) for x in xs]
+        fn = lambda i: ys[i % 16].copy_(xs[i % 16])  # noqa: E731
+    elif args.profile in ("rmsnorm", "matmul"):
         nm = norm_matmul(seed=1, M=M_ROWS, H=H, N=N_COLS)
         x, w, W = d16(nm["x"]), d16(nm["w"]), d16(nm["W"])
         if args.profile == "rmsnorm":
@@ -637,7 +642,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=20.0,
                     help="seconds of oracle work for the cpu_baseline sample")
-    ap.add_argument("--profile", choices=["rmsnorm", "matmul", "decode", "prefill"],
+    ap.add_argument("--profile", choices=["rmsnorm", "matmul", "decode", "prefill", "copy"],
                     help="run one kernel alone on a reduced case (for ncu)")
     ap.add_argument("--profile-batch", type=int, default=32)
     ap.add_argument("--profile-seq", type=int, default=4096)

@@ -752,12 +752,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
 
             if (ok && active && valid && !spill) {
-                if (!p.decode || it.s1 == it.n_splits) {
+                if (!p.decode || (it.s0 == 0 && it.s1 == it.n_splits)) {
                     write_out<D>(O, l, m, static_cast<__nv_bfloat16 *>(p.o) + out_row * D,
                                  p.lse ? p.lse + out_row : nullptr);
                 } else {
-                    // first block of a sequence served by several: hand the
-                    // merged state over split s1-1 to attn_combine
+                    // a block of a sequence served by several: hand the
+                    // merged state over its range (ending at split s1-1) to
+                    // attn_combine (in the invariant build only the first
+                    // block gets here; the others write every split)
                     float *rec = p.ws + ((out_row * p.max_splits) + (it.s1 - 1)) * C::REC;
                     rec[0] = m;
                     rec[1] = l;

@@ -87,8 +87,8 @@ __device__ __forceinline__ void store8(void *y, int64_t idx, const uint4 &xv, co
 // A block handles R rows at a time: all R rows are loaded before any is
 // reduced, so that more bytes are in flight.  R changes only how rows are
 // grouped into blocks; each row's arithmetic is the same for every R.
-template <int ITEMS, int R, bool OUT_F32>
-__global__ void __launch_bounds__(1024) rmsnorm_kernel(const uint4 *__restrict__ x,
+template <int ITEMS, int R, bool OUT_F32, int MAXT>
+__global__ void __launch_bounds__(MAXT, MAXT <= 256 ? 2 : 1) rmsnorm_kernel(const uint4 *__restrict__ x,
                                                        const uint4 *__restrict__ w,
                                                        void *__restrict__ y, int64_t M, int H,
                                                        float eps)
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(1024) rmsnorm_kernel(const uint4 *__restrict__
     }
 }
 
-template <int ITEMS, int R>
+template <int ITEMS, int R, int MAXT>
 cudaError_t launch_rows(const void *x, const void *w, void *y, int64_t M, int H, float eps,
                         bool out_f32, int threads, cudaStream_t s)
 {
@@ -150,24 +150,35 @@ cudaError_t launch_rows(const void *x, const void *w, void *y, int64_t M, int H,
     const int64_t groups = (M + R - 1) / R;
     const unsigned grid = static_cast<unsigned>(groups < cap ? groups : cap);
     if (out_f32)
-        rmsnorm_kernel<ITEMS, R, true><<<grid, threads, 0, s>>>(
+        rmsnorm_kernel<ITEMS, R, true, MAXT><<<grid, threads, 0, s>>>(
             static_cast<const uint4 *>(x), static_cast<const uint4 *>(w), y, M, H, eps);
     else
-        rmsnorm_kernel<ITEMS, R, false><<<grid, threads, 0, s>>>(
+        rmsnorm_kernel<ITEMS, R, false, MAXT><<<grid, threads, 0, s>>>(
             static_cast<const uint4 *>(x), static_cast<const uint4 *>(w), y, M, H, eps);
     return cudaGetLastError();
 }
 
+// Rows per block R with ITEMS * R 16-byte chunks held per thread: up to 16
+// (64 registers) for blocks of at most 256 threads, two blocks per SM;
+// up to 8 for wider blocks.
 template <int ITEMS>
 cudaError_t launch_items(const void *x, const void *w, void *y, int64_t M, int H, float eps,
                          bool out_f32, int threads, int rows_per_block, cudaStream_t s)
 {
-    // ITEMS * rows_per_block <= 8 (the host never asks for more)
-    if constexpr (ITEMS <= 2)
-        if (rows_per_block >= 4) return launch_rows<ITEMS, 4>(x, w, y, M, H, eps, out_f32, threads, s);
+    if (threads <= 256) {
+        if constexpr (ITEMS <= 2)
+            if (rows_per_block >= 8)
+                return launch_rows<ITEMS, 8, 256>(x, w, y, M, H, eps, out_f32, threads, s);
+        if constexpr (ITEMS <= 4)
+            if (rows_per_block >= 4)
+                return launch_rows<ITEMS, 4, 256>(x, w, y, M, H, eps, out_f32, threads, s);
+        if (rows_per_block >= 2) return launch_rows<ITEMS, 2, 256>(x, w, y, M, H, eps, out_f32, threads, s);
+        return launch_rows<ITEMS, 1, 256>(x, w, y, M, H, eps, out_f32, threads, s);
+    }
     if constexpr (ITEMS <= 4)
-        if (rows_per_block >= 2) return launch_rows<ITEMS, 2>(x, w, y, M, H, eps, out_f32, threads, s);
-    return launch_rows<ITEMS, 1>(x, w, y, M, H, eps, out_f32, threads, s);
+        if (rows_per_block >= 2)
+            return launch_rows<ITEMS, 2, 1024>(x, w, y, M, H, eps, out_f32, threads, s);
+    return launch_rows<ITEMS, 1, 1024>(x, w, y, M, H, eps, out_f32, threads, s);
 }
 
 }  // namespace
@@ -199,10 +210,13 @@ cudaError_t launch_rmsnorm(const void *x, const void *w, void *y, int64_t M, int
         threads = static_cast<int>((t + 31) / 32 * 32);
     }
 #endif
-    // Rows per block: enough that one wave of resident blocks covers M.
-    const int64_t resident = int64_t(num_sms) * (2048 / threads);
+    // Rows per block: enough that two blocks per SM cover M in one wave,
+    // within the registers a thread may hold (ITEMS * R <= 16; 8 for blocks
+    // wider than 256 threads).
+    const int64_t blocks = int64_t(num_sms) * (threads <= 256 ? 2 : 1);
+    const int cap = threads <= 256 ? 16 : 8;
     int rpb = 1;
-    while (rpb < 4 && int64_t(rpb) * resident < M && items * rpb < 8) rpb *= 2;
+    while (rpb < 8 && int64_t(rpb) * blocks < M && items * rpb * 2 <= cap) rpb *= 2;
     const int h = static_cast<int>(H);
     switch (items) {
     case 1: return launch_items<1>(x, w, y, M, h, eps, out_f32, threads, rpb, s);
