@@ -118,9 +118,9 @@ bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H
  *   the nn.Linear weight layout);  c : device, [M, N] of out_dtype.
  *   Requirements: K % 8 == 0, N % 8 == 0, M, N, K >= 1, all three pointers
  *   16-byte aligned, c not overlapping a or w.  M == 0 is a no-op.
- *   One fixed 128 x 256 output tile, K consumed in 64-wide slices in
- *   ascending order with fp32 accumulation on the tensor cores; there is no
- *   split-K and no choice of kernel by shape.
+ *   One fixed 256 x 256 output tile computed by a pair of SMs, K consumed in
+ *   64-wide slices in ascending order with fp32 accumulation on the tensor
+ *   cores; there is no split-K and no choice of kernel by shape.
  *   ws / ws_bytes: workspace (device); the invariant build needs none
  *   (bi_matmul_workspace_bytes returns 0, ws may be NULL).  The variant-off
  *   build uses it for split-K partial sums.

@@ -168,8 +168,9 @@ bi_status bi_matmul(const void *a, const void *w, void *c, int64_t M, int64_t N,
     CUtensorMap ta, tw;
     const uint64_t da[2] = {uint64_t(K), uint64_t(M)}, sa[1] = {uint64_t(K) * 2};
     const uint64_t dw[2] = {uint64_t(K), uint64_t(N)}, sw[1] = {uint64_t(K) * 2};
-    const uint32_t ba[2] = {uint32_t(bi::kGemmBK), uint32_t(bi::kGemmBM)};
-    const uint32_t bw[2] = {uint32_t(bi::kGemmBK), uint32_t(bi::kGemmBN)};
+    // each CTA of a pair loads 128 rows of A and 128 rows of W per K slice
+    const uint32_t ba[2] = {uint32_t(bi::kGemmBK), 128u};
+    const uint32_t bw[2] = {uint32_t(bi::kGemmBK), 128u};
     if (!encode(&ta, a, 2, da, sa, ba) || !encode(&tw, w, 2, dw, sw, bw)) return BI_ERR_CUDA;
     return from_cuda(bi::launch_gemm(ta, tw, c, int(M), int(N), int(K), out_dtype == BI_F32,
                                      static_cast<float *>(ws), ks, d->num_sms, d->status,

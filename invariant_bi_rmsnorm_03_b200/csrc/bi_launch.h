@@ -16,7 +16,7 @@ cudaError_t launch_rmsnorm(const void *x, const void *w, void *y, int64_t M, int
                            float eps, bool out_f32, int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- matmul
-constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64, kGemmStages = 4;
+constexpr int kGemmBK = 64;  // K slice; the output tile is 256 x 256 per SM pair
 size_t gemm_smem_bytes();
 // k_splits > 1 only in the variant-off build: fp32 partial sums go to ws
 // ([k_splits, M, N]) and a second kernel adds them.

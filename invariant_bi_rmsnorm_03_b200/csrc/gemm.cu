@@ -6,21 +6,25 @@
 // insight, "技术原理与创新点解析", data-parallel matmul bullet: the output is cut
 // into 2-D tiles and each core computes its tiles' whole dot products.
 //
-// One configuration for every shape: 128 x 256 output tiles, K consumed in
-// 64-wide slices in ascending order, four K=16 MMAs per slice accumulating
-// in fp32 in tensor memory.  Row m of A always lands in tile m / 128 at row
-// m % 128 and column n of W in tile n / 256, whatever M is; the K loop of an
-// output element never depends on M, N or on which block runs the tile.
-// Rows past M and K past the end are zero-filled by TMA.
+// One configuration for every shape: 256 x 256 output tiles, each computed
+// by a pair of SMs (a 2-CTA cluster, tcgen05.mma.cta_group::2), K consumed
+// in 64-wide slices in ascending order, four K=16 MMAs per slice
+// accumulating in fp32 in tensor memory.  Row m of A always lands in tile
+// m / 256 at row m % 256 (CTA (m % 256) / 128 of the pair) and column n of
+// W in tile n / 256, whatever M is; the K loop of an output element never
+// depends on M, N or on which pair runs the tile.  Rows past M and K past
+// the end are zero-filled by TMA.
 //
-// Block of 192 threads, one per SM, persistent over tiles:
-//   warp 0     TMA producer: A [128 x 64] and W [256 x 64] slices, 128-byte
-//              swizzle, into a 4-stage shared-memory ring (48 KB a stage)
-//   warp 1     TMEM allocation (512 columns = two 128 x 256 fp32
-//              accumulators) and MMA issue by one thread
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp reads its
-//              32-lane quarter), fp32 -> bf16 rounding, global stores; the
-//              second accumulator lets the next tile's MMAs run meanwhile.
+// Each CTA of a pair: 192 threads, one per SM, persistent over tiles:
+//   warp 0     TMA producer: this CTA's 128 rows of the A slice and 128 rows
+//              of the W slice (128-byte swizzle, 32 KB a stage, 6 stages),
+//              completing on the leader's barrier
+//   warp 1     TMEM allocation (512 columns: two 128 x 256 fp32
+//              accumulators, the pair allocating together) and, in the
+//              leader, MMA issue by one thread
+//   warps 2-5  epilogue: tcgen05.ld of this CTA's accumulator rows (each warp
+//              its 32-lane quarter), fp32 -> bf16 rounding, global stores;
+//              the second accumulator lets the next tile's MMAs run meanwhile.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -33,15 +37,6 @@
 
 namespace bi {
 namespace {
-
-constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK, STAGES = kGemmStages;
-constexpr int A_BYTES = BM * BK * 2;          // 16 KB
-constexpr int W_BYTES = BN * BK * 2;          // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + W_BYTES;
-constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 512;
-constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = 1024 /* alignment slack */ + STAGES * STAGE_BYTES + BAR_BYTES;
 
 struct Unit {
     int mb, nb, split, kb0, kb1;
@@ -103,10 +98,29 @@ __device__ __forceinline__ void store_row32(const uint32_t (&r)[32], void *c, fl
     }
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmw,
-                void *__restrict__ c, float *__restrict__ ws, int M, int N, int K, int out_f32,
-                int k_splits, unsigned *status, uint64_t timeout_ns)
+// ------------------------------------------------------------------ 2-SM kernel
+//
+// One 256 x 256 output tile per pair of SMs (a cluster of two CTAs): CTA r
+// of the pair owns rows 128r..128r+127 of the tile in its TMEM and holds,
+// per 64-wide K slice, its own 128 rows of A and W rows 128r..128r+127 of
+// the tile's 256 columns; the leader (r = 0) issues tcgen05.mma.cta_group::2
+// with M = 256, N = 256, which reads both CTAs' shared memory.  A CTA reads
+// 32 KB per K slice instead of 48, so six stages fit.
+namespace pair {
+
+constexpr int BM = 256, BN = 256, BK = kGemmBK, STAGES = 6;
+constexpr int A_BYTES = 128 * BK * 2;   // 16 KB: this CTA's half of the A slice
+constexpr int W_BYTES = 128 * BK * 2;   // 16 KB: this CTA's half of the W slice
+constexpr int STAGE_BYTES = A_BYTES + W_BYTES;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;     // two 128-lane x 256-column fp32 accumulators
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmw,
+                     void *__restrict__ c, float *__restrict__ ws, int M, int N, int K, int out_f32,
+                     int k_splits, unsigned *status, uint64_t timeout_ns)
 {
 #if BI_INVARIANT
     k_splits = 1;  // the invariant build never splits K
@@ -116,15 +130,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
     uint8_t *sA = smem;
     uint8_t *sW = smem + STAGES * A_BYTES;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);  // leader's used
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;
-    uint64_t *tempty = tfull + 2;
+    uint64_t *tempty = tfull + 2;   // leader's used: 8 arrivals (4 epilogue warps x 2 CTAs)
     uint64_t *drain = tempty + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -133,22 +149,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 128);
+            mbar_init(&tempty[a], 8);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tma);
-        tma_prefetch_desc(&tmw);
-    }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_holder, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // barriers and TMEM of both CTAs exist before either uses them
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const WaitCtl ctl{abort_flag, status, timeout_ns};
@@ -158,47 +170,44 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int kblocks = (K + BK - 1) / BK;
     const int kb_per = (kblocks + k_splits - 1) / k_splits;
     const int units = num_m * num_n * k_splits;
+    const int pair_id = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
 
     if (warp == 0) {
         if (lane == 0) {
-            // ------------------------------------------------ TMA producer
+            // ------------------------------------------------ TMA producer (both CTAs)
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t armed = 0, armed_parity = 0;  // per-stage bit sets
             bool ok = true;
-            for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
+            for (int u = pair_id; ok && u < units; u += num_pairs) {
                 const Unit t = unit_of(u, num_m, k_splits, kblocks, kb_per);
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
                     if (!wait(&empty[stage], phase ^ 1u, ctl)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-                    tma_load_2d(sA + stage * A_BYTES, &tma, &full[stage], kb * BK, t.mb * BM);
-                    tma_load_2d(sW + stage * W_BYTES, &tmw, &full[stage], kb * BK, t.nb * BN);
-                    armed |= 1u << stage;
-                    armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                    const uint32_t bar = map_to_cta(smem_u32(&full[stage]), 0);
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+                    tma_load_2d_pair(sA + stage * A_BYTES, &tma, bar, kb * BK,
+                                     t.mb * BM + int(rank) * 128);
+                    tma_load_2d_pair(sW + stage * W_BYTES, &tmw, bar, kb * BK,
+                                     t.nb * BN + int(rank) * 128);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
-            if (!ok) {
-                for (int s = 0; s < STAGES; ++s)
-                    if (armed & (1u << s)) wait_drain(&full[s], (armed_parity >> s) & 1u, timeout_ns);
-            }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ------------------------------------------------ MMA issue
+        if (lane == 0 && leader) {
+            // ------------------------------------------------ MMA issue (leader)
             const uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
+            for (int u = pair_id; ok && u < units; u += num_pairs) {
                 const Unit t = unit_of(u, num_m, k_splits, kblocks, kb_per);
                 if (!wait(&tempty[acc], acc_phase ^ 1u, ctl)) {
                     ok = false;
@@ -216,36 +225,38 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint32_t w0 = smem_u32(sW + stage * W_BYTES);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
-                        mma_ss(d, sdesc_sw128(a0 + 32 * k, 16, 1024),
-                               sdesc_sw128(w0 + 32 * k, 16, 1024), idesc,
-                               (kb > t.kb0 || k > 0) ? 1u : 0u);
+                        mma_ss_pair(d, sdesc_sw128(a0 + 32 * k, 16, 1024),
+                                    sdesc_sw128(w0 + 32 * k, 16, 1024), idesc,
+                                    (kb > t.kb0 || k > 0) ? 1u : 0u);
                     }
-                    mma_commit(&empty[stage]);
+                    mma_commit_pair(&empty[stage], 0x3);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                mma_commit(&tfull[acc]);
+                mma_commit_pair(&tfull[acc], 0x3);
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
             }
             if (!ok) {
-                mma_commit(drain);
+                mma_commit_pair(drain, 0x1);
                 wait_drain(drain, 0, timeout_ns);
             }
         }
     } else {
-        // ---------------------------------------------------- epilogue
+        // ---------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;
+        const uint32_t tempty_leader0 = map_to_cta(smem_u32(&tempty[0]), 0);
+        const uint32_t tempty_leader1 = map_to_cta(smem_u32(&tempty[1]), 0);
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int u = blockIdx.x; u < units; u += gridDim.x) {
+        for (int u = pair_id; u < units; u += num_pairs) {
             const Unit t = unit_of(u, num_m, k_splits, kblocks, kb_per);
             if (!wait(&tfull[acc], acc_phase, ctl)) break;
             tc_fence_after();
-            const int64_t row = int64_t(t.mb) * BM + 32 * q + lane;
+            const int64_t row = int64_t(t.mb) * BM + int(rank) * 128 + 32 * q + lane;
 #pragma unroll 1
             for (int cc = 0; cc < BN / 32; ++cc) {
                 uint32_t r[32];
@@ -256,18 +267,23 @@ __global__ void __launch_bounds__(THREADS, 1)
                     store_row32(r, c, ws, row, col0, N, M, t.split, k_splits, out_f32);
             }
             tc_fence_before();
-            mbar_arrive(&tempty[acc]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
     }
 
+    tc_fence_before();
     __syncthreads();
+    cluster_sync();  // no CTA leaves while its peer may still touch its memory
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        tmem_dealloc_pair(tmem, TMEM_COLS);
     }
 }
+
+}  // namespace pair
 
 // Variant-off only: C = sum over splits of the fp32 partials, in split order.
 __global__ void splitk_reduce_kernel(const float *__restrict__ ws, void *__restrict__ c,
@@ -295,7 +311,7 @@ __global__ void splitk_reduce_kernel(const float *__restrict__ ws, void *__restr
 
 }  // namespace
 
-size_t gemm_smem_bytes() { return SMEM_BYTES; }
+size_t gemm_smem_bytes() { return pair::SMEM_BYTES; }
 
 int gemm_k_splits(int64_t M, int64_t N, int64_t K, int num_sms)
 {
@@ -304,10 +320,11 @@ int gemm_k_splits(int64_t M, int64_t N, int64_t K, int num_sms)
     return 1;
 #else
     // Variant-off: split K when the tiles cannot fill the GPU.
-    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-    const int64_t kblocks = (K + BK - 1) / BK;
-    if (tiles >= num_sms || kblocks < 8) return 1;
-    int64_t ks = num_sms / tiles;
+    const int64_t tiles = ((M + pair::BM - 1) / pair::BM) * ((N + pair::BN - 1) / pair::BN);
+    const int64_t kblocks = (K + pair::BK - 1) / pair::BK;
+    const int64_t pairs = num_sms / 2;
+    if (tiles >= pairs || kblocks < 8) return 1;
+    int64_t ks = pairs / tiles;
     if (ks > kblocks / 4) ks = kblocks / 4;
     if (ks < 2) return 1;
     const int64_t per = (kblocks + ks - 1) / ks;
@@ -319,13 +336,37 @@ cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tw, void *c, i
                         int K, bool out_f32, float *ws, int k_splits, int num_sms,
                         unsigned *status, uint64_t timeout_ns, cudaStream_t s)
 {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(pair::gemm_pair_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         pair::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    const int64_t units = int64_t((M + BM - 1) / BM) * ((N + BN - 1) / BN) * k_splits;
-    const int grid = static_cast<int>(units < num_sms ? units : num_sms);
-    gemm_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(ta, tw, c, ws, M, N, K, out_f32 ? 1 : 0,
-                                                  k_splits, status, timeout_ns);
+    // as many pairs as can be resident at once (not every SM can pair up)
+    static int max_pairs[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (max_pairs[dev] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+        cfg.blockDim = dim3(pair::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = pair::SMEM_BYTES;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        e = cudaOccupancyMaxActiveClusters(&clusters, pair::gemm_pair_kernel, &cfg);
+        if (e != cudaSuccess) return e;
+        max_pairs[dev] = clusters > 0 ? clusters : 1;
+    }
+    const int64_t units = int64_t((M + pair::BM - 1) / pair::BM) * ((N + pair::BN - 1) / pair::BN) *
+                          k_splits;
+    const int pairs = static_cast<int>(units < max_pairs[dev] ? units : max_pairs[dev]);
+    pair::gemm_pair_kernel<<<2 * pairs, pair::THREADS, pair::SMEM_BYTES, s>>>(
+        ta, tw, c, ws, M, N, K, out_f32 ? 1 : 0, k_splits, status, timeout_ns);
     e = cudaGetLastError();
     if (e != cudaSuccess || k_splits <= 1) return e;
     const int64_t MN = int64_t(M) * N;
