@@ -55,6 +55,11 @@ class Oracle:
         lib.oracle_matmul.argtypes = [P, P, i64, i64, i64, P]
         lib.oracle_kv_write.argtypes = [P, P, i32, i32, P, P, P, i64]
         lib.oracle_attention.argtypes = [P, i64, i32, P, P, P, i32, P, P, i32, P, i32, f64, P, P]
+        lib.oracle_embedding.argtypes = [P, i64, i64, P, i64, P]
+        lib.oracle_rope.argtypes = [P, i64, i32, i32, P, f64, P]
+        lib.oracle_swiglu.argtypes = [P, i64, i64, P]
+        lib.oracle_add_rmsnorm.argtypes = [P, P, P, i64, i64, f64, P, P]
+        lib.oracle_argmax.argtypes = [P, i64, i64, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
@@ -121,6 +126,55 @@ class Oracle:
                                   _p(lse))
         return (o, lse) if want_lse else o
 
+    # ---------------------------------------------------------- decoder glue
+
+    def embedding(self, table, ids) -> np.ndarray:
+        """Rows of ``table`` [V, H] (bf16 bits) at ``ids`` [T] -> [T, H] bits."""
+        table = _u16(table)
+        ids = np.ascontiguousarray(ids, dtype=np.int32)
+        V, H = table.shape
+        out = np.zeros((ids.shape[0], H), dtype=np.uint16)
+        self.lib.oracle_embedding(_p(table), V, H, _p(ids), ids.shape[0], _p(out))
+        return out
+
+    def rope(self, x, pos, theta: float = 10000.0) -> np.ndarray:
+        """Rotary embedding (rotate-half pairs) of x [T, nh, d] at positions
+        ``pos`` [T] -> float64 [T, nh, d]."""
+        x = _u16(x)
+        T, nh, d = x.shape
+        pos = np.ascontiguousarray(pos, dtype=np.int32)
+        assert pos.shape == (T,) and d % 2 == 0
+        out = np.empty((T, nh, d), dtype=np.float64)
+        self.lib.oracle_rope(_p(x), T, nh, d, _p(pos), float(theta), _p(out))
+        return out
+
+    def swiglu(self, gu) -> np.ndarray:
+        """silu(gate) * up of gu [T, 2F] = [gate | up] -> float64 [T, F]."""
+        gu = _u16(gu)
+        T, F2 = gu.shape
+        assert F2 % 2 == 0
+        out = np.empty((T, F2 // 2), dtype=np.float64)
+        self.lib.oracle_swiglu(_p(gu), T, F2 // 2, _p(out))
+        return out
+
+    def add_rmsnorm(self, x, delta, w, eps: float):
+        """(s, y): s = x + delta, y = RMSNorm(s) * w, all rows; float64."""
+        x, delta, w = _u16(x), _u16(delta), _u16(w)
+        M, H = x.shape
+        assert delta.shape == (M, H) and w.shape == (H,)
+        s = np.empty((M, H), dtype=np.float64)
+        y = np.empty((M, H), dtype=np.float64)
+        self.lib.oracle_add_rmsnorm(_p(x), _p(delta), _p(w), M, H, float(eps), _p(s), _p(y))
+        return s, y
+
+    def argmax(self, logits) -> np.ndarray:
+        """Lowest index of each row's maximum; logits [T, V] float32."""
+        logits = np.ascontiguousarray(logits, dtype=np.float32)
+        T, V = logits.shape
+        out = np.empty((T,), dtype=np.int32)
+        self.lib.oracle_argmax(_p(logits), T, V, _p(out))
+        return out
+
 
 def default() -> Oracle:
     global _lib
@@ -153,6 +207,26 @@ def attention(q_rows, row_seq, row_head, row_pos, Hq: int, k_cache, v_cache, blo
               scale: float | None = None, want_lse: bool = False):
     return default().attention(q_rows, row_seq, row_head, row_pos, Hq, k_cache, v_cache,
                                block_table, scale=scale, want_lse=want_lse)
+
+
+def embedding(table, ids) -> np.ndarray:
+    return default().embedding(table, ids)
+
+
+def rope(x, pos, theta: float = 10000.0) -> np.ndarray:
+    return default().rope(x, pos, theta)
+
+
+def swiglu(gu) -> np.ndarray:
+    return default().swiglu(gu)
+
+
+def add_rmsnorm(x, delta, w, eps: float):
+    return default().add_rmsnorm(x, delta, w, eps)
+
+
+def argmax(logits) -> np.ndarray:
+    return default().argmax(logits)
 
 
 def decode_rows(q, seq_lens, heads=None):

@@ -195,3 +195,113 @@ void oracle_attention(const uint16_t *q, int64_t R, int32_t d,
         if (lse) lse[r] = mx + log(l);
     }
 }
+
+/* ------------------------------------------------------------------------
+ * The toy decoder's glue operations.  The reports on "Defeating
+ * Nondeterminism in LLM Inference" restate an experiment in which one
+ * prompt is completed greedily many times among other requests and the
+ * distinct completions are counted (xitu-tech news, "显著成果与高昂成本";
+ * liuwei.blog, "实验成果").  They name no layer of the model beyond the three
+ * kernels, so the decoder around them is read as the plain pre-norm
+ * transformer: token embedding, rotary position embedding (base theta,
+ * rotate-half pairing), SwiGLU feed-forward, residual additions, greedy
+ * argmax (lowest index on ties).  Each function is that definition in fp64.
+ * ------------------------------------------------------------------------ */
+
+/* out[t, :] = table[ids[t], :]  (bit copy; ids outside 0..V-1 leave the row
+ * untouched). */
+void oracle_embedding(const uint16_t *table, int64_t V, int64_t H, const int32_t *ids,
+                      int64_t T, uint16_t *out)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        int64_t id = ids[t];
+        if (id < 0 || id >= V) continue;
+        memcpy(out + t * H, table + id * H, (size_t)H * sizeof(uint16_t));
+    }
+}
+
+/*
+ * Rotary position embedding of x [T, nh, d] at absolute positions pos[t]:
+ * for i < d/2, with angle = pos * theta^(-2i/d), the pair (x_i, x_{i+d/2})
+ * is rotated by that angle:
+ *   out_i       = x_i cos(angle) - x_{i+d/2} sin(angle)
+ *   out_{i+d/2} = x_{i+d/2} cos(angle) + x_i sin(angle)
+ */
+void oracle_rope(const uint16_t *x, int64_t T, int32_t nh, int32_t d, const int32_t *pos,
+                 double theta, double *out)
+{
+    int32_t half = d / 2;
+    int64_t t;
+#pragma omp parallel for schedule(static)
+    for (t = 0; t < T; ++t) {
+        for (int32_t h = 0; h < nh; ++h) {
+            const uint16_t *xr = x + (t * nh + h) * (int64_t)d;
+            double *orow = out + (t * nh + h) * (int64_t)d;
+            for (int32_t i = 0; i < half; ++i) {
+                double angle = (double)pos[t] * pow(theta, -2.0 * (double)i / (double)d);
+                double c = cos(angle), s = sin(angle);
+                double a = bf16_to_double(xr[i]), b = bf16_to_double(xr[i + half]);
+                orow[i] = a * c - b * s;
+                orow[i + half] = b * c + a * s;
+            }
+        }
+    }
+}
+
+/*
+ * SwiGLU of gu [T, 2F] = [gate | up]:  out[t, j] = silu(g) * u with
+ * g = gu[t, j], u = gu[t, F + j], silu(g) = g / (1 + exp(-g)).
+ */
+void oracle_swiglu(const uint16_t *gu, int64_t T, int64_t F, double *out)
+{
+    int64_t t;
+#pragma omp parallel for schedule(static)
+    for (t = 0; t < T; ++t) {
+        for (int64_t j = 0; j < F; ++j) {
+            double g = bf16_to_double(gu[t * 2 * F + j]);
+            double u = bf16_to_double(gu[t * 2 * F + F + j]);
+            out[t * F + j] = g / (1.0 + exp(-g)) * u;
+        }
+    }
+}
+
+/*
+ * Residual addition followed by RMSNorm of the sum:
+ *   s[r, :] = x[r, :] + delta[r, :]
+ *   y[r, j] = s[r, j] / sqrt( (1/H) * sum_i s[r, i]^2 + eps ) * w[j]
+ * Both s and y are returned.
+ */
+void oracle_add_rmsnorm(const uint16_t *x, const uint16_t *delta, const uint16_t *w, int64_t M,
+                        int64_t H, double eps, double *s, double *y)
+{
+    int64_t r;
+#pragma omp parallel for schedule(static)
+    for (r = 0; r < M; ++r) {
+        double ss = 0.0;
+        for (int64_t i = 0; i < H; ++i) {
+            double v = bf16_to_double(x[r * H + i]) + bf16_to_double(delta[r * H + i]);
+            s[r * H + i] = v;
+            ss += v * v;
+        }
+        double mean_sq = ss / (double)H;
+        double rms = sqrt(mean_sq + eps);
+        for (int64_t j = 0; j < H; ++j)
+            y[r * H + j] = bf16_to_double(w[j]) * (s[r * H + j] / rms);
+    }
+}
+
+/*
+ * Greedy choice: out[t] = the lowest index j with logits[t, j] equal to the
+ * row's maximum.  The logits are taken in the precision they are given in
+ * (fp32), so the decision is the one that precision makes.
+ */
+void oracle_argmax(const float *logits, int64_t T, int64_t V, int32_t *out)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        const float *row = logits + t * V;
+        int64_t best = 0;
+        for (int64_t j = 1; j < V; ++j)
+            if (row[j] > row[best]) best = j;
+        out[t] = (int32_t)best;
+    }
+}

@@ -316,3 +316,138 @@ def test_attention_brute_force_tiny(oracle):
     want = [(2 * e[0] - 2 * e[2]) / Z, (4 * e[1] + 2 * e[2]) / Z]
     np.testing.assert_allclose(o[0], want, rtol=1e-14)
     assert abs(lse[0] - (0.5 + math.log(Z))) < 1e-14
+
+
+# ---------------------------------------------------------------- decoder glue
+# Pins for the toy decoder's elementwise operations (embedding, rotary
+# position embedding, SwiGLU, residual + RMSNorm, greedy argmax).
+
+
+def test_embedding_rows_carry_their_ids(oracle):
+    # Row v of the table holds the value v in every column: the gathered
+    # rows must decode to the requested ids, in the requested order.
+    V, H = 256, 16  # integers up to 256 are exact in bfloat16
+    table = np.repeat(bf(np.arange(V, dtype=np.float32))[:, None], H, axis=1)
+    ids = np.array([5, 0, 255, 5, 17], dtype=np.int32)
+    out = oracle.embedding(table, ids)
+    assert np.array_equal(widen(out), np.repeat(ids[:, None], H, axis=1).astype(np.float64))
+
+
+def test_embedding_matches_fancy_indexing(oracle):
+    g = rng(41)
+    table = normal_bf16(g, (1000, 64))
+    ids = g.integers(0, 1000, size=37).astype(np.int32)
+    assert np.array_equal(oracle.embedding(table, ids), table[ids])
+
+
+def test_rope_position_zero_is_identity(oracle):
+    g = rng(42)
+    x = normal_bf16(g, (3, 2, 8))
+    out = oracle.rope(x, [0, 0, 0])
+    assert np.array_equal(out, widen(x))
+
+
+def test_rope_hand_example(oracle):
+    # d = 4, theta = 10000: pair (x0, x2) turns by pos * 1, pair (x1, x3) by
+    # pos * 10000^(-1/2) = pos / 100.
+    x = bf([1.0, 2.0, 3.0, -1.0]).reshape(1, 1, 4)
+    out = oracle.rope(x, [2])[0, 0]
+    a0, a1 = 2.0, 0.02
+    want = [1.0 * math.cos(a0) - 3.0 * math.sin(a0),
+            2.0 * math.cos(a1) - (-1.0) * math.sin(a1),
+            3.0 * math.cos(a0) + 1.0 * math.sin(a0),
+            -1.0 * math.cos(a1) + 2.0 * math.sin(a1)]
+    np.testing.assert_allclose(out, want, rtol=1e-14, atol=1e-15)
+
+
+def test_rope_matches_complex_rotation(oracle):
+    # The same rotation as multiplication by e^{i angle} of z = x_i + i x_{i+d/2}.
+    g = rng(43)
+    T, nh, d, theta = 5, 3, 128, 10000.0
+    x = normal_bf16(g, (T, nh, d))
+    pos = np.array([0, 1, 63, 300, 32767], dtype=np.int32)
+    out = oracle.rope(x, pos, theta)
+    xf = widen(x)
+    z = xf[..., : d // 2] + 1j * xf[..., d // 2:]
+    inv = theta ** (-np.arange(0, d, 2, dtype=np.float64) / d)
+    rot = np.exp(1j * pos[:, None].astype(np.float64) * inv[None, :])[:, None, :]
+    zr = z * rot
+    # angles up to 32767 rad: the two routes round the angle differently by
+    # up to ~1e-11 rad
+    np.testing.assert_allclose(out[..., : d // 2], zr.real, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(out[..., d // 2:], zr.imag, rtol=1e-10, atol=1e-10)
+
+
+def test_rope_dot_products_depend_on_relative_position(oracle):
+    # <rope(q, m), rope(k, n)> depends on m - n only, and pair norms are kept.
+    g = rng(44)
+    d = 64
+    q = normal_bf16(g, (1, 1, d))
+    k = normal_bf16(g, (1, 1, d))
+    dots = []
+    for m, n in [(10, 3), (107, 100), (7, 0)]:
+        dots.append(float(np.dot(oracle.rope(q, [m])[0, 0], oracle.rope(k, [n])[0, 0])))
+    np.testing.assert_allclose(dots, [dots[0]] * 3, rtol=1e-12)
+    r = oracle.rope(q, [77])[0, 0]
+    qf = widen(q)[0, 0]
+    np.testing.assert_allclose(r[: d // 2] ** 2 + r[d // 2:] ** 2,
+                               qf[: d // 2] ** 2 + qf[d // 2:] ** 2, rtol=1e-12)
+
+
+def test_swiglu_closed_forms(oracle):
+    # Gate first, up second.  silu(0) = 0; silu(1) = 1 / (1 + 1/e)
+    # = 0.7310585786300049; silu(x) - silu(-x) = x.
+    gu = bf([[0.0, 1.0, -3.0, 3.0, 5.0, 2.0, 1.0, 1.0]])
+    out = oracle.swiglu(gu)[0]
+    assert out[0] == 0.0
+    assert abs(out[1] - 2.0 * 0.7310585786300049) < 1e-15
+    assert abs((out[3] - out[2]) - 3.0) < 1e-14
+
+
+def test_swiglu_matches_torch_fp64(oracle):
+    g = rng(45)
+    T, F = 4, 96
+    gu = normal_bf16(g, (T, 2 * F), std=3.0)
+    out = oracle.swiglu(gu)
+    gt = torch.from_numpy(widen(gu))
+    want = torch.nn.functional.silu(gt[:, :F]) * gt[:, F:]
+    np.testing.assert_allclose(out, want.numpy(), rtol=1e-13, atol=1e-15)
+
+
+def test_add_rmsnorm_constant_sum_closed_form(oracle):
+    # x + delta = c * 1  =>  y = c / sqrt(c^2 + eps) * w; s is the exact sum.
+    H, eps = 32, 1e-6
+    g = rng(46)
+    w = uniform_bf16(g, (H,), 0.5, 1.5)
+    x = np.tile(bf([0.75] * H), (2, 1))
+    delta = np.tile(bf([-2.0] * H), (2, 1))
+    s, y = oracle.add_rmsnorm(x, delta, w, eps)
+    c = -1.25
+    np.testing.assert_array_equal(s, np.full((2, H), c))
+    np.testing.assert_allclose(y[1], c / math.sqrt(c * c + eps) * widen(w), rtol=1e-14)
+
+
+def test_add_rmsnorm_matches_torch_fp64(oracle):
+    g = rng(47)
+    M, H, eps = 5, 256, 1e-6
+    x, delta = normal_bf16(g, (M, H)), normal_bf16(g, (M, H), std=0.3)
+    w = uniform_bf16(g, (H,), 0.5, 1.5)
+    s, y = oracle.add_rmsnorm(x, delta, w, eps)
+    st = torch.from_numpy(widen(x) + widen(delta))
+    want = torch.nn.functional.rms_norm(st, (H,), torch.from_numpy(widen(w)), eps)
+    np.testing.assert_allclose(s, st.numpy(), rtol=0, atol=0)
+    np.testing.assert_allclose(y, want.numpy(), rtol=1e-13)
+
+
+def test_argmax_ties_take_the_lowest_index(oracle):
+    logits = np.array([[1.0, 3.0, 3.0, 2.0],
+                       [-np.inf, -5.0, -np.inf, -5.0],
+                       [0.0, 0.0, 0.0, 0.0],
+                       [1.0, 2.0, 3.0, 4.0]], dtype=np.float32)
+    assert oracle.argmax(logits).tolist() == [1, 1, 0, 3]
+
+
+def test_argmax_matches_numpy_first_occurrence(oracle):
+    g = rng(48)
+    logits = g.integers(-3, 4, size=(50, 1000)).astype(np.float32)  # many ties
+    assert np.array_equal(oracle.argmax(logits), np.argmax(logits, axis=1))

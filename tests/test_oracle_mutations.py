@@ -22,7 +22,7 @@ MUTATIONS = [
      [pins.test_rmsnorm_eps_inside_the_root]),
     ("rmsnorm_wrong_weight_index", "* bf16_to_double(w[j])", "* bf16_to_double(w[H - 1 - j])",
      [pins.test_rmsnorm_matches_torch_fp64, pins.test_rmsnorm_hand_example]),
-    ("rmsnorm_mean_over_h_minus_1", "ss / (double)H", "ss / (double)(H - 1)",
+    ("rmsnorm_mean_over_h_minus_1", "sqrt(ss / (double)H + eps)", "sqrt(ss / (double)(H - 1) + eps)",
      [pins.test_rmsnorm_hand_example, pins.test_rmsnorm_matches_torch_fp64]),
     ("matmul_transposed_weight", "s += bf16_to_double(am[k]) * bf16_to_double(wn[k]);",
      "s += bf16_to_double(am[k]) * bf16_to_double(w[k * N + n]);",
@@ -44,6 +44,31 @@ MUTATIONS = [
      [pins.test_attention_paging_is_transparent, pins.test_attention_matches_torch_sdpa_fp64]),
     ("attention_values_not_normalised", "orow[i] /= l;", "orow[i] /= 1.0;",
      [pins.test_attention_identical_keys_give_prefix_mean]),
+    ("embedding_off_by_one_row", "memcpy(out + t * H, table + id * H,",
+     "memcpy(out + t * H, table + ((id + 1) % V) * H,",
+     [pins.test_embedding_rows_carry_their_ids, pins.test_embedding_matches_fancy_indexing]),
+    ("rope_sin_sign_flipped", "orow[i] = a * c - b * s;", "orow[i] = a * c + b * s;",
+     [pins.test_rope_hand_example, pins.test_rope_matches_complex_rotation]),
+    ("rope_interleaved_pairs", "b = bf16_to_double(xr[i + half]);",
+     "b = bf16_to_double(xr[i ^ 1]);",
+     [pins.test_rope_hand_example, pins.test_rope_matches_complex_rotation]),
+    ("rope_frequency_exponent_i_over_d", "pow(theta, -2.0 * (double)i / (double)d)",
+     "pow(theta, -1.0 * (double)i / (double)d)",
+     [pins.test_rope_hand_example, pins.test_rope_matches_complex_rotation]),
+    ("swiglu_gate_and_up_swapped", "double g = bf16_to_double(gu[t * 2 * F + j]);",
+     "double g = bf16_to_double(gu[t * 2 * F + F + j]);",
+     [pins.test_swiglu_closed_forms, pins.test_swiglu_matches_torch_fp64]),
+    ("swiglu_sigmoid_not_silu", "out[t * F + j] = g / (1.0 + exp(-g)) * u;",
+     "out[t * F + j] = 1.0 / (1.0 + exp(-g)) * u;",
+     [pins.test_swiglu_closed_forms, pins.test_swiglu_matches_torch_fp64]),
+    ("add_rmsnorm_norm_ignores_delta", "            ss += v * v;\n        }\n        double mean_sq",
+     "            ss += bf16_to_double(x[r * H + i]) * bf16_to_double(x[r * H + i]);\n        }\n        double mean_sq",
+     [pins.test_add_rmsnorm_constant_sum_closed_form, pins.test_add_rmsnorm_matches_torch_fp64]),
+    ("add_rmsnorm_eps_outside_root", "sqrt(mean_sq + eps)", "(sqrt(mean_sq) + eps)",
+     [pins.test_add_rmsnorm_constant_sum_closed_form, pins.test_add_rmsnorm_matches_torch_fp64]),
+    ("argmax_ties_take_highest_index", "if (row[j] > row[best]) best = j;",
+     "if (row[j] >= row[best]) best = j;",
+     [pins.test_argmax_ties_take_the_lowest_index, pins.test_argmax_matches_numpy_first_occurrence]),
 ]
 
 
