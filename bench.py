@@ -32,9 +32,7 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -159,52 +157,91 @@ class Workload:
 
 # ---------------------------------------------------------------- clocks
 
-class Clocks:
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+def pci_bus_id(props) -> bytes | None:
+    """NVML's bus-id string ("DDDDDDDD:BB:DD.0") for a torch device, built
+    from the integer PCI domain, bus and device numbers torch reports."""
+    try:
+        dom, bus, dv = (int(getattr(props, k)) for k in ("pci_domain_id", "pci_bus_id",
+                                                          "pci_device_id"))
+    except (AttributeError, TypeError, ValueError):
+        return None
+    return ("%08X:%02X:%02X.0" % (dom, bus, dv)).encode()
 
-    def __init__(self, index: int):
-        self.index = index
-        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+class Clocks:
+    """SM clock and clock-event reasons of this process's GPU, read through
+    NVML by a background thread every few milliseconds.  ``mark()`` brackets
+    the timed region; ``stop()`` summarises the samples taken inside it (or
+    the nearest ones when the region is shorter than the sampling period).
+    Read-only: no clock or other GPU setting is changed."""
+
+    NAMES = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+             ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+             ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+             ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, bus_id: bytes | None, index: int, period_s: float = 0.005):
+        import threading
+
+        self.samples, self.window, self.err = [], [None, None], None
         try:
-            self.p = subprocess.Popen(["nvidia-smi", "-i", str(index), "--query-gpu=" + self.Q,
-                                       "--format=csv,noheader,nounits", "-lms", "200"],
-                                      stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.p = None
+            import pynvml as nv
+
+            nv.nvmlInit()
+            self.h = None
+            if isinstance(bus_id, bytes):  # never an int: NVML takes it as a char*
+                try:
+                    self.h = nv.nvmlDeviceGetHandleByPciBusId(bus_id)
+                except Exception:
+                    self.h = None
+            if self.h is None:
+                self.h = nv.nvmlDeviceGetHandleByIndex(index)
+            self.nv = nv
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report it, do not guess
+            self.nv, self.err = None, "nvml unavailable: %s" % e
+            return
+        self.stop_flag = threading.Event()
+        self.period = period_s
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), sm, rs))
+            except Exception as e:
+                self.err = str(e)
+            self.stop_flag.wait(self.period)
+
+    def mark(self, which: int):
+        self.window[which] = time.perf_counter()
 
     def stop(self):
-        if self.p is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.p.terminate()
-        try:
-            self.p.wait(timeout=5)
-        except Exception:
-            self.p.kill()
-        self.f.flush()
-        rows = []
-        with open(self.f.name) as fh:
-            for line in fh:
-                parts = [s.strip() for s in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.f.name)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
-        load = [s for s in sm if s > 0.5 * (max(mx) if mx else 1)] or sm
-        return {"sm_mhz": statistics.median(load) if load else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err]}
+        self.stop_flag.set()
+        self.t.join(timeout=2)
+        t0, t1 = self.window
+        inside = [s for s in self.samples if t0 is not None and t1 is not None and t0 <= s[0] <= t1]
+        if not inside and self.samples and t0 is not None:
+            mid = 0.5 * (t0 + (t1 or t0))
+            inside = sorted(self.samples, key=lambda s: abs(s[0] - mid))[:2]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"]}
+        reasons = sorted({n for _, _, rs in inside for n, attr in self.NAMES
+                          if rs & getattr(self.nv, attr, 0)})
+        return {"sm_mhz": statistics.median([s[1] for s in inside]), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside), "source": "nvml, 5 ms period",
+                "window_ms": (t1 - t0) * 1e3 if t1 and t0 else None}
 
 
 # ---------------------------------------------------------------- ours
 
-def timed_steps(torch, L, wl, steps, warmup, dist=None):
+def timed_steps(torch, L, wl, steps, warmup, dist=None, clocks=None):
     for _ in range(warmup):
         wl.flush.zero_()
         wl.step(L)
@@ -215,10 +252,14 @@ def timed_steps(torch, L, wl, steps, warmup, dist=None):
         dist.barrier()
     torch.cuda.synchronize()
     t0 = time.perf_counter()
+    if clocks is not None:
+        clocks.mark(0)
     for i in range(steps):
         wl.flush.zero_()
         wl.step(L, evs[i])
     torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.mark(1)
     wall = time.perf_counter() - t0
     if dist is not None:
         dist.barrier()
@@ -310,6 +351,37 @@ def invariance_checks(torch, L, wl) -> dict:
     return out
 
 
+def rmsnorm_context(torch, L, wl) -> dict:
+    """What bounds RMSNorm at the step's size: a plain device copy of the same
+    bytes timed the same way, and RMSNorm on 65536 rows (1 GiB moved)."""
+    T = torch
+
+    def timed(fn, reps=20):
+        for _ in range(3):
+            wl.flush.zero_()
+            fn()
+        ev = [(T.cuda.Event(enable_timing=True), T.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in ev:
+            wl.flush.zero_()
+            a.record()
+            fn()
+            b.record()
+        T.cuda.synchronize()
+        return float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+    y = T.empty_like(wl.x)
+    copy_ms = timed(lambda: y.copy_(wl.x))
+    big = T.empty((65536, H), dtype=T.bfloat16, device=wl.x.device)
+    big.copy_(wl.x.repeat(32, 1))
+    big_out = T.empty_like(big)
+    big_ms = timed(lambda: L.bi_rmsnorm(big, wl.w, wl.eps, out=big_out), reps=10)
+    nbytes = 2.0 * 2 * M_ROWS * H
+    big_bytes = 2.0 * 2 * 65536 * H
+    del big, big_out
+    return {"copy_same_bytes_ms": copy_ms, "copy_same_bytes_GB/s": nbytes / (copy_ms * 1e-3) / 1e9,
+            "rmsnorm_M65536_ms": big_ms, "rmsnorm_M65536_GB/s": big_bytes / (big_ms * 1e-3) / 1e9}
+
+
 def cpu_baseline(wl, budget_s: float = 20.0) -> dict:
     """The oracle (fp64, OpenMP) on a bounded sample of the same workload."""
     import oracle
@@ -393,8 +465,8 @@ def run_ours(args):
     wl = Workload(torch, bi, dev, seed_base=0)
     launches = wl.launches_per_step(L)
 
-    clocks = Clocks(local)
-    per, wall = timed_steps(torch, L, wl, args.steps, args.warmup, dist)
+    clocks = Clocks(pci_bus_id(torch.cuda.get_device_properties(dev)), local)
+    per, wall = timed_steps(torch, L, wl, args.steps, args.warmup, dist, clocks)
     clk = clocks.stop()
     mean = per.mean(axis=0)  # ms per kernel group
     step_ms = float(per.sum(axis=1).mean())
@@ -433,6 +505,7 @@ def run_ours(args):
     overhead["step"] = float(per.sum(axis=1).mean() / per_v.sum(axis=1).mean() - 1.0)
 
     checks = invariance_checks(torch, L, wl)
+    rms_ctx = rmsnorm_context(torch, L, wl)
 
     if rank != 0:
         if dist is not None:
@@ -445,7 +518,9 @@ def run_ours(args):
     kernels = {
         "bi_kv_write": {"ms": float(mean[0]), "GB/s": wl.kvw_bytes / (mean[0] * 1e-3) / 1e9},
         "bi_rmsnorm": {"ms": float(mean[1]), "GB/s": wl.norm_bytes / (mean[1] * 1e-3) / 1e9,
-                       "frac_hbm": wl.norm_bytes / (mean[1] * 1e-3) / 1e9 / pk["hbm_gbs"]},
+                       "frac_hbm": wl.norm_bytes / (mean[1] * 1e-3) / 1e9 / pk["hbm_gbs"],
+                       "context": rms_ctx,
+                       "frac_hbm_M65536": rms_ctx["rmsnorm_M65536_GB/s"] / pk["hbm_gbs"]},
         "bi_matmul": {"ms": float(mean[2]), "TFLOP/s": wl.gemm_flops / (mean[2] * 1e-3) / 1e12,
                       "frac_bf16": wl.gemm_flops / (mean[2] * 1e-3) / 1e12 / pk["bf16_tflops"]},
         "bi_attention_decode": {"ms": float(mean[3]), "GB/s": wl.dec_bytes / (mean[3] * 1e-3) / 1e9,
@@ -635,6 +710,9 @@ def run_profile_case(args):
 
 
 def main(argv=None):
+    import faulthandler
+
+    faulthandler.enable()  # a host-side crash prints every thread's stack
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)

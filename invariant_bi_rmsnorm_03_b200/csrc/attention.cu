@@ -15,8 +15,7 @@
 //   S      = Q K_s^T                    tcgen05, M=128 rows, N=256 keys, fp32
 //   x_j    = S_j * scale * log2(e), masked to -inf where key j > t
 //   m_s    = max_j x_j
-//   p_j    = 2^(x_j - m_s),  l_s = sum_j p_j   (fixed order: 32-key chunks
-//            summed by a pairwise tree, chunk sums added left to right)
+//   p_j    = 2^(x_j - m_s),  l_s = sum_j p_j   (a fixed order, tree8 below)
 //   O_s    = bf16(p) V_s                tcgen05, P read from tensor memory
 // and the partials are merged from split 0 upwards, always in that order:
 //   m' = max(m, m_s), a = 2^(m - m'), c = 2^(m_s - m')
@@ -34,17 +33,24 @@
 // split, with the same merge function.  The bits therefore do not depend on
 // how many blocks served a sequence.
 //
-// Block of 192 threads, one per SM (224 KB shared memory, 512 TMEM columns):
+// Block of 320 threads, one per SM (about 225 KB shared memory; 512 TMEM
+// columns as two 256-column buffers, each holding a split's logits, then
+// its P in columns 0-127 and O_s in columns 128-255):
 //   warp 0     producer: Q by TMA once; per split the 16 pages of K and of
 //              V, one bulk copy per page block (gathered through the page
 //              table; the cache keeps each page block in the tensor core's
 //              core-matrix order, so it is used in place), into a 3-slot
-//              ring; the V rows past the sequence end are zero (copies of a
-//              zero page, explicit stores for the partial page) so that
-//              0 * stale never reaches O.
-//   warp 1     TMEM allocation and MMA issue (one thread)
-//   warps 2-5  softmax and merge; warp w owns TMEM lanes 32(w%4)..+31.
-//              Decode spreads the query heads over the four lane quarters.
+//              ring, in the order K0 K1 V0 K2 V1 ...; V rows past the
+//              sequence end are zero (copies of a zero page, explicit stores
+//              for the partial page) so that 0 * stale never reaches O.
+//   warp 1     TMEM allocation and MMA issue (one thread): QK^T of split
+//              s+1 runs while split s is in softmax (double-buffered TMEM).
+//   warps 4-7  softmax of one split; warp w owns TMEM lanes 32(w%4)..+31.
+//              Decode spreads the query heads over the four lane quarters,
+//              and with at most 8 heads per quarter four threads share a
+//              row (softmax_heads16).
+//   warps 2,3,8,9  merge ("fold") of O_s into the running output, one per
+//              lane quarter, overlapping the next split's softmax.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
