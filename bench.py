@@ -506,6 +506,12 @@ def run_ours(args):
 
     checks = invariance_checks(torch, L, wl)
     rms_ctx = rmsnorm_context(torch, L, wl)
+    uc = None
+    if rank == 0 and args.uc_targets > 0:
+        # the end-to-end check on the toy decoder, at a reduced count
+        uc = unique_completions(args.uc_targets, args.uc_targets, span=2 * args.uc_targets)
+        checks["unique_completions"] = uc["invariant"]["unique_completions"]
+        checks["all"] = bool(checks["all"] and checks["unique_completions"] == 1)
 
     if rank != 0:
         if dist is not None:
@@ -574,6 +580,7 @@ def run_ours(args):
         "roofline": roof,
         "kernels": kernels,
         "overhead_vs_variant_off": overhead,
+        "unique_completions": uc,
         "e2e": {"value": world * wl.gemm_flops / (e2e_gemm_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "split_kv_attn_gbs": world * wl.dec_bytes / (e2e_dec_ms * 1e-3) / 1e9},
@@ -709,6 +716,82 @@ def run_profile_case(args):
     print(json.dumps({"profile": args.profile, "ms": ms, "status": int(L.bi_device_status())}))
 
 
+def run_unique_completions(args):
+    print(json.dumps(unique_completions(args.targets, args.others, args.max_batch,
+                                        args.token_budget, args.span)), flush=True)
+
+
+def unique_completions(targets, others, max_batch=256, token_budget=2048, span=2000) -> dict:
+    """One fixed 64-token prompt completed greedily (256 tokens) many times
+    amid random other requests, on the 8-layer hidden-4096 random-init
+    decoder: the number of distinct completions for the invariant and the
+    variant-off build, and where the completions first differ from the
+    prompt's completion when it runs alone."""
+    import torch
+
+    import invariant_bi_rmsnorm_03_b200 as bi
+    from invariant_bi_rmsnorm_03_b200.decoder import (DecoderConfig, PagePool, Request, Scheduler,
+                                                      ToyDecoder, run, weight_shapes)
+    from synth import toy_decoder_weights, unique_completion_workload
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = DecoderConfig()
+    weights = toy_decoder_weights(weight_shapes(cfg), seed=4, device=dev)
+    prompt, spec = unique_completion_workload(seed=4, n_target=targets, n_other=others,
+                                              vocab=cfg.vocab, steps_span=span)
+    pages_per_req = (512 + 256 + 15) // 16
+    num_pages = max_batch * pages_per_req + 64
+    result = {"experiment": "unique completions", "model": "8-layer decoder, hidden 4096, GQA 32/8, "
+              "d 128, SwiGLU 14336, vocab 32000, W~N(0,0.02) seed 4",
+              "prompt_tokens": 64, "new_tokens": 256, "targets": targets,
+              "others": others, "max_batch": max_batch,
+              "token_budget": token_budget, "data": "synthetic"}
+    for variant in (False, True):
+        L = bi.load(variant=variant)
+        model = ToyDecoder(L, cfg, weights, num_pages, dev)
+        solo = Request(-1, prompt, 256)
+        s1 = Scheduler(PagePool(num_pages, seed=1), max_batch=1, token_budget=token_budget)
+        s1.add([solo])
+        run(s1, model)
+        reqs = [Request(d["rid"], d["prompt"], d["max_new"], d["arrival"], d["tag"]) for d in spec]
+        sched = Scheduler(PagePool(num_pages, seed=2), max_batch=max_batch,
+                          token_budget=token_budget)
+        sched.add(reqs)
+        sizes = []
+        orig_plan = sched.plan
+
+        def plan_and_count():
+            p = orig_plan()
+            if p is not None:
+                sizes.append(len(p.dec) + len(p.pre))
+            return p
+
+        sched.plan = plan_and_count
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        steps = run(sched, model)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+        outs = [tuple(r.out) for r in reqs if r.tag == "target"]
+        ref = tuple(solo.out)
+        first_div = [next((i for i, (a, b) in enumerate(zip(o, ref)) if a != b), None) for o in outs]
+        div = [f for f in first_div if f is not None]
+        tokens = sum(len(r.prompt) + r.max_new for r in reqs)
+        result["variant_off" if variant else "invariant"] = {
+            "unique_completions": len(set(outs)),
+            "equal_to_solo_run": sum(o == ref for o in outs),
+            "first_divergent_token": {"min": min(div), "median": float(np.median(div))} if div else None,
+            "steps": steps, "batch_rows_min": int(min(sizes)), "batch_rows_max": int(max(sizes)),
+            "wall_s": wall, "tokens_per_s": tokens / wall,
+            "device_status": int(L.bi_device_status())}
+        del model
+        torch.cuda.empty_cache()
+    del weights
+    torch.cuda.empty_cache()
+    return result
+
+
 def main(argv=None):
     import faulthandler
 
@@ -725,11 +808,23 @@ def main(argv=None):
     ap.add_argument("--profile-batch", type=int, default=32)
     ap.add_argument("--profile-seq", type=int, default=4096)
     ap.add_argument("--variant", action="store_true", help="--profile the variant-off build")
+    ap.add_argument("--unique-completions", action="store_true",
+                    help="run the toy-decoder unique-completion experiment instead")
+    ap.add_argument("--targets", type=int, default=1000)
+    ap.add_argument("--others", type=int, default=1000)
+    ap.add_argument("--max-batch", type=int, default=256)
+    ap.add_argument("--token-budget", type=int, default=2048)
+    ap.add_argument("--span", type=int, default=2000, help="arrival steps are spread over this")
+    ap.add_argument("--uc-targets", type=int, default=200,
+                    help="target copies (and as many others) of the in-bench unique-completion "
+                         "check; 0 skips it")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.profile:
         run_profile_case(args)
+    elif args.unique_completions:
+        run_unique_completions(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

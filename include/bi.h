@@ -106,6 +106,21 @@ bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H
                      bi_dtype out_dtype, void *stream);
 
 /*
+ * bi_add_rmsnorm -- the residual form of bi_rmsnorm used between the
+ * sublayers of a pre-norm decoder: the residual stream x takes the
+ * sublayer's output, then is normalised.
+ *
+ *   x[r, j] <- round( x[r, j] + delta[r, j] )          (fp32 add, bf16 RNE)
+ *   y[r, :]  = bi_rmsnorm(x[r, :]) of the updated row, bit for bit
+ *
+ *   x : device, bf16 [M, H], read and written;  delta : device, bf16 [M, H];
+ *   w, y, eps, out_dtype, requirements: as bi_rmsnorm; y overlaps neither x
+ *   nor delta.  Same one-block-per-row order, fixed by H alone.
+ */
+bi_status bi_add_rmsnorm(void *x, const void *delta, const void *w, void *y, int64_t M,
+                         int64_t H, float eps, bi_dtype out_dtype, void *stream);
+
+/*
  * bi_matmul -- batch-invariant matrix product (xitu-tech news,
  * "构建确定性解决方案", matmul item: no split-K chosen from the input size, one
  * fixed kernel configuration with one tile size; neican.ai insight,
@@ -248,6 +263,67 @@ size_t bi_attention_prefill_workspace_bytes(const bi_paged_kv *kv, int32_t B, in
                                             int32_t max_q_len);
 
 /* Human-readable name of a status code (static string). */
+/*
+ * Decoder glue.  The reports measure invariance end to end by completing one
+ * prompt greedily many times among other requests and counting the distinct
+ * completions (xitu-tech news, "显著成果与高昂成本"; liuwei.blog, "实验成果").
+ * They name no layer beyond RMSNorm, matmul and attention; the decoder around
+ * them is read as the plain pre-norm transformer.  Each operation below
+ * computes an output row from its own input row only.
+ */
+
+/*
+ * bi_embedding -- out[t, :] = table[ids[t], :]  (bit copy; also a row gather
+ * of any [V, H] bf16 matrix).
+ *   table : device, bf16 [V, H];  ids : device, int32 [T];
+ *   out : device, bf16 [T, H].  H % 8 == 0, table and out 16-byte aligned.
+ *   An id outside 0..V-1 leaves its row unwritten and flags
+ *   BI_ERR_DEVICE_INDEX.  T == 0 is a no-op.
+ */
+bi_status bi_embedding(const void *table, int64_t V, int64_t H, const int32_t *ids, void *out,
+                       int64_t T, void *stream);
+
+/*
+ * bi_rope_kv_write -- rotary position embedding of the new tokens' queries
+ * and keys, fused with the write of their keys and values into the paged
+ * cache (the cache is updated before attention runs, as bi_kv_write does).
+ *
+ *   qkv : device, bf16 [T, (Hq + 2 Hkv) * d], each row [q heads | k heads |
+ *         v heads] (the output of one matmul with the stacked q, k, v
+ *         weights);  positions : device, int32 [T], absolute positions;
+ *   slot_mapping : device, int64 [T], as bi_kv_write (slot < 0 skips the
+ *         token's K/V; a slot past the pool flags BI_ERR_DEVICE_INDEX);
+ *   q_out : device, bf16 [T, Hq, d], the rotated queries.
+ *   For i < d/2, angle = pos * theta^(-2i/d) (evaluated in double, its
+ *   cosine and sine rounded to float); the pair (x_i, x_{i + d/2}) becomes
+ *     (x_i cos - x_{i+d/2} sin,  x_{i+d/2} cos + x_i sin)
+ *   in fp32 with every product and sum rounded, then bf16 RNE.  V is copied
+ *   unchanged.  Requirements: Hq % Hkv == 0, d in {64, 128}, theta > 1,
+ *   qkv and q_out 16-byte aligned.
+ */
+bi_status bi_rope_kv_write(const bi_paged_kv *kv, const void *qkv, const int32_t *positions,
+                           const int64_t *slot_mapping, void *q_out, int64_t T, int32_t Hq,
+                           float theta, void *stream);
+
+/*
+ * bi_swiglu -- out[t, j] = round( silu(g) * u ),  g = gu[t, j],
+ * u = gu[t, F + j], silu(g) = g / (1 + e^-g), fp32.
+ *   gu : device, bf16 [T, 2F] (gate columns first, then up: the output of
+ *   one matmul with the stacked gate and up weights);  out : device, bf16
+ *   [T, F].  F % 8 == 0, both 16-byte aligned.
+ */
+bi_status bi_swiglu(const void *gu, void *out, int64_t T, int64_t F, void *stream);
+
+/*
+ * bi_argmax -- greedy choice: out[t] = the lowest index j of the maximum of
+ * logits[t, :].  An exact selection (no rounding), so it does not depend on
+ * the order of the search.  NaN entries are never chosen; a row of NaN only
+ * gives 0.
+ *   logits : device, fp32 [T, V], 16-byte aligned, V % 4 == 0;
+ *   out : device, int32 [T].
+ */
+bi_status bi_argmax(const float *logits, int64_t T, int64_t V, int32_t *out, void *stream);
+
 const char *bi_status_string(bi_status s);
 
 /* 1 for the batch-invariant build, 0 for the variant-off build (split-K

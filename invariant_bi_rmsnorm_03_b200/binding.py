@@ -108,7 +108,8 @@ class Library:
                "bi_attention_decode", "bi_attention_decode_workspace_bytes",
                "bi_attention_prefill", "bi_attention_prefill_workspace_bytes",
                "bi_status_string", "bi_build_invariant", "bi_device_status",
-               "bi_debug_bounded_wait")
+               "bi_debug_bounded_wait", "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write",
+               "bi_swiglu", "bi_argmax")
 
     def __init__(self, path: str):
         if not os.path.exists(path):
@@ -137,8 +138,15 @@ class Library:
         L.bi_debug_bounded_wait.argtypes = [ctypes.c_uint64, P]
         L.bi_attention_decode_noalloc.argtypes = [kvp, P, P, P, P, i32, i32, i32, f32, i32, P]
         L.bi_attention_decode_noalloc.restype = st
+        L.bi_add_rmsnorm.argtypes = [P, P, P, P, i64, i64, f32, st, P]
+        L.bi_embedding.argtypes = [P, i64, i64, P, P, i64, P]
+        L.bi_rope_kv_write.argtypes = [kvp, P, P, P, P, i64, i32, f32, P]
+        L.bi_swiglu.argtypes = [P, P, i64, i64, P]
+        L.bi_argmax.argtypes = [P, i64, i64, P, P]
         for name in ("bi_rmsnorm", "bi_matmul", "bi_kv_write", "bi_attention_decode",
-                     "bi_attention_prefill", "bi_device_status", "bi_debug_bounded_wait"):
+                     "bi_attention_prefill", "bi_device_status", "bi_debug_bounded_wait",
+                     "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write", "bi_swiglu",
+                     "bi_argmax"):
             getattr(L, name).restype = st
         self.lib = L
 
@@ -171,6 +179,22 @@ class Library:
         _need(out, "out", out_dtype, (M, H))
         self._check("bi_rmsnorm", self.lib.bi_rmsnorm(_ptr(x), _ptr(w), _ptr(out), M, H,
                                                       float(eps), _DT[out_dtype], _stream(stream)))
+        return out
+
+    def bi_add_rmsnorm(self, x: torch.Tensor, delta: torch.Tensor, w: torch.Tensor,
+                       eps: float = 1e-6, out=None, out_dtype=torch.bfloat16,
+                       stream=None) -> torch.Tensor:
+        """x <- round(x + delta) in place; returns RMSNorm(x) * w."""
+        _need(x, "x", torch.bfloat16)
+        M, H = x.shape
+        _need(delta, "delta", torch.bfloat16, (M, H))
+        _need(w, "w", torch.bfloat16, (H,))
+        if out is None:
+            out = torch.empty((M, H), dtype=out_dtype, device=x.device)
+        _need(out, "out", out_dtype, (M, H))
+        self._check("bi_add_rmsnorm", self.lib.bi_add_rmsnorm(
+            _ptr(x), _ptr(delta), _ptr(w), _ptr(out), M, H, float(eps), _DT[out_dtype],
+            _stream(stream)))
         return out
 
     # ------------------------------------------------------------ matmul
@@ -209,6 +233,63 @@ class Library:
         c = kv.c_struct()
         self._check("bi_kv_write", self.lib.bi_kv_write(ctypes.byref(c), _ptr(k_new), _ptr(v_new),
                                                         _ptr(slot_mapping), T, _stream(stream)))
+
+    # ------------------------------------------------------------ decoder glue
+    def bi_embedding(self, table: torch.Tensor, ids: torch.Tensor, out=None,
+                     stream=None) -> torch.Tensor:
+        """Rows ``table[ids]`` ([V, H] bf16, int32 ids [T]) -> [T, H]."""
+        _need(table, "table", torch.bfloat16)
+        V, H = table.shape
+        _need(ids, "ids", torch.int32)
+        T = ids.shape[0]
+        if out is None:
+            out = torch.empty((T, H), dtype=torch.bfloat16, device=table.device)
+        _need(out, "out", torch.bfloat16, (T, H))
+        self._check("bi_embedding", self.lib.bi_embedding(_ptr(table), V, H, _ptr(ids), _ptr(out),
+                                                          T, _stream(stream)))
+        return out
+
+    def bi_rope_kv_write(self, kv: PagedKV, qkv: torch.Tensor, positions: torch.Tensor,
+                         slot_mapping: torch.Tensor, Hq: int, theta: float = 10000.0,
+                         q_out=None, stream=None) -> torch.Tensor:
+        """Rotate q and k of ``qkv`` [T, (Hq + 2 Hkv) d]; k and v go to the
+        cache at ``slot_mapping``; returns the rotated q [T, Hq, d]."""
+        _need(qkv, "qkv", torch.bfloat16)
+        T = qkv.shape[0]
+        d, Hkv = kv.head_dim, kv.num_kv_heads
+        _need(qkv, "qkv", torch.bfloat16, (T, (Hq + 2 * Hkv) * d))
+        _need(positions, "positions", torch.int32, (T,))
+        _need(slot_mapping, "slot_mapping", torch.int64, (T,))
+        if q_out is None:
+            q_out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=qkv.device)
+        _need(q_out, "q_out", torch.bfloat16, (T, Hq, d))
+        c = kv.c_struct()
+        self._check("bi_rope_kv_write", self.lib.bi_rope_kv_write(
+            ctypes.byref(c), _ptr(qkv), _ptr(positions), _ptr(slot_mapping), _ptr(q_out), T, Hq,
+            float(theta), _stream(stream)))
+        return q_out
+
+    def bi_swiglu(self, gu: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+        """silu(gate) * up of gu [T, 2F] = [gate | up] -> [T, F]."""
+        _need(gu, "gu", torch.bfloat16)
+        T, F2 = gu.shape
+        if out is None:
+            out = torch.empty((T, F2 // 2), dtype=torch.bfloat16, device=gu.device)
+        _need(out, "out", torch.bfloat16, (T, F2 // 2))
+        self._check("bi_swiglu", self.lib.bi_swiglu(_ptr(gu), _ptr(out), T, F2 // 2,
+                                                    _stream(stream)))
+        return out
+
+    def bi_argmax(self, logits: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+        """Lowest index of each row's maximum; logits [T, V] fp32 -> int32 [T]."""
+        _need(logits, "logits", torch.float32)
+        T, V = logits.shape
+        if out is None:
+            out = torch.empty((T,), dtype=torch.int32, device=logits.device)
+        _need(out, "out", torch.int32, (T,))
+        self._check("bi_argmax", self.lib.bi_argmax(_ptr(logits), T, V, _ptr(out),
+                                                    _stream(stream)))
+        return out
 
     # ------------------------------------------------------------ attention
     def bi_attention_decode_workspace_bytes(self, kv: PagedKV, B: int, Hq: int, max_seq_len: int,

@@ -140,6 +140,23 @@ bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H
                                         static_cast<cudaStream_t>(stream)));
 }
 
+bi_status bi_add_rmsnorm(void *x, const void *delta, const void *w, void *y, int64_t M,
+                         int64_t H, float eps, bi_dtype out_dtype, void *stream)
+{
+    if (M < 0 || H < 8 || H % 8 != 0 || H > 65536) return BI_ERR_INVALID;
+    if (out_dtype != BI_BF16 && out_dtype != BI_F32) return BI_ERR_INVALID;
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return BI_ERR_INVALID;
+    if (M == 0) return BI_OK;
+    if (!x || !delta || !w || !y) return BI_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(delta) || !aligned16(w) || !aligned16(y)) return BI_ERR_INVALID;
+    if (x == y || delta == y) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_add_rmsnorm(x, delta, w, y, M, H, eps, out_dtype == BI_F32,
+                                            d->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
 size_t bi_matmul_workspace_bytes(int64_t M, int64_t N, int64_t K)
 {
     if (M <= 0 || N <= 0 || K <= 0) return 0;
@@ -190,6 +207,60 @@ bi_status bi_kv_write(const bi_paged_kv *kv, const void *k_new, const void *v_ne
     return from_cuda(bi::launch_kv_write(kv->k_cache, kv->v_cache, kv->num_pages, kv->num_kv_heads,
                                          kv->head_dim, k_new, v_new, slot_mapping, T, d->status,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+bi_status bi_embedding(const void *table, int64_t V, int64_t H, const int32_t *ids, void *out,
+                       int64_t T, void *stream)
+{
+    if (V < 1 || H < 8 || H % 8 != 0 || T < 0) return BI_ERR_INVALID;
+    if (T == 0) return BI_OK;
+    if (!table || !ids || !out || !aligned16(table) || !aligned16(out)) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_embedding(table, V, H, ids, out, T, d->status, d->num_sms,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+bi_status bi_rope_kv_write(const bi_paged_kv *kv, const void *qkv, const int32_t *positions,
+                           const int64_t *slot_mapping, void *q_out, int64_t T, int32_t Hq,
+                           float theta, void *stream)
+{
+    if (!kv_ok(kv) || !head_dim_ok(kv->head_dim) || T < 0) return BI_ERR_INVALID;
+    if (Hq < 1 || Hq % kv->num_kv_heads != 0) return BI_ERR_INVALID;
+    if (!(theta > 1.0f) || !std::isfinite(theta)) return BI_ERR_INVALID;
+    if (T == 0) return BI_OK;
+    if (!qkv || !positions || !slot_mapping || !q_out || !aligned16(qkv) || !aligned16(q_out))
+        return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_rope_kv(qkv, positions, slot_mapping, q_out, kv->k_cache,
+                                        kv->v_cache, kv->num_pages, Hq, kv->num_kv_heads,
+                                        kv->head_dim, double(theta), T, d->status, d->num_sms,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+bi_status bi_swiglu(const void *gu, void *out, int64_t T, int64_t F, void *stream)
+{
+    if (T < 0 || F < 8 || F % 8 != 0) return BI_ERR_INVALID;
+    if (T == 0) return BI_OK;
+    if (!gu || !out || !aligned16(gu) || !aligned16(out)) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_swiglu(gu, out, T, F, d->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+bi_status bi_argmax(const float *logits, int64_t T, int64_t V, int32_t *out, void *stream)
+{
+    if (T < 0 || V < 4 || V % 4 != 0 || V > INT32_MAX) return BI_ERR_INVALID;
+    if (T == 0) return BI_OK;
+    if (!logits || !out || !aligned16(logits)) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_argmax(logits, T, V, out, d->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
 static bool attn_common_ok(const bi_paged_kv *kv, int32_t Hq)

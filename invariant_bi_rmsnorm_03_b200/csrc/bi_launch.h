@@ -14,6 +14,9 @@ namespace bi {
 void rmsnorm_shape(int64_t H, int *items, int *threads);
 cudaError_t launch_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H,
                            float eps, bool out_f32, int num_sms, cudaStream_t s);
+// x <- round(x + delta); y <- RMSNorm(x) exactly as launch_rmsnorm computes it
+cudaError_t launch_add_rmsnorm(void *x, const void *delta, const void *w, void *y, int64_t M,
+                               int64_t H, float eps, bool out_f32, int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- matmul
 constexpr int kGemmBK = 64;  // K slice; the output tile is 256 x 256 per SM pair
@@ -67,6 +70,18 @@ cudaError_t launch_attention(const CUtensorMap &tq, const AttnParams &p, int hea
                              cudaStream_t s);
 cudaError_t launch_attn_combine(const AttnParams &p, int head_dim, cudaStream_t s);
 cudaError_t launch_attn_order(const int32_t *seq_lens, int B, int32_t *order, cudaStream_t s);
+
+// ---------------------------------------------------------------- decoder glue
+cudaError_t launch_embedding(const void *table, int64_t V, int64_t H, const int32_t *ids,
+                             void *out, int64_t T, unsigned *status, int num_sms, cudaStream_t s);
+cudaError_t launch_rope_kv(const void *qkv, const int32_t *pos, const int64_t *slots,
+                           void *q_out, void *k_cache, void *v_cache, int64_t num_pages, int Hq,
+                           int Hkv, int d, double theta, int64_t T, unsigned *status, int num_sms,
+                           cudaStream_t s);
+cudaError_t launch_swiglu(const void *gu, void *out, int64_t T, int64_t F, int num_sms,
+                          cudaStream_t s);
+cudaError_t launch_argmax(const float *logits, int64_t T, int64_t V, int32_t *out, int num_sms,
+                          cudaStream_t s);
 
 // ---------------------------------------------------------------- debug
 cudaError_t launch_bounded_wait_probe(unsigned *status, uint64_t timeout_ns, cudaStream_t s);

@@ -1,0 +1,275 @@
+// glue.cu -- the elementwise and per-row operations of a decoder layer around
+// the three batch-invariant kernels: token embedding, rotary position
+// embedding fused with the KV-cache write, SwiGLU, and the greedy argmax.
+//
+// The reports on "Defeating Nondeterminism in LLM Inference" measure
+// invariance end to end by completing one prompt greedily many times among
+// other requests and counting the distinct completions (xitu-tech news,
+// "显著成果与高昂成本"; liuwei.blog, "实验成果").  They name no layer beyond
+// RMSNorm, matmul and attention; the decoder is read as the plain pre-norm
+// transformer.  Every operation here computes each output element (or each
+// row's argmax) from its own row's inputs only, in an order fixed by the
+// row's shape, so it is batch-invariant by construction.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "bi_common.cuh"
+#include "bi_launch.h"
+
+namespace bi {
+namespace {
+
+__device__ __forceinline__ float lo16(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float hi16(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack2(float a, float b)
+{
+    __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&p);
+}
+
+// ---------------------------------------------------------------- embedding
+// out[t, :] = table[ids[t], :]: one thread per 16-byte piece.
+__global__ void embedding_kernel(const uint4 *__restrict__ table, int64_t V, int pieces,
+                                 const int32_t *__restrict__ ids, uint4 *__restrict__ out,
+                                 int64_t T, unsigned *status)
+{
+    const int64_t n = T * pieces;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t t = i / pieces;
+        const int p = static_cast<int>(i - t * pieces);
+        const int64_t id = __ldg(ids + t);
+        if (id < 0 || id >= V) {
+            if (p == 0) record_status(status, BI_DEV_BAD_INDEX);
+            continue;
+        }
+        out[i] = __ldg(table + id * pieces + p);
+    }
+}
+
+// ---------------------------------------------------------------- RoPE
+// One block per token (grid-stride).  The token's d/2 rotation angles
+// angle_i = pos * theta^(-2i/d) and their cosine and sine are evaluated in
+// double precision once per token and rounded to float; then each 16-byte
+// piece pair (values 8c..8c+7 and d/2+8c..d/2+8c+7) of every q and k head
+// is rotated in fp32:
+//   lo' = round(round(lo cos) - round(hi sin)),  hi' = round(round(hi cos) + round(lo sin))
+// and rounded to bf16.  q goes to q_out [T, Hq, d]; the rotated k and the
+// unchanged v go to the token's cache slot (page blocks in core-matrix
+// order: value 8vg + c of token 8kg + r at piece (kg * d/8 + vg) * 8 + r).
+constexpr int kRopeThreads = 256;
+constexpr int kMaxHalf = 64;  // head_dim <= 128
+
+__global__ void __launch_bounds__(kRopeThreads)
+rope_kv_kernel(const uint4 *__restrict__ qkv, const int32_t *__restrict__ pos,
+               const int64_t *__restrict__ slots, uint4 *__restrict__ q_out, uint4 *k_cache,
+               uint4 *v_cache, int64_t num_pages, int Hq, int Hkv, int d, double theta, int64_t T,
+               unsigned *status)
+{
+    __shared__ float cs[kMaxHalf], sn[kMaxHalf];
+    const int half = d / 2;
+    const int pieces = d / 8;          // 16-byte pieces of a head
+    const int hp = half / 8;           // pieces of a half head
+    const int row_pieces = (Hq + 2 * Hkv) * pieces;
+    const int rot_items = (Hq + Hkv) * hp;    // rotated piece pairs of q and k
+    const int items = rot_items + Hkv * pieces;  // + plain v pieces
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        const int32_t p = __ldg(pos + t);
+        const int64_t slot = __ldg(slots + t);
+        __syncthreads();  // the previous token's angles are no longer read
+        if (threadIdx.x < half) {
+            const double inv = pow(theta, -2.0 * double(threadIdx.x) / double(d));
+            double s, c;
+            sincos(double(p) * inv, &s, &c);
+            cs[threadIdx.x] = static_cast<float>(c);
+            sn[threadIdx.x] = static_cast<float>(s);
+        }
+        __syncthreads();
+        bool write_kv = slot >= 0;
+        if (slot >= num_pages * kPage) {
+            write_kv = false;
+            if (threadIdx.x == 0) record_status(status, BI_DEV_BAD_INDEX);
+        }
+        const int64_t page = slot / kPage;
+        const int off = static_cast<int>(slot % kPage);
+        // piece of the cache block holding token `off`, value piece vg
+        const int64_t blk_row = (off >> 3) * (8 * pieces) + (off & 7);
+        const uint4 *row = qkv + t * row_pieces;
+        for (int it = threadIdx.x; it < items; it += blockDim.x) {
+            if (it < rot_items) {
+                const int h = it / hp;          // 0..Hq-1 q heads, then k heads
+                const int c = it - h * hp;      // piece of the low half
+                const uint4 a = row[h * pieces + c];
+                const uint4 b = row[h * pieces + hp + c];
+                const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+                const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
+                uint32_t lo[4], hi[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int i0 = 8 * c + 2 * k;
+                    const float c0 = cs[i0], s0 = sn[i0], c1 = cs[i0 + 1], s1 = sn[i0 + 1];
+                    const float a0 = lo16(av[k]), a1 = hi16(av[k]);
+                    const float b0 = lo16(bv[k]), b1 = hi16(bv[k]);
+                    lo[k] = pack2(__fsub_rn(__fmul_rn(a0, c0), __fmul_rn(b0, s0)),
+                                  __fsub_rn(__fmul_rn(a1, c1), __fmul_rn(b1, s1)));
+                    hi[k] = pack2(__fadd_rn(__fmul_rn(b0, c0), __fmul_rn(a0, s0)),
+                                  __fadd_rn(__fmul_rn(b1, c1), __fmul_rn(a1, s1)));
+                }
+                const uint4 lo4 = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                const uint4 hi4 = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                if (h < Hq) {
+                    uint4 *qo = q_out + (t * Hq + h) * pieces;
+                    qo[c] = lo4;
+                    qo[hp + c] = hi4;
+                } else if (write_kv) {
+                    const int g = h - Hq;
+                    uint4 *blk = k_cache + (page * Hkv + g) * (kPage * pieces) + blk_row;
+                    blk[c * 8] = lo4;
+                    blk[(hp + c) * 8] = hi4;
+                }
+            } else if (write_kv) {
+                const int j = it - rot_items;
+                const int g = j / pieces;
+                const int vg = j - g * pieces;
+                v_cache[(page * Hkv + g) * (kPage * pieces) + blk_row + vg * 8] =
+                    row[(Hq + Hkv + g) * pieces + vg];
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- SwiGLU
+// out[t, j] = round( silu(g) * u ),  g = gu[t, j], u = gu[t, F + j],
+// silu(g) = g / (1 + e^-g), fp32; one thread per 8 outputs.
+__global__ void swiglu_kernel(const uint4 *__restrict__ gu, uint4 *__restrict__ out, int64_t T,
+                              int64_t fp)
+{
+    const int64_t n = T * fp;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t t = i / fp;
+        const int64_t c = i - t * fp;
+        const uint4 g4 = __ldcs(gu + t * 2 * fp + c);
+        const uint4 u4 = __ldcs(gu + t * 2 * fp + fp + c);
+        const uint32_t gv[4] = {g4.x, g4.y, g4.z, g4.w};
+        const uint32_t uv[4] = {u4.x, u4.y, u4.z, u4.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float g0 = lo16(gv[k]), g1 = hi16(gv[k]);
+            const float s0 = __fdiv_rn(g0, __fadd_rn(1.0f, expf(-g0)));
+            const float s1 = __fdiv_rn(g1, __fadd_rn(1.0f, expf(-g1)));
+            o[k] = pack2(__fmul_rn(s0, lo16(uv[k])), __fmul_rn(s1, hi16(uv[k])));
+        }
+        __stcs(out + i, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+}
+
+// ---------------------------------------------------------------- argmax
+// One block per row (grid-stride): each thread scans its float4 pieces in
+// index order, then the (value, index) pairs are combined by a warp
+// butterfly and across warps.  The combination keeps the larger value and,
+// on equal values, the lower index: an exact selection, the same whatever
+// the order of combination.  NaN entries are never selected.
+constexpr int kArgmaxThreads = 512;
+
+struct Best {
+    float v;
+    int32_t i;
+};
+
+__device__ __forceinline__ Best better(Best a, Best b)
+{
+    return (b.v > a.v || (b.v == a.v && b.i < a.i)) ? b : a;
+}
+
+__global__ void __launch_bounds__(kArgmaxThreads)
+argmax_kernel(const float4 *__restrict__ logits, int64_t T, int64_t V, int32_t *__restrict__ out)
+{
+    __shared__ Best part[kArgmaxThreads / 32];
+    const int64_t q = V / 4;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        Best b{-INFINITY, INT32_MAX};
+        const float4 *row = logits + t * q;
+        for (int64_t c = threadIdx.x; c < q; c += blockDim.x) {
+            const float4 v = __ldcs(row + c);
+            const int32_t j = static_cast<int32_t>(4 * c);
+            b = better(b, Best{v.x, j});
+            b = better(b, Best{v.y, j + 1});
+            b = better(b, Best{v.z, j + 2});
+            b = better(b, Best{v.w, j + 3});
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            Best o;
+            o.v = __shfl_xor_sync(0xffffffffu, b.v, off);
+            o.i = __shfl_xor_sync(0xffffffffu, b.i, off);
+            b = better(b, o);
+        }
+        if (lane == 0) part[warp] = b;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            Best r = part[0];
+            for (int k = 1; k < int(blockDim.x >> 5); ++k) r = better(r, part[k]);
+            out[t] = r.i == INT32_MAX ? 0 : r.i;  // a row of NaN only: index 0
+        }
+        __syncthreads();  // part[] is reused by the next row
+    }
+}
+
+unsigned grid_for(int64_t items, int threads, int num_sms)
+{
+    const int64_t blocks = (items + threads - 1) / threads;
+    const int64_t cap = int64_t(num_sms) * 8;
+    return static_cast<unsigned>(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_embedding(const void *table, int64_t V, int64_t H, const int32_t *ids,
+                             void *out, int64_t T, unsigned *status, int num_sms, cudaStream_t s)
+{
+    const int pieces = static_cast<int>(H / 8);
+    embedding_kernel<<<grid_for(T * pieces, 256, num_sms), 256, 0, s>>>(
+        static_cast<const uint4 *>(table), V, pieces, ids, static_cast<uint4 *>(out), T, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rope_kv(const void *qkv, const int32_t *pos, const int64_t *slots,
+                           void *q_out, void *k_cache, void *v_cache, int64_t num_pages, int Hq,
+                           int Hkv, int d, double theta, int64_t T, unsigned *status, int num_sms,
+                           cudaStream_t s)
+{
+    const int64_t cap = int64_t(num_sms) * 8;
+    const unsigned grid = static_cast<unsigned>(T < cap ? T : cap);
+    rope_kv_kernel<<<grid, kRopeThreads, 0, s>>>(
+        static_cast<const uint4 *>(qkv), pos, slots, static_cast<uint4 *>(q_out),
+        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), num_pages, Hq, Hkv, d,
+        theta, T, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu(const void *gu, void *out, int64_t T, int64_t F, int num_sms,
+                          cudaStream_t s)
+{
+    const int64_t fp = F / 8;
+    swiglu_kernel<<<grid_for(T * fp, 256, num_sms), 256, 0, s>>>(
+        static_cast<const uint4 *>(gu), static_cast<uint4 *>(out), T, fp);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_argmax(const float *logits, int64_t T, int64_t V, int32_t *out, int num_sms,
+                          cudaStream_t s)
+{
+    const int64_t cap = int64_t(num_sms) * 4;
+    const unsigned grid = static_cast<unsigned>(T < cap ? T : cap);
+    argmax_kernel<<<grid, kArgmaxThreads, 0, s>>>(reinterpret_cast<const float4 *>(logits), T, V,
+                                                  out);
+    return cudaGetLastError();
+}
+
+}  // namespace bi

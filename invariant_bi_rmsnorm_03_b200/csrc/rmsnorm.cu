@@ -17,10 +17,16 @@
 // T and ITEMS depend only on H, so a row gets the same bits whatever M is,
 // whichever block handles it and wherever it sits in the batch.
 //
-// Memory: rows are loaded once into registers with 128-bit loads (a block
-// loads all of its R rows before reducing any, to keep more bytes in
-// flight), the output is written with 128-bit stores.  The grid strides
-// over groups of R rows.
+// Residual form (between the sublayers of a pre-norm decoder): x is first
+// replaced by round(x + delta) (fp32 add, bf16 RNE) and written back, then
+// normalised by the same code, so its y equals the plain form's y of the
+// updated row bit for bit.
+//
+// Memory: a row is loaded once into registers with 128-bit streaming loads
+// and written with 128-bit stores.  One row per block at a time, with many
+// small blocks resident per SM (8 of 256 threads at H = 4096) so that the
+// loads of some rows overlap the reduction and stores of others; the grid
+// strides over rows.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -84,101 +90,139 @@ __device__ __forceinline__ void store8(void *y, int64_t idx, const uint4 &xv, co
     }
 }
 
-// A block handles R rows at a time: all R rows are loaded before any is
-// reduced, so that more bytes are in flight.  R changes only how rows are
-// grouped into blocks; each row's arithmetic is the same for every R.
-template <int ITEMS, int R, bool OUT_F32, int MAXT>
-__global__ void __launch_bounds__(MAXT, MAXT <= 256 ? 2 : 1) rmsnorm_kernel(const uint4 *__restrict__ x,
+__device__ __forceinline__ uint32_t add_pair(uint32_t a, uint32_t b)
+{
+    __nv_bfloat162 p = __floats2bfloat162_rn(__fadd_rn(bf_lo(a), bf_lo(b)),
+                                             __fadd_rn(bf_hi(a), bf_hi(b)));
+    return *reinterpret_cast<uint32_t *>(&p);
+}
+
+// x <- round(x + delta), element by element in fp32.
+__device__ __forceinline__ uint4 add8(const uint4 &a, const uint4 &b)
+{
+    return make_uint4(add_pair(a.x, b.x), add_pair(a.y, b.y), add_pair(a.z, b.z),
+                      add_pair(a.w, b.w));
+}
+
+// One row per block iteration; the grid strides over rows.
+// ADD: the residual form -- x is first replaced by round(x + delta) (and
+// written back), then normalised exactly as the plain form normalises it.
+template <int ITEMS, bool OUT_F32, int MAXT, bool ADD, int MINB>
+__global__ void __launch_bounds__(MAXT, MINB) rmsnorm_kernel(uint4 *x,
+                                                       const uint4 *__restrict__ delta,
                                                        const uint4 *__restrict__ w,
                                                        void *__restrict__ y, int64_t M, int H,
                                                        float eps)
 {
-    __shared__ float part[R][32];
+    __shared__ float part[32];
     const int chunks = H >> 3;
     const int T = blockDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const float h_den = static_cast<float>(H);
 
-    for (int64_t row0 = int64_t(blockIdx.x) * R; row0 < M; row0 += int64_t(gridDim.x) * R) {
-        uint4 v[R][ITEMS];
-        float acc[R];
+    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+        uint4 v[ITEMS];
+        uint4 dv[ADD ? ITEMS : 1];
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            acc[r] = 0.0f;
-            const int64_t row = row0 + r;
+        for (int it = 0; it < ITEMS; ++it) {
+            const int c = threadIdx.x + it * T;
+            if (c < chunks) {
+                v[it] = __ldcs(x + row * chunks + c);
+                if constexpr (ADD) dv[it] = __ldcs(delta + row * chunks + c);
+            }
+        }
+        float acc = 0.0f;
 #pragma unroll
-            for (int it = 0; it < ITEMS; ++it) {
-                const int c = threadIdx.x + it * T;
-                if (row < M && c < chunks) v[r][it] = __ldcs(x + row * chunks + c);
+        for (int it = 0; it < ITEMS; ++it) {
+            const int c = threadIdx.x + it * T;
+            if (c < chunks) {
+                if constexpr (ADD) {
+                    v[it] = add8(v[it], dv[it]);
+                    x[row * chunks + c] = v[it];
+                }
+                acc = sumsq8(v[it], acc);
             }
         }
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-#pragma unroll
-            for (int it = 0; it < ITEMS; ++it) {
-                const int c = threadIdx.x + it * T;
-                if (row0 + r < M && c < chunks) acc[r] = sumsq8(v[r][it], acc[r]);
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1)
-                acc[r] = __fadd_rn(acc[r], __shfl_xor_sync(0xffffffffu, acc[r], off));
-            if (lane == 0) part[r][warp] = acc[r];
-        }
+        for (int off = 16; off > 0; off >>= 1)
+            acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+        if (lane == 0) part[warp] = acc;
         __syncthreads();
+        float tot = 0.0f;
+        for (int i = 0; i < (T >> 5); ++i) tot = __fadd_rn(tot, part[i]);
+        const float rstd = rsqrtf(__fadd_rn(__fdiv_rn(tot, h_den), eps));
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int64_t row = row0 + r;
-            if (row >= M) break;
-            float tot = 0.0f;
-            for (int i = 0; i < (T >> 5); ++i) tot = __fadd_rn(tot, part[r][i]);
-            const float rstd = rsqrtf(__fadd_rn(__fdiv_rn(tot, h_den), eps));
-#pragma unroll
-            for (int it = 0; it < ITEMS; ++it) {
-                const int c = threadIdx.x + it * T;
-                if (c < chunks) store8<OUT_F32>(y, row * chunks + c, v[r][it], __ldg(w + c), rstd);
-            }
+        for (int it = 0; it < ITEMS; ++it) {
+            const int c = threadIdx.x + it * T;
+            if (c < chunks) store8<OUT_F32>(y, row * chunks + c, v[it], __ldg(w + c), rstd);
         }
-        __syncthreads();  // part[] is reused by the next group of rows
+        __syncthreads();  // part[] is reused by the next row
     }
 }
 
-template <int ITEMS, int R, int MAXT>
-cudaError_t launch_rows(const void *x, const void *w, void *y, int64_t M, int H, float eps,
-                        bool out_f32, int threads, cudaStream_t s)
+struct NormArgs {
+    void *x;
+    const void *delta;  // non-null: the residual form
+    const void *w;
+    void *y;
+    int64_t M;
+    int H;
+    float eps;
+    bool out_f32;
+    int threads;
+    int num_sms;
+};
+
+// Blocks resident per SM: as many as the 2048 threads of an SM hold, within
+// the registers a thread needs (the row's ITEMS 16-byte chunks, twice that
+// for the residual form).
+template <int ITEMS, int MAXT, bool ADD>
+constexpr int min_blocks()
 {
+    constexpr int full = 2048 / MAXT;                     // 8 or 2
+    constexpr int data_regs = 4 * ITEMS * (ADD ? 2 : 1);  // registers of row data
+    return data_regs <= 8 ? full : (data_regs <= 16 ? full / 2 : full / 4 > 0 ? full / 4 : 1);
+}
+
+template <int ITEMS, int MAXT, bool ADD>
+cudaError_t launch_shape(const NormArgs &a, cudaStream_t s)
+{
+    constexpr int MINB = min_blocks<ITEMS, MAXT, ADD>();
+    // Up to two waves of rows: every block takes rows in turn (grid of the
+    // resident blocks); more rows: one block per row, the hardware refills.
+    const int64_t resident = int64_t(a.num_sms) * MINB;
     const int64_t cap = int64_t(1) << 20;
-    const int64_t groups = (M + R - 1) / R;
-    const unsigned grid = static_cast<unsigned>(groups < cap ? groups : cap);
-    if (out_f32)
-        rmsnorm_kernel<ITEMS, R, true, MAXT><<<grid, threads, 0, s>>>(
-            static_cast<const uint4 *>(x), static_cast<const uint4 *>(w), y, M, H, eps);
+    int64_t grid = a.M <= 2 * resident ? (a.M < resident ? a.M : resident) : a.M;
+    if (grid > cap) grid = cap;
+    uint4 *x = static_cast<uint4 *>(a.x);
+    const uint4 *d = static_cast<const uint4 *>(a.delta);
+    const uint4 *w = static_cast<const uint4 *>(a.w);
+    const unsigned g = static_cast<unsigned>(grid);
+    if (a.out_f32)
+        rmsnorm_kernel<ITEMS, true, MAXT, ADD, MINB><<<g, a.threads, 0, s>>>(x, d, w, a.y, a.M,
+                                                                             a.H, a.eps);
     else
-        rmsnorm_kernel<ITEMS, R, false, MAXT><<<grid, threads, 0, s>>>(
-            static_cast<const uint4 *>(x), static_cast<const uint4 *>(w), y, M, H, eps);
+        rmsnorm_kernel<ITEMS, false, MAXT, ADD, MINB><<<g, a.threads, 0, s>>>(x, d, w, a.y, a.M,
+                                                                              a.H, a.eps);
     return cudaGetLastError();
 }
 
-// Rows per block R with ITEMS * R 16-byte chunks held per thread: up to 16
-// (64 registers) for blocks of at most 256 threads, two blocks per SM;
-// up to 8 for wider blocks.
-template <int ITEMS>
-cudaError_t launch_items(const void *x, const void *w, void *y, int64_t M, int H, float eps,
-                         bool out_f32, int threads, int rows_per_block, cudaStream_t s)
+template <int ITEMS, bool ADD>
+cudaError_t launch_items(const NormArgs &a, cudaStream_t s)
 {
-    if (threads <= 256) {
-        if constexpr (ITEMS <= 2)
-            if (rows_per_block >= 8)
-                return launch_rows<ITEMS, 8, 256>(x, w, y, M, H, eps, out_f32, threads, s);
-        if constexpr (ITEMS <= 4)
-            if (rows_per_block >= 4)
-                return launch_rows<ITEMS, 4, 256>(x, w, y, M, H, eps, out_f32, threads, s);
-        if (rows_per_block >= 2) return launch_rows<ITEMS, 2, 256>(x, w, y, M, H, eps, out_f32, threads, s);
-        return launch_rows<ITEMS, 1, 256>(x, w, y, M, H, eps, out_f32, threads, s);
+    return a.threads <= 256 ? launch_shape<ITEMS, 256, ADD>(a, s)
+                            : launch_shape<ITEMS, 1024, ADD>(a, s);
+}
+
+template <bool ADD>
+cudaError_t launch_norm(const NormArgs &a, int items, cudaStream_t s)
+{
+    switch (items) {
+    case 1: return launch_items<1, ADD>(a, s);
+    case 2: return launch_items<2, ADD>(a, s);
+    case 4: return launch_items<4, ADD>(a, s);
+    default: return launch_items<8, ADD>(a, s);
     }
-    if constexpr (ITEMS <= 4)
-        if (rows_per_block >= 2)
-            return launch_rows<ITEMS, 2, 1024>(x, w, y, M, H, eps, out_f32, threads, s);
-    return launch_rows<ITEMS, 1, 1024>(x, w, y, M, H, eps, out_f32, threads, s);
 }
 
 }  // namespace
@@ -196,8 +240,8 @@ void rmsnorm_shape(int64_t H, int *items, int *threads)
     *threads = static_cast<int>(t);
 }
 
-cudaError_t launch_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H,
-                           float eps, bool out_f32, int num_sms, cudaStream_t s)
+static cudaError_t launch_any(void *x, const void *delta, const void *w, void *y, int64_t M,
+                              int64_t H, float eps, bool out_f32, int num_sms, cudaStream_t s)
 {
     int items, threads;
     rmsnorm_shape(H, &items, &threads);
@@ -210,20 +254,20 @@ cudaError_t launch_rmsnorm(const void *x, const void *w, void *y, int64_t M, int
         threads = static_cast<int>((t + 31) / 32 * 32);
     }
 #endif
-    // Rows per block: enough that two blocks per SM cover M in one wave,
-    // within the registers a thread may hold (ITEMS * R <= 16; 8 for blocks
-    // wider than 256 threads).
-    const int64_t blocks = int64_t(num_sms) * (threads <= 256 ? 2 : 1);
-    const int cap = threads <= 256 ? 16 : 8;
-    int rpb = 1;
-    while (rpb < 8 && int64_t(rpb) * blocks < M && items * rpb * 2 <= cap) rpb *= 2;
-    const int h = static_cast<int>(H);
-    switch (items) {
-    case 1: return launch_items<1>(x, w, y, M, h, eps, out_f32, threads, rpb, s);
-    case 2: return launch_items<2>(x, w, y, M, h, eps, out_f32, threads, rpb, s);
-    case 4: return launch_items<4>(x, w, y, M, h, eps, out_f32, threads, rpb, s);
-    default: return launch_items<8>(x, w, y, M, h, eps, out_f32, threads, rpb, s);
-    }
+    const NormArgs a{x, delta, w, y, M, static_cast<int>(H), eps, out_f32, threads, num_sms};
+    return delta ? launch_norm<true>(a, items, s) : launch_norm<false>(a, items, s);
+}
+
+cudaError_t launch_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H,
+                           float eps, bool out_f32, int num_sms, cudaStream_t s)
+{
+    return launch_any(const_cast<void *>(x), nullptr, w, y, M, H, eps, out_f32, num_sms, s);
+}
+
+cudaError_t launch_add_rmsnorm(void *x, const void *delta, const void *w, void *y, int64_t M,
+                               int64_t H, float eps, bool out_f32, int num_sms, cudaStream_t s)
+{
+    return launch_any(x, delta, w, y, M, H, eps, out_f32, num_sms, s);
 }
 
 }  // namespace bi

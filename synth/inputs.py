@@ -230,3 +230,55 @@ def torch_normal_bf16(shape, seed: int, device, std: float = 1.0):
     t = torch.empty(shape, dtype=torch.bfloat16, device=device)
     t.normal_(0.0, std, generator=gen)
     return t
+
+
+# ---------------------------------------------------------------------------
+# the toy decoder's weights and the unique-completion workload
+# ---------------------------------------------------------------------------
+
+def toy_decoder_weights(shapes: dict, seed: int, device, std: float = 0.02) -> dict:
+    """Random-init weights for the toy decoder: every matrix N(0, std) drawn
+    on ``device`` by torch's generator (one seed per tensor, in the order of
+    ``shapes``), every norm weight 1."""
+    import torch
+
+    out = {}
+    for k, (name, shape) in enumerate(shapes.items()):
+        if len(shape) == 1:
+            out[name] = torch.ones(shape, dtype=torch.bfloat16, device=device)
+        else:
+            out[name] = torch_normal_bf16(shape, seed * 1000 + k, device, std=std)
+    return out
+
+
+def unique_completion_workload(seed: int = 4, n_target: int = 1000, n_other: int = 1000,
+                               prompt_len: int = 64, gen_len: int = 256, vocab: int = 32000,
+                               other_prompt_max: int = 512, steps_span: int = 2000):
+    """One fixed prompt (``prompt_len`` ids drawn from ``seed``) to be
+    completed ``n_target`` times, amid ``n_other`` requests with random
+    prompts of U(1, other_prompt_max) tokens and U(1, gen_len) new tokens.
+    Arrival steps are drawn in bursts (each request's step is uniform inside
+    one of several windows of random width over ``steps_span`` steps), so
+    the number of running requests sweeps from 1 up to the scheduler's cap.
+
+    Returns ``(prompt, requests)`` with requests a list of dicts
+    ``{rid, prompt, max_new, arrival, tag}`` in random order."""
+    g = rng(seed)
+    prompt = g.integers(0, vocab, size=prompt_len).astype(np.int32)
+    n = n_target + n_other
+    tags = np.array(["target"] * n_target + ["other"] * n_other)
+    g.shuffle(tags)
+    # bursts: 16 windows with random centres and widths
+    centres = np.sort(g.uniform(0, steps_span, size=16))
+    widths = g.uniform(1, steps_span / 8, size=16)
+    which = g.integers(0, 16, size=n)
+    arrival = np.clip(centres[which] + g.uniform(-0.5, 0.5, size=n) * widths[which], 0, None)
+    reqs = []
+    for i in range(n):
+        if tags[i] == "target":
+            p, m = prompt, gen_len
+        else:
+            p = g.integers(0, vocab, size=int(g.integers(1, other_prompt_max + 1))).astype(np.int32)
+            m = int(g.integers(1, gen_len + 1))
+        reqs.append(dict(rid=i, prompt=p, max_new=m, arrival=int(arrival[i]), tag=str(tags[i])))
+    return prompt, reqs
