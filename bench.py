@@ -442,6 +442,23 @@ def traffic_record(kernel_src: str, name: str):
     return rec.get("dram_bytes_per_launch")
 
 
+def max_over_ranks(v: float, dist=None, device="cpu") -> float:
+    """The largest value of ``v`` over all ranks (every rank gets it)."""
+    if dist is None:
+        return v
+    import torch
+
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Units per second of the whole job: every rank processes
+    ``units_per_rank`` (replicas, weak scaling), over the slowest rank's time."""
+    return world * units_per_rank / (max_ms * 1e-3)
+
+
 def run_ours(args):
     import torch
 
@@ -473,11 +490,7 @@ def run_ours(args):
 
     # whole-job figures: all ranks' work over the slowest rank's time
     def maxall(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks(v, dist, dev)
 
     gemm_ms = maxall(float(mean[2]))
     dec_ms = maxall(float(mean[3]))
@@ -485,8 +498,8 @@ def run_ours(args):
     norm_ms = maxall(float(mean[1]))
     kvw_ms = maxall(float(mean[0]))
     step_ms = maxall(step_ms)
-    gemm_tf = world * wl.gemm_flops / (gemm_ms * 1e-3) / 1e12
-    dec_gbs = world * wl.dec_bytes / (dec_ms * 1e-3) / 1e9
+    gemm_tf = whole_job(wl.gemm_flops, world, gemm_ms) / 1e12
+    dec_gbs = whole_job(wl.dec_bytes, world, dec_ms) / 1e9
 
     # e2e through host buffers
     e2e_per, h2d, d2h = e2e_steps(torch, L, wl, max(2, args.steps // 2), 1)

@@ -33,7 +33,7 @@
 // split, with the same merge function.  The bits therefore do not depend on
 // how many blocks served a sequence.
 //
-// Block of 320 threads, one per SM (about 225 KB shared memory; 512 TMEM
+// Block of 448 threads, one per SM (about 225 KB shared memory; 512 TMEM
 // columns as two 256-column buffers, each holding a split's logits, then
 // its P in columns 0-127 and O_s in columns 128-255):
 //   warp 0     producer: Q by TMA once; per split the 16 pages of K and of
@@ -49,8 +49,9 @@
 //              Decode spreads the query heads over the four lane quarters,
 //              and with at most 8 heads per quarter four threads share a
 //              row (softmax_heads16).
-//   warps 2,3,8,9  merge ("fold") of O_s into the running output, one per
-//              lane quarter, overlapping the next split's softmax.
+//   warps 2,3,8-13  merge ("fold") of O_s into the running output, two per
+//              lane quarter (one per half of the head dim), overlapping the
+//              next split's softmax.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -64,9 +65,11 @@
 namespace bi {
 namespace {
 
-// Warp roles: 0 producer, 1 MMA, 4-7 softmax, 2-3 and 8-9 merge ("fold").
-// Softmax warp w and fold warp w' own TMEM lane quarter w % 4.
-constexpr int THREADS = 320;
+// Warp roles: 0 producer, 1 MMA, 4-7 softmax, 2-3 and 8-13 merge ("fold").
+// Softmax warp w and fold warp w' own TMEM lane quarter w % 4; fold warps
+// 2, 3, 8, 9 take the first half of the head dim, 10-13 the second.
+constexpr int THREADS = 448;
+constexpr int kFoldThreads = 256;
 constexpr float kLn2 = 0.693147180559945309f;
 
 template <int D>
@@ -131,7 +134,7 @@ __device__ __forceinline__ void write_out(const float (&O)[D], float l, float m,
 __device__ bool wait_drain(uint64_t *bar, uint32_t parity, uint64_t timeout_ns)
 {
     const uint64_t t0 = global_ns();
-    while (!mbar_try_wait(bar, parity))
+    while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs))
         if (global_ns() - t0 > timeout_ns) return false;
     return true;
 }
@@ -194,19 +197,6 @@ __device__ __forceinline__ uint32_t page_off(int r, int c)
 
 // ---------------------------------------------------------------- kernel
 
-// 128 columns of one lane quarter into four register arrays, one wait.
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[4][32])
-{
-    tmem_ld32(taddr, r[0]);
-    tmem_ld32(taddr + 32, r[1]);
-    tmem_ld32(taddr + 64, r[2]);
-    tmem_ld32(taddr + 96, r[3]);
-    tmem_wait_ld(r[0]);
-    tmem_wait_ld(r[1]);
-    tmem_wait_ld(r[2]);
-    tmem_wait_ld(r[3]);
-}
-
 // The order of the split sum l_s, shared by both softmax paths below.  The
 // 256 keys of a split are cut into 32-key chunks; inside a chunk, key
 // 32c + 8i + 2u + j (i < 4, u < 4, j < 2) belongs to class u.  For each class
@@ -221,75 +211,104 @@ __device__ __forceinline__ float tree8(float a0, float b0, float a1, float b1, f
                      __fadd_rn(__fadd_rn(a2, b2), __fadd_rn(a3, b3)));
 }
 
-__device__ __forceinline__ float logit(uint32_t s, float cs, float m_s)
+// p = 2^(S * cs - m_s), one rounding (fused multiply-add).  Both softmax
+// paths below use it, so a key's p has the same bits in decode and prefill.
+__device__ __forceinline__ float logit(float s, float cs, float m_s)
 {
-    return ex2(__fsub_rn(__fmul_rn(__uint_as_float(s), cs), m_s));
+    return ex2(__fmaf_rn(s, cs, -m_s));
+}
+
+// Maximum of the visible logits of 32 keys kc .. kc+31.
+__device__ __forceinline__ void chunk_max(const uint32_t (&r)[32], int kc, int t, float (&mx)[8])
+{
+    if (kc + 31 <= t) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[j]));
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (kc + j <= t) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[j]));
+    }
+}
+
+// p of 16 keys kc .. kc+15 (half `hf` of a 32-key chunk): packed bf16 P
+// written to TMEM at `pcol` (8 columns); tr[u] gets this half's part of
+// the chunk's class-u tree: (a_{2hf} + b_{2hf}) + (a_{2hf+1} + b_{2hf+1}).
+__device__ __forceinline__ void piece_exp(const uint32_t (&r)[16], int kc, int t, float cs,
+                                          float m_s, uint32_t pcol, float (&tr)[4])
+{
+    float e[16];
+    if (kc + 15 <= t) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) e[j] = logit(__uint_as_float(r[j]), cs, m_s);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            e[j] = (kc + j <= t) ? logit(__uint_as_float(r[j]), cs, m_s) : 0.0f;
+    }
+    uint32_t pk[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2(e[2 * j], e[2 * j + 1]);
+    tmem_st8(pcol, pk);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        tr[u] = __fadd_rn(__fadd_rn(e[2 * u], e[2 * u + 1]), __fadd_rn(e[8 + 2 * u], e[9 + 2 * u]));
 }
 
 // Softmax of one split, one row per thread (any row layout; used by
 // prefill and by decode with more than 8 query rows per lane quarter).
-// S is read from TMEM columns sb .. sb+255 in two passes of two 128-column
-// loads; P (bf16 pairs) is written over columns sb .. sb+127 as the second
-// pass goes (each store lands on columns this thread has already read).
-// Returns m_s (scaled, log2 units) and l_s.  (P V cannot start before the
-// whole pass is done: it writes O_s over the logits of keys 128..255.)
+// S is read from TMEM columns sb .. sb+255 in two passes of 16-column
+// loads, the next load in flight while a piece is processed; P (bf16 pairs)
+// is written over columns sb .. sb+127 as the second pass goes (each store
+// lands on columns this thread has already read).  Returns m_s (scaled,
+// log2 units) and l_s.  (P V cannot start before the whole pass is done: it
+// writes O_s over the logits of keys 128..255.)
 __device__ __forceinline__ void softmax_rows(uint32_t sb, int k0, int t, float cs, float &m_s,
                                              float &l_s)
 {
+    constexpr int NP = kSplit / 16;  // 16-key pieces
     // pass 1: maximum of the raw logits over the visible keys.  For c > 0,
     // x -> round(x * c) is monotonic, so max_j round(S_j c) = round(max_j S_j * c).
     // (A maximum is exact in any order; eight accumulators break the chain.)
     float mx[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+    // The loops are kept rolled (two loads of each kind per trip): a small
+    // instruction footprint matters more here than unrolling, since the
+    // block's other warps run other code on the same sub-partitions.
+    {
+        // 32-column loads, the next in flight while a chunk is scanned
+        uint32_t ra[32], rb[32];
+        tmem_ld32(sb, ra);
 #pragma unroll 1
-    for (int c = 0; c < kSplit / 32; c += 4) {
-        uint32_t r[4][32];
-        tmem_ld128(sb + 32 * c, r);
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const int kc = k0 + 32 * (c + h);
-            if (kc + 31 <= t) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[h][j]));
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (kc + j <= t) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[h][j]));
-            }
+        for (int c = 0; c < NP / 2; c += 2) {
+            tmem_wait_ld(ra);
+            tmem_ld32(sb + 32 * (c + 1), rb);
+            chunk_max(ra, k0 + 32 * c, t, mx);
+            tmem_wait_ld(rb);
+            if (c + 2 < NP / 2) tmem_ld32(sb + 32 * (c + 2), ra);
+            chunk_max(rb, k0 + 32 * (c + 1), t, mx);
         }
     }
     const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
     m_s = __fmul_rn(mraw, cs);
-    // pass 2: p = 2^(round(S c) - m_s), masked keys 0; P into TMEM; the sum
-    // in the order described above.
+    // pass 2: p = 2^(S c - m_s), masked keys 0; P into TMEM; the sum in the
+    // order of tree8 (a chunk's two halves are its pieces h and h + 1).
     float S[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    uint32_t ra[16], rb[16];
+    tmem_ld16(sb, ra);
 #pragma unroll 1
-    for (int c = 0; c < kSplit / 32; c += 4) {
-        uint32_t r[4][32];
-        tmem_ld128(sb + 32 * c, r);
+    for (int h = 0; h < NP; h += 2) {
+        float t0[4], t1[4];
+        tmem_wait_ld(ra);
+        tmem_ld16(sb + 16 * (h + 1), rb);
+        piece_exp(ra, k0 + 16 * h, t, cs, m_s, sb + 8 * h, t0);
+        tmem_wait_ld(rb);
+        if (h + 2 < NP) tmem_ld16(sb + 16 * (h + 2), ra);
+        piece_exp(rb, k0 + 16 * (h + 1), t, cs, m_s, sb + 8 * (h + 1), t1);
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const int kc = k0 + 32 * (c + h);
-            float e[32];
-            if (kc + 31 <= t) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) e[j] = logit(r[h][j], cs, m_s);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) e[j] = (kc + j <= t) ? logit(r[h][j], cs, m_s) : 0.0f;
-            }
-            uint32_t pk[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(e[2 * j], e[2 * j + 1]);
-            tmem_st16(sb + 16 * (c + h), pk);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                S[u] = __fadd_rn(S[u], tree8(e[2 * u], e[2 * u + 1], e[8 + 2 * u], e[9 + 2 * u],
-                                             e[16 + 2 * u], e[17 + 2 * u], e[24 + 2 * u],
-                                             e[25 + 2 * u]));
-        }
+        for (int u = 0; u < 4; ++u) S[u] = __fadd_rn(S[u], __fadd_rn(t0[u], t1[u]));
     }
     tmem_wait_st();
     l_s = __fadd_rn(__fadd_rn(S[0], S[1]), __fadd_rn(S[2], S[3]));
@@ -298,61 +317,79 @@ __device__ __forceinline__ void softmax_rows(uint32_t sb, int k0, int t, float c
 // Softmax of one split for decode when the query rows of this lane quarter
 // sit in its lanes 0..7: four threads share a row.  Thread t = u + 4 v
 // handles lane v, keys 8m + 2u and 8m + 2u + 1 (m < 32) -- class u of the
-// order above -- read with the 16-lane TMEM shape, and writes the packed P
-// of those keys (P column 4m + u) with the matching 16-lane store.  The
-// arithmetic per row is the same as softmax_rows, so the bits are equal.
-// sb is the TMEM address of lane 0 of the quarter.
+// order above -- read with the 16-lane TMEM shape (64 keys a load, the next
+// load in flight), and writes the packed P of those keys (P column 4m + u)
+// with the matching 16-lane store.  The arithmetic per row is the same as
+// softmax_rows, so the bits are equal.  sb is the TMEM address of lane 0 of
+// the quarter.
 __device__ __forceinline__ void softmax_heads16(uint32_t sb, int k0, int t, float cs, float &m_s,
                                                 float &l_s)
 {
     const int u = threadIdx.x & 3;
-    float v[64];  // v[2m], v[2m+1]: keys 8m + 2u, 8m + 2u + 1
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        uint32_t r[64];
-        tmem_ld_16x256b_x16(sb + 128 * h, r);
-        tmem_wait_ld(r);
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            v[2 * (16 * h + m)] = __uint_as_float(r[4 * m]);
-            v[2 * (16 * h + m) + 1] = __uint_as_float(r[4 * m + 1]);
-        }
-    }
     const bool whole = k0 + kSplit - 1 <= t;  // every key of the split visible
+    // r[4m'], r[4m'+1] of load k: keys 8m + 2u, 8m + 2u + 1 with m = 8k + m'
+    auto vis = [&](int m, int j) { return whole || k0 + 8 * m + 2 * u + j <= t; };
+    uint32_t ra[32], rb[32];
     float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    auto load_max = [&](const uint32_t (&r)[32], int k) {
 #pragma unroll
-    for (int m = 0; m < 32; ++m)
+        for (int mm = 0; mm < 8; ++mm)
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-            if (whole || k0 + 8 * m + 2 * u + j <= t) mx[m & 3] = fmaxf(mx[m & 3], v[2 * m + j]);
+            for (int j = 0; j < 2; ++j) {
+                const int m = 8 * k + mm;
+                if (vis(m, j)) mx[m & 3] = fmaxf(mx[m & 3], __uint_as_float(r[4 * mm + j]));
+            }
+    };
+    // loops kept rolled (small instruction footprint): the load just
+    // waited for is moved to `ra` and the next one issued into `rb`
+    tmem_ld_16x256b_x8(sb, rb);
+#pragma unroll 1
+    for (int k = 0; k < 4; ++k) {
+        tmem_wait_ld(rb);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ra[j] = rb[j];
+        if (k + 1 < 4) tmem_ld_16x256b_x8(sb + 64 * (k + 1), rb);
+        load_max(ra, k);
+    }
     float mraw = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
     mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 1));
     mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 2));
     m_s = __fmul_rn(mraw, cs);
 
+    // Load k covers 32-key chunks 2k and 2k + 1; its P goes to columns
+    // 32k .. 32k + 31 of the quarter's lanes 0..7.
     float S = 0.0f;
-    uint32_t pk[2][32];  // 16x128b store operands: [half][2 * m' + lane-half]
+    auto load_exp = [&](const uint32_t (&r)[32], int k) {
+        uint32_t pk[16];  // 16x128b.x8 store operands: [2 m' + lane-half]
 #pragma unroll
-    for (int c = 0; c < kSplit / 32; ++c) {
-        float e[8];
+        for (int cc = 0; cc < 2; ++cc) {
+            float e[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int m = 4 * c + i;
-                const float x = ex2(__fsub_rn(__fmul_rn(v[2 * m + j], cs), m_s));
-                e[2 * i + j] = (whole || k0 + 8 * m + 2 * u + j <= t) ? x : 0.0f;
+                for (int j = 0; j < 2; ++j) {
+                    const int mm = 4 * cc + i, m = 8 * k + mm;
+                    const float x = logit(__uint_as_float(r[4 * mm + j]), cs, m_s);
+                    e[2 * i + j] = vis(m, j) ? x : 0.0f;
+                }
+            S = __fadd_rn(S, tree8(e[0], e[1], e[2], e[3], e[4], e[5], e[6], e[7]));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                pk[2 * (4 * cc + i)] = pack_bf16x2(e[2 * i], e[2 * i + 1]);
+                pk[2 * (4 * cc + i) + 1] = 0u;  // lanes 8..15 hold no query row
             }
-        S = __fadd_rn(S, tree8(e[0], e[1], e[2], e[3], e[4], e[5], e[6], e[7]));
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int m = 4 * c + i;
-            pk[m >> 4][2 * (m & 15)] = pack_bf16x2(e[2 * i], e[2 * i + 1]);
-            pk[m >> 4][2 * (m & 15) + 1] = 0u;  // lanes 8..15 hold no query row
         }
+        tmem_st_16x128b_x8(sb + 32 * k, pk);
+    };
+    tmem_ld_16x256b_x8(sb, rb);
+#pragma unroll 1
+    for (int k = 0; k < 4; ++k) {
+        tmem_wait_ld(rb);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ra[j] = rb[j];
+        if (k + 1 < 4) tmem_ld_16x256b_x8(sb + 64 * (k + 1), rb);
+        load_exp(ra, k);
     }
-    tmem_st_16x128b_x16(sb, pk[0]);
-    tmem_st_16x128b_x16(sb + 64, pk[1]);
     tmem_wait_st();
     // (S_u + S_u^1) + (S_u^2 + S_u^3): commutativity gives every thread the
     // same bits.
@@ -402,7 +439,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&barS[b], 1);
             mbar_init(&barP[b], 128);
             mbar_init(&barO[b], 1);
-            mbar_init(&barF[b], 128);
+            mbar_init(&barF[b], kFoldThreads);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -615,8 +652,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else {
         // ====================================================== rows
-        // Softmax warps (4-7) and fold warps (2, 3, 8, 9) of lane quarter q
-        // serve the same 32 rows.
+        // Softmax warp 4 + q and fold warps of lane quarter q (two, one per
+        // half of the head dim) serve the same 32 rows.
         const bool is_softmax = warp >= 4 && warp < 8;
         const int q = warp & 3;
         bool valid, active;
@@ -670,6 +707,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         } else {
             // -------------------------------------------------- fold
+            // This warp merges columns col0 .. col0 + HW - 1 of its rows.
+            constexpr int HW = D / 2;
+            const int half = warp >= 10 ? 1 : 0;
+            const int col0 = half * HW;
 #if BI_INVARIANT
             // blocks after a sequence's first write every split's own partial
             const bool spill = p.decode && it.s0 > 0;
@@ -679,14 +720,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             const bool spill = false;
 #endif
             float m = -INFINITY, l = 0.0f;
-            float O[D];
+            float O[HW];
 #pragma unroll
-            for (int j = 0; j < D; ++j) O[j] = 0.0f;
+            for (int j = 0; j < HW; ++j) O[j] = 0.0f;
             bool ok = true;
             for (int s = it.s0; s < it.s1; ++s) {
                 const int b = (s - it.s0) & 1;
                 const uint32_t par = uint32_t((s - it.s0) >> 1) & 1u;
-                const uint32_t ob = lane_base + C::BUF_COLS * uint32_t(b) + C::O_OFF;
+                const uint32_t ob = lane_base + C::BUF_COLS * uint32_t(b) + C::O_OFF + col0;
                 const int k0 = s * kSplit;
                 // barP: (m_s, l_s) of this split are in shared memory;
                 // barO: O_s is in TMEM.
@@ -698,26 +739,28 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const float m_s = sML[(b * 128 + row_id) * 2 + 0];
                 const float l_s = sML[(b * 128 + row_id) * 2 + 1];
                 if (active) {
+                    // 32-column TMEM loads (HW / 32 per split)
+                    constexpr int NCH32 = HW / 32;
                     if (spill) {
                         // not the first block of this sequence: write the
                         // split's own partial for attn_combine
-                        float *rec = p.ws + ((out_row * p.max_splits) + s) * C::REC;
+                        float *rec = p.ws + ((out_row * p.max_splits) + s) * C::REC + 4 + col0;
 #pragma unroll 1
-                        for (int c = 0; c < D / 16; ++c) {
-                            uint32_t r0[16];
-                            tmem_ld16(ob + 16 * c, r0);
-                            tmem_wait_ld(r0);
+                        for (int c = 0; c < NCH32; ++c) {
+                            uint32_t r[32];
+                            tmem_ld32(ob + 32 * c, r);
+                            tmem_wait_ld(r);
                             if (valid) {
 #pragma unroll
-                                for (int j = 0; j < 4; ++j)
-                                    reinterpret_cast<float4 *>(rec + 4 + 16 * c)[j] = make_float4(
-                                        __uint_as_float(r0[4 * j]), __uint_as_float(r0[4 * j + 1]),
-                                        __uint_as_float(r0[4 * j + 2]), __uint_as_float(r0[4 * j + 3]));
+                                for (int j = 0; j < 8; ++j)
+                                    reinterpret_cast<float4 *>(rec + 32 * c)[j] = make_float4(
+                                        __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                        __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
                             }
                         }
-                        if (valid) {
-                            rec[0] = m_s;
-                            rec[1] = l_s;
+                        if (valid && half == 0) {
+                            rec[-4] = m_s;
+                            rec[-3] = l_s;
                         }
                     } else {
                         const bool first = (s == it.s0);
@@ -725,23 +768,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                         float mn, a, cc;
                         merge_scales(m, m_s, mn, a, cc);
 #pragma unroll
-                        for (int c = 0; c < D / 16; c += 2) {
-                            uint32_t r0[16], r1[16];
-                            tmem_ld16(ob + 16 * c, r0);
-                            tmem_ld16(ob + 16 * c + 16, r1);
-                            tmem_wait_ld(r0);
-                            tmem_wait_ld(r1);
+                        for (int c = 0; c < NCH32; ++c) {
+                            uint32_t r[32];
+                            tmem_ld32(ob + 32 * c, r);
+                            tmem_wait_ld(r);
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                const float o0 = __uint_as_float(r0[j]);
-                                const float o1 = __uint_as_float(r1[j]);
-                                if (first) {
-                                    O[16 * c + j] = o0;
-                                    O[16 * c + 16 + j] = o1;
-                                } else if (take) {
-                                    O[16 * c + j] = merge_val(O[16 * c + j], a, o0, cc);
-                                    O[16 * c + 16 + j] = merge_val(O[16 * c + 16 + j], a, o1, cc);
-                                }
+                            for (int j = 0; j < 32; ++j) {
+                                const float o = __uint_as_float(r[j]);
+                                if (first)
+                                    O[32 * c + j] = o;
+                                else if (take)
+                                    O[32 * c + j] = merge_val(O[32 * c + j], a, o, cc);
                             }
                         }
                         if (first) {
@@ -759,19 +796,21 @@ __global__ void __launch_bounds__(THREADS, 1)
 
             if (ok && active && valid && !spill) {
                 if (!p.decode || (it.s0 == 0 && it.s1 == it.n_splits)) {
-                    write_out<D>(O, l, m, static_cast<__nv_bfloat16 *>(p.o) + out_row * D,
-                                 p.lse ? p.lse + out_row : nullptr);
+                    write_out<HW>(O, l, m, static_cast<__nv_bfloat16 *>(p.o) + out_row * D + col0,
+                                  (p.lse && half == 0) ? p.lse + out_row : nullptr);
                 } else {
                     // a block of a sequence served by several: hand the
                     // merged state over its range (ending at split s1-1) to
                     // attn_combine (in the invariant build only the first
                     // block gets here; the others write every split)
                     float *rec = p.ws + ((out_row * p.max_splits) + (it.s1 - 1)) * C::REC;
-                    rec[0] = m;
-                    rec[1] = l;
+                    if (half == 0) {
+                        rec[0] = m;
+                        rec[1] = l;
+                    }
 #pragma unroll
-                    for (int j = 0; j < D / 4; ++j)
-                        reinterpret_cast<float4 *>(rec + 4)[j] =
+                    for (int j = 0; j < HW / 4; ++j)
+                        reinterpret_cast<float4 *>(rec + 4 + col0)[j] =
                             make_float4(O[4 * j], O[4 * j + 1], O[4 * j + 2], O[4 * j + 3]);
                 }
             }

@@ -59,7 +59,7 @@ __device__ __forceinline__ Unit unit_of(int u, int num_m, int k_splits, int kblo
 __device__ bool wait_drain(uint64_t *bar, uint32_t parity, uint64_t timeout_ns)
 {
     const uint64_t t0 = global_ns();
-    while (!mbar_try_wait(bar, parity))
+    while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs))
         if (global_ns() - t0 > timeout_ns) return false;
     return true;
 }
