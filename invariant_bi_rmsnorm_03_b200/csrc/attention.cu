@@ -13,9 +13,9 @@
 // 0..t are cut into splits of 256 keys aligned to key 0.  For each split s,
 // on its own:
 //   S      = Q K_s^T                    tcgen05, M=128 rows, N=256 keys, fp32
-//   x_j    = S_j * scale * log2(e), masked to -inf where key j > t
-//   m_s    = max_j x_j
-//   p_j    = 2^(x_j - m_s),  l_s = sum_j p_j   (a fixed order, tree8 below)
+//   c      = scale * log2(e); keys j > t are masked out
+//   m_s    = round(c * max_j S_j)        (= max_j round(c S_j): c > 0)
+//   p_j    = 2^fma(S_j, c, -m_s),  l_s = sum_j p_j   (a fixed order, tree8 below)
 //   O_s    = bf16(p) V_s                tcgen05, P read from tensor memory
 // and the partials are merged from split 0 upwards, always in that order:
 //   m' = max(m, m_s), a = 2^(m - m'), c = 2^(m_s - m')
@@ -231,34 +231,36 @@ __device__ __forceinline__ void chunk_max(const uint32_t (&r)[32], int kc, int t
     }
 }
 
-// p of 16 keys kc .. kc+15 (half `hf` of a 32-key chunk): packed bf16 P
-// written to TMEM at `pcol` (8 columns); tr[u] gets this half's part of
-// the chunk's class-u tree: (a_{2hf} + b_{2hf}) + (a_{2hf+1} + b_{2hf+1}).
-__device__ __forceinline__ void piece_exp(const uint32_t (&r)[16], int kc, int t, float cs,
-                                          float m_s, uint32_t pcol, float (&tr)[4])
+// p of the 32 keys kc .. kc+31, computed in place (r[j] becomes the bits of
+// p_j): packed bf16 P written to TMEM at `pcol` (16 columns), the class sums
+// S_u advanced by this chunk in the order of tree8.
+__device__ __forceinline__ void chunk_exp(uint32_t (&r)[32], int kc, int t, float cs, float m_s,
+                                          uint32_t pcol, float (&S)[4])
 {
-    float e[16];
-    if (kc + 15 <= t) {
+    if (kc + 31 <= t) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) e[j] = logit(__uint_as_float(r[j]), cs, m_s);
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(logit(__uint_as_float(r[j]), cs, m_s));
     } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            e[j] = (kc + j <= t) ? logit(__uint_as_float(r[j]), cs, m_s) : 0.0f;
+        for (int j = 0; j < 32; ++j)
+            r[j] = (kc + j <= t) ? __float_as_uint(logit(__uint_as_float(r[j]), cs, m_s)) : 0u;
     }
-    uint32_t pk[8];
+    uint32_t pk[16];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2(e[2 * j], e[2 * j + 1]);
-    tmem_st8(pcol, pk);
+    for (int j = 0; j < 16; ++j)
+        pk[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+    tmem_st16(pcol, pk);
+    auto e = [&](int j) { return __uint_as_float(r[j]); };
 #pragma unroll
     for (int u = 0; u < 4; ++u)
-        tr[u] = __fadd_rn(__fadd_rn(e[2 * u], e[2 * u + 1]), __fadd_rn(e[8 + 2 * u], e[9 + 2 * u]));
+        S[u] = __fadd_rn(S[u], tree8(e(2 * u), e(2 * u + 1), e(8 + 2 * u), e(9 + 2 * u),
+                                     e(16 + 2 * u), e(17 + 2 * u), e(24 + 2 * u), e(25 + 2 * u)));
 }
 
 // Softmax of one split, one row per thread (any row layout; used by
 // prefill and by decode with more than 8 query rows per lane quarter).
-// S is read from TMEM columns sb .. sb+255 in two passes of 16-column
-// loads, the next load in flight while a piece is processed; P (bf16 pairs)
+// S is read from TMEM columns sb .. sb+255 in two passes of 32-column
+// loads, the next load in flight while a chunk is processed; P (bf16 pairs)
 // is written over columns sb .. sb+127 as the second pass goes (each store
 // lands on columns this thread has already read).  Returns m_s (scaled,
 // log2 units) and l_s.  (P V cannot start before the whole pass is done: it
@@ -266,7 +268,7 @@ __device__ __forceinline__ void piece_exp(const uint32_t (&r)[16], int kc, int t
 __device__ __forceinline__ void softmax_rows(uint32_t sb, int k0, int t, float cs, float &m_s,
                                              float &l_s)
 {
-    constexpr int NP = kSplit / 16;  // 16-key pieces
+    constexpr int NC = kSplit / 32;  // 32-key chunks
     // pass 1: maximum of the raw logits over the visible keys.  For c > 0,
     // x -> round(x * c) is monotonic, so max_j round(S_j c) = round(max_j S_j * c).
     // (A maximum is exact in any order; eight accumulators break the chain.)
@@ -281,12 +283,12 @@ __device__ __forceinline__ void softmax_rows(uint32_t sb, int k0, int t, float c
         uint32_t ra[32], rb[32];
         tmem_ld32(sb, ra);
 #pragma unroll 1
-        for (int c = 0; c < NP / 2; c += 2) {
+        for (int c = 0; c < NC; c += 2) {
             tmem_wait_ld(ra);
             tmem_ld32(sb + 32 * (c + 1), rb);
             chunk_max(ra, k0 + 32 * c, t, mx);
             tmem_wait_ld(rb);
-            if (c + 2 < NP / 2) tmem_ld32(sb + 32 * (c + 2), ra);
+            if (c + 2 < NC) tmem_ld32(sb + 32 * (c + 2), ra);
             chunk_max(rb, k0 + 32 * (c + 1), t, mx);
         }
     }
@@ -294,21 +296,18 @@ __device__ __forceinline__ void softmax_rows(uint32_t sb, int k0, int t, float c
                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
     m_s = __fmul_rn(mraw, cs);
     // pass 2: p = 2^(S c - m_s), masked keys 0; P into TMEM; the sum in the
-    // order of tree8 (a chunk's two halves are its pieces h and h + 1).
+    // order of tree8.  32-key chunks, the next chunk's load in flight.
     float S[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    uint32_t ra[16], rb[16];
-    tmem_ld16(sb, ra);
+    uint32_t ra[32], rb[32];
+    tmem_ld32(sb, ra);
 #pragma unroll 1
-    for (int h = 0; h < NP; h += 2) {
-        float t0[4], t1[4];
+    for (int c = 0; c < NC; c += 2) {
         tmem_wait_ld(ra);
-        tmem_ld16(sb + 16 * (h + 1), rb);
-        piece_exp(ra, k0 + 16 * h, t, cs, m_s, sb + 8 * h, t0);
+        tmem_ld32(sb + 32 * (c + 1), rb);
+        chunk_exp(ra, k0 + 32 * c, t, cs, m_s, sb + 16 * c, S);
         tmem_wait_ld(rb);
-        if (h + 2 < NP) tmem_ld16(sb + 16 * (h + 2), ra);
-        piece_exp(rb, k0 + 16 * (h + 1), t, cs, m_s, sb + 8 * (h + 1), t1);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) S[u] = __fadd_rn(S[u], __fadd_rn(t0[u], t1[u]));
+        if (c + 2 < NC) tmem_ld32(sb + 32 * (c + 2), ra);
+        chunk_exp(rb, k0 + 32 * (c + 1), t, cs, m_s, sb + 16 * (c + 1), S);
     }
     tmem_wait_st();
     l_s = __fadd_rn(__fadd_rn(S[0], S[1]), __fadd_rn(S[2], S[3]));
