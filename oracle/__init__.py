@@ -60,6 +60,8 @@ class Oracle:
         lib.oracle_swiglu.argtypes = [P, i64, i64, P]
         lib.oracle_add_rmsnorm.argtypes = [P, P, P, i64, i64, f64, P, P]
         lib.oracle_argmax.argtypes = [P, i64, i64, P]
+        lib.oracle_philox4x32_10.argtypes = [P, P, P]
+        lib.oracle_sample.argtypes = [P, i64, i64, P, P, P, P, P, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
@@ -175,6 +177,36 @@ class Oracle:
         self.lib.oracle_argmax(_p(logits), T, V, _p(out))
         return out
 
+    # ---------------------------------------------------------- sampling
+
+    def philox4x32_10(self, ctr, key) -> np.ndarray:
+        """Philox4x32-10 of a 4-word counter and a 2-word key -> 4 words."""
+        c = np.ascontiguousarray(ctr, dtype=np.uint32)
+        k = np.ascontiguousarray(key, dtype=np.uint32)
+        assert c.shape == (4,) and k.shape == (2,)
+        out = np.empty(4, dtype=np.uint32)
+        self.lib.oracle_philox4x32_10(_p(c), _p(k), _p(out))
+        return out
+
+    def sample(self, logits, temperature, top_p, seed, offset, details: bool = False):
+        """One token per row of fp32 logits [T, V] (temperature 0: greedy;
+        else softmax at that temperature, nucleus top_p, the draw from
+        Philox4x32-10 keyed by the row's seed at counter ``offset``).
+        With ``details``, also (r, zk): the draw and the kept mass as
+        fractions of the total weight."""
+        logits = np.ascontiguousarray(logits, dtype=np.float32)
+        T, V = logits.shape
+        temp = np.ascontiguousarray(np.broadcast_to(temperature, (T,)), dtype=np.float32)
+        tp = np.ascontiguousarray(np.broadcast_to(top_p, (T,)), dtype=np.float32)
+        sd = np.ascontiguousarray(np.broadcast_to(seed, (T,)), dtype=np.uint64)
+        off = np.ascontiguousarray(np.broadcast_to(offset, (T,)), dtype=np.uint64)
+        out = np.empty((T,), dtype=np.int32)
+        r = np.empty((T,), dtype=np.float64)
+        zk = np.empty((T,), dtype=np.float64)
+        self.lib.oracle_sample(_p(logits), T, V, _p(temp), _p(tp), _p(sd), _p(off), _p(out),
+                               _p(r), _p(zk))
+        return (out, r, zk) if details else out
+
 
 def default() -> Oracle:
     global _lib
@@ -227,6 +259,14 @@ def add_rmsnorm(x, delta, w, eps: float):
 
 def argmax(logits) -> np.ndarray:
     return default().argmax(logits)
+
+
+def philox4x32_10(ctr, key) -> np.ndarray:
+    return default().philox4x32_10(ctr, key)
+
+
+def sample(logits, temperature, top_p, seed, offset, details: bool = False):
+    return default().sample(logits, temperature, top_p, seed, offset, details)
 
 
 def decode_rows(q, seq_lens, heads=None):

@@ -31,6 +31,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
@@ -303,5 +304,132 @@ void oracle_argmax(const float *logits, int64_t T, int64_t V, int32_t *out)
         for (int64_t j = 1; j < V; ++j)
             if (row[j] > row[best]) best = j;
         out[t] = (int32_t)best;
+    }
+}
+
+/* ------------------------------------------------------------------------
+ * Sampling at temperature > 0 with nucleus (top-p) truncation, each request
+ * drawing from its own counter-based random stream, so that a request's
+ * token never depends on the other requests of the batch.  The reports tie
+ * bitwise-identical sampling to on-policy reinforcement learning (xitu-tech
+ * news, "强化学习的突破"; neican.ai insight, "未来发展路径预测") and set the
+ * random seed aside as the cause of run-to-run differences (vpshk.cn,
+ * "AI随机性的根源探析"); they describe no sampler.  Reading taken: the random
+ * draw belongs to the request -- its seed and its position -- and every
+ * reduction over the vocabulary has a fixed order.
+ *
+ * Generator: Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random
+ * numbers: as easy as 1, 2, 3", SC 2011): a 128-bit counter, a 64-bit key,
+ * ten rounds of two 32x32->64 multiplications with the key bumped by the
+ * Weyl constants between rounds.
+ * ------------------------------------------------------------------------ */
+
+static void philox_round(uint32_t c[4], const uint32_t k[2])
+{
+    uint64_t p0 = (uint64_t)0xD2511F53u * c[0];
+    uint64_t p1 = (uint64_t)0xCD9E8D57u * c[2];
+    uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+    uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+    uint32_t n0 = hi1 ^ c[1] ^ k[0], n2 = hi0 ^ c[3] ^ k[1];
+    c[0] = n0;
+    c[1] = lo1;
+    c[2] = n2;
+    c[3] = lo0;
+}
+
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t c[4] = {ctr[0], ctr[1], ctr[2], ctr[3]};
+    uint32_t k[2] = {key[0], key[1]};
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k[0] += 0x9E3779B9u;
+            k[1] += 0xBB67AE85u;
+        }
+        philox_round(c, k);
+    }
+    for (int i = 0; i < 4; ++i) out[i] = c[i];
+}
+
+static int oracle_cmp_desc(const void *a, const void *b)
+{
+    double x = *(const double *)a, y = *(const double *)b;
+    return (x < y) - (x > y);
+}
+
+/*
+ * One token per row of logits [T, V] (fp32, the precision the lm_head
+ * produces them in):
+ *   temperature 0: the greedy choice (lowest index of the maximum);
+ *   otherwise, with z_i = logits_i / temperature and w_i = exp(z_i - max z):
+ *     kept set K = { i : w_i >= tau }, tau the largest w-value such that the
+ *       weights >= tau hold at least top_p of the total weight (ties at tau
+ *       are all kept);  W_K = sum over K of w_i;
+ *     u = the first Philox4x32-10 output word for key (seed lo, seed hi) and
+ *       counter (offset lo, offset hi, 0, 0), u = (word >> 8) * 2^-24;
+ *     the token is the first i of K, in index order, at which the running
+ *       sum of w over K exceeds u * W_K.
+ * r_out (may be NULL) receives u * W_K / W (the target as a fraction of the
+ * total weight), zk_out (may be NULL) W_K / W.
+ */
+void oracle_sample(const float *logits, int64_t T, int64_t V, const float *temperature,
+                   const float *top_p, const uint64_t *seed, const uint64_t *offset, int32_t *out,
+                   double *r_out, double *zk_out)
+{
+    int64_t t;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (t = 0; t < T; ++t) {
+        const float *row = logits + t * V;
+        int64_t best = 0;
+        for (int64_t j = 1; j < V; ++j)
+            if (row[best] < row[j]) best = j;
+        if (!(temperature[t] > 0.0f)) {
+            out[t] = (int32_t)best;
+            if (r_out) r_out[t] = 0.0;
+            if (zk_out) zk_out[t] = 0.0;
+            continue;
+        }
+        double *w = (double *)malloc((size_t)V * sizeof(double));
+        double *sorted = (double *)malloc((size_t)V * sizeof(double));
+        double mx = (double)row[best] / (double)temperature[t];
+        double total = 0.0;
+        for (int64_t j = 0; j < V; ++j) {
+            w[j] = exp((double)row[j] / (double)temperature[t] - mx);
+            total += w[j];
+            sorted[j] = w[j];
+        }
+        qsort(sorted, (size_t)V, sizeof(double), oracle_cmp_desc);  /* descending */
+        double need = (double)top_p[t] * total, acc = 0.0, tau = sorted[V - 1];
+        for (int64_t j = 0; j < V; ++j) {
+            acc += sorted[j];
+            if (acc >= need) {
+                tau = sorted[j];
+                break;
+            }
+        }
+        double zk = 0.0;
+        for (int64_t j = 0; j < V; ++j)
+            if (w[j] >= tau) zk += w[j];
+        uint32_t ctr[4] = {(uint32_t)offset[t], (uint32_t)(offset[t] >> 32), 0u, 0u};
+        uint32_t key[2] = {(uint32_t)seed[t], (uint32_t)(seed[t] >> 32)};
+        uint32_t rnd[4];
+        oracle_philox4x32_10(ctr, key, rnd);
+        double u = (double)(rnd[0] >> 8) * (1.0 / 16777216.0);
+        double target = u * zk, run = 0.0;
+        int64_t tok = -1, last = -1;
+        for (int64_t j = 0; j < V; ++j) {
+            if (w[j] < tau) continue;
+            last = j;
+            run += w[j];
+            if (run > target) {
+                tok = j;
+                break;
+            }
+        }
+        out[t] = (int32_t)(tok >= 0 ? tok : last);
+        if (r_out) r_out[t] = target / total;
+        if (zk_out) zk_out[t] = zk / total;
+        free(w);
+        free(sorted);
     }
 }

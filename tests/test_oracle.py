@@ -451,3 +451,83 @@ def test_argmax_matches_numpy_first_occurrence(oracle):
     g = rng(48)
     logits = g.integers(-3, 4, size=(50, 1000)).astype(np.float32)  # many ties
     assert np.array_equal(oracle.argmax(logits), np.argmax(logits, axis=1))
+
+
+# ---------------------------------------------------------------- sampling
+
+
+def test_philox_known_answer_vectors(oracle):
+    # Known-answer vectors published with the generator (Salmon et al., SC 2011;
+    # the Random123 distribution's test vectors for philox4x32 with 10 rounds).
+    kat = [((0, 0, 0, 0), (0, 0), (0x6627E8D5, 0xE169C58D, 0xBC57AC4C, 0x9B00DBD8)),
+           ((0xFFFFFFFF,) * 4, (0xFFFFFFFF,) * 2, (0x408F276D, 0x41C83B0E, 0xA20BC7C6, 0x6D5451FD)),
+           ((0x243F6A88, 0x85A308D3, 0x13198A2E, 0x03707344), (0xA4093822, 0x299F31D0),
+            (0xD16CFE09, 0x94FDCCEB, 0x5001E420, 0x24126EA1))]
+    for ctr, key, want in kat:
+        assert tuple(int(x) for x in oracle.philox4x32_10(ctr, key)) == want
+
+
+def _u(oracle, seed, offset):
+    w = oracle.philox4x32_10((offset & 0xFFFFFFFF, offset >> 32, 0, 0),
+                             (seed & 0xFFFFFFFF, seed >> 32))
+    return (int(w[0]) >> 8) / 16777216.0
+
+
+def test_sample_temperature_zero_is_greedy(oracle):
+    g = rng(140)
+    logits = g.integers(-3, 4, size=(30, 500)).astype(np.float32)
+    got = oracle.sample(logits, 0.0, 0.9, np.arange(30, dtype=np.uint64), 7)
+    assert np.array_equal(got, oracle.argmax(logits))
+
+
+def test_sample_uniform_logits_closed_form(oracle):
+    # four equal weights, everything kept: token = floor(4 u)
+    logits = np.zeros((1, 4), dtype=np.float32)
+    for seed in range(200):
+        tok = oracle.sample(logits, 1.0, 1.0, seed, 3 * seed + 1)[0]
+        assert tok == int(4 * _u(oracle, seed, 3 * seed + 1)), seed
+
+
+def test_sample_dominant_logit_and_tiny_top_p(oracle):
+    g = rng(141)
+    logits = g.standard_normal((50, 300)).astype(np.float32)
+    logits[np.arange(50), g.integers(0, 300, size=50)] += 60.0
+    seeds = np.arange(50, dtype=np.uint64) * 7919
+    assert np.array_equal(oracle.sample(logits, 1.0, 1.0, seeds, 5), oracle.argmax(logits))
+    mild = g.standard_normal((50, 300)).astype(np.float32)
+    assert np.array_equal(oracle.sample(mild, 0.8, 1e-6, seeds, 5), oracle.argmax(mild))
+
+
+def test_sample_nucleus_drops_the_tail(oracle):
+    # weights 0.5, 0.3, 0.2 at top_p 0.6: keep {0, 1}; token 2 never drawn,
+    # tokens 0 and 1 in proportion 5 : 3.
+    logits = np.log(np.array([[0.5, 0.3, 0.2]], dtype=np.float64)).astype(np.float32)
+    n = 4000
+    toks = np.array([oracle.sample(logits, 1.0, 0.6, s, 11)[0] for s in range(n)])
+    assert not (toks == 2).any()
+    f0 = (toks == 0).mean()
+    assert abs(f0 - 0.625) < 4 * np.sqrt(0.625 * 0.375 / n)
+
+
+def test_sample_ties_at_the_threshold_are_all_kept(oracle):
+    # weights 1, 1, 1, 0.5 at top_p 0.5: the threshold is 1 and all three
+    # tied weights stay; 0.5 never drawn; the three equally often.
+    logits = np.log(np.array([[1.0, 1.0, 1.0, 0.5]])).astype(np.float32)
+    n = 3000
+    toks = np.array([oracle.sample(logits, 1.0, 0.5, s, 0)[0] for s in range(n)])
+    assert not (toks == 3).any()
+    for k in range(3):
+        assert abs((toks == k).mean() - 1 / 3) < 4 * np.sqrt(2 / 9 / n)
+
+
+def test_sample_frequencies_follow_the_softmax(oracle):
+    logits = np.array([[1.0, 0.0, -1.0, 2.0, 0.5]], dtype=np.float32)
+    T = 0.7
+    p = np.exp(logits[0].astype(np.float64) / T)
+    p /= p.sum()
+    n = 20000
+    rows = np.repeat(logits, n, axis=0)
+    toks = oracle.sample(rows, T, 1.0, np.arange(n, dtype=np.uint64), 99)
+    for k in range(5):
+        f = (toks == k).mean()
+        assert abs(f - p[k]) < 4.5 * np.sqrt(p[k] * (1 - p[k]) / n), (k, f, p[k])

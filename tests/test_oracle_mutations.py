@@ -66,6 +66,19 @@ MUTATIONS = [
      [pins.test_add_rmsnorm_constant_sum_closed_form, pins.test_add_rmsnorm_matches_torch_fp64]),
     ("add_rmsnorm_eps_outside_root", "sqrt(mean_sq + eps)", "(sqrt(mean_sq) + eps)",
      [pins.test_add_rmsnorm_constant_sum_closed_form, pins.test_add_rmsnorm_matches_torch_fp64]),
+    ("philox_hi_lo_swapped", "c[1] = lo1;", "c[1] = hi1;",
+     [pins.test_philox_known_answer_vectors]),
+    ("philox_key_not_bumped", "k[0] += 0x9E3779B9u;", "k[0] += 0u;",
+     [pins.test_philox_known_answer_vectors]),
+    ("sample_temperature_multiplies", "w[j] = exp((double)row[j] / (double)temperature[t] - mx);",
+     "w[j] = exp((double)row[j] * (double)temperature[t] - mx);",
+     [pins.test_sample_frequencies_follow_the_softmax]),
+    ("sample_ties_dropped", "if (w[j] >= tau) zk += w[j];", "if (w[j] > tau) zk += w[j];",
+     [pins.test_sample_ties_at_the_threshold_are_all_kept]),
+    ("sample_wrong_word", "double u = (double)(rnd[0] >> 8)", "double u = (double)(rnd[1] >> 8)",
+     [pins.test_sample_uniform_logits_closed_form]),
+    ("sample_nucleus_ignored", "double need = (double)top_p[t] * total", "double need = total",
+     [pins.test_sample_nucleus_drops_the_tail, pins.test_sample_dominant_logit_and_tiny_top_p]),
     ("argmax_ties_take_highest_index", "if (row[j] > row[best]) best = j;",
      "if (row[j] >= row[best]) best = j;",
      [pins.test_argmax_ties_take_the_lowest_index, pins.test_argmax_matches_numpy_first_occurrence]),
