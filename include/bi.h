@@ -324,6 +324,35 @@ bi_status bi_swiglu(const void *gu, void *out, int64_t T, int64_t F, void *strea
  */
 bi_status bi_argmax(const float *logits, int64_t T, int64_t V, int32_t *out, void *stream);
 
+/*
+ * bi_sample -- one token per row, the random draw belonging to the request,
+ * so that a request's token never depends on the rest of the batch.  The
+ * reports tie bitwise-identical sampling to on-policy reinforcement learning
+ * (xitu-tech news, "强化学习的突破"; neican.ai insight, "未来发展路径预测") and
+ * set the random seed aside as the cause of run-to-run differences
+ * (vpshk.cn, "AI随机性的根源探析"); they describe no sampler, so this one is
+ * the plainest reading.
+ *
+ *   temperature[t] <= 0: the greedy choice (as bi_argmax).  Otherwise, with
+ *   z_j = logits[t, j] / temperature[t] and w_j = e^(z_j - max z):
+ *     kept set K = { j : w_j >= tau }, tau the largest value such that the
+ *       weights >= tau hold at least top_p[t] of the total (ties at tau are
+ *       all kept; top_p >= 1 keeps everything);
+ *     u = (x >> 8) * 2^-24, x the first output word of Philox4x32-10
+ *       (Salmon et al., SC 2011) with key (seed lo, seed hi) and counter
+ *       (offset lo, offset hi, 0, 0) -- e.g. seed per request, offset = the
+ *       token's position;
+ *     the token is the first j of K, in index order, at which the running
+ *       sum of w over K exceeds u * sum_K w.
+ *   Every sum has an order fixed by V alone (fp32).
+ *   logits : device, fp32 [T, V], 1 <= V <= 53248;  temperature, top_p :
+ *   device, fp32 [T];  seed, offset : device, uint64 [T];  out : device,
+ *   int32 [T].  T == 0 is a no-op.
+ */
+bi_status bi_sample(const float *logits, int64_t T, int64_t V, const float *temperature,
+                    const float *top_p, const uint64_t *seed, const uint64_t *offset, int32_t *out,
+                    void *stream);
+
 const char *bi_status_string(bi_status s);
 
 /* 1 for the batch-invariant build, 0 for the variant-off build (split-K

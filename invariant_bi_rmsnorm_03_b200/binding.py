@@ -109,7 +109,7 @@ class Library:
                "bi_attention_prefill", "bi_attention_prefill_workspace_bytes",
                "bi_status_string", "bi_build_invariant", "bi_device_status",
                "bi_debug_bounded_wait", "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write",
-               "bi_swiglu", "bi_argmax")
+               "bi_swiglu", "bi_argmax", "bi_sample")
 
     def __init__(self, path: str):
         if not os.path.exists(path):
@@ -143,10 +143,11 @@ class Library:
         L.bi_rope_kv_write.argtypes = [kvp, P, P, P, P, i64, i32, f32, P]
         L.bi_swiglu.argtypes = [P, P, i64, i64, P]
         L.bi_argmax.argtypes = [P, i64, i64, P, P]
+        L.bi_sample.argtypes = [P, i64, i64, P, P, P, P, P, P]
         for name in ("bi_rmsnorm", "bi_matmul", "bi_kv_write", "bi_attention_decode",
                      "bi_attention_prefill", "bi_device_status", "bi_debug_bounded_wait",
                      "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write", "bi_swiglu",
-                     "bi_argmax"):
+                     "bi_argmax", "bi_sample"):
             getattr(L, name).restype = st
         self.lib = L
 
@@ -289,6 +290,33 @@ class Library:
         _need(out, "out", torch.int32, (T,))
         self._check("bi_argmax", self.lib.bi_argmax(_ptr(logits), T, V, _ptr(out),
                                                     _stream(stream)))
+        return out
+
+    def bi_sample(self, logits: torch.Tensor, temperature, top_p, seed, offset, out=None,
+                  stream=None) -> torch.Tensor:
+        """One token per row of fp32 logits [T, V]; temperature, top_p (fp32),
+        seed and offset (int64/uint64 bit patterns) are per-row tensors [T]
+        on the device, or Python scalars broadcast to every row."""
+        _need(logits, "logits", torch.float32)
+        T, V = logits.shape
+        dev = logits.device
+
+        def col(x, dtype, name):
+            if not isinstance(x, torch.Tensor):
+                x = torch.full((T,), x, dtype=dtype, device=dev)
+            _need(x, name, dtype, (T,))
+            return x
+
+        temperature = col(temperature, torch.float32, "temperature")
+        top_p = col(top_p, torch.float32, "top_p")
+        seed = col(seed, torch.int64, "seed")        # uint64 bits
+        offset = col(offset, torch.int64, "offset")
+        if out is None:
+            out = torch.empty((T,), dtype=torch.int32, device=dev)
+        _need(out, "out", torch.int32, (T,))
+        self._check("bi_sample", self.lib.bi_sample(
+            _ptr(logits), T, V, _ptr(temperature), _ptr(top_p), _ptr(seed), _ptr(offset), _ptr(out),
+            _stream(stream)))
         return out
 
     # ------------------------------------------------------------ attention

@@ -263,6 +263,20 @@ bi_status bi_argmax(const float *logits, int64_t T, int64_t V, int32_t *out, voi
     return from_cuda(bi::launch_argmax(logits, T, V, out, d->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
+bi_status bi_sample(const float *logits, int64_t T, int64_t V, const float *temperature,
+                    const float *top_p, const uint64_t *seed, const uint64_t *offset, int32_t *out,
+                    void *stream)
+{
+    if (T < 0 || V < 1 || V > bi::kMaxSampleVocab) return BI_ERR_INVALID;
+    if (T == 0) return BI_OK;
+    if (!logits || !temperature || !top_p || !seed || !offset || !out) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_sample(logits, T, V, temperature, top_p, seed, offset, out,
+                                       d->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
 static bool attn_common_ok(const bi_paged_kv *kv, int32_t Hq)
 {
     if (!kv_ok(kv)) return false;

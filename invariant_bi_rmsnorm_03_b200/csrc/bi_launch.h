@@ -82,6 +82,11 @@ cudaError_t launch_swiglu(const void *gu, void *out, int64_t T, int64_t F, int n
                           cudaStream_t s);
 cudaError_t launch_argmax(const float *logits, int64_t T, int64_t V, int32_t *out, int num_sms,
                           cudaStream_t s);
+constexpr int64_t kMaxSampleVocab = 53248;  // the row's weights live in shared memory
+size_t sample_smem_bytes(int64_t V);
+cudaError_t launch_sample(const float *logits, int64_t T, int64_t V, const float *temperature,
+                          const float *top_p, const uint64_t *seed, const uint64_t *offset,
+                          int32_t *out, int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- debug
 cudaError_t launch_bounded_wait_probe(unsigned *status, uint64_t timeout_ns, cudaStream_t s);

@@ -221,6 +221,186 @@ argmax_kernel(const float4 *__restrict__ logits, int64_t T, int64_t V, int32_t *
     }
 }
 
+// ---------------------------------------------------------------- sampling
+// One block per row (grid-stride), the row's weights cached in shared
+// memory.  Every reduction has an order fixed by V and the block size alone:
+// thread i takes elements i, i + T, ... in turn, then a warp xor-butterfly
+// (commutative, so every lane gets the same bits), then warps 0..W-1 in
+// order.  The row's draw comes from Philox4x32-10 (Salmon et al., SC 2011)
+// keyed by the request's seed at a counter made of its offset.
+constexpr int kSampleThreads = 512;
+
+struct Philox {
+    uint32_t c[4];
+    uint32_t k[2];
+};
+
+__device__ __forceinline__ uint32_t philox_word0(uint64_t seed, uint64_t offset)
+{
+    uint32_t c0 = uint32_t(offset), c1 = uint32_t(offset >> 32), c2 = 0u, c3 = 0u;
+    uint32_t k0 = uint32_t(seed), k1 = uint32_t(seed >> 32);
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
+        const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
+        const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+        c0 = n0;
+        c1 = lo1;
+        c2 = n2;
+        c3 = lo0;
+        k0 += 0x9E3779B9u;  // the key for the next round
+        k1 += 0xBB67AE85u;
+    }
+    return c0;
+}
+
+// Sum over the block of one value per thread: butterfly in each warp, then
+// the warp sums in order.  `red` holds kSampleThreads / 32 floats.
+__device__ __forceinline__ float block_sum(float v, float *red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();  // red[] free
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float tot = 0.0f;
+    for (int i = 0; i < int(blockDim.x >> 5); ++i) tot = __fadd_rn(tot, red[i]);
+    return tot;
+}
+
+__device__ __forceinline__ float block_max(float v, float *red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float m = red[0];
+    for (int i = 1; i < int(blockDim.x >> 5); ++i) m = fmaxf(m, red[i]);
+    return m;
+}
+
+__device__ __forceinline__ int block_min_int(int v, int *red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    int m = red[0];
+    for (int i = 1; i < int(blockDim.x >> 5); ++i) m = min(m, red[i]);
+    return m;
+}
+
+__global__ void __launch_bounds__(kSampleThreads)
+sample_kernel(const float *__restrict__ logits, int64_t T, int V,
+              const float *__restrict__ temperature, const float *__restrict__ top_p,
+              const uint64_t *__restrict__ seed, const uint64_t *__restrict__ offset,
+              int32_t *__restrict__ out)
+{
+    extern __shared__ float w[];                 // [V] weights of the row
+    __shared__ float redf[kSampleThreads / 32];
+    __shared__ int redi[kSampleThreads / 32];
+    const int tid = threadIdx.x, nt = blockDim.x;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        const float *row = logits + t * int64_t(V);
+        const float temp = temperature[t];
+        if (!(temp > 0.0f)) {
+            // greedy: the largest logit, lowest index on ties
+            float bv = -INFINITY;
+            int bi = INT32_MAX;
+            for (int j = tid; j < V; j += nt) {
+                const float x = row[j];
+                if (x > bv || (x == bv && j < bi)) {
+                    bv = x;
+                    bi = j;
+                }
+            }
+            const float m = block_max(bv, redf);
+            const int idx = block_min_int(bv == m ? bi : INT32_MAX, redi);
+            if (tid == 0) out[t] = idx == INT32_MAX ? 0 : idx;
+            continue;
+        }
+        // z_j = logit_j / temperature; weights w_j = e^(z_j - max z)
+        float mx = -INFINITY;
+        for (int j = tid; j < V; j += nt) mx = fmaxf(mx, __fdiv_rn(row[j], temp));
+        mx = block_max(mx, redf);
+        float part = 0.0f;
+        for (int j = tid; j < V; j += nt) {
+            const float e = expf(__fsub_rn(__fdiv_rn(row[j], temp), mx));
+            w[j] = e;
+            part = __fadd_rn(part, e);
+        }
+        const float total = block_sum(part, redf);
+        // nucleus threshold: the largest tau with sum_{w >= tau} w >= top_p * total,
+        // found by bisection on the bit pattern (positive floats order like
+        // their bits); each probe is a sum in the fixed order above.
+        uint32_t lo = 0u, hi = 0x3F800001u;  // S(0) = total, S(> 1) = 0
+        float zk = total;
+        const float tp = top_p[t];
+        if (tp < 1.0f) {
+            const float need = __fmul_rn(tp, total);
+            while (hi - lo > 1u) {
+                const uint32_t mid = lo + ((hi - lo) >> 1);
+                const float tau = __uint_as_float(mid);
+                float ps = 0.0f;
+                for (int j = tid; j < V; j += nt)
+                    if (w[j] >= tau) ps = __fadd_rn(ps, w[j]);
+                const float S = block_sum(ps, redf);
+                if (S >= need) {
+                    lo = mid;
+                    zk = S;
+                } else {
+                    hi = mid;
+                }
+            }
+            if (lo == 0u) zk = total;
+        }
+        const float tau = __uint_as_float(lo);
+        // the draw and the target mass
+        const float u = float(philox_word0(seed[t], offset[t]) >> 8) * (1.0f / 16777216.0f);
+        const float target = __fmul_rn(u, zk);
+        // walk the kept weights in index order: thread i owns the contiguous
+        // range [i C, (i+1) C); range sums, an exclusive scan of them over the
+        // threads (a fixed tree), then each thread walks its range.
+        const int C = (V + nt - 1) / nt;
+        const int j0 = tid * C, j1 = min(V, j0 + C);
+        float rs = 0.0f;
+        for (int j = j0; j < j1; ++j)
+            if (w[j] >= tau) rs = __fadd_rn(rs, w[j]);
+        float inc = rs;
+        const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc = __fadd_rn(inc, y);
+        }
+        __syncthreads();
+        if (lane == 31) redf[warp] = inc;
+        __syncthreads();
+        float before = 0.0f;  // sum of the warps before this one, in order
+        for (int i = 0; i < warp; ++i) before = __fadd_rn(before, redf[i]);
+        float run = __fadd_rn(before, __fsub_rn(inc, rs));  // exclusive prefix
+        int cand = INT32_MAX, last = -1;
+        for (int j = j0; j < j1; ++j) {
+            if (!(w[j] >= tau)) continue;
+            last = j;
+            run = __fadd_rn(run, w[j]);
+            if (run > target) {
+                cand = j;
+                break;
+            }
+        }
+        int tok = block_min_int(cand, redi);
+        if (tok == INT32_MAX) tok = -block_min_int(-last, redi);  // past the end: the last kept
+        if (tid == 0) out[t] = tok < 0 ? 0 : tok;
+        __syncthreads();  // w[] and the scratch are reused by the next row
+    }
+}
+
 unsigned grid_for(int64_t items, int threads, int num_sms)
 {
     const int64_t blocks = (items + threads - 1) / threads;
@@ -229,6 +409,29 @@ unsigned grid_for(int64_t items, int threads, int num_sms)
 }
 
 }  // namespace
+
+size_t sample_smem_bytes(int64_t V) { return size_t(V) * sizeof(float); }
+
+cudaError_t launch_sample(const float *logits, int64_t T, int64_t V, const float *temperature,
+                          const float *top_p, const uint64_t *seed, const uint64_t *offset,
+                          int32_t *out, int num_sms, cudaStream_t s)
+{
+    const size_t smem = sample_smem_bytes(V);
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(kMaxSampleVocab * sizeof(float)));
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    const int64_t cap = int64_t(num_sms);
+    const unsigned grid = static_cast<unsigned>(T < cap ? T : cap);
+    sample_kernel<<<grid, kSampleThreads, smem, s>>>(logits, T, int(V), temperature, top_p, seed,
+                                                     offset, out);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_embedding(const void *table, int64_t V, int64_t H, const int32_t *ids,
                              void *out, int64_t T, unsigned *status, int num_sms, cudaStream_t s)

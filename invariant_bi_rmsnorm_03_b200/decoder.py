@@ -9,7 +9,9 @@ layer beyond RMSNorm, matmul and attention, so the model here is the plain
 pre-norm transformer (token embedding; per layer RMSNorm -> stacked q/k/v
 matmul -> rotary embedding + KV-cache write -> paged attention -> output
 matmul -> residual + RMSNorm -> stacked gate/up matmul -> SwiGLU -> down
-matmul -> residual; final RMSNorm; lm_head matmul in fp32; greedy argmax).
+matmul -> residual; final RMSNorm; lm_head matmul in fp32; the next token by
+bi_sample: greedy at temperature 0, else nucleus sampling from the request's
+own counter-based random stream).
 
 Every arithmetic step runs in the library's CUDA kernels through the C ABI;
 this module only plans the batch on the host (which request contributes
@@ -69,6 +71,9 @@ class Request:
     max_new: int                  # tokens to generate
     arrival: int = 0              # first step at which it may be admitted
     tag: str = ""
+    temperature: float = 0.0      # 0: greedy
+    top_p: float = 1.0
+    seed: int = 0                 # the request's own random stream
     pages: list = field(default_factory=list)
     done_prompt: int = 0          # prompt tokens already in the cache
     out: list = field(default_factory=list)
@@ -96,6 +101,10 @@ class StepPlan:
     ctx: np.ndarray          # int32 [B_pre]
     sample_rows: np.ndarray  # int32 rows whose next token is taken
     sample_reqs: list        # the request of each sampled row
+    temperature: np.ndarray  # float32 per sampled row
+    top_p: np.ndarray        # float32 per sampled row
+    seed: np.ndarray         # uint64 per sampled row
+    offset: np.ndarray       # uint64 per sampled row: the position of the token drawn
     block_table: np.ndarray  # int32 [B_dec + B_pre, max_pages]
 
 
@@ -186,10 +195,16 @@ class Scheduler:
         bt = np.full((len(rows), max_pages), -1, dtype=np.int32)
         for i, r in enumerate(rows):
             bt[i, :len(r.pages)] = r.pages
+        # the token drawn for request r sits at position len(prompt) + len(out)
         return StepPlan(np.array(tokens, np.int32), np.array(pos, np.int32),
                         np.array(slots, np.int64), dec, np.array(dec_lens, np.int32), pre,
                         np.array(cu, np.int32), np.array(ctx, np.int32),
-                        np.array(sample_rows, np.int32), sample_reqs, bt)
+                        np.array(sample_rows, np.int32), sample_reqs,
+                        np.array([r.temperature for r in sample_reqs], np.float32),
+                        np.array([r.top_p for r in sample_reqs], np.float32),
+                        np.array([r.seed for r in sample_reqs], np.uint64),
+                        np.array([len(r.prompt) + len(r.out) for r in sample_reqs], np.uint64),
+                        bt)
 
     def commit(self, plan: StepPlan, next_tokens: np.ndarray) -> None:
         """Record the step's sampled tokens and retire finished requests."""
@@ -273,7 +288,9 @@ class ToyDecoder:
             n += 8
         last = L.bi_embedding(h, rows)
         logits = L.bi_matmul(last, W["lm_head"], out_dtype=torch.float32)
-        nt = L.bi_argmax(logits)
+        nt = L.bi_sample(logits, self._to_dev(plan.temperature), self._to_dev(plan.top_p),
+                         self._to_dev(plan.seed.view(np.int64)),
+                         self._to_dev(plan.offset.view(np.int64)))
         self.launches += n + 3
         return nt.cpu().numpy()
 

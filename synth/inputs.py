@@ -262,7 +262,9 @@ def unique_completion_workload(seed: int = 4, n_target: int = 1000, n_other: int
     the number of running requests sweeps from 1 up to the scheduler's cap.
 
     Returns ``(prompt, requests)`` with requests a list of dicts
-    ``{rid, prompt, max_new, arrival, tag}`` in random order."""
+    ``{rid, prompt, max_new, arrival, tag, seed}`` in random order; every
+    target copy carries the same sampling seed (the same request sent again),
+    the others seeds of their own."""
     g = rng(seed)
     prompt = g.integers(0, vocab, size=prompt_len).astype(np.int32)
     n = n_target + n_other
@@ -273,12 +275,15 @@ def unique_completion_workload(seed: int = 4, n_target: int = 1000, n_other: int
     widths = g.uniform(1, steps_span / 8, size=16)
     which = g.integers(0, 16, size=n)
     arrival = np.clip(centres[which] + g.uniform(-0.5, 0.5, size=n) * widths[which], 0, None)
+    target_seed = int(g.integers(0, 2 ** 62))
     reqs = []
     for i in range(n):
         if tags[i] == "target":
-            p, m = prompt, gen_len
+            p, m, sd = prompt, gen_len, target_seed
         else:
             p = g.integers(0, vocab, size=int(g.integers(1, other_prompt_max + 1))).astype(np.int32)
             m = int(g.integers(1, gen_len + 1))
-        reqs.append(dict(rid=i, prompt=p, max_new=m, arrival=int(arrival[i]), tag=str(tags[i])))
+            sd = int(g.integers(0, 2 ** 62))
+        reqs.append(dict(rid=i, prompt=p, max_new=m, arrival=int(arrival[i]), tag=str(tags[i]),
+                         seed=sd))
     return prompt, reqs

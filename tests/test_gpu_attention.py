@@ -322,3 +322,21 @@ def test_bounded_wait_gives_up_and_the_context_survives(L):
     assert L.bi_device_status() == bi.Status.OK
     c = tiny_layer()
     decode_parity(L, c["kv"], c["q"])
+
+
+def test_repeat_runs_are_identical(L):
+    # the same decode and prefill calls made 100 times give the same bytes
+    g = rng(51)
+    lens = [5000, 1, 300, 2600]
+    kv = paged_kv(g, lens, 4, 128)
+    q = dev_bf16(normal_bf16(g, (4, 64, 128)))
+    dkv, sl = dev_kv(kv), i32(kv.seq_lens)
+    ref = L.bi_attention_decode(dkv, q, sl, 5000)
+    S = 700
+    qp = dev_bf16(normal_bf16(g, (S, 8, 128)))
+    kp, vp = normal_bf16(g, (S, 2, 128)), normal_bf16(g, (S, 2, 128))
+    pkv, _ = write_sequence(L, S, 2, 128, kp, vp, seed=5)
+    refp = L.bi_attention_prefill(pkv, qp, i32([0, S]), i32([0]), S)
+    for _ in range(100):
+        assert same_bytes(L.bi_attention_decode(dkv, q, sl, 5000), ref)
+        assert same_bytes(L.bi_attention_prefill(pkv, qp, i32([0, S]), i32([0]), S), refp)

@@ -58,3 +58,25 @@ def test_full_size_decoder_step_runs():
         assert alone.out == r.out, r.rid
     torch.cuda.synchronize()
     assert len(together.finished) == 4
+
+
+def test_unique_completion_small_with_sampling():
+    # temperature 0.8, nucleus 0.95: every target copy carries the same seed,
+    # so every copy draws the same tokens however the batch around it looks
+    L = bi.load()
+    w = toy_decoder_weights(weight_shapes(SMALL), seed=4, device="cuda")
+    prompt, spec = unique_completion_workload(seed=5, n_target=24, n_other=120, prompt_len=40,
+                                              gen_len=24, vocab=SMALL.vocab,
+                                              other_prompt_max=300, steps_span=60)
+    tseed = next(d["seed"] for d in spec if d["tag"] == "target")
+    solo = Request(-1, prompt, 24, temperature=0.8, top_p=0.95, seed=tseed)
+    completions(L, SMALL, w, [solo], max_batch=1, budget=16)
+    reqs = [Request(d["rid"], d["prompt"], d["max_new"], d["arrival"], d["tag"], temperature=0.8,
+                    top_p=0.95, seed=d["seed"]) for d in spec]
+    completions(L, SMALL, w, reqs, max_batch=48, budget=256)
+    outs = {tuple(r.out) for r in reqs if r.tag == "target"}
+    assert outs == {tuple(solo.out)}
+    # and sampling did not collapse to the greedy completion
+    greedy = Request(-1, prompt, 24)
+    completions(L, SMALL, w, [greedy], max_batch=1, budget=64)
+    assert tuple(greedy.out) != tuple(solo.out)
