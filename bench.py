@@ -698,6 +698,13 @@ def run_profile_case(args):
             fn = lambda i: L.bi_rmsnorm(xs[i % 16], w, 1e-6)  # noqa: E731
         else:
             fn = lambda i: L.bi_matmul(x, W)  # noqa: E731
+    elif args.profile == "sample":
+        # 256 rows of lm_head logits (vocab 32000), temperature 0.8, nucleus 0.95
+        g = rng(5)
+        lg = T.from_numpy((g.standard_normal((256, 32000)) * 2.0).astype(np.float32)).to(dev)
+        seeds = T.from_numpy(g.integers(0, 2 ** 62, size=256)).to(dev)
+        offs = T.from_numpy(g.integers(0, 2 ** 20, size=256)).to(dev)
+        fn = lambda i: L.bi_sample(lg, 0.8, 0.95, seeds, offs)  # noqa: E731
     elif args.profile == "decode":
         B = args.profile_batch
         g = rng(2)
@@ -830,7 +837,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=20.0,
                     help="seconds of oracle work for the cpu_baseline sample")
-    ap.add_argument("--profile", choices=["rmsnorm", "matmul", "decode", "prefill", "copy"],
+    ap.add_argument("--profile", choices=["rmsnorm", "matmul", "decode", "prefill", "copy",
+                                          "sample"],
                     help="run one kernel alone on a reduced case (for ncu)")
     ap.add_argument("--profile-batch", type=int, default=32)
     ap.add_argument("--profile-seq", type=int, default=4096)

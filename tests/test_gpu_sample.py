@@ -67,6 +67,7 @@ def test_sample_matches_the_oracle(L):
     got = run(L, logits, temp, top_p, seeds, offs)
     want, r, _ = oracle.sample(logits, temp, top_p, seeds, offs, details=True)
     bad = np.nonzero(got != want)[0]
+    print("rows decided differently at a boundary: %d of %d" % (len(bad), len(got)))
     assert len(bad) <= 4, bad
     for t in bad:  # only at a rounding-close boundary
         assert margin(logits[t], temp[t], top_p[t], r[t]) < 1e-5, t
