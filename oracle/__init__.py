@@ -62,6 +62,9 @@ class Oracle:
         lib.oracle_argmax.argtypes = [P, i64, i64, P]
         lib.oracle_philox4x32_10.argtypes = [P, P, P]
         lib.oracle_sample.argtypes = [P, i64, i64, P, P, P, P, P, P, P]
+        lib.oracle_moe_route.argtypes = [P, i64, i32, i32, P, P]
+        lib.oracle_moe_dispatch.argtypes = [P, i64, i32, P, P, P]
+        lib.oracle_moe_combine.argtypes = [P, P, P, i64, i32, i64, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
@@ -207,6 +210,38 @@ class Oracle:
                                _p(r), _p(zk))
         return (out, r, zk) if details else out
 
+    # ---------------------------------------------------------- mixture of experts
+
+    def moe_route(self, logits, k: int):
+        """(experts [T, k] int32, weights [T, k] float64) from fp32 router logits [T, E]."""
+        logits = np.ascontiguousarray(logits, dtype=np.float32)
+        T, E = logits.shape
+        ex = np.empty((T, k), dtype=np.int32)
+        w = np.empty((T, k), dtype=np.float64)
+        self.lib.oracle_moe_route(_p(logits), T, E, k, _p(ex), _p(w))
+        return ex, w
+
+    def moe_dispatch(self, experts, E: int):
+        """(offsets [E+1], order [N], pos [N]) grouping the flat entries by expert."""
+        ex = np.ascontiguousarray(experts, dtype=np.int32).ravel()
+        N = ex.shape[0]
+        off = np.empty(E + 1, dtype=np.int64)
+        order = np.empty(N, dtype=np.int64)
+        pos = np.empty(N, dtype=np.int64)
+        self.lib.oracle_moe_dispatch(_p(ex), N, E, _p(off), _p(order), _p(pos))
+        return off, order, pos
+
+    def moe_combine(self, y, pos, weights) -> np.ndarray:
+        """Gate-weighted sum of each token's expert rows; y [N, H] bf16 bits."""
+        y = _u16(y)
+        w = np.ascontiguousarray(weights, dtype=np.float64)
+        T, k = w.shape
+        ps = np.ascontiguousarray(pos, dtype=np.int64)
+        H = y.shape[1]
+        out = np.empty((T, H), dtype=np.float64)
+        self.lib.oracle_moe_combine(_p(y), _p(ps), _p(w), T, k, H, _p(out))
+        return out
+
 
 def default() -> Oracle:
     global _lib
@@ -267,6 +302,18 @@ def philox4x32_10(ctr, key) -> np.ndarray:
 
 def sample(logits, temperature, top_p, seed, offset, details: bool = False):
     return default().sample(logits, temperature, top_p, seed, offset, details)
+
+
+def moe_route(logits, k: int):
+    return default().moe_route(logits, k)
+
+
+def moe_dispatch(experts, E: int):
+    return default().moe_dispatch(experts, E)
+
+
+def moe_combine(y, pos, weights) -> np.ndarray:
+    return default().moe_combine(y, pos, weights)
 
 
 def decode_rows(q, seq_lens, heads=None):

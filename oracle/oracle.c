@@ -433,3 +433,74 @@ void oracle_sample(const float *logits, int64_t T, int64_t V, const float *tempe
         free(sorted);
     }
 }
+
+/* ------------------------------------------------------------------------
+ * Mixture-of-experts feed-forward.  The model of the reports' experiment is
+ * a mixture of experts (Qwen3-235B-A22B; xitu-tech news, "显著成果与高昂成本";
+ * neican.ai insight, "技术原理与创新点解析"); they describe no router.  Reading
+ * taken (the common top-k router): each token's router logits over E
+ * experts pick its k experts by largest logit (lowest index on ties); the
+ * gate weights are the softmax of the selected logits (the full softmax
+ * renormalised over the k); the token's output is the gate-weighted sum of
+ * its experts' outputs, taken in rank order.
+ * ------------------------------------------------------------------------ */
+
+/* experts[t, i] = the i-th largest logit's index (ties: lower index first);
+ * weights[t, i] = exp(l_i - l_0) / sum_j exp(l_j - l_0) over the k chosen. */
+void oracle_moe_route(const float *logits, int64_t T, int32_t E, int32_t k, int32_t *experts,
+                      double *weights)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        const float *row = logits + t * E;
+        int32_t *ex = experts + t * k;
+        for (int32_t i = 0; i < k; ++i) {
+            int32_t best = -1;
+            for (int32_t e = 0; e < E; ++e) {
+                int taken = 0;
+                for (int32_t j = 0; j < i; ++j)
+                    if (ex[j] == e) taken = 1;
+                if (taken) continue;
+                if (best < 0 || row[e] > row[best]) best = e;
+            }
+            ex[i] = best;
+        }
+        double sum = 0.0;
+        for (int32_t i = 0; i < k; ++i) sum += exp((double)row[ex[i]] - (double)row[ex[0]]);
+        for (int32_t i = 0; i < k; ++i)
+            weights[t * k + i] = exp((double)row[ex[i]] - (double)row[ex[0]]) / sum;
+    }
+}
+
+/* Group the T*k (token, rank) entries by expert: offsets[e] .. offsets[e+1]
+ * hold expert e's entries in increasing entry index (entry = t*k + i);
+ * order[p] is the entry at position p, pos[entry] its position. */
+void oracle_moe_dispatch(const int32_t *experts, int64_t N, int32_t E, int64_t *offsets,
+                         int64_t *order, int64_t *pos)
+{
+    int64_t p = 0;
+    for (int32_t e = 0; e < E; ++e) {
+        offsets[e] = p;
+        for (int64_t i = 0; i < N; ++i)
+            if (experts[i] == e) {
+                order[p] = i;
+                pos[i] = p;
+                ++p;
+            }
+    }
+    offsets[E] = p;
+}
+
+/* out[t, :] = sum over i of weights[t, i] * y[pos[t*k + i], :]. */
+void oracle_moe_combine(const uint16_t *y, const int64_t *pos, const double *weights, int64_t T,
+                        int32_t k, int64_t H, double *out)
+{
+    int64_t t;
+#pragma omp parallel for schedule(static)
+    for (t = 0; t < T; ++t) {
+        for (int64_t h = 0; h < H; ++h) out[t * H + h] = 0.0;
+        for (int32_t i = 0; i < k; ++i) {
+            const uint16_t *yr = y + pos[t * k + i] * H;
+            for (int64_t h = 0; h < H; ++h) out[t * H + h] += weights[t * k + i] * bf16_to_double(yr[h]);
+        }
+    }
+}

@@ -531,3 +531,51 @@ def test_sample_frequencies_follow_the_softmax(oracle):
     for k in range(5):
         f = (toks == k).mean()
         assert abs(f - p[k]) < 4.5 * np.sqrt(p[k] * (1 - p[k]) / n), (k, f, p[k])
+
+
+# ---------------------------------------------------------------- mixture of experts
+
+
+def test_moe_route_hand_example(oracle):
+    logits = np.array([[0.5, 2.0, -1.0, 2.0, 1.0]], dtype=np.float32)
+    ex, w = oracle.moe_route(logits, 3)
+    assert ex.tolist() == [[1, 3, 4]]          # tie 2.0: index 1 before 3
+    e = np.exp([0.0, 0.0, -1.0])
+    np.testing.assert_allclose(w[0], e / e.sum(), rtol=1e-15)
+
+
+def test_moe_route_matches_a_stable_sort(oracle):
+    g = rng(160)
+    logits = g.integers(-4, 5, size=(200, 16)).astype(np.float32)  # many ties
+    ex, w = oracle.moe_route(logits, 4)
+    want = np.argsort(-logits.astype(np.float64), axis=1, kind="stable")[:, :4]
+    assert np.array_equal(ex, want)
+    np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=1e-14)
+    sel = np.take_along_axis(logits, want, axis=1).astype(np.float64)
+    t = torch.softmax(torch.from_numpy(sel), dim=1).numpy()
+    np.testing.assert_allclose(w, t, rtol=1e-13)
+    _, w1 = oracle.moe_route(logits, 1)
+    assert np.all(w1 == 1.0)
+
+
+def test_moe_dispatch_groups_by_expert_stably(oracle):
+    g = rng(161)
+    ex = g.integers(0, 8, size=(50, 3)).astype(np.int32)
+    off, order, pos = oracle.moe_dispatch(ex, 8)
+    flat = ex.ravel()
+    want = np.argsort(flat, kind="stable")
+    assert np.array_equal(order, want)
+    assert np.array_equal(pos[order], np.arange(flat.size))
+    assert np.array_equal(np.diff(off), np.bincount(flat, minlength=8))
+
+
+def test_moe_combine_closed_forms(oracle):
+    g = rng(162)
+    y = normal_bf16(g, (6, 32))
+    pos = np.array([3, 0, 5, 1, 2, 4])           # T = 3 tokens, k = 2
+    w = np.array([[1.0, 0.0], [0.25, 0.75], [0.5, 0.5]])
+    out = oracle.moe_combine(y, pos, w)
+    yf = widen(y)
+    np.testing.assert_array_equal(out[0], yf[3])
+    np.testing.assert_allclose(out[1], 0.25 * yf[5] + 0.75 * yf[1], rtol=1e-15)
+    np.testing.assert_allclose(out[2], 0.5 * (yf[2] + yf[4]), rtol=1e-15)

@@ -79,6 +79,17 @@ MUTATIONS = [
      [pins.test_sample_uniform_logits_closed_form]),
     ("sample_nucleus_ignored", "double need = (double)top_p[t] * total", "double need = total",
      [pins.test_sample_nucleus_drops_the_tail, pins.test_sample_dominant_logit_and_tiny_top_p]),
+    ("moe_route_ties_to_higher_index", "if (best < 0 || row[e] > row[best]) best = e;",
+     "if (best < 0 || row[e] >= row[best]) best = e;",
+     [pins.test_moe_route_hand_example, pins.test_moe_route_matches_a_stable_sort]),
+    ("moe_route_weights_not_renormalised", "weights[t * k + i] = exp((double)row[ex[i]] - (double)row[ex[0]]) / sum;",
+     "weights[t * k + i] = exp((double)row[ex[i]] - (double)row[ex[0]]);",
+     [pins.test_moe_route_hand_example, pins.test_moe_route_matches_a_stable_sort]),
+    ("moe_dispatch_wrong_position", "pos[i] = p;", "pos[i] = p + 1;",
+     [pins.test_moe_dispatch_groups_by_expert_stably]),
+    ("moe_combine_ignores_weights", "out[t * H + h] += weights[t * k + i] * bf16_to_double(yr[h]);",
+     "out[t * H + h] += bf16_to_double(yr[h]);",
+     [pins.test_moe_combine_closed_forms]),
     ("argmax_ties_take_highest_index", "if (row[j] > row[best]) best = j;",
      "if (row[j] >= row[best]) best = j;",
      [pins.test_argmax_ties_take_the_lowest_index, pins.test_argmax_matches_numpy_first_occurrence]),
