@@ -746,11 +746,11 @@ def run_profile_case(args):
 def run_unique_completions(args):
     print(json.dumps(unique_completions(args.targets, args.others, args.max_batch,
                                         args.token_budget, args.span, args.temperature,
-                                        args.top_p)), flush=True)
+                                        args.top_p, args.moe)), flush=True)
 
 
 def unique_completions(targets, others, max_batch=256, token_budget=2048, span=2000,
-                       temperature=0.0, top_p=1.0) -> dict:
+                       temperature=0.0, top_p=1.0, moe=False) -> dict:
     """One fixed 64-token prompt completed greedily (256 tokens) many times
     amid random other requests, on the 8-layer hidden-4096 random-init
     decoder: the number of distinct completions for the invariant and the
@@ -765,14 +765,16 @@ def unique_completions(targets, others, max_batch=256, token_budget=2048, span=2
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    cfg = DecoderConfig()
+    # dense: SwiGLU 14336; mixture of experts: 16 experts of SwiGLU 1408, top 4
+    cfg = DecoderConfig(n_experts=16, top_k=4, expert_ffn=1408) if moe else DecoderConfig()
     weights = toy_decoder_weights(weight_shapes(cfg), seed=4, device=dev)
     prompt, spec = unique_completion_workload(seed=4, n_target=targets, n_other=others,
                                               vocab=cfg.vocab, steps_span=span)
     pages_per_req = (512 + 256 + 15) // 16
     num_pages = max_batch * pages_per_req + 64
+    ffn = ("mixture of 16 experts (SwiGLU 1408, top 4)" if moe else "SwiGLU 14336")
     result = {"experiment": "unique completions", "model": "8-layer decoder, hidden 4096, GQA 32/8, "
-              "d 128, SwiGLU 14336, vocab 32000, W~N(0,0.02) seed 4",
+              "d 128, %s, vocab 32000, W~N(0,0.02) seed 4" % ffn,
               "prompt_tokens": 64, "new_tokens": 256, "targets": targets,
               "others": others, "max_batch": max_batch,
               "token_budget": token_budget, "data": "synthetic",
@@ -853,6 +855,8 @@ def main(argv=None):
     ap.add_argument("--temperature", type=float, default=0.0,
                     help="unique-completion run: 0 = greedy, else sampling at this temperature")
     ap.add_argument("--top-p", type=float, default=1.0)
+    ap.add_argument("--moe", action="store_true",
+                    help="unique-completion run on the mixture-of-experts decoder")
     ap.add_argument("--uc-targets", type=int, default=200,
                     help="target copies (and as many others) of the in-bench unique-completion "
                          "check; 0 skips it")

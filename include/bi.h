@@ -353,6 +353,54 @@ bi_status bi_sample(const float *logits, int64_t T, int64_t V, const float *temp
                     const float *top_p, const uint64_t *seed, const uint64_t *offset, int32_t *out,
                     void *stream);
 
+/*
+ * Mixture-of-experts feed-forward.  The model of the reports' experiment is
+ * a mixture of experts (Qwen3-235B-A22B; xitu-tech news, "显著成果与高昂成本";
+ * neican.ai insight, "技术原理与创新点解析"); they describe no router.  The
+ * plainest reading: each token picks its k experts by largest router logit
+ * (lowest index on ties), its gate weights are the softmax of the selected
+ * logits, its output is the gate-weighted sum of its experts' outputs in
+ * rank order.  The experts' matmuls go through bi_matmul, whose rows do not
+ * depend on how many tokens an expert received, so a token's output does
+ * not depend on the batch.
+ */
+
+/*
+ * bi_moe_route -- experts[t, i] = index of the i-th largest of
+ * logits[t, 0..E-1] (ties: lower index first); weights[t, i] =
+ * e^(l_i - l_0) / sum_j e^(l_j - l_0) over the chosen k (fp32, summed in
+ * rank order).
+ *   logits : device, fp32 [T, E] (finite);  experts : device, int32 [T, k];
+ *   weights : device, fp32 [T, k].  1 <= k <= min(E, 16), E <= 256.
+ */
+bi_status bi_moe_route(const float *logits, int64_t T, int32_t E, int32_t k, int32_t *experts,
+                       float *weights, void *stream);
+
+/*
+ * bi_moe_dispatch -- groups the T*k entries (entry t*k + i = token t's i-th
+ * expert) by expert, keeping entry order inside an expert: offsets[e] ..
+ * offsets[e+1]-1 are expert e's positions; order[p] is the entry at position
+ * p, pos[entry] its position, token_sorted[p] = order[p] / k (the rows to
+ * gather, e.g. with bi_embedding).  Integer work, exact.  An expert id
+ * outside 0..E-1 is skipped (pos = -1) and flags BI_ERR_DEVICE_INDEX.
+ *   experts : device, int32 [T, k];  offsets : device, int64 [E + 1];
+ *   order, pos : device, int64 [T*k];  token_sorted : device, int32 [T*k].
+ */
+bi_status bi_moe_dispatch(const int32_t *experts, int64_t T, int32_t k, int32_t E,
+                          int64_t *offsets, int64_t *order, int64_t *pos, int32_t *token_sorted,
+                          void *stream);
+
+/*
+ * bi_moe_combine -- out[t, :] = round( sum_{i<k} weights[t, i] *
+ * y[pos[t*k + i], :] ), fp32, terms added in rank order, bf16 RNE.
+ *   y : device, bf16 [T*k, H] (the experts' outputs in dispatch order);
+ *   pos : device, int64 [T*k] (from bi_moe_dispatch);  weights : device,
+ *   fp32 [T, k];  out : device, bf16 [T, H].  H % 8 == 0, y and out 16-byte
+ *   aligned.
+ */
+bi_status bi_moe_combine(const void *y, const int64_t *pos, const float *weights, int64_t T,
+                         int32_t k, int64_t H, void *out, void *stream);
+
 const char *bi_status_string(bi_status s);
 
 /* 1 for the batch-invariant build, 0 for the variant-off build (split-K

@@ -109,7 +109,8 @@ class Library:
                "bi_attention_prefill", "bi_attention_prefill_workspace_bytes",
                "bi_status_string", "bi_build_invariant", "bi_device_status",
                "bi_debug_bounded_wait", "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write",
-               "bi_swiglu", "bi_argmax", "bi_sample")
+               "bi_swiglu", "bi_argmax", "bi_sample", "bi_moe_route", "bi_moe_dispatch",
+               "bi_moe_combine")
 
     def __init__(self, path: str):
         if not os.path.exists(path):
@@ -144,10 +145,14 @@ class Library:
         L.bi_swiglu.argtypes = [P, P, i64, i64, P]
         L.bi_argmax.argtypes = [P, i64, i64, P, P]
         L.bi_sample.argtypes = [P, i64, i64, P, P, P, P, P, P]
+        L.bi_moe_route.argtypes = [P, i64, i32, i32, P, P, P]
+        L.bi_moe_dispatch.argtypes = [P, i64, i32, i32, P, P, P, P, P]
+        L.bi_moe_combine.argtypes = [P, P, P, i64, i32, i64, P, P]
         for name in ("bi_rmsnorm", "bi_matmul", "bi_kv_write", "bi_attention_decode",
                      "bi_attention_prefill", "bi_device_status", "bi_debug_bounded_wait",
                      "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write", "bi_swiglu",
-                     "bi_argmax", "bi_sample"):
+                     "bi_argmax", "bi_sample", "bi_moe_route", "bi_moe_dispatch",
+                     "bi_moe_combine"):
             getattr(L, name).restype = st
         self.lib = L
 
@@ -317,6 +322,46 @@ class Library:
         self._check("bi_sample", self.lib.bi_sample(
             _ptr(logits), T, V, _ptr(temperature), _ptr(top_p), _ptr(seed), _ptr(offset), _ptr(out),
             _stream(stream)))
+        return out
+
+    # ------------------------------------------------------------ mixture of experts
+    def bi_moe_route(self, logits: torch.Tensor, k: int, stream=None):
+        """(experts int32 [T, k], weights fp32 [T, k]) from fp32 router logits [T, E]."""
+        _need(logits, "logits", torch.float32)
+        T, E = logits.shape
+        ex = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+        w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+        self._check("bi_moe_route", self.lib.bi_moe_route(_ptr(logits), T, E, k, _ptr(ex), _ptr(w),
+                                                          _stream(stream)))
+        return ex, w
+
+    def bi_moe_dispatch(self, experts: torch.Tensor, E: int, stream=None):
+        """(offsets [E+1], order [T*k], pos [T*k], token_sorted [T*k]) grouping by expert."""
+        _need(experts, "experts", torch.int32)
+        T, k = experts.shape
+        dev = experts.device
+        off = torch.empty((E + 1,), dtype=torch.int64, device=dev)
+        order = torch.empty((T * k,), dtype=torch.int64, device=dev)
+        pos = torch.empty((T * k,), dtype=torch.int64, device=dev)
+        tok = torch.empty((T * k,), dtype=torch.int32, device=dev)
+        self._check("bi_moe_dispatch", self.lib.bi_moe_dispatch(
+            _ptr(experts), T, k, E, _ptr(off), _ptr(order), _ptr(pos), _ptr(tok), _stream(stream)))
+        return off, order, pos, tok
+
+    def bi_moe_combine(self, y: torch.Tensor, pos: torch.Tensor, weights: torch.Tensor, out=None,
+                       stream=None) -> torch.Tensor:
+        """Gate-weighted sum in rank order: y [T*k, H] bf16 (dispatch order) -> [T, H]."""
+        _need(weights, "weights", torch.float32)
+        T, k = weights.shape
+        _need(y, "y", torch.bfloat16)
+        H = y.shape[1]
+        _need(y, "y", torch.bfloat16, (T * k, H))
+        _need(pos, "pos", torch.int64, (T * k,))
+        if out is None:
+            out = torch.empty((T, H), dtype=torch.bfloat16, device=y.device)
+        _need(out, "out", torch.bfloat16, (T, H))
+        self._check("bi_moe_combine", self.lib.bi_moe_combine(
+            _ptr(y), _ptr(pos), _ptr(weights), T, k, H, _ptr(out), _stream(stream)))
         return out
 
     # ------------------------------------------------------------ attention

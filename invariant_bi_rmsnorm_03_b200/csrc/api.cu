@@ -277,6 +277,49 @@ bi_status bi_sample(const float *logits, int64_t T, int64_t V, const float *temp
                                        d->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
+bi_status bi_moe_route(const float *logits, int64_t T, int32_t E, int32_t k, int32_t *experts,
+                       float *weights, void *stream)
+{
+    if (T < 0 || E < 1 || E > bi::kMaxMoeExperts || k < 1 || k > bi::kMaxMoeTopK || k > E)
+        return BI_ERR_INVALID;
+    if (T == 0) return BI_OK;
+    if (!logits || !experts || !weights) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_moe_route(logits, T, E, k, experts, weights, d->num_sms,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+bi_status bi_moe_dispatch(const int32_t *experts, int64_t T, int32_t k, int32_t E,
+                          int64_t *offsets, int64_t *order, int64_t *pos, int32_t *token_sorted,
+                          void *stream)
+{
+    if (T < 0 || E < 1 || E > bi::kMaxMoeExperts || k < 1 || k > bi::kMaxMoeTopK)
+        return BI_ERR_INVALID;
+    if (T > (int64_t(1) << 31) / k) return BI_ERR_INVALID;
+    if (!experts || !offsets || !order || !pos || !token_sorted) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_moe_dispatch(experts, T * k, E, k, offsets, order, pos,
+                                             token_sorted, d->status,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+bi_status bi_moe_combine(const void *y, const int64_t *pos, const float *weights, int64_t T,
+                         int32_t k, int64_t H, void *out, void *stream)
+{
+    if (T < 0 || k < 1 || k > bi::kMaxMoeTopK || H < 8 || H % 8 != 0) return BI_ERR_INVALID;
+    if (T == 0) return BI_OK;
+    if (!y || !pos || !weights || !out || !aligned16(y) || !aligned16(out)) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_moe_combine(y, pos, weights, T, k, H, out, d->status, d->num_sms,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 static bool attn_common_ok(const bi_paged_kv *kv, int32_t Hq)
 {
     if (!kv_ok(kv)) return false;

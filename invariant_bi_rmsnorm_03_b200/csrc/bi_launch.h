@@ -88,6 +88,18 @@ cudaError_t launch_sample(const float *logits, int64_t T, int64_t V, const float
                           const float *top_p, const uint64_t *seed, const uint64_t *offset,
                           int32_t *out, int num_sms, cudaStream_t s);
 
+// ---------------------------------------------------------------- mixture of experts
+constexpr int kMaxMoeExperts = 256;
+constexpr int kMaxMoeTopK = 16;
+cudaError_t launch_moe_route(const float *logits, int64_t T, int E, int k, int32_t *experts,
+                             float *weights, int num_sms, cudaStream_t s);
+cudaError_t launch_moe_dispatch(const int32_t *experts, int64_t N, int E, int k, int64_t *offsets,
+                                int64_t *order, int64_t *pos, int32_t *token_sorted,
+                                unsigned *status, cudaStream_t s);
+cudaError_t launch_moe_combine(const void *y, const int64_t *pos, const float *weights, int64_t T,
+                               int k, int64_t H, void *out, unsigned *status, int num_sms,
+                               cudaStream_t s);
+
 // ---------------------------------------------------------------- debug
 cudaError_t launch_bounded_wait_probe(unsigned *status, uint64_t timeout_ns, cudaStream_t s);
 

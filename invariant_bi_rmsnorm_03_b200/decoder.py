@@ -9,9 +9,11 @@ layer beyond RMSNorm, matmul and attention, so the model here is the plain
 pre-norm transformer (token embedding; per layer RMSNorm -> stacked q/k/v
 matmul -> rotary embedding + KV-cache write -> paged attention -> output
 matmul -> residual + RMSNorm -> stacked gate/up matmul -> SwiGLU -> down
-matmul -> residual; final RMSNorm; lm_head matmul in fp32; the next token by
-bi_sample: greedy at temperature 0, else nucleus sampling from the request's
-own counter-based random stream).
+matmul -> residual, or a mixture of experts in place of the one feed-forward
+(router matmul -> top-k route -> grouping by expert -> each expert's SwiGLU
+feed-forward -> gate-weighted combine); final RMSNorm; lm_head matmul in
+fp32; the next token by bi_sample: greedy at temperature 0, else nucleus
+sampling from the request's own counter-based random stream).
 
 Every arithmetic step runs in the library's CUDA kernels through the C ABI;
 this module only plans the batch on the host (which request contributes
@@ -41,6 +43,9 @@ class DecoderConfig:
     vocab: int = 32000
     theta: float = 10000.0
     eps: float = 1e-6
+    n_experts: int = 0            # > 0: a mixture-of-experts feed-forward
+    top_k: int = 2
+    expert_ffn: int = 1408
 
     @property
     def qkv_dim(self) -> int:
@@ -56,8 +61,14 @@ def weight_shapes(cfg: DecoderConfig) -> dict:
         s["l%d.wqkv" % i] = (cfg.qkv_dim, cfg.hidden)
         s["l%d.wo" % i] = (cfg.hidden, cfg.n_heads * cfg.head_dim)
         s["l%d.mlp_norm" % i] = (cfg.hidden,)
-        s["l%d.wgu" % i] = (2 * cfg.ffn, cfg.hidden)
-        s["l%d.wdown" % i] = (cfg.hidden, cfg.ffn)
+        if cfg.n_experts:
+            s["l%d.router" % i] = (cfg.n_experts, cfg.hidden)
+            for e in range(cfg.n_experts):
+                s["l%d.e%d.wgu" % (i, e)] = (2 * cfg.expert_ffn, cfg.hidden)
+                s["l%d.e%d.wdown" % (i, e)] = (cfg.hidden, cfg.expert_ffn)
+        else:
+            s["l%d.wgu" % i] = (2 * cfg.ffn, cfg.hidden)
+            s["l%d.wdown" % i] = (cfg.hidden, cfg.ffn)
     return s
 
 
@@ -281,11 +292,16 @@ class ToyDecoder:
                 n += 1
             a = L.bi_matmul(o.view(T, c.n_heads * c.head_dim), W["l%d.wo" % i])
             h = L.bi_add_rmsnorm(x, a, W["l%d.mlp_norm" % i], c.eps)
-            f = L.bi_swiglu(L.bi_matmul(h, W["l%d.wgu" % i]))
-            m = L.bi_matmul(f, W["l%d.wdown" % i])
+            if c.n_experts:
+                m, nm = self._moe(h, i)
+                n += nm
+            else:
+                f = L.bi_swiglu(L.bi_matmul(h, W["l%d.wgu" % i]))
+                m = L.bi_matmul(f, W["l%d.wdown" % i])
+                n += 3
             nxt = W["l%d.attn_norm" % (i + 1)] if i + 1 < c.layers else W["final_norm"]
             h = L.bi_add_rmsnorm(x, m, nxt, c.eps)
-            n += 8
+            n += 5
         last = L.bi_embedding(h, rows)
         logits = L.bi_matmul(last, W["lm_head"], out_dtype=torch.float32)
         nt = L.bi_sample(logits, self._to_dev(plan.temperature), self._to_dev(plan.top_p),
@@ -293,6 +309,27 @@ class ToyDecoder:
                          self._to_dev(plan.offset.view(np.int64)))
         self.launches += n + 3
         return nt.cpu().numpy()
+
+
+    def _moe(self, h: torch.Tensor, i: int):
+        """The mixture-of-experts feed-forward of layer i; returns (output,
+        launches).  The expert boundaries are read back to the host to size
+        each expert's matmuls (one synchronisation per layer)."""
+        L, c, W = self.L, self.cfg, self.w
+        logits = L.bi_matmul(h, W["l%d.router" % i], out_dtype=torch.float32)
+        experts, gates = L.bi_moe_route(logits, c.top_k)
+        off, _, pos, tok = L.bi_moe_dispatch(experts, c.n_experts)
+        xs = L.bi_embedding(h, tok)                  # rows grouped by expert
+        ys = torch.empty_like(xs)
+        bounds = off.cpu().tolist()
+        n = 4
+        for e in range(c.n_experts):
+            a, b = bounds[e], bounds[e + 1]
+            if b > a:
+                f = L.bi_swiglu(L.bi_matmul(xs[a:b], W["l%d.e%d.wgu" % (i, e)]))
+                L.bi_matmul(f, W["l%d.e%d.wdown" % (i, e)], out=ys[a:b])
+                n += 3
+        return L.bi_moe_combine(ys, pos, gates), n + 1
 
 
 def run(sched: Scheduler, model: ToyDecoder, max_steps: int = 1_000_000) -> int:

@@ -80,3 +80,19 @@ def test_unique_completion_small_with_sampling():
     greedy = Request(-1, prompt, 24)
     completions(L, SMALL, w, [greedy], max_batch=1, budget=64)
     assert tuple(greedy.out) != tuple(solo.out)
+
+
+def test_unique_completion_small_moe():
+    # the same experiment on a mixture-of-experts decoder (16 experts, top 4)
+    L = bi.load()
+    cfg = DecoderConfig(hidden=512, layers=2, n_heads=8, n_kv_heads=2, head_dim=64, vocab=2000,
+                        n_experts=16, top_k=4, expert_ffn=256)
+    w = toy_decoder_weights(weight_shapes(cfg), seed=6, device="cuda")
+    prompt, spec = unique_completion_workload(seed=7, n_target=16, n_other=80, prompt_len=32,
+                                              gen_len=16, vocab=cfg.vocab, other_prompt_max=200,
+                                              steps_span=40)
+    solo = Request(-1, prompt, 16)
+    completions(L, cfg, w, [solo], max_batch=1, budget=16)
+    reqs = [Request(d["rid"], d["prompt"], d["max_new"], d["arrival"], d["tag"]) for d in spec]
+    completions(L, cfg, w, reqs, max_batch=40, budget=256)
+    assert {tuple(r.out) for r in reqs if r.tag == "target"} == {tuple(solo.out)}
