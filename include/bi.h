@@ -383,6 +383,7 @@ bi_status bi_moe_route(const float *logits, int64_t T, int32_t E, int32_t k, int
  * p, pos[entry] its position, token_sorted[p] = order[p] / k (the rows to
  * gather, e.g. with bi_embedding).  Integer work, exact.  An expert id
  * outside 0..E-1 is skipped (pos = -1) and flags BI_ERR_DEVICE_INDEX.
+ * T == 0 only zeroes the offsets (the other arrays may then be NULL).
  *   experts : device, int32 [T, k];  offsets : device, int64 [E + 1];
  *   order, pos : device, int64 [T*k];  token_sorted : device, int32 [T*k].
  */

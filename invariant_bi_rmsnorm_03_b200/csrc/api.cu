@@ -298,7 +298,8 @@ bi_status bi_moe_dispatch(const int32_t *experts, int64_t T, int32_t k, int32_t 
     if (T < 0 || E < 1 || E > bi::kMaxMoeExperts || k < 1 || k > bi::kMaxMoeTopK)
         return BI_ERR_INVALID;
     if (T > (int64_t(1) << 31) / k) return BI_ERR_INVALID;
-    if (!experts || !offsets || !order || !pos || !token_sorted) return BI_ERR_INVALID;
+    if (!offsets) return BI_ERR_INVALID;
+    if (T > 0 && (!experts || !order || !pos || !token_sorted)) return BI_ERR_INVALID;
     DeviceState *d;
     bi_status st = device_state(&d);
     if (st != BI_OK) return st;

@@ -74,3 +74,34 @@ def test_moe_feed_forward_rows_do_not_depend_on_the_batch(L):
         yd = oracle.matmul(host_bits(f), host_bits(w["l0.e%d.wdown" % e]))
         acc += gw[0, i] * yd[0]
     assert rowwise_normwise(to_f64(full[:1]), acc[None]).max() <= TOL_BF16
+
+
+def test_degenerate_cases(L):
+    g = rng(190)
+    # k = E (every expert), a single expert, an empty batch
+    for T, E, k in ((33, 4, 4), (20, 1, 1)):
+        logits = g.standard_normal((T, E)).astype(np.float32)
+        ex, w = L.bi_moe_route(torch.from_numpy(logits).to(DEV), k)
+        oex, ow = oracle.moe_route(logits, k)
+        assert np.array_equal(ex.cpu().numpy(), oex)
+        assert rowwise_normwise(w.cpu().numpy().astype(np.float64), ow).max() <= TOL_F32
+        off, order, pos, tok = L.bi_moe_dispatch(ex, E)
+        o_off, o_order, o_pos = oracle.moe_dispatch(oex, E)
+        assert np.array_equal(order.cpu().numpy(), o_order)
+        assert np.array_equal(off.cpu().numpy(), o_off)
+    ex0, w0 = L.bi_moe_route(torch.empty((0, 8), device=DEV), 2)
+    assert ex0.shape == (0, 2)
+    off0, _, _, _ = L.bi_moe_dispatch(ex0, 8)
+    assert off0.cpu().numpy().tolist() == [0] * 9
+
+
+def test_bad_expert_id_is_flagged_not_faulted(L):
+    L.bi_device_status()
+    ex = torch.tensor([[0, 1], [9, 2]], dtype=torch.int32, device=DEV)  # 9 >= E = 4
+    off, order, pos, tok = L.bi_moe_dispatch(ex, 4)
+    assert L.bi_device_status() == bi.Status.DEVICE_INDEX
+    assert pos.cpu().numpy()[2] == -1
+    y = torch.zeros((4, 16), dtype=torch.bfloat16, device=DEV)
+    w = torch.full((2, 2), 0.5, dtype=torch.float32, device=DEV)
+    L.bi_moe_combine(y, pos, w)  # the unplaced entry is skipped, not read
+    assert L.bi_device_status() == bi.Status.DEVICE_INDEX

@@ -105,3 +105,24 @@ def test_frequencies_follow_the_softmax(L):
     for k in range(len(row)):
         f = (got == k).mean()
         assert abs(f - p[k]) < 4.5 * np.sqrt(p[k] * (1 - p[k]) / n), (k, f, p[k])
+
+
+def test_degenerate_cases(L):
+    g = rng(154)
+    # one-token vocabulary, odd vocabulary sizes, an empty batch
+    for V in (1, 3, 31999):
+        logits = g.standard_normal((7, V)).astype(np.float32)
+        got = run(L, logits, np.full(7, 0.9, np.float32), np.full(7, 0.9, np.float32),
+                  np.arange(7, dtype=np.uint64), np.zeros(7, np.uint64))
+        want = oracle.sample(logits, 0.9, 0.9, np.arange(7, dtype=np.uint64), 0)
+        assert np.array_equal(got, want), V
+    empty = L.bi_sample(torch.empty((0, 10), device=DEV), 1.0, 1.0, 0, 0)
+    assert empty.shape == (0,)
+    # top_p 0 keeps only the largest weight(s); a tiny temperature is greedy
+    logits = g.standard_normal((50, 1000)).astype(np.float32)
+    greedy = L.bi_argmax(dev(logits, torch.float32)).cpu().numpy()
+    seeds = np.arange(50, dtype=np.uint64)
+    assert np.array_equal(run(L, logits, np.ones(50, np.float32), np.zeros(50, np.float32),
+                              seeds, seeds), greedy)
+    assert np.array_equal(run(L, logits, np.full(50, 1e-6, np.float32), np.ones(50, np.float32),
+                              seeds, seeds), greedy)
