@@ -145,6 +145,28 @@ bi_status bi_matmul(const void *a, const void *w, void *c, int64_t M, int64_t N,
 size_t bi_matmul_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
+ * bi_matmul_grouped -- many matrix products of one shape family in one
+ * launch, as bi_matmul computes each: the rows offsets[g] .. offsets[g+1]-1
+ * of A and C (group g, e.g. the tokens routed to expert g) are multiplied
+ * by group g's weight, rows g*N .. g*N+N-1 of w:
+ *
+ *   C[r, n] = round( sum_k A[r, k] * w[g*N + n, k] )    offsets[g] <= r < offsets[g+1]
+ *
+ *   a : device, bf16 [rows, K];  w : device, bf16 [groups * N, K] (the
+ *   groups' weights stacked, each output-feature-major);  c : device,
+ *   [rows, N] of out_dtype;  offsets : device, int64 [groups + 1],
+ *   non-decreasing within 0..rows (rows outside every group are left
+ *   unwritten).  The tile list is built on the device from the offsets (no
+ *   read-back): each group's rows are cut into the same fixed 256 x 256 tiles
+ *   as bi_matmul, with the same K order, so a row's bits do not depend on
+ *   how many rows its group holds.  1 <= groups <= 256; K, N % 8 == 0;
+ *   pointers 16-byte aligned.  No split-K in either build.
+ */
+bi_status bi_matmul_grouped(const void *a, const void *w, void *c, const int64_t *offsets,
+                            int32_t groups, int64_t rows, int64_t N, int64_t K, bi_dtype out_dtype,
+                            void *stream);
+
+/*
  * bi_kv_write -- write the step's new keys and values into the paged cache
  * before attention runs, so that the attention kernel sees one consistent
  * KV layout (neican.ai insight, "技术原理与创新点解析", batch-invariant

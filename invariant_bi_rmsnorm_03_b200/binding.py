@@ -110,7 +110,7 @@ class Library:
                "bi_status_string", "bi_build_invariant", "bi_device_status",
                "bi_debug_bounded_wait", "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write",
                "bi_swiglu", "bi_argmax", "bi_sample", "bi_moe_route", "bi_moe_dispatch",
-               "bi_moe_combine")
+               "bi_moe_combine", "bi_matmul_grouped")
 
     def __init__(self, path: str):
         if not os.path.exists(path):
@@ -148,11 +148,12 @@ class Library:
         L.bi_moe_route.argtypes = [P, i64, i32, i32, P, P, P]
         L.bi_moe_dispatch.argtypes = [P, i64, i32, i32, P, P, P, P, P]
         L.bi_moe_combine.argtypes = [P, P, P, i64, i32, i64, P, P]
+        L.bi_matmul_grouped.argtypes = [P, P, P, P, i32, i64, i64, i64, st, P]
         for name in ("bi_rmsnorm", "bi_matmul", "bi_kv_write", "bi_attention_decode",
                      "bi_attention_prefill", "bi_device_status", "bi_debug_bounded_wait",
                      "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write", "bi_swiglu",
                      "bi_argmax", "bi_sample", "bi_moe_route", "bi_moe_dispatch",
-                     "bi_moe_combine"):
+                     "bi_moe_combine", "bi_matmul_grouped"):
             getattr(L, name).restype = st
         self.lib = L
 
@@ -226,6 +227,25 @@ class Library:
         self._check("bi_matmul", self.lib.bi_matmul(_ptr(a), _ptr(w), _ptr(out), M, N, K,
                                                     _DT[out_dtype], _ptr(ws), nbytes,
                                                     _stream(stream)))
+        return out
+
+    def bi_matmul_grouped(self, a: torch.Tensor, w: torch.Tensor, offsets: torch.Tensor,
+                          out=None, out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+        """Rows offsets[g]..offsets[g+1]-1 of a [rows, K] times w[g] ([G, N, K]
+        bf16, stacked) -> c [rows, N]; offsets int64 [G + 1] on the device."""
+        _need(a, "a", torch.bfloat16)
+        rows, K = a.shape
+        _need(w, "w", torch.bfloat16)
+        G, N, K2 = w.shape
+        if K2 != K:
+            raise ValueError("w must be [groups, N, K] with K = %d" % K)
+        _need(offsets, "offsets", torch.int64, (G + 1,))
+        if out is None:
+            out = torch.empty((rows, N), dtype=out_dtype, device=a.device)
+        _need(out, "out", out_dtype, (rows, N))
+        self._check("bi_matmul_grouped", self.lib.bi_matmul_grouped(
+            _ptr(a), _ptr(w), _ptr(out), _ptr(offsets), G, rows, N, K, _DT[out_dtype],
+            _stream(stream)))
         return out
 
     # ------------------------------------------------------------ KV cache

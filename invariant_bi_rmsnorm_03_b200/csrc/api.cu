@@ -140,6 +140,32 @@ bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H
                                         static_cast<cudaStream_t>(stream)));
 }
 
+bi_status bi_matmul_grouped(const void *a, const void *w, void *c, const int64_t *offsets,
+                            int32_t groups, int64_t rows, int64_t N, int64_t K, bi_dtype out_dtype,
+                            void *stream)
+{
+    if (rows < 0 || N < 1 || K < 1 || N % 8 != 0 || K % 8 != 0) return BI_ERR_INVALID;
+    if (groups < 1 || groups > bi::kMaxGemmGroups) return BI_ERR_INVALID;
+    if (out_dtype != BI_BF16 && out_dtype != BI_F32) return BI_ERR_INVALID;
+    if (rows > INT32_MAX || int64_t(groups) * N > INT32_MAX || K > INT32_MAX) return BI_ERR_INVALID;
+    if (rows == 0) return BI_OK;
+    if (!a || !w || !c || !offsets || !aligned16(a) || !aligned16(w) || !aligned16(c))
+        return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    CUtensorMap ta, tw;
+    const uint64_t da[2] = {uint64_t(K), uint64_t(rows)}, sa[1] = {uint64_t(K) * 2};
+    const uint64_t dw[2] = {uint64_t(K), uint64_t(groups) * uint64_t(N)}, sw[1] = {uint64_t(K) * 2};
+    const uint32_t ba[2] = {uint32_t(bi::kGemmBK), 128u};
+    const uint32_t bw[2] = {uint32_t(bi::kGemmBK), 128u};
+    if (!encode(&ta, a, 2, da, sa, ba) || !encode(&tw, w, 2, dw, sw, bw)) return BI_ERR_CUDA;
+    return from_cuda(bi::launch_gemm_grouped(ta, tw, c, int(rows), int(N), int(K),
+                                             out_dtype == BI_F32, offsets, groups, d->num_sms,
+                                             d->status, bi::kDefaultTimeoutNs,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 bi_status bi_add_rmsnorm(void *x, const void *delta, const void *w, void *y, int64_t M,
                          int64_t H, float eps, bi_dtype out_dtype, void *stream)
 {

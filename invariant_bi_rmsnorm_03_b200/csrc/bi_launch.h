@@ -27,6 +27,13 @@ int gemm_k_splits(int64_t M, int64_t N, int64_t K, int num_sms);
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tw, void *c, int M, int N,
                         int K, bool out_f32, float *ws, int k_splits, int num_sms,
                         unsigned *status, uint64_t timeout_ns, cudaStream_t s);
+// Grouped: group g's rows offsets[g] .. offsets[g+1]-1 of A and C use rows
+// g*N .. g*N+N-1 of W (the groups' weights stacked); offsets on the device.
+constexpr int kMaxGemmGroups = 256;
+cudaError_t launch_gemm_grouped(const CUtensorMap &ta, const CUtensorMap &tw, void *c, int rows,
+                                int N, int K, bool out_f32, const int64_t *offsets, int groups,
+                                int num_sms, unsigned *status, uint64_t timeout_ns,
+                                cudaStream_t s);
 
 // ---------------------------------------------------------------- KV write
 cudaError_t launch_kv_write(void *k_cache, void *v_cache, int64_t num_pages, int Hkv, int d,

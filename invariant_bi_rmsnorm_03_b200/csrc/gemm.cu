@@ -40,6 +40,9 @@ namespace {
 
 struct Unit {
     int mb, nb, split, kb0, kb1;
+    int64_t row0;    // first row of A and C of the tile
+    int64_t row_end; // rows at or past this one are not stored
+    int64_t w_row0;  // first row of W (stacked groups: group * N + column)
 };
 
 __device__ __forceinline__ Unit unit_of(int u, int num_m, int k_splits, int kblocks, int kb_per)
@@ -115,12 +118,48 @@ constexpr int STAGE_BYTES = A_BYTES + W_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;     // two 128-lane x 256-column fp32 accumulators
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+constexpr int CUM_BYTES = (kMaxGemmGroups + 1) * 4;  // grouped mode: tiles before each group
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + CUM_BYTES;
+
+// The tile of work unit u.  Plain: tiles m-fastest over an M x N output
+// (split-K units only in the variant-off build).  Grouped: the rows of group
+// g are offsets[g] .. offsets[g+1]-1 of A and C and its weight is rows
+// g*N .. g*N+N-1 of W; its tiles (m-fastest) follow those of group g-1.
+__device__ __forceinline__ Unit unit_at(int u, int num_m, int num_n, int k_splits, int kblocks,
+                                        int kb_per, int M, int N, const int64_t *goff,
+                                        const int *cum, int groups)
+{
+    if (!goff) {
+        Unit t = unit_of(u, num_m, k_splits, kblocks, kb_per);
+        t.row0 = int64_t(t.mb) * BM;
+        t.row_end = M;
+        t.w_row0 = int64_t(t.nb) * BN;
+        return t;
+    }
+    int g = 0;
+    while (g + 1 < groups && cum[g + 1] <= u) ++g;
+    const int64_t r0 = goff[g], r1 = goff[g + 1];
+    const int mt = int((r1 - r0 + BM - 1) / BM);
+    const int local = u - cum[g];
+    Unit t;
+    t.split = 0;
+    t.kb0 = 0;
+    t.kb1 = kblocks;
+    t.mb = local % mt;
+    t.nb = local / mt;
+    t.row0 = r0 + int64_t(t.mb) * BM;
+    t.row_end = r1;
+    t.w_row0 = int64_t(g) * N + int64_t(t.nb) * BN;
+    (void)num_m;
+    (void)num_n;
+    return t;
+}
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmw,
                      void *__restrict__ c, float *__restrict__ ws, int M, int N, int K, int out_f32,
-                     int k_splits, unsigned *status, uint64_t timeout_ns)
+                     int k_splits, const int64_t *__restrict__ goff, int groups, unsigned *status,
+                     uint64_t timeout_ns)
 {
 #if BI_INVARIANT
     k_splits = 1;  // the invariant build never splits K
@@ -137,10 +176,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint64_t *drain = tempty + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    int *cum = reinterpret_cast<int *>(smem + STAGES * STAGE_BYTES + BAR_BYTES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
+    const int num_n = (N + BN - 1) / BN;
+    if (goff && threadIdx.x == 64) {
+        // tiles before each group (read once: the offsets come from the device)
+        int acc = 0;
+        for (int g = 0; g < groups; ++g) {
+            cum[g] = acc;
+            const int64_t n = goff[g + 1] - goff[g];
+            acc += int((n > 0 ? (n + BM - 1) / BM : 0) * num_n);
+        }
+        cum[groups] = acc;
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -166,10 +217,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const WaitCtl ctl{abort_flag, status, timeout_ns};
 
     const int num_m = (M + BM - 1) / BM;
-    const int num_n = (N + BN - 1) / BN;
     const int kblocks = (K + BK - 1) / BK;
     const int kb_per = (kblocks + k_splits - 1) / k_splits;
-    const int units = num_m * num_n * k_splits;
+    const int units = goff ? cum[groups] : num_m * num_n * k_splits;
+    auto unit = [&](int u) {
+        return unit_at(u, num_m, num_n, k_splits, kblocks, kb_per, M, N, goff, cum, groups);
+    };
     const int pair_id = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
 
     if (warp == 0) {
@@ -179,7 +232,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             uint32_t phase = 0;
             bool ok = true;
             for (int u = pair_id; ok && u < units; u += num_pairs) {
-                const Unit t = unit_of(u, num_m, k_splits, kblocks, kb_per);
+                const Unit t = unit(u);
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
                     if (!wait(&empty[stage], phase ^ 1u, ctl)) {
                         ok = false;
@@ -188,9 +241,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     const uint32_t bar = map_to_cta(smem_u32(&full[stage]), 0);
                     if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
                     tma_load_2d_pair(sA + stage * A_BYTES, &tma, bar, kb * BK,
-                                     t.mb * BM + int(rank) * 128);
+                                     int(t.row0) + int(rank) * 128);
                     tma_load_2d_pair(sW + stage * W_BYTES, &tmw, bar, kb * BK,
-                                     t.nb * BN + int(rank) * 128);
+                                     int(t.w_row0) + int(rank) * 128);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -208,7 +261,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int u = pair_id; ok && u < units; u += num_pairs) {
-                const Unit t = unit_of(u, num_m, k_splits, kblocks, kb_per);
+                const Unit t = unit(u);
                 if (!wait(&tempty[acc], acc_phase ^ 1u, ctl)) {
                     ok = false;
                     break;
@@ -253,17 +306,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int u = pair_id; u < units; u += num_pairs) {
-            const Unit t = unit_of(u, num_m, k_splits, kblocks, kb_per);
+            const Unit t = unit(u);
             if (!wait(&tfull[acc], acc_phase, ctl)) break;
             tc_fence_after();
-            const int64_t row = int64_t(t.mb) * BM + int(rank) * 128 + 32 * q + lane;
+            const int64_t row = t.row0 + int(rank) * 128 + 32 * q + lane;
 #pragma unroll 1
             for (int cc = 0; cc < BN / 32; ++cc) {
                 uint32_t r[32];
                 tmem_ld32(tmem_addr(tmem, 32 * q, acc * BN + cc * 32), r);
                 tmem_wait_ld(r);
                 const int col0 = t.nb * BN + cc * 32;
-                if (row < M && col0 < N)
+                if (row >= 0 && row < M && row < t.row_end && col0 < N)
                     store_row32(r, c, ws, row, col0, N, M, t.split, k_splits, out_f32);
             }
             tc_fence_before();
@@ -332,9 +385,9 @@ int gemm_k_splits(int64_t M, int64_t N, int64_t K, int num_sms)
 #endif
 }
 
-cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tw, void *c, int M, int N,
-                        int K, bool out_f32, float *ws, int k_splits, int num_sms,
-                        unsigned *status, uint64_t timeout_ns, cudaStream_t s)
+// Pairs of SMs that can be resident at once on this device (not every SM can
+// pair up); the persistent grid is this many clusters.
+static cudaError_t resident_pairs(int num_sms, int *out)
 {
     cudaError_t e = cudaFuncSetAttribute(pair::gemm_pair_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -362,11 +415,36 @@ cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tw, void *c, i
         if (e != cudaSuccess) return e;
         max_pairs[dev] = clusters > 0 ? clusters : 1;
     }
+    *out = max_pairs[dev];
+    return cudaSuccess;
+}
+
+cudaError_t launch_gemm_grouped(const CUtensorMap &ta, const CUtensorMap &tw, void *c, int rows,
+                                int N, int K, bool out_f32, const int64_t *offsets, int groups,
+                                int num_sms, unsigned *status, uint64_t timeout_ns,
+                                cudaStream_t s)
+{
+    int pairs = 0;
+    cudaError_t e = resident_pairs(num_sms, &pairs);
+    if (e != cudaSuccess) return e;
+    // the tile count is only known on the device: every resident pair runs
+    pair::gemm_pair_kernel<<<2 * pairs, pair::THREADS, pair::SMEM_BYTES, s>>>(
+        ta, tw, c, nullptr, rows, N, K, out_f32 ? 1 : 0, 1, offsets, groups, status, timeout_ns);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tw, void *c, int M, int N,
+                        int K, bool out_f32, float *ws, int k_splits, int num_sms,
+                        unsigned *status, uint64_t timeout_ns, cudaStream_t s)
+{
+    int max_pairs = 0;
+    cudaError_t e = resident_pairs(num_sms, &max_pairs);
+    if (e != cudaSuccess) return e;
     const int64_t units = int64_t((M + pair::BM - 1) / pair::BM) * ((N + pair::BN - 1) / pair::BN) *
                           k_splits;
-    const int pairs = static_cast<int>(units < max_pairs[dev] ? units : max_pairs[dev]);
+    const int pairs = static_cast<int>(units < max_pairs ? units : max_pairs);
     pair::gemm_pair_kernel<<<2 * pairs, pair::THREADS, pair::SMEM_BYTES, s>>>(
-        ta, tw, c, ws, M, N, K, out_f32 ? 1 : 0, k_splits, status, timeout_ns);
+        ta, tw, c, ws, M, N, K, out_f32 ? 1 : 0, k_splits, nullptr, 0, status, timeout_ns);
     e = cudaGetLastError();
     if (e != cudaSuccess || k_splits <= 1) return e;
     const int64_t MN = int64_t(M) * N;

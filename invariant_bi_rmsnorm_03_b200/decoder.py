@@ -61,11 +61,10 @@ def weight_shapes(cfg: DecoderConfig) -> dict:
         s["l%d.wqkv" % i] = (cfg.qkv_dim, cfg.hidden)
         s["l%d.wo" % i] = (cfg.hidden, cfg.n_heads * cfg.head_dim)
         s["l%d.mlp_norm" % i] = (cfg.hidden,)
-        if cfg.n_experts:
+        if cfg.n_experts:  # the experts' weights stacked: [E, out, in]
             s["l%d.router" % i] = (cfg.n_experts, cfg.hidden)
-            for e in range(cfg.n_experts):
-                s["l%d.e%d.wgu" % (i, e)] = (2 * cfg.expert_ffn, cfg.hidden)
-                s["l%d.e%d.wdown" % (i, e)] = (cfg.hidden, cfg.expert_ffn)
+            s["l%d.moe_wgu" % i] = (cfg.n_experts, 2 * cfg.expert_ffn, cfg.hidden)
+            s["l%d.moe_wdown" % i] = (cfg.n_experts, cfg.hidden, cfg.expert_ffn)
         else:
             s["l%d.wgu" % i] = (2 * cfg.ffn, cfg.hidden)
             s["l%d.wdown" % i] = (cfg.hidden, cfg.ffn)
@@ -313,23 +312,17 @@ class ToyDecoder:
 
     def _moe(self, h: torch.Tensor, i: int):
         """The mixture-of-experts feed-forward of layer i; returns (output,
-        launches).  The expert boundaries are read back to the host to size
-        each expert's matmuls (one synchronisation per layer)."""
+        launches).  All experts' matmuls run in one grouped launch each, their
+        tiles laid out on the device from the dispatch offsets (no host
+        read-back)."""
         L, c, W = self.L, self.cfg, self.w
         logits = L.bi_matmul(h, W["l%d.router" % i], out_dtype=torch.float32)
         experts, gates = L.bi_moe_route(logits, c.top_k)
         off, _, pos, tok = L.bi_moe_dispatch(experts, c.n_experts)
         xs = L.bi_embedding(h, tok)                  # rows grouped by expert
-        ys = torch.empty_like(xs)
-        bounds = off.cpu().tolist()
-        n = 4
-        for e in range(c.n_experts):
-            a, b = bounds[e], bounds[e + 1]
-            if b > a:
-                f = L.bi_swiglu(L.bi_matmul(xs[a:b], W["l%d.e%d.wgu" % (i, e)]))
-                L.bi_matmul(f, W["l%d.e%d.wdown" % (i, e)], out=ys[a:b])
-                n += 3
-        return L.bi_moe_combine(ys, pos, gates), n + 1
+        f = L.bi_swiglu(L.bi_matmul_grouped(xs, W["l%d.moe_wgu" % i], off))
+        ys = L.bi_matmul_grouped(f, W["l%d.moe_wdown" % i], off)
+        return L.bi_moe_combine(ys, pos, gates), 8
 
 
 def run(sched: Scheduler, model: ToyDecoder, max_steps: int = 1_000_000) -> int:

@@ -67,11 +67,11 @@ def test_moe_feed_forward_rows_do_not_depend_on_the_batch(L):
     ex, gw = oracle.moe_route(rl, cfg.top_k)
     acc = np.zeros(cfg.hidden)
     for i, e in enumerate(ex[0]):
-        gu = L.bi_matmul(h[:1], w["l0.e%d.wgu" % e])
+        gu = L.bi_matmul(h[:1], w["l0.moe_wgu"][e])
         f = L.bi_swiglu(gu)
         want_f = oracle.swiglu(host_bits(gu))
         assert rowwise_normwise(to_f64(f), want_f).max() <= TOL_BF16
-        yd = oracle.matmul(host_bits(f), host_bits(w["l0.e%d.wdown" % e]))
+        yd = oracle.matmul(host_bits(f), host_bits(w["l0.moe_wdown"][e]))
         acc += gw[0, i] * yd[0]
     assert rowwise_normwise(to_f64(full[:1]), acc[None]).max() <= TOL_BF16
 
@@ -105,3 +105,26 @@ def test_bad_expert_id_is_flagged_not_faulted(L):
     w = torch.full((2, 2), 0.5, dtype=torch.float32, device=DEV)
     L.bi_moe_combine(y, pos, w)  # the unplaced entry is skipped, not read
     assert L.bi_device_status() == bi.Status.DEVICE_INDEX
+
+
+@pytest.mark.parametrize("sizes", [[0, 1, 255, 256, 257], [513, 0, 0, 2, 100, 700, 31, 1]])
+def test_grouped_matmul_equals_per_group_matmul_bitwise(L, sizes):
+    # every group's rows through one grouped launch give the bits bi_matmul
+    # gives them alone (same tile, same K order), and match the oracle
+    g = rng(200 + len(sizes))
+    G, N, K = len(sizes), 640, 1024
+    rows = int(sum(sizes))
+    a = normal_bf16(g, (rows, K))
+    w = normal_bf16(g, (G, N, K), std=0.02)
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+    ad, wd = dev_bf16(a), dev_bf16(w)
+    c = L.bi_matmul_grouped(ad, wd, torch.from_numpy(off).to(DEV))
+    for gi in range(G):
+        lo, hi = int(off[gi]), int(off[gi + 1])
+        if hi == lo:
+            continue
+        alone = L.bi_matmul(ad[lo:hi].contiguous(), wd[gi])
+        assert same_bytes(c[lo:hi], alone), gi
+        want = oracle.matmul(a[lo:hi], w[gi])
+        assert rowwise_normwise(to_f64(c[lo:hi]), want).max() <= TOL_BF16
+    assert L.bi_device_status() == bi.Status.OK
