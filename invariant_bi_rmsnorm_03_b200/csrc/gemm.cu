@@ -17,7 +17,7 @@
 //
 // Each CTA of a pair: 192 threads, one per SM, persistent over tiles:
 //   warp 0     TMA producer: this CTA's 128 rows of the A slice and 128 rows
-//              of the W slice (128-byte swizzle, 32 KB a stage, 6 stages),
+//              of the W slice (128-byte swizzle, 32 KB a stage, 7 stages),
 //              completing on the leader's barrier
 //   warp 1     TMEM allocation (512 columns: two 128 x 256 fp32
 //              accumulators, the pair allocating together) and, in the
@@ -108,10 +108,10 @@ __device__ __forceinline__ void store_row32(const uint32_t (&r)[32], void *c, fl
 // per 64-wide K slice, its own 128 rows of A and W rows 128r..128r+127 of
 // the tile's 256 columns; the leader (r = 0) issues tcgen05.mma.cta_group::2
 // with M = 256, N = 256, which reads both CTAs' shared memory.  A CTA reads
-// 32 KB per K slice instead of 48, so six stages fit.
+// 32 KB per K slice instead of 48, so seven stages fit.
 namespace pair {
 
-constexpr int BM = 256, BN = 256, BK = kGemmBK, STAGES = 6;
+constexpr int BM = 256, BN = 256, BK = kGemmBK, STAGES = 7;
 constexpr int A_BYTES = 128 * BK * 2;   // 16 KB: this CTA's half of the A slice
 constexpr int W_BYTES = 128 * BK * 2;   // 16 KB: this CTA's half of the W slice
 constexpr int STAGE_BYTES = A_BYTES + W_BYTES;
