@@ -150,27 +150,36 @@ struct Item {
     int pos0;             // prefill: absolute position of the tile's first row
 };
 
-__device__ __forceinline__ bool make_item(const AttnParams &p, Item &it)
+// Work item idx of a launch.  Decode: idx = x + nblk (g + Hkv z), block x of
+// the split range of kv head g of the z-th sequence of the launch order
+// (longest first).  Prefill: idx = h + Hq (xr + tiles b), query head h of
+// tile tiles-1-xr (longest first) of sequence b.  Items past a sequence's
+// end are empty (false).
+__device__ __forceinline__ bool make_item(const AttnParams &p, int idx, Item &it)
 {
     if (p.decode) {
-        it.b = p.order ? p.order[blockIdx.z] : static_cast<int>(blockIdx.z);
-        it.g = blockIdx.y;
+        const int nblk = (p.max_splits + p.splits_per_cta - 1) / p.splits_per_cta;
+        const int x = idx % nblk, r = idx / nblk;
+        const int z = r / p.Hkv;
+        it.b = p.order ? p.order[z] : z;
+        it.g = r - z * p.Hkv;
         it.h = 0;
         it.kv_len = p.seq_lens[it.b];
         it.n_splits = (it.kv_len + kSplit - 1) / kSplit;
-        it.s0 = blockIdx.x * p.splits_per_cta;
+        it.s0 = x * p.splits_per_cta;
         if (it.n_splits > p.max_splits) {  // longer than the declared maximum
-            if (threadIdx.x == 0 && blockIdx.x == 0) record_status(p.status, BI_DEV_BAD_INDEX);
+            if (threadIdx.x == 0) record_status(p.status, BI_DEV_BAD_INDEX);
             return false;
         }
         if (it.kv_len <= 0 || it.s0 >= it.n_splits) return false;
         it.s1 = min(it.n_splits, it.s0 + p.splits_per_cta);
         it.q_row0 = it.rows = it.pos0 = 0;
     } else {
-        it.b = blockIdx.z;
-        it.h = blockIdx.y;
+        const int r = idx / p.Hq;
+        it.h = idx - r * p.Hq;
+        it.b = r / p.num_q_tiles;
         it.g = it.h / p.group;
-        const int tile = p.num_q_tiles - 1 - static_cast<int>(blockIdx.x);  // long tiles first
+        const int tile = p.num_q_tiles - 1 - (r - it.b * p.num_q_tiles);  // long tiles first
         const int q0 = p.cu_q[it.b];
         const int n = p.cu_q[it.b + 1] - q0;
         if (tile * 128 >= n) return false;
@@ -402,9 +411,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     attn_split_kernel(const __grid_constant__ CUtensorMap tq, const AttnParams p)
 {
     using C = Cfg<D>;
-    Item it;
-    if (!make_item(p, it)) return;
-
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t pad = (1024 - (raw & 1023)) & 1023;
@@ -419,10 +425,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint64_t *full = reinterpret_cast<uint64_t *>(sKV + C::NSLOT * C::KV_BYTES);
     uint64_t *empty = full + C::NSLOT;
     uint64_t *barQ = empty + C::NSLOT;
-    uint64_t *barS = barQ + 1;     // [2] S of buffer b computed
-    uint64_t *barP = barS + 2;     // [2] P and (m_s, l_s) of buffer b written (128 arrivals)
-    uint64_t *barO = barP + 2;     // [2] O_s of buffer b computed
-    uint64_t *barF = barO + 2;     // [2] O_s of buffer b merged, buffer free (128 arrivals)
+    uint64_t *barQfree = barQ + 1;  // the item's last QK done: Q may be replaced
+    uint64_t *barS = barQfree + 1;  // [2] S of buffer b computed
+    uint64_t *barP = barS + 2;      // [2] P and (m_s, l_s) of buffer b written (128 arrivals)
+    uint64_t *barO = barP + 2;      // [2] O_s of buffer b computed
+    uint64_t *barF = barO + 2;      // [2] O_s of buffer b merged, buffer free
     uint64_t *drain = barF + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
@@ -434,6 +441,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(barQ, 1);
+        mbar_init(barQfree, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&barS[b], 1);
             mbar_init(&barP[b], 128);
@@ -453,196 +461,219 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
-    const int32_t *bt_row = p.block_table + int64_t(it.b) * p.max_pages;
 
+    // The block serves work items blockIdx.x, blockIdx.x + gridDim.x, ...
+    // (longest first).  Every role walks the same items and counts the
+    // splits it has seen (gs): split number gs uses TMEM buffer gs & 1 with
+    // barrier parity (gs >> 1) & 1, and its loads are numbers 2 gs, 2 gs + 1
+    // of the ring.  An item's last QK releases the Q buffer for the next.
     if (warp == 0) {
         // ====================================================== producer
-        // Loads in the order K(s0), V(s0), K(s0+1), V(s0+1), ...; load i
-        // goes to ring slot i % NSLOT.
         bool ok = true;
         uint32_t armed = 0, armed_parity = 0;
-        if (lane == 0) {
-            if (p.decode) {
-                const int rpq = p.rows_per_q;
-                mbar_arrive_expect_tx(barQ, 4u * C::KB * rpq * 128u);
-                for (int q = 0; q < 4; ++q)
-                    for (int kb = 0; kb < C::KB; ++kb)
-                        tma_load_3d(sQ + kb * C::Q_KB_BYTES + q * 32 * 128, &tq, barQ, kb * 64,
-                                    it.g * p.group + q * rpq, it.b);
-            } else {
-                mbar_arrive_expect_tx(barQ, uint32_t(C::Q_BYTES));
-                for (int kb = 0; kb < C::KB; ++kb)
-                    tma_load_3d(sQ + kb * C::Q_KB_BYTES, &tq, barQ, kb * 64, it.h, it.q_row0);
-            }
-        }
-        // Lane i < 16 looks up page i of a split ahead of use and issues
-        // that page's boxes itself.  The id is only loaded here; it is
-        // checked where it is used, so the load overlaps other work.
-        auto lookup = [&](int s) -> int {
-            const int lp = s * (kSplit / kPage) + lane;  // logical page
-            if (lane >= kSplit / kPage || lp * kPage >= it.kv_len) return -1;
-            return lp < p.max_pages ? __ldg(bt_row + lp) : -2;
-        };
-        // Load list (relative split j, n splits): K0, K1, V0, K2, V1, K3,
-        // ..., V(n-2), V(n-1): keys two splits ahead of values, which is the
-        // order in which the MMA warp consumes them.  Load i goes to ring
-        // slot i % NSLOT.  Lane i < 16 keeps the page ids of the splits in
-        // flight in a 4-entry ring (looked up ahead of use).
-        const int n = it.s1 - it.s0;
-        int slot = 0;
-        uint32_t phase = 0;
-        int pages[4];
+        int gs = 0, nq = 0;
+        int64_t li = 0;  // running load number: slot li % NSLOT
+        for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
+            Item it;
+            if (!make_item(p, idx, it)) continue;
+            const int32_t *bt_row = p.block_table + int64_t(it.b) * p.max_pages;
+            auto lookup = [&](int s) -> int {
+                const int lp = s * (kSplit / kPage) + lane;  // logical page
+                if (lane >= kSplit / kPage || lp * kPage >= it.kv_len) return -1;
+                return lp < p.max_pages ? __ldg(bt_row + lp) : -2;
+            };
+            // Load list (relative split j, n splits): K0, K1, V0, K2, V1, K3,
+            // ..., V(n-2), V(n-1): keys two splits ahead of values, the order
+            // in which the MMA warp consumes them.  Lane i < 16 looks up page
+            // i of a split ahead of use (4 splits in flight) and issues that
+            // page's copy itself; the id is checked where it is used.
+            const int n = it.s1 - it.s0;
+            int pages[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) pages[e] = e < n ? lookup(it.s0 + e) : -1;
-        auto emit = [&](int which, int j) -> bool {
-            const int s = it.s0 + j;
-            int phys = pages[j & 3];
-            if (phys == -2 || phys >= p.num_pages || phys < -1) {  // bad id: zero box, flagged
-                if (which == 0) record_status(p.status, BI_DEV_BAD_INDEX);
-                phys = -1;
-            }
-            const int nk = min(kSplit, it.kv_len - s * kSplit);  // valid keys, >= 1
-            const int full_pages = nk / kPage;
-            const int npages = (nk + kPage - 1) / kPage;
-            int got = 1;
-            if (lane == 0) got = wait(&empty[slot], phase ^ 1u, ctl) ? 1 : 0;
-            got = __shfl_sync(0xffffffffu, got, 0);
-            if (!got) return false;
-            uint8_t *dst = sKV + slot * C::KV_BYTES;
-            const uint8_t *cache = static_cast<const uint8_t *>(which ? p.v_cache : p.k_cache);
-            const int partial_phys = __shfl_sync(0xffffffffu, phys, full_pages & 31);
-            // V: the partial last page is copied by the whole warp, with the
-            // keys past the sequence end set to zero.
-            if (which == 1 && full_pages < npages) {
-                const int pg = full_pages;
-                const bool good = partial_phys >= 0;
-                const int valid = nk - pg * kPage;
-                const uint8_t *blk =
-                    cache + (int64_t(partial_phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
-                for (int e = lane; e < kPage * (D / 8); e += 32) {
-                    const int r = e / (D / 8), c = e % (D / 8);
-                    const uint32_t off = page_off<D>(r, c);
-                    uint4 v = make_uint4(0, 0, 0, 0);
-                    if (good && r < valid) v = __ldg(reinterpret_cast<const uint4 *>(blk + off));
-                    *reinterpret_cast<uint4 *>(dst + pg * C::PAGE_BYTES + off) = v;
+            for (int e = 0; e < 4; ++e) pages[e] = e < n ? lookup(it.s0 + e) : -1;
+            auto emit = [&](int which, int j) -> bool {
+                const int s = it.s0 + j;
+                const int slot = int(li % C::NSLOT);
+                const uint32_t phase = uint32_t(li / C::NSLOT) & 1u;
+                int phys = pages[j & 3];
+                if (phys == -2 || phys >= p.num_pages || phys < -1) {  // bad id: zero page, flagged
+                    if (which == 0) record_status(p.status, BI_DEV_BAD_INDEX);
+                    phys = -1;
                 }
-                fence_proxy_async_smem();
+                const int nk = min(kSplit, it.kv_len - s * kSplit);  // valid keys, >= 1
+                const int full_pages = nk / kPage;
+                const int npages = (nk + kPage - 1) / kPage;
+                int got = 1;
+                if (lane == 0) got = wait(&empty[slot], phase ^ 1u, ctl) ? 1 : 0;
+                got = __shfl_sync(0xffffffffu, got, 0);
+                if (!got) return false;
+                uint8_t *dst = sKV + slot * C::KV_BYTES;
+                const uint8_t *cache = static_cast<const uint8_t *>(which ? p.v_cache : p.k_cache);
+                const int partial_phys = __shfl_sync(0xffffffffu, phys, full_pages & 31);
+                // V: the partial last page is copied by the whole warp, with
+                // the keys past the sequence end set to zero.
+                if (which == 1 && full_pages < npages) {
+                    const int pg = full_pages;
+                    const bool good = partial_phys >= 0;
+                    const int valid = nk - pg * kPage;
+                    const uint8_t *blk =
+                        cache + (int64_t(partial_phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
+                    for (int e = lane; e < kPage * (D / 8); e += 32) {
+                        const int r = e / (D / 8), c = e % (D / 8);
+                        const uint32_t off = page_off<D>(r, c);
+                        uint4 v = make_uint4(0, 0, 0, 0);
+                        if (good && r < valid) v = __ldg(reinterpret_cast<const uint4 *>(blk + off));
+                        *reinterpret_cast<uint4 *>(dst + pg * C::PAGE_BYTES + off) = v;
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                // K: the pages holding valid keys.  V: whole valid pages plus
+                // all-zero pages past the end.  One bulk copy per page.
+                const int copies = which ? (kSplit / kPage) - (npages - full_pages) : npages;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[slot], uint32_t(copies) * C::PAGE_BYTES);
+                    armed |= 1u << slot;
+                    armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
+                }
                 __syncwarp();
-            }
-            // K: the pages holding valid keys.  V: whole valid pages plus
-            // all-zero pages past the end.  One bulk copy per page.
-            const int copies = which ? (kSplit / kPage) - (npages - full_pages) : npages;
+                const int pg = lane;
+                bool issue;
+                const uint8_t *src = g_zero_page;
+                if (which == 0) {
+                    issue = pg < npages;
+                    if (phys >= 0) src = cache + (int64_t(phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
+                } else {
+                    issue = pg < kSplit / kPage && !(pg == full_pages && full_pages < npages);
+                    if (pg < full_pages && phys >= 0)
+                        src = cache + (int64_t(phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
+                }
+                if (issue) bulk_load(dst + pg * C::PAGE_BYTES, src, C::PAGE_BYTES, &full[slot]);
+                __syncwarp();
+                ++li;
+                return true;
+            };
+            // the first keys go out before Q (their slots free up earlier)
+            if (n > 0) ok = emit(0, 0);
+            if (ok && n > 1) ok = emit(0, 1);
+            // Q of this item once the previous item's QK products are done
+            int gotq = 1;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&full[slot], uint32_t(copies) * C::PAGE_BYTES);
-                armed |= 1u << slot;
-                armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
+                if (nq > 0) gotq = wait(barQfree, uint32_t(nq - 1) & 1u, ctl) ? 1 : 0;
+                if (gotq) {
+                    if (p.decode) {
+                        const int rpq = p.rows_per_q;
+                        mbar_arrive_expect_tx(barQ, 4u * C::KB * rpq * 128u);
+                        for (int q = 0; q < 4; ++q)
+                            for (int kb = 0; kb < C::KB; ++kb)
+                                tma_load_3d(sQ + kb * C::Q_KB_BYTES + q * 32 * 128, &tq, barQ,
+                                            kb * 64, it.g * p.group + q * rpq, it.b);
+                    } else {
+                        mbar_arrive_expect_tx(barQ, uint32_t(C::Q_BYTES));
+                        for (int kb = 0; kb < C::KB; ++kb)
+                            tma_load_3d(sQ + kb * C::Q_KB_BYTES, &tq, barQ, kb * 64, it.h, it.q_row0);
+                    }
+                }
             }
-            __syncwarp();
-            const int pg = lane;
-            bool issue;
-            const uint8_t *src = g_zero_page;
-            if (which == 0) {
-                issue = pg < npages;
-                if (phys >= 0) src = cache + (int64_t(phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
-            } else {
-                issue = pg < kSplit / kPage && !(pg == full_pages && full_pages < npages);
-                if (pg < full_pages && phys >= 0)
-                    src = cache + (int64_t(phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
+            gotq = __shfl_sync(0xffffffffu, gotq, 0);
+            ok = ok && gotq;
+            ++nq;
+            for (int j = 0; ok && j < n; ++j) {
+                ok = emit(1, j);
+                // split j is done with its page ids: look up split j + 4
+                pages[j & 3] = (j + 4 < n) ? lookup(it.s0 + j + 4) : -1;
+                if (ok && j + 2 < n) ok = emit(0, j + 2);
             }
-            if (issue) bulk_load(dst + pg * C::PAGE_BYTES, src, C::PAGE_BYTES, &full[slot]);
-            __syncwarp();
-            if (++slot == C::NSLOT) {
-                slot = 0;
-                phase ^= 1u;
-            }
-            return true;
-        };
-        if (n > 0) ok = emit(0, 0);
-        if (ok && n > 1) ok = emit(0, 1);
-        for (int j = 0; ok && j < n; ++j) {
-            ok = emit(1, j);
-            // split j is done with its page ids: look up split j + 4
-            pages[j & 3] = (j + 4 < n) ? lookup(it.s0 + j + 4) : -1;
-            if (ok && j + 2 < n) ok = emit(0, j + 2);
+            gs += n;
         }
         if (!ok && lane == 0) {
             for (int s = 0; s < C::NSLOT; ++s)
                 if (armed & (1u << s)) wait_drain(&full[s], (armed_parity >> s) & 1u, p.timeout_ns);
-            wait_drain(barQ, 0, p.timeout_ns);
+            if (nq > 0) wait_drain(barQ, uint32_t(nq - 1) & 1u, p.timeout_ns);
         }
+        (void)gs;
     } else if (warp == 1) {
         // ====================================================== MMA issue
-        // Tensor-pipe order: QK(s0), QK(s0+1), PV(s0), QK(s0+2), PV(s0+1),
-        // ... -- the order of the producer's load list; split s uses TMEM
-        // buffer (s - s0) & 1, which QK(s+2) reuses once the fold warps
-        // have merged O_s(s).
+        // Per item, tensor-pipe order QK(0), QK(1), PV(0), QK(2), PV(1), ...
+        // -- the order of the producer's load list.  QK of split gs reuses
+        // TMEM buffer gs & 1 once the fold warps have merged split gs - 2,
+        // which may belong to the previous item.
         if (lane == 0) {
             const uint32_t idesc_qk = idesc_bf16_f32(128, kSplit, 0, 0);
             const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t q_base = smem_u32(sQ);
-            bool ok = wait(barQ, 0, ctl);
-            // index of each load in the producer's list K0, K1, V0, K2, V1, ...
-            const int n = it.s1 - it.s0;
-            auto k_index = [](int j) { return j < 2 ? j : 2 * j - 1; };
-            auto v_index = [n](int j) { return min(2 + 2 * j, 2 * n - 1); };
-            auto issue_qk = [&](int s) -> bool {
-                const int i = k_index(s - it.s0);
-                const int slot = i % C::NSLOT;
-                if (!wait(&full[slot], uint32_t(i / C::NSLOT) & 1u, ctl)) return false;
-                tc_fence_after();
-                const uint32_t d = tmem + C::BUF_COLS * uint32_t((s - it.s0) & 1);
-                const uint32_t k_base = smem_u32(sKV + slot * C::KV_BYTES);
+            bool ok = true;
+            int gs = 0, nq = 0;
+            for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
+                Item it;
+                if (!make_item(p, idx, it)) continue;
+                const int n = it.s1 - it.s0;
+                const int64_t base = 2 * int64_t(gs);  // load number of K0
+                // load numbers of K(j) and V(j) in the list K0, K1, V0, K2, V1, ...
+                auto k_load = [&](int j) { return base + (j < 2 ? j : 2 * j - 1); };
+                auto v_load = [&](int j) { return base + min(2 + 2 * j, 2 * n - 1); };
+                auto issue_qk = [&](int j) -> bool {
+                    const int g = gs + j;
+                    if (g >= 2) {  // buffer g & 1 still holds split g - 2 until merged
+                        if (!wait(&barF[g & 1], uint32_t((g - 2) >> 1) & 1u, ctl)) return false;
+                        tc_fence_after();
+                    }
+                    const int64_t i = k_load(j);
+                    const int slot = int(i % C::NSLOT);
+                    if (!wait(&full[slot], uint32_t(i / C::NSLOT) & 1u, ctl)) return false;
+                    tc_fence_after();
+                    const uint32_t d = tmem + C::BUF_COLS * uint32_t(g & 1);
+                    const uint32_t k_base = smem_u32(sKV + slot * C::KV_BYTES);
 #pragma unroll
-                for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t kb = k >> 2, kk = k & 3;
-                    // K: K-major, core matrices; 16 values of the head dim
-                    // are two core matrices 128 bytes apart, 8-key groups
-                    // are KGROUP_BYTES apart (also across pages).
-                    mma_ss(d, sdesc_sw128(q_base + kb * C::Q_KB_BYTES + kk * 32, 16, 1024),
-                           sdesc_plain(k_base + k * 256, 128, C::KGROUP_BYTES), idesc_qk,
-                           k > 0 ? 1u : 0u);
-                }
-                mma_commit(&barS[(s - it.s0) & 1]);
-                mma_commit(&empty[slot]);
-                return true;
-            };
-            if (ok) ok = issue_qk(it.s0);
-            if (ok && it.s0 + 1 < it.s1) ok = issue_qk(it.s0 + 1);
-            for (int s = it.s0; ok && s < it.s1; ++s) {
-                const int b = (s - it.s0) & 1;
-                const uint32_t par = uint32_t((s - it.s0) >> 1) & 1u;
-                const int i = v_index(s - it.s0);
-                const int slot = i % C::NSLOT;
-                if (!wait(&full[slot], uint32_t(i / C::NSLOT) & 1u, ctl)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t buf = tmem + C::BUF_COLS * uint32_t(b);
-                const uint32_t v_base = smem_u32(sKV + slot * C::KV_BYTES);
-                if (!wait(&barP[b], par, ctl)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-#pragma unroll
-                for (int j = 0; j < kSplit / 16; ++j) {
-                    // V: MN-major, core matrices; step j is page j; its two
-                    // 8-key groups are KGROUP_BYTES apart, 8-value blocks of
-                    // the head dim 128 bytes apart.
-                    mma_ts(buf + C::O_OFF, buf + C::P_OFF + 8 * j,
-                           sdesc_plain(v_base + j * C::PAGE_BYTES, C::KGROUP_BYTES, 128), idesc_pv,
-                           j > 0 ? 1u : 0u);
-                }
-                mma_commit(&barO[b]);
-                mma_commit(&empty[slot]);
-                if (s + 2 < it.s1) {
-                    if (!wait(&barF[b], par, ctl)) {
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint32_t kb = k >> 2, kk = k & 3;
+                        // K: K-major, core matrices; 16 values of the head
+                        // dim are two core matrices 128 bytes apart, 8-key
+                        // groups KGROUP_BYTES apart (also across pages).
+                        mma_ss(d, sdesc_sw128(q_base + kb * C::Q_KB_BYTES + kk * 32, 16, 1024),
+                               sdesc_plain(k_base + k * 256, 128, C::KGROUP_BYTES), idesc_qk,
+                               k > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&barS[g & 1]);
+                    mma_commit(&empty[slot]);
+                    if (j == n - 1) mma_commit(barQfree);  // the item's last use of Q
+                    return true;
+                };
+                ok = wait(barQ, uint32_t(nq) & 1u, ctl);
+                ++nq;
+                if (ok) ok = issue_qk(0);
+                if (ok && n > 1) ok = issue_qk(1);
+                for (int j = 0; ok && j < n; ++j) {
+                    const int g = gs + j;
+                    const int b = g & 1;
+                    const uint32_t par = uint32_t(g >> 1) & 1u;
+                    const int64_t i = v_load(j);
+                    const int slot = int(i % C::NSLOT);
+                    if (!wait(&full[slot], uint32_t(i / C::NSLOT) & 1u, ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t buf = tmem + C::BUF_COLS * uint32_t(b);
+                    const uint32_t v_base = smem_u32(sKV + slot * C::KV_BYTES);
+                    if (!wait(&barP[b], par, ctl)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    ok = issue_qk(s + 2);
+#pragma unroll
+                    for (int jj = 0; jj < kSplit / 16; ++jj) {
+                        // V: MN-major, core matrices; step jj is page jj;
+                        // its two 8-key groups are KGROUP_BYTES apart,
+                        // 8-value blocks of the head dim 128 bytes apart.
+                        mma_ts(buf + C::O_OFF, buf + C::P_OFF + 8 * jj,
+                               sdesc_plain(v_base + jj * C::PAGE_BYTES, C::KGROUP_BYTES, 128),
+                               idesc_pv, jj > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&barO[b]);
+                    mma_commit(&empty[slot]);
+                    if (j + 2 < n) ok = issue_qk(j + 2);
                 }
+                gs += n;
             }
             if (!ok) {
                 mma_commit(drain);
@@ -655,164 +686,174 @@ __global__ void __launch_bounds__(THREADS, 1)
         // half of the head dim) serve the same 32 rows.
         const bool is_softmax = warp >= 4 && warp < 8;
         const int q = warp & 3;
-        bool valid, active;
-        int t, local;
-        int64_t out_row;
-        if (p.decode) {
-            local = q * p.rows_per_q + lane;
-            valid = lane < p.rows_per_q && local < p.group;
-            t = it.kv_len - 1;
-            const int head = it.g * p.group + local;
-            out_row = int64_t(it.b) * p.Hq + head;
-            active = q * p.rows_per_q < p.group;
-        } else {
-            local = 32 * q + lane;
-            valid = local < it.rows;
-            t = it.pos0 + local;
-            out_row = int64_t(it.q_row0 + local) * p.Hq + it.h;
-            active = 32 * q < it.rows;
-        }
         const uint32_t lane_base = tmem_addr(tmem, 32 * q, 0);
         const int row_id = 32 * q + lane;  // TMEM lane of this row
-
-        if (is_softmax) {
-            // -------------------------------------------------- softmax
-            const float cs = p.scale_log2;
-            const uint32_t quarter_base = tmem_addr(tmem, 32 * q, 0);
-            // decode with at most 8 query rows per quarter: the 16-lane path
-            const bool heads16 = p.decode && p.rows_per_q <= 8 && active;
-            for (int s = it.s0; s < it.s1; ++s) {
-                const int b = (s - it.s0) & 1;
-                const uint32_t par = uint32_t((s - it.s0) >> 1) & 1u;
-                const uint32_t sb = lane_base + C::BUF_COLS * uint32_t(b);
-                if (!wait(&barS[b], par, ctl)) break;
-                tc_fence_after();
-                float m_s = -INFINITY, l_s = 0.0f;
-                if (heads16) {
-                    // rows of this quarter in lanes 0..7, four threads a row
-                    softmax_heads16(quarter_base + C::BUF_COLS * uint32_t(b) + C::P_OFF, s * kSplit,
-                                    t, cs, m_s, l_s);
-                    if ((lane & 3) == 0) {
-                        sML[(b * 128 + 32 * q + (lane >> 2)) * 2 + 0] = m_s;
-                        sML[(b * 128 + 32 * q + (lane >> 2)) * 2 + 1] = l_s;
-                    }
-                } else {
-                    if (active) softmax_rows(sb + C::P_OFF, s * kSplit, t, cs, m_s, l_s);
-                    sML[(b * 128 + row_id) * 2 + 0] = m_s;
-                    sML[(b * 128 + row_id) * 2 + 1] = l_s;
-                }
-                tc_fence_before();
-                mbar_arrive(&barP[b]);
+        int gs = 0;
+        bool ok = true;
+        for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
+            Item it;
+            if (!make_item(p, idx, it)) continue;
+            bool valid, active;
+            int t, local;
+            int64_t out_row;
+            if (p.decode) {
+                local = q * p.rows_per_q + lane;
+                valid = lane < p.rows_per_q && local < p.group;
+                t = it.kv_len - 1;
+                const int head = it.g * p.group + local;
+                out_row = int64_t(it.b) * p.Hq + head;
+                active = q * p.rows_per_q < p.group;
+            } else {
+                local = 32 * q + lane;
+                valid = local < it.rows;
+                t = it.pos0 + local;
+                out_row = int64_t(it.q_row0 + local) * p.Hq + it.h;
+                active = 32 * q < it.rows;
             }
-        } else {
-            // -------------------------------------------------- fold
-            // This warp merges columns col0 .. col0 + HW - 1 of its rows.
-            constexpr int HW = D / 2;
-            const int half = warp >= 10 ? 1 : 0;
-            const int col0 = half * HW;
-#if BI_INVARIANT
-            // blocks after a sequence's first write every split's own partial
-            const bool spill = p.decode && it.s0 > 0;
-#else
-            // variant-off: every block merges its own range (the grouping of
-            // the merge then depends on how many blocks served the sequence)
-            const bool spill = false;
-#endif
-            float m = -INFINITY, l = 0.0f;
-            float O[HW];
-#pragma unroll
-            for (int j = 0; j < HW; ++j) O[j] = 0.0f;
-            bool ok = true;
-            for (int s = it.s0; s < it.s1; ++s) {
-                const int b = (s - it.s0) & 1;
-                const uint32_t par = uint32_t((s - it.s0) >> 1) & 1u;
-                const uint32_t ob = lane_base + C::BUF_COLS * uint32_t(b) + C::O_OFF + col0;
-                const int k0 = s * kSplit;
-                // barP: (m_s, l_s) of this split are in shared memory;
-                // barO: O_s is in TMEM.
-                if (!wait(&barP[b], par, ctl) || !wait(&barO[b], par, ctl)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const float m_s = sML[(b * 128 + row_id) * 2 + 0];
-                const float l_s = sML[(b * 128 + row_id) * 2 + 1];
-                if (active) {
-                    // 32-column TMEM loads (HW / 32 per split)
-                    constexpr int NCH32 = HW / 32;
-                    if (spill) {
-                        // not the first block of this sequence: write the
-                        // split's own partial for attn_combine
-                        float *rec = p.ws + ((out_row * p.max_splits) + s) * C::REC + 4 + col0;
-#pragma unroll 1
-                        for (int c = 0; c < NCH32; ++c) {
-                            uint32_t r[32];
-                            tmem_ld32(ob + 32 * c, r);
-                            tmem_wait_ld(r);
-                            if (valid) {
-#pragma unroll
-                                for (int j = 0; j < 8; ++j)
-                                    reinterpret_cast<float4 *>(rec + 32 * c)[j] = make_float4(
-                                        __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                        __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-                            }
-                        }
-                        if (valid && half == 0) {
-                            rec[-4] = m_s;
-                            rec[-3] = l_s;
+            if (is_softmax) {
+                // -------------------------------------------------- softmax
+                const float cs = p.scale_log2;
+                // decode with at most 8 query rows per quarter: the 16-lane path
+                const bool heads16 = p.decode && p.rows_per_q <= 8 && active;
+                for (int s = it.s0; s < it.s1; ++s) {
+                    const int g = gs + (s - it.s0);
+                    const int b = g & 1;
+                    const uint32_t par = uint32_t(g >> 1) & 1u;
+                    const uint32_t sb = lane_base + C::BUF_COLS * uint32_t(b);
+                    if (!wait(&barS[b], par, ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    float m_s = -INFINITY, l_s = 0.0f;
+                    if (heads16) {
+                        // rows of this quarter in lanes 0..7, four threads a row
+                        softmax_heads16(lane_base + C::BUF_COLS * uint32_t(b) + C::P_OFF,
+                                        s * kSplit, t, cs, m_s, l_s);
+                        if ((lane & 3) == 0) {
+                            sML[(b * 128 + 32 * q + (lane >> 2)) * 2 + 0] = m_s;
+                            sML[(b * 128 + 32 * q + (lane >> 2)) * 2 + 1] = l_s;
                         }
                     } else {
-                        const bool first = (s == it.s0);
-                        const bool take = k0 <= t;  // the row sees at least key k0
-                        float mn, a, cc;
-                        merge_scales(m, m_s, mn, a, cc);
+                        if (active) softmax_rows(sb + C::P_OFF, s * kSplit, t, cs, m_s, l_s);
+                        sML[(b * 128 + row_id) * 2 + 0] = m_s;
+                        sML[(b * 128 + row_id) * 2 + 1] = l_s;
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&barP[b]);
+                }
+            } else {
+                // -------------------------------------------------- fold
+                // This warp merges columns col0 .. col0 + HW - 1 of its rows.
+                constexpr int HW = D / 2;
+                const int half = warp >= 10 ? 1 : 0;
+                const int col0 = half * HW;
+#if BI_INVARIANT
+                // blocks after a sequence's first write every split's own partial
+                const bool spill = p.decode && it.s0 > 0;
+#else
+                // variant-off: every block merges its own range (the grouping
+                // of the merge then depends on how many blocks served it)
+                const bool spill = false;
+#endif
+                float m = -INFINITY, l = 0.0f;
+                float O[HW];
 #pragma unroll
-                        for (int c = 0; c < NCH32; ++c) {
-                            uint32_t r[32];
-                            tmem_ld32(ob + 32 * c, r);
-                            tmem_wait_ld(r);
+                for (int j = 0; j < HW; ++j) O[j] = 0.0f;
+                for (int s = it.s0; s < it.s1; ++s) {
+                    const int g = gs + (s - it.s0);
+                    const int b = g & 1;
+                    const uint32_t par = uint32_t(g >> 1) & 1u;
+                    const uint32_t ob = lane_base + C::BUF_COLS * uint32_t(b) + C::O_OFF + col0;
+                    const int k0 = s * kSplit;
+                    // barP: (m_s, l_s) of this split are in shared memory;
+                    // barO: O_s is in TMEM.
+                    if (!wait(&barP[b], par, ctl) || !wait(&barO[b], par, ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const float m_s = sML[(b * 128 + row_id) * 2 + 0];
+                    const float l_s = sML[(b * 128 + row_id) * 2 + 1];
+                    if (active) {
+                        // 32-column TMEM loads (HW / 32 per split)
+                        constexpr int NCH32 = HW / 32;
+                        if (spill) {
+                            // not the first block of this sequence: write the
+                            // split's own partial for attn_combine
+                            float *rec = p.ws + ((out_row * p.max_splits) + s) * C::REC + 4 + col0;
+#pragma unroll 1
+                            for (int c = 0; c < NCH32; ++c) {
+                                uint32_t r[32];
+                                tmem_ld32(ob + 32 * c, r);
+                                tmem_wait_ld(r);
+                                if (valid) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                const float o = __uint_as_float(r[j]);
-                                if (first)
-                                    O[32 * c + j] = o;
-                                else if (take)
-                                    O[32 * c + j] = merge_val(O[32 * c + j], a, o, cc);
+                                    for (int j = 0; j < 8; ++j)
+                                        reinterpret_cast<float4 *>(rec + 32 * c)[j] = make_float4(
+                                            __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                            __uint_as_float(r[4 * j + 2]),
+                                            __uint_as_float(r[4 * j + 3]));
+                                }
+                            }
+                            if (valid && half == 0) {
+                                rec[-4] = m_s;
+                                rec[-3] = l_s;
+                            }
+                        } else {
+                            const bool first = (s == it.s0);
+                            const bool take = k0 <= t;  // the row sees at least key k0
+                            float mn, a, cc;
+                            merge_scales(m, m_s, mn, a, cc);
+#pragma unroll
+                            for (int c = 0; c < NCH32; ++c) {
+                                uint32_t r[32];
+                                tmem_ld32(ob + 32 * c, r);
+                                tmem_wait_ld(r);
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) {
+                                    const float o = __uint_as_float(r[j]);
+                                    if (first)
+                                        O[32 * c + j] = o;
+                                    else if (take)
+                                        O[32 * c + j] = merge_val(O[32 * c + j], a, o, cc);
+                                }
+                            }
+                            if (first) {
+                                m = m_s;
+                                l = l_s;
+                            } else if (take) {
+                                l = merge_val(l, a, l_s, cc);
+                                m = mn;
                             }
                         }
-                        if (first) {
-                            m = m_s;
-                            l = l_s;
-                        } else if (take) {
-                            l = merge_val(l, a, l_s, cc);
-                            m = mn;
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&barF[b]);
+                }
+                if (ok && active && valid && !spill) {
+                    if (!p.decode || (it.s0 == 0 && it.s1 == it.n_splits)) {
+                        write_out<HW>(O, l, m,
+                                      static_cast<__nv_bfloat16 *>(p.o) + out_row * D + col0,
+                                      (p.lse && half == 0) ? p.lse + out_row : nullptr);
+                    } else {
+                        // a block of a sequence served by several: hand the
+                        // merged state over its range (ending at split s1-1)
+                        // to attn_combine (in the invariant build only the
+                        // first block gets here; the others write every split)
+                        float *rec = p.ws + ((out_row * p.max_splits) + (it.s1 - 1)) * C::REC;
+                        if (half == 0) {
+                            rec[0] = m;
+                            rec[1] = l;
                         }
-                    }
-                }
-                tc_fence_before();
-                mbar_arrive(&barF[b]);
-            }
-
-            if (ok && active && valid && !spill) {
-                if (!p.decode || (it.s0 == 0 && it.s1 == it.n_splits)) {
-                    write_out<HW>(O, l, m, static_cast<__nv_bfloat16 *>(p.o) + out_row * D + col0,
-                                  (p.lse && half == 0) ? p.lse + out_row : nullptr);
-                } else {
-                    // a block of a sequence served by several: hand the
-                    // merged state over its range (ending at split s1-1) to
-                    // attn_combine (in the invariant build only the first
-                    // block gets here; the others write every split)
-                    float *rec = p.ws + ((out_row * p.max_splits) + (it.s1 - 1)) * C::REC;
-                    if (half == 0) {
-                        rec[0] = m;
-                        rec[1] = l;
-                    }
 #pragma unroll
-                    for (int j = 0; j < HW / 4; ++j)
-                        reinterpret_cast<float4 *>(rec + 4 + col0)[j] =
-                            make_float4(O[4 * j], O[4 * j + 1], O[4 * j + 2], O[4 * j + 3]);
+                        for (int j = 0; j < HW / 4; ++j)
+                            reinterpret_cast<float4 *>(rec + 4 + col0)[j] =
+                                make_float4(O[4 * j], O[4 * j + 1], O[4 * j + 2], O[4 * j + 3]);
+                    }
                 }
             }
+            gs += it.s1 - it.s0;
         }
     }
 
@@ -922,14 +963,35 @@ size_t attn_ws_bytes(int B, int Hq, int head_dim, int max_splits, int max_chunks
     return size_t(B) * Hq * max_splits * (head_dim + 4) * sizeof(float);
 }
 
-cudaError_t launch_attention(const CUtensorMap &tq, const AttnParams &p, int head_dim,
+cudaError_t launch_attention(const CUtensorMap &tq, const AttnParams &p_in, int head_dim,
                              cudaStream_t s)
 {
-    dim3 grid;
+    // Prefill: persistent, one block per SM (at most), each walking items
+    // blockIdx.x, blockIdx.x + gridDim.x, ... (longest first; the tiles'
+    // lengths fall in steps, so the static assignment stays balanced, and a
+    // block's next item overlaps the current one's tail).  Decode: one block
+    // per item -- request lengths vary too much for a static assignment, and
+    // the hardware hands each free SM the next block of the longest-first
+    // order.
+    AttnParams p = p_in;
+    int64_t items;
     if (p.decode)
-        grid = dim3((p.max_splits + p.splits_per_cta - 1) / p.splits_per_cta, p.Hkv, p.B);
+        items = int64_t((p.max_splits + p.splits_per_cta - 1) / p.splits_per_cta) * p.Hkv * p.B;
     else
-        grid = dim3(p.num_q_tiles, p.Hq, p.B);
+        items = int64_t(p.num_q_tiles) * p.Hq * p.B;
+    if (items > INT32_MAX) return cudaErrorInvalidValue;
+    p.items = static_cast<int32_t>(items);
+    if (p.items == 0) return cudaSuccess;
+    static int sms[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (sms[dev] == 0) {
+        cudaError_t e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+    }
+    const unsigned grid =
+        static_cast<unsigned>(p.decode ? p.items : (p.items < sms[dev] ? p.items : sms[dev]));
     cudaError_t e;
     if (head_dim == 128) {
         e = cudaFuncSetAttribute(attn_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,

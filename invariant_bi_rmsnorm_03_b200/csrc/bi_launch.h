@@ -62,6 +62,7 @@ struct AttnParams {
     int32_t splits_per_cta;    // decode work division
     int32_t max_splits;        // decode: splits of the longest sequence
     int32_t num_q_tiles;       // prefill: tiles of the longest chunk
+    int32_t items;             // work items of the launch (set by launch_attention)
     float scale_log2;          // softmax scale * log2(e)
     // outputs
     void *o;
