@@ -65,6 +65,9 @@ class Oracle:
         lib.oracle_moe_route.argtypes = [P, i64, i32, i32, P, P]
         lib.oracle_moe_dispatch.argtypes = [P, i64, i32, P, P, P]
         lib.oracle_moe_combine.argtypes = [P, P, P, i64, i32, i64, P]
+        lib.oracle_fold_norm_weight.argtypes = [P, P, i64, i64, P]
+        lib.oracle_rmsnorm_matmul.argtypes = [P, P, i64, i64, i64, f64, P]
+        lib.oracle_matmul_residual.argtypes = [P, P, P, i64, i64, i64, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
@@ -242,6 +245,38 @@ class Oracle:
         self.lib.oracle_moe_combine(_p(y), _p(ps), _p(w), T, k, H, _p(out))
         return out
 
+    # ---------------------------------------------------------- fused matmuls
+
+    def fold_norm_weight(self, W, w) -> np.ndarray:
+        """wf[n, k] = W[n, k] * w[k]; W [N, K], w [K] (bf16 bits) -> float64."""
+        W, w = _u16(W), _u16(w)
+        N, K = W.shape
+        assert w.shape == (K,)
+        out = np.empty((N, K), dtype=np.float64)
+        self.lib.oracle_fold_norm_weight(_p(W), _p(w), N, K, _p(out))
+        return out
+
+    def rmsnorm_matmul(self, x, wf, eps: float) -> np.ndarray:
+        """C = RMSNorm(x) @ wf.T with the norm weight already in wf; x [M, K],
+        wf [N, K] (bf16 bits) -> float64 [M, N]."""
+        x, wf = _u16(x), _u16(wf)
+        M, K = x.shape
+        N, K2 = wf.shape
+        assert K == K2
+        c = np.empty((M, N), dtype=np.float64)
+        self.lib.oracle_rmsnorm_matmul(_p(x), _p(wf), M, N, K, float(eps), _p(c))
+        return c
+
+    def matmul_residual(self, r, a, w) -> np.ndarray:
+        """C = R + A @ W.T; r [M, N], a [M, K], w [N, K] (bf16 bits) -> float64."""
+        r, a, w = _u16(r), _u16(a), _u16(w)
+        M, K = a.shape
+        N, K2 = w.shape
+        assert K == K2 and r.shape == (M, N)
+        c = np.empty((M, N), dtype=np.float64)
+        self.lib.oracle_matmul_residual(_p(r), _p(a), _p(w), M, N, K, _p(c))
+        return c
+
 
 def default() -> Oracle:
     global _lib
@@ -314,6 +349,18 @@ def moe_dispatch(experts, E: int):
 
 def moe_combine(y, pos, weights) -> np.ndarray:
     return default().moe_combine(y, pos, weights)
+
+
+def fold_norm_weight(W, w) -> np.ndarray:
+    return default().fold_norm_weight(W, w)
+
+
+def rmsnorm_matmul(x, wf, eps: float) -> np.ndarray:
+    return default().rmsnorm_matmul(x, wf, eps)
+
+
+def matmul_residual(r, a, w) -> np.ndarray:
+    return default().matmul_residual(r, a, w)
 
 
 def decode_rows(q, seq_lens, heads=None):

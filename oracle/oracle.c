@@ -504,3 +504,66 @@ void oracle_moe_combine(const uint16_t *y, const int64_t *pos, const double *wei
         }
     }
 }
+
+/*
+ * Fused forms of the adjacent RMSNorm and matmul steps (xitu-tech news,
+ * "构建确定性解决方案": the RMSNorm item followed by the matmul item; each
+ * transformer block normalises a row and multiplies it by a weight).
+ *
+ * Norm weight folded into a matmul weight:
+ *   wf[n, k] = W[n, k] * w[k]
+ * (the product of two bfloat16 values, exact in double).
+ */
+void oracle_fold_norm_weight(const uint16_t *W, const uint16_t *w, int64_t N, int64_t K,
+                             double *wf)
+{
+    int64_t n;
+#pragma omp parallel for schedule(static)
+    for (n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            wf[n * K + k] = bf16_to_double(W[n * K + k]) * bf16_to_double(w[k]);
+}
+
+/*
+ * RMSNorm (weight folded into wf) followed by the matrix product:
+ *   y[m, k] = x[m, k] / sqrt( (1/K) * sum_i x[m, i]^2 + eps )
+ *   C[m, n] = sum_k y[m, k] * wf[n, k]             x: [M, K], wf: [N, K]
+ */
+void oracle_rmsnorm_matmul(const uint16_t *x, const uint16_t *wf, int64_t M, int64_t N,
+                           int64_t K, double eps, double *c)
+{
+    int64_t m;
+#pragma omp parallel for schedule(static)
+    for (m = 0; m < M; ++m) {
+        const uint16_t *xm = x + m * K;
+        double sum_sq = 0.0;
+        for (int64_t i = 0; i < K; ++i) sum_sq += bf16_to_double(xm[i]) * bf16_to_double(xm[i]);
+        const double root = sqrt(sum_sq / (double)K + eps);
+        for (int64_t n = 0; n < N; ++n) {
+            const uint16_t *wn = wf + n * K;
+            double s = 0.0;
+            for (int64_t k = 0; k < K; ++k) s += (bf16_to_double(xm[k]) / root) * bf16_to_double(wn[k]);
+            c[m * N + n] = s;
+        }
+    }
+}
+
+/*
+ * Matrix product added to the residual stream (the residual connection of a
+ * transformer block):
+ *   C[m, n] = R[m, n] + sum_k A[m, k] * W[n, k]    R: [M, N], A: [M, K], W: [N, K]
+ */
+void oracle_matmul_residual(const uint16_t *r, const uint16_t *a, const uint16_t *w, int64_t M,
+                            int64_t N, int64_t K, double *c)
+{
+    int64_t m;
+#pragma omp parallel for schedule(static)
+    for (m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double dot = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                dot += bf16_to_double(a[m * K + k]) * bf16_to_double(w[n * K + k]);
+            c[m * N + n] = bf16_to_double(r[m * N + n]) + dot;
+        }
+    }
+}

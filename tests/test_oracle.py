@@ -579,3 +579,95 @@ def test_moe_combine_closed_forms(oracle):
     np.testing.assert_array_equal(out[0], yf[3])
     np.testing.assert_allclose(out[1], 0.25 * yf[5] + 0.75 * yf[1], rtol=1e-15)
     np.testing.assert_allclose(out[2], 0.5 * (yf[2] + yf[4]), rtol=1e-15)
+
+
+# ---------------------------------------------------------------- fused matmuls
+
+
+def test_fold_norm_weight_closed_forms(oracle):
+    g = rng(80)
+    W = normal_bf16(g, (6, 20), std=0.02)
+    # w = 1 leaves W; powers of two scale exactly; a one-hot w keeps one column
+    np.testing.assert_array_equal(oracle.fold_norm_weight(W, bf(np.ones(20))), widen(W))
+    p2 = 2.0 ** np.arange(-4, 16)
+    np.testing.assert_array_equal(oracle.fold_norm_weight(W, bf(p2)), widen(W) * p2[None, :])
+    one = np.zeros(20)
+    one[13] = 1.0
+    got = oracle.fold_norm_weight(W, bf(one))
+    assert np.count_nonzero(got[:, np.arange(20) != 13]) == 0
+    np.testing.assert_array_equal(got[:, 13], widen(W)[:, 13])
+
+
+def test_fold_norm_weight_small_integers(oracle):
+    # N=3, K=4: distinct sizes, so indexing w by the row fails
+    W = np.array([[1, -2, 3, 4], [0, 5, -6, 7], [8, 1, 2, -3]])
+    w = np.array([2, -1, 3, 5])
+    got = oracle.fold_norm_weight(bf(W), bf(w))
+    for n in range(3):
+        for k in range(4):
+            assert got[n, k] == W[n, k] * w[k]
+
+
+def test_rmsnorm_matmul_hand_example(oracle):
+    # x = [3, 4]: mean square 12.5; with eps = 0 each output is (w . x) / sqrt(12.5)
+    c = oracle.rmsnorm_matmul(bf([[3, 4]]), bf([[1, 1], [1, -1], [2, 0]]), 0.0)
+    np.testing.assert_allclose(c[0], np.array([7.0, -1.0, 6.0]) / math.sqrt(12.5), rtol=1e-15)
+
+
+def test_rmsnorm_matmul_one_hot_rows_closed_form(oracle):
+    # row m = v e_j: mean square v^2 / K, so C[m, n] = v / sqrt(v^2/K + eps) * wf[n, j].
+    # v = 2^-10 makes eps (1e-6) dominate v^2 / K, so a dropped or misplaced eps shows.
+    g = rng(81)
+    K, N = 64, 9
+    wf = normal_bf16(g, (N, K), std=0.5)
+    cols = [0, 17, 63]
+    vals = [2.0 ** -10, -3.0, 40.0]
+    x = np.zeros((3, K))
+    for m, (j, v) in enumerate(zip(cols, vals)):
+        x[m, j] = v
+    c = oracle.rmsnorm_matmul(bf(x), wf, 1e-6)
+    for m, (j, v) in enumerate(zip(cols, vals)):
+        np.testing.assert_allclose(c[m], v / math.sqrt(v * v / K + 1e-6) * widen(wf)[:, j],
+                                   rtol=1e-13)
+
+
+def test_rmsnorm_matmul_scale_invariance_without_eps(oracle):
+    g = rng(82)
+    x = normal_bf16(g, (4, 48))
+    wf = normal_bf16(g, (5, 48), std=0.1)
+    x2 = bf(widen(x) * 8.0)
+    np.testing.assert_allclose(oracle.rmsnorm_matmul(x, wf, 0.0),
+                               oracle.rmsnorm_matmul(x2, wf, 0.0), rtol=1e-13)
+
+
+def test_rmsnorm_matmul_matches_torch_fp64(oracle):
+    g = rng(83)
+    x = normal_bf16(g, (6, 72))
+    wf = normal_bf16(g, (11, 72), std=0.05)
+    xt = torch.from_numpy(widen(x))
+    y = torch.nn.functional.rms_norm(xt, (72,), eps=1e-6)
+    want = y @ torch.from_numpy(widen(wf)).T
+    np.testing.assert_allclose(oracle.rmsnorm_matmul(x, wf, 1e-6), want.numpy(), rtol=1e-11,
+                               atol=1e-14)
+
+
+def test_matmul_residual_small_integers_brute_force(oracle):
+    # M=2, N=3, K=4, all distinct, so a transposed operand or residual fails
+    g = rng(84)
+    R = g.integers(-20, 21, size=(2, 3))
+    A = g.integers(-5, 6, size=(2, 4))
+    W = g.integers(-5, 6, size=(3, 4))
+    c = oracle.matmul_residual(bf(R), bf(A), bf(W))
+    for m in range(2):
+        for n in range(3):
+            assert c[m, n] == R[m, n] + sum(int(A[m, k]) * int(W[n, k]) for k in range(4))
+
+
+def test_matmul_residual_degenerate_cases(oracle):
+    g = rng(85)
+    R = normal_bf16(g, (5, 24))
+    A = normal_bf16(g, (5, 16))
+    W = normal_bf16(g, (24, 16), std=0.1)
+    np.testing.assert_array_equal(oracle.matmul_residual(R, A, bf(np.zeros((24, 16)))), widen(R))
+    np.testing.assert_allclose(oracle.matmul_residual(bf(np.zeros((5, 24))), A, W),
+                               oracle.matmul(A, W), rtol=1e-15)

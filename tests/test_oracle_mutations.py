@@ -27,7 +27,8 @@ MUTATIONS = [
     ("matmul_transposed_weight", "s += bf16_to_double(am[k]) * bf16_to_double(wn[k]);",
      "s += bf16_to_double(am[k]) * bf16_to_double(w[k * N + n]);",
      [pins.test_matmul_small_integers_brute_force, pins.test_matmul_matches_torch_fp64]),
-    ("matmul_drops_last_k", "for (int64_t k = 0; k < K; ++k)", "for (int64_t k = 0; k < K - 1; ++k)",
+    ("matmul_drops_last_k", "for (int64_t k = 0; k < K; ++k)\n                s += bf16_to_double(am[k])",
+     "for (int64_t k = 0; k < K - 1; ++k)\n                s += bf16_to_double(am[k])",
      [pins.test_matmul_identity_weight, pins.test_matmul_hand_example]),
     ("kv_write_wrong_offset", "off = slot % ORACLE_PAGE", "off = (slot + 1) % ORACLE_PAGE",
      [pins.test_kv_write_matches_direct_scatter]),
@@ -93,6 +94,25 @@ MUTATIONS = [
     ("argmax_ties_take_highest_index", "if (row[j] > row[best]) best = j;",
      "if (row[j] >= row[best]) best = j;",
      [pins.test_argmax_ties_take_the_lowest_index, pins.test_argmax_matches_numpy_first_occurrence]),
+    ("fold_indexes_w_by_row", "* bf16_to_double(w[k]);", "* bf16_to_double(w[n % K]);",
+     [pins.test_fold_norm_weight_closed_forms, pins.test_fold_norm_weight_small_integers]),
+    ("rmsnorm_matmul_drops_eps", "sqrt(sum_sq / (double)K + eps)", "sqrt(sum_sq / (double)K)",
+     [pins.test_rmsnorm_matmul_one_hot_rows_closed_form]),
+    ("rmsnorm_matmul_mean_over_n", "sqrt(sum_sq / (double)K + eps)", "sqrt(sum_sq / (double)N + eps)",
+     [pins.test_rmsnorm_matmul_hand_example, pins.test_rmsnorm_matmul_one_hot_rows_closed_form]),
+    ("rmsnorm_matmul_not_normalised", "s += (bf16_to_double(xm[k]) / root) * bf16_to_double(wn[k]);",
+     "s += bf16_to_double(xm[k]) * bf16_to_double(wn[k]);",
+     [pins.test_rmsnorm_matmul_hand_example, pins.test_rmsnorm_matmul_matches_torch_fp64]),
+    ("rmsnorm_matmul_transposed_weight",
+     "s += (bf16_to_double(xm[k]) / root) * bf16_to_double(wn[k]);",
+     "s += (bf16_to_double(xm[k]) / root) * bf16_to_double(wf[(k * N + n) % (N * K)]);",
+     [pins.test_rmsnorm_matmul_hand_example, pins.test_rmsnorm_matmul_matches_torch_fp64]),
+    ("matmul_residual_drops_residual", "c[m * N + n] = bf16_to_double(r[m * N + n]) + dot;",
+     "c[m * N + n] = dot;",
+     [pins.test_matmul_residual_small_integers_brute_force, pins.test_matmul_residual_degenerate_cases]),
+    ("matmul_residual_transposed_residual", "c[m * N + n] = bf16_to_double(r[m * N + n]) + dot;",
+     "c[m * N + n] = bf16_to_double(r[(n * M + m) % (M * N)]) + dot;",
+     [pins.test_matmul_residual_small_integers_brute_force, pins.test_matmul_residual_degenerate_cases]),
 ]
 
 
