@@ -698,6 +698,27 @@ def run_profile_case(args):
             fn = lambda i: L.bi_rmsnorm(xs[i % 16], w, 1e-6)  # noqa: E731
         else:
             fn = lambda i: L.bi_matmul(x, W)  # noqa: E731
+    elif args.profile in ("rmsnorm_matmul", "rmsnorm_then_matmul", "matmul_residual",
+                          "matmul_rows"):
+        # fused forms against their unfused launches, M = --profile-rows rows
+        # of hidden 4096 times N = 12288; two weight copies rotate (201 MB > L2)
+        M = args.profile_rows
+        nm = norm_matmul(seed=1, M=M, H=H, N=N_COLS)
+        x, w = d16(nm["x"]), d16(nm["w"])
+        Ws = [d16(nm["W"]), d16(norm_matmul(seed=11, M=1, H=H, N=N_COLS)["W"])]
+        c = T.empty((M, N_COLS), dtype=T.bfloat16, device=dev)
+        if args.profile == "rmsnorm_matmul":
+            wfs = [L.bi_fold_norm_weight(W, w) for W in Ws]
+            fn = lambda i: L.bi_rmsnorm_matmul(x, wfs[i % 2], 1e-6, out=c)  # noqa: E731
+        elif args.profile == "rmsnorm_then_matmul":
+            y = T.empty_like(x)
+            fn = lambda i: L.bi_matmul(L.bi_rmsnorm(x, w, 1e-6, out=y), Ws[i % 2],  # noqa: E731
+                                       out=c)
+        elif args.profile == "matmul_residual":
+            r = d16(normal_bf16(rng(12), (M, N_COLS)))
+            fn = lambda i: L.bi_matmul_residual(x, Ws[i % 2], r, out=c)  # noqa: E731
+        else:
+            fn = lambda i: L.bi_matmul(x, Ws[i % 2], out=c)  # noqa: E731
     elif args.profile == "sample":
         # 256 rows of lm_head logits (vocab 32000), temperature 0.8, nucleus 0.95
         g = rng(5)
@@ -746,11 +767,11 @@ def run_profile_case(args):
 def run_unique_completions(args):
     print(json.dumps(unique_completions(args.targets, args.others, args.max_batch,
                                         args.token_budget, args.span, args.temperature,
-                                        args.top_p, args.moe)), flush=True)
+                                        args.top_p, args.moe, args.fused)), flush=True)
 
 
 def unique_completions(targets, others, max_batch=256, token_budget=2048, span=2000,
-                       temperature=0.0, top_p=1.0, moe=False) -> dict:
+                       temperature=0.0, top_p=1.0, moe=False, fused=False) -> dict:
     """One fixed 64-token prompt completed greedily (256 tokens) many times
     amid random other requests, on the 8-layer hidden-4096 random-init
     decoder: the number of distinct completions for the invariant and the
@@ -766,7 +787,7 @@ def unique_completions(targets, others, max_batch=256, token_budget=2048, span=2
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     # dense: SwiGLU 14336; mixture of experts: 16 experts of SwiGLU 1408, top 4
-    cfg = DecoderConfig(n_experts=16, top_k=4, expert_ffn=1408) if moe else DecoderConfig()
+    cfg = DecoderConfig(n_experts=16, top_k=4, expert_ffn=1408) if moe else DecoderConfig(fused=fused)
     weights = toy_decoder_weights(weight_shapes(cfg), seed=4, device=dev)
     prompt, spec = unique_completion_workload(seed=4, n_target=targets, n_other=others,
                                               vocab=cfg.vocab, steps_span=span)
@@ -778,6 +799,8 @@ def unique_completions(targets, others, max_batch=256, token_budget=2048, span=2
               "prompt_tokens": 64, "new_tokens": 256, "targets": targets,
               "others": others, "max_batch": max_batch,
               "token_budget": token_budget, "data": "synthetic",
+              "fused": ("RMSNorm folded into the next matmul, residual adds in the matmul "
+                        "epilogue" if cfg.fused else False),
               "sampling": ("greedy" if temperature <= 0 else
                            {"temperature": temperature, "top_p": top_p,
                             "seed": "one per request; every target copy the same"})}
@@ -840,10 +863,13 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=20.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--profile", choices=["rmsnorm", "matmul", "decode", "prefill", "copy",
-                                          "sample"],
+                                          "sample", "rmsnorm_matmul", "rmsnorm_then_matmul",
+                                          "matmul_residual", "matmul_rows"],
                     help="run one kernel alone on a reduced case (for ncu)")
     ap.add_argument("--profile-batch", type=int, default=32)
     ap.add_argument("--profile-seq", type=int, default=4096)
+    ap.add_argument("--profile-rows", type=int, default=M_ROWS,
+                    help="rows of the fused-matmul --profile cases")
     ap.add_argument("--variant", action="store_true", help="--profile the variant-off build")
     ap.add_argument("--unique-completions", action="store_true",
                     help="run the toy-decoder unique-completion experiment instead")
@@ -857,6 +883,8 @@ def main(argv=None):
     ap.add_argument("--top-p", type=float, default=1.0)
     ap.add_argument("--moe", action="store_true",
                     help="unique-completion run on the mixture-of-experts decoder")
+    ap.add_argument("--fused", action="store_true",
+                    help="unique-completion run with the fused RMSNorm/residual matmuls")
     ap.add_argument("--uc-targets", type=int, default=200,
                     help="target copies (and as many others) of the in-bench unique-completion "
                          "check; 0 skips it")

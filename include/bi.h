@@ -167,6 +167,48 @@ bi_status bi_matmul_grouped(const void *a, const void *w, void *c, const int64_t
                             void *stream);
 
 /*
+ * Fused forms of the RMSNorm and residual steps around a transformer block's
+ * matmuls (the RMSNorm item beside the matmul item of xitu-tech news,
+ * "构建确定性解决方案").  Both run the bi_matmul product (same tiles, same
+ * K order, no split-K in either build) and change only its epilogue, row by
+ * row, so every row stays independent of M.
+ *
+ * bi_fold_norm_weight -- wf[n, k] = round(W[n, k] * w[k]): a matmul weight
+ *   with the preceding RMSNorm's weight folded in (once, at load time).
+ *   W, wf : device, bf16 [N, K];  w : device, bf16 [K].  K % 8 == 0, N >= 0,
+ *   16-byte aligned; wf may be W (in place), no other overlap.  The product
+ *   of two bf16 values is exact in fp32, so wf is the correctly rounded
+ *   product.
+ *
+ * bi_rmsnorm_matmul -- RMSNorm of each row of x followed by the product with
+ *   a folded weight, in one launch:
+ *
+ *     r[m]    = rsqrt( (1/K) * sum_k x[m, k]^2 + eps )          (fp32)
+ *     C[m, n] = round( r[m] * sum_k x[m, k] * wf[n, k] )
+ *
+ *   x : device, bf16 [M, K];  wf : device, bf16 [N, K];  c : device, [M, N]
+ *   of out_dtype.  The sum of squares is taken from the A tiles already in
+ *   shared memory (K ascending, eight fixed partial sums), so x is read
+ *   once; the normalised row is never rounded to bf16.  Requirements as
+ *   bi_matmul, and eps finite and >= 0.
+ *
+ * bi_matmul_residual -- the product added to a residual stream:
+ *
+ *     C[m, n] = round( R[m, n] + round( sum_k A[m, k] * W[n, k] ) )
+ *
+ *   (the inner rounding is bi_matmul's, so the result equals bi_matmul
+ *   followed by the addition bit for bit).  a : bf16 [M, K];  w : bf16
+ *   [N, K];  r, c : bf16 [M, N], c may be r (in place), no other overlap.
+ *   Requirements as bi_matmul.
+ */
+bi_status bi_fold_norm_weight(const void *W, const void *w, void *wf, int64_t N, int64_t K,
+                              void *stream);
+bi_status bi_rmsnorm_matmul(const void *x, const void *wf, void *c, int64_t M, int64_t N,
+                            int64_t K, float eps, bi_dtype out_dtype, void *stream);
+bi_status bi_matmul_residual(const void *a, const void *w, const void *r, void *c, int64_t M,
+                             int64_t N, int64_t K, void *stream);
+
+/*
  * bi_kv_write -- write the step's new keys and values into the paged cache
  * before attention runs, so that the attention kernel sees one consistent
  * KV layout (neican.ai insight, "技术原理与创新点解析", batch-invariant

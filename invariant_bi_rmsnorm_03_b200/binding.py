@@ -110,7 +110,8 @@ class Library:
                "bi_status_string", "bi_build_invariant", "bi_device_status",
                "bi_debug_bounded_wait", "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write",
                "bi_swiglu", "bi_argmax", "bi_sample", "bi_moe_route", "bi_moe_dispatch",
-               "bi_moe_combine", "bi_matmul_grouped")
+               "bi_moe_combine", "bi_matmul_grouped", "bi_fold_norm_weight",
+               "bi_rmsnorm_matmul", "bi_matmul_residual")
 
     def __init__(self, path: str):
         if not os.path.exists(path):
@@ -149,11 +150,15 @@ class Library:
         L.bi_moe_dispatch.argtypes = [P, i64, i32, i32, P, P, P, P, P]
         L.bi_moe_combine.argtypes = [P, P, P, i64, i32, i64, P, P]
         L.bi_matmul_grouped.argtypes = [P, P, P, P, i32, i64, i64, i64, st, P]
+        L.bi_fold_norm_weight.argtypes = [P, P, P, i64, i64, P]
+        L.bi_rmsnorm_matmul.argtypes = [P, P, P, i64, i64, i64, f32, st, P]
+        L.bi_matmul_residual.argtypes = [P, P, P, P, i64, i64, i64, P]
         for name in ("bi_rmsnorm", "bi_matmul", "bi_kv_write", "bi_attention_decode",
                      "bi_attention_prefill", "bi_device_status", "bi_debug_bounded_wait",
                      "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write", "bi_swiglu",
                      "bi_argmax", "bi_sample", "bi_moe_route", "bi_moe_dispatch",
-                     "bi_moe_combine", "bi_matmul_grouped"):
+                     "bi_moe_combine", "bi_matmul_grouped", "bi_fold_norm_weight",
+                     "bi_rmsnorm_matmul", "bi_matmul_residual"):
             getattr(L, name).restype = st
         self.lib = L
 
@@ -227,6 +232,58 @@ class Library:
         self._check("bi_matmul", self.lib.bi_matmul(_ptr(a), _ptr(w), _ptr(out), M, N, K,
                                                     _DT[out_dtype], _ptr(ws), nbytes,
                                                     _stream(stream)))
+        return out
+
+    def bi_fold_norm_weight(self, W: torch.Tensor, w: torch.Tensor, out=None,
+                            stream=None) -> torch.Tensor:
+        """wf = round(W * w[None, :]) for W [N, K] and w [K] (bf16)."""
+        _need(W, "W", torch.bfloat16)
+        N, K = W.shape
+        _need(w, "w", torch.bfloat16, (K,))
+        if out is None:
+            out = torch.empty_like(W)
+        _need(out, "out", torch.bfloat16, (N, K))
+        self._check("bi_fold_norm_weight",
+                    self.lib.bi_fold_norm_weight(_ptr(W), _ptr(w), _ptr(out), N, K,
+                                                 _stream(stream)))
+        return out
+
+    def bi_rmsnorm_matmul(self, x: torch.Tensor, wf: torch.Tensor, eps: float, out=None,
+                          out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+        """C = RMSNorm(x) @ wf.T in one launch; x [M, K], wf [N, K] the weight with
+        the norm weight folded in (bi_fold_norm_weight)."""
+        _need(x, "x", torch.bfloat16)
+        M, K = x.shape
+        _need(wf, "wf", torch.bfloat16)
+        N = wf.shape[0]
+        if wf.shape[1] != K:
+            raise ValueError("wf must be [N, K] with K = %d" % K)
+        if out is None:
+            out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+        _need(out, "out", out_dtype, (M, N))
+        self._check("bi_rmsnorm_matmul",
+                    self.lib.bi_rmsnorm_matmul(_ptr(x), _ptr(wf), _ptr(out), M, N, K, float(eps),
+                                               _DT[out_dtype], _stream(stream)))
+        return out
+
+    def bi_matmul_residual(self, a: torch.Tensor, w: torch.Tensor, r: torch.Tensor, out=None,
+                           stream=None) -> torch.Tensor:
+        """C = round(r + round(a @ w.T)); a [M, K], w [N, K], r [M, N] (bf16).
+        ``out`` may be ``r`` (in place); by default the result goes to a new
+        tensor."""
+        _need(a, "a", torch.bfloat16)
+        M, K = a.shape
+        _need(w, "w", torch.bfloat16)
+        N = w.shape[0]
+        if w.shape[1] != K:
+            raise ValueError("w must be [N, K] with K = %d" % K)
+        _need(r, "r", torch.bfloat16, (M, N))
+        if out is None:
+            out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+        _need(out, "out", torch.bfloat16, (M, N))
+        self._check("bi_matmul_residual",
+                    self.lib.bi_matmul_residual(_ptr(a), _ptr(w), _ptr(r), _ptr(out), M, N, K,
+                                                _stream(stream)))
         return out
 
     def bi_matmul_grouped(self, a: torch.Tensor, w: torch.Tensor, offsets: torch.Tensor,

@@ -166,6 +166,73 @@ bi_status bi_matmul_grouped(const void *a, const void *w, void *c, const int64_t
                                              static_cast<cudaStream_t>(stream)));
 }
 
+static bool gemm_shape_ok(int64_t M, int64_t N, int64_t K)
+{
+    return M >= 0 && N >= 1 && K >= 1 && N % 8 == 0 && K % 8 == 0 && M <= INT32_MAX &&
+           N <= INT32_MAX && K <= INT32_MAX;
+}
+
+static bi_status gemm_maps(const void *a, const void *w, int64_t M, int64_t N, int64_t K,
+                           CUtensorMap *ta, CUtensorMap *tw)
+{
+    const uint64_t da[2] = {uint64_t(K), uint64_t(M)}, sa[1] = {uint64_t(K) * 2};
+    const uint64_t dw[2] = {uint64_t(K), uint64_t(N)}, sw[1] = {uint64_t(K) * 2};
+    // each CTA of a pair loads 128 rows of A and 128 rows of W per K slice
+    const uint32_t box[2] = {uint32_t(bi::kGemmBK), 128u};
+    if (!encode(ta, a, 2, da, sa, box) || !encode(tw, w, 2, dw, sw, box)) return BI_ERR_CUDA;
+    return BI_OK;
+}
+
+bi_status bi_fold_norm_weight(const void *W, const void *w, void *wf, int64_t N, int64_t K,
+                              void *stream)
+{
+    if (N < 0 || K < 8 || K % 8 != 0) return BI_ERR_INVALID;
+    if (N == 0) return BI_OK;
+    if (!W || !w || !wf || !aligned16(W) || !aligned16(w) || !aligned16(wf)) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_fold_norm_weight(W, w, wf, N, K, d->num_sms,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
+bi_status bi_rmsnorm_matmul(const void *x, const void *wf, void *c, int64_t M, int64_t N,
+                            int64_t K, float eps, bi_dtype out_dtype, void *stream)
+{
+    if (!gemm_shape_ok(M, N, K)) return BI_ERR_INVALID;
+    if (out_dtype != BI_BF16 && out_dtype != BI_F32) return BI_ERR_INVALID;
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return BI_ERR_INVALID;
+    if (M == 0) return BI_OK;
+    if (!x || !wf || !c || !aligned16(x) || !aligned16(wf) || !aligned16(c)) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    CUtensorMap ta, tw;
+    if ((st = gemm_maps(x, wf, M, N, K, &ta, &tw)) != BI_OK) return st;
+    bi::GemmEpi epi{1, eps, nullptr};
+    return from_cuda(bi::launch_gemm_fused(ta, tw, c, int(M), int(N), int(K), out_dtype == BI_F32,
+                                           epi, d->num_sms, d->status, bi::kDefaultTimeoutNs,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+bi_status bi_matmul_residual(const void *a, const void *w, const void *r, void *c, int64_t M,
+                             int64_t N, int64_t K, void *stream)
+{
+    if (!gemm_shape_ok(M, N, K)) return BI_ERR_INVALID;
+    if (M == 0) return BI_OK;
+    if (!a || !w || !r || !c || !aligned16(a) || !aligned16(w) || !aligned16(r) || !aligned16(c))
+        return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    CUtensorMap ta, tw;
+    if ((st = gemm_maps(a, w, M, N, K, &ta, &tw)) != BI_OK) return st;
+    bi::GemmEpi epi{0, 0.0f, r};
+    return from_cuda(bi::launch_gemm_fused(ta, tw, c, int(M), int(N), int(K), false, epi,
+                                           d->num_sms, d->status, bi::kDefaultTimeoutNs,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
 bi_status bi_add_rmsnorm(void *x, const void *delta, const void *w, void *y, int64_t M,
                          int64_t H, float eps, bi_dtype out_dtype, void *stream)
 {

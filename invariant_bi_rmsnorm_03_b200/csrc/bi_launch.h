@@ -34,6 +34,20 @@ cudaError_t launch_gemm_grouped(const CUtensorMap &ta, const CUtensorMap &tw, vo
                                 int N, int K, bool out_f32, const int64_t *offsets, int groups,
                                 int num_sms, unsigned *status, uint64_t timeout_ns,
                                 cudaStream_t s);
+// Fused epilogues of the plain product (never split along K):
+//   norm:     C[m, :] = round(rsqrt(mean_k A[m, k]^2 + eps) * acc[m, :])
+//   residual: C[m, :] = round(R[m, :] + round(acc[m, :]))   (R may be C)
+struct GemmEpi {
+    int norm;
+    float eps;
+    const void *residual;
+};
+cudaError_t launch_gemm_fused(const CUtensorMap &ta, const CUtensorMap &tw, void *c, int M, int N,
+                              int K, bool out_f32, const GemmEpi &epi, int num_sms,
+                              unsigned *status, uint64_t timeout_ns, cudaStream_t s);
+// wf[n, k] = round(W[n, k] * w[k])
+cudaError_t launch_fold_norm_weight(const void *W, const void *w, void *wf, int64_t N, int64_t K,
+                                    int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- KV write
 cudaError_t launch_kv_write(void *k_cache, void *v_cache, int64_t num_pages, int Hkv, int d,

@@ -124,6 +124,12 @@ __device__ __forceinline__ void fence_proxy_async_smem()
 
 // ---------------------------------------------------------------- TMA
 
+// Brings the 128-byte line holding p into L2 (no register is written).
+__device__ __forceinline__ void prefetch_l2(const void *p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const void *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -379,6 +385,16 @@ __device__ __forceinline__ uint32_t map_to_cta(uint32_t saddr, uint32_t rank)
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+// The same with relaxed ordering: it orders none of this thread's earlier
+// memory operations, and does not stall the thread for the round trip a
+// release across CTAs takes.  For forwarding a completion that carries no
+// data of this thread's own.
+__device__ __forceinline__ void mbar_arrive_relaxed_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                  : "memory");
 }
 

@@ -25,6 +25,25 @@
 //   warps 2-5  epilogue: tcgen05.ld of this CTA's accumulator rows (each warp
 //              its 32-lane quarter), fp32 -> bf16 rounding, global stores;
 //              the second accumulator lets the next tile's MMAs run meanwhile.
+//
+// Fused forms (the RMSNorm and residual steps around a transformer block's
+// matmuls, adjacent to the matmul item of xitu-tech news, "构建确定性解决方案"):
+//   norm      C[m, :] = rsqrt(mean_k A[m, k]^2 + eps) * (A W^T)[m, :], with the
+//             norm weight folded into W beforehand.  Four more warps (6-9)
+//             per CTA read each A slice of their CTA as soon as it lands,
+//             while the MMAs run, adding the squares of their row (one row
+//             per thread, K ascending, eight fixed partial sums); a stage is
+//             refilled only after they have read it, and the epilogue scales
+//             its row by the resulting rsqrt.  No second pass over A, and the
+//             MMA operands are the stored bf16 values.  The peer's A slice
+//             completes on a barrier of its own, so that its norm warps can
+//             see it; the peer's otherwise idle MMA warp forwards each
+//             completion to the leader's barrier with a relaxed arrive (a
+//             release arrive across the pair stalls the arriving thread for
+//             about a microsecond, which would throttle the pipeline).
+//   residual  C[m, :] = round(R[m, :] + round(acc[m, :])), R read in the
+//             epilogue (it may be C itself).
+// Neither changes the K order of the product; both are per-row.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -101,6 +120,43 @@ __device__ __forceinline__ void store_row32(const uint32_t (&r)[32], void *c, fl
     }
 }
 
+// The residual row[col0 .. col0+31] (pieces past N read as zero).
+__device__ __forceinline__ void load_res32(const void *res, int64_t row, int col0, int N,
+                                           uint4 (&v)[4])
+{
+    const uint4 *src =
+        reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(res) + row * N + col0);
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+        v[g] = (col0 + 8 * g < N) ? __ldcs(src + g) : make_uint4(0u, 0u, 0u, 0u);
+}
+
+// out[row, col0 .. col0+31] = round(res + round(acc)) in bf16, res loaded
+// beforehand (it may be c itself).
+__device__ __forceinline__ void store_row32_res(const uint32_t (&r)[32], void *c,
+                                                const uint4 (&rv)[4], int64_t row, int col0, int N)
+{
+    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(c) + row * N + col0;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        if (col0 + 8 * g < N) {
+            const uint32_t ru[4] = {rv[g].x, rv[g].y, rv[g].z, rv[g].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                // round the product to bf16 first, as a separate matmul would
+                const uint32_t p = pack_bf16x2(__uint_as_float(r[8 * g + 2 * j]),
+                                               __uint_as_float(r[8 * g + 2 * j + 1]));
+                const float lo = __fadd_rn(__uint_as_float(ru[j] << 16), __uint_as_float(p << 16));
+                const float hi = __fadd_rn(__uint_as_float(ru[j] & 0xFFFF0000u),
+                                           __uint_as_float(p & 0xFFFF0000u));
+                o[j] = pack_bf16x2(lo, hi);
+            }
+            *reinterpret_cast<uint4 *>(dst + 8 * g) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ 2-SM kernel
 //
 // One 256 x 256 output tile per pair of SMs (a cluster of two CTAs): CTA r
@@ -116,9 +172,13 @@ constexpr int A_BYTES = 128 * BK * 2;   // 16 KB: this CTA's half of the A slice
 constexpr int W_BYTES = 128 * BK * 2;   // 16 KB: this CTA's half of the W slice
 constexpr int STAGE_BYTES = A_BYTES + W_BYTES;
 constexpr int THREADS = 192;
+constexpr int FUSED_THREADS = 320;      // + warps 6-9: the row sums of squares (norm form)
 constexpr uint32_t TMEM_COLS = 512;     // two 128-lane x 256-column fp32 accumulators
 constexpr int BAR_BYTES = 256;
-constexpr int CUM_BYTES = (kMaxGemmGroups + 1) * 4;  // grouped mode: tiles before each group
+constexpr int CUM_BYTES = (kMaxGemmGroups + 1) * 4;  // grouped mode: tiles before each group;
+                                                    // norm form: two 128-row rsqrt buffers
+static_assert(CUM_BYTES >= 2 * 128 * 4, "the rsqrt buffers share the group table's room");
+static_assert((3 * STAGES + 9) * 8 + 8 <= BAR_BYTES, "barriers, TMEM address and abort flag");
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + CUM_BYTES;
 
 // The tile of work unit u.  Plain: tiles m-fastest over an M x N output
@@ -155,15 +215,23 @@ __device__ __forceinline__ Unit unit_at(int u, int num_m, int num_n, int k_split
     return t;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+template <bool FUSED>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FUSED ? FUSED_THREADS : THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmw,
-                     void *__restrict__ c, float *__restrict__ ws, int M, int N, int K, int out_f32,
-                     int k_splits, const int64_t *__restrict__ goff, int groups, unsigned *status,
-                     uint64_t timeout_ns)
+                     void *c, float *__restrict__ ws, int M, int N, int K, int out_f32,
+                     int k_splits, const int64_t *__restrict__ goff, int groups, GemmEpi epi,
+                     unsigned *status, uint64_t timeout_ns)
 {
 #if BI_INVARIANT
     k_splits = 1;  // the invariant build never splits K
 #endif
+    // fused forms: plain tiles only (no groups, no split K)
+    const bool nrm = FUSED && epi.norm;
+    const void *res = FUSED ? epi.residual : nullptr;
+    if (FUSED) {
+        k_splits = 1;
+        goff = nullptr;
+    }
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
@@ -174,9 +242,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 2;   // leader's used: 8 arrivals (4 epilogue warps x 2 CTAs)
     uint64_t *drain = tempty + 2;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *afull = drain + 1;       // norm form, peer: its own A slice landed
+    uint64_t *rfull = afull + STAGES;  // norm form: rsqrt buffer written (4 norm warps)
+    uint64_t *rempty = rfull + 2;      // norm form: rsqrt buffer read (4 epilogue warps)
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(rempty + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
     int *cum = reinterpret_cast<int *>(smem + STAGES * STAGE_BYTES + BAR_BYTES);
+    float *rsq = reinterpret_cast<float *>(cum);  // norm form: [2][128]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -195,12 +267,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            // norm form: the leader's full also counts the peer's forward, and a
+            // stage is free once the MMAs and the 4 norm warps have read it
+            mbar_init(&full[s], nrm ? 2 : 1);
+            mbar_init(&empty[s], nrm ? 5 : 1);
+            mbar_init(&afull[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
             mbar_init(&tempty[a], 8);
+            mbar_init(&rfull[a], 4);
+            mbar_init(&rempty[a], 4);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -239,8 +316,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         break;
                     }
                     const uint32_t bar = map_to_cta(smem_u32(&full[stage]), 0);
-                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
-                    tma_load_2d_pair(sA + stage * A_BYTES, &tma, bar, kb * BK,
+                    // norm form: the peer's A slice completes on its own barrier
+                    uint32_t abar = bar;
+                    if (leader) {
+                        mbar_arrive_expect_tx(&full[stage],
+                                              nrm ? 2 * STAGE_BYTES - A_BYTES : 2 * STAGE_BYTES);
+                    } else if (nrm) {
+                        mbar_arrive_expect_tx(&afull[stage], A_BYTES);
+                        abar = map_to_cta(smem_u32(&afull[stage]), rank);
+                    }
+                    tma_load_2d_pair(sA + stage * A_BYTES, &tma, abar, kb * BK,
                                      int(t.row0) + int(rank) * 128);
                     tma_load_2d_pair(sW + stage * W_BYTES, &tmw, bar, kb * BK,
                                      int(t.w_row0) + int(rank) * 128);
@@ -252,6 +337,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
         }
     } else if (warp == 1) {
+        if (nrm && lane == 0 && !leader) {
+            // ------------------------------------ norm form, peer: forward
+            // each landed A slice of this CTA to the leader's full barrier
+            const uint32_t full_leader = map_to_cta(smem_u32(&full[0]), 0);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int u = pair_id; ok && u < units; u += num_pairs) {
+                const Unit t = unit(u);
+                for (int kb = t.kb0; kb < t.kb1; ++kb) {
+                    if (!wait(&afull[stage], phase, ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_relaxed_cluster(full_leader + 8u * uint32_t(stage));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
         if (lane == 0 && leader) {
             // ------------------------------------------------ MMA issue (leader)
             const uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
@@ -298,7 +405,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 wait_drain(drain, 0, timeout_ns);
             }
         }
-    } else {
+    } else if (warp < 6) {
         // ---------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;
         const uint32_t tempty_leader0 = map_to_cta(smem_u32(&tempty[0]), 0);
@@ -307,23 +414,113 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         uint32_t acc_phase = 0;
         for (int u = pair_id; u < units; u += num_pairs) {
             const Unit t = unit(u);
+            const int64_t row = t.row0 + int(rank) * 128 + 32 * q + lane;
+            const bool row_ok = row >= 0 && row < M && row < t.row_end;
+            // residual form: this row's 256 residual values are fetched while
+            // the MMAs still run (into L2, and the first 32 into registers),
+            // so that the stores below do not wait on memory in turn
+            uint4 rcur[4];
+            if (FUSED && res && row_ok) {
+                const __nv_bfloat16 *rp = static_cast<const __nv_bfloat16 *>(res) + row * N;
+#pragma unroll
+                for (int l = 0; l < BN / 64; ++l) {
+                    const int col = t.nb * BN + 64 * l;
+                    if (col < N) prefetch_l2(rp + col);
+                }
+                load_res32(res, row, t.nb * BN, N, rcur);
+            }
             if (!wait(&tfull[acc], acc_phase, ctl)) break;
             tc_fence_after();
-            const int64_t row = t.row0 + int(rank) * 128 + 32 * q + lane;
+            float rscale = 1.0f;
+            if (nrm) {
+                if (!wait(&rfull[acc], acc_phase, ctl)) break;
+                rscale = rsq[acc * 128 + 32 * q + lane];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&rempty[acc]);
+            }
 #pragma unroll 1
             for (int cc = 0; cc < BN / 32; ++cc) {
+                uint4 rnext[4];
+                if (FUSED && res && row_ok && cc + 1 < BN / 32)
+                    load_res32(res, row, t.nb * BN + (cc + 1) * 32, N, rnext);
                 uint32_t r[32];
                 tmem_ld32(tmem_addr(tmem, 32 * q, acc * BN + cc * 32), r);
                 tmem_wait_ld(r);
+                if (nrm) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        r[j] = __float_as_uint(__fmul_rn(__uint_as_float(r[j]), rscale));
+                }
                 const int col0 = t.nb * BN + cc * 32;
-                if (row >= 0 && row < M && row < t.row_end && col0 < N)
-                    store_row32(r, c, ws, row, col0, N, M, t.split, k_splits, out_f32);
+                if (row_ok && col0 < N) {
+                    if (FUSED && res)
+                        store_row32_res(r, c, rcur, row, col0, N);
+                    else
+                        store_row32(r, c, ws, row, col0, N, M, t.split, k_splits, out_f32);
+                }
+                if (FUSED && res) {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) rcur[g] = rnext[g];
+                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
+        }
+    } else if (nrm) {
+        // ---------------------------------------- norm form: row sums of squares
+        // Thread i owns row i of this CTA's 128.  An A slice row is 128
+        // bytes, its 16-byte piece p stored at p ^ (i % 8) (128-byte
+        // swizzle); squares are added K-ascending into eight partial sums,
+        // one per position within a piece.
+        const int i = 32 * (warp & 3) + lane;
+        uint64_t *ready = leader ? full : afull;
+        int stage = 0;
+        uint32_t phase = 0;
+        int buf = 0;
+        uint32_t buf_phase = 0;
+        bool ok = true;
+        for (int u = pair_id; ok && u < units; u += num_pairs) {
+            const Unit t = unit(u);
+            float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int kb = t.kb0; kb < t.kb1; ++kb) {
+                if (!wait(&ready[stage], phase, ctl)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t *rowp = sA + stage * A_BYTES + i * 128;
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(rowp + ((p ^ (i & 7)) << 4));
+                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float lo = __uint_as_float(w4[j] << 16);
+                        const float hi = __uint_as_float(w4[j] & 0xFFFF0000u);
+                        part[2 * j] = __fmaf_rn(lo, lo, part[2 * j]);
+                        part[2 * j + 1] = __fmaf_rn(hi, hi, part[2 * j + 1]);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            const float ss = __fadd_rn(
+                __fadd_rn(__fadd_rn(part[0], part[1]), __fadd_rn(part[2], part[3])),
+                __fadd_rn(__fadd_rn(part[4], part[5]), __fadd_rn(part[6], part[7])));
+            const float r = rsqrtf(__fadd_rn(__fdiv_rn(ss, float(K)), epi.eps));
+            if (!wait(&rempty[buf], buf_phase ^ 1u, ctl)) break;
+            rsq[buf * 128 + i] = r;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&rfull[buf]);
+            buf ^= 1;
+            if (buf == 0) buf_phase ^= 1u;
         }
     }
 
@@ -389,9 +586,12 @@ int gemm_k_splits(int64_t M, int64_t N, int64_t K, int num_sms)
 // pair up); the persistent grid is this many clusters.
 static cudaError_t resident_pairs(int num_sms, int *out)
 {
-    cudaError_t e = cudaFuncSetAttribute(pair::gemm_pair_kernel,
+    cudaError_t e = cudaFuncSetAttribute(pair::gemm_pair_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          pair::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(pair::gemm_pair_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, pair::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     // as many pairs as can be resident at once (not every SM can pair up)
     static int max_pairs[64] = {0};
@@ -411,7 +611,7 @@ static cudaError_t resident_pairs(int num_sms, int *out)
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        e = cudaOccupancyMaxActiveClusters(&clusters, pair::gemm_pair_kernel, &cfg);
+        e = cudaOccupancyMaxActiveClusters(&clusters, pair::gemm_pair_kernel<false>, &cfg);
         if (e != cudaSuccess) return e;
         max_pairs[dev] = clusters > 0 ? clusters : 1;
     }
@@ -428,8 +628,9 @@ cudaError_t launch_gemm_grouped(const CUtensorMap &ta, const CUtensorMap &tw, vo
     cudaError_t e = resident_pairs(num_sms, &pairs);
     if (e != cudaSuccess) return e;
     // the tile count is only known on the device: every resident pair runs
-    pair::gemm_pair_kernel<<<2 * pairs, pair::THREADS, pair::SMEM_BYTES, s>>>(
-        ta, tw, c, nullptr, rows, N, K, out_f32 ? 1 : 0, 1, offsets, groups, status, timeout_ns);
+    pair::gemm_pair_kernel<false><<<2 * pairs, pair::THREADS, pair::SMEM_BYTES, s>>>(
+        ta, tw, c, nullptr, rows, N, K, out_f32 ? 1 : 0, 1, offsets, groups, GemmEpi{}, status,
+        timeout_ns);
     return cudaGetLastError();
 }
 
@@ -443,14 +644,31 @@ cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tw, void *c, i
     const int64_t units = int64_t((M + pair::BM - 1) / pair::BM) * ((N + pair::BN - 1) / pair::BN) *
                           k_splits;
     const int pairs = static_cast<int>(units < max_pairs ? units : max_pairs);
-    pair::gemm_pair_kernel<<<2 * pairs, pair::THREADS, pair::SMEM_BYTES, s>>>(
-        ta, tw, c, ws, M, N, K, out_f32 ? 1 : 0, k_splits, nullptr, 0, status, timeout_ns);
+    pair::gemm_pair_kernel<false><<<2 * pairs, pair::THREADS, pair::SMEM_BYTES, s>>>(
+        ta, tw, c, ws, M, N, K, out_f32 ? 1 : 0, k_splits, nullptr, 0, GemmEpi{}, status,
+        timeout_ns);
     e = cudaGetLastError();
     if (e != cudaSuccess || k_splits <= 1) return e;
     const int64_t MN = int64_t(M) * N;
     const int64_t thr = (MN / 4 + 255) / 256;
     splitk_reduce_kernel<<<static_cast<unsigned>(thr), 256, 0, s>>>(ws, c, MN, k_splits,
                                                                     out_f32 ? 1 : 0);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_fused(const CUtensorMap &ta, const CUtensorMap &tw, void *c, int M, int N,
+                              int K, bool out_f32, const GemmEpi &epi, int num_sms,
+                              unsigned *status, uint64_t timeout_ns, cudaStream_t s)
+{
+    int max_pairs = 0;
+    cudaError_t e = resident_pairs(num_sms, &max_pairs);
+    if (e != cudaSuccess) return e;
+    const int64_t units = int64_t((M + pair::BM - 1) / pair::BM) * ((N + pair::BN - 1) / pair::BN);
+    const int pairs = static_cast<int>(units < max_pairs ? units : max_pairs);
+    // the norm warps exist only in the norm form
+    const int threads = epi.norm ? pair::FUSED_THREADS : pair::THREADS;
+    pair::gemm_pair_kernel<true><<<2 * pairs, threads, pair::SMEM_BYTES, s>>>(
+        ta, tw, c, nullptr, M, N, K, out_f32 ? 1 : 0, 1, nullptr, 0, epi, status, timeout_ns);
     return cudaGetLastError();
 }
 

@@ -168,6 +168,26 @@ __global__ void swiglu_kernel(const uint4 *__restrict__ gu, uint4 *__restrict__ 
     }
 }
 
+// ---------------------------------------------------------------- norm-weight fold
+// wf[n, k] = round(W[n, k] * w[k]): the product of two bf16 values is exact
+// in fp32, so this is the correctly rounded product.  Eight per thread.
+__global__ void fold_norm_weight_kernel(const uint4 *__restrict__ W, const uint4 *__restrict__ w,
+                                        uint4 *__restrict__ wf, int64_t N, int64_t kp)
+{
+    const int64_t n = N * kp;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t k = i % kp;
+        const uint4 a = W[i], b = __ldg(w + k);
+        const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            o[j] = pack2(__fmul_rn(lo16(av[j]), lo16(bv[j])), __fmul_rn(hi16(av[j]), hi16(bv[j])));
+        wf[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
 // ---------------------------------------------------------------- argmax
 // One block per row (grid-stride): each thread scans its float4 pieces in
 // index order, then the (value, index) pairs are combined by a warp
@@ -462,6 +482,16 @@ cudaError_t launch_swiglu(const void *gu, void *out, int64_t T, int64_t F, int n
     const int64_t fp = F / 8;
     swiglu_kernel<<<grid_for(T * fp, 256, num_sms), 256, 0, s>>>(
         static_cast<const uint4 *>(gu), static_cast<uint4 *>(out), T, fp);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fold_norm_weight(const void *W, const void *w, void *wf, int64_t N, int64_t K,
+                                    int num_sms, cudaStream_t s)
+{
+    const int64_t kp = K / 8;
+    fold_norm_weight_kernel<<<grid_for(N * kp, 256, num_sms), 256, 0, s>>>(
+        static_cast<const uint4 *>(W), static_cast<const uint4 *>(w), static_cast<uint4 *>(wf), N,
+        kp);
     return cudaGetLastError();
 }
 

@@ -46,6 +46,8 @@ class DecoderConfig:
     n_experts: int = 0            # > 0: a mixture-of-experts feed-forward
     top_k: int = 2
     expert_ffn: int = 1408
+    fused: bool = False           # RMSNorm folded into the next matmul, residual adds
+                                  # into the matmul epilogue (dense feed-forward only)
 
     @property
     def qkv_dim(self) -> int:
@@ -255,6 +257,19 @@ class ToyDecoder:
                         for _ in range(cfg.layers)]
         self.num_pages = num_pages
         self.launches = 0
+        # fused form: each matmul that follows an RMSNorm takes its weight with
+        # the norm weight folded in (once, here)
+        self.wf = {}
+        if cfg.fused:
+            if cfg.n_experts:
+                raise ValueError("the fused form covers the dense feed-forward only")
+            for i in range(cfg.layers):
+                self.wf["l%d.wqkv" % i] = lib.bi_fold_norm_weight(weights["l%d.wqkv" % i],
+                                                                  weights["l%d.attn_norm" % i])
+                self.wf["l%d.wgu" % i] = lib.bi_fold_norm_weight(weights["l%d.wgu" % i],
+                                                                 weights["l%d.mlp_norm" % i])
+            self.wf["lm_head"] = lib.bi_fold_norm_weight(weights["lm_head"],
+                                                         weights["final_norm"])
 
     def _to_dev(self, a: np.ndarray) -> torch.Tensor:
         return torch.from_numpy(np.ascontiguousarray(a)).to(self.dev, non_blocking=False)
@@ -274,11 +289,16 @@ class ToyDecoder:
         max_chunk = int(np.diff(plan.cu_q).max()) if plan.pre else 0
 
         x = L.bi_embedding(W["embed"], tokens)
-        h = L.bi_rmsnorm(x, W["l0.attn_norm"], c.eps)
-        n = 2
         o = torch.empty((T, c.n_heads, c.head_dim), dtype=torch.bfloat16, device=self.dev)
+        if c.fused:
+            h, n = None, 1
+        else:
+            h, n = L.bi_rmsnorm(x, W["l0.attn_norm"], c.eps), 2
         for i in range(c.layers):
-            qkv = L.bi_matmul(h, W["l%d.wqkv" % i])
+            if c.fused:
+                qkv = L.bi_rmsnorm_matmul(x, self.wf["l%d.wqkv" % i], c.eps)
+            else:
+                qkv = L.bi_matmul(h, W["l%d.wqkv" % i])
             kv_all = PagedKV(self.k_cache[i], self.v_cache[i], bt)
             q = L.bi_rope_kv_write(kv_all, qkv, pos, slots, c.n_heads, c.theta)
             if Bd:
@@ -289,6 +309,14 @@ class ToyDecoder:
                 kv = PagedKV(self.k_cache[i], self.v_cache[i], bt[Bd:])
                 L.bi_attention_prefill(kv, q[Bd:], cu, ctx, max_chunk, out=o[Bd:])
                 n += 1
+            if c.fused:
+                # x += o Wo^T; x += swiglu(RMSNorm(x) Wgu^T) Wdown^T
+                L.bi_matmul_residual(o.view(T, c.n_heads * c.head_dim), W["l%d.wo" % i], x,
+                                     out=x)
+                f = L.bi_swiglu(L.bi_rmsnorm_matmul(x, self.wf["l%d.wgu" % i], c.eps))
+                L.bi_matmul_residual(f, W["l%d.wdown" % i], x, out=x)
+                n += 6
+                continue
             a = L.bi_matmul(o.view(T, c.n_heads * c.head_dim), W["l%d.wo" % i])
             h = L.bi_add_rmsnorm(x, a, W["l%d.mlp_norm" % i], c.eps)
             if c.n_experts:
@@ -301,8 +329,12 @@ class ToyDecoder:
             nxt = W["l%d.attn_norm" % (i + 1)] if i + 1 < c.layers else W["final_norm"]
             h = L.bi_add_rmsnorm(x, m, nxt, c.eps)
             n += 5
-        last = L.bi_embedding(h, rows)
-        logits = L.bi_matmul(last, W["lm_head"], out_dtype=torch.float32)
+        if c.fused:
+            last = L.bi_embedding(x, rows)
+            logits = L.bi_rmsnorm_matmul(last, self.wf["lm_head"], c.eps, out_dtype=torch.float32)
+        else:
+            last = L.bi_embedding(h, rows)
+            logits = L.bi_matmul(last, W["lm_head"], out_dtype=torch.float32)
         nt = L.bi_sample(logits, self._to_dev(plan.temperature), self._to_dev(plan.top_p),
                          self._to_dev(plan.seed.view(np.int64)),
                          self._to_dev(plan.offset.view(np.int64)))

@@ -3,11 +3,15 @@ greedily many times amid random other requests (random prompt lengths,
 arrival steps, chunked prefill, decode/prefill mixes, batch sizes from 1 up
 to the cap) gives exactly one completion, equal to the prompt's completion
 when it runs alone."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
 
 import invariant_bi_rmsnorm_03_b200 as bi
+import oracle
+from gpu_util import TOL_BF16, host_bits, rowwise_normwise, to_f64
 from invariant_bi_rmsnorm_03_b200.decoder import (DecoderConfig, PagePool, Request, Scheduler,
                                                   ToyDecoder, run, weight_shapes)
 from synth import toy_decoder_weights, unique_completion_workload
@@ -40,6 +44,46 @@ def test_unique_completion_small():
     outs = {tuple(r.out) for r in reqs if r.tag == "target"}
     assert len(solo.out) == 24
     assert outs == {tuple(solo.out)}
+
+
+def test_unique_completion_small_fused():
+    # RMSNorm folded into the following matmul and the residual adds into
+    # the matmul epilogue: other bits than the unfused decoder, but again
+    # one completion, the prompt's own.
+    cfg = dataclasses.replace(SMALL, fused=True)
+    L = bi.load()
+    w = toy_decoder_weights(weight_shapes(cfg), seed=4, device="cuda")
+    prompt, spec = unique_completion_workload(seed=5, n_target=24, n_other=120, prompt_len=40,
+                                              gen_len=24, vocab=cfg.vocab,
+                                              other_prompt_max=300, steps_span=60)
+    solo = Request(-1, prompt, 24)
+    completions(L, cfg, w, [solo], max_batch=1, budget=16)
+    reqs = [Request(d["rid"], d["prompt"], d["max_new"], d["arrival"], d["tag"]) for d in spec]
+    completions(L, cfg, w, reqs, max_batch=48, budget=256)
+    outs = {tuple(r.out) for r in reqs if r.tag == "target"}
+    assert outs == {tuple(solo.out)}
+
+
+def test_fused_decoder_pieces_match_the_oracle():
+    # The fused model's feed-forward pieces on its own folded weights against
+    # the oracle, each fed the GPU's bf16 inputs: RMSNorm folded into the
+    # gate/up matmul, and the down matmul added to the residual in place.
+    cfg = dataclasses.replace(SMALL, fused=True, layers=1)
+    L = bi.load()
+    w = toy_decoder_weights(weight_shapes(cfg), seed=6, device="cuda")
+    model = ToyDecoder(L, cfg, w, 64, "cuda")
+    # the model's norm weights are ones, so the folded weights are the weights
+    assert torch.equal(model.wf["l0.wqkv"].view(torch.int16), w["l0.wqkv"].view(torch.int16))
+    x = torch.from_numpy(np.random.default_rng(7).standard_normal((37, cfg.hidden))
+                         .astype(np.float32)).to("cuda").to(torch.bfloat16)
+    gu = L.bi_rmsnorm_matmul(x, model.wf["l0.wgu"], cfg.eps)
+    ref = oracle.rmsnorm_matmul(host_bits(x), host_bits(model.wf["l0.wgu"]), cfg.eps)
+    assert rowwise_normwise(to_f64(gu), ref).max() <= TOL_BF16
+    f = L.bi_swiglu(gu)
+    x2 = x.clone()
+    L.bi_matmul_residual(f, w["l0.wdown"], x2, out=x2)
+    ref2 = oracle.matmul_residual(host_bits(x), host_bits(f), host_bits(w["l0.wdown"]))
+    assert rowwise_normwise(to_f64(x2), ref2).max() <= TOL_BF16
 
 
 def test_full_size_decoder_step_runs():

@@ -1,0 +1,143 @@
+"""The fused matmul forms on the GPU: the norm-weight fold (bit-exact: the
+correctly rounded product), RMSNorm folded into the matmul (parity with the
+fp64 oracle, bitwise batch invariance) and the residual matmul (equal bit for
+bit to bi_matmul followed by the addition; parity with the oracle)."""
+import numpy as np
+import pytest
+import torch
+
+import invariant_bi_rmsnorm_03_b200 as bi
+import oracle
+from gpu_util import (TOL_BF16, TOL_F32, dev_bf16, host_bits, rowwise_normwise, same_bytes,
+                      to_f64)
+from synth import bf16_bits_to_f32, f32_to_bf16_bits, norm_matmul, normal_bf16, rng, uniform_bf16
+
+pytestmark = pytest.mark.gpu
+
+EPS = 1e-6
+SHAPES = [(1, 8, 8), (3, 264, 72), (129, 512, 136), (200, 776, 1000), (257, 256, 64),
+          (300, 4096, 4096), (600, 1024, 8), (2048, 8192, 64)]
+
+
+@pytest.fixture(scope="module")
+def L():
+    return bi.load()
+
+
+def scaled_rows(g, M, K):
+    """N(0, 1) rows times per-row scales 2^U(-6, 6): the norm has work to do."""
+    x = normal_bf16(g, (M, K))
+    s = np.exp2(g.uniform(-6, 6, size=(M, 1))).astype(np.float32)
+    return f32_to_bf16_bits(bf16_bits_to_f32(x) * s)
+
+
+def test_fold_is_the_correctly_rounded_product(L):
+    g = rng(300)
+    W = normal_bf16(g, (777, 520), std=0.02)
+    w = uniform_bf16(g, (520,), 0.5, 1.5)
+    want = f32_to_bf16_bits(oracle.fold_norm_weight(W, w).astype(np.float32))  # exact in fp32
+    got = host_bits(L.bi_fold_norm_weight(dev_bf16(W), dev_bf16(w)))
+    np.testing.assert_array_equal(got, want)
+    Wd = dev_bf16(W)
+    L.bi_fold_norm_weight(Wd, dev_bf16(w), out=Wd)  # in place
+    np.testing.assert_array_equal(host_bits(Wd), want)
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_rmsnorm_matmul_parity(L, M, N, K):
+    g = rng(310 + M + N + K)
+    x = scaled_rows(g, M, K)
+    wf = normal_bf16(g, (N, K), std=0.05)
+    rows = np.arange(M) if M <= 300 else np.unique(np.concatenate(
+        [[0, 127, 128, 255, 256, M - 1], g.integers(0, M, 40)]))
+    ref = oracle.rmsnorm_matmul(x[rows], wf, EPS)
+    for dt, tol in ((torch.bfloat16, TOL_BF16), (torch.float32, TOL_F32)):
+        c = L.bi_rmsnorm_matmul(dev_bf16(x), dev_bf16(wf), EPS, out_dtype=dt)
+        err = rowwise_normwise(to_f64(c)[rows], ref)
+        assert err.max() <= tol, (dt, rows[err.argmax()], err.max())
+
+
+def test_rmsnorm_matmul_full_size_sampled_rows(L):
+    c = norm_matmul(M=2048, N=12288)
+    g = rng(320)
+    w = c["w"]
+    wf = L.bi_fold_norm_weight(dev_bf16(c["W"]), dev_bf16(w))
+    rows = np.unique(np.concatenate([[0, 127, 128, 2047], g.integers(0, 2048, 24)]))
+    ref = oracle.rmsnorm_matmul(c["x"][rows], host_bits(wf), EPS)
+    out = L.bi_rmsnorm_matmul(dev_bf16(c["x"]), wf, EPS)
+    err = rowwise_normwise(to_f64(out)[rows], ref)
+    assert err.max() <= TOL_BF16, err.max()
+    # the composition the fold stands for: RMSNorm with weight w, then W
+    ref2 = oracle.matmul(f32_to_bf16_bits(oracle.rmsnorm(c["x"][rows], w, EPS).astype(np.float32)),
+                         c["W"])
+    assert rowwise_normwise(to_f64(out)[rows], ref2).max() <= TOL_BF16
+
+
+def test_rmsnorm_matmul_rows_do_not_depend_on_the_batch(L):
+    g = rng(330)
+    x = dev_bf16(scaled_rows(g, 2048, 4096))
+    wf = dev_bf16(normal_bf16(g, (4096, 4096), std=0.02))
+    full = L.bi_rmsnorm_matmul(x, wf, EPS)
+    for M in (1, 2, 3, 31, 127, 128, 129, 255, 256, 257, 1000, 1500, 2047):
+        assert same_bytes(L.bi_rmsnorm_matmul(x[:M], wf, EPS), full[:M]), M
+    perm = torch.from_numpy(g.permutation(2048)).to(x.device)
+    assert same_bytes(L.bi_rmsnorm_matmul(x[perm].contiguous(), wf, EPS), full[perm])
+    for _ in range(5):
+        assert same_bytes(L.bi_rmsnorm_matmul(x, wf, EPS), full)
+
+
+def test_rmsnorm_matmul_edge_rows(L):
+    g = rng(340)
+    x = scaled_rows(g, 5, 256)
+    x[1] = 0                       # a zero row: rsqrt(eps) * 0 = 0
+    x[3] = f32_to_bf16_bits(np.full(256, 3.0, np.float32))  # constant row: y = sign
+    wf = normal_bf16(g, (264, 256), std=0.1)
+    c = to_f64(L.bi_rmsnorm_matmul(dev_bf16(x), dev_bf16(wf), EPS, out_dtype=torch.float32))
+    assert np.all(c[1] == 0.0)
+    ref = oracle.rmsnorm_matmul(x, wf, EPS)
+    assert rowwise_normwise(c, ref).max() <= TOL_F32
+    assert L.bi_rmsnorm_matmul(dev_bf16(x[:0]), dev_bf16(wf), EPS).shape == (0, 264)
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_residual_equals_matmul_then_add(L, M, N, K):
+    g = rng(350 + M + N + K)
+    a = dev_bf16(normal_bf16(g, (M, K)))
+    w = dev_bf16(normal_bf16(g, (N, K), std=0.05))
+    r = dev_bf16(normal_bf16(g, (M, N)))
+    want = (r.float() + L.bi_matmul(a, w).float()).to(torch.bfloat16)
+    assert same_bytes(L.bi_matmul_residual(a, w, r), want)
+    r2 = r.clone()
+    L.bi_matmul_residual(a, w, r2, out=r2)  # in place
+    assert same_bytes(r2, want)
+
+
+def test_residual_parity_with_the_oracle(L):
+    g = rng(360)
+    a, w, r = normal_bf16(g, (300, 1000)), normal_bf16(g, (776, 1000), std=0.05), \
+        normal_bf16(g, (300, 776))
+    out = L.bi_matmul_residual(dev_bf16(a), dev_bf16(w), dev_bf16(r))
+    err = rowwise_normwise(to_f64(out), oracle.matmul_residual(r, a, w))
+    assert err.max() <= TOL_BF16, err.max()
+
+
+def test_residual_rows_do_not_depend_on_the_batch(L):
+    c = norm_matmul(M=2048, N=4096)
+    g = rng(370)
+    a, w = dev_bf16(c["x"]), dev_bf16(c["W"])
+    r = dev_bf16(normal_bf16(g, (2048, 4096)))
+    full = L.bi_matmul_residual(a, w, r)
+    for M in (1, 3, 129, 256, 257, 2047):
+        assert same_bytes(L.bi_matmul_residual(a[:M], w, r[:M]), full[:M]), M
+
+
+def test_fused_argument_errors(L):
+    x = torch.zeros((4, 12), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(RuntimeError):
+        L.bi_rmsnorm_matmul(x, torch.zeros((8, 12), dtype=torch.bfloat16, device="cuda"), EPS)
+    x = torch.zeros((4, 16), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(RuntimeError):
+        L.bi_rmsnorm_matmul(x, torch.zeros((8, 16), dtype=torch.bfloat16, device="cuda"), -1.0)
+    with pytest.raises(RuntimeError):
+        L.bi_matmul_residual(x, torch.zeros((12, 16), dtype=torch.bfloat16, device="cuda"),
+                             torch.zeros((4, 12), dtype=torch.bfloat16, device="cuda"))
