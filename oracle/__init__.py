@@ -68,6 +68,7 @@ class Oracle:
         lib.oracle_fold_norm_weight.argtypes = [P, P, i64, i64, P]
         lib.oracle_rmsnorm_matmul.argtypes = [P, P, i64, i64, i64, f64, P]
         lib.oracle_matmul_residual.argtypes = [P, P, P, i64, i64, i64, P]
+        lib.oracle_rope_angles.argtypes = [i32, i32, f64, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
@@ -154,6 +155,12 @@ class Oracle:
         assert pos.shape == (T,) and d % 2 == 0
         out = np.empty((T, nh, d), dtype=np.float64)
         self.lib.oracle_rope(_p(x), T, nh, d, _p(pos), float(theta), _p(out))
+        return out
+
+    def rope_angles(self, P: int, d: int, theta: float = 10000.0) -> np.ndarray:
+        """(cos, sin) of p * theta^(-2i/d) -> float64 [P, d/2, 2]."""
+        out = np.empty((P, d // 2, 2), dtype=np.float64)
+        self.lib.oracle_rope_angles(int(P), int(d), float(theta), _p(out))
         return out
 
     def swiglu(self, gu) -> np.ndarray:
@@ -317,6 +324,10 @@ def embedding(table, ids) -> np.ndarray:
 
 def rope(x, pos, theta: float = 10000.0) -> np.ndarray:
     return default().rope(x, pos, theta)
+
+
+def rope_angles(P: int, d: int, theta: float = 10000.0) -> np.ndarray:
+    return default().rope_angles(P, d, theta)
 
 
 def swiglu(gu) -> np.ndarray:

@@ -567,3 +567,21 @@ void oracle_matmul_residual(const uint16_t *r, const uint16_t *a, const uint16_t
         }
     }
 }
+
+/*
+ * The rotary angles as a table: out[p][i] = (cos a, sin a) with
+ * a = p * theta^(-2i/d), for positions p < P and i < d/2 -- the angles of
+ * oracle_rope above, listed once per position.
+ */
+void oracle_rope_angles(int32_t P, int32_t d, double theta, double *out)
+{
+    int32_t p;
+#pragma omp parallel for schedule(static)
+    for (p = 0; p < P; ++p) {
+        for (int32_t i = 0; i < d / 2; ++i) {
+            const double freq = pow(theta, -(double)(2 * i) / (double)d);
+            out[((int64_t)p * (d / 2) + i) * 2] = cos((double)p * freq);
+            out[((int64_t)p * (d / 2) + i) * 2 + 1] = sin((double)p * freq);
+        }
+    }
+}

@@ -671,3 +671,27 @@ def test_matmul_residual_degenerate_cases(oracle):
     np.testing.assert_array_equal(oracle.matmul_residual(R, A, bf(np.zeros((24, 16)))), widen(R))
     np.testing.assert_allclose(oracle.matmul_residual(bf(np.zeros((5, 24))), A, W),
                                oracle.matmul(A, W), rtol=1e-15)
+
+
+def test_rope_angles_closed_forms(oracle):
+    t = oracle.rope_angles(40, 8, 10000.0)
+    np.testing.assert_array_equal(t[0, :, 0], 1.0)   # position 0: no rotation
+    np.testing.assert_array_equal(t[0, :, 1], 0.0)
+    p = np.arange(40)
+    np.testing.assert_allclose(t[:, 0, 0], np.cos(p), rtol=0, atol=1e-15)  # i = 0: frequency 1
+    np.testing.assert_allclose(t[:, 0, 1], np.sin(p), rtol=0, atol=1e-15)
+    # d = 4, theta = 100: i = 1 has frequency 100^(-1/2) = 0.1; position 10 turns by 1 radian
+    h = oracle.rope_angles(11, 4, 100.0)
+    np.testing.assert_allclose(h[10, 1], [math.cos(1.0), math.sin(1.0)], rtol=1e-14)
+    np.testing.assert_allclose(t[..., 0] ** 2 + t[..., 1] ** 2, 1.0, rtol=1e-15)
+
+
+def test_rope_angles_rotate_like_rope(oracle):
+    g = rng(90)
+    x = normal_bf16(g, (6, 3, 16))
+    pos = g.integers(0, 50, size=6).astype(np.int32)
+    t = oracle.rope_angles(50, 16, 10000.0)
+    xw = widen(x)
+    c, s = t[pos, :, 0][:, None, :], t[pos, :, 1][:, None, :]
+    want = np.concatenate([xw[..., :8] * c - xw[..., 8:] * s, xw[..., 8:] * c + xw[..., :8] * s], -1)
+    np.testing.assert_allclose(oracle.rope(x, pos), want, rtol=1e-13, atol=1e-15)

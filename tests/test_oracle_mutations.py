@@ -107,6 +107,11 @@ MUTATIONS = [
      "s += (bf16_to_double(xm[k]) / root) * bf16_to_double(wn[k]);",
      "s += (bf16_to_double(xm[k]) / root) * bf16_to_double(wf[(k * N + n) % (N * K)]);",
      [pins.test_rmsnorm_matmul_hand_example, pins.test_rmsnorm_matmul_matches_torch_fp64]),
+    ("rope_angles_exponent_i_over_d", "pow(theta, -(double)(2 * i) / (double)d)",
+     "pow(theta, -(double)(i) / (double)d)",
+     [pins.test_rope_angles_closed_forms, pins.test_rope_angles_rotate_like_rope]),
+    ("rope_angles_cos_sin_swapped", "* 2] = cos((double)p * freq);", "* 2] = sin((double)p * freq);",
+     [pins.test_rope_angles_closed_forms]),
     ("matmul_residual_drops_residual", "c[m * N + n] = bf16_to_double(r[m * N + n]) + dot;",
      "c[m * N + n] = dot;",
      [pins.test_matmul_residual_small_integers_brute_force, pins.test_matmul_residual_degenerate_cases]),
