@@ -719,6 +719,33 @@ def run_profile_case(args):
             fn = lambda i: L.bi_matmul_residual(x, Ws[i % 2], r, out=c)  # noqa: E731
         else:
             fn = lambda i: L.bi_matmul(x, Ws[i % 2], out=c)  # noqa: E731
+    elif args.profile in ("qkv_fused", "qkv_unfused"):
+        # the attention input of one layer of the toy decoder (hidden 4096, 32 q and
+        # 8 kv heads of 128), M = --profile-rows tokens: RMSNorm, QKV matmul, RoPE and
+        # the cache write, in one launch or as RMSNorm + matmul + RoPE/cache write
+        M, Hq, Hkv, d = args.profile_rows, 32, 8, D
+        g = rng(13)
+        nm = norm_matmul(seed=1, M=M, H=H, N=8)
+        x, w = d16(nm["x"]), d16(nm["w"])
+        Wq = d16(normal_bf16(g, ((Hq + 2 * Hkv) * d, H), std=0.02))
+        npages = M // 16 + 16
+        kv = bi.PagedKV(T.zeros((npages, Hkv, 16, d), dtype=T.bfloat16, device=dev),
+                        T.zeros((npages, Hkv, 16, d), dtype=T.bfloat16, device=dev),
+                        T.zeros((1, 1), dtype=T.int32, device=dev))
+        pos = T.from_numpy(g.integers(0, 4096, size=M).astype(np.int32)).to(dev)
+        slots = T.from_numpy(g.permutation(npages * 16)[:M].astype(np.int64)).to(dev)
+        q = T.empty((M, Hq, d), dtype=T.bfloat16, device=dev)
+        if args.profile == "qkv_fused":
+            wf = L.bi_fold_norm_weight(Wq, w)
+            table = L.bi_rope_table(4096, d)
+            fn = lambda i: L.bi_rmsnorm_matmul_rope_kv(x, wf, 1e-6, kv, table, pos,  # noqa: E731
+                                                       slots, Hq, q_out=q)
+        else:
+            y = T.empty_like(x)
+            qkv = T.empty((M, (Hq + 2 * Hkv) * d), dtype=T.bfloat16, device=dev)
+            fn = lambda i: L.bi_rope_kv_write(  # noqa: E731
+                kv, L.bi_matmul(L.bi_rmsnorm(x, w, 1e-6, out=y), Wq, out=qkv), pos, slots, Hq,
+                q_out=q)
     elif args.profile == "sample":
         # 256 rows of lm_head logits (vocab 32000), temperature 0.8, nucleus 0.95
         g = rng(5)
@@ -799,8 +826,9 @@ def unique_completions(targets, others, max_batch=256, token_budget=2048, span=2
               "prompt_tokens": 64, "new_tokens": 256, "targets": targets,
               "others": others, "max_batch": max_batch,
               "token_budget": token_budget, "data": "synthetic",
-              "fused": ("RMSNorm folded into the next matmul, residual adds in the matmul "
-                        "epilogue" if cfg.fused else False),
+              "fused": ("RMSNorm folded into the next matmul, RoPE and the cache write in "
+                        "the QKV matmul's epilogue, residual adds in the matmul epilogue"
+                        if cfg.fused else False),
               "sampling": ("greedy" if temperature <= 0 else
                            {"temperature": temperature, "top_p": top_p,
                             "seed": "one per request; every target copy the same"})}
@@ -864,7 +892,8 @@ def main(argv=None):
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--profile", choices=["rmsnorm", "matmul", "decode", "prefill", "copy",
                                           "sample", "rmsnorm_matmul", "rmsnorm_then_matmul",
-                                          "matmul_residual", "matmul_rows"],
+                                          "matmul_residual", "matmul_rows", "qkv_fused",
+                                          "qkv_unfused"],
                     help="run one kernel alone on a reduced case (for ncu)")
     ap.add_argument("--profile-batch", type=int, default=32)
     ap.add_argument("--profile-seq", type=int, default=4096)
@@ -884,7 +913,7 @@ def main(argv=None):
     ap.add_argument("--moe", action="store_true",
                     help="unique-completion run on the mixture-of-experts decoder")
     ap.add_argument("--fused", action="store_true",
-                    help="unique-completion run with the fused RMSNorm/residual matmuls")
+                    help="unique-completion run with the fused matmul forms")
     ap.add_argument("--uc-targets", type=int, default=200,
                     help="target copies (and as many others) of the in-bench unique-completion "
                          "check; 0 skips it")

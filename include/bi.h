@@ -201,6 +201,36 @@ bi_status bi_matmul_grouped(const void *a, const void *w, void *c, const int64_t
  *   [N, K];  r, c : bf16 [M, N], c may be r (in place), no other overlap.
  *   Requirements as bi_matmul.
  */
+/*
+ * bi_rope_table -- the rotary angles of bi_rope_kv_write as a table:
+ *   table[p, i] = ( cos(p theta^(-2i/d)), sin(p theta^(-2i/d)) ),  p < max_pos, i < d/2
+ * evaluated in double precision and rounded to fp32 exactly as
+ * bi_rope_kv_write evaluates them (the same floats).  table : device, fp32
+ * [max_pos, d/2, 2], 16-byte aligned.  d = head_dim in {64, 128}; theta > 1.
+ *
+ * bi_rmsnorm_matmul_rope_kv -- the attention input of a transformer block in
+ * one launch: RMSNorm of x folded into the QKV matmul (as bi_rmsnorm_matmul,
+ * wf the folded [N, K] weight, N = (Hq + 2 Hkv) d), then RoPE of the q and k
+ * heads and the cache write of k and v, in the matmul's epilogue.  The
+ * result is bi_rmsnorm_matmul followed by bi_rope_kv_write bit for bit (the
+ * product is rounded to bf16 first, the rotation uses the table's angles
+ * and the same fp32 operations); the [T, N] product is never stored.
+ *   x : device, bf16 [T, K];  positions : device, int32 [T], each in
+ *   [0, max_pos) (a row outside writes nothing and sets BI_ERR_DEVICE_INDEX
+ *   in the status word);  slot_mapping : device, int64 [T] (< 0: no cache
+ *   write; >= num_pages * 16: no write and BI_ERR_DEVICE_INDEX);  q_out :
+ *   device, bf16 [T, Hq, d];  the cache as in bi_kv_write.  Requirements as
+ *   bi_matmul for (T, N, K), Hq % Hkv == 0.  The cache pages written must be
+ *   distinct from the pages the same launch's other rows write (one slot per
+ *   token).
+ */
+bi_status bi_rope_table(float *table, int32_t max_pos, int32_t head_dim, float theta,
+                        void *stream);
+bi_status bi_rmsnorm_matmul_rope_kv(const void *x, const void *wf, float eps,
+                                    const bi_paged_kv *kv, const float *rope_table,
+                                    int32_t max_pos, const int32_t *positions,
+                                    const int64_t *slot_mapping, void *q_out, int64_t T,
+                                    int64_t K, int32_t Hq, void *stream);
 bi_status bi_fold_norm_weight(const void *W, const void *w, void *wf, int64_t N, int64_t K,
                               void *stream);
 bi_status bi_rmsnorm_matmul(const void *x, const void *wf, void *c, int64_t M, int64_t N,

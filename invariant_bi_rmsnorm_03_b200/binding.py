@@ -111,7 +111,8 @@ class Library:
                "bi_debug_bounded_wait", "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write",
                "bi_swiglu", "bi_argmax", "bi_sample", "bi_moe_route", "bi_moe_dispatch",
                "bi_moe_combine", "bi_matmul_grouped", "bi_fold_norm_weight",
-               "bi_rmsnorm_matmul", "bi_matmul_residual")
+               "bi_rmsnorm_matmul", "bi_matmul_residual", "bi_rope_table",
+               "bi_rmsnorm_matmul_rope_kv")
 
     def __init__(self, path: str):
         if not os.path.exists(path):
@@ -153,12 +154,15 @@ class Library:
         L.bi_fold_norm_weight.argtypes = [P, P, P, i64, i64, P]
         L.bi_rmsnorm_matmul.argtypes = [P, P, P, i64, i64, i64, f32, st, P]
         L.bi_matmul_residual.argtypes = [P, P, P, P, i64, i64, i64, P]
+        L.bi_rope_table.argtypes = [P, i32, i32, f32, P]
+        L.bi_rmsnorm_matmul_rope_kv.argtypes = [P, P, f32, kvp, P, i32, P, P, P, i64, i64, i32, P]
         for name in ("bi_rmsnorm", "bi_matmul", "bi_kv_write", "bi_attention_decode",
                      "bi_attention_prefill", "bi_device_status", "bi_debug_bounded_wait",
                      "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write", "bi_swiglu",
                      "bi_argmax", "bi_sample", "bi_moe_route", "bi_moe_dispatch",
                      "bi_moe_combine", "bi_matmul_grouped", "bi_fold_norm_weight",
-                     "bi_rmsnorm_matmul", "bi_matmul_residual"):
+                     "bi_rmsnorm_matmul", "bi_matmul_residual", "bi_rope_table",
+                     "bi_rmsnorm_matmul_rope_kv"):
             getattr(L, name).restype = st
         self.lib = L
 
@@ -350,6 +354,42 @@ class Library:
         self._check("bi_rope_kv_write", self.lib.bi_rope_kv_write(
             ctypes.byref(c), _ptr(qkv), _ptr(positions), _ptr(slot_mapping), _ptr(q_out), T, Hq,
             float(theta), _stream(stream)))
+        return q_out
+
+    def bi_rope_table(self, max_pos: int, head_dim: int, theta: float = 10000.0, device="cuda",
+                      stream=None) -> torch.Tensor:
+        """(cos, sin) of p theta^(-2i/d) as fp32 [max_pos, d/2, 2], the same floats
+        bi_rope_kv_write evaluates."""
+        table = torch.empty((max_pos, head_dim // 2, 2), dtype=torch.float32, device=device)
+        self._check("bi_rope_table", self.lib.bi_rope_table(_ptr(table), int(max_pos),
+                                                            int(head_dim), float(theta),
+                                                            _stream(stream)))
+        return table
+
+    def bi_rmsnorm_matmul_rope_kv(self, x: torch.Tensor, wf: torch.Tensor, eps: float,
+                                  kv: PagedKV, rope_table: torch.Tensor, positions: torch.Tensor,
+                                  slot_mapping: torch.Tensor, Hq: int, q_out=None,
+                                  stream=None) -> torch.Tensor:
+        """RMSNorm(x) @ wf.T, then RoPE and the cache write of k and v, in one
+        launch (bit for bit bi_rmsnorm_matmul + bi_rope_kv_write); returns the
+        rotated q [T, Hq, d]."""
+        _need(x, "x", torch.bfloat16)
+        T, K = x.shape
+        d, Hkv = kv.head_dim, kv.num_kv_heads
+        _need(wf, "wf", torch.bfloat16, ((Hq + 2 * Hkv) * d, K))
+        _need(rope_table, "rope_table", torch.float32)
+        if rope_table.dim() != 3 or rope_table.shape[1:] != (d // 2, 2):
+            raise ValueError("rope_table must be [max_pos, %d, 2]" % (d // 2))
+        _need(positions, "positions", torch.int32, (T,))
+        _need(slot_mapping, "slot_mapping", torch.int64, (T,))
+        if q_out is None:
+            q_out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=x.device)
+        _need(q_out, "q_out", torch.bfloat16, (T, Hq, d))
+        c = kv.c_struct()
+        self._check("bi_rmsnorm_matmul_rope_kv", self.lib.bi_rmsnorm_matmul_rope_kv(
+            _ptr(x), _ptr(wf), float(eps), ctypes.byref(c), _ptr(rope_table),
+            int(rope_table.shape[0]), _ptr(positions), _ptr(slot_mapping), _ptr(q_out), T, K, Hq,
+            _stream(stream)))
         return q_out
 
     def bi_swiglu(self, gu: torch.Tensor, out=None, stream=None) -> torch.Tensor:

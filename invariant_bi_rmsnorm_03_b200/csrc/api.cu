@@ -215,6 +215,58 @@ bi_status bi_rmsnorm_matmul(const void *x, const void *wf, void *c, int64_t M, i
                                            static_cast<cudaStream_t>(stream)));
 }
 
+bi_status bi_rope_table(float *table, int32_t max_pos, int32_t head_dim, float theta,
+                        void *stream)
+{
+    if (max_pos < 1 || !head_dim_ok(head_dim)) return BI_ERR_INVALID;
+    if (!(theta > 1.0f) || !std::isfinite(theta)) return BI_ERR_INVALID;
+    if (!table || !aligned16(table)) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_rope_table(table, max_pos, head_dim, double(theta), d->num_sms,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+bi_status bi_rmsnorm_matmul_rope_kv(const void *x, const void *wf, float eps,
+                                    const bi_paged_kv *kv, const float *rope_table,
+                                    int32_t max_pos, const int32_t *positions,
+                                    const int64_t *slot_mapping, void *q_out, int64_t T,
+                                    int64_t K, int32_t Hq, void *stream)
+{
+    if (!kv_ok(kv) || !head_dim_ok(kv->head_dim)) return BI_ERR_INVALID;
+    if (Hq < 1 || Hq % kv->num_kv_heads != 0 || max_pos < 1) return BI_ERR_INVALID;
+    const int64_t N = int64_t(Hq + 2 * kv->num_kv_heads) * kv->head_dim;
+    if (!gemm_shape_ok(T, N, K)) return BI_ERR_INVALID;
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return BI_ERR_INVALID;
+    if (T == 0) return BI_OK;
+    if (!x || !wf || !rope_table || !positions || !slot_mapping || !q_out || !aligned16(x) ||
+        !aligned16(wf) || !aligned16(rope_table) || !aligned16(q_out))
+        return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    CUtensorMap ta, tw;
+    if ((st = gemm_maps(x, wf, T, N, K, &ta, &tw)) != BI_OK) return st;
+    bi::GemmEpi epi{};
+    epi.norm = 1;
+    epi.eps = eps;
+    epi.rope = rope_table;
+    epi.max_pos = max_pos;
+    epi.pos = positions;
+    epi.slots = slot_mapping;
+    epi.q_out = q_out;
+    epi.k_cache = kv->k_cache;
+    epi.v_cache = kv->v_cache;
+    epi.num_pages = kv->num_pages;
+    epi.Hq = Hq;
+    epi.Hkv = kv->num_kv_heads;
+    epi.head_dim = kv->head_dim;
+    return from_cuda(bi::launch_gemm_fused(ta, tw, nullptr, int(T), int(N), int(K), false, epi,
+                                           d->num_sms, d->status, bi::kDefaultTimeoutNs,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
 bi_status bi_matmul_residual(const void *a, const void *w, const void *r, void *c, int64_t M,
                              int64_t N, int64_t K, void *stream)
 {

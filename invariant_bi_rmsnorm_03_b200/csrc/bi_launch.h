@@ -37,14 +37,29 @@ cudaError_t launch_gemm_grouped(const CUtensorMap &ta, const CUtensorMap &tw, vo
 // Fused epilogues of the plain product (never split along K):
 //   norm:     C[m, :] = round(rsqrt(mean_k A[m, k]^2 + eps) * acc[m, :])
 //   residual: C[m, :] = round(R[m, :] + round(acc[m, :]))   (R may be C)
+//   QKV (rope non-null): the N = (Hq + 2 Hkv) head_dim columns of the
+//             rounded product are q, k and v heads; q and k are rotated by
+//             the angles of the row's position (rope_kv_kernel's arithmetic)
+//             and q goes to q_out [M, Hq, head_dim], k and v to the row's
+//             cache slot; C is not written.
 struct GemmEpi {
     int norm;
     float eps;
     const void *residual;
+    const float *rope;      // [max_pos, head_dim / 2, 2]: cos, sin
+    int max_pos;
+    const int32_t *pos;     // [M]
+    const int64_t *slots;   // [M]; < 0: no cache write
+    void *q_out, *k_cache, *v_cache;
+    int64_t num_pages;
+    int Hq, Hkv, head_dim;
 };
 cudaError_t launch_gemm_fused(const CUtensorMap &ta, const CUtensorMap &tw, void *c, int M, int N,
                               int K, bool out_f32, const GemmEpi &epi, int num_sms,
                               unsigned *status, uint64_t timeout_ns, cudaStream_t s);
+// table[p, i] = (cos, sin) of p theta^(-2i/d), evaluated as rope_kv_kernel does
+cudaError_t launch_rope_table(float *table, int P, int d, double theta, int num_sms,
+                              cudaStream_t s);
 // wf[n, k] = round(W[n, k] * w[k])
 cudaError_t launch_fold_norm_weight(const void *W, const void *w, void *wf, int64_t N, int64_t K,
                                     int num_sms, cudaStream_t s);

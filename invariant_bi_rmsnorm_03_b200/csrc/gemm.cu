@@ -43,6 +43,9 @@
 //             about a microsecond, which would throttle the pipeline).
 //   residual  C[m, :] = round(R[m, :] + round(acc[m, :])), R read in the
 //             epilogue (it may be C itself).
+//   QKV       the columns are q, k and v heads: the rounded product goes
+//             through RoPE and the cache write in the epilogue (qkv_epilogue),
+//             with or without the norm form.
 // Neither changes the K order of the product; both are per-row.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -153,6 +156,96 @@ __device__ __forceinline__ void store_row32_res(const uint32_t (&r)[32], void *c
                 o[j] = pack_bf16x2(lo, hi);
             }
             *reinterpret_cast<uint4 *>(dst + 8 * g) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+// QKV form of the epilogue, for one accumulator row (one token): the tile's
+// 256 columns are 256 / d whole heads of the (Hq + 2 Hkv) d columns.  Each
+// value is first rounded to bf16 exactly as the product's output would be
+// (after the norm scale), then q and k heads are rotated with the table's
+// angles for the token's position using rope_kv_kernel's fp32 operations,
+// so that the result is the plain product followed by bi_rope_kv_write bit
+// for bit.  q goes to q_out, k and v to the token's cache slot (page blocks
+// in core-matrix order).  The tensor-memory loads are warp-wide; only the
+// stores depend on the row.
+__device__ __noinline__ void qkv_epilogue(const GemmEpi &epi, uint32_t tbase, int nb, int64_t row,
+                                          bool row_ok, float rscale, int N, unsigned *status)
+{
+    const int d = epi.head_dim, half = d / 2, pieces = d / 8;
+    int32_t p = 0;
+    int64_t slot = -1;
+    if (row_ok) {
+        p = __ldg(epi.pos + row);
+        slot = __ldg(epi.slots + row);
+        if (p < 0 || p >= epi.max_pos) record_status(status, BI_DEV_BAD_INDEX);
+        if (slot >= epi.num_pages * kPage) {
+            record_status(status, BI_DEV_BAD_INDEX);
+            slot = -1;
+        }
+    }
+    const bool ok = row_ok && p >= 0 && p < epi.max_pos;  // else the row writes nothing
+    const int64_t page = slot >= 0 ? slot / kPage : 0;
+    const int off = slot >= 0 ? int(slot % kPage) : 0;
+    const int64_t blk_row = (off >> 3) * (8 * pieces) + (off & 7);
+#pragma unroll 1
+    for (int hh = 0; hh < 256 / d; ++hh) {
+        const int n0 = nb * 256 + hh * d;
+        if (n0 >= N) break;  // the same for the whole warp
+        const int gh = n0 / d;  // q heads, then k heads, then v heads
+        const bool rotated = gh < epi.Hq + epi.Hkv;
+#pragma unroll 1
+        for (int a = 0; a < half / 32; ++a) {
+            uint32_t lo[32], hi[32];
+            tmem_ld32(tbase + uint32_t(hh * d + 32 * a), lo);
+            tmem_ld32(tbase + uint32_t(hh * d + half + 32 * a), hi);
+            tmem_wait_ld(lo);
+            tmem_wait_ld(hi);
+            uint32_t plo[16], phi[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                plo[j] = pack_bf16x2(__fmul_rn(__uint_as_float(lo[2 * j]), rscale),
+                                     __fmul_rn(__uint_as_float(lo[2 * j + 1]), rscale));
+                phi[j] = pack_bf16x2(__fmul_rn(__uint_as_float(hi[2 * j]), rscale),
+                                     __fmul_rn(__uint_as_float(hi[2 * j + 1]), rscale));
+            }
+            if (!ok) continue;
+            if (rotated) {
+                const float4 *cs =
+                    reinterpret_cast<const float4 *>(epi.rope + (int64_t(p) * half + 32 * a) * 2);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float4 c = __ldg(cs + j);  // cos, sin of values 2j and 2j + 1
+                    const float a0 = __uint_as_float(plo[j] << 16);
+                    const float a1 = __uint_as_float(plo[j] & 0xFFFF0000u);
+                    const float b0 = __uint_as_float(phi[j] << 16);
+                    const float b1 = __uint_as_float(phi[j] & 0xFFFF0000u);
+                    plo[j] = pack_bf16x2(__fsub_rn(__fmul_rn(a0, c.x), __fmul_rn(b0, c.y)),
+                                         __fsub_rn(__fmul_rn(a1, c.z), __fmul_rn(b1, c.w)));
+                    phi[j] = pack_bf16x2(__fadd_rn(__fmul_rn(b0, c.x), __fmul_rn(a0, c.y)),
+                                         __fadd_rn(__fmul_rn(b1, c.z), __fmul_rn(a1, c.w)));
+                }
+            }
+            if (gh < epi.Hq) {
+                uint4 *qo = static_cast<uint4 *>(epi.q_out) + (row * epi.Hq + gh) * pieces;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    qo[4 * a + u] = make_uint4(plo[4 * u], plo[4 * u + 1], plo[4 * u + 2], plo[4 * u + 3]);
+                    qo[half / 8 + 4 * a + u] =
+                        make_uint4(phi[4 * u], phi[4 * u + 1], phi[4 * u + 2], phi[4 * u + 3]);
+                }
+            } else if (slot >= 0) {
+                const int g = rotated ? gh - epi.Hq : gh - epi.Hq - epi.Hkv;
+                uint4 *blk = static_cast<uint4 *>(rotated ? epi.k_cache : epi.v_cache) +
+                             (page * epi.Hkv + g) * (kPage * pieces) + blk_row;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    blk[(4 * a + u) * 8] =
+                        make_uint4(plo[4 * u], plo[4 * u + 1], plo[4 * u + 2], plo[4 * u + 3]);
+                    blk[(half / 8 + 4 * a + u) * 8] =
+                        make_uint4(phi[4 * u], phi[4 * u + 1], phi[4 * u + 2], phi[4 * u + 3]);
+                }
+            }
         }
     }
 }
@@ -438,6 +531,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FUSED ? FUSED_THREAD
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&rempty[acc]);
             }
+            if (FUSED && epi.rope) {
+                qkv_epilogue(epi, tmem_addr(tmem, 32 * q, acc * BN), t.nb, row, row_ok, rscale, N,
+                             status);
+            } else {
 #pragma unroll 1
             for (int cc = 0; cc < BN / 32; ++cc) {
                 uint4 rnext[4];
@@ -462,6 +559,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FUSED ? FUSED_THREAD
 #pragma unroll
                     for (int g = 0; g < 4; ++g) rcur[g] = rnext[g];
                 }
+            }
             }
             tc_fence_before();
             __syncwarp();

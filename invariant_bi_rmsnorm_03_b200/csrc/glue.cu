@@ -168,6 +168,23 @@ __global__ void swiglu_kernel(const uint4 *__restrict__ gu, uint4 *__restrict__ 
     }
 }
 
+// The same angles as a table [P, d/2] of (cos, sin), for the QKV epilogue
+// of the matmul: the same expressions, so the same floats.
+__global__ void rope_table_kernel(float2 *__restrict__ table, int P, int d, double theta)
+{
+    const int half = d / 2;
+    const int64_t n = int64_t(P) * half;
+    for (int64_t k = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; k < n;
+         k += int64_t(gridDim.x) * blockDim.x) {
+        const int p = static_cast<int>(k / half);
+        const int i = static_cast<int>(k - int64_t(p) * half);
+        const double inv = pow(theta, -2.0 * double(i) / double(d));
+        double sv, cv;
+        sincos(double(p) * inv, &sv, &cv);
+        table[k] = make_float2(static_cast<float>(cv), static_cast<float>(sv));
+    }
+}
+
 // ---------------------------------------------------------------- norm-weight fold
 // wf[n, k] = round(W[n, k] * w[k]): the product of two bf16 values is exact
 // in fp32, so this is the correctly rounded product.  Eight per thread.
@@ -482,6 +499,14 @@ cudaError_t launch_swiglu(const void *gu, void *out, int64_t T, int64_t F, int n
     const int64_t fp = F / 8;
     swiglu_kernel<<<grid_for(T * fp, 256, num_sms), 256, 0, s>>>(
         static_cast<const uint4 *>(gu), static_cast<uint4 *>(out), T, fp);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rope_table(float *table, int P, int d, double theta, int num_sms,
+                              cudaStream_t s)
+{
+    rope_table_kernel<<<grid_for(int64_t(P) * (d / 2), 256, num_sms), 256, 0, s>>>(
+        reinterpret_cast<float2 *>(table), P, d, theta);
     return cudaGetLastError();
 }
 

@@ -46,8 +46,10 @@ class DecoderConfig:
     n_experts: int = 0            # > 0: a mixture-of-experts feed-forward
     top_k: int = 2
     expert_ffn: int = 1408
-    fused: bool = False           # RMSNorm folded into the next matmul, residual adds
-                                  # into the matmul epilogue (dense feed-forward only)
+    fused: bool = False           # RMSNorm folded into the next matmul, RoPE and the
+                                  # cache write in the QKV matmul's epilogue, residual
+                                  # adds in the matmul epilogue (dense feed-forward only)
+    max_pos: int = 8192           # fused form: positions covered by the rotary table
 
     @property
     def qkv_dim(self) -> int:
@@ -270,6 +272,7 @@ class ToyDecoder:
                                                                  weights["l%d.mlp_norm" % i])
             self.wf["lm_head"] = lib.bi_fold_norm_weight(weights["lm_head"],
                                                          weights["final_norm"])
+            self.rope = lib.bi_rope_table(cfg.max_pos, cfg.head_dim, cfg.theta, device=self.dev)
 
     def _to_dev(self, a: np.ndarray) -> torch.Tensor:
         return torch.from_numpy(np.ascontiguousarray(a)).to(self.dev, non_blocking=False)
@@ -295,12 +298,14 @@ class ToyDecoder:
         else:
             h, n = L.bi_rmsnorm(x, W["l0.attn_norm"], c.eps), 2
         for i in range(c.layers):
+            kv_all = PagedKV(self.k_cache[i], self.v_cache[i], bt)
             if c.fused:
-                qkv = L.bi_rmsnorm_matmul(x, self.wf["l%d.wqkv" % i], c.eps)
+                # RMSNorm, the QKV matmul, RoPE and the cache write in one launch
+                q = L.bi_rmsnorm_matmul_rope_kv(x, self.wf["l%d.wqkv" % i], c.eps, kv_all,
+                                                self.rope, pos, slots, c.n_heads)
             else:
                 qkv = L.bi_matmul(h, W["l%d.wqkv" % i])
-            kv_all = PagedKV(self.k_cache[i], self.v_cache[i], bt)
-            q = L.bi_rope_kv_write(kv_all, qkv, pos, slots, c.n_heads, c.theta)
+                q = L.bi_rope_kv_write(kv_all, qkv, pos, slots, c.n_heads, c.theta)
             if Bd:
                 kv = PagedKV(self.k_cache[i], self.v_cache[i], bt[:Bd])
                 L.bi_attention_decode(kv, q[:Bd], dec_lens, max_len, out=o[:Bd])
@@ -315,7 +320,7 @@ class ToyDecoder:
                                      out=x)
                 f = L.bi_swiglu(L.bi_rmsnorm_matmul(x, self.wf["l%d.wgu" % i], c.eps))
                 L.bi_matmul_residual(f, W["l%d.wdown" % i], x, out=x)
-                n += 6
+                n += 5
                 continue
             a = L.bi_matmul(o.view(T, c.n_heads * c.head_dim), W["l%d.wo" % i])
             h = L.bi_add_rmsnorm(x, a, W["l%d.mlp_norm" % i], c.eps)

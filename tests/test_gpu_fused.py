@@ -141,3 +141,104 @@ def test_fused_argument_errors(L):
     with pytest.raises(RuntimeError):
         L.bi_matmul_residual(x, torch.zeros((12, 16), dtype=torch.bfloat16, device="cuda"),
                              torch.zeros((4, 12), dtype=torch.bfloat16, device="cuda"))
+
+
+# ---------------------------------------------------------------- QKV epilogue
+
+THETA = 10000.0
+
+
+def qkv_case(seed, T, Hq, Hkv, d, K, num_pages=64, max_pos=4096):
+    g = rng(seed)
+    x = scaled_rows(g, T, K)
+    wf = normal_bf16(g, ((Hq + 2 * Hkv) * d, K), std=0.05)
+    pos = g.integers(0, max_pos, size=T).astype(np.int32)
+    slots = g.permutation(num_pages * 16)[:T].astype(np.int64)  # one slot per token
+    slots[::7] = -1                                           # rows that write no cache
+    return x, wf, pos, slots
+
+
+def caches(num_pages, Hkv, d):
+    return [torch.zeros((num_pages, Hkv, 16, d), dtype=torch.bfloat16, device="cuda")
+            for _ in range(2)]
+
+
+@pytest.mark.parametrize("T,Hq,Hkv,d,K", [(1, 32, 8, 128, 4096), (3, 8, 2, 64, 512),
+                                          (130, 32, 8, 128, 4096), (300, 8, 2, 128, 1000),
+                                          (257, 4, 4, 64, 256), (129, 3, 1, 128, 256)])
+def test_qkv_epilogue_equals_the_two_launches(L, T, Hq, Hkv, d, K):
+    # one tile may hold q and k heads, or k and v heads; N need not fill the last tile
+    x, wf, pos, slots = qkv_case(400 + T + d, T, Hq, Hkv, d, K, num_pages=max(64, T // 8))
+    np_ = max(64, T // 8)
+    table = L.bi_rope_table(4096, d, THETA)
+    bt = torch.zeros((1, 1), dtype=torch.int32, device="cuda")
+    k1, v1 = caches(np_, Hkv, d)
+    k2, v2 = caches(np_, Hkv, d)
+    xd, wd = dev_bf16(x), dev_bf16(wf)
+    pd, sd = torch.from_numpy(pos).cuda(), torch.from_numpy(slots).cuda()
+    L.bi_device_status()
+    q1 = L.bi_rmsnorm_matmul_rope_kv(xd, wd, EPS, bi.PagedKV(k1, v1, bt), table, pd, sd, Hq)
+    qkv = L.bi_rmsnorm_matmul(xd, wd, EPS)
+    q2 = L.bi_rope_kv_write(bi.PagedKV(k2, v2, bt), qkv, pd, sd, Hq, THETA)
+    assert L.bi_device_status() == bi.Status.OK
+    assert same_bytes(q1, q2)
+    assert same_bytes(k1, k2) and same_bytes(v1, v2)
+    if (slots >= 0).any():  # some row wrote its slot
+        assert bool(torch.any(k1 != 0)) and bool(torch.any(v1 != 0))
+
+
+def test_qkv_epilogue_parity_with_the_oracle(L):
+    T, Hq, Hkv, d, K = 40, 8, 2, 128, 512
+    x, wf, pos, slots = qkv_case(410, T, Hq, Hkv, d, K)
+    table = L.bi_rope_table(4096, d, THETA)
+    q = L.bi_rmsnorm_matmul_rope_kv(dev_bf16(x), dev_bf16(wf), EPS,
+                                    bi.PagedKV(*caches(64, Hkv, d),
+                                               torch.zeros((1, 1), dtype=torch.int32,
+                                                           device="cuda")),
+                                    table, torch.from_numpy(pos).cuda(),
+                                    torch.from_numpy(slots).cuda(), Hq)
+    # the oracle's chain: RMSNorm -> matmul (rounded to bf16, as the fused op's
+    # product is) -> RoPE at each token's position
+    prod = f32_to_bf16_bits(oracle.rmsnorm_matmul(x, wf, EPS).astype(np.float32))
+    want = oracle.rope(prod[:, :Hq * d].reshape(T, Hq, d), pos, THETA)
+    err = rowwise_normwise(to_f64(q).reshape(T, -1), want.reshape(T, -1))
+    assert err.max() <= TOL_BF16, err.max()
+
+
+def test_qkv_epilogue_rows_do_not_depend_on_the_batch(L):
+    T, Hq, Hkv, d, K = 300, 32, 8, 128, 4096
+    x, wf, pos, slots = qkv_case(420, T, Hq, Hkv, d, K)
+    slots[:] = -1  # q only
+    table = L.bi_rope_table(4096, d, THETA)
+    kv = bi.PagedKV(*caches(64, Hkv, d), torch.zeros((1, 1), dtype=torch.int32, device="cuda"))
+    xd, wd = dev_bf16(x), dev_bf16(wf)
+    pd, sd = torch.from_numpy(pos).cuda(), torch.from_numpy(slots).cuda()
+    full = L.bi_rmsnorm_matmul_rope_kv(xd, wd, EPS, kv, table, pd, sd, Hq)
+    for M in (1, 2, 129, 256, 257):
+        part = L.bi_rmsnorm_matmul_rope_kv(xd[:M], wd, EPS, kv, table, pd[:M], sd[:M], Hq)
+        assert same_bytes(part, full[:M]), M
+
+
+def test_rope_table_is_the_rounded_angles(L):
+    for d in (64, 128):
+        got = L.bi_rope_table(3000, d, THETA).cpu().numpy().astype(np.float64)
+        want = oracle.rope_angles(3000, d, THETA)
+        ulp = np.spacing(np.abs(want).astype(np.float32)).astype(np.float64)
+        assert np.all(np.abs(got - want) <= ulp), d
+
+
+def test_qkv_epilogue_bad_position_and_slot(L):
+    T, Hq, Hkv, d, K = 20, 4, 2, 64, 256
+    x, wf, pos, slots = qkv_case(430, T, Hq, Hkv, d, K, max_pos=100)
+    table = L.bi_rope_table(100, d, THETA)
+    bt = torch.zeros((1, 1), dtype=torch.int32, device="cuda")
+    kv = bi.PagedKV(*caches(64, Hkv, d), bt)
+    pos[5] = 100           # past the table: the row writes nothing
+    slots[6] = 64 * 16     # past the cache: q is written, k and v are not
+    q = torch.zeros((T, Hq, d), dtype=torch.bfloat16, device="cuda")
+    L.bi_device_status()
+    L.bi_rmsnorm_matmul_rope_kv(dev_bf16(x), dev_bf16(wf), EPS, kv, table,
+                                torch.from_numpy(pos).cuda(), torch.from_numpy(slots).cuda(), Hq,
+                                q_out=q)
+    assert L.bi_device_status() == bi.Status.DEVICE_INDEX
+    assert not bool(torch.any(q[5] != 0)) and bool(torch.any(q[6] != 0))
