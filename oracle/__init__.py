@@ -69,6 +69,7 @@ class Oracle:
         lib.oracle_rmsnorm_matmul.argtypes = [P, P, i64, i64, i64, f64, P]
         lib.oracle_matmul_residual.argtypes = [P, P, P, i64, i64, i64, P]
         lib.oracle_rope_angles.argtypes = [i32, i32, f64, P]
+        lib.oracle_rmsnorm_backward.argtypes = [P, P, P, i64, i64, f64, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
@@ -252,6 +253,18 @@ class Oracle:
         self.lib.oracle_moe_combine(_p(y), _p(ps), _p(w), T, k, H, _p(out))
         return out
 
+    # ---------------------------------------------------------- backward
+
+    def rmsnorm_backward(self, x, w, dy, eps: float):
+        """(dx [M, H], dw [H]) of y = RMSNorm(x) * w for upstream dy; float64."""
+        x, w, dy = _u16(x), _u16(w), _u16(dy)
+        M, H = x.shape
+        assert w.shape == (H,) and dy.shape == (M, H)
+        dx = np.empty((M, H), dtype=np.float64)
+        dw = np.empty((H,), dtype=np.float64)
+        self.lib.oracle_rmsnorm_backward(_p(x), _p(w), _p(dy), M, H, float(eps), _p(dx), _p(dw))
+        return dx, dw
+
     # ---------------------------------------------------------- fused matmuls
 
     def fold_norm_weight(self, W, w) -> np.ndarray:
@@ -364,6 +377,10 @@ def moe_combine(y, pos, weights) -> np.ndarray:
 
 def fold_norm_weight(W, w) -> np.ndarray:
     return default().fold_norm_weight(W, w)
+
+
+def rmsnorm_backward(x, w, dy, eps: float):
+    return default().rmsnorm_backward(x, w, dy, eps)
 
 
 def rmsnorm_matmul(x, wf, eps: float) -> np.ndarray:

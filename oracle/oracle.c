@@ -585,3 +585,40 @@ void oracle_rope_angles(int32_t P, int32_t d, double theta, double *out)
         }
     }
 }
+
+/*
+ * Backward of the RMSNorm above, for the trainer side of on-policy RL
+ * (xitu-tech news, "强化学习的突破": the trainer must reproduce the sampler's
+ * numbers, so its passes run on the same deterministic kernels).  With
+ * r = 1 / sqrt((1/H) sum_i x_i^2 + eps) and y_j = x_j r w_j, the gradients of
+ * a loss with upstream gradient dy are
+ *   dx_j = r w_j dy_j - x_j (r^3 / H) sum_i w_i dy_i x_i        (per row)
+ *   dw_j = sum over rows of dy_j x_j r
+ */
+void oracle_rmsnorm_backward(const uint16_t *x, const uint16_t *w, const uint16_t *dy,
+                             int64_t M, int64_t H, double eps, double *dx, double *dw)
+{
+    double *rs = (double *)malloc((size_t)(M > 0 ? M : 1) * sizeof(double));
+    int64_t r;
+#pragma omp parallel for schedule(static)
+    for (r = 0; r < M; ++r) {
+        double sq = 0.0, dot = 0.0;
+        for (int64_t i = 0; i < H; ++i) {
+            const double xi = bf16_to_double(x[r * H + i]);
+            sq += xi * xi;
+            dot += bf16_to_double(w[i]) * bf16_to_double(dy[r * H + i]) * xi;
+        }
+        const double inv = 1.0 / sqrt(sq / (double)H + eps);
+        rs[r] = inv;
+        for (int64_t j = 0; j < H; ++j)
+            dx[r * H + j] = bf16_to_double(w[j]) * inv * bf16_to_double(dy[r * H + j]) -
+                            bf16_to_double(x[r * H + j]) * inv * inv * inv / (double)H * dot;
+    }
+    for (int64_t j = 0; j < H; ++j) {
+        double acc = 0.0;
+        for (int64_t m = 0; m < M; ++m)
+            acc += bf16_to_double(dy[m * H + j]) * bf16_to_double(x[m * H + j]) * rs[m];
+        dw[j] = acc;
+    }
+    free(rs);
+}

@@ -695,3 +695,62 @@ def test_rope_angles_rotate_like_rope(oracle):
     c, s = t[pos, :, 0][:, None, :], t[pos, :, 1][:, None, :]
     want = np.concatenate([xw[..., :8] * c - xw[..., 8:] * s, xw[..., 8:] * c + xw[..., :8] * s], -1)
     np.testing.assert_allclose(oracle.rope(x, pos), want, rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------- backward
+
+
+def _loss_grad_fd(oracle, x, w, dy, eps, h=1e-6):
+    """Central differences of L = sum(dy * RMSNorm(x) * w) in x and w, taken
+    on the oracle's forward in float64 (inputs perturbed off the bf16 grid
+    through the exact forward formula restated with numpy)."""
+    xw, ww, dyw = widen(x), widen(w), widen(dy)
+
+    def loss(xv, wv):
+        r = 1.0 / np.sqrt((xv * xv).mean(axis=1, keepdims=True) + eps)
+        return float((dyw * xv * r * wv).sum())
+
+    gx = np.zeros_like(xw)
+    for idx in np.ndindex(*xw.shape):
+        a, b = xw.copy(), xw.copy()
+        a[idx] += h
+        b[idx] -= h
+        gx[idx] = (loss(a, ww) - loss(b, ww)) / (2 * h)
+    gw = np.zeros_like(ww)
+    for j in range(ww.shape[0]):
+        a, b = ww.copy(), ww.copy()
+        a[j] += h
+        b[j] -= h
+        gw[j] = (loss(xw, a) - loss(xw, b)) / (2 * h)
+    return gx, gw
+
+
+def test_rmsnorm_backward_matches_finite_differences(oracle):
+    g = rng(95)
+    x = normal_bf16(g, (3, 10))
+    w = uniform_bf16(g, (10,), 0.5, 1.5)
+    dy = normal_bf16(g, (3, 10))
+    dx, dw = oracle.rmsnorm_backward(x, w, dy, 1e-6)
+    gx, gw = _loss_grad_fd(oracle, x, w, dy, 1e-6)
+    np.testing.assert_allclose(dx, gx, rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(dw, gw, rtol=1e-6, atol=1e-7)
+    # the forward the differences were taken on is the oracle's own
+    xw, ww = widen(x), widen(w)
+    r = 1.0 / np.sqrt((xw * xw).mean(axis=1, keepdims=True) + 1e-6)
+    np.testing.assert_allclose(oracle.rmsnorm(x, w, 1e-6), xw * r * ww, rtol=1e-14)
+
+
+def test_rmsnorm_backward_closed_forms(oracle):
+    # dy parallel to y's direction: a row-scale-invariant map has dx orthogonal
+    # to x when eps = 0 (sum_j x_j dx_j = 0); dw with dy = 1 is sum over rows of x r
+    g = rng(96)
+    x = normal_bf16(g, (4, 16))
+    w = bf(np.ones(16))
+    dy = normal_bf16(g, (4, 16))
+    dx, _ = oracle.rmsnorm_backward(x, w, dy, 0.0)
+    np.testing.assert_allclose((dx * widen(x)).sum(axis=1), 0.0, atol=1e-12)
+    ones = bf(np.ones((4, 16)))
+    _, dw = oracle.rmsnorm_backward(x, w, ones, 1e-6)
+    xw = widen(x)
+    r = 1.0 / np.sqrt((xw * xw).mean(axis=1, keepdims=True) + 1e-6)
+    np.testing.assert_allclose(dw, (xw * r).sum(axis=0), rtol=1e-13)

@@ -112,6 +112,16 @@ MUTATIONS = [
      [pins.test_rope_angles_closed_forms, pins.test_rope_angles_rotate_like_rope]),
     ("rope_angles_cos_sin_swapped", "* 2] = cos((double)p * freq);", "* 2] = sin((double)p * freq);",
      [pins.test_rope_angles_closed_forms]),
+    ("rmsnorm_backward_r_squared", "bf16_to_double(x[r * H + j]) * inv * inv * inv / (double)H * dot;",
+     "bf16_to_double(x[r * H + j]) * inv * inv / (double)H * dot;",
+     [pins.test_rmsnorm_backward_matches_finite_differences, pins.test_rmsnorm_backward_closed_forms]),
+    ("rmsnorm_backward_dw_without_r",
+     "acc += bf16_to_double(dy[m * H + j]) * bf16_to_double(x[m * H + j]) * rs[m];",
+     "acc += bf16_to_double(dy[m * H + j]) * bf16_to_double(x[m * H + j]);",
+     [pins.test_rmsnorm_backward_matches_finite_differences, pins.test_rmsnorm_backward_closed_forms]),
+    ("rmsnorm_backward_dot_without_w", "dot += bf16_to_double(w[i]) * bf16_to_double(dy[r * H + i]) * xi;",
+     "dot += bf16_to_double(dy[r * H + i]) * xi;",
+     [pins.test_rmsnorm_backward_matches_finite_differences]),
     ("matmul_residual_drops_residual", "c[m * N + n] = bf16_to_double(r[m * N + n]) + dot;",
      "c[m * N + n] = dot;",
      [pins.test_matmul_residual_small_integers_brute_force, pins.test_matmul_residual_degenerate_cases]),
