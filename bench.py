@@ -746,6 +746,19 @@ def run_profile_case(args):
             fn = lambda i: L.bi_rope_kv_write(  # noqa: E731
                 kv, L.bi_matmul(L.bi_rmsnorm(x, w, 1e-6, out=y), Wq, out=qkv), pos, slots, Hq,
                 q_out=q)
+    elif args.profile in ("rmsnorm_backward", "matmul_backward"):
+        # the backward passes at the hidden-4096 sizes: RMSNorm of x[M, 4096];
+        # the matmul C = x W^T with W [12288, 4096] (dA and dW, 2 x 2MNK flop)
+        M = args.profile_rows
+        g = rng(14)
+        nm = norm_matmul(seed=1, M=M, H=H, N=N_COLS)
+        x, w, W = d16(nm["x"]), d16(nm["w"]), d16(nm["W"])
+        if args.profile == "rmsnorm_backward":
+            dy = d16(normal_bf16(g, (M, H)))
+            fn = lambda i: L.bi_rmsnorm_backward(x, w, dy, 1e-6)  # noqa: E731
+        else:
+            dc = d16(normal_bf16(g, (M, N_COLS)))
+            fn = lambda i: L.bi_matmul_backward(dc, x, W)  # noqa: E731
     elif args.profile == "sample":
         # 256 rows of lm_head logits (vocab 32000), temperature 0.8, nucleus 0.95
         g = rng(5)
@@ -893,7 +906,7 @@ def main(argv=None):
     ap.add_argument("--profile", choices=["rmsnorm", "matmul", "decode", "prefill", "copy",
                                           "sample", "rmsnorm_matmul", "rmsnorm_then_matmul",
                                           "matmul_residual", "matmul_rows", "qkv_fused",
-                                          "qkv_unfused"],
+                                          "qkv_unfused", "rmsnorm_backward", "matmul_backward"],
                     help="run one kernel alone on a reduced case (for ncu)")
     ap.add_argument("--profile-batch", type=int, default=32)
     ap.add_argument("--profile-seq", type=int, default=4096)

@@ -202,6 +202,45 @@ bi_status bi_matmul_grouped(const void *a, const void *w, void *c, const int64_t
  *   Requirements as bi_matmul.
  */
 /*
+ * Backward passes for a trainer that must reproduce the sampler's numbers
+ * (on-policy RL; xitu-tech news, "强化学习的突破").  Every reduction runs in
+ * a fixed order, so the results are the same bits on every run.
+ *
+ * bi_rmsnorm_backward -- gradients of y = RMSNorm(x) * w (bi_rmsnorm) for an
+ *   upstream gradient dy, with r = rsqrt(mean_i x_i^2 + eps):
+ *     dx[m, j] = r w_j dy[m, j] - x[m, j] (r^3 / H) sum_i w_i dy[m, i] x[m, i]
+ *     dw[j]    = sum_m dy[m, j] x[m, j] r[m]
+ *   x, dy : device bf16 [M, H];  w : bf16 [H];  dx : [M, H], dw : [H] of
+ *   out_dtype.  A row's dx depends on that row only (one block per row, sums
+ *   in an order fixed by H); dw adds the rows in chunks of 256 from row 0,
+ *   each chunk ascending, then the chunks ascending.  ws : device workspace
+ *   of bi_rmsnorm_backward_workspace_bytes(M, H) bytes.  H % 8 == 0,
+ *   8 <= H <= 65536, 16-byte aligned pointers.
+ *
+ * bi_transpose -- out[c, r] = a[r, c] for bf16 a [R, C]; out has rows of
+ *   ld_out >= R values, those past R set to 0.  A bit copy.
+ *
+ * bi_matmul_backward -- for C = A W^T (bi_matmul):  dA = dC W  [M, K]  and
+ *   dW = dC^T A  [N, K], both on the invariant matmul (the transposes of W,
+ *   dC and A made in the workspace by bi_transpose; dW's sum over the M rows
+ *   is that matmul's K loop, rows padded to a multiple of 8 with zeros).
+ *   dc : bf16 [M, N];  a : bf16 [M, K];  w : bf16 [N, K];  da, dw : of
+ *   out_dtype, either may be NULL.  ws : bi_matmul_backward_workspace_bytes
+ *   (M, N, K) bytes.  Requirements as bi_matmul.  A row of dA depends on
+ *   that row of dC only.
+ */
+size_t bi_rmsnorm_backward_workspace_bytes(int64_t M, int64_t H);
+bi_status bi_rmsnorm_backward(const void *x, const void *w, const void *dy, void *dx, void *dw,
+                              int64_t M, int64_t H, float eps, bi_dtype out_dtype, void *ws,
+                              size_t ws_bytes, void *stream);
+bi_status bi_transpose(const void *a, void *out, int64_t R, int64_t C, int64_t ld_out,
+                       void *stream);
+size_t bi_matmul_backward_workspace_bytes(int64_t M, int64_t N, int64_t K);
+bi_status bi_matmul_backward(const void *dc, const void *a, const void *w, void *da, void *dw,
+                             int64_t M, int64_t N, int64_t K, bi_dtype out_dtype, void *ws,
+                             size_t ws_bytes, void *stream);
+
+/*
  * bi_rope_table -- the rotary angles of bi_rope_kv_write as a table:
  *   table[p, i] = ( cos(p theta^(-2i/d)), sin(p theta^(-2i/d)) ),  p < max_pos, i < d/2
  * evaluated in double precision and rounded to fp32 exactly as

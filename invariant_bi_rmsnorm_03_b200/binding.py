@@ -112,7 +112,9 @@ class Library:
                "bi_swiglu", "bi_argmax", "bi_sample", "bi_moe_route", "bi_moe_dispatch",
                "bi_moe_combine", "bi_matmul_grouped", "bi_fold_norm_weight",
                "bi_rmsnorm_matmul", "bi_matmul_residual", "bi_rope_table",
-               "bi_rmsnorm_matmul_rope_kv")
+               "bi_rmsnorm_matmul_rope_kv", "bi_rmsnorm_backward",
+               "bi_rmsnorm_backward_workspace_bytes", "bi_transpose", "bi_matmul_backward",
+               "bi_matmul_backward_workspace_bytes")
 
     def __init__(self, path: str):
         if not os.path.exists(path):
@@ -156,13 +158,21 @@ class Library:
         L.bi_matmul_residual.argtypes = [P, P, P, P, i64, i64, i64, P]
         L.bi_rope_table.argtypes = [P, i32, i32, f32, P]
         L.bi_rmsnorm_matmul_rope_kv.argtypes = [P, P, f32, kvp, P, i32, P, P, P, i64, i64, i32, P]
+        L.bi_rmsnorm_backward_workspace_bytes.argtypes = [i64, i64]
+        L.bi_rmsnorm_backward_workspace_bytes.restype = sz
+        L.bi_rmsnorm_backward.argtypes = [P, P, P, P, P, i64, i64, f32, st, P, sz, P]
+        L.bi_transpose.argtypes = [P, P, i64, i64, i64, P]
+        L.bi_matmul_backward_workspace_bytes.argtypes = [i64, i64, i64]
+        L.bi_matmul_backward_workspace_bytes.restype = sz
+        L.bi_matmul_backward.argtypes = [P, P, P, P, P, i64, i64, i64, st, P, sz, P]
         for name in ("bi_rmsnorm", "bi_matmul", "bi_kv_write", "bi_attention_decode",
                      "bi_attention_prefill", "bi_device_status", "bi_debug_bounded_wait",
                      "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write", "bi_swiglu",
                      "bi_argmax", "bi_sample", "bi_moe_route", "bi_moe_dispatch",
                      "bi_moe_combine", "bi_matmul_grouped", "bi_fold_norm_weight",
                      "bi_rmsnorm_matmul", "bi_matmul_residual", "bi_rope_table",
-                     "bi_rmsnorm_matmul_rope_kv"):
+                     "bi_rmsnorm_matmul_rope_kv", "bi_rmsnorm_backward", "bi_transpose",
+                     "bi_matmul_backward"):
             getattr(L, name).restype = st
         self.lib = L
 
@@ -391,6 +401,52 @@ class Library:
             int(rope_table.shape[0]), _ptr(positions), _ptr(slot_mapping), _ptr(q_out), T, K, Hq,
             _stream(stream)))
         return q_out
+
+    # ------------------------------------------------------------ backward
+    def bi_rmsnorm_backward(self, x: torch.Tensor, w: torch.Tensor, dy: torch.Tensor,
+                            eps: float = 1e-6, out_dtype=torch.bfloat16, stream=None):
+        """(dx [M, H], dw [H]) of y = RMSNorm(x) * w for the upstream gradient dy."""
+        _need(x, "x", torch.bfloat16)
+        M, H = x.shape
+        _need(w, "w", torch.bfloat16, (H,))
+        _need(dy, "dy", torch.bfloat16, (M, H))
+        dx = torch.empty((M, H), dtype=out_dtype, device=x.device)
+        dw = torch.empty((H,), dtype=out_dtype, device=x.device)
+        need = int(self.lib.bi_rmsnorm_backward_workspace_bytes(M, H))
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+        self._check("bi_rmsnorm_backward", self.lib.bi_rmsnorm_backward(
+            _ptr(x), _ptr(w), _ptr(dy), _ptr(dx), _ptr(dw), M, H, float(eps), _DT[out_dtype],
+            _ptr(ws), ws.numel(), _stream(stream)))
+        return dx, dw
+
+    def bi_transpose(self, a: torch.Tensor, ld_out: int | None = None, stream=None) -> torch.Tensor:
+        """a.T for bf16 a [R, C], as [C, ld_out] with the columns past R zero."""
+        _need(a, "a", torch.bfloat16)
+        R, C = a.shape
+        ld = R if ld_out is None else int(ld_out)
+        out = torch.empty((C, ld), dtype=torch.bfloat16, device=a.device)
+        self._check("bi_transpose", self.lib.bi_transpose(_ptr(a), _ptr(out), R, C, ld,
+                                                          _stream(stream)))
+        return out
+
+    def bi_matmul_backward(self, dc: torch.Tensor, a: torch.Tensor, w: torch.Tensor,
+                           out_dtype=torch.bfloat16, want_da: bool = True, want_dw: bool = True,
+                           stream=None):
+        """(dA, dW) for C = a @ w.T: dA = dc @ w [M, K], dW = dc.T @ a [N, K]."""
+        _need(dc, "dc", torch.bfloat16)
+        M, N = dc.shape
+        _need(a, "a", torch.bfloat16)
+        K = a.shape[1]
+        _need(a, "a", torch.bfloat16, (M, K))
+        _need(w, "w", torch.bfloat16, (N, K))
+        da = torch.empty((M, K), dtype=out_dtype, device=dc.device) if want_da else None
+        dw = torch.empty((N, K), dtype=out_dtype, device=dc.device) if want_dw else None
+        need = int(self.lib.bi_matmul_backward_workspace_bytes(M, N, K))
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dc.device)
+        self._check("bi_matmul_backward", self.lib.bi_matmul_backward(
+            _ptr(dc), _ptr(a), _ptr(w), _ptr(da), _ptr(dw), M, N, K, _DT[out_dtype], _ptr(ws),
+            ws.numel(), _stream(stream)))
+        return da, dw
 
     def bi_swiglu(self, gu: torch.Tensor, out=None, stream=None) -> torch.Tensor:
         """silu(gate) * up of gu [T, 2F] = [gate | up] -> [T, F]."""

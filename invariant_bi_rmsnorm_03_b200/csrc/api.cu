@@ -285,6 +285,108 @@ bi_status bi_matmul_residual(const void *a, const void *w, const void *r, void *
                                            static_cast<cudaStream_t>(stream)));
 }
 
+size_t bi_rmsnorm_backward_workspace_bytes(int64_t M, int64_t H)
+{
+    if (M <= 0 || H <= 0) return 0;
+    return bi::rmsnorm_backward_ws_bytes(M, H);
+}
+
+bi_status bi_rmsnorm_backward(const void *x, const void *w, const void *dy, void *dx, void *dw,
+                              int64_t M, int64_t H, float eps, bi_dtype out_dtype, void *ws,
+                              size_t ws_bytes, void *stream)
+{
+    if (M < 0 || H < 8 || H % 8 != 0 || H > 65536) return BI_ERR_INVALID;
+    if (out_dtype != BI_BF16 && out_dtype != BI_F32) return BI_ERR_INVALID;
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return BI_ERR_INVALID;
+    if (M == 0) return BI_OK;
+    if (!x || !w || !dy || !dx || !dw || !aligned16(x) || !aligned16(w) || !aligned16(dy) ||
+        !aligned16(dx) || !aligned16(dw))
+        return BI_ERR_INVALID;
+    if (!ws || ws_bytes < bi::rmsnorm_backward_ws_bytes(M, H) || !aligned16(ws))
+        return BI_ERR_WORKSPACE;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_rmsnorm_backward(x, w, dy, dx, dw, M, H, eps, out_dtype == BI_F32,
+                                                 ws, d->num_sms,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
+bi_status bi_transpose(const void *a, void *out, int64_t R, int64_t C, int64_t ld_out,
+                       void *stream)
+{
+    if (R < 0 || C < 0 || ld_out < R) return BI_ERR_INVALID;
+    if (R == 0 || C == 0) return BI_OK;
+    if (!a || !out) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_transpose(a, out, R, C, ld_out, d->num_sms,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+int64_t round8(int64_t v) { return (v + 7) / 8 * 8; }
+size_t region(int64_t elems) { return (size_t(elems) * 2 + 255) / 256 * 256; }
+}  // namespace
+
+size_t bi_matmul_backward_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    const int64_t M8 = round8(M);
+    return region(K * N) + region(N * M8) + region(K * M8);
+}
+
+bi_status bi_matmul_backward(const void *dc, const void *a, const void *w, void *da, void *dw,
+                             int64_t M, int64_t N, int64_t K, bi_dtype out_dtype, void *ws,
+                             size_t ws_bytes, void *stream)
+{
+    if (!gemm_shape_ok(M, N, K)) return BI_ERR_INVALID;
+    if (out_dtype != BI_BF16 && out_dtype != BI_F32) return BI_ERR_INVALID;
+    if (M == 0) return BI_OK;
+    if (!dc || !a || !w || (!da && !dw)) return BI_ERR_INVALID;
+    if (!aligned16(dc) || !aligned16(a) || !aligned16(w) || (da && !aligned16(da)) ||
+        (dw && !aligned16(dw)))
+        return BI_ERR_INVALID;
+    const int64_t M8 = round8(M);
+    if (M8 > INT32_MAX) return BI_ERR_INVALID;
+    if (!ws || ws_bytes < bi_matmul_backward_workspace_bytes(M, N, K) || !aligned16(ws))
+        return BI_ERR_WORKSPACE;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    void *wt = base;                                  // W^T  [K, N]
+    void *dct = base + region(K * N);                 // dC^T [N, M8]
+    void *at = base + region(K * N) + region(N * M8); // A^T  [K, M8]
+    const bool f32 = out_dtype == BI_F32;
+    cudaError_t e;
+    if (da) {
+        // dA [M, K] = dC [M, N] (W^T [K, N])^T
+        if ((e = bi::launch_transpose(w, wt, N, K, N, d->num_sms, s)) != cudaSuccess)
+            return from_cuda(e);
+        CUtensorMap ta, tw;
+        if ((st = gemm_maps(dc, wt, M, K, N, &ta, &tw)) != BI_OK) return st;
+        if ((e = bi::launch_gemm(ta, tw, da, int(M), int(K), int(N), f32, nullptr, 1, d->num_sms,
+                                 d->status, bi::kDefaultTimeoutNs, s)) != cudaSuccess)
+            return from_cuda(e);
+    }
+    if (dw) {
+        // dW [N, K] = dC^T [N, M8] (A^T [K, M8])^T; the zero columns past M add nothing
+        if ((e = bi::launch_transpose(dc, dct, M, N, M8, d->num_sms, s)) != cudaSuccess)
+            return from_cuda(e);
+        if ((e = bi::launch_transpose(a, at, M, K, M8, d->num_sms, s)) != cudaSuccess)
+            return from_cuda(e);
+        CUtensorMap ta, tw;
+        if ((st = gemm_maps(dct, at, N, K, M8, &ta, &tw)) != BI_OK) return st;
+        if ((e = bi::launch_gemm(ta, tw, dw, int(N), int(K), int(M8), f32, nullptr, 1, d->num_sms,
+                                 d->status, bi::kDefaultTimeoutNs, s)) != cudaSuccess)
+            return from_cuda(e);
+    }
+    return BI_OK;
+}
+
 bi_status bi_add_rmsnorm(void *x, const void *delta, const void *w, void *y, int64_t M,
                          int64_t H, float eps, bi_dtype out_dtype, void *stream)
 {

@@ -64,6 +64,15 @@ cudaError_t launch_rope_table(float *table, int P, int d, double theta, int num_
 cudaError_t launch_fold_norm_weight(const void *W, const void *w, void *wf, int64_t N, int64_t K,
                                     int num_sms, cudaStream_t s);
 
+// ---------------------------------------------------------------- backward
+size_t rmsnorm_backward_ws_bytes(int64_t M, int64_t H);
+cudaError_t launch_rmsnorm_backward(const void *x, const void *w, const void *dy, void *dx,
+                                    void *dw, int64_t M, int64_t H, float eps, bool out_f32,
+                                    void *ws, int num_sms, cudaStream_t s);
+// out[c, r] = a[r, c] (bf16), rows of out padded with zeros to ld_out >= R
+cudaError_t launch_transpose(const void *a, void *out, int64_t R, int64_t C, int64_t ld_out,
+                             int num_sms, cudaStream_t s);
+
 // ---------------------------------------------------------------- KV write
 cudaError_t launch_kv_write(void *k_cache, void *v_cache, int64_t num_pages, int Hkv, int d,
                             const void *k_new, const void *v_new, const int64_t *slots,
