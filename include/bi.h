@@ -212,7 +212,7 @@ bi_status bi_matmul_grouped(const void *a, const void *w, void *c, const int64_t
  *     dw[j]    = sum_m dy[m, j] x[m, j] r[m]
  *   x, dy : device bf16 [M, H];  w : bf16 [H];  dx : [M, H], dw : [H] of
  *   out_dtype.  A row's dx depends on that row only (one block per row, sums
- *   in an order fixed by H); dw adds the rows in chunks of 256 from row 0,
+ *   in an order fixed by H); dw adds the rows in chunks of 64 from row 0,
  *   each chunk ascending, then the chunks ascending.  ws : device workspace
  *   of bi_rmsnorm_backward_workspace_bytes(M, H) bytes.  H % 8 == 0,
  *   8 <= H <= 65536, 16-byte aligned pointers.

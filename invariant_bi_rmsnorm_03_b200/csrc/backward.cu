@@ -5,7 +5,7 @@
 //
 //   RMSNorm   dx: one block per row, every sum in a fixed order that depends
 //             on H only, so a row's dx does not depend on the batch.
-//             dw: a sum over rows -- in chunks of 256 rows counted from row 0,
+//             dw: a sum over rows -- in chunks of 64 rows counted from row 0,
 //             each chunk's rows in ascending order, then the chunks in
 //             ascending order: the same bits on every run.
 //   matmul    through the invariant GEMM: dA = dC W as dC (W^T)^T and
@@ -23,7 +23,8 @@ namespace bi {
 namespace {
 
 constexpr int kBwdThreads = 256;
-constexpr int kDwChunk = 256;  // rows per partial sum of dw
+constexpr int kDwChunk = 64;   // rows per partial sum of dw
+constexpr int kDwBatch = 8;    // rows whose loads are in flight together
 
 __device__ __forceinline__ float lo_f(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float hi_f(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
@@ -120,15 +121,29 @@ __global__ void rmsnorm_bwd_dw_partial_kernel(const uint4 *__restrict__ x,
         const int64_t ch = it / pieces, p = it - ch * pieces;
         const int64_t m1 = (ch + 1) * kDwChunk < M ? (ch + 1) * kDwChunk : M;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int64_t m = ch * kDwChunk; m < m1; ++m) {
-            const uint4 a = __ldg(x + m * pieces + p), b = __ldg(dy + m * pieces + p);
-            const float r = __ldg(rs + m);
-            const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+        for (int64_t m0 = ch * kDwChunk; m0 < m1; m0 += kDwBatch) {
+            // the loads of up to kDwBatch rows first, then their terms in row order
+            uint4 a[kDwBatch], b[kDwBatch];
+            float r[kDwBatch];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                acc[2 * j] = __fadd_rn(acc[2 * j], __fmul_rn(__fmul_rn(lo_f(bv[j]), lo_f(av[j])), r));
-                acc[2 * j + 1] =
-                    __fadd_rn(acc[2 * j + 1], __fmul_rn(__fmul_rn(hi_f(bv[j]), hi_f(av[j])), r));
+            for (int u = 0; u < kDwBatch; ++u) {
+                const bool in = m0 + u < m1;
+                a[u] = in ? __ldg(x + (m0 + u) * pieces + p) : make_uint4(0u, 0u, 0u, 0u);
+                b[u] = in ? __ldg(dy + (m0 + u) * pieces + p) : make_uint4(0u, 0u, 0u, 0u);
+                r[u] = in ? __ldg(rs + m0 + u) : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < kDwBatch; ++u) {
+                if (m0 + u >= m1) break;
+                const uint32_t av[4] = {a[u].x, a[u].y, a[u].z, a[u].w};
+                const uint32_t bv[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[2 * j] =
+                        __fadd_rn(acc[2 * j], __fmul_rn(__fmul_rn(lo_f(bv[j]), lo_f(av[j])), r[u]));
+                    acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1],
+                                               __fmul_rn(__fmul_rn(hi_f(bv[j]), hi_f(av[j])), r[u]));
+                }
             }
         }
         float4 *dst = reinterpret_cast<float4 *>(partial + ch * H + 8 * p);
