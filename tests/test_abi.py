@@ -108,3 +108,53 @@ def test_debug_wait_rejects_out_of_range_limits(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(ImportError):
         binding.Library(str(tmp_path / "libbi.so"))
+
+
+def test_fused_matmuls_reject_bad_arguments(lib):
+    L, INV, OK = lib.lib, binding.Status.INVALID, binding.Status.OK
+    assert L.bi_fold_norm_weight(FAKE, FAKE, FAKE, 4, 12, None) == INV          # K % 8
+    assert L.bi_fold_norm_weight(None, FAKE, FAKE, 4, 64, None) == INV
+    assert L.bi_fold_norm_weight(None, None, None, 0, 64, None) == OK           # N == 0
+    assert L.bi_rmsnorm_matmul(FAKE, FAKE, FAKE, 4, 12, 64, 1e-6, 0, None) == INV  # N % 8
+    assert L.bi_rmsnorm_matmul(FAKE, FAKE, FAKE, 4, 64, 64, -1.0, 0, None) == INV  # eps < 0
+    assert L.bi_rmsnorm_matmul(FAKE, FAKE, FAKE, 4, 64, 64, float("inf"), 0, None) == INV
+    assert L.bi_rmsnorm_matmul(FAKE, FAKE, FAKE, 4, 64, 64, 1e-6, 9, None) == INV   # dtype
+    assert L.bi_rmsnorm_matmul(None, None, None, 0, 64, 64, 1e-6, 0, None) == OK    # M == 0
+    assert L.bi_matmul_residual(FAKE, FAKE, FAKE, FAKE, 4, 64, 12, None) == INV     # K % 8
+    assert L.bi_matmul_residual(FAKE, FAKE, None, FAKE, 4, 64, 64, None) == INV     # no R
+    assert L.bi_matmul_residual(None, None, None, None, 0, 64, 64, None) == OK
+
+
+def test_qkv_epilogue_and_angle_table_reject_bad_arguments(lib):
+    L, INV, OK = lib.lib, binding.Status.INVALID, binding.Status.OK
+    assert L.bi_rope_table(FAKE, 0, 128, 10000.0, None) == INV                  # no positions
+    assert L.bi_rope_table(FAKE, 16, 96, 10000.0, None) == INV                  # head_dim
+    assert L.bi_rope_table(FAKE, 16, 128, 1.0, None) == INV                     # theta <= 1
+    assert L.bi_rope_table(P(0x10004), 16, 128, 10000.0, None) == INV           # alignment
+    call = lambda kv, Hq=4, T=3, K=64: L.bi_rmsnorm_matmul_rope_kv(  # noqa: E731
+        FAKE, FAKE, 1e-6, ctypes.byref(kv), FAKE, 4096, FAKE, FAKE, FAKE, T, K, Hq, None)
+    assert call(_kv(page_size=8)) == INV
+    assert call(_kv(), Hq=3) == INV                                             # Hq % Hkv
+    assert call(_kv(), K=12) == INV                                             # K % 8
+    assert call(_kv(), T=0) == OK
+
+
+def test_backward_passes_reject_bad_arguments(lib):
+    L, INV, OK, WS = lib.lib, binding.Status.INVALID, binding.Status.OK, binding.Status.WORKSPACE
+    bwd = lambda M=4, H=64, ws=FAKE, nb=1 << 20, eps=1e-6: L.bi_rmsnorm_backward(  # noqa: E731
+        FAKE, FAKE, FAKE, FAKE, FAKE, M, H, eps, 0, ws, nb, None)
+    assert bwd(H=12) == INV
+    assert bwd(eps=float("nan")) == INV
+    assert bwd(nb=0) == WS
+    assert bwd(ws=None) == WS
+    assert bwd(M=0) == OK
+    assert L.bi_rmsnorm_backward_workspace_bytes(300, 64) >= 300 * 4 + 5 * 64 * 4
+    assert L.bi_transpose(FAKE, FAKE, 8, 4, 7, None) == INV                     # ld_out < R
+    assert L.bi_transpose(None, None, 0, 4, 0, None) == OK
+    mb = lambda da=FAKE, dw=FAKE, M=4, nb=1 << 30: L.bi_matmul_backward(  # noqa: E731
+        FAKE, FAKE, FAKE, da, dw, M, 64, 64, 0, FAKE, nb, None)
+    assert mb(da=None, dw=None) == INV
+    assert mb(nb=16) == WS
+    assert mb(M=0) == OK
+    # W^T, dC^T and A^T, each region rounded up to 256 bytes, rows padded to 8
+    assert L.bi_matmul_backward_workspace_bytes(5, 64, 32) == 4096 + 1024 + 512
