@@ -44,9 +44,9 @@
 //   residual  C[m, :] = round(R[m, :] + round(acc[m, :])), R read in the
 //             epilogue (it may be C itself).
 //   QKV       the columns are q, k and v heads: the rounded product goes
-//             through RoPE and the cache write in the epilogue (qkv_epilogue),
-//             with or without the norm form.
-// Neither changes the K order of the product; both are per-row.
+//             through RoPE and the cache write in the epilogue (qkv_epilogue);
+//             the library uses it together with the norm form.
+// None of them changes the K order of the product; all of them act per row.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
