@@ -282,6 +282,9 @@ class ToyDecoder:
         L, c, W = self.L, self.cfg, self.w
         T = len(plan.tokens)
         Bd = len(plan.dec)
+        if c.fused and T and int(plan.positions.max()) >= c.max_pos:
+            raise ValueError("position %d is past the rotary table (max_pos %d)"
+                             % (int(plan.positions.max()), c.max_pos))
         tokens, pos, slots = self._to_dev(plan.tokens), self._to_dev(plan.positions), \
             self._to_dev(plan.slots)
         bt = self._to_dev(plan.block_table)
