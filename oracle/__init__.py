@@ -70,6 +70,8 @@ class Oracle:
         lib.oracle_matmul_residual.argtypes = [P, P, P, i64, i64, i64, P]
         lib.oracle_rope_angles.argtypes = [i32, i32, f64, P]
         lib.oracle_rmsnorm_backward.argtypes = [P, P, P, i64, i64, f64, P, P]
+        lib.oracle_attention_backward.argtypes = [P, P, i64, i32, P, P, P, i32, P, P, i32, i32,
+                                                  P, i32, f64, P, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
@@ -265,6 +267,30 @@ class Oracle:
         self.lib.oracle_rmsnorm_backward(_p(x), _p(w), _p(dy), M, H, float(eps), _p(dx), _p(dw))
         return dx, dw
 
+    def attention_backward(self, q_rows, dout_rows, row_seq, row_head, row_pos, Hq: int,
+                           k_cache, v_cache, block_table, scale: float | None = None):
+        """(dq [R, d], dk, dv [num_pages, Hkv, 16, d]) of ``attention`` for the
+        upstream gradients ``dout_rows`` [R, d] (bf16 bits); float64."""
+        q_rows, dout_rows = _u16(q_rows), _u16(dout_rows)
+        k_cache, v_cache = _u16(k_cache), _u16(v_cache)
+        R, d = q_rows.shape
+        num_pages, Hkv, page, d2 = k_cache.shape
+        assert page == 16 and d2 == d and Hq % Hkv == 0 and dout_rows.shape == (R, d)
+        bt = np.ascontiguousarray(block_table, dtype=np.int32)
+        rs = np.ascontiguousarray(row_seq, dtype=np.int32)
+        rh = np.ascontiguousarray(row_head, dtype=np.int32)
+        rp = np.ascontiguousarray(row_pos, dtype=np.int32)
+        if scale is None:
+            scale = 1.0 / np.sqrt(d)
+        dq = np.empty((R, d), dtype=np.float64)
+        dk = np.empty(k_cache.shape, dtype=np.float64)
+        dv = np.empty(k_cache.shape, dtype=np.float64)
+        self.lib.oracle_attention_backward(_p(q_rows), _p(dout_rows), R, d, _p(rs), _p(rh),
+                                           _p(rp), Hq, _p(k_cache), _p(v_cache), Hkv, num_pages,
+                                           _p(bt), bt.shape[1], float(scale), _p(dq), _p(dk),
+                                           _p(dv))
+        return dq, dk, dv
+
     # ---------------------------------------------------------- fused matmuls
 
     def fold_norm_weight(self, W, w) -> np.ndarray:
@@ -381,6 +407,12 @@ def fold_norm_weight(W, w) -> np.ndarray:
 
 def rmsnorm_backward(x, w, dy, eps: float):
     return default().rmsnorm_backward(x, w, dy, eps)
+
+
+def attention_backward(q_rows, dout_rows, row_seq, row_head, row_pos, Hq: int, k_cache,
+                       v_cache, block_table, scale: float | None = None):
+    return default().attention_backward(q_rows, dout_rows, row_seq, row_head, row_pos, Hq,
+                                        k_cache, v_cache, block_table, scale)
 
 
 def rmsnorm_matmul(x, wf, eps: float) -> np.ndarray:

@@ -622,3 +622,73 @@ void oracle_rmsnorm_backward(const uint16_t *x, const uint16_t *w, const uint16_
     }
     free(rs);
 }
+
+/*
+ * Backward of oracle_attention for an upstream gradient dO of each query row
+ * (the trainer side of on-policy RL; xitu-tech news, "强化学习的突破").  With
+ * p_j the softmax weights of the visible keys and o = sum_j p_j v_j:
+ *   dv_j += p_j dO,   dp_j = dO . v_j,   ds_j = p_j (dp_j - sum_i p_i dp_i),
+ *   dq = scale sum_j ds_j k_j,           dk_j += scale ds_j q.
+ * dk and dv are sums over every row that sees the key (all query heads of
+ * the kv group, all positions), returned in the logical cache layout
+ * [num_pages, Hkv, 16, d].  Rows are taken one after another.
+ */
+void oracle_attention_backward(const uint16_t *q, const uint16_t *dout, int64_t R, int32_t d,
+                               const int32_t *row_seq, const int32_t *row_head,
+                               const int32_t *row_pos, int32_t Hq, const uint16_t *k_cache,
+                               const uint16_t *v_cache, int32_t Hkv, int32_t num_pages,
+                               const int32_t *block_table, int32_t max_pages, double scale,
+                               double *dq, double *dk, double *dv)
+{
+    const int64_t cache_elems = (int64_t)num_pages * Hkv * ORACLE_PAGE * d;
+    for (int64_t e = 0; e < cache_elems; ++e) {
+        dk[e] = 0.0;
+        dv[e] = 0.0;
+    }
+    for (int64_t r = 0; r < R; ++r) {
+        const int32_t kvh = row_head[r] / (Hq / Hkv);
+        const int64_t visible = (int64_t)row_pos[r] + 1;
+        const uint16_t *qr = q + r * d, *gr = dout + r * d;
+        double *logit = (double *)malloc((size_t)visible * sizeof(double));
+        double *wt = (double *)malloc((size_t)visible * sizeof(double));
+        double *dp = (double *)malloc((size_t)visible * sizeof(double));
+        int64_t *off = (int64_t *)malloc((size_t)visible * sizeof(int64_t));
+        double top = -INFINITY;
+        for (int64_t key = 0; key < visible; ++key) {
+            const int64_t phys = block_table[(int64_t)row_seq[r] * max_pages + key / ORACLE_PAGE];
+            off[key] = ((phys * Hkv + kvh) * ORACLE_PAGE + key % ORACLE_PAGE) * d;
+            double dot = 0.0;
+            for (int32_t i = 0; i < d; ++i)
+                dot += bf16_to_double(qr[i]) * bf16_to_double(k_cache[off[key] + i]);
+            logit[key] = scale * dot;
+            if (logit[key] > top) top = logit[key];
+        }
+        double total = 0.0;
+        for (int64_t key = 0; key < visible; ++key) {
+            wt[key] = exp(logit[key] - top);
+            total += wt[key];
+        }
+        double mean_dp = 0.0;
+        for (int64_t key = 0; key < visible; ++key) {
+            wt[key] /= total;
+            double s = 0.0;
+            for (int32_t i = 0; i < d; ++i)
+                s += bf16_to_double(gr[i]) * bf16_to_double(v_cache[off[key] + i]);
+            dp[key] = s;
+            mean_dp += wt[key] * dp[key];
+        }
+        for (int32_t i = 0; i < d; ++i) dq[r * d + i] = 0.0;
+        for (int64_t key = 0; key < visible; ++key) {
+            const double ds = wt[key] * (dp[key] - mean_dp);
+            for (int32_t i = 0; i < d; ++i) {
+                dq[r * d + i] += scale * ds * bf16_to_double(k_cache[off[key] + i]);
+                dk[off[key] + i] += scale * ds * bf16_to_double(qr[i]);
+                dv[off[key] + i] += wt[key] * bf16_to_double(gr[i]);
+            }
+        }
+        free(logit);
+        free(wt);
+        free(dp);
+        free(off);
+    }
+}

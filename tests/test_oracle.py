@@ -754,3 +754,80 @@ def test_rmsnorm_backward_closed_forms(oracle):
     xw = widen(x)
     r = 1.0 / np.sqrt((xw * xw).mean(axis=1, keepdims=True) + 1e-6)
     np.testing.assert_allclose(dw, (xw * r).sum(axis=0), rtol=1e-13)
+
+
+def _attn_case(seed, L=7, Hq=4, Hkv=2, d=4):
+    g = rng(seed)
+    K, V = normal_bf16(g, (L, Hkv, d)), normal_bf16(g, (L, Hkv, d))
+    kc, vc, bt = _contig_cache(K, V)
+    rows = [(h, t) for h in range(Hq) for t in (2, L - 1)]
+    q = normal_bf16(g, (len(rows), d))
+    do = normal_bf16(g, (len(rows), d))
+    heads = np.array([h for h, _ in rows])
+    pos = np.array([t for _, t in rows])
+    return q, do, heads, pos, kc, vc, bt
+
+
+def _attn_forward_np(q, kc, vc, heads, pos, Hq, scale):
+    """softmax(scale q.k) v over keys 0..t of the contiguous cache, float64."""
+    Hkv, d = kc.shape[1], kc.shape[3]
+    Kl = kc.transpose(0, 2, 1, 3).reshape(-1, Hkv, d)
+    Vl = vc.transpose(0, 2, 1, 3).reshape(-1, Hkv, d)
+    out = np.zeros_like(q)
+    for r in range(q.shape[0]):
+        g, t = heads[r] // (Hq // Hkv), pos[r]
+        s = scale * (Kl[: t + 1, g] @ q[r])
+        p = np.exp(s - s.max())
+        out[r] = (p / p.sum()) @ Vl[: t + 1, g]
+    return out
+
+
+def test_attention_backward_matches_finite_differences(oracle):
+    Hq, d = 4, 4
+    q, do, heads, pos, kc, vc, bt = _attn_case(97, Hq=Hq, d=d)
+    R, scale = q.shape[0], 0.7
+    dq, dk, dv = oracle.attention_backward(q, do, np.zeros(R), heads, pos, Hq, kc, vc, bt, scale)
+    qw, dow, kw, vw = widen(q), widen(do), widen(kc), widen(vc)
+    # the numpy forward is the oracle's forward
+    np.testing.assert_allclose(_attn_forward_np(qw, kw, vw, heads, pos, Hq, scale),
+                               oracle.attention(q, np.zeros(R), heads, pos, Hq, kc, vc, bt,
+                                                scale=scale), rtol=1e-13, atol=1e-15)
+
+    def loss(qv, kv, vv):
+        return float((dow * _attn_forward_np(qv, kv, vv, heads, pos, Hq, scale)).sum())
+
+    h = 1e-6
+    for arr, grad, which in ((qw, dq, 0), (kw, dk, 1), (vw, dv, 2)):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(*arr.shape):
+            a, b = arr.copy(), arr.copy()
+            a[idx] += h
+            b[idx] -= h
+            args_a = [qw, kw, vw]
+            args_b = [qw, kw, vw]
+            args_a[which], args_b[which] = a, b
+            fd[idx] = (loss(*args_a) - loss(*args_b)) / (2 * h)
+        np.testing.assert_allclose(grad, fd, rtol=1e-6, atol=1e-8)
+
+
+def test_attention_backward_closed_forms(oracle):
+    # identical keys: uniform weights, so sum_j ds_j = 0 and dq = 0; and each
+    # visible value row gets dO / (t + 1) from every row that sees it
+    g = rng(98)
+    L, d = 6, 4
+    K = np.tile(normal_bf16(g, (d,)), (L, 1, 1))
+    V = normal_bf16(g, (L, 1, d))
+    kc, vc, bt = _contig_cache(K, V)
+    q, do = normal_bf16(g, (2, d)), normal_bf16(g, (2, d))
+    pos = np.array([1, 5])
+    dq, dk, dv = oracle.attention_backward(q, do, np.zeros(2), np.zeros(2), pos, 1, kc, vc, bt)
+    assert np.abs(dq).max() < 1e-12
+    dow = widen(do)
+    for j in range(L):
+        want = dow[1] / 6 + (dow[0] / 2 if j <= 1 else 0.0)
+        np.testing.assert_allclose(dv[0, 0, j], want, rtol=1e-13, atol=1e-15)
+    # a single visible key: weight 1, no gradient to q or k, dv = dO
+    dq1, dk1, dv1 = oracle.attention_backward(q[:1], do[:1], [0], [0], [0], 1, kc, vc, bt)
+    assert np.all(dq1 == 0) and np.all(dk1 == 0)
+    np.testing.assert_array_equal(dv1[0, 0, 0], dow[0])
+    assert np.all(dv1[0, 0, 1:] == 0)

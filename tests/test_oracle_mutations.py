@@ -122,6 +122,18 @@ MUTATIONS = [
     ("rmsnorm_backward_dot_without_w", "dot += bf16_to_double(w[i]) * bf16_to_double(dy[r * H + i]) * xi;",
      "dot += bf16_to_double(dy[r * H + i]) * xi;",
      [pins.test_rmsnorm_backward_matches_finite_differences]),
+    ("attention_backward_ds_without_mean", "const double ds = wt[key] * (dp[key] - mean_dp);",
+     "const double ds = wt[key] * dp[key];",
+     [pins.test_attention_backward_matches_finite_differences, pins.test_attention_backward_closed_forms]),
+    ("attention_backward_dk_without_scale", "dk[off[key] + i] += scale * ds * bf16_to_double(qr[i]);",
+     "dk[off[key] + i] += ds * bf16_to_double(qr[i]);",
+     [pins.test_attention_backward_matches_finite_differences]),
+    ("attention_backward_dv_from_ds", "dv[off[key] + i] += wt[key] * bf16_to_double(gr[i]);",
+     "dv[off[key] + i] += (wt[key] - 0.5 * (dp[key] - mean_dp)) * bf16_to_double(gr[i]);",
+     [pins.test_attention_backward_matches_finite_differences, pins.test_attention_backward_closed_forms]),
+    ("attention_backward_sees_one_key_less", "const int64_t visible = (int64_t)row_pos[r] + 1;",
+     "const int64_t visible = (int64_t)row_pos[r] + (row_pos[r] > 0 ? 0 : 1);",
+     [pins.test_attention_backward_matches_finite_differences, pins.test_attention_backward_closed_forms]),
     ("matmul_residual_drops_residual", "c[m * N + n] = bf16_to_double(r[m * N + n]) + dot;",
      "c[m * N + n] = dot;",
      [pins.test_matmul_residual_small_integers_brute_force, pins.test_matmul_residual_degenerate_cases]),
