@@ -70,6 +70,8 @@ class Oracle:
         lib.oracle_matmul_residual.argtypes = [P, P, P, i64, i64, i64, P]
         lib.oracle_rope_angles.argtypes = [i32, i32, f64, P]
         lib.oracle_rmsnorm_backward.argtypes = [P, P, P, i64, i64, f64, P, P]
+        lib.oracle_swiglu_backward.argtypes = [P, P, i64, i64, P]
+        lib.oracle_rope_backward.argtypes = [P, i64, i32, i32, P, f64, P]
         lib.oracle_attention_backward.argtypes = [P, P, i64, i32, P, P, P, i32, P, P, i32, i32,
                                                   P, i32, f64, P, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -267,6 +269,24 @@ class Oracle:
         self.lib.oracle_rmsnorm_backward(_p(x), _p(w), _p(dy), M, H, float(eps), _p(dx), _p(dw))
         return dx, dw
 
+    def swiglu_backward(self, gu, dout) -> np.ndarray:
+        """[dgate | dup] [T, 2F] of swiglu for the upstream gradient dout [T, F]."""
+        gu, dout = _u16(gu), _u16(dout)
+        T, F2 = gu.shape
+        assert dout.shape == (T, F2 // 2)
+        out = np.empty((T, F2), dtype=np.float64)
+        self.lib.oracle_swiglu_backward(_p(gu), _p(dout), T, F2 // 2, _p(out))
+        return out
+
+    def rope_backward(self, dy, pos, theta: float = 10000.0) -> np.ndarray:
+        """Gradient of rope's input for the upstream gradient dy [T, nh, d]."""
+        dy = _u16(dy)
+        T, nh, d = dy.shape
+        pos = np.ascontiguousarray(pos, dtype=np.int32)
+        out = np.empty((T, nh, d), dtype=np.float64)
+        self.lib.oracle_rope_backward(_p(dy), T, nh, d, _p(pos), float(theta), _p(out))
+        return out
+
     def attention_backward(self, q_rows, dout_rows, row_seq, row_head, row_pos, Hq: int,
                            k_cache, v_cache, block_table, scale: float | None = None):
         """(dq [R, d], dk, dv [num_pages, Hkv, 16, d]) of ``attention`` for the
@@ -407,6 +427,14 @@ def fold_norm_weight(W, w) -> np.ndarray:
 
 def rmsnorm_backward(x, w, dy, eps: float):
     return default().rmsnorm_backward(x, w, dy, eps)
+
+
+def swiglu_backward(gu, dout) -> np.ndarray:
+    return default().swiglu_backward(gu, dout)
+
+
+def rope_backward(dy, pos, theta: float = 10000.0) -> np.ndarray:
+    return default().rope_backward(dy, pos, theta)
 
 
 def attention_backward(q_rows, dout_rows, row_seq, row_head, row_pos, Hq: int, k_cache,

@@ -692,3 +692,52 @@ void oracle_attention_backward(const uint16_t *q, const uint16_t *dout, int64_t 
         free(off);
     }
 }
+
+/*
+ * Backward of oracle_swiglu: with s = 1 / (1 + e^(-g)) and out = g s u,
+ *   dgate = dout u s (1 + g (1 - s)),   dup = dout g s.
+ * gu [T, 2F] = [gate | up], dout [T, F] -> dgu [T, 2F] = [dgate | dup].
+ */
+void oracle_swiglu_backward(const uint16_t *gu, const uint16_t *dout, int64_t T, int64_t F,
+                            double *dgu)
+{
+    int64_t t;
+#pragma omp parallel for schedule(static)
+    for (t = 0; t < T; ++t) {
+        for (int64_t j = 0; j < F; ++j) {
+            const double gate = bf16_to_double(gu[t * 2 * F + j]);
+            const double up = bf16_to_double(gu[t * 2 * F + F + j]);
+            const double sig = 1.0 / (1.0 + exp(-gate));
+            const double dy = bf16_to_double(dout[t * F + j]);
+            dgu[t * 2 * F + j] = dy * up * sig * (1.0 + gate * (1.0 - sig));
+            dgu[t * 2 * F + F + j] = dy * gate * sig;
+        }
+    }
+}
+
+/*
+ * Backward of oracle_rope: the rotation by the angle is orthogonal, so the
+ * gradient is the upstream gradient rotated back by the same angle:
+ *   dx_i       =  dy_i cos(a) + dy_{i+d/2} sin(a)
+ *   dx_{i+d/2} = -dy_i sin(a) + dy_{i+d/2} cos(a),   a = pos theta^(-2i/d).
+ */
+void oracle_rope_backward(const uint16_t *dy, int64_t T, int32_t nh, int32_t d,
+                          const int32_t *pos, double theta, double *dx)
+{
+    const int32_t half = d / 2;
+    int64_t t;
+#pragma omp parallel for schedule(static)
+    for (t = 0; t < T; ++t) {
+        for (int32_t h = 0; h < nh; ++h) {
+            const uint16_t *gr = dy + (t * nh + h) * (int64_t)d;
+            double *xr = dx + (t * nh + h) * (int64_t)d;
+            for (int32_t i = 0; i < half; ++i) {
+                const double ang = (double)pos[t] / pow(theta, (double)(2 * i) / (double)d);
+                const double cs = cos(ang), sn = sin(ang);
+                const double lo = bf16_to_double(gr[i]), hi = bf16_to_double(gr[i + half]);
+                xr[i] = lo * cs + hi * sn;
+                xr[i + half] = hi * cs - lo * sn;
+            }
+        }
+    }
+}

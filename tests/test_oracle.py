@@ -831,3 +831,48 @@ def test_attention_backward_closed_forms(oracle):
     assert np.all(dq1 == 0) and np.all(dk1 == 0)
     np.testing.assert_array_equal(dv1[0, 0, 0], dow[0])
     assert np.all(dv1[0, 0, 1:] == 0)
+
+
+def test_swiglu_backward_matches_finite_differences(oracle):
+    g = rng(99)
+    gu = normal_bf16(g, (3, 10), std=2.0)
+    dout = normal_bf16(g, (3, 5))
+    grad = oracle.swiglu_backward(gu, dout)
+    guw, dw = widen(gu), widen(dout)
+    np.testing.assert_allclose(oracle.swiglu(gu), guw[:, :5] / (1 + np.exp(-guw[:, :5])) * guw[:, 5:],
+                               rtol=1e-14)
+
+    def loss(v):
+        return float((dw * v[:, :5] / (1 + np.exp(-v[:, :5])) * v[:, 5:]).sum())
+
+    h = 1e-6
+    fd = np.zeros_like(guw)
+    for idx in np.ndindex(*guw.shape):
+        a, b = guw.copy(), guw.copy()
+        a[idx] += h
+        b[idx] -= h
+        fd[idx] = (loss(a) - loss(b)) / (2 * h)
+    np.testing.assert_allclose(grad, fd, rtol=1e-6, atol=1e-9)
+    # closed forms at gate 0: dgate = dout * up / 2, dup = 0
+    z = bf([[0.0, 0.0, 3.0, -1.0]])
+    np.testing.assert_array_equal(oracle.swiglu_backward(z, bf([[2.0, 1.0]])), [[3.0, -0.5, 0.0, 0.0]])
+
+
+def test_rope_backward_is_the_inverse_rotation(oracle):
+    g = rng(100)
+    dy = normal_bf16(g, (5, 2, 8))
+    pos = g.integers(0, 500, size=5).astype(np.int32)
+    dx = oracle.rope_backward(dy, pos)
+    # the forward is linear with an orthogonal matrix per (t, pair): its
+    # gradient is the transpose, so rotating dx forward gives dy back
+    t = oracle.rope_angles(500, 8)
+    c, s = t[pos, :, 0][:, None, :], t[pos, :, 1][:, None, :]
+    fwd = np.concatenate([dx[..., :4] * c - dx[..., 4:] * s, dx[..., 4:] * c + dx[..., :4] * s], -1)
+    np.testing.assert_allclose(fwd, widen(dy), rtol=1e-12, atol=1e-14)
+    # position 0: identity
+    np.testing.assert_array_equal(oracle.rope_backward(dy, np.zeros(5, np.int32)), widen(dy))
+    # the adjoint identity <rope(x), dy> = <x, rope_backward(dy)> on bf16 inputs
+    x = normal_bf16(g, (5, 2, 8))
+    lhs = float((oracle.rope(x, pos) * widen(dy)).sum())
+    rhs = float((widen(x) * dx).sum())
+    assert abs(lhs - rhs) < 1e-10 * max(1.0, abs(lhs))

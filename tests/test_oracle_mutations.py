@@ -134,6 +134,14 @@ MUTATIONS = [
     ("attention_backward_sees_one_key_less", "const int64_t visible = (int64_t)row_pos[r] + 1;",
      "const int64_t visible = (int64_t)row_pos[r] + (row_pos[r] > 0 ? 0 : 1);",
      [pins.test_attention_backward_matches_finite_differences, pins.test_attention_backward_closed_forms]),
+    ("swiglu_backward_drops_sigmoid_slope", "dy * up * sig * (1.0 + gate * (1.0 - sig));",
+     "dy * up * sig;",
+     [pins.test_swiglu_backward_matches_finite_differences]),
+    ("swiglu_backward_dup_uses_up", "dgu[t * 2 * F + F + j] = dy * gate * sig;",
+     "dgu[t * 2 * F + F + j] = dy * up * sig;",
+     [pins.test_swiglu_backward_matches_finite_differences]),
+    ("rope_backward_rotates_forward", "xr[i] = lo * cs + hi * sn;", "xr[i] = lo * cs - hi * sn;",
+     [pins.test_rope_backward_is_the_inverse_rotation]),
     ("matmul_residual_drops_residual", "c[m * N + n] = bf16_to_double(r[m * N + n]) + dot;",
      "c[m * N + n] = dot;",
      [pins.test_matmul_residual_small_integers_brute_force, pins.test_matmul_residual_degenerate_cases]),
