@@ -346,19 +346,22 @@ size_t bi_attention_decode_workspace_bytes(const bi_paged_kv *kv, int32_t B, int
  * the process exits.  The caller still passes q, o, lse and seq_lens.
  *
  * Arguments, layouts and output bits are exactly those of
- * bi_attention_decode.  With splits_per_cta == 0 the work division is picked
- * so that the scratch fits (falling back to one block per sequence, which
- * changes only the speed); a request that cannot fit -- an explicit
- * splits_per_cta whose partials exceed the array, or more sequences than
- * the array can order -- returns BI_ERR_WORKSPACE before any launch.
+ * bi_attention_decode (both entry points share one launcher).  With
+ * splits_per_cta == 0 the work division is picked so that the scratch fits
+ * (falling back to one block per sequence, which changes only the speed);
+ * an explicit splits_per_cta whose partials exceed the array returns
+ * BI_ERR_WORKSPACE before any launch.  (The launch order of the largest
+ * batch, 65535 sequences, always fits.)
  *
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any
- * stream capture.  Every call on a device shares the one array and each
- * call writes all of the scratch it later reads, so nothing has to start at
- * zero; two calls whose work overlaps on the GPU (different streams without
- * ordering) race on the array and must not be issued.  No device memory is
- * allocated or freed.
+ * stream capture.  The address is kept for the life of the process: this
+ * entry point does not support a device reset (cudaDeviceReset) between
+ * calls.  Every call on a device shares the one array and each call writes
+ * all of the scratch it later reads, so nothing has to start at zero; two
+ * calls whose work overlaps on the GPU (different streams without ordering)
+ * race on the array and must not be issued.  No device memory is allocated
+ * or freed.
  */
 #define BI_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 bi_status bi_attention_decode_noalloc(const bi_paged_kv *kv, const void *q, void *o, float *lse,
@@ -395,7 +398,6 @@ bi_status bi_attention_prefill(const bi_paged_kv *kv, const void *q, void *o, fl
 size_t bi_attention_prefill_workspace_bytes(const bi_paged_kv *kv, int32_t B, int32_t Hq,
                                             int32_t max_q_len);
 
-/* Human-readable name of a status code (static string). */
 /*
  * Decoder glue.  The reports measure invariance end to end by completing one
  * prompt greedily many times among other requests and counting the distinct
@@ -535,6 +537,7 @@ bi_status bi_moe_dispatch(const int32_t *experts, int64_t T, int32_t k, int32_t 
 bi_status bi_moe_combine(const void *y, const int64_t *pos, const float *weights, int64_t T,
                          int32_t k, int64_t H, void *out, void *stream);
 
+/* Human-readable name of a status code (static string). */
 const char *bi_status_string(bi_status s);
 
 /* 1 for the batch-invariant build, 0 for the variant-off build (split-K

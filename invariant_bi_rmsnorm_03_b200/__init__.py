@@ -6,7 +6,8 @@ torch tensors out).  Functions of the same names as the C entry points are
 re-exported from the default (batch-invariant) build; ``load(variant=True)``
 gives the variant-off build used to measure the cost of invariance.
 """
-from .binding import BIError, Library, PagedKV, Status, load, PAGE_SIZE, SPLIT_KEYS  # noqa: F401
+from .binding import (BIError, Library, PagedKV, Status, load, NOALLOC_SCRATCH_BYTES,  # noqa: F401
+                      PAGE_SIZE, SPLIT_KEYS)
 
 
 def _default():

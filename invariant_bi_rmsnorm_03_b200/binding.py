@@ -19,6 +19,7 @@ import torch
 LIBDIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib")
 PAGE_SIZE = 16
 SPLIT_KEYS = 256
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # BI_NOALLOC_SCRATCH_BYTES of include/bi.h
 
 
 class Status(enum.IntEnum):

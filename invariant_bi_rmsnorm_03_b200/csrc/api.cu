@@ -588,10 +588,10 @@ size_t bi_attention_decode_workspace_bytes(const bi_paged_kv *kv, int32_t B, int
     return order_bytes(B) + bi::attn_ws_bytes(B, Hq, kv->head_dim, max_splits, chunks);
 }
 
-bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, float *lse,
-                              const int32_t *seq_lens, int32_t B, int32_t Hq,
-                              int32_t max_seq_len, float scale, int32_t splits_per_cta,
-                              void *ws, size_t ws_bytes, void *stream)
+// Argument checks shared by both decode entry points.
+static bi_status decode_args_ok(const bi_paged_kv *kv, const void *q, const void *o,
+                                const int32_t *seq_lens, int32_t B, int32_t Hq,
+                                int32_t max_seq_len, float scale, int32_t splits_per_cta)
 {
     if (!attn_common_ok(kv, Hq)) return BI_ERR_INVALID;
     if (!head_dim_ok(kv->head_dim)) return BI_ERR_UNSUPPORTED;
@@ -601,19 +601,20 @@ bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, flo
     if (B == 0) return BI_OK;
     if (B > 65535) return BI_ERR_UNSUPPORTED;
     if (!q || !o || !seq_lens || !aligned16(q) || !aligned16(o)) return BI_ERR_INVALID;
-    DeviceState *d;
-    bi_status st = device_state(&d);
-    if (st != BI_OK) return st;
+    return BI_OK;
+}
 
+// The launches of one decode call, given its scratch: `order` (int32 [B],
+// the launch order of the sequences) and, when a sequence is split over
+// several blocks (chunks > 1), `partials` (the fp32 split records).  Both
+// decode entry points go through here, so they launch the same kernels with
+// the same parameters and give the same bits.
+static bi_status decode_launch(const DeviceState *d, const bi_paged_kv *kv, const void *q,
+                               void *o, float *lse, const int32_t *seq_lens, int32_t B,
+                               int32_t Hq, int max_splits, int splits_per_cta, int chunks,
+                               float scale, int32_t *order, float *partials, cudaStream_t s)
+{
     const int D = kv->head_dim, Hkv = kv->num_kv_heads, group = Hq / Hkv;
-    const int max_splits = (max_seq_len + bi::kSplit - 1) / bi::kSplit;
-    const int c = decode_splits_per_cta(B, Hkv, max_splits, splits_per_cta, d->num_sms);
-    const int chunks = (max_splits + c - 1) / c;
-    const size_t need = order_bytes(B) + bi::attn_ws_bytes(B, Hq, D, max_splits, chunks);
-    if (!ws || ws_bytes < need || !aligned16(ws)) return BI_ERR_WORKSPACE;
-    int32_t *order = static_cast<int32_t *>(ws);
-    float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + order_bytes(B));
-
     bi::AttnParams p{};
     p.k_cache = kv->k_cache;
     p.v_cache = kv->v_cache;
@@ -628,7 +629,7 @@ bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, flo
     p.B = B;
     p.seq_lens = seq_lens;
     p.order = order;
-    p.splits_per_cta = c;
+    p.splits_per_cta = splits_per_cta;
     p.max_splits = max_splits;
     p.scale_log2 = float(double(scale) * 1.4426950408889634);
     p.o = o;
@@ -642,13 +643,33 @@ bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, flo
     const uint64_t sq[2] = {uint64_t(D) * 2, uint64_t(Hq) * D * 2};
     const uint32_t bq[3] = {64, uint32_t(p.rows_per_q), 1};
     if (!encode(&tq, q, 3, dq, sq, bq)) return BI_ERR_CUDA;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = bi::launch_attn_order(seq_lens, B, order, s);
     if (e != cudaSuccess) return BI_ERR_CUDA;
     e = bi::launch_attention(tq, p, D, s);
     if (e != cudaSuccess) return BI_ERR_CUDA;
     if (chunks > 1) e = bi::launch_attn_combine(p, D, s);
     return from_cuda(e);
+}
+
+bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, float *lse,
+                              const int32_t *seq_lens, int32_t B, int32_t Hq,
+                              int32_t max_seq_len, float scale, int32_t splits_per_cta,
+                              void *ws, size_t ws_bytes, void *stream)
+{
+    bi_status st = decode_args_ok(kv, q, o, seq_lens, B, Hq, max_seq_len, scale, splits_per_cta);
+    if (st != BI_OK || B == 0) return st;
+    DeviceState *d;
+    if ((st = device_state(&d)) != BI_OK) return st;
+
+    const int max_splits = (max_seq_len + bi::kSplit - 1) / bi::kSplit;
+    const int c = decode_splits_per_cta(B, kv->num_kv_heads, max_splits, splits_per_cta, d->num_sms);
+    const int chunks = (max_splits + c - 1) / c;
+    const size_t need = order_bytes(B) + bi::attn_ws_bytes(B, Hq, kv->head_dim, max_splits, chunks);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return BI_ERR_WORKSPACE;
+    int32_t *order = static_cast<int32_t *>(ws);
+    float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + order_bytes(B));
+    return decode_launch(d, kv, q, o, lse, seq_lens, B, Hq, max_splits, c, chunks, scale, order,
+                         partials, static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------- no-alloc decode
@@ -658,6 +679,10 @@ bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, flo
 // sequences and the split partials) is this fixed array, which every GPU
 // that loads the library holds until the process exits.
 static __device__ __align__(256) uint8_t g_decode_scratch[BI_NOALLOC_SCRATCH_BYTES];
+
+// The launch order of the largest batch always fits beside some partials.
+static_assert(((65535 * 4 + 255) / 256) * 256 < BI_NOALLOC_SCRATCH_BYTES,
+              "the launch order of 65535 sequences fits in the scratch array");
 
 static std::mutex g_scratch_mu;
 static void *g_scratch_addr[kMaxDevices];
@@ -685,26 +710,17 @@ bi_status bi_attention_decode_noalloc(const bi_paged_kv *kv, const void *q, void
                                       int32_t max_seq_len, float scale, int32_t splits_per_cta,
                                       void *stream)
 {
-    if (!attn_common_ok(kv, Hq)) return BI_ERR_INVALID;
-    if (!head_dim_ok(kv->head_dim)) return BI_ERR_UNSUPPORTED;
-    if (B < 0 || max_seq_len < 1 || splits_per_cta < 0 || !std::isfinite(scale))
-        return BI_ERR_INVALID;
-    if (int64_t(max_seq_len) > int64_t(kv->max_pages_per_seq) * BI_PAGE_SIZE) return BI_ERR_INVALID;
-    if (B == 0) return BI_OK;
-    if (B > 65535) return BI_ERR_UNSUPPORTED;
-    if (!q || !o || !seq_lens || !aligned16(q) || !aligned16(o)) return BI_ERR_INVALID;
+    bi_status st = decode_args_ok(kv, q, o, seq_lens, B, Hq, max_seq_len, scale, splits_per_cta);
+    if (st != BI_OK || B == 0) return st;
     DeviceState *d;
-    bi_status st = device_state(&d);
-    if (st != BI_OK) return st;
+    if ((st = device_state(&d)) != BI_OK) return st;
     void *scratch = nullptr;
-    st = decode_scratch(&scratch);
-    if (st != BI_OK) return st;
+    if ((st = decode_scratch(&scratch)) != BI_OK) return st;
 
-    const int D = kv->head_dim, Hkv = kv->num_kv_heads, group = Hq / Hkv;
     const int max_splits = (max_seq_len + bi::kSplit - 1) / bi::kSplit;
-    int c = decode_splits_per_cta(B, Hkv, max_splits, splits_per_cta, d->num_sms);
+    int c = decode_splits_per_cta(B, kv->num_kv_heads, max_splits, splits_per_cta, d->num_sms);
     int chunks = (max_splits + c - 1) / c;
-    size_t need = order_bytes(B) + bi::attn_ws_bytes(B, Hq, D, max_splits, chunks);
+    size_t need = order_bytes(B) + bi::attn_ws_bytes(B, Hq, kv->head_dim, max_splits, chunks);
     if (need > BI_NOALLOC_SCRATCH_BYTES && splits_per_cta == 0) {
         // The work division chosen from the load would need more partials
         // than the array holds: give each sequence one block instead (the
@@ -716,42 +732,8 @@ bi_status bi_attention_decode_noalloc(const bi_paged_kv *kv, const void *q, void
     if (need > BI_NOALLOC_SCRATCH_BYTES) return BI_ERR_WORKSPACE;
     int32_t *order = static_cast<int32_t *>(scratch);
     float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(scratch) + order_bytes(B));
-
-    bi::AttnParams p{};
-    p.k_cache = kv->k_cache;
-    p.v_cache = kv->v_cache;
-    p.block_table = kv->block_table;
-    p.max_pages = kv->max_pages_per_seq;
-    p.num_pages = kv->num_pages;
-    p.Hkv = Hkv;
-    p.Hq = Hq;
-    p.group = group;
-    p.rows_per_q = (group + 3) / 4;
-    p.decode = 1;
-    p.B = B;
-    p.seq_lens = seq_lens;
-    p.order = order;
-    p.splits_per_cta = c;
-    p.max_splits = max_splits;
-    p.scale_log2 = float(double(scale) * 1.4426950408889634);
-    p.o = o;
-    p.lse = lse;
-    p.ws = partials;
-    p.status = d->status;
-    p.timeout_ns = bi::kDefaultTimeoutNs;
-
-    CUtensorMap tq;
-    const uint64_t dq[3] = {uint64_t(D), uint64_t(Hq), uint64_t(B)};
-    const uint64_t sq[2] = {uint64_t(D) * 2, uint64_t(Hq) * D * 2};
-    const uint32_t bq[3] = {64, uint32_t(p.rows_per_q), 1};
-    if (!encode(&tq, q, 3, dq, sq, bq)) return BI_ERR_CUDA;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = bi::launch_attn_order(seq_lens, B, order, s);
-    if (e != cudaSuccess) return BI_ERR_CUDA;
-    e = bi::launch_attention(tq, p, D, s);
-    if (e != cudaSuccess) return BI_ERR_CUDA;
-    if (chunks > 1) e = bi::launch_attn_combine(p, D, s);
-    return from_cuda(e);
+    return decode_launch(d, kv, q, o, lse, seq_lens, B, Hq, max_splits, c, chunks, scale, order,
+                         partials, static_cast<cudaStream_t>(stream));
 }
 
 size_t bi_attention_prefill_workspace_bytes(const bi_paged_kv *kv, int32_t B, int32_t Hq,

@@ -38,6 +38,15 @@ def test_library_exports_every_declared_symbol(lib):
         assert ctypes.cast(getattr(lib.lib, s), ctypes.c_void_p).value
 
 
+def test_header_constants_match_the_binding():
+    text = open(HEADER).read()
+    m = re.search(r"#define BI_NOALLOC_SCRATCH_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", text)
+    assert m, "BI_NOALLOC_SCRATCH_BYTES not found"
+    assert int(m.group(1)) * int(m.group(2)) * int(m.group(3)) == bi.NOALLOC_SCRATCH_BYTES
+    assert re.search(r"#define BI_PAGE_SIZE %d\b" % bi.PAGE_SIZE, text)
+    assert re.search(r"#define BI_SPLIT_KEYS %d\b" % bi.SPLIT_KEYS, text)
+
+
 def test_build_flavour(lib):
     want = 0 if lib.path.endswith("libbi_variant.so") else 1
     assert lib.bi_build_invariant() == want

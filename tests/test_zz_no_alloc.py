@@ -8,9 +8,10 @@ library instead of a caller workspace.
 The test calls the entry point through the C ABI twice in a row and checks
 both outputs against bi_attention_decode's on the same inputs: within the
 parity tolerance the other tests use, and (since the work division never
-changes the bits) byte for byte.  This file is collected last so that a run
-that stops at the first failure has run every other test before it; it
-passes alone in a fresh process as well."""
+changes the bits) byte for byte; the outputs are also checked against the
+fp64 oracle.  This file is collected last so that a run that stops at the
+first failure has run every other test before it; it passes alone in a
+fresh process as well."""
 import ctypes
 
 import numpy as np
@@ -18,7 +19,9 @@ import pytest
 import torch
 
 import invariant_bi_rmsnorm_03_b200 as bi
-from gpu_util import DEV, TOL_BF16, TOL_F32, dev_bf16, rowwise_normwise, same_bytes, to_f64
+import oracle
+from gpu_util import (DEV, TOL_BF16, TOL_F32, dev_bf16, host_bits as bits_of, rowwise_normwise,
+                      same_bytes, to_f64)
 from synth import kv_to_blocks, normal_bf16, paged_kv, rng, tiny_layer
 
 pytestmark = pytest.mark.gpu
@@ -27,6 +30,17 @@ pytestmark = pytest.mark.gpu
 def _dev_kv(kv):
     return bi.PagedKV(dev_bf16(kv_to_blocks(kv.k_cache)), dev_bf16(kv_to_blocks(kv.v_cache)),
                       torch.from_numpy(np.ascontiguousarray(kv.block_table)).to(DEV))
+
+
+def _oracle_check(kv, q, o, lse):
+    """The outputs against the fp64 oracle, per request (o) and per row (lse)."""
+    B, Hq, d = q.shape
+    rows = oracle.decode_rows(q, kv.seq_lens)
+    ro, rl = oracle.attention(*rows, Hq, kv.k_cache, kv.v_cache, kv.block_table, want_lse=True)
+    err = rowwise_normwise(to_f64(o).reshape(B, Hq * d), ro.reshape(B, Hq * d))
+    assert err.max() <= TOL_BF16, "request %d: %.3g" % (err.argmax(), err.max())
+    lerr = rowwise_normwise(to_f64(lse).reshape(B, Hq), rl.reshape(B, Hq))
+    assert lerr.max() <= TOL_F32, "lse of request %d: %.3g" % (lerr.argmax(), lerr.max())
 
 
 def _cases():
@@ -66,6 +80,8 @@ def test_noalloc_matches_workspace_entry_point_twice(name, kv, q):
         assert lerr.max() <= TOL_F32, (call, lerr.max())
         assert same_bytes(o, ref_o), call
         assert same_bytes(lse, ref_l), call
+        if call == 0:
+            _oracle_check(kv, q, o, lse)
     assert L.bi_device_status() == bi.Status.OK
 
 
@@ -84,7 +100,16 @@ def test_noalloc_rejects_what_the_array_cannot_hold():
     with pytest.raises(bi.BIError) as e:
         L.bi_attention_decode_noalloc(dkv, q, sl, 65536, splits_per_cta=1)
     assert e.value.status == bi.Status.WORKSPACE
-    # with the division left to the library it fits, and matches the
-    # workspace entry point
-    o = L.bi_attention_decode_noalloc(dkv, q, sl, 65536)
-    assert same_bytes(o, L.bi_attention_decode(dkv, q, sl, 65536))
+    # With the division left to the library the division it would pick from
+    # the load needs more scratch than the array holds (the workspace query
+    # of the other entry point says how much), so the call falls back to one
+    # block per sequence -- and still matches the workspace entry point and
+    # the oracle.
+    need = L.bi_attention_decode_workspace_bytes(dkv, 4, 64, 65536)
+    assert need > bi.NOALLOC_SCRATCH_BYTES, need
+    o, lse = L.bi_attention_decode_noalloc(dkv, q, sl, 65536, want_lse=True)
+    ref_o, ref_l = L.bi_attention_decode(dkv, q, sl, 65536, want_lse=True)
+    assert same_bytes(o, ref_o)
+    assert same_bytes(lse, ref_l)
+    _oracle_check(kv, bits_of(q), o, lse)
+    assert L.bi_device_status() == bi.Status.OK
