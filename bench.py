@@ -382,6 +382,95 @@ def rmsnorm_context(torch, L, wl) -> dict:
             "rmsnorm_M65536_ms": big_ms, "rmsnorm_M65536_GB/s": big_bytes / (big_ms * 1e-3) / 1e9}
 
 
+def _median_ms(torch, fn, flush, reps=15, warm=3):
+    """Median CUDA-event time of fn() on the current stream, L2 flushed
+    (a 512 MB write) before every launch."""
+    T = torch
+    for _ in range(warm):
+        flush.zero_()
+        fn()
+    ev = [(T.cuda.Event(enable_timing=True), T.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        fn()
+        b.record()
+    T.cuda.synchronize()
+    return float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+
+def cost_of_invariance(torch, L, Lv, wl) -> dict:
+    """Each kernel of the step at several sizes in both builds (the
+    invariant build and the variant-off build, whose matmul splits K when the
+    tiles cannot fill the GPU and whose decode blocks pre-merge their own
+    range), the cuBLAS product (torch.matmul) at the same shapes as context,
+    and the weight bandwidth of the small-M products.  Medians of CUDA-event
+    times, L2 flushed before each launch."""
+    T = torch
+    dev = wl.x.device
+    pk, _ = peaks()
+    out = {"matmul": [], "rmsnorm": [], "attention_decode": [], "attention_prefill": []}
+    # matmul: M rows of the step's normalised x times W [N, 4096]
+    Ws = {N_COLS: wl.W}
+    for N in (4096, 28672):
+        Ws[N] = T.randn((N, H), device=dev, dtype=T.float32).mul_(0.02).to(T.bfloat16)
+    for M in (64, 256, 2048):
+        for N in (4096, N_COLS, 28672):
+            if M == 2048 and N != N_COLS:
+                continue
+            a, W = wl.y[:M], Ws[N]
+            c = T.empty((M, N), dtype=T.bfloat16, device=dev)
+            need = max(Lv.bi_matmul_workspace_bytes(M, N, H), 16)
+            ws = T.empty(need, dtype=T.uint8, device=dev)
+            ms_i = _median_ms(T, lambda: L.bi_matmul(a, W, out=c), wl.flush)
+            ms_v = _median_ms(T, lambda: Lv.bi_matmul(a, W, out=c, ws=ws), wl.flush)
+            ms_cb = _median_ms(T, lambda: T.matmul(a, W.t()), wl.flush)
+            flops = 2.0 * M * N * H
+            wbytes = 2.0 * N * H
+            out["matmul"].append({
+                "M": M, "N": N, "K": H, "invariant_ms": ms_i, "variant_off_ms": ms_v,
+                "overhead": ms_i / ms_v - 1.0, "k_splits_variant_off":
+                    (need // (4 * M * N)) if need > 16 else 1,
+                "cublas_ms": ms_cb, "vs_cublas": ms_i / ms_cb - 1.0,
+                "TFLOP/s": flops / (ms_i * 1e-3) / 1e12,
+                "frac_bf16": flops / (ms_i * 1e-3) / 1e12 / pk["bf16_tflops"],
+                "weight_GB/s": wbytes / (ms_i * 1e-3) / 1e9,
+                "weight_frac_hbm": wbytes / (ms_i * 1e-3) / 1e9 / pk["hbm_gbs"]})
+    del Ws
+    for M in (64, 256, 2048):
+        x = wl.x[:M]
+        y = T.empty_like(x)
+        ms_i = _median_ms(T, lambda: L.bi_rmsnorm(x, wl.w, wl.eps, out=y), wl.flush)
+        ms_v = _median_ms(T, lambda: Lv.bi_rmsnorm(x, wl.w, wl.eps, out=y), wl.flush)
+        out["rmsnorm"].append({"M": M, "H": H, "invariant_ms": ms_i, "variant_off_ms": ms_v,
+                               "overhead": ms_i / ms_v - 1.0})
+    # decode: the first B requests of the step's batch
+    for B in (1, 16, DEC_B):
+        kv = type(wl.dec_kv)(wl.dec_kv.k_cache, wl.dec_kv.v_cache,
+                             wl.dec_kv.block_table[:B].contiguous())
+        q, sl = wl.dec_q[:B].contiguous(), wl.dec_lens[:B].contiguous()
+        o = T.empty_like(q)
+        mx = int(wl.dec_lens_np[:B].max())
+        need = max(L.bi_attention_decode_workspace_bytes(kv, B, DEC_HQ, mx),
+                   Lv.bi_attention_decode_workspace_bytes(kv, B, DEC_HQ, mx), 16)
+        ws = T.empty(need, dtype=T.uint8, device=dev)
+        ms_i = _median_ms(T, lambda: L.bi_attention_decode(kv, q, sl, mx, out=o, ws=ws), wl.flush)
+        ms_v = _median_ms(T, lambda: Lv.bi_attention_decode(kv, q, sl, mx, out=o, ws=ws), wl.flush)
+        nbytes = float(wl.dec_lens_np[:B].astype(np.int64).sum()) * DEC_HKV * D * 4
+        out["attention_decode"].append({
+            "B": B, "kv_tokens": int(wl.dec_lens_np[:B].sum()), "invariant_ms": ms_i,
+            "variant_off_ms": ms_v, "overhead": ms_i / ms_v - 1.0,
+            "GB/s": nbytes / (ms_i * 1e-3) / 1e9})
+    ms_i = _median_ms(T, lambda: L.bi_attention_prefill(wl.pre_kv, wl.pre_q, wl.pre_cu, wl.pre_ctx,
+                                                         PRE_S, out=wl.pre_o), wl.flush, reps=7)
+    ms_v = _median_ms(T, lambda: Lv.bi_attention_prefill(wl.pre_kv, wl.pre_q, wl.pre_cu, wl.pre_ctx,
+                                                          PRE_S, out=wl.pre_o), wl.flush, reps=7)
+    out["attention_prefill"].append({"S": PRE_S, "invariant_ms": ms_i, "variant_off_ms": ms_v,
+                                     "overhead": ms_i / ms_v - 1.0,
+                                     "note": "one prefill kernel in both builds"})
+    return out
+
+
 def cpu_baseline(wl, budget_s: float = 20.0) -> dict:
     """The oracle (fp64, OpenMP) on a bounded sample of the same workload."""
     import oracle
@@ -505,6 +594,8 @@ def run_ours(args):
     e2e_per, h2d, d2h = e2e_steps(torch, L, wl, max(2, args.steps // 2), 1)
     e2e_gemm_ms = maxall(float(e2e_per[:, 0].mean()))
     e2e_dec_ms = maxall(float(e2e_per[:, 1].mean()))
+    e2e_step_ms = maxall(float(e2e_per.sum(axis=1).mean()))
+    e2e_pre_ms = maxall(float(e2e_per[:, 2].mean()))
 
     # variant-off build on the same step (the cost of invariance)
     Lv = bi.load(variant=True)
@@ -517,12 +608,15 @@ def run_ours(args):
     overhead = {n: float(mean[i] / mean_v[i] - 1.0) for i, n in enumerate(names)}
     overhead["step"] = float(per.sum(axis=1).mean() / per_v.sum(axis=1).mean() - 1.0)
 
+    coi = cost_of_invariance(torch, L, Lv, wl) if rank == 0 else None
     checks = invariance_checks(torch, L, wl)
     rms_ctx = rmsnorm_context(torch, L, wl)
     uc = None
     if rank == 0 and args.uc_targets > 0:
-        # the end-to-end check on the toy decoder, at a reduced count
-        uc = unique_completions(args.uc_targets, args.uc_targets, span=2 * args.uc_targets)
+        # the end-to-end check on the toy decoder: one prompt completed by
+        # --uc-targets copies amid as many other requests, in both builds
+        uc = unique_completions(args.uc_targets, args.uc_targets,
+                                span=min(2000, 2 * args.uc_targets))
         checks["unique_completions"] = uc["invariant"]["unique_completions"]
         checks["all"] = bool(checks["all"] and checks["unique_completions"] == 1)
 
@@ -600,10 +694,16 @@ def run_ours(args):
         "roofline": roof,
         "kernels": kernels,
         "overhead_vs_variant_off": overhead,
+        "cost_of_invariance": coi,
         "unique_completions": uc,
         "e2e": {"value": world * wl.gemm_flops / (e2e_gemm_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "split_kv_attn_gbs": world * wl.dec_bytes / (e2e_dec_ms * 1e-3) / 1e9},
+                "split_kv_attn_gbs": world * wl.dec_bytes / (e2e_dec_ms * 1e-3) / 1e9,
+                "step_ms": e2e_step_ms,
+                "legs_ms": {"rmsnorm_matmul": e2e_gemm_ms, "kv_write_decode": e2e_dec_ms,
+                            "kv_write_prefill": e2e_pre_ms},
+                "note": "step_ms: the whole step (all three legs) through the public calls, "
+                        "inputs copied in from pinned host memory and results copied out"},
         "gpu_launches": launches * args.steps,
         "clocks": clk,
         "cpu_baseline": cpu,
@@ -701,12 +801,13 @@ def run_profile_case(args):
     elif args.profile in ("rmsnorm_matmul", "rmsnorm_then_matmul", "matmul_residual",
                           "matmul_rows"):
         # fused forms against their unfused launches, M = --profile-rows rows
-        # of hidden 4096 times N = 12288; two weight copies rotate (201 MB > L2)
-        M = args.profile_rows
-        nm = norm_matmul(seed=1, M=M, H=H, N=N_COLS)
+        # of hidden 4096 times N = --profile-cols (12288); two weight copies
+        # rotate (201 MB > L2 at N = 12288)
+        M, NC = args.profile_rows, args.profile_cols
+        nm = norm_matmul(seed=1, M=M, H=H, N=NC)
         x, w = d16(nm["x"]), d16(nm["w"])
-        Ws = [d16(nm["W"]), d16(norm_matmul(seed=11, M=1, H=H, N=N_COLS)["W"])]
-        c = T.empty((M, N_COLS), dtype=T.bfloat16, device=dev)
+        Ws = [d16(nm["W"]), d16(norm_matmul(seed=11, M=1, H=H, N=NC)["W"])]
+        c = T.empty((M, NC), dtype=T.bfloat16, device=dev)
         if args.profile == "rmsnorm_matmul":
             wfs = [L.bi_fold_norm_weight(W, w) for W in Ws]
             fn = lambda i: L.bi_rmsnorm_matmul(x, wfs[i % 2], 1e-6, out=c)  # noqa: E731
@@ -715,7 +816,7 @@ def run_profile_case(args):
             fn = lambda i: L.bi_matmul(L.bi_rmsnorm(x, w, 1e-6, out=y), Ws[i % 2],  # noqa: E731
                                        out=c)
         elif args.profile == "matmul_residual":
-            r = d16(normal_bf16(rng(12), (M, N_COLS)))
+            r = d16(normal_bf16(rng(12), (M, NC)))
             fn = lambda i: L.bi_matmul_residual(x, Ws[i % 2], r, out=c)  # noqa: E731
         else:
             fn = lambda i: L.bi_matmul(x, Ws[i % 2], out=c)  # noqa: E731
@@ -759,6 +860,39 @@ def run_profile_case(args):
         else:
             dc = d16(normal_bf16(g, (M, N_COLS)))
             fn = lambda i: L.bi_matmul_backward(dc, x, W)  # noqa: E731
+    elif args.profile in ("attention_backward", "swiglu_backward", "rope_backward"):
+        # the toy decoder's shapes: 32 query / 8 kv heads of 128 over one
+        # causal prompt of --profile-seq tokens; SwiGLU 14336 and RoPE of the
+        # q heads over the same tokens
+        g = rng(15)
+        S = args.profile_seq
+        if args.profile == "attention_backward":
+            Hq, Hkv = 32, 8
+            q = d16(normal_bf16(g, (S, Hq, D)))
+            k = d16(normal_bf16(g, (S, Hkv, D)))
+            v = d16(normal_bf16(g, (S, Hkv, D)))
+            dout = d16(normal_bf16(g, (S, Hq, D)))
+            pbt, pnp = page_table(g, [S])
+            kv = bi.PagedKV(T.zeros((pnp, Hkv, 16, D), dtype=T.bfloat16, device=dev),
+                            T.zeros((pnp, Hkv, 16, D), dtype=T.bfloat16, device=dev),
+                            T.from_numpy(pbt).to(dev))
+            L.bi_kv_write(kv, k, v, T.from_numpy(slot_mapping(pbt, 0, np.arange(S))).to(dev))
+            cu = T.tensor([0, S], dtype=T.int32, device=dev)
+            ctx = T.tensor([0], dtype=T.int32, device=dev)
+            o, lse = L.bi_attention_prefill(kv, q, cu, ctx, S, want_lse=True)
+            dk, dv = T.zeros_like(kv.k_cache), T.zeros_like(kv.v_cache)
+            fn = lambda i: L.bi_attention_backward(kv, q, o, dout, lse, cu, ctx, S, S,  # noqa: E731
+                                                   dk=dk, dv=dv)
+        elif args.profile == "swiglu_backward":
+            gu = d16(normal_bf16(g, (S, 2 * 14336)))
+            dout = d16(normal_bf16(g, (S, 14336)))
+            out = T.empty_like(gu)
+            fn = lambda i: L.bi_swiglu_backward(gu, dout, out=out)  # noqa: E731
+        else:
+            dy = d16(normal_bf16(g, (S, 32, D)))
+            pos = T.from_numpy(np.arange(S, dtype=np.int32)).to(dev)
+            out = T.empty_like(dy)
+            fn = lambda i: L.bi_rope_backward(dy, pos, out=out)  # noqa: E731
     elif args.profile == "sample":
         # 256 rows of lm_head logits (vocab 32000), temperature 0.8, nucleus 0.95
         g = rng(5)
@@ -906,12 +1040,16 @@ def main(argv=None):
     ap.add_argument("--profile", choices=["rmsnorm", "matmul", "decode", "prefill", "copy",
                                           "sample", "rmsnorm_matmul", "rmsnorm_then_matmul",
                                           "matmul_residual", "matmul_rows", "qkv_fused",
-                                          "qkv_unfused", "rmsnorm_backward", "matmul_backward"],
+                                          "qkv_unfused", "rmsnorm_backward", "matmul_backward",
+                                          "attention_backward", "swiglu_backward",
+                                          "rope_backward"],
                     help="run one kernel alone on a reduced case (for ncu)")
     ap.add_argument("--profile-batch", type=int, default=32)
     ap.add_argument("--profile-seq", type=int, default=4096)
     ap.add_argument("--profile-rows", type=int, default=M_ROWS,
                     help="rows of the fused-matmul --profile cases")
+    ap.add_argument("--profile-cols", type=int, default=N_COLS,
+                    help="output columns of the fused-matmul --profile cases")
     ap.add_argument("--variant", action="store_true", help="--profile the variant-off build")
     ap.add_argument("--unique-completions", action="store_true",
                     help="run the toy-decoder unique-completion experiment instead")
@@ -927,7 +1065,7 @@ def main(argv=None):
                     help="unique-completion run on the mixture-of-experts decoder")
     ap.add_argument("--fused", action="store_true",
                     help="unique-completion run with the fused matmul forms")
-    ap.add_argument("--uc-targets", type=int, default=200,
+    ap.add_argument("--uc-targets", type=int, default=1000,
                     help="target copies (and as many others) of the in-bench unique-completion "
                          "check; 0 skips it")
     args = ap.parse_args(argv)

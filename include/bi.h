@@ -181,16 +181,19 @@ bi_status bi_matmul_grouped(const void *a, const void *w, void *c, const int64_t
  *   product.
  *
  * bi_rmsnorm_matmul -- RMSNorm of each row of x followed by the product with
- *   a folded weight, in one launch:
+ *   a folded weight:
  *
  *     r[m]    = rsqrt( (1/K) * sum_k x[m, k]^2 + eps )          (fp32)
  *     C[m, n] = round( r[m] * sum_k x[m, k] * wf[n, k] )
  *
  *   x : device, bf16 [M, K];  wf : device, bf16 [N, K];  c : device, [M, N]
- *   of out_dtype.  The sum of squares is taken from the A tiles already in
- *   shared memory (K ascending, eight fixed partial sums), so x is read
- *   once; the normalised row is never rounded to bf16.  Requirements as
- *   bi_matmul, and eps finite and >= 0.
+ *   of out_dtype.  r is computed first by bi_rmsnorm's own reduction (the
+ *   same order, so r[m] has the bits of bi_rmsnorm's rstd of that row) into
+ *   the workspace -- M floats instead of the normalised [M, K] rows -- and
+ *   the matmul's epilogue scales each row by it; the normalised row is never
+ *   rounded to bf16.  ws : device workspace of
+ *   bi_rmsnorm_matmul_workspace_bytes(M) bytes, 16-byte aligned.
+ *   Requirements as bi_matmul, K <= 65536, and eps finite and >= 0.
  *
  * bi_matmul_residual -- the product added to a residual stream:
  *
@@ -228,6 +231,29 @@ bi_status bi_matmul_grouped(const void *a, const void *w, void *c, const int64_t
  *   out_dtype, either may be NULL.  ws : bi_matmul_backward_workspace_bytes
  *   (M, N, K) bytes.  Requirements as bi_matmul.  A row of dA depends on
  *   that row of dC only.
+ *
+ * bi_swiglu_backward -- gradients of out = silu(g) * u (bi_swiglu) for an
+ *   upstream gradient dout, with s = 1 / (1 + e^-g):
+ *     dgate = dout * u * (s + g s (1 - s)),   dup = dout * g * s
+ *   (1 - s evaluated as 1 / (1 + e^g)); fp32, every operation rounded.
+ *   gu : device, bf16 [T, 2F] (gate columns, then up);  dout : device, bf16
+ *   [T, F];  dgu : device, [T, 2F] of out_dtype (dgate, then dup: the layout
+ *   of gu, ready for the stacked gate/up matmul's backward).  F % 8 == 0,
+ *   16-byte aligned pointers, dgu overlapping neither input.  Each element
+ *   depends on its own inputs only.
+ *
+ * bi_rope_backward -- gradient of bi_rope_kv_write's rotation: the rotation
+ *   by the negative angle,
+ *     dx_i       = dy_i cos(a) + dy_{i+d/2} sin(a)
+ *     dx_{i+d/2} = dy_{i+d/2} cos(a) - dy_i sin(a),   a = pos * theta^(-2i/d)
+ *   with cos and sin evaluated in double precision and rounded to float as
+ *   the forward evaluates them; fp32, every product and sum rounded.
+ *   dy : device, bf16, T rows of num_heads heads of head_dim values, rows
+ *   ld_dy values apart;  dx : device, of out_dtype, same shape, rows ld_dx
+ *   values apart (so a head set inside a wider row, e.g. the q or k part of
+ *   a fused q/k/v gradient, can be read and written in place of a copy);
+ *   positions : device, int32 [T].  head_dim in {64, 128}, ld % 8 == 0,
+ *   ld >= num_heads * head_dim, theta > 1, 16-byte aligned dy and dx.
  */
 size_t bi_rmsnorm_backward_workspace_bytes(int64_t M, int64_t H);
 bi_status bi_rmsnorm_backward(const void *x, const void *w, const void *dy, void *dx, void *dw,
@@ -235,6 +261,11 @@ bi_status bi_rmsnorm_backward(const void *x, const void *w, const void *dy, void
                               size_t ws_bytes, void *stream);
 bi_status bi_transpose(const void *a, void *out, int64_t R, int64_t C, int64_t ld_out,
                        void *stream);
+bi_status bi_swiglu_backward(const void *gu, const void *dout, void *dgu, int64_t T, int64_t F,
+                             bi_dtype out_dtype, void *stream);
+bi_status bi_rope_backward(const void *dy, int64_t ld_dy, const int32_t *positions, void *dx,
+                           int64_t ld_dx, int64_t T, int32_t num_heads, int32_t head_dim,
+                           float theta, bi_dtype out_dtype, void *stream);
 size_t bi_matmul_backward_workspace_bytes(int64_t M, int64_t N, int64_t K);
 bi_status bi_matmul_backward(const void *dc, const void *a, const void *w, void *da, void *dw,
                              int64_t M, int64_t N, int64_t K, bi_dtype out_dtype, void *ws,
@@ -247,9 +278,10 @@ bi_status bi_matmul_backward(const void *dc, const void *a, const void *w, void 
  * bi_rope_kv_write evaluates them (the same floats).  table : device, fp32
  * [max_pos, d/2, 2], 16-byte aligned.  d = head_dim in {64, 128}; theta > 1.
  *
- * bi_rmsnorm_matmul_rope_kv -- the attention input of a transformer block in
- * one launch: RMSNorm of x folded into the QKV matmul (as bi_rmsnorm_matmul,
- * wf the folded [N, K] weight, N = (Hq + 2 Hkv) d), then RoPE of the q and k
+ * bi_rmsnorm_matmul_rope_kv -- the attention input of a transformer block:
+ * RMSNorm of x folded into the QKV matmul (as bi_rmsnorm_matmul, wf the
+ * folded [N, K] weight, N = (Hq + 2 Hkv) d, its row statistics in ws, of
+ * bi_rmsnorm_matmul_workspace_bytes(T) bytes), then RoPE of the q and k
  * heads and the cache write of k and v, in the matmul's epilogue.  The
  * result is bi_rmsnorm_matmul followed by bi_rope_kv_write bit for bit (the
  * product is rounded to bf16 first, the rotation uses the table's angles
@@ -269,11 +301,14 @@ bi_status bi_rmsnorm_matmul_rope_kv(const void *x, const void *wf, float eps,
                                     const bi_paged_kv *kv, const float *rope_table,
                                     int32_t max_pos, const int32_t *positions,
                                     const int64_t *slot_mapping, void *q_out, int64_t T,
-                                    int64_t K, int32_t Hq, void *stream);
+                                    int64_t K, int32_t Hq, void *ws, size_t ws_bytes,
+                                    void *stream);
 bi_status bi_fold_norm_weight(const void *W, const void *w, void *wf, int64_t N, int64_t K,
                               void *stream);
+size_t bi_rmsnorm_matmul_workspace_bytes(int64_t M);
 bi_status bi_rmsnorm_matmul(const void *x, const void *wf, void *c, int64_t M, int64_t N,
-                            int64_t K, float eps, bi_dtype out_dtype, void *stream);
+                            int64_t K, float eps, bi_dtype out_dtype, void *ws, size_t ws_bytes,
+                            void *stream);
 bi_status bi_matmul_residual(const void *a, const void *w, const void *r, void *c, int64_t M,
                              int64_t N, int64_t K, void *stream);
 
@@ -397,6 +432,47 @@ bi_status bi_attention_prefill(const bi_paged_kv *kv, const void *q, void *o, fl
                                void *ws, size_t ws_bytes, void *stream);
 size_t bi_attention_prefill_workspace_bytes(const bi_paged_kv *kv, int32_t B, int32_t Hq,
                                             int32_t max_q_len);
+
+/*
+ * bi_attention_backward -- gradients of bi_attention_prefill (and of decode,
+ * which is prefill with one row per sequence) for an upstream gradient dO,
+ * for the trainer side of on-policy RL (xitu-tech news, "强化学习的突破").
+ * With P_ij = exp(scale q_i.k_j - lse_i) over the visible keys j <= t_i,
+ * dP_ij = dO_i.v_j, Delta_i = dO_i.o_i and dS_ij = P_ij (dP_ij - Delta_i):
+ *   dq_i = scale sum_j dS_ij k_j
+ *   dk_j = scale sum_i dS_ij q_i,   dv_j = sum_i P_ij dO_i
+ * the sums for dk_j, dv_j over every row of the call's chunk of key j's
+ * sequence that sees it, in all query heads of its kv group.
+ *
+ *   kv, q, cu_q, ctx_lens, B, Hq, T_total, max_q_len, scale : as the
+ *     bi_attention_prefill call whose gradient is taken;
+ *   o    : device, bf16 [T_total, Hq, d], that call's output;
+ *   lse  : device, fp32 [T_total, Hq], that call's lse (natural log);
+ *   dout : device, bf16 [T_total, Hq, d], the upstream gradient;
+ *   max_kv_len : host int >= every ctx_lens[b] + chunk length;
+ *   dq   : device, bf16 [T_total, Hq, d];
+ *   dk_cache, dv_cache : device, bf16, shaped and laid out like the caches
+ *     (page blocks in core-matrix order).  For each sequence, every slot of
+ *     its pages up to its last key is written (slots past its length in the
+ *     last page get 0); other pages are not touched.  No page may belong to
+ *     two sequences of the call; dk_cache and dv_cache overlap neither cache
+ *     nor each other.
+ *   ws, ws_bytes : device workspace of bi_attention_backward_workspace_bytes
+ *     (Hq, T_total) bytes (Delta and lse log2 e per row), 16-byte aligned.
+ * Fixed orders: dk_j and dv_j sum the query heads of the group ascending,
+ * then the 128-row query tiles of the chunk ascending, each tile's rows
+ * reduced on the tensor core; dq_i sums the 128-key blocks from key 0
+ * ascending -- a row's dq depends on that row only.  P and dS enter the
+ * tensor core as bf16 (as the forward's P does); the rest is fp32.
+ * Requirements: as bi_attention_prefill; d in {64, 128}.
+ */
+size_t bi_attention_backward_workspace_bytes(int32_t Hq, int64_t T_total);
+bi_status bi_attention_backward(const bi_paged_kv *kv, const void *q, const void *o,
+                                const void *dout, const float *lse, const int32_t *cu_q,
+                                const int32_t *ctx_lens, int32_t B, int32_t Hq, int64_t T_total,
+                                int32_t max_q_len, int32_t max_kv_len, float scale, void *dq,
+                                void *dk_cache, void *dv_cache, void *ws, size_t ws_bytes,
+                                void *stream);
 
 /*
  * Decoder glue.  The reports measure invariance end to end by completing one

@@ -115,7 +115,9 @@ class Library:
                "bi_rmsnorm_matmul", "bi_matmul_residual", "bi_rope_table",
                "bi_rmsnorm_matmul_rope_kv", "bi_rmsnorm_backward",
                "bi_rmsnorm_backward_workspace_bytes", "bi_transpose", "bi_matmul_backward",
-               "bi_matmul_backward_workspace_bytes")
+               "bi_matmul_backward_workspace_bytes", "bi_swiglu_backward", "bi_rope_backward",
+               "bi_attention_backward", "bi_attention_backward_workspace_bytes",
+               "bi_rmsnorm_matmul_workspace_bytes")
 
     def __init__(self, path: str):
         if not os.path.exists(path):
@@ -155,10 +157,13 @@ class Library:
         L.bi_moe_combine.argtypes = [P, P, P, i64, i32, i64, P, P]
         L.bi_matmul_grouped.argtypes = [P, P, P, P, i32, i64, i64, i64, st, P]
         L.bi_fold_norm_weight.argtypes = [P, P, P, i64, i64, P]
-        L.bi_rmsnorm_matmul.argtypes = [P, P, P, i64, i64, i64, f32, st, P]
+        L.bi_rmsnorm_matmul.argtypes = [P, P, P, i64, i64, i64, f32, st, P, sz, P]
+        L.bi_rmsnorm_matmul_workspace_bytes.argtypes = [i64]
+        L.bi_rmsnorm_matmul_workspace_bytes.restype = sz
         L.bi_matmul_residual.argtypes = [P, P, P, P, i64, i64, i64, P]
         L.bi_rope_table.argtypes = [P, i32, i32, f32, P]
-        L.bi_rmsnorm_matmul_rope_kv.argtypes = [P, P, f32, kvp, P, i32, P, P, P, i64, i64, i32, P]
+        L.bi_rmsnorm_matmul_rope_kv.argtypes = [P, P, f32, kvp, P, i32, P, P, P, i64, i64, i32, P,
+                                                sz, P]
         L.bi_rmsnorm_backward_workspace_bytes.argtypes = [i64, i64]
         L.bi_rmsnorm_backward_workspace_bytes.restype = sz
         L.bi_rmsnorm_backward.argtypes = [P, P, P, P, P, i64, i64, f32, st, P, sz, P]
@@ -166,6 +171,12 @@ class Library:
         L.bi_matmul_backward_workspace_bytes.argtypes = [i64, i64, i64]
         L.bi_matmul_backward_workspace_bytes.restype = sz
         L.bi_matmul_backward.argtypes = [P, P, P, P, P, i64, i64, i64, st, P, sz, P]
+        L.bi_swiglu_backward.argtypes = [P, P, P, i64, i64, st, P]
+        L.bi_rope_backward.argtypes = [P, i64, P, P, i64, i64, i32, i32, f32, st, P]
+        L.bi_attention_backward.argtypes = [kvp, P, P, P, P, P, P, i32, i32, i64, i32, i32, f32,
+                                            P, P, P, P, sz, P]
+        L.bi_attention_backward_workspace_bytes.argtypes = [i32, i64]
+        L.bi_attention_backward_workspace_bytes.restype = sz
         for name in ("bi_rmsnorm", "bi_matmul", "bi_kv_write", "bi_attention_decode",
                      "bi_attention_prefill", "bi_device_status", "bi_debug_bounded_wait",
                      "bi_add_rmsnorm", "bi_embedding", "bi_rope_kv_write", "bi_swiglu",
@@ -173,7 +184,8 @@ class Library:
                      "bi_moe_combine", "bi_matmul_grouped", "bi_fold_norm_weight",
                      "bi_rmsnorm_matmul", "bi_matmul_residual", "bi_rope_table",
                      "bi_rmsnorm_matmul_rope_kv", "bi_rmsnorm_backward", "bi_transpose",
-                     "bi_matmul_backward"):
+                     "bi_matmul_backward", "bi_swiglu_backward", "bi_rope_backward",
+                     "bi_attention_backward"):
             getattr(L, name).restype = st
         self.lib = L
 
@@ -264,9 +276,10 @@ class Library:
         return out
 
     def bi_rmsnorm_matmul(self, x: torch.Tensor, wf: torch.Tensor, eps: float, out=None,
-                          out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
-        """C = RMSNorm(x) @ wf.T in one launch; x [M, K], wf [N, K] the weight with
-        the norm weight folded in (bi_fold_norm_weight)."""
+                          out_dtype=torch.bfloat16, ws=None, stream=None) -> torch.Tensor:
+        """C = RMSNorm(x) @ wf.T; x [M, K], wf [N, K] the weight with the norm
+        weight folded in (bi_fold_norm_weight).  `ws` (uint8, optional): the
+        workspace for the M row statistics."""
         _need(x, "x", torch.bfloat16)
         M, K = x.shape
         _need(wf, "wf", torch.bfloat16)
@@ -276,10 +289,20 @@ class Library:
         if out is None:
             out = torch.empty((M, N), dtype=out_dtype, device=x.device)
         _need(out, "out", out_dtype, (M, N))
+        ws = self._norm_ws(M, x.device, ws)
         self._check("bi_rmsnorm_matmul",
                     self.lib.bi_rmsnorm_matmul(_ptr(x), _ptr(wf), _ptr(out), M, N, K, float(eps),
-                                               _DT[out_dtype], _stream(stream)))
+                                               _DT[out_dtype], _ptr(ws), ws.numel(),
+                                               _stream(stream)))
         return out
+
+    def _norm_ws(self, M: int, device, ws=None) -> torch.Tensor:
+        """The fused norm forms' workspace (M row statistics): the caller's
+        `ws` if it is large enough, else a new one."""
+        need = max(int(self.lib.bi_rmsnorm_matmul_workspace_bytes(M)), 16)
+        if ws is None or ws.numel() * ws.element_size() < need:
+            ws = torch.empty(need, dtype=torch.uint8, device=device)
+        return ws
 
     def bi_matmul_residual(self, a: torch.Tensor, w: torch.Tensor, r: torch.Tensor, out=None,
                            stream=None) -> torch.Tensor:
@@ -379,11 +402,11 @@ class Library:
 
     def bi_rmsnorm_matmul_rope_kv(self, x: torch.Tensor, wf: torch.Tensor, eps: float,
                                   kv: PagedKV, rope_table: torch.Tensor, positions: torch.Tensor,
-                                  slot_mapping: torch.Tensor, Hq: int, q_out=None,
+                                  slot_mapping: torch.Tensor, Hq: int, q_out=None, ws=None,
                                   stream=None) -> torch.Tensor:
-        """RMSNorm(x) @ wf.T, then RoPE and the cache write of k and v, in one
-        launch (bit for bit bi_rmsnorm_matmul + bi_rope_kv_write); returns the
-        rotated q [T, Hq, d]."""
+        """RMSNorm(x) @ wf.T, then RoPE and the cache write of k and v in the
+        matmul's epilogue (bit for bit bi_rmsnorm_matmul + bi_rope_kv_write);
+        returns the rotated q [T, Hq, d]."""
         _need(x, "x", torch.bfloat16)
         T, K = x.shape
         d, Hkv = kv.head_dim, kv.num_kv_heads
@@ -397,10 +420,11 @@ class Library:
             q_out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=x.device)
         _need(q_out, "q_out", torch.bfloat16, (T, Hq, d))
         c = kv.c_struct()
+        ws = self._norm_ws(T, x.device, ws)
         self._check("bi_rmsnorm_matmul_rope_kv", self.lib.bi_rmsnorm_matmul_rope_kv(
             _ptr(x), _ptr(wf), float(eps), ctypes.byref(c), _ptr(rope_table),
             int(rope_table.shape[0]), _ptr(positions), _ptr(slot_mapping), _ptr(q_out), T, K, Hq,
-            _stream(stream)))
+            _ptr(ws), ws.numel(), _stream(stream)))
         return q_out
 
     # ------------------------------------------------------------ backward
@@ -448,6 +472,39 @@ class Library:
             _ptr(dc), _ptr(a), _ptr(w), _ptr(da), _ptr(dw), M, N, K, _DT[out_dtype], _ptr(ws),
             ws.numel(), _stream(stream)))
         return da, dw
+
+    def bi_swiglu_backward(self, gu: torch.Tensor, dout: torch.Tensor, out=None,
+                           out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+        """[dgate | dup] [T, 2F] of out = silu(gate) * up for the upstream dout [T, F]."""
+        _need(gu, "gu", torch.bfloat16)
+        T, F2 = gu.shape
+        _need(dout, "dout", torch.bfloat16, (T, F2 // 2))
+        if out is None:
+            out = torch.empty((T, F2), dtype=out_dtype, device=gu.device)
+        _need(out, "out", out_dtype, (T, F2))
+        self._check("bi_swiglu_backward", self.lib.bi_swiglu_backward(
+            _ptr(gu), _ptr(dout), _ptr(out), T, F2 // 2, _DT[out_dtype], _stream(stream)))
+        return out
+
+    def bi_rope_backward(self, dy: torch.Tensor, positions: torch.Tensor, theta: float = 10000.0,
+                         out=None, out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+        """Gradient of the rotary rotation's input for the upstream dy [T, nh, d]
+        (dy and out may be column slices of wider rows, e.g. of a q/k/v gradient)."""
+        if dy.dtype != torch.bfloat16 or dy.dim() != 3 or dy.stride(2) != 1 or \
+                dy.stride(1) != dy.shape[2] or not dy.is_cuda:
+            raise ValueError("dy: bf16 [T, nh, d] with dense heads")
+        T, nh, d = dy.shape
+        _need(positions, "positions", torch.int32, (T,))
+        if out is None:
+            out = torch.empty((T, nh, d), dtype=out_dtype, device=dy.device)
+        if out.dtype != out_dtype or tuple(out.shape) != (T, nh, d) or out.stride(2) != 1 or \
+                out.stride(1) != d:
+            raise ValueError("out: [T, nh, d] of out_dtype with dense heads")
+        self._check("bi_rope_backward", self.lib.bi_rope_backward(
+            ctypes.c_void_p(dy.data_ptr()), dy.stride(0), _ptr(positions),
+            ctypes.c_void_p(out.data_ptr()), out.stride(0), T, nh, d, float(theta),
+            _DT[out_dtype], _stream(stream)))
+        return out
 
     def bi_swiglu(self, gu: torch.Tensor, out=None, stream=None) -> torch.Tensor:
         """silu(gate) * up of gu [T, 2F] = [gate | up] -> [T, F]."""
@@ -597,6 +654,40 @@ class Library:
             ctypes.byref(c), _ptr(q), _ptr(out), _ptr(lse), _ptr(seq_lens), B, Hq,
             int(max_seq_len), float(scale), int(splits_per_cta), _stream(stream)))
         return (out, lse) if want_lse else out
+
+    def bi_attention_backward(self, kv: PagedKV, q: torch.Tensor, o: torch.Tensor,
+                              dout: torch.Tensor, lse: torch.Tensor, cu_q: torch.Tensor,
+                              ctx_lens: torch.Tensor, max_q_len: int, max_kv_len: int,
+                              scale: float | None = None, dk=None, dv=None, stream=None):
+        """(dq [T, Hq, d], dk, dv) of bi_attention_prefill's output o (with its
+        lse) for the upstream gradient dout.  dk and dv are shaped like the
+        caches; they start as zeros unless given (pages no sequence of the
+        call owns are not written)."""
+        _need(q, "q", torch.bfloat16)
+        T, Hq, d = q.shape
+        B = ctx_lens.shape[0]
+        _need(o, "o", torch.bfloat16, (T, Hq, d))
+        _need(dout, "dout", torch.bfloat16, (T, Hq, d))
+        _need(lse, "lse", torch.float32, (T, Hq))
+        _need(cu_q, "cu_q", torch.int32, (B + 1,))
+        _need(ctx_lens, "ctx_lens", torch.int32, (B,))
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        dq = torch.empty_like(q)
+        if dk is None:
+            dk = torch.zeros_like(kv.k_cache)
+        if dv is None:
+            dv = torch.zeros_like(kv.v_cache)
+        _need(dk, "dk", torch.bfloat16, tuple(kv.k_cache.shape))
+        _need(dv, "dv", torch.bfloat16, tuple(kv.v_cache.shape))
+        need = int(self.lib.bi_attention_backward_workspace_bytes(Hq, T))
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        c = kv.c_struct()
+        self._check("bi_attention_backward", self.lib.bi_attention_backward(
+            ctypes.byref(c), _ptr(q), _ptr(o), _ptr(dout), _ptr(lse), _ptr(cu_q), _ptr(ctx_lens),
+            B, Hq, T, int(max_q_len), int(max_kv_len), float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+            _ptr(ws), ws.numel(), _stream(stream)))
+        return dq, dk, dv
 
     def bi_attention_prefill(self, kv: PagedKV, q: torch.Tensor, cu_q: torch.Tensor,
                              ctx_lens: torch.Tensor, max_q_len: int, scale: float | None = None,

@@ -196,23 +196,35 @@ bi_status bi_fold_norm_weight(const void *W, const void *w, void *wf, int64_t N,
                                                  static_cast<cudaStream_t>(stream)));
 }
 
-bi_status bi_rmsnorm_matmul(const void *x, const void *wf, void *c, int64_t M, int64_t N,
-                            int64_t K, float eps, bi_dtype out_dtype, void *stream)
+size_t bi_rmsnorm_matmul_workspace_bytes(int64_t M)
 {
-    if (!gemm_shape_ok(M, N, K)) return BI_ERR_INVALID;
+    return M > 0 ? (size_t(M) * sizeof(float) + 255) / 256 * 256 : 0;
+}
+
+bi_status bi_rmsnorm_matmul(const void *x, const void *wf, void *c, int64_t M, int64_t N,
+                            int64_t K, float eps, bi_dtype out_dtype, void *ws, size_t ws_bytes,
+                            void *stream)
+{
+    if (!gemm_shape_ok(M, N, K) || K > 65536) return BI_ERR_INVALID;
     if (out_dtype != BI_BF16 && out_dtype != BI_F32) return BI_ERR_INVALID;
     if (!(eps >= 0.0f) || !std::isfinite(eps)) return BI_ERR_INVALID;
     if (M == 0) return BI_OK;
     if (!x || !wf || !c || !aligned16(x) || !aligned16(wf) || !aligned16(c)) return BI_ERR_INVALID;
+    if (!ws || ws_bytes < bi_rmsnorm_matmul_workspace_bytes(M) || !aligned16(ws))
+        return BI_ERR_WORKSPACE;
     DeviceState *d;
     bi_status st = device_state(&d);
     if (st != BI_OK) return st;
     CUtensorMap ta, tw;
     if ((st = gemm_maps(x, wf, M, N, K, &ta, &tw)) != BI_OK) return st;
-    bi::GemmEpi epi{1, eps, nullptr};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float *r = static_cast<float *>(ws);
+    cudaError_t e = bi::launch_row_rstd(x, r, M, K, eps, d->num_sms, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    bi::GemmEpi epi{};
+    epi.rs = r;
     return from_cuda(bi::launch_gemm_fused(ta, tw, c, int(M), int(N), int(K), out_dtype == BI_F32,
-                                           epi, d->num_sms, d->status, bi::kDefaultTimeoutNs,
-                                           static_cast<cudaStream_t>(stream)));
+                                           epi, d->num_sms, d->status, bi::kDefaultTimeoutNs, s));
 }
 
 bi_status bi_rope_table(float *table, int32_t max_pos, int32_t head_dim, float theta,
@@ -232,25 +244,31 @@ bi_status bi_rmsnorm_matmul_rope_kv(const void *x, const void *wf, float eps,
                                     const bi_paged_kv *kv, const float *rope_table,
                                     int32_t max_pos, const int32_t *positions,
                                     const int64_t *slot_mapping, void *q_out, int64_t T,
-                                    int64_t K, int32_t Hq, void *stream)
+                                    int64_t K, int32_t Hq, void *ws, size_t ws_bytes,
+                                    void *stream)
 {
     if (!kv_ok(kv) || !head_dim_ok(kv->head_dim)) return BI_ERR_INVALID;
     if (Hq < 1 || Hq % kv->num_kv_heads != 0 || max_pos < 1) return BI_ERR_INVALID;
     const int64_t N = int64_t(Hq + 2 * kv->num_kv_heads) * kv->head_dim;
-    if (!gemm_shape_ok(T, N, K)) return BI_ERR_INVALID;
+    if (!gemm_shape_ok(T, N, K) || K > 65536) return BI_ERR_INVALID;
     if (!(eps >= 0.0f) || !std::isfinite(eps)) return BI_ERR_INVALID;
     if (T == 0) return BI_OK;
     if (!x || !wf || !rope_table || !positions || !slot_mapping || !q_out || !aligned16(x) ||
         !aligned16(wf) || !aligned16(rope_table) || !aligned16(q_out))
         return BI_ERR_INVALID;
+    if (!ws || ws_bytes < bi_rmsnorm_matmul_workspace_bytes(T) || !aligned16(ws))
+        return BI_ERR_WORKSPACE;
     DeviceState *d;
     bi_status st = device_state(&d);
     if (st != BI_OK) return st;
     CUtensorMap ta, tw;
     if ((st = gemm_maps(x, wf, T, N, K, &ta, &tw)) != BI_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float *r = static_cast<float *>(ws);
+    cudaError_t e = bi::launch_row_rstd(x, r, T, K, eps, d->num_sms, s);
+    if (e != cudaSuccess) return from_cuda(e);
     bi::GemmEpi epi{};
-    epi.norm = 1;
-    epi.eps = eps;
+    epi.rs = r;
     epi.rope = rope_table;
     epi.max_pos = max_pos;
     epi.pos = positions;
@@ -263,8 +281,7 @@ bi_status bi_rmsnorm_matmul_rope_kv(const void *x, const void *wf, float eps,
     epi.Hkv = kv->num_kv_heads;
     epi.head_dim = kv->head_dim;
     return from_cuda(bi::launch_gemm_fused(ta, tw, nullptr, int(T), int(N), int(K), false, epi,
-                                           d->num_sms, d->status, bi::kDefaultTimeoutNs,
-                                           static_cast<cudaStream_t>(stream)));
+                                           d->num_sms, d->status, bi::kDefaultTimeoutNs, s));
 }
 
 bi_status bi_matmul_residual(const void *a, const void *w, const void *r, void *c, int64_t M,
@@ -279,7 +296,8 @@ bi_status bi_matmul_residual(const void *a, const void *w, const void *r, void *
     if (st != BI_OK) return st;
     CUtensorMap ta, tw;
     if ((st = gemm_maps(a, w, M, N, K, &ta, &tw)) != BI_OK) return st;
-    bi::GemmEpi epi{0, 0.0f, r};
+    bi::GemmEpi epi{};
+    epi.residual = r;
     return from_cuda(bi::launch_gemm_fused(ta, tw, c, int(M), int(N), int(K), false, epi,
                                            d->num_sms, d->status, bi::kDefaultTimeoutNs,
                                            static_cast<cudaStream_t>(stream)));
@@ -385,6 +403,40 @@ bi_status bi_matmul_backward(const void *dc, const void *a, const void *w, void 
             return from_cuda(e);
     }
     return BI_OK;
+}
+
+bi_status bi_swiglu_backward(const void *gu, const void *dout, void *dgu, int64_t T, int64_t F,
+                             bi_dtype out_dtype, void *stream)
+{
+    if (T < 0 || F < 8 || F % 8 != 0) return BI_ERR_INVALID;
+    if (out_dtype != BI_BF16 && out_dtype != BI_F32) return BI_ERR_INVALID;
+    if (T == 0) return BI_OK;
+    if (!gu || !dout || !dgu || !aligned16(gu) || !aligned16(dout) || !aligned16(dgu))
+        return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_swiglu_backward(gu, dout, dgu, T, F, out_dtype == BI_F32,
+                                                d->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+bi_status bi_rope_backward(const void *dy, int64_t ld_dy, const int32_t *positions, void *dx,
+                           int64_t ld_dx, int64_t T, int32_t num_heads, int32_t head_dim,
+                           float theta, bi_dtype out_dtype, void *stream)
+{
+    if (T < 0 || num_heads < 1 || !head_dim_ok(head_dim)) return BI_ERR_INVALID;
+    if (out_dtype != BI_BF16 && out_dtype != BI_F32) return BI_ERR_INVALID;
+    if (!(theta > 1.0f) || !std::isfinite(theta)) return BI_ERR_INVALID;
+    const int64_t row = int64_t(num_heads) * head_dim;
+    if (ld_dy < row || ld_dx < row || ld_dy % 8 != 0 || ld_dx % 8 != 0) return BI_ERR_INVALID;
+    if (T == 0) return BI_OK;
+    if (!dy || !positions || !dx || !aligned16(dy) || !aligned16(dx)) return BI_ERR_INVALID;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+    return from_cuda(bi::launch_rope_backward(dy, ld_dy, positions, dx, ld_dx, T, num_heads,
+                                              head_dim, double(theta), out_dtype == BI_F32,
+                                              d->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
 bi_status bi_add_rmsnorm(void *x, const void *delta, const void *w, void *y, int64_t M,
@@ -788,6 +840,73 @@ bi_status bi_attention_prefill(const bi_paged_kv *kv, const void *q, void *o, fl
     const uint32_t bq[3] = {64, 1, 128};
     if (!encode(&tq, q, 3, dq, sq, bq)) return BI_ERR_CUDA;
     return from_cuda(bi::launch_attention(tq, p, D, static_cast<cudaStream_t>(stream)));
+}
+
+size_t bi_attention_backward_workspace_bytes(int32_t Hq, int64_t T_total)
+{
+    if (Hq < 1 || T_total < 1) return 0;
+    return bi::attn_bwd_ws_bytes(int64_t(Hq) * T_total);
+}
+
+bi_status bi_attention_backward(const bi_paged_kv *kv, const void *q, const void *o,
+                                const void *dout, const float *lse, const int32_t *cu_q,
+                                const int32_t *ctx_lens, int32_t B, int32_t Hq, int64_t T_total,
+                                int32_t max_q_len, int32_t max_kv_len, float scale, void *dq,
+                                void *dk_cache, void *dv_cache, void *ws, size_t ws_bytes,
+                                void *stream)
+{
+    if (!attn_common_ok(kv, Hq)) return BI_ERR_INVALID;
+    if (!head_dim_ok(kv->head_dim)) return BI_ERR_UNSUPPORTED;
+    if (B < 0 || T_total < 0 || max_q_len < 0 || max_kv_len < 0 || !std::isfinite(scale))
+        return BI_ERR_INVALID;
+    if (int64_t(max_kv_len) > int64_t(kv->max_pages_per_seq) * BI_PAGE_SIZE) return BI_ERR_INVALID;
+    if (T_total > INT32_MAX) return BI_ERR_UNSUPPORTED;
+    if (B == 0 || T_total == 0 || max_q_len == 0) return BI_OK;
+    if (max_kv_len < max_q_len) return BI_ERR_INVALID;
+    if (B > 65535) return BI_ERR_UNSUPPORTED;
+    if (!q || !o || !dout || !lse || !cu_q || !ctx_lens || !dq || !dk_cache || !dv_cache)
+        return BI_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk_cache) || !aligned16(dv_cache))
+        return BI_ERR_INVALID;
+    if (dk_cache == kv->k_cache || dk_cache == kv->v_cache || dv_cache == kv->k_cache ||
+        dv_cache == kv->v_cache || dk_cache == dv_cache)
+        return BI_ERR_INVALID;
+    const int64_t rows = T_total * Hq;
+    if (!ws || ws_bytes < bi::attn_bwd_ws_bytes(rows) || !aligned16(ws)) return BI_ERR_WORKSPACE;
+    DeviceState *d;
+    bi_status st = device_state(&d);
+    if (st != BI_OK) return st;
+
+    bi::AttnBwdParams p{};
+    p.k_cache = kv->k_cache;
+    p.v_cache = kv->v_cache;
+    p.block_table = kv->block_table;
+    p.max_pages = kv->max_pages_per_seq;
+    p.num_pages = kv->num_pages;
+    p.Hkv = kv->num_kv_heads;
+    p.Hq = Hq;
+    p.group = Hq / kv->num_kv_heads;
+    p.B = B;
+    p.cu_q = cu_q;
+    p.ctx_lens = ctx_lens;
+    p.num_q_tiles = (max_q_len + 127) / 128;
+    p.num_key_blocks = (max_kv_len + 127) / 128;
+    p.scale = scale;
+    p.scale_log2 = float(double(scale) * 1.4426950408889634);
+    p.q = q;
+    p.o = o;
+    p.dout = dout;
+    p.lse = lse;
+    p.lse2 = static_cast<float *>(ws);
+    p.delta = static_cast<float *>(ws) + rows;
+    p.dq = dq;
+    p.dk = dk_cache;
+    p.dv = dv_cache;
+    p.status = d->status;
+    p.timeout_ns = bi::kDefaultTimeoutNs;
+    return from_cuda(bi::launch_attention_backward(p, kv->head_dim, rows, d->num_sms,
+                                                   static_cast<cudaStream_t>(stream)));
 }
 
 bi_status bi_device_status(void *stream)

@@ -145,10 +145,43 @@ struct Item {
     int b, g, h;          // sequence, kv head, query head (prefill)
     int s0, s1, n_splits; // split range of this block; splits of the sequence
     int kv_len;           // keys in the cache for this sequence
+    int key0, kend;       // keys key0 .. kend-1 of the sequence are this block's;
+                          // split s covers key0 + (s - s0) 256 .. +255 (below kend)
     int q_row0;           // prefill: first packed token of the tile
     int rows;             // prefill: valid tokens in the tile
     int pos0;             // prefill: absolute position of the tile's first row
 };
+
+__device__ __forceinline__ int key_of(const Item &it, int s) { return it.key0 + (s - it.s0) * kSplit; }
+
+// Decode: whether this block alone covers the whole sequence, and the index
+// of the record a block that does not hands its merged range over in.
+__device__ __forceinline__ bool item_whole(const Item &it)
+{
+    return it.key0 == 0 && it.kend == it.kv_len && it.s1 == it.n_splits;
+}
+__device__ __forceinline__ int item_rec(const Item &it)
+{
+#if BI_INVARIANT
+    return it.s1 - 1;  // its last split
+#else
+    return it.s0;      // its block number
+#endif
+}
+
+#if !BI_INVARIANT
+// Variant-off decode: the sequence's keys are cut into cnt ranges of R keys
+// (R a whole number of pages), cnt = min(blocks per sequence, its 256-key
+// splits) -- the split SIZE follows the load.  Block x covers keys x R ..
+// min((x + 1) R, L) - 1 in 256-key pieces counted from x R.
+__device__ __forceinline__ int variant_range(int L, int nblk)
+{
+    const int n = (L + kSplit - 1) / kSplit;
+    const int cnt = min(nblk, n);
+    const int per = (L + cnt - 1) / cnt;
+    return (per + kPage - 1) / kPage * kPage;
+}
+#endif
 
 // Work item idx of a launch.  Decode: idx = x + nblk (g + Hkv z), block x of
 // the split range of kv head g of the z-th sequence of the launch order
@@ -166,13 +199,25 @@ __device__ __forceinline__ bool make_item(const AttnParams &p, int idx, Item &it
         it.h = 0;
         it.kv_len = p.seq_lens[it.b];
         it.n_splits = (it.kv_len + kSplit - 1) / kSplit;
-        it.s0 = x * p.splits_per_cta;
         if (it.n_splits > p.max_splits) {  // longer than the declared maximum
             if (threadIdx.x == 0) record_status(p.status, BI_DEV_BAD_INDEX);
             return false;
         }
-        if (it.kv_len <= 0 || it.s0 >= it.n_splits) return false;
+        if (it.kv_len <= 0) return false;
+#if BI_INVARIANT
+        it.s0 = x * p.splits_per_cta;
+        if (it.s0 >= it.n_splits) return false;
         it.s1 = min(it.n_splits, it.s0 + p.splits_per_cta);
+        it.key0 = it.s0 * kSplit;
+        it.kend = it.kv_len;
+#else
+        const int R = variant_range(it.kv_len, nblk);
+        it.key0 = x * R;
+        if (it.key0 >= it.kv_len) return false;
+        it.kend = min(it.kv_len, it.key0 + R);
+        it.s0 = x;
+        it.s1 = x + (it.kend - it.key0 + kSplit - 1) / kSplit;
+#endif
         it.q_row0 = it.rows = it.pos0 = 0;
     } else {
         const int r = idx / p.Hq;
@@ -192,6 +237,8 @@ __device__ __forceinline__ bool make_item(const AttnParams &p, int idx, Item &it
         it.s0 = 0;
         it.s1 = t_max / kSplit + 1;
         it.n_splits = (it.kv_len + kSplit - 1) / kSplit;
+        it.key0 = 0;
+        it.kend = it.kv_len;
     }
     return true;
 }
@@ -227,19 +274,6 @@ __device__ __forceinline__ float logit(float s, float cs, float m_s)
     return ex2(__fmaf_rn(s, cs, -m_s));
 }
 
-// Maximum of the visible logits of 32 keys kc .. kc+31.
-__device__ __forceinline__ void chunk_max(const uint32_t (&r)[32], int kc, int t, float (&mx)[8])
-{
-    if (kc + 31 <= t) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[j]));
-    } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-            if (kc + j <= t) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[j]));
-    }
-}
-
 // p of the 32 keys kc .. kc+31, computed in place (r[j] becomes the bits of
 // p_j): packed bf16 P written to TMEM at `pcol` (16 columns), the class sums
 // S_u advanced by this chunk in the order of tree8.
@@ -266,46 +300,58 @@ __device__ __forceinline__ void chunk_exp(uint32_t (&r)[32], int kc, int t, floa
                                      e(16 + 2 * u), e(17 + 2 * u), e(24 + 2 * u), e(25 + 2 * u)));
 }
 
-// Softmax of one split, one row per thread (any row layout; used by
-// prefill and by decode with more than 8 query rows per lane quarter).
-// S is read from TMEM columns sb .. sb+255 in two passes of 32-column
-// loads, the next load in flight while a chunk is processed; P (bf16 pairs)
-// is written over columns sb .. sb+127 as the second pass goes (each store
-// lands on columns this thread has already read).  Returns m_s (scaled,
-// log2 units) and l_s.  (P V cannot start before the whole pass is done: it
-// writes O_s over the logits of keys 128..255.)
-__device__ __forceinline__ void softmax_rows(uint32_t sb, int k0, int t, float cs, float &m_s,
-                                             float &l_s)
+// Row maximum of one split's visible logits, scaled: m_s = round(c max_j S_j)
+// (for c > 0, x -> round(x c) is monotonic, so this equals max_j round(S_j c);
+// a maximum is exact in any order).  S is read from TMEM columns
+// sb .. sb+255 in 16-column loads, the next load in flight while a chunk is
+// scanned; eight accumulators break the dependency chain.  The loop is kept
+// rolled (two loads per trip): a small instruction footprint matters more
+// here than unrolling, since the block's other warps run other code on the
+// same sub-partitions.
+__device__ __forceinline__ float row_max(uint32_t sb, int k0, int t, float cs)
 {
-    constexpr int NC = kSplit / 32;  // 32-key chunks
-    // pass 1: maximum of the raw logits over the visible keys.  For c > 0,
-    // x -> round(x * c) is monotonic, so max_j round(S_j c) = round(max_j S_j * c).
-    // (A maximum is exact in any order; eight accumulators break the chain.)
+    constexpr int NC = kSplit / 16;  // 16-key chunks (small loads: this runs on the
+                                     // fold warps, whose registers hold the output)
     float mx[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-    // The loops are kept rolled (two loads of each kind per trip): a small
-    // instruction footprint matters more here than unrolling, since the
-    // block's other warps run other code on the same sub-partitions.
-    {
-        // 32-column loads, the next in flight while a chunk is scanned
-        uint32_t ra[32], rb[32];
-        tmem_ld32(sb, ra);
-#pragma unroll 1
-        for (int c = 0; c < NC; c += 2) {
-            tmem_wait_ld(ra);
-            tmem_ld32(sb + 32 * (c + 1), rb);
-            chunk_max(ra, k0 + 32 * c, t, mx);
-            tmem_wait_ld(rb);
-            if (c + 2 < NC) tmem_ld32(sb + 32 * (c + 2), ra);
-            chunk_max(rb, k0 + 32 * (c + 1), t, mx);
+    auto scan = [&](const uint32_t (&r)[16], int kc) {
+        if (kc + 15 <= t) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[j]));
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (kc + j <= t) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[j]));
         }
+    };
+    uint32_t ra[16], rb[16];
+    tmem_ld16(sb, ra);
+#pragma unroll 1
+    for (int c = 0; c < NC; c += 2) {
+        tmem_wait_ld16(ra);
+        tmem_ld16(sb + 16 * (c + 1), rb);
+        scan(ra, k0 + 16 * c);
+        tmem_wait_ld16(rb);
+        if (c + 2 < NC) tmem_ld16(sb + 16 * (c + 2), ra);
+        scan(rb, k0 + 16 * (c + 1));
     }
     const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-    m_s = __fmul_rn(mraw, cs);
-    // pass 2: p = 2^(S c - m_s), masked keys 0; P into TMEM; the sum in the
-    // order of tree8.  32-key chunks, the next chunk's load in flight.
+    return __fmul_rn(mraw, cs);
+}
+
+// The exponent pass of one split, one row per thread (any row layout; used
+// by prefill and by decode with more than 8 query rows per lane quarter),
+// given the row's m_s (row_max, computed by another warp one split ahead):
+// p = 2^(S c - m_s) with masked keys 0, P (bf16 pairs) written over TMEM
+// columns sb .. sb+127 as the pass goes (each store lands on columns this
+// thread has already read), l_s summed in the order of tree8; 32-key chunks,
+// the next chunk's load in flight.  (P V cannot start before the whole pass
+// is done: it writes O_s over the logits of keys 128..255.)
+__device__ __forceinline__ float softmax_exp(uint32_t sb, int k0, int t, float cs, float m_s)
+{
+    constexpr int NC = kSplit / 32;
     float S[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     uint32_t ra[32], rb[32];
     tmem_ld32(sb, ra);
@@ -319,7 +365,7 @@ __device__ __forceinline__ void softmax_rows(uint32_t sb, int k0, int t, float c
         chunk_exp(rb, k0 + 32 * (c + 1), t, cs, m_s, sb + 16 * (c + 1), S);
     }
     tmem_wait_st();
-    l_s = __fadd_rn(__fadd_rn(S[0], S[1]), __fadd_rn(S[2], S[3]));
+    return __fadd_rn(__fadd_rn(S[0], S[1]), __fadd_rn(S[2], S[3]));
 }
 
 // Softmax of one split for decode when the query rows of this lane quarter
@@ -430,7 +476,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint64_t *barP = barS + 2;      // [2] P and (m_s, l_s) of buffer b written (128 arrivals)
     uint64_t *barO = barP + 2;      // [2] O_s of buffer b computed
     uint64_t *barF = barO + 2;      // [2] O_s of buffer b merged, buffer free
-    uint64_t *drain = barF + 2;
+    uint64_t *barM = barF + 2;      // [2] row maxima of buffer b's split written (128 arrivals)
+    uint64_t *drain = barM + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
@@ -447,6 +494,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&barP[b], 128);
             mbar_init(&barO[b], 1);
             mbar_init(&barF[b], kFoldThreads);
+            mbar_init(&barM[b], 128);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -478,8 +526,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!make_item(p, idx, it)) continue;
             const int32_t *bt_row = p.block_table + int64_t(it.b) * p.max_pages;
             auto lookup = [&](int s) -> int {
-                const int lp = s * (kSplit / kPage) + lane;  // logical page
-                if (lane >= kSplit / kPage || lp * kPage >= it.kv_len) return -1;
+                const int lp = key_of(it, s) / kPage + lane;  // logical page
+                if (lane >= kSplit / kPage || lp * kPage >= it.kend) return -1;
                 return lp < p.max_pages ? __ldg(bt_row + lp) : -2;
             };
             // Load list (relative split j, n splits): K0, K1, V0, K2, V1, K3,
@@ -500,7 +548,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (which == 0) record_status(p.status, BI_DEV_BAD_INDEX);
                     phys = -1;
                 }
-                const int nk = min(kSplit, it.kv_len - s * kSplit);  // valid keys, >= 1
+                const int nk = min(kSplit, it.kend - key_of(it, s));  // valid keys, >= 1
                 const int full_pages = nk / kPage;
                 const int npages = (nk + kPage - 1) / kPage;
                 int got = 1;
@@ -688,28 +736,57 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int q = warp & 3;
         const uint32_t lane_base = tmem_addr(tmem, 32 * q, 0);
         const int row_id = 32 * q + lane;  // TMEM lane of this row
-        int gs = 0;
-        bool ok = true;
-        for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
-            Item it;
-            if (!make_item(p, idx, it)) continue;
-            bool valid, active;
-            int t, local;
-            int64_t out_row;
+        // Rows whose softmax reads one row per thread (all but decode with at
+        // most 8 rows per lane quarter) get their maxima from the first-half
+        // fold warp of the quarter (warps 2, 3, 8, 9), one split ahead, so
+        // the softmax warp only runs the exponent pass.  The maximum is exact
+        // in any order: the bits are those of a one-warp softmax.
+        const bool max_ahead = !(p.decode && p.rows_per_q <= 8);
+        const bool max_warp = max_ahead && !is_softmax && warp < 10;
+        // This thread's row of an item: its last visible key t, whether its
+        // lane quarter holds any row, whether the row is a real one, and
+        // where its output goes.
+        auto row_of = [&](const Item &it, int &t, bool &active, bool &valid, int64_t &out_row) {
             if (p.decode) {
-                local = q * p.rows_per_q + lane;
+                const int local = q * p.rows_per_q + lane;
                 valid = lane < p.rows_per_q && local < p.group;
-                t = it.kv_len - 1;
-                const int head = it.g * p.group + local;
-                out_row = int64_t(it.b) * p.Hq + head;
+                t = it.kend - 1;  // the block's last key (the sequence's, but for a
+                                  // variant-off range that ends before it)
+                out_row = int64_t(it.b) * p.Hq + it.g * p.group + local;
                 active = q * p.rows_per_q < p.group;
             } else {
-                local = 32 * q + lane;
+                const int local = 32 * q + lane;
                 valid = local < it.rows;
                 t = it.pos0 + local;
                 out_row = int64_t(it.q_row0 + local) * p.Hq + it.h;
                 active = 32 * q < it.rows;
             }
+        };
+        // The scaled maximum of split number g (key base k0) for this row,
+        // written to sML and signalled on barM.
+        auto max_split = [&](int g, int k0, int t_row, bool act) -> bool {
+            const int b = g & 1;
+            const uint32_t par = uint32_t(g >> 1) & 1u;
+            if (!wait(&barS[b], par, ctl)) return false;
+            tc_fence_after();
+            const float m_s =
+                act ? row_max(lane_base + C::BUF_COLS * uint32_t(b) + C::P_OFF, k0, t_row, p.scale_log2)
+                    : -INFINITY;
+            sML[(b * 128 + row_id) * 2 + 0] = m_s;
+            tc_fence_before();
+            mbar_arrive(&barM[b]);
+            return true;
+        };
+        int gs = 0;
+        bool ok = true;
+        bool ahead = false;  // the maximum of this item's first split is already written
+        for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
+            Item it;
+            if (!make_item(p, idx, it)) continue;
+            bool valid, active;
+            int t;
+            int64_t out_row;
+            row_of(it, t, active, valid, out_row);
             if (is_softmax) {
                 // -------------------------------------------------- softmax
                 const float cs = p.scale_log2;
@@ -729,13 +806,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (heads16) {
                         // rows of this quarter in lanes 0..7, four threads a row
                         softmax_heads16(lane_base + C::BUF_COLS * uint32_t(b) + C::P_OFF,
-                                        s * kSplit, t, cs, m_s, l_s);
+                                        key_of(it, s), t, cs, m_s, l_s);
                         if ((lane & 3) == 0) {
                             sML[(b * 128 + 32 * q + (lane >> 2)) * 2 + 0] = m_s;
                             sML[(b * 128 + 32 * q + (lane >> 2)) * 2 + 1] = l_s;
                         }
                     } else {
-                        if (active) softmax_rows(sb + C::P_OFF, s * kSplit, t, cs, m_s, l_s);
+                        if (max_ahead) {
+                            if (!wait(&barM[b], par, ctl)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            m_s = sML[(b * 128 + row_id) * 2 + 0];
+                        }
+                        if (active) l_s = softmax_exp(sb + C::P_OFF, key_of(it, s), t, cs, m_s);
                         sML[(b * 128 + row_id) * 2 + 0] = m_s;
                         sML[(b * 128 + row_id) * 2 + 1] = l_s;
                     }
@@ -760,12 +845,45 @@ __global__ void __launch_bounds__(THREADS, 1)
                 float O[HW];
 #pragma unroll
                 for (int j = 0; j < HW; ++j) O[j] = 0.0f;
+                if (max_warp && !ahead && it.s1 > it.s0 && !max_split(gs, it.key0, t, active)) {
+                    ok = false;
+                    break;
+                }
+                ahead = false;
                 for (int s = it.s0; s < it.s1; ++s) {
                     const int g = gs + (s - it.s0);
                     const int b = g & 1;
                     const uint32_t par = uint32_t(g >> 1) & 1u;
+                    if (max_warp) {
+                        // the next split's maximum, before this split's merge:
+                        // the next split of this item, or the first split of
+                        // the block's next item
+                        if (s + 1 < it.s1) {
+                            if (!max_split(g + 1, key_of(it, s + 1), t, active)) {
+                                ok = false;
+                                break;
+                            }
+                        } else if (!p.decode) {
+                            // (decode runs one block per item: no next item)
+                            for (int nidx = idx + int(gridDim.x); nidx < p.items; nidx += gridDim.x) {
+                                // the prefill item nidx (as make_item): this
+                                // row's last visible key, its quarter's rows
+                                const int r = nidx / p.Hq;
+                                const int nb = r / p.num_q_tiles;
+                                const int tile = p.num_q_tiles - 1 - (r - nb * p.num_q_tiles);
+                                const int n = p.cu_q[nb + 1] - p.cu_q[nb];
+                                if (tile * 128 >= n) continue;
+                                const int npos0 = p.ctx_lens[nb] + tile * 128;
+                                const bool nact = 32 * q < n - tile * 128;
+                                if (!max_split(g + 1, 0, npos0 + 32 * q + lane, nact)) ok = false;
+                                ahead = ok;
+                                break;
+                            }
+                            if (!ok) break;
+                        }
+                    }
                     const uint32_t ob = lane_base + C::BUF_COLS * uint32_t(b) + C::O_OFF + col0;
-                    const int k0 = s * kSplit;
+                    const int k0 = key_of(it, s);
                     // barP: (m_s, l_s) of this split are in shared memory;
                     // barO: O_s is in TMEM.
                     if (!wait(&barP[b], par, ctl) || !wait(&barO[b], par, ctl)) {
@@ -832,7 +950,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     mbar_arrive(&barF[b]);
                 }
                 if (ok && active && valid && !spill) {
-                    if (!p.decode || (it.s0 == 0 && it.s1 == it.n_splits)) {
+                    if (!p.decode || item_whole(it)) {
                         write_out<HW>(O, l, m,
                                       static_cast<__nv_bfloat16 *>(p.o) + out_row * D + col0,
                                       (p.lse && half == 0) ? p.lse + out_row : nullptr);
@@ -841,7 +959,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         // merged state over its range (ending at split s1-1)
                         // to attn_combine (in the invariant build only the
                         // first block gets here; the others write every split)
-                        float *rec = p.ws + ((out_row * p.max_splits) + (it.s1 - 1)) * C::REC;
+                        float *rec = p.ws + ((out_row * p.max_splits) + item_rec(it)) * C::REC;
                         if (half == 0) {
                             rec[0] = m;
                             rec[1] = l;
@@ -922,10 +1040,19 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p)
     const int b = static_cast<int>(row / p.Hq);
     const int L = p.seq_lens[b];
     const int n = (L + kSplit - 1) / kSplit;
+    const float *base = p.ws + row * p.max_splits * C::REC;
+#if BI_INVARIANT
     const int first_end = p.splits_per_cta;  // splits merged by the first block
     if (L <= 0 || n <= first_end || n > p.max_splits) return;
-    const float *base = p.ws + row * p.max_splits * C::REC;
     const float *rec = base + int64_t(first_end - 1) * C::REC;
+#else
+    // variant-off: one record per block of keys x R .. (x + 1) R - 1
+    const int nblk = (p.max_splits + p.splits_per_cta - 1) / p.splits_per_cta;
+    if (L <= 0 || n > p.max_splits) return;
+    const int R = variant_range(L, nblk);
+    if (R >= L) return;  // one block: its output is written
+    const float *rec = base;
+#endif
     float m = rec[0], l = rec[1];
     float O[PER];
 #pragma unroll
@@ -934,9 +1061,8 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p)
     for (int s = first_end; s < n; ++s) {
         rec = base + int64_t(s) * C::REC;
 #else
-    // variant-off: one record per block, at the block's last split
-    for (int e = 2 * first_end; e < n + first_end; e += first_end) {
-        rec = base + int64_t(min(e, n) - 1) * C::REC;
+    for (int x = 1; x * R < L; ++x) {
+        rec = base + int64_t(x) * C::REC;
 #endif
         const float ms = rec[0], ls = rec[1];
         float mn, a, cc;

@@ -1,0 +1,605 @@
+// attention_bwd.cu -- backward of the paged causal attention, for the trainer
+// side of on-policy RL (xitu-tech news, "强化学习的突破": the trainer must
+// reproduce the sampler's numbers, so its passes run on fixed, deterministic
+// reduction orders).
+//
+// For a query row i (absolute position t_i, visible keys j <= t_i) with the
+// forward's log-sum-exp lse_i and output o_i, and an upstream gradient dO_i:
+//   P_ij  = exp(scale q_i . k_j - lse_i)                 (the forward's weights)
+//   dP_ij = dO_i . v_j,   Delta_i = dO_i . o_i           (= sum_j P_ij dP_ij)
+//   dS_ij = P_ij (dP_ij - Delta_i)
+//   dq_i  = scale sum_j dS_ij k_j
+//   dk_j  = scale sum_i dS_ij q_i,   dv_j = sum_i P_ij dO_i
+// where the sums for dk_j and dv_j run over every query row of the sequence's
+// chunk that sees key j, in all query heads of k_j's group.
+//
+// Three kernels, no atomics:
+//   attn_bwd_prep_kernel   Delta_i (fp32, a fixed order) and lse_i log2(e).
+//   attn_bwd_dkv_kernel    one block per (sequence, kv head, 128-key block):
+//                          for each query head of the group (ascending) and
+//                          each 128-row query tile (ascending):
+//                            S^T = K Q^T,  dP^T = V dO^T        (tcgen05)
+//                            P^T, dS^T elementwise (one key row per thread)
+//                            dV += P^T dO,  dK += dS^T Q         (P^T, dS^T
+//                                                                 from TMEM)
+//                          so a key's dk and dv are sums in one fixed order
+//                          over its own sequence's rows.
+//   attn_bwd_dq_kernel     one block per (sequence, query head, 128-row tile):
+//                          for each 128-key block ascending:
+//                            S = Q K^T,  dP = dO V^T;  P, dS elementwise (one
+//                            query row per thread);  dQ += dS K.
+//                          A row's dq depends on that row alone.
+// P and dS are rounded to bf16 to enter the tensor core (as the forward
+// rounds P before P V); every other quantity is fp32.
+//
+// Shared-memory operands are in the tensor core's no-swizzle core-matrix
+// layout (8 rows x 16 bytes = 128 contiguous bytes): a 128-row tile of q or dO
+// as [value block d/8][row 128][8 values], a 128-key block of the cache as its
+// eight page blocks, already in that layout.  Every tile is loaded by the
+// threads with 16-byte loads (rows outside the sequence or the chunk become
+// zeros), so that a masked product never meets a stale NaN.
+//
+// Block of 128 threads (4 warps; warp w owns TMEM lanes 32w .. 32w+31).
+// Thread 0 issues the MMAs; every wait is bounded and its outcome is agreed
+// on by the whole block (__syncthreads_and), so that a timeout ends every
+// thread's loop at the same point.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "bi_common.cuh"
+#include "bi_launch.h"
+#include "bi_ptx.cuh"
+
+namespace bi {
+namespace {
+
+constexpr int kBwdThreads = 128;
+constexpr int kKeyBlock = 128;  // keys per block of the dk/dv kernel and per step of dq
+constexpr int kQTile = 128;     // query rows per tile
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BwdCfg {
+    static constexpr int TILE_BYTES = kQTile * D * 2;          // q or dO tile
+    static constexpr int PAGE_BYTES = kPage * D * 2;           // one page block
+    static constexpr int KGROUP_BYTES = PAGE_BYTES / 2;        // 8-key groups
+    static constexpr int BLOCK_BYTES = (kKeyBlock / kPage) * PAGE_BYTES;  // 128 keys
+    static constexpr int VEC_BYTES = 2 * kQTile * 4;           // lse2, Delta of 128 rows
+    static constexpr int SLACK = 1024;
+    static constexpr int SMEM = SLACK + 2 * TILE_BYTES + 2 * BLOCK_BYTES + VEC_BYTES + 64;
+    // TMEM columns: S (128), dP (128), two d-wide accumulators (dV, dK) or one (dQ)
+    static constexpr uint32_t S_COL = 0, DP_COL = 128, ACC0 = 256, ACC1 = 256 + D;
+    static constexpr uint32_t TMEM_COLS = 512;
+};
+
+// Byte offset of values 8c .. 8c+7 of row r in a 128-row tile.
+__device__ __forceinline__ uint32_t tile_off(int r, int c) { return (uint32_t(c) * 128u + r) * 16u; }
+
+// Byte offset, inside a page block of head dim D, of values 8c .. 8c+7 of key r.
+template <int D>
+__device__ __forceinline__ uint32_t page_off(int r, int c)
+{
+    return uint32_t(r >> 3) * (D * 16) + uint32_t(c) * 128u + uint32_t(r & 7) * 16u;
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b)
+{
+    __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&p);
+}
+
+// Rows row0 .. row0+127 of one head of a [T, H, D] bf16 tensor into a tile;
+// rows at or past `rows` are zero.
+template <int D>
+__device__ __forceinline__ void load_tile(uint8_t *tile, const uint4 *src, int64_t row0, int rows,
+                                          int H, int h)
+{
+    constexpr int P = D / 8;
+    for (int e = threadIdx.x; e < kQTile * P; e += kBwdThreads) {
+        const int r = e % kQTile, c = e / kQTile;  // rows fastest: conflict-free stores
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r < rows) v = __ldg(src + ((row0 + r) * H + h) * P + c);
+        *reinterpret_cast<uint4 *>(tile + tile_off(r, c)) = v;
+    }
+}
+
+// Keys k0 .. k0+127 of kv head g of one sequence (its page-table row `bt`)
+// into eight page blocks; keys at or past kv_len are zero.
+template <int D>
+__device__ __forceinline__ void load_keys(uint8_t *dst, const uint8_t *cache, const int32_t *bt,
+                                          int k0, int kv_len, int Hkv, int g, int num_pages,
+                                          unsigned *status)
+{
+    using C = BwdCfg<D>;
+    constexpr int PP = C::PAGE_BYTES / 16;  // 16-byte pieces of a page block
+    for (int e = threadIdx.x; e < (kKeyBlock / kPage) * PP; e += kBwdThreads) {
+        const int pg = e / PP, piece = e - pg * PP;
+        const uint32_t off = uint32_t(piece) * 16u;
+        // piece -> key: off = kg * 16D + c * 128 + r * 16
+        const int kg = int(off / (D * 16)), r = int(off % 128) / 16;
+        const int key = k0 + pg * kPage + kg * 8 + r;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (key < kv_len) {
+            const int phys = __ldg(bt + (k0 / kPage + pg));
+            if (phys >= 0 && phys < num_pages)
+                v = __ldg(reinterpret_cast<const uint4 *>(
+                            cache + (int64_t(phys) * Hkv + g) * int64_t(C::PAGE_BYTES) + off));
+            else if (piece == 0)
+                record_status(status, BI_DEV_BAD_INDEX);
+        }
+        *reinterpret_cast<uint4 *>(dst + pg * C::PAGE_BYTES + off) = v;
+    }
+}
+
+// Waits for phase `parity` of `bar` on every thread; the block agrees on the
+// outcome (true only if every thread saw the phase complete).
+__device__ __forceinline__ bool block_wait(uint64_t *bar, uint32_t parity, const WaitCtl &ctl)
+{
+    const bool ok = wait(bar, parity, ctl);
+    return __syncthreads_and(ok ? 1 : 0) != 0;
+}
+
+__device__ bool drain_wait(uint64_t *bar, uint32_t parity, uint64_t timeout_ns)
+{
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs))
+        if (global_ns() - t0 > timeout_ns) return false;
+    return true;
+}
+
+// ---------------------------------------------------------------- prep
+// delta[r] = sum_v dO[r, v] o[r, v] (fp32: lane-strided fused multiply-adds
+// in value order, then a xor butterfly); lse2[r] = lse[r] log2(e).  One warp
+// per (token, head) row.
+__global__ void attn_bwd_prep_kernel(const uint16_t *__restrict__ o, const uint16_t *__restrict__ dout,
+                                     const float *__restrict__ lse, int64_t rows, int d,
+                                     float *__restrict__ lse2, float *__restrict__ delta)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t r = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+         r += warps) {
+        float acc = 0.0f;
+        for (int v = lane; v < d; v += 32) {
+            const float a = __uint_as_float(uint32_t(o[r * d + v]) << 16);
+            const float b = __uint_as_float(uint32_t(dout[r * d + v]) << 16);
+            acc = __fmaf_rn(a, b, acc);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+        if (lane == 0) {
+            delta[r] = acc;
+            lse2[r] = __fmul_rn(lse[r], kLog2e);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- dK, dV
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const AttnBwdParams p)
+{
+    using C = BwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
+    uint8_t *sQ = smem;
+    uint8_t *sDO = sQ + C::TILE_BYTES;
+    uint8_t *sK = sDO + C::TILE_BYTES;
+    uint8_t *sV = sK + C::BLOCK_BYTES;
+    float *sLse = reinterpret_cast<float *>(sV + C::BLOCK_BYTES);
+    float *sDelta = sLse + kQTile;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sDelta + kQTile);
+    uint64_t *drain = bar + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    // block -> (sequence, kv head, key block)
+    const int nkb = p.num_key_blocks;
+    const int kb = blockIdx.x % nkb;
+    const int g = (blockIdx.x / nkb) % p.Hkv;
+    const int b = blockIdx.x / (nkb * p.Hkv);
+    const int q0 = p.cu_q[b], n = p.cu_q[b + 1] - q0, ctx = p.ctx_lens[b];
+    const int kv_len = ctx + n;
+    const int k0 = kb * kKeyBlock;
+    if (n <= 0 || k0 >= kv_len) return;
+    if (kv_len > p.max_pages * kPage) {  // the page table cannot hold the sequence
+        if (threadIdx.x == 0) record_status(p.status, BI_DEV_BAD_INDEX);
+        return;
+    }
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    const int32_t *bt = p.block_table + int64_t(b) * p.max_pages;
+    load_keys<D>(sK, static_cast<const uint8_t *>(p.k_cache), bt, k0, kv_len, p.Hkv, g,
+                 p.num_pages, p.status);
+    load_keys<D>(sV, static_cast<const uint8_t *>(p.v_cache), bt, k0, kv_len, p.Hkv, g,
+                 p.num_pages, p.status);
+    fence_proxy_async_smem();  // the key block is read by the tensor core
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
+    const uint32_t lane_base = tmem_addr(tmem, 32 * warp, 0);
+    const int key = k0 + 32 * warp + lane;  // this thread's key (TMEM lane)
+    const float cs = p.scale_log2;
+
+    const uint32_t idesc_s = idesc_bf16_f32(128, kQTile, 0, 0);
+    const uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
+    const uint32_t kb_addr = smem_u32(sK), vb_addr = smem_u32(sV);
+    const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
+    uint32_t phase = 0;
+    bool ok = true, first = true;
+    const int ntiles = (n + kQTile - 1) / kQTile;
+    for (int hh = 0; ok && hh < p.group; ++hh) {
+        const int h = g * p.group + hh;
+        for (int qt = 0; ok && qt < ntiles; ++qt) {
+            const int rows = min(kQTile, n - qt * kQTile);
+            const int pos0 = ctx + qt * kQTile;
+            if (pos0 + rows - 1 < k0) continue;  // no row of the tile sees this block
+            // ------------------------------------------------ load the tile
+            load_tile<D>(sQ, static_cast<const uint4 *>(p.q), q0 + int64_t(qt) * kQTile, rows,
+                         p.Hq, h);
+            load_tile<D>(sDO, static_cast<const uint4 *>(p.dout), q0 + int64_t(qt) * kQTile, rows,
+                         p.Hq, h);
+            {
+                const int r = threadIdx.x;
+                const int64_t row = (int64_t(q0) + qt * kQTile + r) * p.Hq + h;
+                sLse[r] = r < rows ? p.lse2[row] : 0.0f;
+                sDelta[r] = r < rows ? p.delta[row] : 0.0f;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            // ------------------------------------------------ S^T, dP^T
+            if (threadIdx.x == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    mma_ss(tmem + C::S_COL, sdesc_plain(kb_addr + 256 * k, 128, C::KGROUP_BYTES),
+                           sdesc_plain(q_addr + 4096 * k, 2048, 128), idesc_s, k > 0 ? 1u : 0u);
+                    mma_ss(tmem + C::DP_COL, sdesc_plain(vb_addr + 256 * k, 128, C::KGROUP_BYTES),
+                           sdesc_plain(do_addr + 4096 * k, 2048, 128), idesc_s, k > 0 ? 1u : 0u);
+                }
+                mma_commit(bar);
+            }
+            ok = block_wait(bar, phase, ctl);
+            phase ^= 1u;
+            if (!ok) break;
+            tc_fence_after();
+            // ------------------------------------------------ P^T, dS^T (row = key)
+#pragma unroll 1
+            for (int c = 0; c < kQTile / 32; ++c) {
+                uint32_t s[32], dp[32];
+                tmem_ld32(lane_base + C::S_COL + 32 * c, s);
+                tmem_ld32(lane_base + C::DP_COL + 32 * c, dp);
+                tmem_wait_ld(s);
+                tmem_wait_ld(dp);
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    float pv[2], dv[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int i = 32 * c + j + u;  // query column
+                        const bool vis = i < rows && key <= pos0 + i;
+                        const float pr = ex2(__fmaf_rn(__uint_as_float(s[j + u]), cs, -sLse[i]));
+                        const float ds = __fmul_rn(pr, __fsub_rn(__uint_as_float(dp[j + u]), sDelta[i]));
+                        pv[u] = vis ? pr : 0.0f;
+                        dv[u] = vis ? ds : 0.0f;
+                    }
+                    pk[j / 2] = pack2(pv[0], pv[1]);
+                    dk[j / 2] = pack2(dv[0], dv[1]);
+                }
+                tmem_st16(lane_base + C::S_COL + 16 * c, pk);
+                tmem_st16(lane_base + C::DP_COL + 16 * c, dk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncthreads();
+            // ------------------------------------------------ dV += P^T dO, dK += dS^T Q
+            if (threadIdx.x == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int jj = 0; jj < kQTile / 16; ++jj) {
+                    const uint32_t acc = (first && jj == 0) ? 0u : 1u;
+                    mma_ts(tmem + C::ACC0, tmem + C::S_COL + 8 * jj,
+                           sdesc_plain(do_addr + 256 * jj, 128, 2048), idesc_acc, acc);
+                    mma_ts(tmem + C::ACC1, tmem + C::DP_COL + 8 * jj,
+                           sdesc_plain(q_addr + 256 * jj, 128, 2048), idesc_acc, acc);
+                }
+                mma_commit(bar);
+            }
+            first = false;
+            ok = block_wait(bar, phase, ctl);
+            phase ^= 1u;
+            if (!ok) break;
+            tc_fence_after();
+        }
+    }
+    if (!ok) {
+        if (threadIdx.x == 0) {
+            mma_commit(drain);
+            drain_wait(drain, 0, p.timeout_ns);
+        }
+    } else {
+        // ---------------------------------------------------- write dV, dK
+        // The keys of this block in pages the sequence owns (slots past its
+        // length are zeros: their rows of P^T and dS^T were zero).
+        const int n_pages = (kv_len + kPage - 1) / kPage;
+        const int lp = key / kPage;
+        const bool mine = lp < n_pages;
+        int phys = -1;
+        if (mine) phys = __ldg(bt + lp);
+        const bool good = mine && phys >= 0 && phys < p.num_pages;
+        const int r = key % kPage;
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {
+            uint8_t *dst = static_cast<uint8_t *>(which ? p.dk : p.dv);
+            const float mul = which ? p.scale : 1.0f;
+            const uint32_t col = which ? C::ACC1 : C::ACC0;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t a[32];
+                tmem_ld32(lane_base + col + 32 * c, a);
+                tmem_wait_ld(a);
+                if (good) {
+                    uint8_t *blk = dst + (int64_t(phys) * p.Hkv + g) * int64_t(C::PAGE_BYTES);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 v;
+                        v.x = pack2(__fmul_rn(__uint_as_float(a[8 * q + 0]), mul),
+                                    __fmul_rn(__uint_as_float(a[8 * q + 1]), mul));
+                        v.y = pack2(__fmul_rn(__uint_as_float(a[8 * q + 2]), mul),
+                                    __fmul_rn(__uint_as_float(a[8 * q + 3]), mul));
+                        v.z = pack2(__fmul_rn(__uint_as_float(a[8 * q + 4]), mul),
+                                    __fmul_rn(__uint_as_float(a[8 * q + 5]), mul));
+                        v.w = pack2(__fmul_rn(__uint_as_float(a[8 * q + 6]), mul),
+                                    __fmul_rn(__uint_as_float(a[8 * q + 7]), mul));
+                        *reinterpret_cast<uint4 *>(blk + page_off<D>(r, 4 * c + q)) = v;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- dQ
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnBwdParams p)
+{
+    using C = BwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
+    uint8_t *sQ = smem;
+    uint8_t *sDO = sQ + C::TILE_BYTES;
+    uint8_t *sK = sDO + C::TILE_BYTES;
+    uint8_t *sV = sK + C::BLOCK_BYTES;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sV + C::BLOCK_BYTES + C::VEC_BYTES);
+    uint64_t *drain = bar + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    // block -> (sequence, query head, query tile)
+    const int nqt = p.num_q_tiles;
+    const int qt = blockIdx.x % nqt;
+    const int h = (blockIdx.x / nqt) % p.Hq;
+    const int b = blockIdx.x / (nqt * p.Hq);
+    const int q0 = p.cu_q[b], n = p.cu_q[b + 1] - q0, ctx = p.ctx_lens[b];
+    const int kv_len = ctx + n;
+    if (qt * kQTile >= n) return;
+    if (kv_len > p.max_pages * kPage) {
+        if (threadIdx.x == 0) record_status(p.status, BI_DEV_BAD_INDEX);
+        return;
+    }
+    const int rows = min(kQTile, n - qt * kQTile);
+    const int pos0 = ctx + qt * kQTile;
+    const int g = h / p.group;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    const int64_t row0 = int64_t(q0) + qt * kQTile;
+    load_tile<D>(sQ, static_cast<const uint4 *>(p.q), row0, rows, p.Hq, h);
+    load_tile<D>(sDO, static_cast<const uint4 *>(p.dout), row0, rows, p.Hq, h);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
+    const uint32_t lane_base = tmem_addr(tmem, 32 * warp, 0);
+    const int i = 32 * warp + lane;  // this thread's query row (TMEM lane)
+    const bool row_ok = i < rows;
+    const int t = pos0 + i;          // its absolute position
+    const float lse2 = row_ok ? p.lse2[(row0 + i) * p.Hq + h] : 0.0f;
+    const float delta = row_ok ? p.delta[(row0 + i) * p.Hq + h] : 0.0f;
+    const float cs = p.scale_log2;
+    const int32_t *bt = p.block_table + int64_t(b) * p.max_pages;
+
+    const uint32_t idesc_s = idesc_bf16_f32(128, kKeyBlock, 0, 0);
+    const uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
+    const uint32_t kb_addr = smem_u32(sK), vb_addr = smem_u32(sV);
+    const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
+    uint32_t phase = 0;
+    bool ok = true;
+    const int last_key = pos0 + rows - 1;  // the tile's last visible key
+    for (int kb = 0; ok && kb * kKeyBlock <= last_key; ++kb) {
+        const int k0 = kb * kKeyBlock;
+        // the previous block's dQ MMAs have completed (waited below)
+        load_keys<D>(sK, static_cast<const uint8_t *>(p.k_cache), bt, k0, kv_len, p.Hkv, g,
+                     p.num_pages, p.status);
+        load_keys<D>(sV, static_cast<const uint8_t *>(p.v_cache), bt, k0, kv_len, p.Hkv, g,
+                     p.num_pages, p.status);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                mma_ss(tmem + C::S_COL, sdesc_plain(q_addr + 4096 * k, 2048, 128),
+                       sdesc_plain(kb_addr + 256 * k, 128, C::KGROUP_BYTES), idesc_s, k > 0 ? 1u : 0u);
+                mma_ss(tmem + C::DP_COL, sdesc_plain(do_addr + 4096 * k, 2048, 128),
+                       sdesc_plain(vb_addr + 256 * k, 128, C::KGROUP_BYTES), idesc_s, k > 0 ? 1u : 0u);
+            }
+            mma_commit(bar);
+        }
+        ok = block_wait(bar, phase, ctl);
+        phase ^= 1u;
+        if (!ok) break;
+        tc_fence_after();
+        // ---------------------------------------------------- dS (row = query)
+#pragma unroll 1
+        for (int c = 0; c < kKeyBlock / 32; ++c) {
+            uint32_t s[32], dp[32];
+            tmem_ld32(lane_base + C::S_COL + 32 * c, s);
+            tmem_ld32(lane_base + C::DP_COL + 32 * c, dp);
+            tmem_wait_ld(s);
+            tmem_wait_ld(dp);
+            uint32_t dk[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                float dv[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int key = k0 + 32 * c + j + u;
+                    const bool vis = row_ok && key <= t;
+                    const float pr = ex2(__fmaf_rn(__uint_as_float(s[j + u]), cs, -lse2));
+                    const float ds = __fmul_rn(pr, __fsub_rn(__uint_as_float(dp[j + u]), delta));
+                    dv[u] = vis ? ds : 0.0f;
+                }
+                dk[j / 2] = pack2(dv[0], dv[1]);
+            }
+            tmem_st16(lane_base + C::S_COL + 16 * c, dk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        // ---------------------------------------------------- dQ += dS K
+        if (threadIdx.x == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int jj = 0; jj < kKeyBlock / 16; ++jj)
+                mma_ts(tmem + C::ACC0, tmem + C::S_COL + 8 * jj,
+                       sdesc_plain(kb_addr + jj * C::PAGE_BYTES, C::KGROUP_BYTES, 128), idesc_acc,
+                       (kb > 0 || jj > 0) ? 1u : 0u);
+            mma_commit(bar);
+        }
+        ok = block_wait(bar, phase, ctl);
+        phase ^= 1u;
+        if (!ok) break;
+        tc_fence_after();
+    }
+    if (!ok) {
+        if (threadIdx.x == 0) {
+            mma_commit(drain);
+            drain_wait(drain, 0, p.timeout_ns);
+        }
+    } else {
+        // every thread takes part in the warp's TMEM loads; rows past the
+        // chunk store nothing
+        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dq) + ((row0 + i) * p.Hq + h) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t a[32];
+            tmem_ld32(lane_base + C::ACC0 + 32 * c, a);
+            tmem_wait_ld(a);
+            if (!row_ok) continue;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint4 v;
+                v.x = pack2(__fmul_rn(__uint_as_float(a[8 * q + 0]), p.scale),
+                            __fmul_rn(__uint_as_float(a[8 * q + 1]), p.scale));
+                v.y = pack2(__fmul_rn(__uint_as_float(a[8 * q + 2]), p.scale),
+                            __fmul_rn(__uint_as_float(a[8 * q + 3]), p.scale));
+                v.z = pack2(__fmul_rn(__uint_as_float(a[8 * q + 4]), p.scale),
+                            __fmul_rn(__uint_as_float(a[8 * q + 5]), p.scale));
+                v.w = pack2(__fmul_rn(__uint_as_float(a[8 * q + 6]), p.scale),
+                            __fmul_rn(__uint_as_float(a[8 * q + 7]), p.scale));
+                reinterpret_cast<uint4 *>(dst + 32 * c)[q] = v;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+size_t attn_bwd_ws_bytes(int64_t rows) { return size_t(rows) * 2 * sizeof(float); }
+
+cudaError_t launch_attention_backward(const AttnBwdParams &p_in, int head_dim, int64_t rows,
+                                      int num_sms, cudaStream_t s)
+{
+    AttnBwdParams p = p_in;
+    // Delta and lse2 of every (token, head) row, in the workspace
+    {
+        const int64_t blocks = (rows + 7) / 8, cap = int64_t(num_sms) * 16;
+        attn_bwd_prep_kernel<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, s>>>(
+            static_cast<const uint16_t *>(p.o), static_cast<const uint16_t *>(p.dout), p.lse, rows,
+            head_dim, p.lse2, p.delta);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t dkv_blocks = int64_t(p.B) * p.Hkv * p.num_key_blocks;
+    const int64_t dq_blocks = int64_t(p.B) * p.Hq * p.num_q_tiles;
+    if (dkv_blocks > INT32_MAX || dq_blocks > INT32_MAX) return cudaErrorInvalidValue;
+    cudaError_t e;
+    if (head_dim == 128) {
+        using C = BwdCfg<128>;
+        if ((e = cudaFuncSetAttribute(attn_bwd_dkv_kernel<128>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(attn_bwd_dq_kernel<128>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM)) != cudaSuccess)
+            return e;
+        attn_bwd_dkv_kernel<128><<<unsigned(dkv_blocks), kBwdThreads, C::SMEM, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        attn_bwd_dq_kernel<128><<<unsigned(dq_blocks), kBwdThreads, C::SMEM, s>>>(p);
+    } else {
+        using C = BwdCfg<64>;
+        if ((e = cudaFuncSetAttribute(attn_bwd_dkv_kernel<64>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(attn_bwd_dq_kernel<64>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM)) != cudaSuccess)
+            return e;
+        attn_bwd_dkv_kernel<64><<<unsigned(dkv_blocks), kBwdThreads, C::SMEM, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        attn_bwd_dq_kernel<64><<<unsigned(dq_blocks), kBwdThreads, C::SMEM, s>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace bi

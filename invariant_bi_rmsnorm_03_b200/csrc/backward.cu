@@ -11,6 +11,9 @@
 //   matmul    through the invariant GEMM: dA = dC W as dC (W^T)^T and
 //             dW = dC^T A as (dC^T) (A^T)^T, the transposes made by
 //             transpose_kernel (bit copies).
+//   SwiGLU    elementwise: each gradient from its own (gate, up, dout) only.
+//   RoPE      elementwise per pair: the rotation by the negative angle, with
+//             the forward's angles (double precision, rounded to float).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -189,6 +192,124 @@ __global__ void transpose_kernel(const uint16_t *__restrict__ a, uint16_t *__res
     }
 }
 
+// ---------------------------------------------------------------- SwiGLU
+// With s = 1 / (1 + e^-g) (the sigmoid), out = g s u:
+//   dup   = dout (g s)
+//   dgate = (dout u) (s + (g s) s'),   s' = 1 / (1 + e^g) = 1 - s
+// s' is evaluated as its own sigmoid rather than as 1 - s, which loses the
+// small values of 1 - s for large g; neither form overflows to NaN.  fp32,
+// every operation rounded; one thread per 8 outputs of each half.
+template <bool OUT_F32>
+__global__ void swiglu_bwd_kernel(const uint4 *__restrict__ gu, const uint4 *__restrict__ dout,
+                                  void *__restrict__ dgu, int64_t T, int64_t fp)
+{
+    const int64_t n = T * fp;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t t = i / fp;
+        const int64_t c = i - t * fp;
+        const uint4 g4 = __ldcs(gu + t * 2 * fp + c);
+        const uint4 u4 = __ldcs(gu + t * 2 * fp + fp + c);
+        const uint4 d4 = __ldcs(dout + i);
+        const uint32_t gv[4] = {g4.x, g4.y, g4.z, g4.w};
+        const uint32_t uv[4] = {u4.x, u4.y, u4.z, u4.w};
+        const uint32_t dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        float dg[8], du[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float g = (k & 1) ? hi_f(gv[k >> 1]) : lo_f(gv[k >> 1]);
+            const float u = (k & 1) ? hi_f(uv[k >> 1]) : lo_f(uv[k >> 1]);
+            const float d = (k & 1) ? hi_f(dv[k >> 1]) : lo_f(dv[k >> 1]);
+            const float s = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-g)));
+            const float sc = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(g)));
+            const float gs = __fmul_rn(g, s);
+            du[k] = __fmul_rn(d, gs);
+            dg[k] = __fmul_rn(__fmul_rn(d, u), __fadd_rn(s, __fmul_rn(gs, sc)));
+        }
+        const int64_t og = t * 2 * fp + c, ou = og + fp;  // 8-value pieces of dgate, dup
+        if constexpr (OUT_F32) {
+            float4 *o = static_cast<float4 *>(dgu);
+            o[2 * og] = make_float4(dg[0], dg[1], dg[2], dg[3]);
+            o[2 * og + 1] = make_float4(dg[4], dg[5], dg[6], dg[7]);
+            o[2 * ou] = make_float4(du[0], du[1], du[2], du[3]);
+            o[2 * ou + 1] = make_float4(du[4], du[5], du[6], du[7]);
+        } else {
+            uint4 *o = static_cast<uint4 *>(dgu);
+            o[og] = make_uint4(pack_rn(dg[0], dg[1]), pack_rn(dg[2], dg[3]), pack_rn(dg[4], dg[5]),
+                               pack_rn(dg[6], dg[7]));
+            o[ou] = make_uint4(pack_rn(du[0], du[1]), pack_rn(du[2], du[3]), pack_rn(du[4], du[5]),
+                               pack_rn(du[6], du[7]));
+        }
+    }
+}
+
+// ---------------------------------------------------------------- RoPE
+// The forward rotates the pair (x_i, x_{i+d/2}) by the angle
+// a_i = pos theta^(-2i/d); its transpose rotates the upstream gradient back:
+//   dx_i       = round(round(dy_i cos) + round(dy_{i+d/2} sin))
+//   dx_{i+d/2} = round(round(dy_{i+d/2} cos) - round(dy_i sin))
+// with cos and sin evaluated in double precision and rounded to float, as
+// the forward does.  One block per token (grid-stride); each thread rotates
+// a pair of 8-value pieces of one head.  dy and dx rows are ld_dy / ld_dx
+// values apart (a head set inside a wider row, e.g. the q part of a fused
+// q/k/v gradient).
+constexpr int kRopeBwdThreads = 256;
+
+template <bool OUT_F32>
+__global__ void __launch_bounds__(kRopeBwdThreads)
+rope_bwd_kernel(const uint16_t *__restrict__ dy, int64_t ld_dy, const int32_t *__restrict__ pos,
+                void *__restrict__ dx, int64_t ld_dx, int64_t T, int nh, int d, double theta)
+{
+    __shared__ float cs[64], sn[64];
+    const int half = d / 2, hp = half / 8;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        const int32_t p = __ldg(pos + t);
+        __syncthreads();  // the previous token's angles are no longer read
+        if (threadIdx.x < half) {
+            const double inv = pow(theta, -2.0 * double(threadIdx.x) / double(d));
+            double sv, cv;
+            sincos(double(p) * inv, &sv, &cv);
+            cs[threadIdx.x] = static_cast<float>(cv);
+            sn[threadIdx.x] = static_cast<float>(sv);
+        }
+        __syncthreads();
+        for (int it = threadIdx.x; it < nh * hp; it += blockDim.x) {
+            const int h = it / hp, c = it - h * hp;
+            const uint16_t *row = dy + t * ld_dy + int64_t(h) * d;
+            const uint4 a = *reinterpret_cast<const uint4 *>(row + 8 * c);
+            const uint4 b = *reinterpret_cast<const uint4 *>(row + half + 8 * c);
+            const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+            float lo[8], hi[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int i = 8 * c + k;
+                const float l = (k & 1) ? hi_f(av[k >> 1]) : lo_f(av[k >> 1]);
+                const float u = (k & 1) ? hi_f(bv[k >> 1]) : lo_f(bv[k >> 1]);
+                lo[k] = __fadd_rn(__fmul_rn(l, cs[i]), __fmul_rn(u, sn[i]));
+                hi[k] = __fsub_rn(__fmul_rn(u, cs[i]), __fmul_rn(l, sn[i]));
+            }
+            const int64_t o = t * ld_dx + int64_t(h) * d;
+            if constexpr (OUT_F32) {
+                float *orow = static_cast<float *>(dx) + o;
+                float4 *ol = reinterpret_cast<float4 *>(orow + 8 * c);
+                float4 *oh = reinterpret_cast<float4 *>(orow + half + 8 * c);
+                ol[0] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+                ol[1] = make_float4(lo[4], lo[5], lo[6], lo[7]);
+                oh[0] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+                oh[1] = make_float4(hi[4], hi[5], hi[6], hi[7]);
+            } else {
+                uint16_t *orow = static_cast<uint16_t *>(dx) + o;
+                *reinterpret_cast<uint4 *>(orow + 8 * c) =
+                    make_uint4(pack_rn(lo[0], lo[1]), pack_rn(lo[2], lo[3]), pack_rn(lo[4], lo[5]),
+                               pack_rn(lo[6], lo[7]));
+                *reinterpret_cast<uint4 *>(orow + half + 8 * c) =
+                    make_uint4(pack_rn(hi[0], hi[1]), pack_rn(hi[2], hi[3]), pack_rn(hi[4], hi[5]),
+                               pack_rn(hi[6], hi[7]));
+            }
+        }
+    }
+}
+
 }  // namespace
 
 size_t rmsnorm_backward_ws_bytes(int64_t M, int64_t H)
@@ -232,6 +353,36 @@ cudaError_t launch_transpose(const void *a, void *out, int64_t R, int64_t C, int
     const int64_t cap = int64_t(num_sms) * 16;
     transpose_kernel<<<static_cast<unsigned>(tiles < cap ? tiles : cap), dim3(32, 8), 0, s>>>(
         static_cast<const uint16_t *>(a), static_cast<uint16_t *>(out), R, C, ld_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu_backward(const void *gu, const void *dout, void *dgu, int64_t T,
+                                   int64_t F, bool out_f32, int num_sms, cudaStream_t s)
+{
+    const int64_t fp = F / 8, items = T * fp;
+    const int64_t blocks = (items + 255) / 256, cap = int64_t(num_sms) * 8;
+    const unsigned g = static_cast<unsigned>(blocks < cap ? blocks : cap);
+    const uint4 *a = static_cast<const uint4 *>(gu), *b = static_cast<const uint4 *>(dout);
+    if (out_f32)
+        swiglu_bwd_kernel<true><<<g, 256, 0, s>>>(a, b, dgu, T, fp);
+    else
+        swiglu_bwd_kernel<false><<<g, 256, 0, s>>>(a, b, dgu, T, fp);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rope_backward(const void *dy, int64_t ld_dy, const int32_t *pos, void *dx,
+                                 int64_t ld_dx, int64_t T, int nh, int d, double theta,
+                                 bool out_f32, int num_sms, cudaStream_t s)
+{
+    const int64_t cap = int64_t(num_sms) * 8;
+    const unsigned g = static_cast<unsigned>(T < cap ? T : cap);
+    const uint16_t *src = static_cast<const uint16_t *>(dy);
+    if (out_f32)
+        rope_bwd_kernel<true><<<g, kRopeBwdThreads, 0, s>>>(src, ld_dy, pos, dx, ld_dx, T, nh, d,
+                                                              theta);
+    else
+        rope_bwd_kernel<false><<<g, kRopeBwdThreads, 0, s>>>(src, ld_dy, pos, dx, ld_dx, T, nh, d,
+                                                               theta);
     return cudaGetLastError();
 }
 

@@ -17,6 +17,10 @@ cudaError_t launch_rmsnorm(const void *x, const void *w, void *y, int64_t M, int
 // x <- round(x + delta); y <- RMSNorm(x) exactly as launch_rmsnorm computes it
 cudaError_t launch_add_rmsnorm(void *x, const void *delta, const void *w, void *y, int64_t M,
                                int64_t H, float eps, bool out_f32, int num_sms, cudaStream_t s);
+// r[m] = rsqrt(sum_k x[m, k]^2 / H + eps): launch_rmsnorm's reduction of the
+// row (the same order, the same bits as its rstd), with nothing else written
+cudaError_t launch_row_rstd(const void *x, float *r, int64_t M, int64_t H, float eps, int num_sms,
+                            cudaStream_t s);
 
 // ---------------------------------------------------------------- matmul
 constexpr int kGemmBK = 64;  // K slice; the output tile is 256 x 256 per SM pair
@@ -35,7 +39,8 @@ cudaError_t launch_gemm_grouped(const CUtensorMap &ta, const CUtensorMap &tw, vo
                                 int num_sms, unsigned *status, uint64_t timeout_ns,
                                 cudaStream_t s);
 // Fused epilogues of the plain product (never split along K):
-//   norm:     C[m, :] = round(rsqrt(mean_k A[m, k]^2 + eps) * acc[m, :])
+//   norm:     C[m, :] = round(rs[m] * acc[m, :]), rs[m] = rsqrt(mean_k A[m, k]^2 + eps)
+//             from launch_row_rstd
 //   residual: C[m, :] = round(R[m, :] + round(acc[m, :]))   (R may be C)
 //   QKV (rope non-null): the N = (Hq + 2 Hkv) head_dim columns of the
 //             rounded product are q, k and v heads; q and k are rotated by
@@ -43,8 +48,7 @@ cudaError_t launch_gemm_grouped(const CUtensorMap &ta, const CUtensorMap &tw, vo
 //             and q goes to q_out [M, Hq, head_dim], k and v to the row's
 //             cache slot; C is not written.
 struct GemmEpi {
-    int norm;
-    float eps;
+    const float *rs;        // [M] row scales (norm form) or null
     const void *residual;
     const float *rope;      // [max_pos, head_dim / 2, 2]: cos, sin
     int max_pos;
@@ -72,6 +76,14 @@ cudaError_t launch_rmsnorm_backward(const void *x, const void *w, const void *dy
 // out[c, r] = a[r, c] (bf16), rows of out padded with zeros to ld_out >= R
 cudaError_t launch_transpose(const void *a, void *out, int64_t R, int64_t C, int64_t ld_out,
                              int num_sms, cudaStream_t s);
+// dgu [T, 2F] = [dgate | dup] of out = silu(gate) * up for the upstream dout [T, F]
+cudaError_t launch_swiglu_backward(const void *gu, const void *dout, void *dgu, int64_t T,
+                                   int64_t F, bool out_f32, int num_sms, cudaStream_t s);
+// dx = the transpose of the rotary rotation applied to dy ([T, nh, d] heads,
+// rows ld_dy / ld_dx values apart)
+cudaError_t launch_rope_backward(const void *dy, int64_t ld_dy, const int32_t *pos, void *dx,
+                                 int64_t ld_dx, int64_t T, int nh, int d, double theta,
+                                 bool out_f32, int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- KV write
 cudaError_t launch_kv_write(void *k_cache, void *v_cache, int64_t num_pages, int Hkv, int d,
@@ -116,6 +128,35 @@ cudaError_t launch_attention(const CUtensorMap &tq, const AttnParams &p, int hea
                              cudaStream_t s);
 cudaError_t launch_attn_combine(const AttnParams &p, int head_dim, cudaStream_t s);
 cudaError_t launch_attn_order(const int32_t *seq_lens, int B, int32_t *order, cudaStream_t s);
+
+// ---------------------------------------------------------------- attention backward
+struct AttnBwdParams {
+    const void *k_cache;
+    const void *v_cache;
+    const int32_t *block_table;
+    int32_t max_pages;
+    int32_t num_pages;
+    int32_t Hkv;
+    int32_t Hq;
+    int32_t group;             // Hq / Hkv
+    int32_t B;
+    const int32_t *cu_q;       // [B + 1]
+    const int32_t *ctx_lens;   // [B]
+    int32_t num_q_tiles;       // 128-row tiles of the longest chunk
+    int32_t num_key_blocks;    // 128-key blocks of the longest sequence
+    float scale;               // softmax scale
+    float scale_log2;          // scale * log2(e)
+    const void *q, *o, *dout;  // [T, Hq, d] bf16
+    const float *lse;          // [T, Hq] natural log
+    float *lse2, *delta;       // workspace [T, Hq] each
+    void *dq;                  // [T, Hq, d] bf16
+    void *dk, *dv;             // cache-shaped bf16
+    unsigned *status;
+    uint64_t timeout_ns;
+};
+size_t attn_bwd_ws_bytes(int64_t rows);
+cudaError_t launch_attention_backward(const AttnBwdParams &p, int head_dim, int64_t rows,
+                                      int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- decoder glue
 cudaError_t launch_embedding(const void *table, int64_t V, int64_t H, const int32_t *ids,

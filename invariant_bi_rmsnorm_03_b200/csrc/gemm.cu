@@ -28,19 +28,14 @@
 //
 // Fused forms (the RMSNorm and residual steps around a transformer block's
 // matmuls, adjacent to the matmul item of xitu-tech news, "构建确定性解决方案"):
-//   norm      C[m, :] = rsqrt(mean_k A[m, k]^2 + eps) * (A W^T)[m, :], with the
-//             norm weight folded into W beforehand.  Four more warps (6-9)
-//             per CTA read each A slice of their CTA as soon as it lands,
-//             while the MMAs run, adding the squares of their row (one row
-//             per thread, K ascending, eight fixed partial sums); a stage is
-//             refilled only after they have read it, and the epilogue scales
-//             its row by the resulting rsqrt.  No second pass over A, and the
-//             MMA operands are the stored bf16 values.  The peer's A slice
-//             completes on a barrier of its own, so that its norm warps can
-//             see it; the peer's otherwise idle MMA warp forwards each
-//             completion to the leader's barrier with a relaxed arrive (a
-//             release arrive across the pair stalls the arriving thread for
-//             about a microsecond, which would throttle the pipeline).
+//   norm      C[m, :] = r[m] * (A W^T)[m, :], r[m] = rsqrt(mean_k A[m, k]^2 +
+//             eps) computed beforehand by the RMSNorm kernel's own reduction
+//             (one read of A, M floats written), with the norm weight folded
+//             into W beforehand: the epilogue scales its row by r[m].  The MMA
+//             operands are the stored bf16 values, and A is not read again
+//             from shared memory for the statistics (which, done once per
+//             output tile, took shared-memory bandwidth the tensor cores
+//             need).
 //   residual  C[m, :] = round(R[m, :] + round(acc[m, :])), R read in the
 //             epilogue (it may be C itself).
 //   QKV       the columns are q, k and v heads: the rounded product goes
@@ -265,13 +260,10 @@ constexpr int A_BYTES = 128 * BK * 2;   // 16 KB: this CTA's half of the A slice
 constexpr int W_BYTES = 128 * BK * 2;   // 16 KB: this CTA's half of the W slice
 constexpr int STAGE_BYTES = A_BYTES + W_BYTES;
 constexpr int THREADS = 192;
-constexpr int FUSED_THREADS = 320;      // + warps 6-9: the row sums of squares (norm form)
 constexpr uint32_t TMEM_COLS = 512;     // two 128-lane x 256-column fp32 accumulators
 constexpr int BAR_BYTES = 256;
-constexpr int CUM_BYTES = (kMaxGemmGroups + 1) * 4;  // grouped mode: tiles before each group;
-                                                    // norm form: two 128-row rsqrt buffers
-static_assert(CUM_BYTES >= 2 * 128 * 4, "the rsqrt buffers share the group table's room");
-static_assert((3 * STAGES + 9) * 8 + 8 <= BAR_BYTES, "barriers, TMEM address and abort flag");
+constexpr int CUM_BYTES = (kMaxGemmGroups + 1) * 4;  // grouped mode: tiles before each group
+static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barriers, TMEM address and abort flag");
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + CUM_BYTES;
 
 // The tile of work unit u.  Plain: tiles m-fastest over an M x N output
@@ -309,7 +301,7 @@ __device__ __forceinline__ Unit unit_at(int u, int num_m, int num_n, int k_split
 }
 
 template <bool FUSED>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FUSED ? FUSED_THREADS : THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmw,
                      void *c, float *__restrict__ ws, int M, int N, int K, int out_f32,
                      int k_splits, const int64_t *__restrict__ goff, int groups, GemmEpi epi,
@@ -319,7 +311,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FUSED ? FUSED_THREAD
     k_splits = 1;  // the invariant build never splits K
 #endif
     // fused forms: plain tiles only (no groups, no split K)
-    const bool nrm = FUSED && epi.norm;
+    const float *row_scale = FUSED ? epi.rs : nullptr;
     const void *res = FUSED ? epi.residual : nullptr;
     if (FUSED) {
         k_splits = 1;
@@ -335,13 +327,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FUSED ? FUSED_THREAD
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 2;   // leader's used: 8 arrivals (4 epilogue warps x 2 CTAs)
     uint64_t *drain = tempty + 2;
-    uint64_t *afull = drain + 1;       // norm form, peer: its own A slice landed
-    uint64_t *rfull = afull + STAGES;  // norm form: rsqrt buffer written (4 norm warps)
-    uint64_t *rempty = rfull + 2;      // norm form: rsqrt buffer read (4 epilogue warps)
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(rempty + 2);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
     int *cum = reinterpret_cast<int *>(smem + STAGES * STAGE_BYTES + BAR_BYTES);
-    float *rsq = reinterpret_cast<float *>(cum);  // norm form: [2][128]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -360,17 +348,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FUSED ? FUSED_THREAD
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            // norm form: the leader's full also counts the peer's forward, and a
-            // stage is free once the MMAs and the 4 norm warps have read it
-            mbar_init(&full[s], nrm ? 2 : 1);
-            mbar_init(&empty[s], nrm ? 5 : 1);
-            mbar_init(&afull[s], 1);
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
             mbar_init(&tempty[a], 8);
-            mbar_init(&rfull[a], 4);
-            mbar_init(&rempty[a], 4);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -409,16 +392,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FUSED ? FUSED_THREAD
                         break;
                     }
                     const uint32_t bar = map_to_cta(smem_u32(&full[stage]), 0);
-                    // norm form: the peer's A slice completes on its own barrier
-                    uint32_t abar = bar;
-                    if (leader) {
-                        mbar_arrive_expect_tx(&full[stage],
-                                              nrm ? 2 * STAGE_BYTES - A_BYTES : 2 * STAGE_BYTES);
-                    } else if (nrm) {
-                        mbar_arrive_expect_tx(&afull[stage], A_BYTES);
-                        abar = map_to_cta(smem_u32(&afull[stage]), rank);
-                    }
-                    tma_load_2d_pair(sA + stage * A_BYTES, &tma, abar, kb * BK,
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+                    tma_load_2d_pair(sA + stage * A_BYTES, &tma, bar, kb * BK,
                                      int(t.row0) + int(rank) * 128);
                     tma_load_2d_pair(sW + stage * W_BYTES, &tmw, bar, kb * BK,
                                      int(t.w_row0) + int(rank) * 128);
@@ -430,28 +405,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FUSED ? FUSED_THREAD
             }
         }
     } else if (warp == 1) {
-        if (nrm && lane == 0 && !leader) {
-            // ------------------------------------ norm form, peer: forward
-            // each landed A slice of this CTA to the leader's full barrier
-            const uint32_t full_leader = map_to_cta(smem_u32(&full[0]), 0);
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int u = pair_id; ok && u < units; u += num_pairs) {
-                const Unit t = unit(u);
-                for (int kb = t.kb0; kb < t.kb1; ++kb) {
-                    if (!wait(&afull[stage], phase, ctl)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_relaxed_cluster(full_leader + 8u * uint32_t(stage));
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-            }
-        }
         if (lane == 0 && leader) {
             // ------------------------------------------------ MMA issue (leader)
             const uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
@@ -524,13 +477,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FUSED ? FUSED_THREAD
             }
             if (!wait(&tfull[acc], acc_phase, ctl)) break;
             tc_fence_after();
-            float rscale = 1.0f;
-            if (nrm) {
-                if (!wait(&rfull[acc], acc_phase, ctl)) break;
-                rscale = rsq[acc * 128 + 32 * q + lane];
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&rempty[acc]);
-            }
+            // norm form: this row's rsqrt (computed before the launch)
+            const float rscale = (row_scale && row_ok) ? __ldg(row_scale + row) : 1.0f;
             if (FUSED && epi.rope) {
                 qkv_epilogue(epi, tmem_addr(tmem, 32 * q, acc * BN), t.nb, row, row_ok, rscale, N,
                              status);
@@ -543,7 +491,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FUSED ? FUSED_THREAD
                 uint32_t r[32];
                 tmem_ld32(tmem_addr(tmem, 32 * q, acc * BN + cc * 32), r);
                 tmem_wait_ld(r);
-                if (nrm) {
+                if (row_scale) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         r[j] = __float_as_uint(__fmul_rn(__uint_as_float(r[j]), rscale));
@@ -566,59 +514,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FUSED ? FUSED_THREAD
             if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
-        }
-    } else if (nrm) {
-        // ---------------------------------------- norm form: row sums of squares
-        // Thread i owns row i of this CTA's 128.  An A slice row is 128
-        // bytes, its 16-byte piece p stored at p ^ (i % 8) (128-byte
-        // swizzle); squares are added K-ascending into eight partial sums,
-        // one per position within a piece.
-        const int i = 32 * (warp & 3) + lane;
-        uint64_t *ready = leader ? full : afull;
-        int stage = 0;
-        uint32_t phase = 0;
-        int buf = 0;
-        uint32_t buf_phase = 0;
-        bool ok = true;
-        for (int u = pair_id; ok && u < units; u += num_pairs) {
-            const Unit t = unit(u);
-            float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            for (int kb = t.kb0; kb < t.kb1; ++kb) {
-                if (!wait(&ready[stage], phase, ctl)) {
-                    ok = false;
-                    break;
-                }
-                const uint8_t *rowp = sA + stage * A_BYTES + i * 128;
-#pragma unroll
-                for (int p = 0; p < 8; ++p) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(rowp + ((p ^ (i & 7)) << 4));
-                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float lo = __uint_as_float(w4[j] << 16);
-                        const float hi = __uint_as_float(w4[j] & 0xFFFF0000u);
-                        part[2 * j] = __fmaf_rn(lo, lo, part[2 * j]);
-                        part[2 * j + 1] = __fmaf_rn(hi, hi, part[2 * j + 1]);
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[stage]);
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-            if (!ok) break;
-            const float ss = __fadd_rn(
-                __fadd_rn(__fadd_rn(part[0], part[1]), __fadd_rn(part[2], part[3])),
-                __fadd_rn(__fadd_rn(part[4], part[5]), __fadd_rn(part[6], part[7])));
-            const float r = rsqrtf(__fadd_rn(__fdiv_rn(ss, float(K)), epi.eps));
-            if (!wait(&rempty[buf], buf_phase ^ 1u, ctl)) break;
-            rsq[buf * 128 + i] = r;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&rfull[buf]);
-            buf ^= 1;
-            if (buf == 0) buf_phase ^= 1u;
         }
     }
 
@@ -667,16 +562,30 @@ int gemm_k_splits(int64_t M, int64_t N, int64_t K, int num_sms)
     (void)M, (void)N, (void)K, (void)num_sms;
     return 1;
 #else
-    // Variant-off: split K when the tiles cannot fill the GPU.
+    // Variant-off: split K when the tiles cannot fill the GPU, with the
+    // count that minimises a simple time model: the K slices the busiest
+    // pair walks (waves x slices per split, ~0.6 us a slice, measured on a
+    // B200 at M = 256) plus one pass of the fp32 partial sums out to memory
+    // and back (~6.5 TB/s).
     const int64_t tiles = ((M + pair::BM - 1) / pair::BM) * ((N + pair::BN - 1) / pair::BN);
     const int64_t kblocks = (K + pair::BK - 1) / pair::BK;
     const int64_t pairs = num_sms / 2;
-    if (tiles >= pairs || kblocks < 8) return 1;
-    int64_t ks = pairs / tiles;
-    if (ks > kblocks / 4) ks = kblocks / 4;
-    if (ks < 2) return 1;
-    const int64_t per = (kblocks + ks - 1) / ks;
-    return static_cast<int>((kblocks + per - 1) / per);
+    if (tiles >= pairs || kblocks < 8 || pairs < 1) return 1;
+    const double slice_us = 0.6, bytes_per_us = 6.5e6;
+    int64_t best = 1;
+    double best_us = double(kblocks) * slice_us;  // one wave of whole-K tiles
+    for (int64_t ks = 2; ks <= 16 && ks <= kblocks / 4; ++ks) {
+        const int64_t per = (kblocks + ks - 1) / ks;
+        const int64_t splits = (kblocks + per - 1) / per;
+        const int64_t waves = (tiles * splits + pairs - 1) / pairs;
+        const double us = double(waves * per) * slice_us +
+                          2.0 * double(splits) * double(M) * double(N) * 4.0 / bytes_per_us;
+        if (us < best_us) {
+            best = splits;
+            best_us = us;
+        }
+    }
+    return static_cast<int>(best);
 #endif
 }
 
@@ -763,9 +672,7 @@ cudaError_t launch_gemm_fused(const CUtensorMap &ta, const CUtensorMap &tw, void
     if (e != cudaSuccess) return e;
     const int64_t units = int64_t((M + pair::BM - 1) / pair::BM) * ((N + pair::BN - 1) / pair::BN);
     const int pairs = static_cast<int>(units < max_pairs ? units : max_pairs);
-    // the norm warps exist only in the norm form
-    const int threads = epi.norm ? pair::FUSED_THREADS : pair::THREADS;
-    pair::gemm_pair_kernel<true><<<2 * pairs, threads, pair::SMEM_BYTES, s>>>(
+    pair::gemm_pair_kernel<true><<<2 * pairs, pair::THREADS, pair::SMEM_BYTES, s>>>(
         ta, tw, c, nullptr, M, N, K, out_f32 ? 1 : 0, 1, nullptr, 0, epi, status, timeout_ns);
     return cudaGetLastError();
 }

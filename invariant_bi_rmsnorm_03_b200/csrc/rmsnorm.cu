@@ -107,7 +107,8 @@ __device__ __forceinline__ uint4 add8(const uint4 &a, const uint4 &b)
 // One row per block iteration; the grid strides over rows.
 // ADD: the residual form -- x is first replaced by round(x + delta) (and
 // written back), then normalised exactly as the plain form normalises it.
-template <int ITEMS, bool OUT_F32, int MAXT, bool ADD, int MINB>
+// STATS: only the row's rstd is written, to ((float *) y)[row].
+template <int ITEMS, bool OUT_F32, int MAXT, bool ADD, int MINB, bool STATS = false>
 __global__ void __launch_bounds__(MAXT, MINB) rmsnorm_kernel(uint4 *x,
                                                        const uint4 *__restrict__ delta,
                                                        const uint4 *__restrict__ w,
@@ -151,10 +152,14 @@ __global__ void __launch_bounds__(MAXT, MINB) rmsnorm_kernel(uint4 *x,
         float tot = 0.0f;
         for (int i = 0; i < (T >> 5); ++i) tot = __fadd_rn(tot, part[i]);
         const float rstd = rsqrtf(__fadd_rn(__fdiv_rn(tot, h_den), eps));
+        if constexpr (STATS) {
+            if (threadIdx.x == 0) static_cast<float *>(y)[row] = rstd;
+        } else {
 #pragma unroll
-        for (int it = 0; it < ITEMS; ++it) {
-            const int c = threadIdx.x + it * T;
-            if (c < chunks) store8<OUT_F32>(y, row * chunks + c, v[it], __ldg(w + c), rstd);
+            for (int it = 0; it < ITEMS; ++it) {
+                const int c = threadIdx.x + it * T;
+                if (c < chunks) store8<OUT_F32>(y, row * chunks + c, v[it], __ldg(w + c), rstd);
+            }
         }
         __syncthreads();  // part[] is reused by the next row
     }
@@ -163,6 +168,7 @@ __global__ void __launch_bounds__(MAXT, MINB) rmsnorm_kernel(uint4 *x,
 struct NormArgs {
     void *x;
     const void *delta;  // non-null: the residual form
+    bool stats;         // write only each row's rstd (y is float [M])
     const void *w;
     void *y;
     int64_t M;
@@ -198,7 +204,10 @@ cudaError_t launch_shape(const NormArgs &a, cudaStream_t s)
     const uint4 *d = static_cast<const uint4 *>(a.delta);
     const uint4 *w = static_cast<const uint4 *>(a.w);
     const unsigned g = static_cast<unsigned>(grid);
-    if (a.out_f32)
+    if (a.stats)
+        rmsnorm_kernel<ITEMS, false, MAXT, false, MINB, true><<<g, a.threads, 0, s>>>(
+            x, d, w, a.y, a.M, a.H, a.eps);
+    else if (a.out_f32)
         rmsnorm_kernel<ITEMS, true, MAXT, ADD, MINB><<<g, a.threads, 0, s>>>(x, d, w, a.y, a.M,
                                                                              a.H, a.eps);
     else
@@ -241,7 +250,8 @@ void rmsnorm_shape(int64_t H, int *items, int *threads)
 }
 
 static cudaError_t launch_any(void *x, const void *delta, const void *w, void *y, int64_t M,
-                              int64_t H, float eps, bool out_f32, int num_sms, cudaStream_t s)
+                              int64_t H, float eps, bool out_f32, int num_sms, cudaStream_t s,
+                              bool stats = false)
 {
     int items, threads;
     rmsnorm_shape(H, &items, &threads);
@@ -254,7 +264,7 @@ static cudaError_t launch_any(void *x, const void *delta, const void *w, void *y
         threads = static_cast<int>((t + 31) / 32 * 32);
     }
 #endif
-    const NormArgs a{x, delta, w, y, M, static_cast<int>(H), eps, out_f32, threads, num_sms};
+    const NormArgs a{x, delta, stats, w, y, M, static_cast<int>(H), eps, out_f32, threads, num_sms};
     return delta ? launch_norm<true>(a, items, s) : launch_norm<false>(a, items, s);
 }
 
@@ -268,6 +278,13 @@ cudaError_t launch_add_rmsnorm(void *x, const void *delta, const void *w, void *
                                int64_t H, float eps, bool out_f32, int num_sms, cudaStream_t s)
 {
     return launch_any(x, delta, w, y, M, H, eps, out_f32, num_sms, s);
+}
+
+cudaError_t launch_row_rstd(const void *x, float *r, int64_t M, int64_t H, float eps, int num_sms,
+                            cudaStream_t s)
+{
+    return launch_any(const_cast<void *>(x), nullptr, nullptr, r, M, H, eps, false, num_sms, s,
+                      true);
 }
 
 }  // namespace bi

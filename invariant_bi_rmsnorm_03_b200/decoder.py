@@ -296,6 +296,8 @@ class ToyDecoder:
 
         x = L.bi_embedding(W["embed"], tokens)
         o = torch.empty((T, c.n_heads, c.head_dim), dtype=torch.bfloat16, device=self.dev)
+        # the fused norm forms' row statistics, one buffer for the whole step
+        nws = L._norm_ws(T, self.dev) if c.fused else None
         if c.fused:
             h, n = None, 1
         else:
@@ -303,9 +305,10 @@ class ToyDecoder:
         for i in range(c.layers):
             kv_all = PagedKV(self.k_cache[i], self.v_cache[i], bt)
             if c.fused:
-                # RMSNorm, the QKV matmul, RoPE and the cache write in one launch
+                # RMSNorm, the QKV matmul, RoPE and the cache write: the row
+                # statistics, then one matmul launch
                 q = L.bi_rmsnorm_matmul_rope_kv(x, self.wf["l%d.wqkv" % i], c.eps, kv_all,
-                                                self.rope, pos, slots, c.n_heads)
+                                                self.rope, pos, slots, c.n_heads, ws=nws)
             else:
                 qkv = L.bi_matmul(h, W["l%d.wqkv" % i])
                 q = L.bi_rope_kv_write(kv_all, qkv, pos, slots, c.n_heads, c.theta)
@@ -321,9 +324,9 @@ class ToyDecoder:
                 # x += o Wo^T; x += swiglu(RMSNorm(x) Wgu^T) Wdown^T
                 L.bi_matmul_residual(o.view(T, c.n_heads * c.head_dim), W["l%d.wo" % i], x,
                                      out=x)
-                f = L.bi_swiglu(L.bi_rmsnorm_matmul(x, self.wf["l%d.wgu" % i], c.eps))
+                f = L.bi_swiglu(L.bi_rmsnorm_matmul(x, self.wf["l%d.wgu" % i], c.eps, ws=nws))
                 L.bi_matmul_residual(f, W["l%d.wdown" % i], x, out=x)
-                n += 5
+                n += 7  # each norm form: the row statistics, then the matmul
                 continue
             a = L.bi_matmul(o.view(T, c.n_heads * c.head_dim), W["l%d.wo" % i])
             h = L.bi_add_rmsnorm(x, a, W["l%d.mlp_norm" % i], c.eps)
@@ -339,14 +342,15 @@ class ToyDecoder:
             n += 5
         if c.fused:
             last = L.bi_embedding(x, rows)
-            logits = L.bi_rmsnorm_matmul(last, self.wf["lm_head"], c.eps, out_dtype=torch.float32)
+            logits = L.bi_rmsnorm_matmul(last, self.wf["lm_head"], c.eps, out_dtype=torch.float32,
+                                         ws=nws)
         else:
             last = L.bi_embedding(h, rows)
             logits = L.bi_matmul(last, W["lm_head"], out_dtype=torch.float32)
         nt = L.bi_sample(logits, self._to_dev(plan.temperature), self._to_dev(plan.top_p),
                          self._to_dev(plan.seed.view(np.int64)),
                          self._to_dev(plan.offset.view(np.int64)))
-        self.launches += n + 3
+        self.launches += n + (4 if c.fused else 3)
         return nt.cpu().numpy()
 
 

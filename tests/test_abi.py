@@ -124,11 +124,17 @@ def test_fused_matmuls_reject_bad_arguments(lib):
     assert L.bi_fold_norm_weight(FAKE, FAKE, FAKE, 4, 12, None) == INV          # K % 8
     assert L.bi_fold_norm_weight(None, FAKE, FAKE, 4, 64, None) == INV
     assert L.bi_fold_norm_weight(None, None, None, 0, 64, None) == OK           # N == 0
-    assert L.bi_rmsnorm_matmul(FAKE, FAKE, FAKE, 4, 12, 64, 1e-6, 0, None) == INV  # N % 8
-    assert L.bi_rmsnorm_matmul(FAKE, FAKE, FAKE, 4, 64, 64, -1.0, 0, None) == INV  # eps < 0
-    assert L.bi_rmsnorm_matmul(FAKE, FAKE, FAKE, 4, 64, 64, float("inf"), 0, None) == INV
-    assert L.bi_rmsnorm_matmul(FAKE, FAKE, FAKE, 4, 64, 64, 1e-6, 9, None) == INV   # dtype
-    assert L.bi_rmsnorm_matmul(None, None, None, 0, 64, 64, 1e-6, 0, None) == OK    # M == 0
+    rm = lambda M=4, N=64, K=64, eps=1e-6, dt=0, ws=FAKE, nb=1024: L.bi_rmsnorm_matmul(  # noqa: E731
+        FAKE, FAKE, FAKE, M, N, K, eps, dt, ws, nb, None)
+    assert rm(N=12) == INV                 # N % 8
+    assert rm(eps=-1.0) == INV
+    assert rm(eps=float("inf")) == INV
+    assert rm(dt=9) == INV
+    assert rm(K=65544) == INV              # beyond the row reduction's limit
+    assert rm(nb=8) == binding.Status.WORKSPACE
+    assert rm(ws=None) == binding.Status.WORKSPACE
+    assert L.bi_rmsnorm_matmul(None, None, None, 0, 64, 64, 1e-6, 0, None, 0, None) == OK  # M == 0
+    assert L.bi_rmsnorm_matmul_workspace_bytes(5) == 256
     assert L.bi_matmul_residual(FAKE, FAKE, FAKE, FAKE, 4, 64, 12, None) == INV     # K % 8
     assert L.bi_matmul_residual(FAKE, FAKE, None, FAKE, 4, 64, 64, None) == INV     # no R
     assert L.bi_matmul_residual(None, None, None, None, 0, 64, 64, None) == OK
@@ -140,8 +146,9 @@ def test_qkv_epilogue_and_angle_table_reject_bad_arguments(lib):
     assert L.bi_rope_table(FAKE, 16, 96, 10000.0, None) == INV                  # head_dim
     assert L.bi_rope_table(FAKE, 16, 128, 1.0, None) == INV                     # theta <= 1
     assert L.bi_rope_table(P(0x10004), 16, 128, 10000.0, None) == INV           # alignment
-    call = lambda kv, Hq=4, T=3, K=64: L.bi_rmsnorm_matmul_rope_kv(  # noqa: E731
-        FAKE, FAKE, 1e-6, ctypes.byref(kv), FAKE, 4096, FAKE, FAKE, FAKE, T, K, Hq, None)
+    call = lambda kv, Hq=4, T=3, K=64, ws=FAKE: L.bi_rmsnorm_matmul_rope_kv(  # noqa: E731
+        FAKE, FAKE, 1e-6, ctypes.byref(kv), FAKE, 4096, FAKE, FAKE, FAKE, T, K, Hq, ws, 256, None)
+    assert call(_kv(), ws=None) == binding.Status.WORKSPACE
     assert call(_kv(page_size=8)) == INV
     assert call(_kv(), Hq=3) == INV                                             # Hq % Hkv
     assert call(_kv(), K=12) == INV                                             # K % 8
@@ -167,3 +174,50 @@ def test_backward_passes_reject_bad_arguments(lib):
     assert mb(M=0) == OK
     # W^T, dC^T and A^T, each region rounded up to 256 bytes, rows padded to 8
     assert L.bi_matmul_backward_workspace_bytes(5, 64, 32) == 4096 + 1024 + 512
+
+
+def test_swiglu_and_rope_backward_reject_bad_arguments(lib):
+    L, INV, OK = lib.lib, binding.Status.INVALID, binding.Status.OK
+    sw = lambda T=4, F=64, dt=0, p=FAKE: L.bi_swiglu_backward(p, FAKE, FAKE, T, F, dt, None)  # noqa: E731
+    assert sw(F=12) == INV
+    assert sw(F=0) == INV
+    assert sw(T=-1) == INV
+    assert sw(dt=5) == INV
+    assert sw(p=P(0x10008)) == INV       # misaligned
+    assert sw(T=0) == OK
+    rb = lambda T=4, nh=2, d=128, ld=256, ldo=256, th=1e4, dt=0: L.bi_rope_backward(  # noqa: E731
+        FAKE, ld, FAKE, FAKE, ldo, T, nh, d, th, dt, None)
+    assert rb(d=96) == INV
+    assert rb(nh=0) == INV
+    assert rb(ld=255) == INV             # shorter than the heads it holds
+    assert rb(ldo=260 - 2) == INV        # not a multiple of 8
+    assert rb(th=1.0) == INV
+    assert rb(th=float("inf")) == INV
+    assert rb(dt=3) == INV
+    assert rb(T=0) == OK
+
+
+def test_attention_backward_rejects_bad_arguments(lib):
+    import ctypes as C
+    L, INV, OK, WS = lib.lib, binding.Status.INVALID, binding.Status.OK, binding.Status.WORKSPACE
+    UNS = binding.Status.UNSUPPORTED
+
+    def kv(d=128, heads=2, pages=8, mp=4):
+        return binding._PagedKV(0x10000, 0x20000, 0x30000, mp, pages, 16, heads, d)
+
+    def ab(k=None, Hq=8, B=2, T=10, mq=5, mkv=40, ws=FAKE, nb=1 << 20, dk=P(0x40000),
+           dv=P(0x50000)):
+        k = k or kv()
+        return L.bi_attention_backward(C.byref(k), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, B, Hq, T,
+                                       mq, mkv, 0.1, FAKE, dk, dv, ws, nb, None)
+    assert ab(Hq=7) == INV                 # Hq % Hkv
+    assert ab(k=kv(d=96)) == UNS
+    assert ab(mkv=65) == INV               # beyond the page table (4 pages)
+    assert ab(mq=50, mkv=40) == INV        # a chunk longer than its sequence
+    assert ab(dk=P(0x10000)) == INV        # dk aliases the k cache
+    assert ab(dk=P(0x50000)) == INV        # dk aliases dv
+    assert ab(nb=8) == WS
+    assert ab(ws=None) == WS
+    assert ab(T=0) == OK
+    assert ab(B=0) == OK
+    assert L.bi_attention_backward_workspace_bytes(8, 10) == 2 * 8 * 10 * 4

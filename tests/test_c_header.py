@@ -38,7 +38,11 @@ int main(void)
     EXPECT(bi_rmsnorm(NULL, NULL, NULL, 0, 64, 1e-6f, BI_BF16, NULL) == BI_OK);
     EXPECT(bi_matmul(fake, fake, fake, 4, 64, 12, BI_BF16, NULL, 0, NULL) == BI_ERR_INVALID);
     EXPECT(bi_kv_write(&kv, fake, fake, (const int64_t *)fake, 4, NULL) == BI_ERR_INVALID);
-    EXPECT(bi_rmsnorm_matmul(fake, fake, fake, 4, 64, 64, -1.0f, BI_BF16, NULL) == BI_ERR_INVALID);
+    EXPECT(bi_rmsnorm_matmul(fake, fake, fake, 4, 64, 64, -1.0f, BI_BF16, fake, 256, NULL) ==
+           BI_ERR_INVALID);
+    EXPECT(bi_rmsnorm_matmul_workspace_bytes(5) == 256);
+    EXPECT(bi_swiglu_backward(fake, fake, fake, 4, 12, BI_BF16, NULL) == BI_ERR_INVALID);
+    EXPECT(bi_attention_backward_workspace_bytes(8, 10) == 640);
     EXPECT(bi_transpose(fake, fake, 8, 4, 7, NULL) == BI_ERR_INVALID);
     EXPECT(bi_matmul_backward_workspace_bytes(5, 64, 32) == 4096 + 1024 + 512);
     EXPECT(bi_matmul_workspace_bytes(2048, 4096, 4096) == 0 || !EXPECTED_FLAVOUR);

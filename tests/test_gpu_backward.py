@@ -2,7 +2,8 @@
 oracle, dx rows independent of the batch, dw the same bits on every run),
 the transpose (a bit copy), and the matmul backward on the invariant GEMM
 (parity with the oracle's products, exact on small integers, dA rows
-independent of the batch)."""
+independent of the batch), and the SwiGLU and RoPE backward (parity with
+the oracle, rows independent of the batch, head sets inside wider rows)."""
 import numpy as np
 import pytest
 import torch
@@ -93,3 +94,62 @@ def test_matmul_backward_da_rows_do_not_depend_on_the_batch(L):
         assert same_bytes(da, full[:M]), M
     _, dw = L.bi_matmul_backward(dcd, ad, wd, want_da=False)
     assert same_bytes(dw, dw_full)
+
+
+@pytest.mark.parametrize("T,F", [(1, 8), (37, 1408), (300, 120), (5, 14336)])
+def test_swiglu_backward_parity(L, T, F):
+    g = rng(560 + T + F)
+    gate = normal_bf16(g, (T, F), std=2.0)
+    gate[0, :4] = f32_to_bf16_bits(np.array([-100.0, -20.0, 20.0, 100.0], dtype=np.float32))[: min(4, F)]
+    gu = np.concatenate([gate, normal_bf16(g, (T, F))], axis=1)
+    dout = normal_bf16(g, (T, F))
+    ref = oracle.swiglu_backward(gu, dout)
+    for dt, tol in ((torch.bfloat16, TOL_BF16), (torch.float32, TOL_F32)):
+        out = L.bi_swiglu_backward(dev_bf16(gu), dev_bf16(dout), out_dtype=dt)
+        assert np.all(np.isfinite(to_f64(out)))
+        assert rowwise_normwise(to_f64(out), ref).max() <= tol, dt
+
+
+def test_swiglu_backward_rows_do_not_depend_on_the_batch(L):
+    g = rng(570)
+    gu, dout = normal_bf16(g, (300, 2 * 1408), std=2.0), normal_bf16(g, (300, 1408))
+    gud, dd = dev_bf16(gu), dev_bf16(dout)
+    full = L.bi_swiglu_backward(gud, dd)
+    for M in (1, 7, 299):
+        assert same_bytes(L.bi_swiglu_backward(gud[:M], dd[:M]), full[:M]), M
+
+
+@pytest.mark.parametrize("nh,d", [(8, 128), (32, 128), (3, 64)])
+def test_rope_backward_parity(L, nh, d):
+    g = rng(580 + nh + d)
+    T = 77
+    dy = normal_bf16(g, (T, nh, d))
+    pos = g.integers(0, 32768, size=T).astype(np.int32)
+    pos[0] = 0
+    ref = oracle.rope_backward(dy, pos)
+    pd = torch.from_numpy(pos).to("cuda")
+    for dt, tol in ((torch.bfloat16, TOL_BF16), (torch.float32, TOL_F32)):
+        out = L.bi_rope_backward(dev_bf16(dy), pd, out_dtype=dt)
+        assert rowwise_normwise(to_f64(out).reshape(T, -1), ref.reshape(T, -1)).max() <= tol, dt
+    # position 0 is the identity
+    out = L.bi_rope_backward(dev_bf16(dy), pd, out_dtype=torch.float32)
+    np.testing.assert_array_equal(to_f64(out)[0], bf16_bits_to_f32(dy[0]).astype(np.float64))
+
+
+def test_rope_backward_reads_and_writes_head_sets_of_wider_rows(L):
+    # the q heads (first 32) and the k heads (next 8) of a fused q/k/v
+    # gradient [T, (32 + 2 * 8) * 128], rotated in place of a copy
+    g = rng(590)
+    T, Hq, Hkv, d = 40, 32, 8, 128
+    dqkv = normal_bf16(g, (T, (Hq + 2 * Hkv) * d))
+    pos = torch.from_numpy(g.integers(0, 4096, size=T).astype(np.int32)).to("cuda")
+    src = dev_bf16(dqkv)
+    out = torch.zeros_like(src)
+    v3 = lambda t, h0, n: t.view(T, Hq + 2 * Hkv, d)[:, h0:h0 + n]  # noqa: E731
+    L.bi_rope_backward(v3(src, 0, Hq), pos, out=v3(out, 0, Hq))
+    L.bi_rope_backward(v3(src, Hq, Hkv), pos, out=v3(out, Hq, Hkv))
+    q_ref = L.bi_rope_backward(v3(src, 0, Hq).contiguous(), pos)
+    k_ref = L.bi_rope_backward(v3(src, Hq, Hkv).contiguous(), pos)
+    assert same_bytes(v3(out, 0, Hq).contiguous(), q_ref)
+    assert same_bytes(v3(out, Hq, Hkv).contiguous(), k_ref)
+    assert torch.count_nonzero(v3(out, Hq + Hkv, Hkv)) == 0  # the v part is untouched

@@ -125,10 +125,13 @@ def test_prefill_8192_modes_bitwise_and_sampled_parity(L):
 
     # sampled tokens and heads against the fp64 oracle
     kc, vc = kv_from_blocks(host_bits(kv.k_cache)), kv_from_blocks(host_bits(kv.v_cache))
-    ts = np.array([0, 1, 255, 256, 257, 4095, 8191])
-    heads = np.array([0, 13, 31])
-    tt, hh = np.meshgrid(ts, heads, indexing="ij")
-    tt, hh = tt.ravel(), hh.ravel()
+    # the split and tile edges in every head, plus 256 random (token, head)
+    # pairs over the whole prompt
+    ts = np.array([0, 1, 127, 128, 255, 256, 257, 4095, 8191])
+    tt, hh = np.meshgrid(ts, np.arange(Hq), indexing="ij")
+    gs = np.random.default_rng(7)
+    tt = np.concatenate([tt.ravel(), gs.integers(0, S, 256)])
+    hh = np.concatenate([hh.ravel(), gs.integers(0, Hq, 256)])
     rows = np.stack([c["q"][t, h] for t, h in zip(tt, hh)])
     want, want_lse = oracle.attention(rows, np.zeros(len(tt)), hh, tt, Hq, kc, vc, bt_np,
                                       want_lse=True)

@@ -1,6 +1,7 @@
 """The fused matmul forms on the GPU: the norm-weight fold (bit-exact: the
 correctly rounded product), RMSNorm folded into the matmul (parity with the
-fp64 oracle, bitwise batch invariance) and the residual matmul (equal bit for
+fp64 oracle, bitwise batch invariance, its row statistics bi_rmsnorm's own)
+and the residual matmul (equal bit for
 bit to bi_matmul followed by the addition; parity with the oracle)."""
 import numpy as np
 import pytest
@@ -41,6 +42,21 @@ def test_fold_is_the_correctly_rounded_product(L):
     Wd = dev_bf16(W)
     L.bi_fold_norm_weight(Wd, dev_bf16(w), out=Wd)  # in place
     np.testing.assert_array_equal(host_bits(Wd), want)
+
+
+@pytest.mark.parametrize("M,K", [(1, 64), (37, 256), (300, 4096), (2048, 4096)])
+def test_rmsnorm_matmul_row_scale_is_the_rmsnorm_rstd(L, M, K):
+    # With the identity as the folded weight the product is x itself (exact
+    # in fp32), so the fused form is round(r * x) -- which must equal
+    # bi_rmsnorm with unit weights, round((x * rstd) * 1), bit for bit: the
+    # row statistics are bi_rmsnorm's own reduction.
+    g = rng(310 + M + K)
+    x = dev_bf16(scaled_rows(g, M, K))
+    eye = dev_bf16(f32_to_bf16_bits(np.eye(K, dtype=np.float32)))
+    ones = dev_bf16(f32_to_bf16_bits(np.ones(K, dtype=np.float32)))
+    for dt in (torch.bfloat16, torch.float32):
+        assert same_bytes(L.bi_rmsnorm_matmul(x, eye, EPS, out_dtype=dt),
+                          L.bi_rmsnorm(x, ones, EPS, out_dtype=dt)), dt
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)

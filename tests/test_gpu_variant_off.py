@@ -1,5 +1,6 @@
 """Negative controls: the variant-off build (split-K matmul, load-dependent
-RMSNorm strategy, decode blocks that pre-merge their own split range) must
+RMSNorm strategy, decode split ranges whose size follows the load, each
+block pre-merging its own range) must
 FAIL the invariance checks that the batch-invariant build passes.  This shows
 the byte comparisons can detect a batch-dependent reduction order, and that
 the invariant build passes them for the reason it is built for (float
@@ -80,4 +81,40 @@ def test_variant_decode_bits_change_with_work_division(V, L):
         differs |= not same_bytes(o_v, ref_v)
         err = rowwise_normwise(to_f64(o_v).reshape(3, -1), to_f64(ref_v).reshape(3, -1))
         assert err.max() <= TOL_BF16
+    assert differs
+
+
+def test_variant_decode_split_size_follows_the_load(V, L):
+    # The variant-off decode cuts each sequence into ranges of ceil(L / count)
+    # keys (count chosen from the load), so a token's decode output differs
+    # from its prefill output -- the mismatch the invariant build removes
+    # (there, decode of the last token equals prefill bit for bit).
+    from synth import page_table, slot_mapping
+    g = rng(82)
+    S, Hq, Hkv, d = 2900, 8, 2, 128
+    q = normal_bf16(g, (S, Hq, d))
+    k, v = normal_bf16(g, (S, Hkv, d)), normal_bf16(g, (S, Hkv, d))
+    bt, npg = page_table(g, [S])
+    i32 = lambda a: torch.tensor(a, dtype=torch.int32, device=DEV)  # noqa: E731
+    differs = False
+    for lib, invariant in ((L, True), (V, False)):
+        kv = bi.PagedKV(torch.zeros((npg, Hkv, 16, d), dtype=torch.bfloat16, device=DEV),
+                        torch.zeros((npg, Hkv, 16, d), dtype=torch.bfloat16, device=DEV),
+                        torch.from_numpy(bt).to(DEV))
+        lib.bi_kv_write(kv, dev_bf16(k), dev_bf16(v),
+                        torch.from_numpy(slot_mapping(bt, 0, np.arange(S))).to(DEV))
+        op = lib.bi_attention_prefill(kv, dev_bf16(q), i32([0, S]), i32([0]), S)
+        # the last token decoded in a batch of 16 copies: 16 x 2 kv heads
+        # against 148 SMs gives 6 blocks per sequence, so the variant cuts
+        # the 2900 keys into ranges of 496 (pieces at 0, 256, 496, 752, ...)
+        dec = bi.PagedKV(kv.k_cache, kv.v_cache, torch.from_numpy(np.repeat(bt, 16, axis=0)).to(DEV))
+        qd = dev_bf16(np.repeat(q[S - 1:], 16, axis=0))
+        od = lib.bi_attention_decode(dec, qd, i32([S] * 16), S)
+        same = same_bytes(od[0], op[S - 1])
+        if invariant:
+            assert same
+        else:
+            differs = not same
+            err = rowwise_normwise(to_f64(od[0]).reshape(1, -1), to_f64(op[S - 1]).reshape(1, -1))
+            assert err.max() <= TOL_BF16
     assert differs
