@@ -664,7 +664,8 @@ static bi_status decode_args_ok(const bi_paged_kv *kv, const void *q, const void
 static bi_status decode_launch(const DeviceState *d, const bi_paged_kv *kv, const void *q,
                                void *o, float *lse, const int32_t *seq_lens, int32_t B,
                                int32_t Hq, int max_splits, int splits_per_cta, int chunks,
-                               float scale, int32_t *order, float *partials, cudaStream_t s)
+                               bool per_sequence, float scale, int32_t *order, float *partials,
+                               cudaStream_t s)
 {
     const int D = kv->head_dim, Hkv = kv->num_kv_heads, group = Hq / Hkv;
     bi::AttnParams p{};
@@ -682,6 +683,9 @@ static bi_status decode_launch(const DeviceState *d, const bi_paged_kv *kv, cons
     p.seq_lens = seq_lens;
     p.order = order;
     p.splits_per_cta = splits_per_cta;
+    // a division chosen from the load cuts each sequence into `chunks`
+    // blocks of its own length; an explicit one uses splits_per_cta for all
+    p.blocks_per_seq = per_sequence ? chunks : 0;
     p.max_splits = max_splits;
     p.scale_log2 = float(double(scale) * 1.4426950408889634);
     p.o = o;
@@ -720,8 +724,9 @@ bi_status bi_attention_decode(const bi_paged_kv *kv, const void *q, void *o, flo
     if (!ws || ws_bytes < need || !aligned16(ws)) return BI_ERR_WORKSPACE;
     int32_t *order = static_cast<int32_t *>(ws);
     float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + order_bytes(B));
-    return decode_launch(d, kv, q, o, lse, seq_lens, B, Hq, max_splits, c, chunks, scale, order,
-                         partials, static_cast<cudaStream_t>(stream));
+    return decode_launch(d, kv, q, o, lse, seq_lens, B, Hq, max_splits, c, chunks,
+                         splits_per_cta == 0, scale, order, partials,
+                         static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------- no-alloc decode
@@ -784,8 +789,9 @@ bi_status bi_attention_decode_noalloc(const bi_paged_kv *kv, const void *q, void
     if (need > BI_NOALLOC_SCRATCH_BYTES) return BI_ERR_WORKSPACE;
     int32_t *order = static_cast<int32_t *>(scratch);
     float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(scratch) + order_bytes(B));
-    return decode_launch(d, kv, q, o, lse, seq_lens, B, Hq, max_splits, c, chunks, scale, order,
-                         partials, static_cast<cudaStream_t>(stream));
+    return decode_launch(d, kv, q, o, lse, seq_lens, B, Hq, max_splits, c, chunks,
+                         splits_per_cta == 0, scale, order, partials,
+                         static_cast<cudaStream_t>(stream));
 }
 
 size_t bi_attention_prefill_workspace_bytes(const bi_paged_kv *kv, int32_t B, int32_t Hq,

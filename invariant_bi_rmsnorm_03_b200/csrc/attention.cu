@@ -154,6 +154,25 @@ struct Item {
 
 __device__ __forceinline__ int key_of(const Item &it, int s) { return it.key0 + (s - it.s0) * kSplit; }
 
+// Decode work division: blocks per sequence, and the splits a block of a
+// sequence of n splits covers (its first block merges splits 0 .. c-1).
+// With blocks_per_seq set, each sequence is cut into that many blocks of
+// ceil(n / blocks_per_seq) splits, so a long sequence gets long blocks and a
+// short one short blocks; otherwise every block covers splits_per_cta.
+// The division never changes the output bits.
+__device__ __forceinline__ int decode_blocks(const AttnParams &p)
+{
+    return p.blocks_per_seq > 0 ? p.blocks_per_seq
+                                : (p.max_splits + p.splits_per_cta - 1) / p.splits_per_cta;
+}
+#if BI_INVARIANT
+__device__ __forceinline__ int decode_chunk(const AttnParams &p, int n)
+{
+    return p.blocks_per_seq > 0 ? max(1, (n + p.blocks_per_seq - 1) / p.blocks_per_seq)
+                                : p.splits_per_cta;
+}
+#endif
+
 // Decode: whether this block alone covers the whole sequence, and the index
 // of the record a block that does not hands its merged range over in.
 __device__ __forceinline__ bool item_whole(const Item &it)
@@ -191,7 +210,7 @@ __device__ __forceinline__ int variant_range(int L, int nblk)
 __device__ __forceinline__ bool make_item(const AttnParams &p, int idx, Item &it)
 {
     if (p.decode) {
-        const int nblk = (p.max_splits + p.splits_per_cta - 1) / p.splits_per_cta;
+        const int nblk = decode_blocks(p);
         const int x = idx % nblk, r = idx / nblk;
         const int z = r / p.Hkv;
         it.b = p.order ? p.order[z] : z;
@@ -205,9 +224,10 @@ __device__ __forceinline__ bool make_item(const AttnParams &p, int idx, Item &it
         }
         if (it.kv_len <= 0) return false;
 #if BI_INVARIANT
-        it.s0 = x * p.splits_per_cta;
+        const int c = decode_chunk(p, it.n_splits);
+        it.s0 = x * c;
         if (it.s0 >= it.n_splits) return false;
-        it.s1 = min(it.n_splits, it.s0 + p.splits_per_cta);
+        it.s1 = min(it.n_splits, it.s0 + c);
         it.key0 = it.s0 * kSplit;
         it.kend = it.kv_len;
 #else
@@ -274,6 +294,19 @@ __device__ __forceinline__ float logit(float s, float cs, float m_s)
     return ex2(__fmaf_rn(s, cs, -m_s));
 }
 
+// Maximum of the visible logits of 32 keys kc .. kc+31.
+__device__ __forceinline__ void chunk_max(const uint32_t (&r)[32], int kc, int t, float (&mx)[8])
+{
+    if (kc + 31 <= t) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[j]));
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (kc + j <= t) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[j]));
+    }
+}
+
 // p of the 32 keys kc .. kc+31, computed in place (r[j] becomes the bits of
 // p_j): packed bf16 P written to TMEM at `pcol` (16 columns), the class sums
 // S_u advanced by this chunk in the order of tree8.
@@ -300,58 +333,46 @@ __device__ __forceinline__ void chunk_exp(uint32_t (&r)[32], int kc, int t, floa
                                      e(16 + 2 * u), e(17 + 2 * u), e(24 + 2 * u), e(25 + 2 * u)));
 }
 
-// Row maximum of one split's visible logits, scaled: m_s = round(c max_j S_j)
-// (for c > 0, x -> round(x c) is monotonic, so this equals max_j round(S_j c);
-// a maximum is exact in any order).  S is read from TMEM columns
-// sb .. sb+255 in 16-column loads, the next load in flight while a chunk is
-// scanned; eight accumulators break the dependency chain.  The loop is kept
-// rolled (two loads per trip): a small instruction footprint matters more
-// here than unrolling, since the block's other warps run other code on the
-// same sub-partitions.
-__device__ __forceinline__ float row_max(uint32_t sb, int k0, int t, float cs)
+// Softmax of one split, one row per thread (any row layout; used by
+// prefill and by decode with more than 8 query rows per lane quarter).
+// S is read from TMEM columns sb .. sb+255 in two passes of 32-column
+// loads, the next load in flight while a chunk is processed; P (bf16 pairs)
+// is written over columns sb .. sb+127 as the second pass goes (each store
+// lands on columns this thread has already read).  Returns m_s (scaled,
+// log2 units) and l_s.  (P V cannot start before the whole pass is done: it
+// writes O_s over the logits of keys 128..255.)
+__device__ __forceinline__ void softmax_rows(uint32_t sb, int k0, int t, float cs, float &m_s,
+                                             float &l_s)
 {
-    constexpr int NC = kSplit / 16;  // 16-key chunks (small loads: this runs on the
-                                     // fold warps, whose registers hold the output)
+    constexpr int NC = kSplit / 32;  // 32-key chunks
+    // pass 1: maximum of the raw logits over the visible keys.  For c > 0,
+    // x -> round(x * c) is monotonic, so max_j round(S_j c) = round(max_j S_j * c).
+    // (A maximum is exact in any order; eight accumulators break the chain.)
     float mx[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-    auto scan = [&](const uint32_t (&r)[16], int kc) {
-        if (kc + 15 <= t) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[j]));
-        } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-                if (kc + j <= t) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[j]));
-        }
-    };
-    uint32_t ra[16], rb[16];
-    tmem_ld16(sb, ra);
+    // The loops are kept rolled (two loads of each kind per trip): a small
+    // instruction footprint matters more here than unrolling, since the
+    // block's other warps run other code on the same sub-partitions.
+    {
+        // 32-column loads, the next in flight while a chunk is scanned
+        uint32_t ra[32], rb[32];
+        tmem_ld32(sb, ra);
 #pragma unroll 1
-    for (int c = 0; c < NC; c += 2) {
-        tmem_wait_ld16(ra);
-        tmem_ld16(sb + 16 * (c + 1), rb);
-        scan(ra, k0 + 16 * c);
-        tmem_wait_ld16(rb);
-        if (c + 2 < NC) tmem_ld16(sb + 16 * (c + 2), ra);
-        scan(rb, k0 + 16 * (c + 1));
+        for (int c = 0; c < NC; c += 2) {
+            tmem_wait_ld(ra);
+            tmem_ld32(sb + 32 * (c + 1), rb);
+            chunk_max(ra, k0 + 32 * c, t, mx);
+            tmem_wait_ld(rb);
+            if (c + 2 < NC) tmem_ld32(sb + 32 * (c + 2), ra);
+            chunk_max(rb, k0 + 32 * (c + 1), t, mx);
+        }
     }
     const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-    return __fmul_rn(mraw, cs);
-}
-
-// The exponent pass of one split, one row per thread (any row layout; used
-// by prefill and by decode with more than 8 query rows per lane quarter),
-// given the row's m_s (row_max, computed by another warp one split ahead):
-// p = 2^(S c - m_s) with masked keys 0, P (bf16 pairs) written over TMEM
-// columns sb .. sb+127 as the pass goes (each store lands on columns this
-// thread has already read), l_s summed in the order of tree8; 32-key chunks,
-// the next chunk's load in flight.  (P V cannot start before the whole pass
-// is done: it writes O_s over the logits of keys 128..255.)
-__device__ __forceinline__ float softmax_exp(uint32_t sb, int k0, int t, float cs, float m_s)
-{
-    constexpr int NC = kSplit / 32;
+    m_s = __fmul_rn(mraw, cs);
+    // pass 2: p = 2^(S c - m_s), masked keys 0; P into TMEM; the sum in the
+    // order of tree8.  32-key chunks, the next chunk's load in flight.
     float S[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     uint32_t ra[32], rb[32];
     tmem_ld32(sb, ra);
@@ -365,7 +386,7 @@ __device__ __forceinline__ float softmax_exp(uint32_t sb, int k0, int t, float c
         chunk_exp(rb, k0 + 32 * (c + 1), t, cs, m_s, sb + 16 * (c + 1), S);
     }
     tmem_wait_st();
-    return __fadd_rn(__fadd_rn(S[0], S[1]), __fadd_rn(S[2], S[3]));
+    l_s = __fadd_rn(__fadd_rn(S[0], S[1]), __fadd_rn(S[2], S[3]));
 }
 
 // Softmax of one split for decode when the query rows of this lane quarter
@@ -476,8 +497,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint64_t *barP = barS + 2;      // [2] P and (m_s, l_s) of buffer b written (128 arrivals)
     uint64_t *barO = barP + 2;      // [2] O_s of buffer b computed
     uint64_t *barF = barO + 2;      // [2] O_s of buffer b merged, buffer free
-    uint64_t *barM = barF + 2;      // [2] row maxima of buffer b's split written (128 arrivals)
-    uint64_t *drain = barM + 2;
+    uint64_t *drain = barF + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
@@ -494,7 +514,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&barP[b], 128);
             mbar_init(&barO[b], 1);
             mbar_init(&barF[b], kFoldThreads);
-            mbar_init(&barM[b], 128);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -736,13 +755,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int q = warp & 3;
         const uint32_t lane_base = tmem_addr(tmem, 32 * q, 0);
         const int row_id = 32 * q + lane;  // TMEM lane of this row
-        // Rows whose softmax reads one row per thread (all but decode with at
-        // most 8 rows per lane quarter) get their maxima from the first-half
-        // fold warp of the quarter (warps 2, 3, 8, 9), one split ahead, so
-        // the softmax warp only runs the exponent pass.  The maximum is exact
-        // in any order: the bits are those of a one-warp softmax.
-        const bool max_ahead = !(p.decode && p.rows_per_q <= 8);
-        const bool max_warp = max_ahead && !is_softmax && warp < 10;
         // This thread's row of an item: its last visible key t, whether its
         // lane quarter holds any row, whether the row is a real one, and
         // where its output goes.
@@ -762,24 +774,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 active = 32 * q < it.rows;
             }
         };
-        // The scaled maximum of split number g (key base k0) for this row,
-        // written to sML and signalled on barM.
-        auto max_split = [&](int g, int k0, int t_row, bool act) -> bool {
-            const int b = g & 1;
-            const uint32_t par = uint32_t(g >> 1) & 1u;
-            if (!wait(&barS[b], par, ctl)) return false;
-            tc_fence_after();
-            const float m_s =
-                act ? row_max(lane_base + C::BUF_COLS * uint32_t(b) + C::P_OFF, k0, t_row, p.scale_log2)
-                    : -INFINITY;
-            sML[(b * 128 + row_id) * 2 + 0] = m_s;
-            tc_fence_before();
-            mbar_arrive(&barM[b]);
-            return true;
-        };
         int gs = 0;
         bool ok = true;
-        bool ahead = false;  // the maximum of this item's first split is already written
         for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
             Item it;
             if (!make_item(p, idx, it)) continue;
@@ -812,15 +808,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                             sML[(b * 128 + 32 * q + (lane >> 2)) * 2 + 1] = l_s;
                         }
                     } else {
-                        if (max_ahead) {
-                            if (!wait(&barM[b], par, ctl)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            m_s = sML[(b * 128 + row_id) * 2 + 0];
-                        }
-                        if (active) l_s = softmax_exp(sb + C::P_OFF, key_of(it, s), t, cs, m_s);
+                        if (active) softmax_rows(sb + C::P_OFF, key_of(it, s), t, cs, m_s, l_s);
                         sML[(b * 128 + row_id) * 2 + 0] = m_s;
                         sML[(b * 128 + row_id) * 2 + 1] = l_s;
                     }
@@ -845,43 +833,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 float O[HW];
 #pragma unroll
                 for (int j = 0; j < HW; ++j) O[j] = 0.0f;
-                if (max_warp && !ahead && it.s1 > it.s0 && !max_split(gs, it.key0, t, active)) {
-                    ok = false;
-                    break;
-                }
-                ahead = false;
                 for (int s = it.s0; s < it.s1; ++s) {
                     const int g = gs + (s - it.s0);
                     const int b = g & 1;
                     const uint32_t par = uint32_t(g >> 1) & 1u;
-                    if (max_warp) {
-                        // the next split's maximum, before this split's merge:
-                        // the next split of this item, or the first split of
-                        // the block's next item
-                        if (s + 1 < it.s1) {
-                            if (!max_split(g + 1, key_of(it, s + 1), t, active)) {
-                                ok = false;
-                                break;
-                            }
-                        } else if (!p.decode) {
-                            // (decode runs one block per item: no next item)
-                            for (int nidx = idx + int(gridDim.x); nidx < p.items; nidx += gridDim.x) {
-                                // the prefill item nidx (as make_item): this
-                                // row's last visible key, its quarter's rows
-                                const int r = nidx / p.Hq;
-                                const int nb = r / p.num_q_tiles;
-                                const int tile = p.num_q_tiles - 1 - (r - nb * p.num_q_tiles);
-                                const int n = p.cu_q[nb + 1] - p.cu_q[nb];
-                                if (tile * 128 >= n) continue;
-                                const int npos0 = p.ctx_lens[nb] + tile * 128;
-                                const bool nact = 32 * q < n - tile * 128;
-                                if (!max_split(g + 1, 0, npos0 + 32 * q + lane, nact)) ok = false;
-                                ahead = ok;
-                                break;
-                            }
-                            if (!ok) break;
-                        }
-                    }
                     const uint32_t ob = lane_base + C::BUF_COLS * uint32_t(b) + C::O_OFF + col0;
                     const int k0 = key_of(it, s);
                     // barP: (m_s, l_s) of this split are in shared memory;
@@ -1042,35 +997,54 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p)
     const int n = (L + kSplit - 1) / kSplit;
     const float *base = p.ws + row * p.max_splits * C::REC;
 #if BI_INVARIANT
-    const int first_end = p.splits_per_cta;  // splits merged by the first block
-    if (L <= 0 || n <= first_end || n > p.max_splits) return;
+    if (L <= 0 || n > p.max_splits) return;
+    const int first_end = decode_chunk(p, n);  // splits merged by the first block
+    if (n <= first_end) return;
     const float *rec = base + int64_t(first_end - 1) * C::REC;
 #else
     // variant-off: one record per block of keys x R .. (x + 1) R - 1
-    const int nblk = (p.max_splits + p.splits_per_cta - 1) / p.splits_per_cta;
+    const int nblk = decode_blocks(p);
     if (L <= 0 || n > p.max_splits) return;
     const int R = variant_range(L, nblk);
     if (R >= L) return;  // one block: its output is written
     const float *rec = base;
 #endif
-    float m = rec[0], l = rec[1];
+#if BI_INVARIANT
+    const int rec0 = first_end, count = n - first_end;  // records split by split
+#else
+    const int rec0 = 1, count = (L + R - 1) / R - 1;    // records block by block
+#endif
+    float m = __ldg(rec), l = __ldg(rec + 1);
     float O[PER];
 #pragma unroll
-    for (int j = 0; j < PER; ++j) O[j] = rec[4 + lane * PER + j];
-#if BI_INVARIANT
-    for (int s = first_end; s < n; ++s) {
-        rec = base + int64_t(s) * C::REC;
-#else
-    for (int x = 1; x * R < L; ++x) {
-        rec = base + int64_t(x) * C::REC;
-#endif
-        const float ms = rec[0], ls = rec[1];
-        float mn, a, cc;
-        merge_scales(m, ms, mn, a, cc);
+    for (int j = 0; j < PER; ++j) O[j] = __ldg(rec + 4 + lane * PER + j);
+    // The records are folded one after another in ascending order; their
+    // loads are issued AHEAD at a time, ahead of the merges that use them,
+    // so that a long sequence does not pay one memory latency per split.
+    constexpr int AHEAD = 16;
+    for (int i0 = 0; i0 < count; i0 += AHEAD) {
+        float rm[AHEAD], rl[AHEAD], ro[AHEAD][PER];
 #pragma unroll
-        for (int j = 0; j < PER; ++j) O[j] = merge_val(O[j], a, rec[4 + lane * PER + j], cc);
-        l = merge_val(l, a, ls, cc);
-        m = mn;
+        for (int i = 0; i < AHEAD; ++i) {
+            if (i0 + i < count) {
+                const float *r = base + int64_t(rec0 + i0 + i) * C::REC;
+                rm[i] = __ldg(r);
+                rl[i] = __ldg(r + 1);
+#pragma unroll
+                for (int j = 0; j < PER; ++j) ro[i][j] = __ldg(r + 4 + lane * PER + j);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < AHEAD; ++i) {
+            if (i0 + i < count) {
+                float mn, a, cc;
+                merge_scales(m, rm[i], mn, a, cc);
+#pragma unroll
+                for (int j = 0; j < PER; ++j) O[j] = merge_val(O[j], a, ro[i][j], cc);
+                l = merge_val(l, a, rl[i], cc);
+                m = mn;
+            }
+        }
     }
     __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.o) + row * D + lane * PER;
 #pragma unroll
@@ -1102,7 +1076,9 @@ cudaError_t launch_attention(const CUtensorMap &tq, const AttnParams &p_in, int 
     AttnParams p = p_in;
     int64_t items;
     if (p.decode)
-        items = int64_t((p.max_splits + p.splits_per_cta - 1) / p.splits_per_cta) * p.Hkv * p.B;
+        items = int64_t(p.blocks_per_seq > 0 ? p.blocks_per_seq
+                                             : (p.max_splits + p.splits_per_cta - 1) / p.splits_per_cta) *
+                p.Hkv * p.B;
     else
         items = int64_t(p.num_q_tiles) * p.Hq * p.B;
     if (items > INT32_MAX) return cudaErrorInvalidValue;

@@ -69,7 +69,11 @@ struct BwdCfg {
     static constexpr int BLOCK_BYTES = (kKeyBlock / kPage) * PAGE_BYTES;  // 128 keys
     static constexpr int VEC_BYTES = 2 * kQTile * 4;           // lse2, Delta of 128 rows
     static constexpr int SLACK = 1024;
-    static constexpr int SMEM = SLACK + 2 * TILE_BYTES + 2 * BLOCK_BYTES + VEC_BYTES + 64;
+    // two buffers of what streams (q and dO tiles in the dk/dv kernel, key
+    // blocks in the dq kernel), one of what stays
+    static constexpr int SMEM = SLACK + 4 * TILE_BYTES + 2 * BLOCK_BYTES + 2 * VEC_BYTES + 64;
+    static_assert(4 * TILE_BYTES + 2 * BLOCK_BYTES == 2 * TILE_BYTES + 4 * BLOCK_BYTES,
+                  "both kernels fit the same shared-memory size");
     // TMEM columns: S (128), dP (128), two d-wide accumulators (dV, dK) or one (dQ)
     static constexpr uint32_t S_COL = 0, DP_COL = 128, ACC0 = 256, ACC1 = 256 + D;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -91,46 +95,58 @@ __device__ __forceinline__ uint32_t pack2(float a, float b)
     return *reinterpret_cast<uint32_t *>(&p);
 }
 
-// Rows row0 .. row0+127 of one head of a [T, H, D] bf16 tensor into a tile;
-// rows at or past `rows` are zero.
+// Rows row0 .. row0+127 of one head of a [T, H, D] bf16 tensor into a tile,
+// asynchronously (the caller commits and waits); rows at or past `rows` are
+// zero.  A warp moves blocks of 8 rows x 4 pieces (64 contiguous bytes of
+// each row: whole 32-byte sectors; the 8 threads of a store phase write 8
+// consecutive 16-byte cells of the tile: no bank conflict).
 template <int D>
-__device__ __forceinline__ void load_tile(uint8_t *tile, const uint4 *src, int64_t row0, int rows,
+__device__ __forceinline__ void copy_tile(uint8_t *tile, const uint4 *src, int64_t row0, int rows,
                                           int H, int h)
 {
-    constexpr int P = D / 8;
-    for (int e = threadIdx.x; e < kQTile * P; e += kBwdThreads) {
-        const int r = e % kQTile, c = e / kQTile;  // rows fastest: conflict-free stores
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r < rows) v = __ldg(src + ((row0 + r) * H + h) * P + c);
-        *reinterpret_cast<uint4 *>(tile + tile_off(r, c)) = v;
+    constexpr int P = D / 8;                         // 16-byte pieces of a row
+    constexpr int ITER = kQTile * P / kBwdThreads;   // pieces per thread
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+    for (int i = 0; i < ITER; ++i) {
+        const int blk = warp + 4 * i;                // blocks of 8 rows x 4 pieces
+        const int r = (blk % (kQTile / 8)) * 8 + (lane & 7);
+        const int c = (blk / (kQTile / 8)) * 4 + (lane >> 3);
+        const bool ok = r < rows;                    // (row 0 always exists)
+        cp_async16(tile + tile_off(r, c), src + ((row0 + (ok ? r : 0)) * H + h) * P + c, ok);
     }
 }
 
 // Keys k0 .. k0+127 of kv head g of one sequence (its page-table row `bt`)
-// into eight page blocks; keys at or past kv_len are zero.
+// into eight page blocks, asynchronously; keys at or past kv_len are zero.
 template <int D>
-__device__ __forceinline__ void load_keys(uint8_t *dst, const uint8_t *cache, const int32_t *bt,
+__device__ __forceinline__ void copy_keys(uint8_t *dst, const uint8_t *cache, const int32_t *bt,
                                           int k0, int kv_len, int Hkv, int g, int num_pages,
                                           unsigned *status)
 {
     using C = BwdCfg<D>;
     constexpr int PP = C::PAGE_BYTES / 16;  // 16-byte pieces of a page block
-    for (int e = threadIdx.x; e < (kKeyBlock / kPage) * PP; e += kBwdThreads) {
+    constexpr int ITER = (kKeyBlock / kPage) * PP / kBwdThreads;
+#pragma unroll
+    for (int i = 0; i < ITER; ++i) {
+        const int e = threadIdx.x + i * kBwdThreads;
         const int pg = e / PP, piece = e - pg * PP;
         const uint32_t off = uint32_t(piece) * 16u;
         // piece -> key: off = kg * 16D + c * 128 + r * 16
         const int kg = int(off / (D * 16)), r = int(off % 128) / 16;
         const int key = k0 + pg * kPage + kg * 8 + r;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        const uint8_t *src = cache;
+        bool ok = false;
         if (key < kv_len) {
             const int phys = __ldg(bt + (k0 / kPage + pg));
-            if (phys >= 0 && phys < num_pages)
-                v = __ldg(reinterpret_cast<const uint4 *>(
-                            cache + (int64_t(phys) * Hkv + g) * int64_t(C::PAGE_BYTES) + off));
-            else if (piece == 0)
+            if (phys >= 0 && phys < num_pages) {
+                src = cache + (int64_t(phys) * Hkv + g) * int64_t(C::PAGE_BYTES) + off;
+                ok = true;
+            } else if (piece == 0) {
                 record_status(status, BI_DEV_BAD_INDEX);
+            }
         }
-        *reinterpret_cast<uint4 *>(dst + pg * C::PAGE_BYTES + off) = v;
+        cp_async16(dst + pg * C::PAGE_BYTES + off, src, ok);
     }
 }
 
@@ -186,13 +202,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
-    uint8_t *sQ = smem;
-    uint8_t *sDO = sQ + C::TILE_BYTES;
-    uint8_t *sK = sDO + C::TILE_BYTES;
+    // q tiles [2], dO tiles [2] (the step's and the next step's), K, V
+    auto sQ = [&](int buf) { return smem + buf * C::TILE_BYTES; };
+    auto sDO = [&](int buf) { return smem + (2 + buf) * C::TILE_BYTES; };
+    uint8_t *sK = smem + 4 * C::TILE_BYTES;
     uint8_t *sV = sK + C::BLOCK_BYTES;
-    float *sLse = reinterpret_cast<float *>(sV + C::BLOCK_BYTES);
-    float *sDelta = sLse + kQTile;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sDelta + kQTile);
+    float *sLse = reinterpret_cast<float *>(sV + C::BLOCK_BYTES);  // [2][128]
+    float *sDelta = sLse + 2 * kQTile;                             // [2][128]
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sDelta + 2 * kQTile);
     uint64_t *drain = bar + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
@@ -211,6 +228,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
         return;
     }
 
+    // Steps j = hh * ntiles + qt: query head hh of the group (ascending),
+    // then the chunk's 128-row tile qt (ascending); a tile whose last row
+    // comes before this key block sees none of it and is skipped.
+    const int ntiles = (n + kQTile - 1) / kQTile;
+    const int nsteps = p.group * ntiles;
+    auto sees = [&](int j) {
+        const int qt = j % ntiles;
+        return ctx + min(n, (qt + 1) * kQTile) - 1 >= k0;
+    };
+    auto next_step = [&](int j) {
+        while (j < nsteps && !sees(j)) ++j;
+        return j;
+    };
+    // the step's tiles (async) and this thread's row of its lse2 / Delta
+    auto fetch = [&](int j, int buf, float &lse_r, float &delta_r) {
+        const int h = g * p.group + j / ntiles, qt = j % ntiles;
+        const int rows = min(kQTile, n - qt * kQTile);
+        const int64_t row0 = int64_t(q0) + int64_t(qt) * kQTile;
+        copy_tile<D>(sQ(buf), static_cast<const uint4 *>(p.q), row0, rows, p.Hq, h);
+        copy_tile<D>(sDO(buf), static_cast<const uint4 *>(p.dout), row0, rows, p.Hq, h);
+        cp_async_commit();
+        const int r = threadIdx.x;
+        lse_r = r < rows ? p.lse2[(row0 + r) * p.Hq + h] : 0.0f;
+        delta_r = r < rows ? p.delta[(row0 + r) * p.Hq + h] : 0.0f;
+    };
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         mbar_init(bar, 1);
@@ -223,11 +266,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
         tmem_relinquish();
     }
     const int32_t *bt = p.block_table + int64_t(b) * p.max_pages;
-    load_keys<D>(sK, static_cast<const uint8_t *>(p.k_cache), bt, k0, kv_len, p.Hkv, g,
+    copy_keys<D>(sK, static_cast<const uint8_t *>(p.k_cache), bt, k0, kv_len, p.Hkv, g,
                  p.num_pages, p.status);
-    load_keys<D>(sV, static_cast<const uint8_t *>(p.v_cache), bt, k0, kv_len, p.Hkv, g,
+    copy_keys<D>(sV, static_cast<const uint8_t *>(p.v_cache), bt, k0, kv_len, p.Hkv, g,
                  p.num_pages, p.status);
-    fence_proxy_async_smem();  // the key block is read by the tensor core
+    cp_async_commit();
+    int j = next_step(0);  // (the sequence's last row sees every key block of it)
+    float lse_r = 0.0f, delta_r = 0.0f;
+    fetch(j, 0, lse_r, delta_r);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -240,96 +286,93 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
     const uint32_t idesc_s = idesc_bf16_f32(128, kQTile, 0, 0);
     const uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
     const uint32_t kb_addr = smem_u32(sK), vb_addr = smem_u32(sV);
-    const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
     uint32_t phase = 0;
     bool ok = true, first = true;
-    const int ntiles = (n + kQTile - 1) / kQTile;
-    for (int hh = 0; ok && hh < p.group; ++hh) {
-        const int h = g * p.group + hh;
-        for (int qt = 0; ok && qt < ntiles; ++qt) {
-            const int rows = min(kQTile, n - qt * kQTile);
-            const int pos0 = ctx + qt * kQTile;
-            if (pos0 + rows - 1 < k0) continue;  // no row of the tile sees this block
-            // ------------------------------------------------ load the tile
-            load_tile<D>(sQ, static_cast<const uint4 *>(p.q), q0 + int64_t(qt) * kQTile, rows,
-                         p.Hq, h);
-            load_tile<D>(sDO, static_cast<const uint4 *>(p.dout), q0 + int64_t(qt) * kQTile, rows,
-                         p.Hq, h);
-            {
-                const int r = threadIdx.x;
-                const int64_t row = (int64_t(q0) + qt * kQTile + r) * p.Hq + h;
-                sLse[r] = r < rows ? p.lse2[row] : 0.0f;
-                sDelta[r] = r < rows ? p.delta[row] : 0.0f;
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            // ------------------------------------------------ S^T, dP^T
-            if (threadIdx.x == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < D / 16; ++k) {
-                    mma_ss(tmem + C::S_COL, sdesc_plain(kb_addr + 256 * k, 128, C::KGROUP_BYTES),
-                           sdesc_plain(q_addr + 4096 * k, 2048, 128), idesc_s, k > 0 ? 1u : 0u);
-                    mma_ss(tmem + C::DP_COL, sdesc_plain(vb_addr + 256 * k, 128, C::KGROUP_BYTES),
-                           sdesc_plain(do_addr + 4096 * k, 2048, 128), idesc_s, k > 0 ? 1u : 0u);
-                }
-                mma_commit(bar);
-            }
-            ok = block_wait(bar, phase, ctl);
-            phase ^= 1u;
-            if (!ok) break;
+    int buf = 0;
+    while (ok && j < nsteps) {
+        const int qt = j % ntiles;
+        const int rows = min(kQTile, n - qt * kQTile);
+        const int pos0 = ctx + qt * kQTile;
+        const uint32_t q_addr = smem_u32(sQ(buf)), do_addr = smem_u32(sDO(buf));
+        float *lse_s = sLse + buf * kQTile, *delta_s = sDelta + buf * kQTile;
+        lse_s[threadIdx.x] = lse_r;
+        delta_s[threadIdx.x] = delta_r;
+        cp_async_wait<0>();        // this step's tiles (and, first, the key block) landed
+        fence_proxy_async_smem();  // ... and are read by the tensor core
+        tc_fence_before();
+        __syncthreads();
+        // ------------------------------------------------ S^T, dP^T
+        if (threadIdx.x == 0) {
             tc_fence_after();
-            // ------------------------------------------------ P^T, dS^T (row = key)
-#pragma unroll 1
-            for (int c = 0; c < kQTile / 32; ++c) {
-                uint32_t s[32], dp[32];
-                tmem_ld32(lane_base + C::S_COL + 32 * c, s);
-                tmem_ld32(lane_base + C::DP_COL + 32 * c, dp);
-                tmem_wait_ld(s);
-                tmem_wait_ld(dp);
-                uint32_t pk[16], dk[16];
 #pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    float pv[2], dv[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int i = 32 * c + j + u;  // query column
-                        const bool vis = i < rows && key <= pos0 + i;
-                        const float pr = ex2(__fmaf_rn(__uint_as_float(s[j + u]), cs, -sLse[i]));
-                        const float ds = __fmul_rn(pr, __fsub_rn(__uint_as_float(dp[j + u]), sDelta[i]));
-                        pv[u] = vis ? pr : 0.0f;
-                        dv[u] = vis ? ds : 0.0f;
-                    }
-                    pk[j / 2] = pack2(pv[0], pv[1]);
-                    dk[j / 2] = pack2(dv[0], dv[1]);
-                }
-                tmem_st16(lane_base + C::S_COL + 16 * c, pk);
-                tmem_st16(lane_base + C::DP_COL + 16 * c, dk);
+            for (int k = 0; k < D / 16; ++k) {
+                mma_ss(tmem + C::S_COL, sdesc_plain(kb_addr + 256 * k, 128, C::KGROUP_BYTES),
+                       sdesc_plain(q_addr + 4096 * k, 2048, 128), idesc_s, k > 0 ? 1u : 0u);
+                mma_ss(tmem + C::DP_COL, sdesc_plain(vb_addr + 256 * k, 128, C::KGROUP_BYTES),
+                       sdesc_plain(do_addr + 4096 * k, 2048, 128), idesc_s, k > 0 ? 1u : 0u);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncthreads();
-            // ------------------------------------------------ dV += P^T dO, dK += dS^T Q
-            if (threadIdx.x == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int jj = 0; jj < kQTile / 16; ++jj) {
-                    const uint32_t acc = (first && jj == 0) ? 0u : 1u;
-                    mma_ts(tmem + C::ACC0, tmem + C::S_COL + 8 * jj,
-                           sdesc_plain(do_addr + 256 * jj, 128, 2048), idesc_acc, acc);
-                    mma_ts(tmem + C::ACC1, tmem + C::DP_COL + 8 * jj,
-                           sdesc_plain(q_addr + 256 * jj, 128, 2048), idesc_acc, acc);
-                }
-                mma_commit(bar);
-            }
-            first = false;
-            ok = block_wait(bar, phase, ctl);
-            phase ^= 1u;
-            if (!ok) break;
-            tc_fence_after();
+            mma_commit(bar);
         }
+        // the next step's tiles stream into the other buffer meanwhile (the
+        // previous step's products, which read it, have completed)
+        const int jn = next_step(j + 1);
+        if (jn < nsteps) fetch(jn, buf ^ 1, lse_r, delta_r);
+        ok = block_wait(bar, phase, ctl);
+        phase ^= 1u;
+        if (!ok) break;
+        tc_fence_after();
+        // ------------------------------------------------ P^T, dS^T (row = key)
+#pragma unroll 1
+        for (int c = 0; c < kQTile / 32; ++c) {
+            uint32_t sv[32], dp[32];
+            tmem_ld32(lane_base + C::S_COL + 32 * c, sv);
+            tmem_ld32(lane_base + C::DP_COL + 32 * c, dp);
+            tmem_wait_ld(sv);
+            tmem_wait_ld(dp);
+            uint32_t pk[16], dk[16];
+#pragma unroll
+            for (int jj = 0; jj < 32; jj += 2) {
+                float pv[2], dv[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int i = 32 * c + jj + u;  // query column
+                    const bool vis = i < rows && key <= pos0 + i;
+                    const float pr = ex2(__fmaf_rn(__uint_as_float(sv[jj + u]), cs, -lse_s[i]));
+                    const float ds = __fmul_rn(pr, __fsub_rn(__uint_as_float(dp[jj + u]), delta_s[i]));
+                    pv[u] = vis ? pr : 0.0f;
+                    dv[u] = vis ? ds : 0.0f;
+                }
+                pk[jj / 2] = pack2(pv[0], pv[1]);
+                dk[jj / 2] = pack2(dv[0], dv[1]);
+            }
+            tmem_st16(lane_base + C::S_COL + 16 * c, pk);
+            tmem_st16(lane_base + C::DP_COL + 16 * c, dk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        // ------------------------------------------------ dV += P^T dO, dK += dS^T Q
+        if (threadIdx.x == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int jj = 0; jj < kQTile / 16; ++jj) {
+                const uint32_t acc = (first && jj == 0) ? 0u : 1u;
+                mma_ts(tmem + C::ACC0, tmem + C::S_COL + 8 * jj,
+                       sdesc_plain(do_addr + 256 * jj, 128, 2048), idesc_acc, acc);
+                mma_ts(tmem + C::ACC1, tmem + C::DP_COL + 8 * jj,
+                       sdesc_plain(q_addr + 256 * jj, 128, 2048), idesc_acc, acc);
+            }
+            mma_commit(bar);
+        }
+        first = false;
+        ok = block_wait(bar, phase, ctl);
+        phase ^= 1u;
+        if (!ok) break;
+        tc_fence_after();
+        buf ^= 1;
+        j = jn;
     }
+    cp_async_wait<0>();  // no copy may still be landing when the block leaves
     if (!ok) {
         if (threadIdx.x == 0) {
             mma_commit(drain);
@@ -394,9 +437,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
     uint8_t *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
     uint8_t *sQ = smem;
     uint8_t *sDO = sQ + C::TILE_BYTES;
-    uint8_t *sK = sDO + C::TILE_BYTES;
-    uint8_t *sV = sK + C::BLOCK_BYTES;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sV + C::BLOCK_BYTES + C::VEC_BYTES);
+    // K blocks [2], V blocks [2]: the step's and the next step's
+    uint8_t *kv_base = sDO + C::TILE_BYTES;
+    auto sK = [&](int buf) { return kv_base + buf * C::BLOCK_BYTES; };
+    auto sV = [&](int buf) { return kv_base + (2 + buf) * C::BLOCK_BYTES; };
+    uint64_t *bar = reinterpret_cast<uint64_t *>(kv_base + 4 * C::BLOCK_BYTES + 2 * C::VEC_BYTES);
     uint64_t *drain = bar + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
@@ -429,8 +474,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
         tmem_relinquish();
     }
     const int64_t row0 = int64_t(q0) + qt * kQTile;
-    load_tile<D>(sQ, static_cast<const uint4 *>(p.q), row0, rows, p.Hq, h);
-    load_tile<D>(sDO, static_cast<const uint4 *>(p.dout), row0, rows, p.Hq, h);
+    const int32_t *bt = p.block_table + int64_t(b) * p.max_pages;
+    auto fetch = [&](int kb, int buf) {
+        copy_keys<D>(sK(buf), static_cast<const uint8_t *>(p.k_cache), bt, kb * kKeyBlock, kv_len,
+                     p.Hkv, g, p.num_pages, p.status);
+        copy_keys<D>(sV(buf), static_cast<const uint8_t *>(p.v_cache), bt, kb * kKeyBlock, kv_len,
+                     p.Hkv, g, p.num_pages, p.status);
+        cp_async_commit();
+    };
+    copy_tile<D>(sQ, static_cast<const uint4 *>(p.q), row0, rows, p.Hq, h);
+    copy_tile<D>(sDO, static_cast<const uint4 *>(p.dout), row0, rows, p.Hq, h);
+    fetch(0, 0);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -443,22 +497,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
     const float lse2 = row_ok ? p.lse2[(row0 + i) * p.Hq + h] : 0.0f;
     const float delta = row_ok ? p.delta[(row0 + i) * p.Hq + h] : 0.0f;
     const float cs = p.scale_log2;
-    const int32_t *bt = p.block_table + int64_t(b) * p.max_pages;
 
     const uint32_t idesc_s = idesc_bf16_f32(128, kKeyBlock, 0, 0);
     const uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
-    const uint32_t kb_addr = smem_u32(sK), vb_addr = smem_u32(sV);
     const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
     uint32_t phase = 0;
     bool ok = true;
     const int last_key = pos0 + rows - 1;  // the tile's last visible key
+    int buf = 0;
     for (int kb = 0; ok && kb * kKeyBlock <= last_key; ++kb) {
         const int k0 = kb * kKeyBlock;
-        // the previous block's dQ MMAs have completed (waited below)
-        load_keys<D>(sK, static_cast<const uint8_t *>(p.k_cache), bt, k0, kv_len, p.Hkv, g,
-                     p.num_pages, p.status);
-        load_keys<D>(sV, static_cast<const uint8_t *>(p.v_cache), bt, k0, kv_len, p.Hkv, g,
-                     p.num_pages, p.status);
+        const uint32_t kb_addr = smem_u32(sK(buf)), vb_addr = smem_u32(sV(buf));
+        cp_async_wait<0>();        // this block's keys (and, first, the tile) landed
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -473,6 +523,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
             }
             mma_commit(bar);
         }
+        // the next key block streams into the other buffer meanwhile (the
+        // previous block's products, which read it, have completed)
+        if ((kb + 1) * kKeyBlock <= last_key) fetch(kb + 1, buf ^ 1);
         ok = block_wait(bar, phase, ctl);
         phase ^= 1u;
         if (!ok) break;
@@ -480,10 +533,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
         // ---------------------------------------------------- dS (row = query)
 #pragma unroll 1
         for (int c = 0; c < kKeyBlock / 32; ++c) {
-            uint32_t s[32], dp[32];
-            tmem_ld32(lane_base + C::S_COL + 32 * c, s);
+            uint32_t sv[32], dp[32];
+            tmem_ld32(lane_base + C::S_COL + 32 * c, sv);
             tmem_ld32(lane_base + C::DP_COL + 32 * c, dp);
-            tmem_wait_ld(s);
+            tmem_wait_ld(sv);
             tmem_wait_ld(dp);
             uint32_t dk[16];
 #pragma unroll
@@ -493,7 +546,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
                 for (int u = 0; u < 2; ++u) {
                     const int key = k0 + 32 * c + j + u;
                     const bool vis = row_ok && key <= t;
-                    const float pr = ex2(__fmaf_rn(__uint_as_float(s[j + u]), cs, -lse2));
+                    const float pr = ex2(__fmaf_rn(__uint_as_float(sv[j + u]), cs, -lse2));
                     const float ds = __fmul_rn(pr, __fsub_rn(__uint_as_float(dp[j + u]), delta));
                     dv[u] = vis ? ds : 0.0f;
                 }
@@ -518,7 +571,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
         phase ^= 1u;
         if (!ok) break;
         tc_fence_after();
+        buf ^= 1;
     }
+    cp_async_wait<0>();  // no copy may still be landing when the block leaves
     if (!ok) {
         if (threadIdx.x == 0) {
             mma_commit(drain);

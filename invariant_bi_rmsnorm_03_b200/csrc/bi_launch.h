@@ -109,7 +109,9 @@ struct AttnParams {
     const int32_t *order;      // decode: launch order of the sequences (or null)
     const int32_t *cu_q;       // prefill
     const int32_t *ctx_lens;   // prefill
-    int32_t splits_per_cta;    // decode work division
+    int32_t splits_per_cta;    // decode work division: splits per block (uniform) ...
+    int32_t blocks_per_seq;    // ... or, if > 0, this many blocks per sequence, each of
+                               // ceil(its splits / blocks_per_seq) splits
     int32_t max_splits;        // decode: splits of the longest sequence
     int32_t num_q_tiles;       // prefill: tiles of the longest chunk
     int32_t items;             // work items of the launch (set by launch_attention)

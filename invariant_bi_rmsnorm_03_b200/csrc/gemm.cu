@@ -566,20 +566,23 @@ int gemm_k_splits(int64_t M, int64_t N, int64_t K, int num_sms)
     // count that minimises a simple time model: the K slices the busiest
     // pair walks (waves x slices per split, ~0.6 us a slice, measured on a
     // B200 at M = 256) plus one pass of the fp32 partial sums out to memory
-    // and back (~6.5 TB/s).
+    // and back (~6.5 TB/s) and the reduction's launch (~3 us); taken only
+    // when the model saves a fifth or more.
     const int64_t tiles = ((M + pair::BM - 1) / pair::BM) * ((N + pair::BN - 1) / pair::BN);
     const int64_t kblocks = (K + pair::BK - 1) / pair::BK;
     const int64_t pairs = num_sms / 2;
     if (tiles >= pairs || kblocks < 8 || pairs < 1) return 1;
-    const double slice_us = 0.6, bytes_per_us = 6.5e6;
+    const double slice_us = 0.6, bytes_per_us = 6.5e6, reduce_us = 3.0;
+    const double whole_us = double(kblocks) * slice_us;  // one wave of whole-K tiles
     int64_t best = 1;
-    double best_us = double(kblocks) * slice_us;  // one wave of whole-K tiles
+    double best_us = 0.8 * whole_us;
     for (int64_t ks = 2; ks <= 16 && ks <= kblocks / 4; ++ks) {
         const int64_t per = (kblocks + ks - 1) / ks;
         const int64_t splits = (kblocks + per - 1) / per;
         const int64_t waves = (tiles * splits + pairs - 1) / pairs;
         const double us = double(waves * per) * slice_us +
-                          2.0 * double(splits) * double(M) * double(N) * 4.0 / bytes_per_us;
+                          2.0 * double(splits) * double(M) * double(N) * 4.0 / bytes_per_us +
+                          reduce_us;
         if (us < best_us) {
             best = splits;
             best_us = us;
