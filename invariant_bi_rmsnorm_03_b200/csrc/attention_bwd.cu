@@ -19,15 +19,15 @@
 //                          for each query head of the group (ascending) and
 //                          each 128-row query tile (ascending):
 //                            S^T = K Q^T,  dP^T = V dO^T        (tcgen05)
-//                            P^T, dS^T elementwise (one key row per thread)
+//                            P^T, dS^T elementwise (a key row per TMEM lane)
 //                            dV += P^T dO,  dK += dS^T Q         (P^T, dS^T
 //                                                                 from TMEM)
 //                          so a key's dk and dv are sums in one fixed order
 //                          over its own sequence's rows.
 //   attn_bwd_dq_kernel     one block per (sequence, query head, 128-row tile):
 //                          for each 128-key block ascending:
-//                            S = Q K^T,  dP = dO V^T;  P, dS elementwise (one
-//                            query row per thread);  dQ += dS K.
+//                            S = Q K^T,  dP = dO V^T;  P, dS elementwise (a
+//                            query row per TMEM lane);  dQ += dS K.
 //                          A row's dq depends on that row alone.
 // P and dS are rounded to bf16 to enter the tensor core (as the forward
 // rounds P before P V); every other quantity is fp32.
@@ -35,14 +35,16 @@
 // Shared-memory operands are in the tensor core's no-swizzle core-matrix
 // layout (8 rows x 16 bytes = 128 contiguous bytes): a 128-row tile of q or dO
 // as [value block d/8][row 128][8 values], a 128-key block of the cache as its
-// eight page blocks, already in that layout.  Every tile is loaded by the
-// threads with 16-byte loads (rows outside the sequence or the chunk become
-// zeros), so that a masked product never meets a stale NaN.
+// eight page blocks, already in that layout.  Every tile is copied by the
+// threads with 16-byte asynchronous copies (cp.async; rows outside the
+// sequence or the chunk become zeros, so that a masked product never meets
+// a stale NaN) into a second buffer while the current step computes.
 //
-// Block of 128 threads (4 warps; warp w owns TMEM lanes 32w .. 32w+31).
-// Thread 0 issues the MMAs; every wait is bounded and its outcome is agreed
-// on by the whole block (__syncthreads_and), so that a timeout ends every
-// thread's loop at the same point.
+// Block of 256 threads (8 warps; warps w and w + 4 share TMEM lanes
+// 32(w%4) .. +31, each taking half of the columns).  Thread 0 issues the
+// MMAs; every wait is bounded and its outcome is agreed on by the whole
+// block (__syncthreads_and), so that a timeout ends every thread's loop at
+// the same point.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -56,7 +58,7 @@
 namespace bi {
 namespace {
 
-constexpr int kBwdThreads = 128;
+constexpr int kBwdThreads = 256;  // 8 warps: two per TMEM lane quarter
 constexpr int kKeyBlock = 128;  // keys per block of the dk/dv kernel and per step of dq
 constexpr int kQTile = 128;     // query rows per tile
 constexpr float kLog2e = 1.4426950408889634f;
@@ -78,6 +80,17 @@ struct BwdCfg {
     static constexpr uint32_t S_COL = 0, DP_COL = 128, ACC0 = 256, ACC1 = 256 + D;
     static constexpr uint32_t TMEM_COLS = 512;
 };
+
+// The two warps of a TMEM lane quarter each turn half of the 128 fp32
+// columns of S (or dP) into bf16 pairs and store them back in place.  Chunk c
+// (columns 32c .. 32c+31) packs into 16 columns inside its own half
+// [64 (c/2), 64 (c/2) + 64), which only that half's warp reads, and only
+// after it has read them: one warp never overwrites a column the other has
+// still to read.  packed_step_col(j) is where values 16 j .. 16 j + 15 (the
+// K step j of the product that reads them) start.
+static_assert(kQTile == 128 && kKeyBlock == 128, "four 32-column chunks, two per half");
+__device__ __forceinline__ uint32_t packed_chunk_col(int c) { return 64u * (c >> 1) + 16u * (c & 1); }
+__device__ __forceinline__ uint32_t packed_step_col(int j) { return 64u * (j >> 2) + 8u * (j & 3); }
 
 // Byte offset of values 8c .. 8c+7 of row r in a 128-row tile.
 __device__ __forceinline__ uint32_t tile_off(int r, int c) { return (uint32_t(c) * 128u + r) * 16u; }
@@ -109,7 +122,7 @@ __device__ __forceinline__ void copy_tile(uint8_t *tile, const uint4 *src, int64
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
     for (int i = 0; i < ITER; ++i) {
-        const int blk = warp + 4 * i;                // blocks of 8 rows x 4 pieces
+        const int blk = warp + (kBwdThreads / 32) * i;  // blocks of 8 rows x 4 pieces
         const int r = (blk % (kQTile / 8)) * 8 + (lane & 7);
         const int c = (blk / (kQTile / 8)) * 4 + (lane >> 3);
         const bool ok = r < rows;                    // (row 0 always exists)
@@ -249,7 +262,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
         copy_tile<D>(sQ(buf), static_cast<const uint4 *>(p.q), row0, rows, p.Hq, h);
         copy_tile<D>(sDO(buf), static_cast<const uint4 *>(p.dout), row0, rows, p.Hq, h);
         cp_async_commit();
-        const int r = threadIdx.x;
+        const int r = threadIdx.x;  // threads 0..127: one row each
         lse_r = r < rows ? p.lse2[(row0 + r) * p.Hq + h] : 0.0f;
         delta_r = r < rows ? p.delta[(row0 + r) * p.Hq + h] : 0.0f;
     };
@@ -279,8 +292,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
-    const uint32_t lane_base = tmem_addr(tmem, 32 * warp, 0);
-    const int key = k0 + 32 * warp + lane;  // this thread's key (TMEM lane)
+    // warps w and w + 4 share TMEM lane quarter w % 4, each taking half of
+    // the columns
+    const int quarter = warp & 3, half = warp >> 2;
+    const uint32_t lane_base = tmem_addr(tmem, 32 * quarter, 0);
+    const int key = k0 + 32 * quarter + lane;  // this thread's key (TMEM lane)
     const float cs = p.scale_log2;
 
     const uint32_t idesc_s = idesc_bf16_f32(128, kQTile, 0, 0);
@@ -295,8 +311,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
         const int pos0 = ctx + qt * kQTile;
         const uint32_t q_addr = smem_u32(sQ(buf)), do_addr = smem_u32(sDO(buf));
         float *lse_s = sLse + buf * kQTile, *delta_s = sDelta + buf * kQTile;
-        lse_s[threadIdx.x] = lse_r;
-        delta_s[threadIdx.x] = delta_r;
+        if (threadIdx.x < kQTile) {
+            lse_s[threadIdx.x] = lse_r;
+            delta_s[threadIdx.x] = delta_r;
+        }
         cp_async_wait<0>();        // this step's tiles (and, first, the key block) landed
         fence_proxy_async_smem();  // ... and are read by the tensor core
         tc_fence_before();
@@ -323,7 +341,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
         tc_fence_after();
         // ------------------------------------------------ P^T, dS^T (row = key)
 #pragma unroll 1
-        for (int c = 0; c < kQTile / 32; ++c) {
+        for (int c = half * (kQTile / 64); c < (half + 1) * (kQTile / 64); ++c) {
             uint32_t sv[32], dp[32];
             tmem_ld32(lane_base + C::S_COL + 32 * c, sv);
             tmem_ld32(lane_base + C::DP_COL + 32 * c, dp);
@@ -345,8 +363,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
                 pk[jj / 2] = pack2(pv[0], pv[1]);
                 dk[jj / 2] = pack2(dv[0], dv[1]);
             }
-            tmem_st16(lane_base + C::S_COL + 16 * c, pk);
-            tmem_st16(lane_base + C::DP_COL + 16 * c, dk);
+            tmem_st16(lane_base + C::S_COL + packed_chunk_col(c), pk);
+            tmem_st16(lane_base + C::DP_COL + packed_chunk_col(c), dk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -357,9 +375,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
 #pragma unroll
             for (int jj = 0; jj < kQTile / 16; ++jj) {
                 const uint32_t acc = (first && jj == 0) ? 0u : 1u;
-                mma_ts(tmem + C::ACC0, tmem + C::S_COL + 8 * jj,
+                mma_ts(tmem + C::ACC0, tmem + C::S_COL + packed_step_col(jj),
                        sdesc_plain(do_addr + 256 * jj, 128, 2048), idesc_acc, acc);
-                mma_ts(tmem + C::ACC1, tmem + C::DP_COL + 8 * jj,
+                mma_ts(tmem + C::ACC1, tmem + C::DP_COL + packed_step_col(jj),
                        sdesc_plain(q_addr + 256 * jj, 128, 2048), idesc_acc, acc);
             }
             mma_commit(bar);
@@ -395,7 +413,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
             const float mul = which ? p.scale : 1.0f;
             const uint32_t col = which ? C::ACC1 : C::ACC0;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
                 uint32_t a[32];
                 tmem_ld32(lane_base + col + 32 * c, a);
                 tmem_wait_ld(a);
@@ -490,8 +508,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
-    const uint32_t lane_base = tmem_addr(tmem, 32 * warp, 0);
-    const int i = 32 * warp + lane;  // this thread's query row (TMEM lane)
+    // warps w and w + 4 share TMEM lane quarter w % 4, each taking half of
+    // the columns
+    const int quarter = warp & 3, half = warp >> 2;
+    const uint32_t lane_base = tmem_addr(tmem, 32 * quarter, 0);
+    const int i = 32 * quarter + lane;  // this thread's query row (TMEM lane)
     const bool row_ok = i < rows;
     const int t = pos0 + i;          // its absolute position
     const float lse2 = row_ok ? p.lse2[(row0 + i) * p.Hq + h] : 0.0f;
@@ -532,7 +553,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
         tc_fence_after();
         // ---------------------------------------------------- dS (row = query)
 #pragma unroll 1
-        for (int c = 0; c < kKeyBlock / 32; ++c) {
+        for (int c = half * (kKeyBlock / 64); c < (half + 1) * (kKeyBlock / 64); ++c) {
             uint32_t sv[32], dp[32];
             tmem_ld32(lane_base + C::S_COL + 32 * c, sv);
             tmem_ld32(lane_base + C::DP_COL + 32 * c, dp);
@@ -552,7 +573,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
                 }
                 dk[j / 2] = pack2(dv[0], dv[1]);
             }
-            tmem_st16(lane_base + C::S_COL + 16 * c, dk);
+            tmem_st16(lane_base + C::S_COL + packed_chunk_col(c), dk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -562,7 +583,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
             tc_fence_after();
 #pragma unroll
             for (int jj = 0; jj < kKeyBlock / 16; ++jj)
-                mma_ts(tmem + C::ACC0, tmem + C::S_COL + 8 * jj,
+                mma_ts(tmem + C::ACC0, tmem + C::S_COL + packed_step_col(jj),
                        sdesc_plain(kb_addr + jj * C::PAGE_BYTES, C::KGROUP_BYTES, 128), idesc_acc,
                        (kb > 0 || jj > 0) ? 1u : 0u);
             mma_commit(bar);
@@ -584,7 +605,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
         // chunk store nothing
         __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dq) + ((row0 + i) * p.Hq + h) * D;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
             uint32_t a[32];
             tmem_ld32(lane_base + C::ACC0 + 32 * c, a);
             tmem_wait_ld(a);
