@@ -33,7 +33,7 @@
 // split, with the same merge function.  The bits therefore do not depend on
 // how many blocks served a sequence.
 //
-// Block of 448 threads, one per SM (about 225 KB shared memory; 512 TMEM
+// Block of 640 threads, one per SM (about 225 KB shared memory; 512 TMEM
 // columns as two 256-column buffers, each holding a split's logits, then
 // its P in columns 0-127 and O_s in columns 128-255):
 //   warp 0     producer: Q by TMA once; per split the 16 pages of K and of
@@ -45,13 +45,15 @@
 //              for the partial page) so that 0 * stale never reaches O.
 //   warp 1     TMEM allocation and MMA issue (one thread): QK^T of split
 //              s+1 runs while split s is in softmax (double-buffered TMEM).
-//   warps 4-7  softmax of one split; warp w owns TMEM lanes 32(w%4)..+31.
-//              Decode spreads the query heads over the four lane quarters,
-//              and with at most 8 heads per quarter four threads share a
-//              row (softmax_heads16).
-//   warps 2,3,8-13  merge ("fold") of O_s into the running output, two per
-//              lane quarter (one per half of the head dim), overlapping the
-//              next split's softmax.
+//   warps 4-7, 16-19  softmax of one split, two warps per TMEM lane
+//              quarter (warp w may only reach lanes 32(w%4)..+31): warps
+//              4-7 take the first 16 lanes of their quarter, 16-19 the last
+//              16, four threads a row (softmax_lanes16).  Decode spreads the
+//              query heads over the four lane quarters.
+//   warps 8-15 merge ("fold") of O_s into the running output, two per lane
+//              quarter (one per half of the head dim), overlapping the next
+//              split's softmax; warps 2-3 idle (they fill the producer's
+//              warpgroup, whose registers go to the fold warps).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -65,10 +67,21 @@
 namespace bi {
 namespace {
 
-// Warp roles: 0 producer, 1 MMA, 4-7 softmax, 2-3 and 8-13 merge ("fold").
-// Softmax warp w and fold warp w' own TMEM lane quarter w % 4; fold warps
-// 2, 3, 8, 9 take the first half of the head dim, 10-13 the second.
-constexpr int THREADS = 448;
+// Warp roles, by warpgroup (four warps): group 0 = producer (warp 0), MMA
+// (warp 1) and two idle warps; group 1 (warps 4-7) and group 4 (16-19)
+// softmax; groups 2 and 3 (warps 8-15) merge ("fold").  Softmax and fold
+// warp w serve TMEM lane quarter w % 4; softmax warps 4-7 take lanes 0-15 of
+// their quarter, 16-19 lanes 16-31; fold warps 8-11 take the first half of
+// the head dim, 12-15 the second.  The block is launched with 96 registers a
+// thread; group 0 gives back all but kRegsCtl and the fold groups take
+// kRegsFold (setmaxnreg), so that a fold thread holds its half row of the
+// output in registers:
+//   128 (kRegsCtl + 96 + 2 kRegsFold + 96) <= 640 * 96.
+constexpr int THREADS = 640;
+constexpr int kLaunchRegs = 96;
+constexpr int kRegsCtl = 56, kRegsFold = 104;
+static_assert(128 * (kRegsCtl + 2 * kLaunchRegs + 2 * kRegsFold) <= THREADS * kLaunchRegs,
+              "the register split must fit the block's launch allocation");
 constexpr int kFoldThreads = 256;
 constexpr float kLn2 = 0.693147180559945309f;
 
@@ -294,183 +307,138 @@ __device__ __forceinline__ float logit(float s, float cs, float m_s)
     return ex2(__fmaf_rn(s, cs, -m_s));
 }
 
-// Maximum of the visible logits of 32 keys kc .. kc+31.
-__device__ __forceinline__ void chunk_max(const uint32_t (&r)[32], int kc, int t, float (&mx)[8])
-{
-    if (kc + 31 <= t) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[j]));
-    } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-            if (kc + j <= t) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(r[j]));
-    }
-}
-
-// p of the 32 keys kc .. kc+31, computed in place (r[j] becomes the bits of
-// p_j): packed bf16 P written to TMEM at `pcol` (16 columns), the class sums
-// S_u advanced by this chunk in the order of tree8.
-__device__ __forceinline__ void chunk_exp(uint32_t (&r)[32], int kc, int t, float cs, float m_s,
-                                          uint32_t pcol, float (&S)[4])
-{
-    if (kc + 31 <= t) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(logit(__uint_as_float(r[j]), cs, m_s));
-    } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-            r[j] = (kc + j <= t) ? __float_as_uint(logit(__uint_as_float(r[j]), cs, m_s)) : 0u;
-    }
-    uint32_t pk[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-        pk[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-    tmem_st16(pcol, pk);
-    auto e = [&](int j) { return __uint_as_float(r[j]); };
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-        S[u] = __fadd_rn(S[u], tree8(e(2 * u), e(2 * u + 1), e(8 + 2 * u), e(9 + 2 * u),
-                                     e(16 + 2 * u), e(17 + 2 * u), e(24 + 2 * u), e(25 + 2 * u)));
-}
-
-// Softmax of one split, one row per thread (any row layout; used by
-// prefill and by decode with more than 8 query rows per lane quarter).
-// S is read from TMEM columns sb .. sb+255 in two passes of 32-column
-// loads, the next load in flight while a chunk is processed; P (bf16 pairs)
-// is written over columns sb .. sb+127 as the second pass goes (each store
-// lands on columns this thread has already read).  Returns m_s (scaled,
-// log2 units) and l_s.  (P V cannot start before the whole pass is done: it
-// writes O_s over the logits of keys 128..255.)
-__device__ __forceinline__ void softmax_rows(uint32_t sb, int k0, int t, float cs, float &m_s,
-                                             float &l_s)
+// Softmax of one split for 16 TMEM lanes of a lane quarter (one warp; the
+// quarter's other 16 lanes belong to its second softmax warp).  Thread
+// t = u + 4 v holds rows v and v + 8 of the 16 lanes and, of each row and
+// each 32-key chunk c, the keys 32c + 8i + 2u and 32c + 8i + 2u + 1 (i < 4)
+// -- class u of the order above -- read with the 16-lane TMEM shape, a chunk
+// a load, the next load in flight.  Pass 1 takes the row maximum (exact in
+// any order; four accumulators a row break the chain, two xor shuffles join
+// the row's four threads).  Pass 2 computes p, writes the chunk's packed P
+// (P column 16c + 4i + u, the matching 16-lane store) over columns this warp
+// has already read, and adds the chunk's eight class-u values to the class
+// sum as tree8 does; the two xor shuffles at the end give
+// (S_u + S_u^1) + (S_u^2 + S_u^3), which commutativity makes
+// (S_0 + S_1) + (S_2 + S_3) on every thread.  So a row's m_s, l_s and P have
+// the same bits whichever lanes and warp hold the row.  sb is the TMEM
+// address of the first of the 16 lanes at the buffer's first column; t_lo
+// and t_hi are the last visible keys of rows v and v + 8; HI says whether
+// rows 8..15 are computed.  A chunk whose 32 keys every row of the thread
+// sees takes a path without masks.
+template <bool HI>
+__device__ __forceinline__ void softmax_lanes16(uint32_t sb, int k0, int t_lo, int t_hi, float cs,
+                                                float (&m_s)[2], float (&l_s)[2])
 {
     constexpr int NC = kSplit / 32;  // 32-key chunks
-    // pass 1: maximum of the raw logits over the visible keys.  For c > 0,
-    // x -> round(x * c) is monotonic, so max_j round(S_j c) = round(max_j S_j * c).
-    // (A maximum is exact in any order; eight accumulators break the chain.)
-    float mx[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-    // The loops are kept rolled (two loads of each kind per trip): a small
-    // instruction footprint matters more here than unrolling, since the
-    // block's other warps run other code on the same sub-partitions.
-    {
-        // 32-column loads, the next in flight while a chunk is scanned
-        uint32_t ra[32], rb[32];
-        tmem_ld32(sb, ra);
-#pragma unroll 1
-        for (int c = 0; c < NC; c += 2) {
-            tmem_wait_ld(ra);
-            tmem_ld32(sb + 32 * (c + 1), rb);
-            chunk_max(ra, k0 + 32 * c, t, mx);
-            tmem_wait_ld(rb);
-            if (c + 2 < NC) tmem_ld32(sb + 32 * (c + 2), ra);
-            chunk_max(rb, k0 + 32 * (c + 1), t, mx);
-        }
-    }
-    const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-    m_s = __fmul_rn(mraw, cs);
-    // pass 2: p = 2^(S c - m_s), masked keys 0; P into TMEM; the sum in the
-    // order of tree8.  32-key chunks, the next chunk's load in flight.
-    float S[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    uint32_t ra[32], rb[32];
-    tmem_ld32(sb, ra);
-#pragma unroll 1
-    for (int c = 0; c < NC; c += 2) {
-        tmem_wait_ld(ra);
-        tmem_ld32(sb + 32 * (c + 1), rb);
-        chunk_exp(ra, k0 + 32 * c, t, cs, m_s, sb + 16 * c, S);
-        tmem_wait_ld(rb);
-        if (c + 2 < NC) tmem_ld32(sb + 32 * (c + 2), ra);
-        chunk_exp(rb, k0 + 32 * (c + 1), t, cs, m_s, sb + 16 * (c + 1), S);
-    }
-    tmem_wait_st();
-    l_s = __fadd_rn(__fadd_rn(S[0], S[1]), __fadd_rn(S[2], S[3]));
-}
-
-// Softmax of one split for decode when the query rows of this lane quarter
-// sit in its lanes 0..7: four threads share a row.  Thread t = u + 4 v
-// handles lane v, keys 8m + 2u and 8m + 2u + 1 (m < 32) -- class u of the
-// order above -- read with the 16-lane TMEM shape (64 keys a load, the next
-// load in flight), and writes the packed P of those keys (P column 4m + u)
-// with the matching 16-lane store.  The arithmetic per row is the same as
-// softmax_rows, so the bits are equal.  sb is the TMEM address of lane 0 of
-// the quarter.
-__device__ __forceinline__ void softmax_heads16(uint32_t sb, int k0, int t, float cs, float &m_s,
-                                                float &l_s)
-{
     const int u = threadIdx.x & 3;
-    const bool whole = k0 + kSplit - 1 <= t;  // every key of the split visible
-    // r[4m'], r[4m'+1] of load k: keys 8m + 2u, 8m + 2u + 1 with m = 8k + m'
-    auto vis = [&](int m, int j) { return whole || k0 + 8 * m + 2 * u + j <= t; };
-    uint32_t ra[32], rb[32];
-    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-    auto load_max = [&](const uint32_t (&r)[32], int k) {
+    // last key visible to both of this thread's rows; a chunk whose keys all
+    // come at or before it takes the path without masks
+    const int t_min = HI ? min(t_lo, t_hi) : t_lo;
+    // r[4 i + 2 h + j] of chunk c: key k0 + 32 c + 8 i + 2 u + j of row h
+    auto key = [&](int c, int i, int j) { return k0 + 32 * c + 8 * i + 2 * u + j; };
+    auto whole = [&](int c) { return k0 + 32 * c + 31 <= t_min; };
+    float mx[2][4];
 #pragma unroll
-        for (int mm = 0; mm < 8; ++mm)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int m = 8 * k + mm;
-                if (vis(m, j)) mx[m & 3] = fmaxf(mx[m & 3], __uint_as_float(r[4 * mm + j]));
-            }
-    };
-    // loops kept rolled (small instruction footprint): the load just
-    // waited for is moved to `ra` and the next one issued into `rb`
-    tmem_ld_16x256b_x8(sb, rb);
-#pragma unroll 1
-    for (int k = 0; k < 4; ++k) {
-        tmem_wait_ld(rb);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) ra[j] = rb[j];
-        if (k + 1 < 4) tmem_ld_16x256b_x8(sb + 64 * (k + 1), rb);
-        load_max(ra, k);
-    }
-    float mraw = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-    mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 1));
-    mraw = fmaxf(mraw, __shfl_xor_sync(0xffffffffu, mraw, 2));
-    m_s = __fmul_rn(mraw, cs);
-
-    // Load k covers 32-key chunks 2k and 2k + 1; its P goes to columns
-    // 32k .. 32k + 31 of the quarter's lanes 0..7.
-    float S = 0.0f;
-    auto load_exp = [&](const uint32_t (&r)[32], int k) {
-        uint32_t pk[16];  // 16x128b.x8 store operands: [2 m' + lane-half]
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            float e[8];
+    for (int i = 0; i < 4; ++i) mx[0][i] = mx[1][i] = -INFINITY;
+    auto chunk_max = [&](const uint32_t (&r)[16], int c) {
+        if (whole(c)) {
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int mm = 4 * cc + i, m = 8 * k + mm;
-                    const float x = logit(__uint_as_float(r[4 * mm + j]), cs, m_s);
-                    e[2 * i + j] = vis(m, j) ? x : 0.0f;
+                    mx[0][i] = fmaxf(mx[0][i], __uint_as_float(r[4 * i + j]));
+                    if (HI) mx[1][i] = fmaxf(mx[1][i], __uint_as_float(r[4 * i + 2 + j]));
                 }
-            S = __fadd_rn(S, tree8(e[0], e[1], e[2], e[3], e[4], e[5], e[6], e[7]));
+        } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                pk[2 * (4 * cc + i)] = pack_bf16x2(e[2 * i], e[2 * i + 1]);
-                pk[2 * (4 * cc + i) + 1] = 0u;  // lanes 8..15 hold no query row
-            }
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int kj = key(c, i, j);
+                    if (kj <= t_lo) mx[0][i] = fmaxf(mx[0][i], __uint_as_float(r[4 * i + j]));
+                    if (HI && kj <= t_hi)
+                        mx[1][i] = fmaxf(mx[1][i], __uint_as_float(r[4 * i + 2 + j]));
+                }
         }
-        tmem_st_16x128b_x8(sb + 32 * k, pk);
     };
-    tmem_ld_16x256b_x8(sb, rb);
+    // loops kept rolled (a small instruction footprint: the block's other
+    // warps run other code on the same sub-partitions), two chunks a trip
+    uint32_t ra[16], rb[16];
+    tmem_ld_16x256b_x4(sb, ra);
 #pragma unroll 1
-    for (int k = 0; k < 4; ++k) {
-        tmem_wait_ld(rb);
+    for (int c = 0; c < NC; c += 2) {
+        tmem_wait_ld16(ra);
+        tmem_ld_16x256b_x4(sb + 32 * (c + 1), rb);
+        chunk_max(ra, c);
+        tmem_wait_ld16(rb);
+        if (c + 2 < NC) tmem_ld_16x256b_x4(sb + 32 * (c + 2), ra);
+        chunk_max(rb, c + 1);
+    }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) ra[j] = rb[j];
-        if (k + 1 < 4) tmem_ld_16x256b_x8(sb + 64 * (k + 1), rb);
-        load_exp(ra, k);
+    for (int h = 0; h < 2; ++h) {
+        float mr = fmaxf(fmaxf(mx[h][0], mx[h][1]), fmaxf(mx[h][2], mx[h][3]));
+        mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, 1));
+        mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, 2));
+        m_s[h] = __fmul_rn(mr, cs);
+    }
+
+    // Chunk c's P goes to columns 16c .. 16c + 15, which the loads of chunks
+    // c/2 .. c have read (waited for); the load in flight reads columns from
+    // 32(c + 1) on.
+    float S[2] = {0.0f, 0.0f};
+    auto chunk_exp = [&](const uint32_t (&r)[16], int c) {
+        float e0[8], e1[8];
+        if (whole(c)) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    e0[2 * i + j] = logit(__uint_as_float(r[4 * i + j]), cs, m_s[0]);
+                    e1[2 * i + j] = HI ? logit(__uint_as_float(r[4 * i + 2 + j]), cs, m_s[1]) : 0.0f;
+                }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int kj = key(c, i, j);
+                    const float x0 = logit(__uint_as_float(r[4 * i + j]), cs, m_s[0]);
+                    e0[2 * i + j] = kj <= t_lo ? x0 : 0.0f;
+                    e1[2 * i + j] = 0.0f;
+                    if (HI) {
+                        const float x1 = logit(__uint_as_float(r[4 * i + 2 + j]), cs, m_s[1]);
+                        e1[2 * i + j] = kj <= t_hi ? x1 : 0.0f;
+                    }
+                }
+        }
+        S[0] = __fadd_rn(S[0], tree8(e0[0], e0[1], e0[2], e0[3], e0[4], e0[5], e0[6], e0[7]));
+        if (HI) S[1] = __fadd_rn(S[1], tree8(e1[0], e1[1], e1[2], e1[3], e1[4], e1[5], e1[6], e1[7]));
+        uint32_t pk[8];  // 16x128b.x4 store operands: [2 i + row h]
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            pk[2 * i] = pack_bf16x2(e0[2 * i], e0[2 * i + 1]);
+            pk[2 * i + 1] = HI ? pack_bf16x2(e1[2 * i], e1[2 * i + 1]) : 0u;
+        }
+        __syncwarp();  // the rows of a warp may have taken different paths
+        tmem_st_16x128b_x4(sb + 16 * c, pk);
+    };
+    tmem_ld_16x256b_x4(sb, ra);
+#pragma unroll 1
+    for (int c = 0; c < NC; c += 2) {
+        tmem_wait_ld16(ra);
+        tmem_ld_16x256b_x4(sb + 32 * (c + 1), rb);
+        chunk_exp(ra, c);
+        tmem_wait_ld16(rb);
+        if (c + 2 < NC) tmem_ld_16x256b_x4(sb + 32 * (c + 2), ra);
+        chunk_exp(rb, c + 1);
     }
     tmem_wait_st();
-    // (S_u + S_u^1) + (S_u^2 + S_u^3): commutativity gives every thread the
-    // same bits.
-    S = __fadd_rn(S, __shfl_xor_sync(0xffffffffu, S, 1));
-    S = __fadd_rn(S, __shfl_xor_sync(0xffffffffu, S, 2));
-    l_s = S;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        S[h] = __fadd_rn(S[h], __shfl_xor_sync(0xffffffffu, S[h], 1));
+        S[h] = __fadd_rn(S[h], __shfl_xor_sync(0xffffffffu, S[h], 2));
+        l_s[h] = S[h];
+    }
 }
 
 template <int D>
@@ -494,7 +462,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint64_t *barQ = empty + C::NSLOT;
     uint64_t *barQfree = barQ + 1;  // the item's last QK done: Q may be replaced
     uint64_t *barS = barQfree + 1;  // [2] S of buffer b computed
-    uint64_t *barP = barS + 2;      // [2] P and (m_s, l_s) of buffer b written (128 arrivals)
+    uint64_t *barP = barS + 2;      // [2] P and (m_s, l_s) of buffer b written (256 arrivals)
     uint64_t *barO = barP + 2;      // [2] O_s of buffer b computed
     uint64_t *barF = barO + 2;      // [2] O_s of buffer b merged, buffer free
     uint64_t *drain = barF + 2;
@@ -511,7 +479,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(barQfree, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&barS[b], 1);
-            mbar_init(&barP[b], 128);
+            mbar_init(&barP[b], 256);
             mbar_init(&barO[b], 1);
             mbar_init(&barF[b], kFoldThreads);
         }
@@ -534,224 +502,282 @@ __global__ void __launch_bounds__(THREADS, 1)
     // splits it has seen (gs): split number gs uses TMEM buffer gs & 1 with
     // barrier parity (gs >> 1) & 1, and its loads are numbers 2 gs, 2 gs + 1
     // of the ring.  An item's last QK releases the Q buffer for the next.
-    if (warp == 0) {
-        // ====================================================== producer
-        bool ok = true;
-        uint32_t armed = 0, armed_parity = 0;
-        int gs = 0, nq = 0;
-        int64_t li = 0;  // running load number: slot li % NSLOT
-        for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
-            Item it;
-            if (!make_item(p, idx, it)) continue;
-            const int32_t *bt_row = p.block_table + int64_t(it.b) * p.max_pages;
-            auto lookup = [&](int s) -> int {
-                const int lp = key_of(it, s) / kPage + lane;  // logical page
-                if (lane >= kSplit / kPage || lp * kPage >= it.kend) return -1;
-                return lp < p.max_pages ? __ldg(bt_row + lp) : -2;
-            };
-            // Load list (relative split j, n splits): K0, K1, V0, K2, V1, K3,
-            // ..., V(n-2), V(n-1): keys two splits ahead of values, the order
-            // in which the MMA warp consumes them.  Lane i < 16 looks up page
-            // i of a split ahead of use (4 splits in flight) and issues that
-            // page's copy itself; the id is checked where it is used.
-            const int n = it.s1 - it.s0;
-            int pages[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) pages[e] = e < n ? lookup(it.s0 + e) : -1;
-            auto emit = [&](int which, int j) -> bool {
-                const int s = it.s0 + j;
-                const int slot = int(li % C::NSLOT);
-                const uint32_t phase = uint32_t(li / C::NSLOT) & 1u;
-                int phys = pages[j & 3];
-                if (phys == -2 || phys >= p.num_pages || phys < -1) {  // bad id: zero page, flagged
-                    if (which == 0) record_status(p.status, BI_DEV_BAD_INDEX);
-                    phys = -1;
-                }
-                const int nk = min(kSplit, it.kend - key_of(it, s));  // valid keys, >= 1
-                const int full_pages = nk / kPage;
-                const int npages = (nk + kPage - 1) / kPage;
-                int got = 1;
-                if (lane == 0) got = wait(&empty[slot], phase ^ 1u, ctl) ? 1 : 0;
-                got = __shfl_sync(0xffffffffu, got, 0);
-                if (!got) return false;
-                uint8_t *dst = sKV + slot * C::KV_BYTES;
-                const uint8_t *cache = static_cast<const uint8_t *>(which ? p.v_cache : p.k_cache);
-                const int partial_phys = __shfl_sync(0xffffffffu, phys, full_pages & 31);
-                // V: the partial last page is copied by the whole warp, with
-                // the keys past the sequence end set to zero.
-                if (which == 1 && full_pages < npages) {
-                    const int pg = full_pages;
-                    const bool good = partial_phys >= 0;
-                    const int valid = nk - pg * kPage;
-                    const uint8_t *blk =
-                        cache + (int64_t(partial_phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
-                    for (int e = lane; e < kPage * (D / 8); e += 32) {
-                        const int r = e / (D / 8), c = e % (D / 8);
-                        const uint32_t off = page_off<D>(r, c);
-                        uint4 v = make_uint4(0, 0, 0, 0);
-                        if (good && r < valid) v = __ldg(reinterpret_cast<const uint4 *>(blk + off));
-                        *reinterpret_cast<uint4 *>(dst + pg * C::PAGE_BYTES + off) = v;
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                }
-                // K: the pages holding valid keys.  V: whole valid pages plus
-                // all-zero pages past the end.  One bulk copy per page.
-                const int copies = which ? (kSplit / kPage) - (npages - full_pages) : npages;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[slot], uint32_t(copies) * C::PAGE_BYTES);
-                    armed |= 1u << slot;
-                    armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
-                }
-                __syncwarp();
-                const int pg = lane;
-                bool issue;
-                const uint8_t *src = g_zero_page;
-                if (which == 0) {
-                    issue = pg < npages;
-                    if (phys >= 0) src = cache + (int64_t(phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
-                } else {
-                    issue = pg < kSplit / kPage && !(pg == full_pages && full_pages < npages);
-                    if (pg < full_pages && phys >= 0)
-                        src = cache + (int64_t(phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
-                }
-                if (issue) bulk_load(dst + pg * C::PAGE_BYTES, src, C::PAGE_BYTES, &full[slot]);
-                __syncwarp();
-                ++li;
-                return true;
-            };
-            // the first keys go out before Q (their slots free up earlier)
-            if (n > 0) ok = emit(0, 0);
-            if (ok && n > 1) ok = emit(0, 1);
-            // Q of this item once the previous item's QK products are done
-            int gotq = 1;
-            if (lane == 0) {
-                if (nq > 0) gotq = wait(barQfree, uint32_t(nq - 1) & 1u, ctl) ? 1 : 0;
-                if (gotq) {
-                    if (p.decode) {
-                        const int rpq = p.rows_per_q;
-                        mbar_arrive_expect_tx(barQ, 4u * C::KB * rpq * 128u);
-                        for (int q = 0; q < 4; ++q)
-                            for (int kb = 0; kb < C::KB; ++kb)
-                                tma_load_3d(sQ + kb * C::Q_KB_BYTES + q * 32 * 128, &tq, barQ,
-                                            kb * 64, it.g * p.group + q * rpq, it.b);
-                    } else {
-                        mbar_arrive_expect_tx(barQ, uint32_t(C::Q_BYTES));
-                        for (int kb = 0; kb < C::KB; ++kb)
-                            tma_load_3d(sQ + kb * C::Q_KB_BYTES, &tq, barQ, kb * 64, it.h, it.q_row0);
-                    }
-                }
-            }
-            gotq = __shfl_sync(0xffffffffu, gotq, 0);
-            ok = ok && gotq;
-            ++nq;
-            for (int j = 0; ok && j < n; ++j) {
-                ok = emit(1, j);
-                // split j is done with its page ids: look up split j + 4
-                pages[j & 3] = (j + 4 < n) ? lookup(it.s0 + j + 4) : -1;
-                if (ok && j + 2 < n) ok = emit(0, j + 2);
-            }
-            gs += n;
-        }
-        if (!ok && lane == 0) {
-            for (int s = 0; s < C::NSLOT; ++s)
-                if (armed & (1u << s)) wait_drain(&full[s], (armed_parity >> s) & 1u, p.timeout_ns);
-            if (nq > 0) wait_drain(barQ, uint32_t(nq - 1) & 1u, p.timeout_ns);
-        }
-        (void)gs;
-    } else if (warp == 1) {
-        // ====================================================== MMA issue
-        // Per item, tensor-pipe order QK(0), QK(1), PV(0), QK(2), PV(1), ...
-        // -- the order of the producer's load list.  QK of split gs reuses
-        // TMEM buffer gs & 1 once the fold warps have merged split gs - 2,
-        // which may belong to the previous item.
-        if (lane == 0) {
-            const uint32_t idesc_qk = idesc_bf16_f32(128, kSplit, 0, 0);
-            const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-            const uint32_t q_base = smem_u32(sQ);
+    // Each warpgroup sets its registers once, at one instruction for all its
+    // warps, before its warps take their roles: warpgroup 0 gives back, the
+    // fold warpgroups take, the softmax ones keep the launch's.
+    if (warp < 4) {
+        regs_release<kRegsCtl>();
+        if (warp == 0) {
+            // ====================================================== producer
             bool ok = true;
+            uint32_t armed = 0, armed_parity = 0;
             int gs = 0, nq = 0;
+            int64_t li = 0;  // running load number: slot li % NSLOT
             for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
                 Item it;
                 if (!make_item(p, idx, it)) continue;
+                const int32_t *bt_row = p.block_table + int64_t(it.b) * p.max_pages;
+                auto lookup = [&](int s) -> int {
+                    const int lp = key_of(it, s) / kPage + lane;  // logical page
+                    if (lane >= kSplit / kPage || lp * kPage >= it.kend) return -1;
+                    return lp < p.max_pages ? __ldg(bt_row + lp) : -2;
+                };
+                // Load list (relative split j, n splits): K0, K1, V0, K2, V1, K3,
+                // ..., V(n-2), V(n-1): keys two splits ahead of values, the order
+                // in which the MMA warp consumes them.  Lane i < 16 looks up page
+                // i of a split ahead of use (4 splits in flight) and issues that
+                // page's copy itself; the id is checked where it is used.
                 const int n = it.s1 - it.s0;
-                const int64_t base = 2 * int64_t(gs);  // load number of K0
-                // load numbers of K(j) and V(j) in the list K0, K1, V0, K2, V1, ...
-                auto k_load = [&](int j) { return base + (j < 2 ? j : 2 * j - 1); };
-                auto v_load = [&](int j) { return base + min(2 + 2 * j, 2 * n - 1); };
-                auto issue_qk = [&](int j) -> bool {
-                    const int g = gs + j;
-                    if (g >= 2) {  // buffer g & 1 still holds split g - 2 until merged
-                        if (!wait(&barF[g & 1], uint32_t((g - 2) >> 1) & 1u, ctl)) return false;
-                        tc_fence_after();
+                int pages[4];
+    #pragma unroll
+                for (int e = 0; e < 4; ++e) pages[e] = e < n ? lookup(it.s0 + e) : -1;
+                auto emit = [&](int which, int j) -> bool {
+                    const int s = it.s0 + j;
+                    const int slot = int(li % C::NSLOT);
+                    const uint32_t phase = uint32_t(li / C::NSLOT) & 1u;
+                    int phys = pages[j & 3];
+                    if (phys == -2 || phys >= p.num_pages || phys < -1) {  // bad id: zero page, flagged
+                        if (which == 0) record_status(p.status, BI_DEV_BAD_INDEX);
+                        phys = -1;
                     }
-                    const int64_t i = k_load(j);
-                    const int slot = int(i % C::NSLOT);
-                    if (!wait(&full[slot], uint32_t(i / C::NSLOT) & 1u, ctl)) return false;
-                    tc_fence_after();
-                    const uint32_t d = tmem + C::BUF_COLS * uint32_t(g & 1);
-                    const uint32_t k_base = smem_u32(sKV + slot * C::KV_BYTES);
-#pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        const uint32_t kb = k >> 2, kk = k & 3;
-                        // K: K-major, core matrices; 16 values of the head
-                        // dim are two core matrices 128 bytes apart, 8-key
-                        // groups KGROUP_BYTES apart (also across pages).
-                        mma_ss(d, sdesc_sw128(q_base + kb * C::Q_KB_BYTES + kk * 32, 16, 1024),
-                               sdesc_plain(k_base + k * 256, 128, C::KGROUP_BYTES), idesc_qk,
-                               k > 0 ? 1u : 0u);
+                    const int nk = min(kSplit, it.kend - key_of(it, s));  // valid keys, >= 1
+                    const int full_pages = nk / kPage;
+                    const int npages = (nk + kPage - 1) / kPage;
+                    int got = 1;
+                    if (lane == 0) got = wait_inl(&empty[slot], phase ^ 1u, ctl) ? 1 : 0;
+                    got = __shfl_sync(0xffffffffu, got, 0);
+                    if (!got) return false;
+                    uint8_t *dst = sKV + slot * C::KV_BYTES;
+                    const uint8_t *cache = static_cast<const uint8_t *>(which ? p.v_cache : p.k_cache);
+                    const int partial_phys = __shfl_sync(0xffffffffu, phys, full_pages & 31);
+                    // V: the partial last page is copied by the whole warp, with
+                    // the keys past the sequence end set to zero.
+                    if (which == 1 && full_pages < npages) {
+                        const int pg = full_pages;
+                        const bool good = partial_phys >= 0;
+                        const int valid = nk - pg * kPage;
+                        const uint8_t *blk =
+                            cache + (int64_t(partial_phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
+                        for (int e = lane; e < kPage * (D / 8); e += 32) {
+                            const int r = e / (D / 8), c = e % (D / 8);
+                            const uint32_t off = page_off<D>(r, c);
+                            uint4 v = make_uint4(0, 0, 0, 0);
+                            if (good && r < valid) v = __ldg(reinterpret_cast<const uint4 *>(blk + off));
+                            *reinterpret_cast<uint4 *>(dst + pg * C::PAGE_BYTES + off) = v;
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
                     }
-                    mma_commit(&barS[g & 1]);
-                    mma_commit(&empty[slot]);
-                    if (j == n - 1) mma_commit(barQfree);  // the item's last use of Q
+                    // K: the pages holding valid keys.  V: whole valid pages plus
+                    // all-zero pages past the end.  One bulk copy per page.
+                    const int copies = which ? (kSplit / kPage) - (npages - full_pages) : npages;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&full[slot], uint32_t(copies) * C::PAGE_BYTES);
+                        armed |= 1u << slot;
+                        armed_parity = (armed_parity & ~(1u << slot)) | (phase << slot);
+                    }
+                    __syncwarp();
+                    const int pg = lane;
+                    bool issue;
+                    const uint8_t *src = g_zero_page;
+                    if (which == 0) {
+                        issue = pg < npages;
+                        if (phys >= 0) src = cache + (int64_t(phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
+                    } else {
+                        issue = pg < kSplit / kPage && !(pg == full_pages && full_pages < npages);
+                        if (pg < full_pages && phys >= 0)
+                            src = cache + (int64_t(phys) * p.Hkv + it.g) * int64_t(C::PAGE_BYTES);
+                    }
+                    if (issue) bulk_load(dst + pg * C::PAGE_BYTES, src, C::PAGE_BYTES, &full[slot]);
+                    __syncwarp();
+                    ++li;
                     return true;
                 };
-                ok = wait(barQ, uint32_t(nq) & 1u, ctl);
+                // the first keys go out before Q (their slots free up earlier)
+                if (n > 0) ok = emit(0, 0);
+                if (ok && n > 1) ok = emit(0, 1);
+                // Q of this item once the previous item's QK products are done
+                int gotq = 1;
+                if (lane == 0) {
+                    if (nq > 0) gotq = wait_inl(barQfree, uint32_t(nq - 1) & 1u, ctl) ? 1 : 0;
+                    if (gotq) {
+                        if (p.decode) {
+                            const int rpq = p.rows_per_q;
+                            mbar_arrive_expect_tx(barQ, 4u * C::KB * rpq * 128u);
+                            for (int q = 0; q < 4; ++q)
+                                for (int kb = 0; kb < C::KB; ++kb)
+                                    tma_load_3d(sQ + kb * C::Q_KB_BYTES + q * 32 * 128, &tq, barQ,
+                                                kb * 64, it.g * p.group + q * rpq, it.b);
+                        } else {
+                            mbar_arrive_expect_tx(barQ, uint32_t(C::Q_BYTES));
+                            for (int kb = 0; kb < C::KB; ++kb)
+                                tma_load_3d(sQ + kb * C::Q_KB_BYTES, &tq, barQ, kb * 64, it.h, it.q_row0);
+                        }
+                    }
+                }
+                gotq = __shfl_sync(0xffffffffu, gotq, 0);
+                ok = ok && gotq;
                 ++nq;
-                if (ok) ok = issue_qk(0);
-                if (ok && n > 1) ok = issue_qk(1);
                 for (int j = 0; ok && j < n; ++j) {
-                    const int g = gs + j;
-                    const int b = g & 1;
-                    const uint32_t par = uint32_t(g >> 1) & 1u;
-                    const int64_t i = v_load(j);
-                    const int slot = int(i % C::NSLOT);
-                    if (!wait(&full[slot], uint32_t(i / C::NSLOT) & 1u, ctl)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t buf = tmem + C::BUF_COLS * uint32_t(b);
-                    const uint32_t v_base = smem_u32(sKV + slot * C::KV_BYTES);
-                    if (!wait(&barP[b], par, ctl)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-#pragma unroll
-                    for (int jj = 0; jj < kSplit / 16; ++jj) {
-                        // V: MN-major, core matrices; step jj is page jj;
-                        // its two 8-key groups are KGROUP_BYTES apart,
-                        // 8-value blocks of the head dim 128 bytes apart.
-                        mma_ts(buf + C::O_OFF, buf + C::P_OFF + 8 * jj,
-                               sdesc_plain(v_base + jj * C::PAGE_BYTES, C::KGROUP_BYTES, 128),
-                               idesc_pv, jj > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&barO[b]);
-                    mma_commit(&empty[slot]);
-                    if (j + 2 < n) ok = issue_qk(j + 2);
+                    ok = emit(1, j);
+                    // split j is done with its page ids: look up split j + 4
+                    pages[j & 3] = (j + 4 < n) ? lookup(it.s0 + j + 4) : -1;
+                    if (ok && j + 2 < n) ok = emit(0, j + 2);
                 }
                 gs += n;
             }
-            if (!ok) {
-                mma_commit(drain);
-                wait_drain(drain, 0, p.timeout_ns);
+            if (!ok && lane == 0) {
+                for (int s = 0; s < C::NSLOT; ++s)
+                    if (armed & (1u << s)) wait_drain(&full[s], (armed_parity >> s) & 1u, p.timeout_ns);
+                if (nq > 0) wait_drain(barQ, uint32_t(nq - 1) & 1u, p.timeout_ns);
+            }
+            (void)gs;
+        } else if (warp == 1) {
+            // ====================================================== MMA issue
+            // Per item, tensor-pipe order QK(0), QK(1), PV(0), QK(2), PV(1), ...
+            // -- the order of the producer's load list.  QK of split gs reuses
+            // TMEM buffer gs & 1 once the fold warps have merged split gs - 2,
+            // which may belong to the previous item.
+            if (lane == 0) {
+                const uint32_t idesc_qk = idesc_bf16_f32(128, kSplit, 0, 0);
+                const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+                const uint32_t q_base = smem_u32(sQ);
+                bool ok = true;
+                int gs = 0, nq = 0;
+                for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
+                    Item it;
+                    if (!make_item(p, idx, it)) continue;
+                    const int n = it.s1 - it.s0;
+                    const int64_t base = 2 * int64_t(gs);  // load number of K0
+                    // load numbers of K(j) and V(j) in the list K0, K1, V0, K2, V1, ...
+                    auto k_load = [&](int j) { return base + (j < 2 ? j : 2 * j - 1); };
+                    auto v_load = [&](int j) { return base + min(2 + 2 * j, 2 * n - 1); };
+                    auto issue_qk = [&](int j) -> bool {
+                        const int g = gs + j;
+                        if (g >= 2) {  // buffer g & 1 still holds split g - 2 until merged
+                            if (!wait_inl(&barF[g & 1], uint32_t((g - 2) >> 1) & 1u, ctl)) return false;
+                            tc_fence_after();
+                        }
+                        const int64_t i = k_load(j);
+                        const int slot = int(i % C::NSLOT);
+                        if (!wait_inl(&full[slot], uint32_t(i / C::NSLOT) & 1u, ctl)) return false;
+                        tc_fence_after();
+                        const uint32_t d = tmem + C::BUF_COLS * uint32_t(g & 1);
+                        const uint32_t k_base = smem_u32(sKV + slot * C::KV_BYTES);
+    #pragma unroll
+                        for (int k = 0; k < D / 16; ++k) {
+                            const uint32_t kb = k >> 2, kk = k & 3;
+                            // K: K-major, core matrices; 16 values of the head
+                            // dim are two core matrices 128 bytes apart, 8-key
+                            // groups KGROUP_BYTES apart (also across pages).
+                            mma_ss(d, sdesc_sw128(q_base + kb * C::Q_KB_BYTES + kk * 32, 16, 1024),
+                                   sdesc_plain(k_base + k * 256, 128, C::KGROUP_BYTES), idesc_qk,
+                                   k > 0 ? 1u : 0u);
+                        }
+                        mma_commit(&barS[g & 1]);
+                        mma_commit(&empty[slot]);
+                        if (j == n - 1) mma_commit(barQfree);  // the item's last use of Q
+                        return true;
+                    };
+                    ok = wait_inl(barQ, uint32_t(nq) & 1u, ctl);
+                    ++nq;
+                    if (ok) ok = issue_qk(0);
+                    if (ok && n > 1) ok = issue_qk(1);
+                    for (int j = 0; ok && j < n; ++j) {
+                        const int g = gs + j;
+                        const int b = g & 1;
+                        const uint32_t par = uint32_t(g >> 1) & 1u;
+                        const int64_t i = v_load(j);
+                        const int slot = int(i % C::NSLOT);
+                        if (!wait_inl(&full[slot], uint32_t(i / C::NSLOT) & 1u, ctl)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t buf = tmem + C::BUF_COLS * uint32_t(b);
+                        const uint32_t v_base = smem_u32(sKV + slot * C::KV_BYTES);
+                        if (!wait_inl(&barP[b], par, ctl)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+    #pragma unroll
+                        for (int jj = 0; jj < kSplit / 16; ++jj) {
+                            // V: MN-major, core matrices; step jj is page jj;
+                            // its two 8-key groups are KGROUP_BYTES apart,
+                            // 8-value blocks of the head dim 128 bytes apart.
+                            mma_ts(buf + C::O_OFF, buf + C::P_OFF + 8 * jj,
+                                   sdesc_plain(v_base + jj * C::PAGE_BYTES, C::KGROUP_BYTES, 128),
+                                   idesc_pv, jj > 0 ? 1u : 0u);
+                        }
+                        mma_commit(&barO[b]);
+                        mma_commit(&empty[slot]);
+                        if (j + 2 < n) ok = issue_qk(j + 2);
+                    }
+                    gs += n;
+                }
+                if (!ok) {
+                    mma_commit(drain);
+                    wait_drain(drain, 0, p.timeout_ns);
+                }
             }
         }
+        // warps 2 and 3: no role
+    } else if ((warp >= 4 && warp < 8) || warp >= 16) {
+        // ====================================================== softmax
+        // The softmax warps of lane quarter q (two, 16 lanes each) and its
+        // fold warps (two, one per half of the head dim) serve the same 32
+        // rows; each role walks the items on its own, so that the code after
+        // a role's register budget is that role's alone.
+        const int q = warp & 3;
+        int gs = 0;
+        bool ok = true;
+        for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
+            Item it;
+            if (!make_item(p, idx, it)) continue;
+            // whether lane quarter q holds any row of the item
+            const bool active = p.decode ? q * p.rows_per_q < p.group : 32 * q < it.rows;
+            const float cs = p.scale_log2;
+            // this warp's 16 lanes of the quarter: lane0 .. lane0 + 15;
+            // this thread's rows lane0 + v and lane0 + v + 8
+            const int lane0 = 32 * q + (warp >= 16 ? 16 : 0), v = lane >> 2;
+            // lanes of the quarter that hold rows (from lane 0 up)
+            const int n_lanes = !active ? 0
+                                : p.decode ? min(p.rows_per_q, p.group - q * p.rows_per_q)
+                                           : min(32, it.rows - 32 * q);
+            const bool lo = n_lanes > lane0 - 32 * q, hi = n_lanes > lane0 - 32 * q + 8;
+            const int t_lo = p.decode ? it.kend - 1 : it.pos0 + lane0 + v;
+            const int t_hi = p.decode ? it.kend - 1 : it.pos0 + lane0 + v + 8;
+            const uint32_t lanes16 = tmem_addr(tmem, uint32_t(lane0), 0);
+            for (int s = it.s0; s < it.s1; ++s) {
+                const int g = gs + (s - it.s0);
+                const int b = g & 1;
+                const uint32_t par = uint32_t(g >> 1) & 1u;
+                if (!wait_inl(&barS[b], par, ctl)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                float m_s[2] = {-INFINITY, -INFINITY}, l_s[2] = {0.0f, 0.0f};
+                const uint32_t sb = lanes16 + C::BUF_COLS * uint32_t(b) + C::P_OFF;
+                if (hi)
+                    softmax_lanes16<true>(sb, key_of(it, s), t_lo, t_hi, cs, m_s, l_s);
+                else if (lo)
+                    softmax_lanes16<false>(sb, key_of(it, s), t_lo, t_hi, cs, m_s, l_s);
+                if ((lane & 3) == 0) {
+                    float *ml = sML + (b * 128 + lane0 + v) * 2;
+                    ml[0] = m_s[0];
+                    ml[1] = l_s[0];
+                    ml[16] = m_s[1];  // row lane0 + v + 8
+                    ml[17] = l_s[1];
+                }
+                tc_fence_before();
+                mbar_arrive(&barP[b]);
+            }
+            gs += it.s1 - it.s0;
+        }
     } else {
-        // ====================================================== rows
-        // Softmax warp 4 + q and fold warps of lane quarter q (two, one per
-        // half of the head dim) serve the same 32 rows.
-        const bool is_softmax = warp >= 4 && warp < 8;
+        // ====================================================== fold
+        regs_take<kRegsFold>();
         const int q = warp & 3;
         const uint32_t lane_base = tmem_addr(tmem, 32 * q, 0);
         const int row_id = 32 * q + lane;  // TMEM lane of this row
@@ -783,153 +809,119 @@ __global__ void __launch_bounds__(THREADS, 1)
             int t;
             int64_t out_row;
             row_of(it, t, active, valid, out_row);
-            if (is_softmax) {
-                // -------------------------------------------------- softmax
-                const float cs = p.scale_log2;
-                // decode with at most 8 query rows per quarter: the 16-lane path
-                const bool heads16 = p.decode && p.rows_per_q <= 8 && active;
-                for (int s = it.s0; s < it.s1; ++s) {
-                    const int g = gs + (s - it.s0);
-                    const int b = g & 1;
-                    const uint32_t par = uint32_t(g >> 1) & 1u;
-                    const uint32_t sb = lane_base + C::BUF_COLS * uint32_t(b);
-                    if (!wait(&barS[b], par, ctl)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    float m_s = -INFINITY, l_s = 0.0f;
-                    if (heads16) {
-                        // rows of this quarter in lanes 0..7, four threads a row
-                        softmax_heads16(lane_base + C::BUF_COLS * uint32_t(b) + C::P_OFF,
-                                        key_of(it, s), t, cs, m_s, l_s);
-                        if ((lane & 3) == 0) {
-                            sML[(b * 128 + 32 * q + (lane >> 2)) * 2 + 0] = m_s;
-                            sML[(b * 128 + 32 * q + (lane >> 2)) * 2 + 1] = l_s;
-                        }
-                    } else {
-                        if (active) softmax_rows(sb + C::P_OFF, key_of(it, s), t, cs, m_s, l_s);
-                        sML[(b * 128 + row_id) * 2 + 0] = m_s;
-                        sML[(b * 128 + row_id) * 2 + 1] = l_s;
-                    }
-                    tc_fence_before();
-                    mbar_arrive(&barP[b]);
-                }
-            } else {
-                // -------------------------------------------------- fold
-                // This warp merges columns col0 .. col0 + HW - 1 of its rows.
-                constexpr int HW = D / 2;
-                const int half = warp >= 10 ? 1 : 0;
-                const int col0 = half * HW;
+            // This warp merges columns col0 .. col0 + HW - 1 of its rows.
+            constexpr int HW = D / 2;
+            const int half = warp >= 12 ? 1 : 0;
+            const int col0 = half * HW;
 #if BI_INVARIANT
-                // blocks after a sequence's first write every split's own partial
-                const bool spill = p.decode && it.s0 > 0;
+            // blocks after a sequence's first write every split's own partial
+            const bool spill = p.decode && it.s0 > 0;
 #else
-                // variant-off: every block merges its own range (the grouping
-                // of the merge then depends on how many blocks served it)
-                const bool spill = false;
+            // variant-off: every block merges its own range (the grouping
+            // of the merge then depends on how many blocks served it)
+            const bool spill = false;
 #endif
-                float m = -INFINITY, l = 0.0f;
-                float O[HW];
+            float m = -INFINITY, l = 0.0f;
+            float O[HW];
 #pragma unroll
-                for (int j = 0; j < HW; ++j) O[j] = 0.0f;
-                for (int s = it.s0; s < it.s1; ++s) {
-                    const int g = gs + (s - it.s0);
-                    const int b = g & 1;
-                    const uint32_t par = uint32_t(g >> 1) & 1u;
-                    const uint32_t ob = lane_base + C::BUF_COLS * uint32_t(b) + C::O_OFF + col0;
-                    const int k0 = key_of(it, s);
-                    // barP: (m_s, l_s) of this split are in shared memory;
-                    // barO: O_s is in TMEM.
-                    if (!wait(&barP[b], par, ctl) || !wait(&barO[b], par, ctl)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const float m_s = sML[(b * 128 + row_id) * 2 + 0];
-                    const float l_s = sML[(b * 128 + row_id) * 2 + 1];
-                    if (active) {
-                        // 32-column TMEM loads (HW / 32 per split)
-                        constexpr int NCH32 = HW / 32;
-                        if (spill) {
-                            // not the first block of this sequence: write the
-                            // split's own partial for attn_combine
-                            float *rec = p.ws + ((out_row * p.max_splits) + s) * C::REC + 4 + col0;
-#pragma unroll 1
-                            for (int c = 0; c < NCH32; ++c) {
-                                uint32_t r[32];
-                                tmem_ld32(ob + 32 * c, r);
-                                tmem_wait_ld(r);
-                                if (valid) {
-#pragma unroll
-                                    for (int j = 0; j < 8; ++j)
-                                        reinterpret_cast<float4 *>(rec + 32 * c)[j] = make_float4(
-                                            __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                            __uint_as_float(r[4 * j + 2]),
-                                            __uint_as_float(r[4 * j + 3]));
-                                }
-                            }
-                            if (valid && half == 0) {
-                                rec[-4] = m_s;
-                                rec[-3] = l_s;
-                            }
-                        } else {
-                            const bool first = (s == it.s0);
-                            const bool take = k0 <= t;  // the row sees at least key k0
-                            float mn, a, cc;
-                            merge_scales(m, m_s, mn, a, cc);
-#pragma unroll
-                            for (int c = 0; c < NCH32; ++c) {
-                                uint32_t r[32];
-                                tmem_ld32(ob + 32 * c, r);
-                                tmem_wait_ld(r);
-#pragma unroll
-                                for (int j = 0; j < 32; ++j) {
-                                    const float o = __uint_as_float(r[j]);
-                                    if (first)
-                                        O[32 * c + j] = o;
-                                    else if (take)
-                                        O[32 * c + j] = merge_val(O[32 * c + j], a, o, cc);
-                                }
-                            }
-                            if (first) {
-                                m = m_s;
-                                l = l_s;
-                            } else if (take) {
-                                l = merge_val(l, a, l_s, cc);
-                                m = mn;
-                            }
-                        }
-                    }
-                    tc_fence_before();
-                    mbar_arrive(&barF[b]);
+            for (int j = 0; j < HW; ++j) O[j] = 0.0f;
+            for (int s = it.s0; s < it.s1; ++s) {
+                const int g = gs + (s - it.s0);
+                const int b = g & 1;
+                const uint32_t par = uint32_t(g >> 1) & 1u;
+                const uint32_t ob = lane_base + C::BUF_COLS * uint32_t(b) + C::O_OFF + col0;
+                const int k0 = key_of(it, s);
+                // barP: (m_s, l_s) of this split are in shared memory;
+                // barO: O_s is in TMEM.
+                if (!wait_inl(&barP[b], par, ctl) || !wait_inl(&barO[b], par, ctl)) {
+                    ok = false;
+                    break;
                 }
-                if (ok && active && valid && !spill) {
-                    if (!p.decode || item_whole(it)) {
-                        write_out<HW>(O, l, m,
-                                      static_cast<__nv_bfloat16 *>(p.o) + out_row * D + col0,
-                                      (p.lse && half == 0) ? p.lse + out_row : nullptr);
-                    } else {
-                        // a block of a sequence served by several: hand the
-                        // merged state over its range (ending at split s1-1)
-                        // to attn_combine (in the invariant build only the
-                        // first block gets here; the others write every split)
-                        float *rec = p.ws + ((out_row * p.max_splits) + item_rec(it)) * C::REC;
-                        if (half == 0) {
-                            rec[0] = m;
-                            rec[1] = l;
-                        }
+                tc_fence_after();
+                const float m_s = sML[(b * 128 + row_id) * 2 + 0];
+                const float l_s = sML[(b * 128 + row_id) * 2 + 1];
+                if (active) {
+                    // 16-column TMEM loads (HW / 16 per split; one load's
+                    // registers at a time beside O, within the 96 a
+                    // thread of this block has)
+                    constexpr int NCH16 = HW / 16;
+                    if (spill) {
+                        // not the first block of this sequence: write the
+                        // split's own partial for attn_combine
+                        float *rec = p.ws + ((out_row * p.max_splits) + s) * C::REC + 4 + col0;
+#pragma unroll 1
+                        for (int c = 0; c < NCH16; ++c) {
+                            uint32_t r[16];
+                            tmem_ld32x16(ob + 16 * c, r);
+                            tmem_wait_ld16(r);
+                            if (valid) {
 #pragma unroll
-                        for (int j = 0; j < HW / 4; ++j)
-                            reinterpret_cast<float4 *>(rec + 4 + col0)[j] =
-                                make_float4(O[4 * j], O[4 * j + 1], O[4 * j + 2], O[4 * j + 3]);
+                                for (int j = 0; j < 4; ++j)
+                                    reinterpret_cast<float4 *>(rec + 16 * c)[j] = make_float4(
+                                        __uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                        __uint_as_float(r[4 * j + 2]),
+                                        __uint_as_float(r[4 * j + 3]));
+                            }
+                        }
+                        if (valid && half == 0) {
+                            rec[-4] = m_s;
+                            rec[-3] = l_s;
+                        }
+                    } else {
+                        const bool first = (s == it.s0);
+                        const bool take = k0 <= t;  // the row sees at least key k0
+                        float mn, a, cc;
+                        merge_scales(m, m_s, mn, a, cc);
+#pragma unroll
+                        for (int c = 0; c < NCH16; ++c) {
+                            uint32_t r[16];
+                            tmem_ld32x16(ob + 16 * c, r);
+                            tmem_wait_ld16(r);
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const float o = __uint_as_float(r[j]);
+                                if (first)
+                                    O[16 * c + j] = o;
+                                else if (take)
+                                    O[16 * c + j] = merge_val(O[16 * c + j], a, o, cc);
+                            }
+                        }
+                        if (first) {
+                            m = m_s;
+                            l = l_s;
+                        } else if (take) {
+                            l = merge_val(l, a, l_s, cc);
+                            m = mn;
+                        }
                     }
+                }
+                tc_fence_before();
+                mbar_arrive(&barF[b]);
+            }
+            if (ok && active && valid && !spill) {
+                if (!p.decode || item_whole(it)) {
+                    write_out<HW>(O, l, m,
+                                  static_cast<__nv_bfloat16 *>(p.o) + out_row * D + col0,
+                                  (p.lse && half == 0) ? p.lse + out_row : nullptr);
+                } else {
+                    // a block of a sequence served by several: hand the
+                    // merged state over its range (ending at split s1-1)
+                    // to attn_combine (in the invariant build only the
+                    // first block gets here; the others write every split)
+                    float *rec = p.ws + ((out_row * p.max_splits) + item_rec(it)) * C::REC;
+                    if (half == 0) {
+                        rec[0] = m;
+                        rec[1] = l;
+                    }
+#pragma unroll
+                    for (int j = 0; j < HW / 4; ++j)
+                        reinterpret_cast<float4 *>(rec + 4 + col0)[j] =
+                            make_float4(O[4 * j], O[4 * j + 1], O[4 * j + 2], O[4 * j + 3]);
                 }
             }
             gs += it.s1 - it.s0;
         }
     }
-
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -1063,6 +1055,25 @@ size_t attn_ws_bytes(int B, int Hq, int head_dim, int max_splits, int max_chunks
     return size_t(B) * Hq * max_splits * (head_dim + 4) * sizeof(float);
 }
 
+// The block's register split (setmaxnreg: warpgroup 0 down to kRegsCtl,
+// the fold warpgroups up to kRegsFold) must fit the registers the block is
+// launched with, i.e. what the compiled kernel declares a thread -- a split
+// above that would leave the fold warps waiting for registers forever.
+// Checked once per kernel; a kernel that does not fit is never launched.
+template <int D>
+cudaError_t check_register_split()
+{
+    static int verdict = 0;  // 0 not yet checked, 1 fits, -1 does not
+    if (verdict == 0) {
+        cudaFuncAttributes a;
+        const cudaError_t e = cudaFuncGetAttributes(&a, attn_split_kernel<D>);
+        if (e != cudaSuccess) return e;
+        const long r = a.numRegs;
+        verdict = (128L * (kRegsCtl + 2 * r + 2 * kRegsFold) <= long(THREADS) * r) ? 1 : -1;
+    }
+    return verdict > 0 ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
 cudaError_t launch_attention(const CUtensorMap &tq, const AttnParams &p_in, int head_dim,
                              cudaStream_t s)
 {
@@ -1094,7 +1105,8 @@ cudaError_t launch_attention(const CUtensorMap &tq, const AttnParams &p_in, int 
     }
     const unsigned grid =
         static_cast<unsigned>(p.decode ? p.items : (p.items < sms[dev] ? p.items : sms[dev]));
-    cudaError_t e;
+    cudaError_t e = head_dim == 128 ? check_register_split<128>() : check_register_split<64>();
+    if (e != cudaSuccess) return e;
     if (head_dim == 128) {
         e = cudaFuncSetAttribute(attn_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg<128>::SMEM);

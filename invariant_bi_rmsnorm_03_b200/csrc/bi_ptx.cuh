@@ -98,7 +98,10 @@ struct WaitCtl {
 // Waits for the phase of `bar` with parity `parity` to complete.  Returns
 // false if the block is aborting or the wait ran past the limit (then the
 // status word records BI_ERR_TIMEOUT and the block's abort flag is raised).
-static __device__ __noinline__ bool wait(uint64_t *bar, uint32_t parity, const WaitCtl &ctl)
+// wait_inl is the inlined form, for kernels whose warpgroups run with
+// different register budgets (setmaxnreg): a called function would have to
+// fit all of them.
+__device__ __forceinline__ bool wait_inl(uint64_t *bar, uint32_t parity, const WaitCtl &ctl)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
@@ -111,6 +114,11 @@ static __device__ __noinline__ bool wait(uint64_t *bar, uint32_t parity, const W
             return false;
         }
     }
+}
+
+static __device__ __noinline__ bool wait(uint64_t *bar, uint32_t parity, const WaitCtl &ctl)
+{
+    return wait_inl(bar, parity, ctl);
 }
 
 // ---------------------------------------------------------------- proxies
@@ -350,6 +358,75 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
         "r"(r[15])
         : "memory");
+}
+
+// Per-warpgroup register budget (setmaxnreg): every warp of a warpgroup
+// executes the same one.  regs_release lowers the warpgroup's registers a
+// thread to N and returns the rest to the block's pool; regs_take raises
+// them to N from that pool, waiting until it holds enough -- so the block's
+// launch allocation must cover every warpgroup's final budget.
+template <uint32_t N>
+__device__ __forceinline__ void regs_release()
+{
+    static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg range");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_take()
+{
+    static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg range");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// 32 lanes x 16 columns into 16 registers per thread (thread i gets lane
+// base+i); valid after tmem_wait_ld16(r).
+__device__ __forceinline__ void tmem_ld32x16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+                   "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr)
+                 : "memory");
+}
+
+// 16 lanes x 256 bits, repeated 4 times (32 columns), into 16 registers per
+// thread.  Thread t = t0 + 4 t1 (t0 < 4) gets, for repetition m < 4,
+// r[4m], r[4m+1] = columns 8m + 2 t0, 8m + 2 t0 + 1 of lane t1 and
+// r[4m+2], r[4m+3] = the same columns of lane t1 + 8.
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+                   "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr)
+                 : "memory");
+}
+
+// Waits for this thread's outstanding TMEM loads; r (16 registers) is tied
+// to the wait so that no use of it moves above it.
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16])
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
+
+// 8 registers per thread into 16 lanes x 128 bits, repeated 4 times (16
+// columns).  Thread t = t0 + 4 t1 writes r[2m] to column 4m + t0 of lane t1
+// and r[2m+1] to the same column of lane t1 + 8 (m < 4).
+__device__ __forceinline__ void tmem_st_16x128b_x4(uint32_t taddr, const uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                 "r"(r[7])
+                 : "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_st()
