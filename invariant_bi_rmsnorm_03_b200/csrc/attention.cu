@@ -340,7 +340,7 @@ __device__ __forceinline__ void softmax_lanes16(uint32_t sb, int k0, int t_lo, i
     float mx[2][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) mx[0][i] = mx[1][i] = -INFINITY;
-    auto chunk_max = [&](const uint32_t (&r)[16], int c) {
+    auto chunk_max = [&](const uint32_t *r, int c) {
         if (whole(c)) {
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -361,18 +361,22 @@ __device__ __forceinline__ void softmax_lanes16(uint32_t sb, int k0, int t_lo, i
                 }
         }
     };
-    // loops kept rolled (a small instruction footprint: the block's other
-    // warps run other code on the same sub-partitions), two chunks a trip
-    uint32_t ra[16], rb[16];
-    tmem_ld_16x256b_x4(sb, ra);
+    // Pass 1 holds four chunks' loads in flight (two 64-key loads, one
+    // wait): a TMEM load under the block's load takes ~150 cycles, far more
+    // than the 16 maxima of a chunk.
+    {
+        uint32_t ra[32], rb[32];
 #pragma unroll 1
-    for (int c = 0; c < NC; c += 2) {
-        tmem_wait_ld16(ra);
-        tmem_ld_16x256b_x4(sb + 32 * (c + 1), rb);
-        chunk_max(ra, c);
-        tmem_wait_ld16(rb);
-        if (c + 2 < NC) tmem_ld_16x256b_x4(sb + 32 * (c + 2), ra);
-        chunk_max(rb, c + 1);
+        for (int c = 0; c < NC; c += 4) {
+            tmem_ld_16x256b_x8(sb + 32 * c, ra);
+            tmem_ld_16x256b_x8(sb + 32 * (c + 2), rb);
+            tmem_wait_ld(ra);
+            tmem_wait_ld(rb);
+            chunk_max(ra, c);
+            chunk_max(ra + 16, c + 1);
+            chunk_max(rb, c + 2);
+            chunk_max(rb + 16, c + 3);
+        }
     }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -422,6 +426,9 @@ __device__ __forceinline__ void softmax_lanes16(uint32_t sb, int k0, int t_lo, i
         __syncwarp();  // the rows of a warp may have taken different paths
         tmem_st_16x128b_x4(sb + 16 * c, pk);
     };
+    // loops kept rolled (a small instruction footprint: the block's other
+    // warps run other code on the same sub-partitions), two chunks a trip
+    uint32_t ra[16], rb[16];
     tmem_ld_16x256b_x4(sb, ra);
 #pragma unroll 1
     for (int c = 0; c < NC; c += 2) {
@@ -838,6 +845,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     break;
                 }
                 tc_fence_after();
+                bool released = false;
                 const float m_s = sML[(b * 128 + row_id) * 2 + 0];
                 const float l_s = sML[(b * 128 + row_id) * 2 + 1];
                 if (active) {
@@ -877,6 +885,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                             uint32_t r[16];
                             tmem_ld32x16(ob + 16 * c, r);
                             tmem_wait_ld16(r);
+                            if (c == NCH16 - 1) {  // O_s read: the buffer is free
+                                tc_fence_before();
+                                mbar_arrive(&barF[b]);
+                                released = true;
+                            }
 #pragma unroll
                             for (int j = 0; j < 16; ++j) {
                                 const float o = __uint_as_float(r[j]);
@@ -895,8 +908,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                         }
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(&barF[b]);
+                if (!released) {
+                    tc_fence_before();
+                    mbar_arrive(&barF[b]);
+                }
             }
             if (ok && active && valid && !spill) {
                 if (!p.decode || item_whole(it)) {
