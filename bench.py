@@ -241,6 +241,18 @@ class Clocks:
 
 # ---------------------------------------------------------------- ours
 
+HOST_AHEAD_CYCLES = 2_000_000  # ~1 ms of GPU clock
+
+
+def host_ahead(torch):
+    """A GPU spin of ~1 ms queued after the L2 flush and before the timed
+    region, so that the host has queued every launch of the timed region
+    before it starts: the device times then never include a wait for the
+    host (the ctypes calls take tens of microseconds each, longer than the
+    shortest kernels)."""
+    torch.cuda._sleep(HOST_AHEAD_CYCLES)
+
+
 def timed_steps(torch, L, wl, steps, warmup, dist=None, clocks=None):
     for _ in range(warmup):
         wl.flush.zero_()
@@ -256,6 +268,7 @@ def timed_steps(torch, L, wl, steps, warmup, dist=None, clocks=None):
         clocks.mark(0)
     for i in range(steps):
         wl.flush.zero_()
+        host_ahead(torch)
         wl.step(L, evs[i])
     torch.cuda.synchronize()
     if clocks is not None:
@@ -363,6 +376,7 @@ def rmsnorm_context(torch, L, wl) -> dict:
         ev = [(T.cuda.Event(enable_timing=True), T.cuda.Event(enable_timing=True)) for _ in range(reps)]
         for a, b in ev:
             wl.flush.zero_()
+            host_ahead(T)
             a.record()
             fn()
             b.record()
@@ -384,7 +398,8 @@ def rmsnorm_context(torch, L, wl) -> dict:
 
 def _median_ms(torch, fn, flush, reps=15, warm=3):
     """Median CUDA-event time of fn() on the current stream, L2 flushed
-    (a 512 MB write) before every launch."""
+    (a 512 MB write) before every launch and the launch queued before its
+    start event runs (host_ahead)."""
     T = torch
     for _ in range(warm):
         flush.zero_()
@@ -392,6 +407,7 @@ def _median_ms(torch, fn, flush, reps=15, warm=3):
     ev = [(T.cuda.Event(enable_timing=True), T.cuda.Event(enable_timing=True)) for _ in range(reps)]
     for a, b in ev:
         flush.zero_()
+        host_ahead(T)
         a.record()
         fn()
         b.record()
@@ -929,6 +945,8 @@ def run_profile_case(args):
         fn(i)
     torch.cuda.synchronize()
     ev = [T.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    # launches back to back: ~1 ms of GPU spin per 10 of them queued first
+    T.cuda._sleep(HOST_AHEAD_CYCLES * max(1, (args.steps + 9) // 10))
     for i in range(args.steps):
         ev[i].record()
         fn(i)
