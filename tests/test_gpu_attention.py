@@ -71,6 +71,26 @@ def test_decode_split_boundaries(L, d):
     decode_parity(L, kv, q, splits_per_cta=1)
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(40, 2), (48, 1), (100, 1), (128, 1)])
+def test_decode_large_groups(L, Hq, Hkv):
+    # Groups of 20, 48, 100 and 128 query heads: 5, 12, 25 and 32 rows in a
+    # TMEM lane quarter, so the quarter's second softmax warp (rows 16..31)
+    # and the upper 8 rows of each warp are used in decode too; the last
+    # quarter of the 100-head group is ragged.  Oracle parity, and decode of
+    # a sequence's last token equals its prefill bit for bit.
+    g = rng(24 + Hq)
+    lens = [1, 300, 777, 2049]
+    kv = paged_kv(g, lens, Hkv, 128)
+    q = normal_bf16(g, (len(lens), Hq, 128))
+    o, _ = decode_parity(L, kv, q)
+    S = lens[-1]
+    qp = normal_bf16(rng(25 + Hq), (S, Hq, 128))
+    qp[S - 1] = q[-1]
+    one = PagedKV(kv.k_cache, kv.v_cache, kv.block_table[-1:], kv.seq_lens[-1:], Hkv, 128)
+    op = L.bi_attention_prefill(dev_kv(one), dev_bf16(qp), i32([0, S]), i32([0]), S)
+    assert same_bytes(op[S - 1], o[-1])
+
+
 def test_decode_bits_do_not_depend_on_work_division(L):
     g = rng(23)
     lens = [5, 700, 2049, 4000, 300, 1]
