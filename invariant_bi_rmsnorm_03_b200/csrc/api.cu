@@ -911,7 +911,14 @@ bi_status bi_attention_backward(const bi_paged_kv *kv, const void *q, const void
     p.dv = dv_cache;
     p.status = d->status;
     p.timeout_ns = bi::kDefaultTimeoutNs;
-    return from_cuda(bi::launch_attention_backward(p, kv->head_dim, rows, d->num_sms,
+    CUtensorMap tq, tdo;
+    const int D = kv->head_dim;
+    const uint64_t dq3[3] = {uint64_t(D), uint64_t(Hq), uint64_t(T_total)};
+    const uint64_t sq3[2] = {uint64_t(D) * 2, uint64_t(Hq) * D * 2};
+    const uint32_t bq3[3] = {64, 1, 128};
+    if (!encode(&tq, q, 3, dq3, sq3, bq3) || !encode(&tdo, dout, 3, dq3, sq3, bq3))
+        return BI_ERR_CUDA;
+    return from_cuda(bi::launch_attention_backward(tq, tdo, p, kv->head_dim, rows, d->num_sms,
                                                    static_cast<cudaStream_t>(stream)));
 }
 

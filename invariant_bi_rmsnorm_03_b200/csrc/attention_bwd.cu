@@ -66,6 +66,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 template <int D>
 struct BwdCfg {
     static constexpr int TILE_BYTES = kQTile * D * 2;          // q or dO tile
+    static constexpr int BOX_BYTES = kQTile * 64 * 2;          // 64 values of 128 rows
     static constexpr int PAGE_BYTES = kPage * D * 2;           // one page block
     static constexpr int KGROUP_BYTES = PAGE_BYTES / 2;        // 8-key groups
     static constexpr int BLOCK_BYTES = (kKeyBlock / kPage) * PAGE_BYTES;  // 128 keys
@@ -209,7 +210,9 @@ __global__ void attn_bwd_prep_kernel(const uint16_t *__restrict__ o, const uint1
 // ---------------------------------------------------------------- dK, dV
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const AttnBwdParams p)
+__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq,
+                                                              const __grid_constant__ CUtensorMap tdo,
+                                                              const AttnBwdParams p)
 {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -224,7 +227,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
     float *sDelta = sLse + 2 * kQTile;                             // [2][128]
     uint64_t *bar = reinterpret_cast<uint64_t *>(sDelta + 2 * kQTile);
     uint64_t *drain = bar + 1;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *tbar = drain + 1;  // [2] the q and dO tiles of buffer b landed (TMA)
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(tbar + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     // block -> (sequence, kv head, key block)
@@ -254,14 +258,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
         while (j < nsteps && !sees(j)) ++j;
         return j;
     };
-    // the step's tiles (async) and this thread's row of its lse2 / Delta
+    // the step's q and dO tiles (TMA, thread 0: 64-value boxes of 128 rows,
+    // 128-byte swizzle, rows past the tensor zero) and this thread's row of
+    // its lse2 / Delta
+    uint32_t tphase = 0, tpending = 0;  // per buffer: parity to wait for, copy in flight
     auto fetch = [&](int j, int buf, float &lse_r, float &delta_r) {
         const int h = g * p.group + j / ntiles, qt = j % ntiles;
         const int rows = min(kQTile, n - qt * kQTile);
         const int64_t row0 = int64_t(q0) + int64_t(qt) * kQTile;
-        copy_tile<D>(sQ(buf), static_cast<const uint4 *>(p.q), row0, rows, p.Hq, h);
-        copy_tile<D>(sDO(buf), static_cast<const uint4 *>(p.dout), row0, rows, p.Hq, h);
-        cp_async_commit();
+        if (threadIdx.x == 0) {
+            mbar_arrive_expect_tx(&tbar[buf], 2u * C::TILE_BYTES);
+#pragma unroll
+            for (int x = 0; x < D / 64; ++x) {
+                tma_load_3d(sQ(buf) + x * C::BOX_BYTES, &tq, &tbar[buf], 64 * x, h, int(row0));
+                tma_load_3d(sDO(buf) + x * C::BOX_BYTES, &tdo, &tbar[buf], 64 * x, h, int(row0));
+            }
+        }
+        tpending |= 1u << buf;
         const int r = threadIdx.x;  // threads 0..127: one row each
         lse_r = r < rows ? p.lse2[(row0 + r) * p.Hq + h] : 0.0f;
         delta_r = r < rows ? p.delta[(row0 + r) * p.Hq + h] : 0.0f;
@@ -271,6 +284,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
     if (threadIdx.x == 0) {
         mbar_init(bar, 1);
         mbar_init(drain, 1);
+        mbar_init(&tbar[0], 1);
+        mbar_init(&tbar[1], 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -315,8 +330,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
             lse_s[threadIdx.x] = lse_r;
             delta_s[threadIdx.x] = delta_r;
         }
-        cp_async_wait<0>();        // this step's tiles (and, first, the key block) landed
-        fence_proxy_async_smem();  // ... and are read by the tensor core
+        cp_async_wait<0>();  // (first step) this thread's part of the key block landed
+        ok = block_wait(&tbar[buf], (tphase >> buf) & 1u, ctl);  // this step's tiles
+        if (!ok) break;
+        tphase ^= 1u << buf;
+        tpending &= ~(1u << buf);
+        if (rows < kQTile) {
+            // rows past the chunk (the next sequence's, or zeros past the
+            // tensor) become zeros: 128 bytes a row in each box (the swizzle
+            // moves 16-byte pieces only within their row)
+            const int per = (kQTile - rows) * 8;  // 16-byte pieces per box
+            for (int e = threadIdx.x; e < 2 * (D / 64) * per; e += kBwdThreads) {
+                const int box = e / per, off = e - box * per;
+                uint8_t *t = (box & 1 ? sDO(buf) : sQ(buf)) + (box >> 1) * C::BOX_BYTES;
+                reinterpret_cast<uint4 *>(t + rows * 128)[off] = make_uint4(0, 0, 0, 0);
+            }
+        }
+        fence_proxy_async_smem();  // the tiles (and the zeros) are read by the tensor core
         tc_fence_before();
         __syncthreads();
         // ------------------------------------------------ S^T, dP^T
@@ -324,10 +354,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
+                // q and dO as K-major operands: 16 values = 32 bytes of a
+                // swizzled 128-byte row, 64-value boxes BOX_BYTES apart
+                const uint32_t koff = (k >> 2) * C::BOX_BYTES + (k & 3) * 32;
                 mma_ss(tmem + C::S_COL, sdesc_plain(kb_addr + 256 * k, 128, C::KGROUP_BYTES),
-                       sdesc_plain(q_addr + 4096 * k, 2048, 128), idesc_s, k > 0 ? 1u : 0u);
+                       sdesc_sw128(q_addr + koff, 16, 1024), idesc_s, k > 0 ? 1u : 0u);
                 mma_ss(tmem + C::DP_COL, sdesc_plain(vb_addr + 256 * k, 128, C::KGROUP_BYTES),
-                       sdesc_plain(do_addr + 4096 * k, 2048, 128), idesc_s, k > 0 ? 1u : 0u);
+                       sdesc_sw128(do_addr + koff, 16, 1024), idesc_s, k > 0 ? 1u : 0u);
             }
             mma_commit(bar);
         }
@@ -375,10 +408,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
 #pragma unroll
             for (int jj = 0; jj < kQTile / 16; ++jj) {
                 const uint32_t acc = (first && jj == 0) ? 0u : 1u;
+                // dO and q as MN-major operands (N = head dim): 16 rows =
+                // 2048 bytes per K step, 8-row groups 1024 bytes apart,
+                // 64-value boxes BOX_BYTES apart along N
                 mma_ts(tmem + C::ACC0, tmem + C::S_COL + packed_step_col(jj),
-                       sdesc_plain(do_addr + 256 * jj, 128, 2048), idesc_acc, acc);
+                       sdesc_sw128(do_addr + 2048 * jj, C::BOX_BYTES, 1024), idesc_acc, acc);
                 mma_ts(tmem + C::ACC1, tmem + C::DP_COL + packed_step_col(jj),
-                       sdesc_plain(q_addr + 256 * jj, 128, 2048), idesc_acc, acc);
+                       sdesc_sw128(q_addr + 2048 * jj, C::BOX_BYTES, 1024), idesc_acc, acc);
             }
             mma_commit(bar);
         }
@@ -395,6 +431,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
         if (threadIdx.x == 0) {
             mma_commit(drain);
             drain_wait(drain, 0, p.timeout_ns);
+            for (int bb = 0; bb < 2; ++bb)
+                if (tpending & (1u << bb)) drain_wait(&tbar[bb], (tphase >> bb) & 1u, p.timeout_ns);
         }
     } else {
         // ---------------------------------------------------- write dV, dK
@@ -447,7 +485,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const Attn
 // ---------------------------------------------------------------- dQ
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnBwdParams p)
+__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq,
+                                                             const __grid_constant__ CUtensorMap tdo,
+                                                             const AttnBwdParams p)
 {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -461,7 +501,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
     auto sV = [&](int buf) { return kv_base + (2 + buf) * C::BLOCK_BYTES; };
     uint64_t *bar = reinterpret_cast<uint64_t *>(kv_base + 4 * C::BLOCK_BYTES + 2 * C::VEC_BYTES);
     uint64_t *drain = bar + 1;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *kvbar = drain + 1;  // [2] the K and V pages of buffer b landed (bulk copies)
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(kvbar + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     // block -> (sequence, query head, query tile)
@@ -484,6 +525,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
     if (threadIdx.x == 0) {
         mbar_init(bar, 1);
         mbar_init(drain, 1);
+        mbar_init(&kvbar[0], 1);
+        mbar_init(&kvbar[1], 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -493,12 +536,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
     }
     const int64_t row0 = int64_t(q0) + qt * kQTile;
     const int32_t *bt = p.block_table + int64_t(b) * p.max_pages;
+    // Page pg of key block kb: its physical page, or -1 when no key of it
+    // is in the sequence or its id is out of range (then it is zeroed).
+    auto page_of = [&](int kb, int pg) -> int {
+        const int lp = kb * (kKeyBlock / kPage) + pg;
+        if (lp * kPage >= kv_len) return -1;
+        const int phys = __ldg(bt + lp);
+        return (phys >= 0 && phys < p.num_pages) ? phys : -1;
+    };
+    // The block's K and V pages, one bulk copy per page block (thread 0).
+    uint32_t kvphase = 0, kvpending = 0;
     auto fetch = [&](int kb, int buf) {
-        copy_keys<D>(sK(buf), static_cast<const uint8_t *>(p.k_cache), bt, kb * kKeyBlock, kv_len,
-                     p.Hkv, g, p.num_pages, p.status);
-        copy_keys<D>(sV(buf), static_cast<const uint8_t *>(p.v_cache), bt, kb * kKeyBlock, kv_len,
-                     p.Hkv, g, p.num_pages, p.status);
-        cp_async_commit();
+        if (threadIdx.x == 0) {
+            uint32_t bytes = 0;
+            for (int pg = 0; pg < kKeyBlock / kPage; ++pg)
+                if (page_of(kb, pg) >= 0) bytes += 2u * C::PAGE_BYTES;
+            mbar_arrive_expect_tx(&kvbar[buf], bytes);
+            for (int pg = 0; pg < kKeyBlock / kPage; ++pg) {
+                const int phys = page_of(kb, pg);
+                const int lp = kb * (kKeyBlock / kPage) + pg;
+                if (phys < 0) {
+                    if (lp * kPage < kv_len) record_status(p.status, BI_DEV_BAD_INDEX);
+                    continue;
+                }
+                const int64_t off = (int64_t(phys) * p.Hkv + g) * int64_t(C::PAGE_BYTES);
+                bulk_load(sK(buf) + pg * C::PAGE_BYTES, static_cast<const uint8_t *>(p.k_cache) + off,
+                          C::PAGE_BYTES, &kvbar[buf]);
+                bulk_load(sV(buf) + pg * C::PAGE_BYTES, static_cast<const uint8_t *>(p.v_cache) + off,
+                          C::PAGE_BYTES, &kvbar[buf]);
+            }
+        }
+        kvpending |= 1u << buf;
     };
     copy_tile<D>(sQ, static_cast<const uint4 *>(p.q), row0, rows, p.Hq, h);
     copy_tile<D>(sDO, static_cast<const uint4 *>(p.dout), row0, rows, p.Hq, h);
@@ -529,7 +597,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
     for (int kb = 0; ok && kb * kKeyBlock <= last_key; ++kb) {
         const int k0 = kb * kKeyBlock;
         const uint32_t kb_addr = smem_u32(sK(buf)), vb_addr = smem_u32(sV(buf));
-        cp_async_wait<0>();        // this block's keys (and, first, the tile) landed
+        cp_async_wait<0>();  // (first step) this thread's part of the q and dO tiles landed
+        ok = block_wait(&kvbar[buf], (kvphase >> buf) & 1u, ctl);  // this block's K and V
+        if (!ok) break;
+        kvphase ^= 1u << buf;
+        kvpending &= ~(1u << buf);
+        // Pages not copied become zeros, and so do the keys past the sequence
+        // in its last page: K enters dQ += dS K, where a masked key's zero
+        // dS must not meet a stale NaN (V only enters dP, masked by
+        // selection, but is zeroed alike).
+        {
+            constexpr int PP = C::PAGE_BYTES / 16;  // 16-byte pieces of a page block
+            for (int pg = 0; pg < kKeyBlock / kPage; ++pg) {
+                const int key0 = k0 + pg * kPage;
+                const bool whole = page_of(kb, pg) < 0;
+                if (!whole && key0 + kPage <= kv_len) continue;  // copied, every key in
+                const int valid = whole ? 0 : kv_len - key0;     // keys of the page in the sequence
+                for (int e = threadIdx.x; e < 2 * PP; e += kBwdThreads) {
+                    const int piece = e % PP;
+                    const uint32_t off = uint32_t(piece) * 16u;
+                    const int r = int(off / (D * 16)) * 8 + int(off % 128) / 16;  // key of the piece
+                    if (r < valid) continue;
+                    uint8_t *dst = (e < PP ? sK(buf) : sV(buf)) + pg * C::PAGE_BYTES + off;
+                    *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+                }
+            }
+        }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -599,6 +692,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
         if (threadIdx.x == 0) {
             mma_commit(drain);
             drain_wait(drain, 0, p.timeout_ns);
+            for (int bb = 0; bb < 2; ++bb)
+                if (kvpending & (1u << bb)) drain_wait(&kvbar[bb], (kvphase >> bb) & 1u, p.timeout_ns);
         }
     } else {
         // every thread takes part in the warp's TMEM loads; rows past the
@@ -637,7 +732,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const AttnB
 
 size_t attn_bwd_ws_bytes(int64_t rows) { return size_t(rows) * 2 * sizeof(float); }
 
-cudaError_t launch_attention_backward(const AttnBwdParams &p_in, int head_dim, int64_t rows,
+cudaError_t launch_attention_backward(const CUtensorMap &tq, const CUtensorMap &tdo,
+                                      const AttnBwdParams &p_in, int head_dim, int64_t rows,
                                       int num_sms, cudaStream_t s)
 {
     AttnBwdParams p = p_in;
@@ -661,9 +757,9 @@ cudaError_t launch_attention_backward(const AttnBwdParams &p_in, int head_dim, i
             (e = cudaFuncSetAttribute(attn_bwd_dq_kernel<128>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM)) != cudaSuccess)
             return e;
-        attn_bwd_dkv_kernel<128><<<unsigned(dkv_blocks), kBwdThreads, C::SMEM, s>>>(p);
+        attn_bwd_dkv_kernel<128><<<unsigned(dkv_blocks), kBwdThreads, C::SMEM, s>>>(tq, tdo, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        attn_bwd_dq_kernel<128><<<unsigned(dq_blocks), kBwdThreads, C::SMEM, s>>>(p);
+        attn_bwd_dq_kernel<128><<<unsigned(dq_blocks), kBwdThreads, C::SMEM, s>>>(tq, tdo, p);
     } else {
         using C = BwdCfg<64>;
         if ((e = cudaFuncSetAttribute(attn_bwd_dkv_kernel<64>,
@@ -671,9 +767,9 @@ cudaError_t launch_attention_backward(const AttnBwdParams &p_in, int head_dim, i
             (e = cudaFuncSetAttribute(attn_bwd_dq_kernel<64>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM)) != cudaSuccess)
             return e;
-        attn_bwd_dkv_kernel<64><<<unsigned(dkv_blocks), kBwdThreads, C::SMEM, s>>>(p);
+        attn_bwd_dkv_kernel<64><<<unsigned(dkv_blocks), kBwdThreads, C::SMEM, s>>>(tq, tdo, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        attn_bwd_dq_kernel<64><<<unsigned(dq_blocks), kBwdThreads, C::SMEM, s>>>(p);
+        attn_bwd_dq_kernel<64><<<unsigned(dq_blocks), kBwdThreads, C::SMEM, s>>>(tq, tdo, p);
     }
     return cudaGetLastError();
 }

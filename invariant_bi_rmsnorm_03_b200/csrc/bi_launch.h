@@ -157,7 +157,10 @@ struct AttnBwdParams {
     uint64_t timeout_ns;
 };
 size_t attn_bwd_ws_bytes(int64_t rows);
-cudaError_t launch_attention_backward(const AttnBwdParams &p, int head_dim, int64_t rows,
+// tq, tdo: 3D tensor maps (D, Hq, T) of q and dO, boxes of 64 x 1 x 128,
+// 128-byte swizzle (the dK/dV kernel's tile loads).
+cudaError_t launch_attention_backward(const CUtensorMap &tq, const CUtensorMap &tdo,
+                                      const AttnBwdParams &p, int head_dim, int64_t rows,
                                       int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- decoder glue
