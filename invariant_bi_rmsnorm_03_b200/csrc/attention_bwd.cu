@@ -32,13 +32,17 @@
 // P and dS are rounded to bf16 to enter the tensor core (as the forward
 // rounds P before P V); every other quantity is fp32.
 //
-// Shared-memory operands are in the tensor core's no-swizzle core-matrix
-// layout (8 rows x 16 bytes = 128 contiguous bytes): a 128-row tile of q or dO
-// as [value block d/8][row 128][8 values], a 128-key block of the cache as its
-// eight page blocks, already in that layout.  Every tile is copied by the
-// threads with 16-byte asynchronous copies (cp.async; rows outside the
-// sequence or the chunk become zeros, so that a masked product never meets
-// a stale NaN) into a second buffer while the current step computes.
+// Shared-memory operands: a 128-row tile of q or dO is loaded by TMA as
+// 64-value boxes of 128 rows with the 128-byte swizzle, which serves both as
+// a K-major operand (for S^T, dP^T, S, dP) and as an MN-major one (for dV,
+// dK); a 128-key block of the cache is its eight page blocks, already in the
+// no-swizzle core-matrix order, copied whole (the dK/dV kernel's, once, by
+// the threads; the dQ kernel's, per step, by one bulk copy per page block).
+// The next step's tiles or block land in a second buffer while the current
+// step computes.  Rows a masked product could meet as 0 x NaN are zeroed in
+// shared memory first: q/dO rows past the chunk in the dK/dV kernel (they
+// enter dV and dK through a zero P or dS) and keys past the sequence in the
+// dQ kernel (they enter dQ through a zero dS).
 //
 // Block of 256 threads (8 warps; warps w and w + 4 share TMEM lanes
 // 32(w%4) .. +31, each taking half of the columns).  Thread 0 issues the
@@ -93,9 +97,6 @@ static_assert(kQTile == 128 && kKeyBlock == 128, "four 32-column chunks, two per
 __device__ __forceinline__ uint32_t packed_chunk_col(int c) { return 64u * (c >> 1) + 16u * (c & 1); }
 __device__ __forceinline__ uint32_t packed_step_col(int j) { return 64u * (j >> 2) + 8u * (j & 3); }
 
-// Byte offset of values 8c .. 8c+7 of row r in a 128-row tile.
-__device__ __forceinline__ uint32_t tile_off(int r, int c) { return (uint32_t(c) * 128u + r) * 16u; }
-
 // Byte offset, inside a page block of head dim D, of values 8c .. 8c+7 of key r.
 template <int D>
 __device__ __forceinline__ uint32_t page_off(int r, int c)
@@ -107,28 +108,6 @@ __device__ __forceinline__ uint32_t pack2(float a, float b)
 {
     __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t *>(&p);
-}
-
-// Rows row0 .. row0+127 of one head of a [T, H, D] bf16 tensor into a tile,
-// asynchronously (the caller commits and waits); rows at or past `rows` are
-// zero.  A warp moves blocks of 8 rows x 4 pieces (64 contiguous bytes of
-// each row: whole 32-byte sectors; the 8 threads of a store phase write 8
-// consecutive 16-byte cells of the tile: no bank conflict).
-template <int D>
-__device__ __forceinline__ void copy_tile(uint8_t *tile, const uint4 *src, int64_t row0, int rows,
-                                          int H, int h)
-{
-    constexpr int P = D / 8;                         // 16-byte pieces of a row
-    constexpr int ITER = kQTile * P / kBwdThreads;   // pieces per thread
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#pragma unroll
-    for (int i = 0; i < ITER; ++i) {
-        const int blk = warp + (kBwdThreads / 32) * i;  // blocks of 8 rows x 4 pieces
-        const int r = (blk % (kQTile / 8)) * 8 + (lane & 7);
-        const int c = (blk / (kQTile / 8)) * 4 + (lane >> 3);
-        const bool ok = r < rows;                    // (row 0 always exists)
-        cp_async16(tile + tile_off(r, c), src + ((row0 + (ok ? r : 0)) * H + h) * P + c, ok);
-    }
 }
 
 // Keys k0 .. k0+127 of kv head g of one sequence (its page-table row `bt`)
@@ -232,10 +211,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     // block -> (sequence, kv head, key block)
-    const int nkb = p.num_key_blocks;
-    const int kb = blockIdx.x % nkb;
-    const int g = (blockIdx.x / nkb) % p.Hkv;
-    const int b = blockIdx.x / (nkb * p.Hkv);
+    // (key blocks slowest, ascending: the blocks with the most query tiles
+    // start first -- a longest-first schedule of the waves)
+    const int bh = blockIdx.x % (p.B * p.Hkv);
+    const int kb = blockIdx.x / (p.B * p.Hkv);
+    const int g = bh % p.Hkv;
+    const int b = bh / p.Hkv;
     const int q0 = p.cu_q[b], n = p.cu_q[b + 1] - q0, ctx = p.ctx_lens[b];
     const int kv_len = ctx + n;
     const int k0 = kb * kKeyBlock;
@@ -502,14 +483,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
     uint64_t *bar = reinterpret_cast<uint64_t *>(kv_base + 4 * C::BLOCK_BYTES + 2 * C::VEC_BYTES);
     uint64_t *drain = bar + 1;
     uint64_t *kvbar = drain + 1;  // [2] the K and V pages of buffer b landed (bulk copies)
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(kvbar + 2);
+    uint64_t *qbar = kvbar + 2;   // the q and dO tiles landed (TMA)
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(qbar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     // block -> (sequence, query head, query tile)
+    // (tiles slowest, the last -- longest -- first: a longest-first
+    // schedule of the waves)
     const int nqt = p.num_q_tiles;
-    const int qt = blockIdx.x % nqt;
-    const int h = (blockIdx.x / nqt) % p.Hq;
-    const int b = blockIdx.x / (nqt * p.Hq);
+    const int bh = blockIdx.x % (p.B * p.Hq);
+    const int qt = nqt - 1 - blockIdx.x / (p.B * p.Hq);
+    const int h = bh % p.Hq;
+    const int b = bh / p.Hq;
     const int q0 = p.cu_q[b], n = p.cu_q[b + 1] - q0, ctx = p.ctx_lens[b];
     const int kv_len = ctx + n;
     if (qt * kQTile >= n) return;
@@ -527,6 +512,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
         mbar_init(drain, 1);
         mbar_init(&kvbar[0], 1);
         mbar_init(&kvbar[1], 1);
+        mbar_init(qbar, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -568,8 +554,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
         }
         kvpending |= 1u << buf;
     };
-    copy_tile<D>(sQ, static_cast<const uint4 *>(p.q), row0, rows, p.Hq, h);
-    copy_tile<D>(sDO, static_cast<const uint4 *>(p.dout), row0, rows, p.Hq, h);
+    // the tile's q and dO rows (TMA, 64-value boxes, 128-byte swizzle; rows
+    // past the chunk are other rows' data or zeros, and a row's dQ depends
+    // on that row alone, so they are left as they land)
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(qbar, 2u * C::TILE_BYTES);
+#pragma unroll
+        for (int x = 0; x < D / 64; ++x) {
+            tma_load_3d(sQ + x * C::BOX_BYTES, &tq, qbar, 64 * x, h, int(row0));
+            tma_load_3d(sDO + x * C::BOX_BYTES, &tdo, qbar, 64 * x, h, int(row0));
+        }
+    }
+    bool qpending = true;
     fetch(0, 0);
     tc_fence_before();
     __syncthreads();
@@ -597,7 +593,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
     for (int kb = 0; ok && kb * kKeyBlock <= last_key; ++kb) {
         const int k0 = kb * kKeyBlock;
         const uint32_t kb_addr = smem_u32(sK(buf)), vb_addr = smem_u32(sV(buf));
-        cp_async_wait<0>();  // (first step) this thread's part of the q and dO tiles landed
+        if (qpending) {  // (first step) the q and dO tiles
+            ok = block_wait(qbar, 0, ctl);
+            if (!ok) break;
+            qpending = false;
+        }
         ok = block_wait(&kvbar[buf], (kvphase >> buf) & 1u, ctl);  // this block's K and V
         if (!ok) break;
         kvphase ^= 1u << buf;
@@ -630,9 +630,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
-                mma_ss(tmem + C::S_COL, sdesc_plain(q_addr + 4096 * k, 2048, 128),
+                const uint32_t koff = (k >> 2) * C::BOX_BYTES + (k & 3) * 32;  // K-major, swizzled
+                mma_ss(tmem + C::S_COL, sdesc_sw128(q_addr + koff, 16, 1024),
                        sdesc_plain(kb_addr + 256 * k, 128, C::KGROUP_BYTES), idesc_s, k > 0 ? 1u : 0u);
-                mma_ss(tmem + C::DP_COL, sdesc_plain(do_addr + 4096 * k, 2048, 128),
+                mma_ss(tmem + C::DP_COL, sdesc_sw128(do_addr + koff, 16, 1024),
                        sdesc_plain(vb_addr + 256 * k, 128, C::KGROUP_BYTES), idesc_s, k > 0 ? 1u : 0u);
             }
             mma_commit(bar);
@@ -694,6 +695,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
             drain_wait(drain, 0, p.timeout_ns);
             for (int bb = 0; bb < 2; ++bb)
                 if (kvpending & (1u << bb)) drain_wait(&kvbar[bb], (kvphase >> bb) & 1u, p.timeout_ns);
+            if (qpending) drain_wait(qbar, 0, p.timeout_ns);
         }
     } else {
         // every thread takes part in the warp's TMEM loads; rows past the
