@@ -341,7 +341,8 @@ def e2e_pipelined(torch, L, wl, steps, legs=("gemm", "decode", "prefill")):
     are copied out on a third.  Device inputs and outputs are double
     buffered; every copy and every launch of the K steps is inside the timed
     region (first copy-in to last copy-out), each step starts with the L2
-    flush.  Returns the mean time of a step in ms."""
+    flush.  Returns the mean time of a step in ms and whether the last
+    step's results, copied out, equal the step computed plainly bit for bit."""
     T = torch
     dev = wl.x.device
     host_in = {"x": wl.x, "dec_q": wl.dec_q, "dec_knew": wl.dec_knew, "dec_vnew": wl.dec_vnew,
@@ -411,8 +412,18 @@ def e2e_pipelined(torch, L, wl, steps, legs=("gemm", "decode", "prefill")):
 
     run(3, False)
     ms = run(steps, True)
-    del bufs
-    return ms
+    # the pipeline's last results against the same step run plainly
+    ref = {n: T.empty_like(outs[n]) for n in names_out}
+    with T.cuda.stream(s_c):
+        bf = dict(bufs[0])
+        for n in names_in:
+            bf[n].copy_(hin[n])
+        bf.update(ref)
+        compute(bf)
+    T.cuda.synchronize()
+    same = all(T.equal(hout[n].view(T.int16), ref[n].cpu().view(T.int16)) for n in names_out)
+    del bufs, ref
+    return ms, same
 
 
 def invariance_checks(torch, L, wl) -> dict:
@@ -726,9 +737,10 @@ def run_ours(args):
     # e2e through host buffers
     e2e_per, h2d, d2h = e2e_steps(torch, L, wl, max(2, args.steps // 2), 1)
     pipe_steps = max(4, args.steps // 2)
-    pipe_gemm_ms = maxall(e2e_pipelined(torch, L, wl, pipe_steps, ("gemm",)))
-    pipe_dec_ms = maxall(e2e_pipelined(torch, L, wl, pipe_steps, ("decode",)))
-    pipe_step_ms = maxall(e2e_pipelined(torch, L, wl, pipe_steps))
+    pipe = [e2e_pipelined(torch, L, wl, pipe_steps, legs)
+            for legs in (("gemm",), ("decode",), ("gemm", "decode", "prefill"))]
+    pipe_gemm_ms, pipe_dec_ms, pipe_step_ms = (maxall(ms) for ms, _ in pipe)
+    pipe_same = all(same for _, same in pipe)
     e2e_gemm_ms = maxall(float(e2e_per[:, 0].mean()))
     e2e_dec_ms = maxall(float(e2e_per[:, 1].mean()))
     e2e_step_ms = maxall(float(e2e_per.sum(axis=1).mean()))
@@ -841,6 +853,7 @@ def run_ours(args):
                 "split_kv_attn_gbs": world * wl.dec_bytes / (pipe_dec_ms * 1e-3) / 1e9,
                 "step_ms": pipe_step_ms,
                 "legs_ms": {"rmsnorm_matmul": pipe_gemm_ms, "kv_write_decode": pipe_dec_ms},
+                "results_equal_serial": pipe_same,
                 "serial": {"step_ms": e2e_step_ms,
                            "legs_ms": {"rmsnorm_matmul": e2e_gemm_ms, "kv_write_decode": e2e_dec_ms,
                                        "kv_write_prefill": e2e_pre_ms},
