@@ -151,8 +151,13 @@ class Workload:
         rec(5)
 
     def launches_per_step(self, L) -> int:
+        # two cache writes, RMSNorm, matmul, the decode launch order (the
+        # bench's batch has more blocks than SMs), decode attention, its
+        # combine when a sequence is split over blocks (the workspace then
+        # holds split records beyond the order array), prefill
         ws = L.bi_attention_decode_workspace_bytes(self.dec_kv, DEC_B, DEC_HQ, DEC_MAXLEN)
-        return 2 + 1 + 1 + 1 + (1 if ws > 0 else 0) + 1
+        order = (4 * DEC_B + 255) // 256 * 256
+        return 2 + 1 + 1 + 1 + 1 + (1 if ws > order else 0) + 1
 
 
 # ---------------------------------------------------------------- clocks

@@ -681,7 +681,14 @@ static bi_status decode_launch(const DeviceState *d, const bi_paged_kv *kv, cons
     p.decode = 1;
     p.B = B;
     p.seq_lens = seq_lens;
-    p.order = order;
+    // The launch order only decides which blocks start first; when every
+    // block of the launch fits in one wave (one block per SM) nothing waits,
+    // so the sorting launch is skipped (the kernel reads a null order as the
+    // identity).
+    const int64_t items = int64_t(per_sequence ? chunks : (max_splits + splits_per_cta - 1) /
+                                                              splits_per_cta) * Hkv * B;
+    const bool sort = B > 1 && items > d->num_sms;
+    p.order = sort ? order : nullptr;
     p.splits_per_cta = splits_per_cta;
     // a division chosen from the load cuts each sequence into `chunks`
     // blocks of its own length; an explicit one uses splits_per_cta for all
@@ -699,8 +706,11 @@ static bi_status decode_launch(const DeviceState *d, const bi_paged_kv *kv, cons
     const uint64_t sq[2] = {uint64_t(D) * 2, uint64_t(Hq) * D * 2};
     const uint32_t bq[3] = {64, uint32_t(p.rows_per_q), 1};
     if (!encode(&tq, q, 3, dq, sq, bq)) return BI_ERR_CUDA;
-    cudaError_t e = bi::launch_attn_order(seq_lens, B, order, s);
-    if (e != cudaSuccess) return BI_ERR_CUDA;
+    cudaError_t e = cudaSuccess;
+    if (sort) {
+        e = bi::launch_attn_order(seq_lens, B, order, s);
+        if (e != cudaSuccess) return BI_ERR_CUDA;
+    }
     e = bi::launch_attention(tq, p, D, s);
     if (e != cudaSuccess) return BI_ERR_CUDA;
     if (chunks > 1) e = bi::launch_attn_combine(p, D, s);

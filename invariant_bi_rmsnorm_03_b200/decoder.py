@@ -258,7 +258,6 @@ class ToyDecoder:
         self.v_cache = [torch.zeros(shape, dtype=torch.bfloat16, device=self.dev)
                         for _ in range(cfg.layers)]
         self.num_pages = num_pages
-        self.launches = 0
         # fused form: each matmul that follows an RMSNorm takes its weight with
         # the norm weight folded in (once, here)
         self.wf = {}
@@ -298,10 +297,7 @@ class ToyDecoder:
         o = torch.empty((T, c.n_heads, c.head_dim), dtype=torch.bfloat16, device=self.dev)
         # the fused norm forms' row statistics, one buffer for the whole step
         nws = L._norm_ws(T, self.dev) if c.fused else None
-        if c.fused:
-            h, n = None, 1
-        else:
-            h, n = L.bi_rmsnorm(x, W["l0.attn_norm"], c.eps), 2
+        h = None if c.fused else L.bi_rmsnorm(x, W["l0.attn_norm"], c.eps)
         for i in range(c.layers):
             kv_all = PagedKV(self.k_cache[i], self.v_cache[i], bt)
             if c.fused:
@@ -315,31 +311,25 @@ class ToyDecoder:
             if Bd:
                 kv = PagedKV(self.k_cache[i], self.v_cache[i], bt[:Bd])
                 L.bi_attention_decode(kv, q[:Bd], dec_lens, max_len, out=o[:Bd])
-                n += 2
             if plan.pre:
                 kv = PagedKV(self.k_cache[i], self.v_cache[i], bt[Bd:])
                 L.bi_attention_prefill(kv, q[Bd:], cu, ctx, max_chunk, out=o[Bd:])
-                n += 1
             if c.fused:
                 # x += o Wo^T; x += swiglu(RMSNorm(x) Wgu^T) Wdown^T
                 L.bi_matmul_residual(o.view(T, c.n_heads * c.head_dim), W["l%d.wo" % i], x,
                                      out=x)
                 f = L.bi_swiglu(L.bi_rmsnorm_matmul(x, self.wf["l%d.wgu" % i], c.eps, ws=nws))
                 L.bi_matmul_residual(f, W["l%d.wdown" % i], x, out=x)
-                n += 7  # each norm form: the row statistics, then the matmul
                 continue
             a = L.bi_matmul(o.view(T, c.n_heads * c.head_dim), W["l%d.wo" % i])
             h = L.bi_add_rmsnorm(x, a, W["l%d.mlp_norm" % i], c.eps)
             if c.n_experts:
-                m, nm = self._moe(h, i)
-                n += nm
+                m = self._moe(h, i)
             else:
                 f = L.bi_swiglu(L.bi_matmul(h, W["l%d.wgu" % i]))
                 m = L.bi_matmul(f, W["l%d.wdown" % i])
-                n += 3
             nxt = W["l%d.attn_norm" % (i + 1)] if i + 1 < c.layers else W["final_norm"]
             h = L.bi_add_rmsnorm(x, m, nxt, c.eps)
-            n += 5
         if c.fused:
             last = L.bi_embedding(x, rows)
             logits = L.bi_rmsnorm_matmul(last, self.wf["lm_head"], c.eps, out_dtype=torch.float32,
@@ -350,13 +340,12 @@ class ToyDecoder:
         nt = L.bi_sample(logits, self._to_dev(plan.temperature), self._to_dev(plan.top_p),
                          self._to_dev(plan.seed.view(np.int64)),
                          self._to_dev(plan.offset.view(np.int64)))
-        self.launches += n + (4 if c.fused else 3)
         return nt.cpu().numpy()
 
 
     def _moe(self, h: torch.Tensor, i: int):
-        """The mixture-of-experts feed-forward of layer i; returns (output,
-        launches).  All experts' matmuls run in one grouped launch each, their
+        """The mixture-of-experts feed-forward of layer i; returns its output.
+        All experts' matmuls run in one grouped launch each, their
         tiles laid out on the device from the dispatch offsets (no host
         read-back)."""
         L, c, W = self.L, self.cfg, self.w
@@ -366,7 +355,7 @@ class ToyDecoder:
         xs = L.bi_embedding(h, tok)                  # rows grouped by expert
         f = L.bi_swiglu(L.bi_matmul_grouped(xs, W["l%d.moe_wgu" % i], off))
         ys = L.bi_matmul_grouped(f, W["l%d.moe_wdown" % i], off)
-        return L.bi_moe_combine(ys, pos, gates), 8
+        return L.bi_moe_combine(ys, pos, gates)
 
 
 def run(sched: Scheduler, model: ToyDecoder, max_steps: int = 1_000_000) -> int:
