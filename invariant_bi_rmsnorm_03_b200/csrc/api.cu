@@ -140,6 +140,17 @@ bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H
                                         static_cast<cudaStream_t>(stream)));
 }
 
+static bi_status gemm_maps(const void *a, const void *w, int64_t M, int64_t N, int64_t K,
+                           CUtensorMap *ta, CUtensorMap *tw)
+{
+    const uint64_t da[2] = {uint64_t(K), uint64_t(M)}, sa[1] = {uint64_t(K) * 2};
+    const uint64_t dw[2] = {uint64_t(K), uint64_t(N)}, sw[1] = {uint64_t(K) * 2};
+    // each CTA of a pair loads kGemmCtaRows rows of A and of W per K slice
+    const uint32_t box[2] = {uint32_t(bi::kGemmBK), uint32_t(bi::kGemmCtaRows)};
+    if (!encode(ta, a, 2, da, sa, box) || !encode(tw, w, 2, dw, sw, box)) return BI_ERR_CUDA;
+    return BI_OK;
+}
+
 bi_status bi_matmul_grouped(const void *a, const void *w, void *c, const int64_t *offsets,
                             int32_t groups, int64_t rows, int64_t N, int64_t K, bi_dtype out_dtype,
                             void *stream)
@@ -155,11 +166,7 @@ bi_status bi_matmul_grouped(const void *a, const void *w, void *c, const int64_t
     bi_status st = device_state(&d);
     if (st != BI_OK) return st;
     CUtensorMap ta, tw;
-    const uint64_t da[2] = {uint64_t(K), uint64_t(rows)}, sa[1] = {uint64_t(K) * 2};
-    const uint64_t dw[2] = {uint64_t(K), uint64_t(groups) * uint64_t(N)}, sw[1] = {uint64_t(K) * 2};
-    const uint32_t ba[2] = {uint32_t(bi::kGemmBK), 128u};
-    const uint32_t bw[2] = {uint32_t(bi::kGemmBK), 128u};
-    if (!encode(&ta, a, 2, da, sa, ba) || !encode(&tw, w, 2, dw, sw, bw)) return BI_ERR_CUDA;
+    if ((st = gemm_maps(a, w, rows, int64_t(groups) * N, K, &ta, &tw)) != BI_OK) return st;
     return from_cuda(bi::launch_gemm_grouped(ta, tw, c, int(rows), int(N), int(K),
                                              out_dtype == BI_F32, offsets, groups, d->num_sms,
                                              d->status, bi::kDefaultTimeoutNs,
@@ -172,16 +179,6 @@ static bool gemm_shape_ok(int64_t M, int64_t N, int64_t K)
            N <= INT32_MAX && K <= INT32_MAX;
 }
 
-static bi_status gemm_maps(const void *a, const void *w, int64_t M, int64_t N, int64_t K,
-                           CUtensorMap *ta, CUtensorMap *tw)
-{
-    const uint64_t da[2] = {uint64_t(K), uint64_t(M)}, sa[1] = {uint64_t(K) * 2};
-    const uint64_t dw[2] = {uint64_t(K), uint64_t(N)}, sw[1] = {uint64_t(K) * 2};
-    // each CTA of a pair loads 128 rows of A and 128 rows of W per K slice
-    const uint32_t box[2] = {uint32_t(bi::kGemmBK), 128u};
-    if (!encode(ta, a, 2, da, sa, box) || !encode(tw, w, 2, dw, sw, box)) return BI_ERR_CUDA;
-    return BI_OK;
-}
 
 bi_status bi_fold_norm_weight(const void *W, const void *w, void *wf, int64_t N, int64_t K,
                               void *stream)
@@ -482,12 +479,7 @@ bi_status bi_matmul(const void *a, const void *w, void *c, int64_t M, int64_t N,
             return BI_ERR_WORKSPACE;
     }
     CUtensorMap ta, tw;
-    const uint64_t da[2] = {uint64_t(K), uint64_t(M)}, sa[1] = {uint64_t(K) * 2};
-    const uint64_t dw[2] = {uint64_t(K), uint64_t(N)}, sw[1] = {uint64_t(K) * 2};
-    // each CTA of a pair loads 128 rows of A and 128 rows of W per K slice
-    const uint32_t ba[2] = {uint32_t(bi::kGemmBK), 128u};
-    const uint32_t bw[2] = {uint32_t(bi::kGemmBK), 128u};
-    if (!encode(&ta, a, 2, da, sa, ba) || !encode(&tw, w, 2, dw, sw, bw)) return BI_ERR_CUDA;
+    if ((st = gemm_maps(a, w, M, N, K, &ta, &tw)) != BI_OK) return st;
     return from_cuda(bi::launch_gemm(ta, tw, c, int(M), int(N), int(K), out_dtype == BI_F32,
                                      static_cast<float *>(ws), ks, d->num_sms, d->status,
                                      bi::kDefaultTimeoutNs, static_cast<cudaStream_t>(stream)));

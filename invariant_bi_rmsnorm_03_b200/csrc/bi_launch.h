@@ -24,6 +24,10 @@ cudaError_t launch_row_rstd(const void *x, float *r, int64_t M, int64_t H, float
 
 // ---------------------------------------------------------------- matmul
 constexpr int kGemmBK = 64;  // K slice; the output tile is 256 x 256 per SM pair
+// Rows of A and of W that each CTA of a pair loads per K slice: the box of
+// both tensor maps (every form encodes them through one function) and the
+// kernel's stage layout.
+constexpr int kGemmCtaRows = 128;
 size_t gemm_smem_bytes();
 // k_splits > 1 only in the variant-off build: fp32 partial sums go to ws
 // ([k_splits, M, N]) and a second kernel adds them.

@@ -256,9 +256,10 @@ __device__ __noinline__ void qkv_epilogue(const GemmEpi &epi, uint32_t tbase, in
 namespace pair {
 
 constexpr int BM = 256, BN = 256, BK = kGemmBK, STAGES = 7;
-constexpr int A_BYTES = 128 * BK * 2;   // 16 KB: this CTA's half of the A slice
-constexpr int W_BYTES = 128 * BK * 2;   // 16 KB: this CTA's half of the W slice
+constexpr int A_BYTES = kGemmCtaRows * BK * 2;  // 16 KB: this CTA's half of the A slice
+constexpr int W_BYTES = kGemmCtaRows * BK * 2;  // 16 KB: this CTA's half of the W slice
 constexpr int STAGE_BYTES = A_BYTES + W_BYTES;
+static_assert(2 * kGemmCtaRows == BM && 2 * kGemmCtaRows == BN, "a pair's two CTAs cover the tile");
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;     // two 128-lane x 256-column fp32 accumulators
 constexpr int BAR_BYTES = 256;
@@ -394,9 +395,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     const uint32_t bar = map_to_cta(smem_u32(&full[stage]), 0);
                     if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
                     tma_load_2d_pair(sA + stage * A_BYTES, &tma, bar, kb * BK,
-                                     int(t.row0) + int(rank) * 128);
+                                     int(t.row0) + int(rank) * kGemmCtaRows);
                     tma_load_2d_pair(sW + stage * W_BYTES, &tmw, bar, kb * BK,
-                                     int(t.w_row0) + int(rank) * 128);
+                                     int(t.w_row0) + int(rank) * kGemmCtaRows);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
