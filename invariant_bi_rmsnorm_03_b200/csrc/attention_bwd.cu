@@ -144,10 +144,11 @@ __device__ __forceinline__ void copy_keys(uint8_t *dst, const uint8_t *cache, co
 }
 
 // Waits for phase `parity` of `bar` on every thread; the block agrees on the
-// outcome (true only if every thread saw the phase complete).
+// outcome (true only if every thread saw the phase complete).  The whole
+// block waits on each step's products, so the wait polls before it sleeps.
 __device__ __forceinline__ bool block_wait(uint64_t *bar, uint32_t parity, const WaitCtl &ctl)
 {
-    const bool ok = wait(bar, parity, ctl);
+    const bool ok = wait_spin(bar, parity, ctl);
     return __syncthreads_and(ok ? 1 : 0) != 0;
 }
 

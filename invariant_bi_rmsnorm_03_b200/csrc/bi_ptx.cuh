@@ -67,6 +67,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // As mbar_try_wait, but the thread may sleep up to `hint_ns` nanoseconds
 // for the phase to complete instead of returning at once: a waiting warp
 // then takes no issue slots from the warps doing the work.
@@ -119,6 +133,17 @@ __device__ __forceinline__ bool wait_inl(uint64_t *bar, uint32_t parity, const W
 static __device__ __noinline__ bool wait(uint64_t *bar, uint32_t parity, const WaitCtl &ctl)
 {
     return wait_inl(bar, parity, ctl);
+}
+
+// For a thread whose waits pace a pipeline (the one that issues the MMAs):
+// polls the phase a bounded number of times first, since a suspended
+// thread resumes some hundred cycles after the phase completes, then waits
+// as `wait` does.
+__device__ __forceinline__ bool wait_spin(uint64_t *bar, uint32_t parity, const WaitCtl &ctl)
+{
+    for (int i = 0; i < 2048; ++i)
+        if (mbar_test_wait(bar, parity)) return true;
+    return wait(bar, parity, ctl);
 }
 
 // ---------------------------------------------------------------- proxies

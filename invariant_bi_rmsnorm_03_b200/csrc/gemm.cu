@@ -388,7 +388,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             for (int u = pair_id; ok && u < units; u += num_pairs) {
                 const Unit t = unit(u);
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
-                    if (!wait(&empty[stage], phase ^ 1u, ctl)) {
+                    if (!wait_spin(&empty[stage], phase ^ 1u, ctl)) {
                         ok = false;
                         break;
                     }
@@ -423,7 +423,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 tc_fence_after();
                 const uint32_t d = tmem + uint32_t(acc * BN);
                 for (int kb = t.kb0; kb < t.kb1; ++kb) {
-                    if (!wait(&full[stage], phase, ctl)) {
+                    if (!wait_spin(&full[stage], phase, ctl)) {
                         ok = false;
                         break;
                     }

@@ -58,9 +58,9 @@ def test_moe_feed_forward_rows_do_not_depend_on_the_batch(L):
     model = ToyDecoder(L, cfg, w, 4, DEV)
     g = rng(181)
     h = dev_bf16(normal_bf16(g, (300, cfg.hidden)))
-    full, _ = model._moe(h, 0)
+    full = model._moe(h, 0)
     for sel in (np.array([5]), np.arange(10, 40), g.choice(300, 150, replace=False)):
-        part, _ = model._moe(h[torch.from_numpy(sel).to(DEV)].contiguous(), 0)
+        part = model._moe(h[torch.from_numpy(sel).to(DEV)].contiguous(), 0)
         assert same_bytes(part, full[torch.from_numpy(sel).to(DEV)]), len(sel)
     # and one token against the oracle: route, its k experts' feed-forwards, combine
     rl = L.bi_matmul(h[:1], w["l0.router"], out_dtype=torch.float32).cpu().numpy()
