@@ -266,6 +266,8 @@ constexpr int BAR_BYTES = 256;
 constexpr int CUM_BYTES = (kMaxGemmGroups + 1) * 4;  // grouped mode: tiles before each group
 static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barriers, TMEM address and abort flag");
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + CUM_BYTES;
+// shared addresses fit the 14-bit field (16-byte units) of a matrix descriptor
+static_assert(SMEM_BYTES + 4096 <= (1 << 18), "descriptor address field");
 
 // The tile of work unit u.  Plain: tiles m-fastest over an M x N output
 // (split-K units only in the variant-off build).  Grouped: the rows of group
@@ -409,6 +411,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (lane == 0 && leader) {
             // ------------------------------------------------ MMA issue (leader)
             const uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
+            const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA), 16, 1024);
+            const uint64_t w_desc0 = sdesc_sw128(smem_u32(sW), 16, 1024);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -416,7 +420,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             bool ok = true;
             for (int u = pair_id; ok && u < units; u += num_pairs) {
                 const Unit t = unit(u);
-                if (!wait(&tempty[acc], acc_phase ^ 1u, ctl)) {
+                if (!wait_spin(&tempty[acc], acc_phase ^ 1u, ctl)) {
                     ok = false;
                     break;
                 }
@@ -428,14 +432,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
-                    const uint32_t w0 = smem_u32(sW + stage * W_BYTES);
+                    // the descriptors of stage 0 plus the stage's and the K
+                    // step's offsets, in the 16-byte units of the address
+                    // field (every address stays below 2^18 bytes, so the
+                    // sums never carry out of the field)
+                    const uint64_t ad = a_desc0 + uint64_t(stage * (A_BYTES >> 4));
+                    const uint64_t wd = w_desc0 + uint64_t(stage * (W_BYTES >> 4));
+                    mma_ss_pair(d, ad, wd, idesc, kb > t.kb0 ? 1u : 0u);
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k) {
-                        mma_ss_pair(d, sdesc_sw128(a0 + 32 * k, 16, 1024),
-                                    sdesc_sw128(w0 + 32 * k, 16, 1024), idesc,
-                                    (kb > t.kb0 || k > 0) ? 1u : 0u);
-                    }
+                    for (int k = 1; k < BK / 16; ++k)
+                        mma_ss_pair(d, ad + 2 * k, wd + 2 * k, idesc, 1u);
                     mma_commit_pair(&empty[stage], 0x3);
                     if (++stage == STAGES) {
                         stage = 0;
