@@ -67,12 +67,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
-// Barrier `id` (1..15) among `count` threads (whole warps) of the block.
-__device__ __forceinline__ void named_barrier_sync(int id, int count)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // Non-blocking test of the phase with the given parity.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
 {
