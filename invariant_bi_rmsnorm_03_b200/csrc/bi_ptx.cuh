@@ -135,10 +135,12 @@ static __device__ __noinline__ bool wait(uint64_t *bar, uint32_t parity, const W
     return wait_inl(bar, parity, ctl);
 }
 
-// For a thread whose waits pace a pipeline (the one that issues the MMAs):
-// polls the phase a bounded number of times first, since a suspended
-// thread resumes some hundred cycles after the phase completes, then waits
-// as `wait` does.
+// For waits that pace a pipeline (the matmul's producer and MMA threads,
+// the attention backward's whole-block waits on its products): polls the
+// phase a bounded number of times first, since a suspended thread resumes
+// some hundred cycles after the phase completes, then waits as `wait` does.
+// Polling takes issue slots, so warps that share their sub-partitions with
+// busy ones keep the sleeping `wait`.
 __device__ __forceinline__ bool wait_spin(uint64_t *bar, uint32_t parity, const WaitCtl &ctl)
 {
     for (int i = 0; i < 2048; ++i)
