@@ -503,8 +503,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
+    // The item of this block's r-th round: items are ordered longest first
+    // and dealt to the blocks in a snake (round r even: block b takes item
+    // r G + b; odd: r G + G - 1 - b), so that every block's total is close to
+    // the mean instead of block 0 taking the longest item of every round.
+    // Every role walks the same sequence.
+    const auto item_of = [&](int rnd) {
+        const int G = int(gridDim.x), b = int(blockIdx.x);
+        return rnd * G + ((rnd & 1) ? G - 1 - b : b);
+    };
 
-    // The block serves work items blockIdx.x, blockIdx.x + gridDim.x, ...
+    // The block serves work items item_of(0), item_of(1), ...
     // (longest first).  Every role walks the same items and counts the
     // splits it has seen (gs): split number gs uses TMEM buffer gs & 1 with
     // barrier parity (gs >> 1) & 1, and its loads are numbers 2 gs, 2 gs + 1
@@ -520,7 +529,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t armed = 0, armed_parity = 0;
             int gs = 0, nq = 0;
             int64_t li = 0;  // running load number: slot li % NSLOT
-            for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
+            for (int rnd = 0, idx = item_of(0); ok && idx < p.items; idx = item_of(++rnd)) {
                 Item it;
                 if (!make_item(p, idx, it)) continue;
                 const int32_t *bt_row = p.block_table + int64_t(it.b) * p.max_pages;
@@ -651,7 +660,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t q_base = smem_u32(sQ);
                 bool ok = true;
                 int gs = 0, nq = 0;
-                for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
+                for (int rnd = 0, idx = item_of(0); ok && idx < p.items; idx = item_of(++rnd)) {
                     Item it;
                     if (!make_item(p, idx, it)) continue;
                     const int n = it.s1 - it.s0;
@@ -738,7 +747,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int q = warp & 3;
         int gs = 0;
         bool ok = true;
-        for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
+        for (int rnd = 0, idx = item_of(0); ok && idx < p.items; idx = item_of(++rnd)) {
             Item it;
             if (!make_item(p, idx, it)) continue;
             // whether lane quarter q holds any row of the item
@@ -809,7 +818,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         };
         int gs = 0;
         bool ok = true;
-        for (int idx = blockIdx.x; ok && idx < p.items; idx += gridDim.x) {
+        for (int rnd = 0, idx = item_of(0); ok && idx < p.items; idx = item_of(++rnd)) {
             Item it;
             if (!make_item(p, idx, it)) continue;
             bool valid, active;
