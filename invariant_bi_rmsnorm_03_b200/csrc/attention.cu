@@ -1101,8 +1101,8 @@ cudaError_t check_register_split()
 cudaError_t launch_attention(const CUtensorMap &tq, const AttnParams &p_in, int head_dim,
                              cudaStream_t s)
 {
-    // Prefill: persistent, one block per SM (at most), each walking items
-    // blockIdx.x, blockIdx.x + gridDim.x, ... (longest first; the tiles'
+    // Prefill: persistent, one block per SM (at most), each walking its
+    // items in the snake order of item_of (longest first; the tiles'
     // lengths fall in steps, so the static assignment stays balanced, and a
     // block's next item overlaps the current one's tail).  Decode: one block
     // per item -- request lengths vary too much for a static assignment, and
