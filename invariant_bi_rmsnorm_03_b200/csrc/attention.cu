@@ -100,6 +100,8 @@ struct Cfg {
     static constexpr int BAR_BYTES = 256;
     static constexpr int SLACK = 768;                  // alignment slack of the base
     static constexpr int SMEM = SLACK + ML_BYTES + Q_BYTES + NSLOT * KV_BYTES + BAR_BYTES;
+    // shared addresses fit the 14-bit field (16-byte units) of a matrix descriptor
+    static_assert(SMEM + 4096 <= (1 << 18), "descriptor address field");
     // TMEM: two buffers of 256 columns.  In buffer b: S over all 256
     // columns; P (bf16 pairs) written over its first 128; O_s in the next D.
     static constexpr uint32_t BUF_COLS = 256, P_OFF = 0, O_OFF = 128, TMEM_COLS = 512;
@@ -658,6 +660,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t idesc_qk = idesc_bf16_f32(128, kSplit, 0, 0);
                 const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
                 const uint32_t q_base = smem_u32(sQ);
+                const uint64_t q_desc0 = sdesc_sw128(q_base, 16, 1024);
                 bool ok = true;
                 int gs = 0, nq = 0;
                 for (int rnd = 0, idx = item_of(0); ok && idx < p.items; idx = item_of(++rnd)) {
@@ -680,15 +683,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                         tc_fence_after();
                         const uint32_t d = tmem + C::BUF_COLS * uint32_t(g & 1);
                         const uint32_t k_base = smem_u32(sKV + slot * C::KV_BYTES);
+                        // K: K-major, core matrices; 16 values of the head
+                        // dim are two core matrices 128 bytes apart, 8-key
+                        // groups KGROUP_BYTES apart (also across pages).
+                        // Descriptors by offset (16-byte units) from the
+                        // step-0 ones: shared addresses stay below 2^18, so
+                        // no sum carries out of the address field.
+                        const uint64_t kd0 = sdesc_plain(k_base, 128, C::KGROUP_BYTES);
     #pragma unroll
                         for (int k = 0; k < D / 16; ++k) {
                             const uint32_t kb = k >> 2, kk = k & 3;
-                            // K: K-major, core matrices; 16 values of the head
-                            // dim are two core matrices 128 bytes apart, 8-key
-                            // groups KGROUP_BYTES apart (also across pages).
-                            mma_ss(d, sdesc_sw128(q_base + kb * C::Q_KB_BYTES + kk * 32, 16, 1024),
-                                   sdesc_plain(k_base + k * 256, 128, C::KGROUP_BYTES), idesc_qk,
-                                   k > 0 ? 1u : 0u);
+                            mma_ss(d, q_desc0 + (kb * C::Q_KB_BYTES + kk * 32) / 16, kd0 + 16 * k,
+                                   idesc_qk, k > 0 ? 1u : 0u);
                         }
                         mma_commit(&barS[g & 1]);
                         mma_commit(&empty[slot]);
@@ -716,15 +722,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                             break;
                         }
                         tc_fence_after();
+                        // V: MN-major, core matrices; step jj is page jj;
+                        // its two 8-key groups are KGROUP_BYTES apart, 8-value
+                        // blocks of the head dim 128 bytes apart.
+                        const uint64_t vd0 = sdesc_plain(v_base, C::KGROUP_BYTES, 128);
     #pragma unroll
-                        for (int jj = 0; jj < kSplit / 16; ++jj) {
-                            // V: MN-major, core matrices; step jj is page jj;
-                            // its two 8-key groups are KGROUP_BYTES apart,
-                            // 8-value blocks of the head dim 128 bytes apart.
+                        for (int jj = 0; jj < kSplit / 16; ++jj)
                             mma_ts(buf + C::O_OFF, buf + C::P_OFF + 8 * jj,
-                                   sdesc_plain(v_base + jj * C::PAGE_BYTES, C::KGROUP_BYTES, 128),
-                                   idesc_pv, jj > 0 ? 1u : 0u);
-                        }
+                                   vd0 + uint64_t(jj) * (C::PAGE_BYTES / 16), idesc_pv, jj > 0 ? 1u : 0u);
                         mma_commit(&barO[b]);
                         mma_commit(&empty[slot]);
                         if (j + 2 < n) ok = issue_qk(j + 2);
