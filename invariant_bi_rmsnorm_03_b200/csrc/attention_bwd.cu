@@ -79,6 +79,9 @@ struct BwdCfg {
     // two buffers of what streams (q and dO tiles in the dk/dv kernel, key
     // blocks in the dq kernel), one of what stays
     static constexpr int SMEM = SLACK + 4 * TILE_BYTES + 2 * BLOCK_BYTES + 2 * VEC_BYTES + 64;
+    // shared addresses fit the 14-bit field (16-byte units) of a matrix
+    // descriptor, so descriptors are formed by adding offsets to one
+    static_assert(SMEM + 4096 <= (1 << 18), "descriptor address field");
     static_assert(4 * TILE_BYTES + 2 * BLOCK_BYTES == 2 * TILE_BYTES + 4 * BLOCK_BYTES,
                   "both kernels fit the same shared-memory size");
     // TMEM columns: S (128), dP (128), two d-wide accumulators (dV, dK) or one (dQ)
@@ -299,6 +302,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
     const uint32_t idesc_s = idesc_bf16_f32(128, kQTile, 0, 0);
     const uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
     const uint32_t kb_addr = smem_u32(sK), vb_addr = smem_u32(sV);
+    const uint64_t kd0 = sdesc_plain(kb_addr, 128, C::KGROUP_BYTES);  // K, V: K-major
+    const uint64_t vd0 = sdesc_plain(vb_addr, 128, C::KGROUP_BYTES);
     uint32_t phase = 0;
     bool ok = true, first = true;
     int buf = 0;
@@ -334,15 +339,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
         // ------------------------------------------------ S^T, dP^T
         if (threadIdx.x == 0) {
             tc_fence_after();
+            // descriptors by offset (16-byte units) from the step-0 ones
+            const uint64_t qd = sdesc_sw128(q_addr, 16, 1024), dd = sdesc_sw128(do_addr, 16, 1024);
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 // q and dO as K-major operands: 16 values = 32 bytes of a
                 // swizzled 128-byte row, 64-value boxes BOX_BYTES apart
-                const uint32_t koff = (k >> 2) * C::BOX_BYTES + (k & 3) * 32;
-                mma_ss(tmem + C::S_COL, sdesc_plain(kb_addr + 256 * k, 128, C::KGROUP_BYTES),
-                       sdesc_sw128(q_addr + koff, 16, 1024), idesc_s, k > 0 ? 1u : 0u);
-                mma_ss(tmem + C::DP_COL, sdesc_plain(vb_addr + 256 * k, 128, C::KGROUP_BYTES),
-                       sdesc_sw128(do_addr + koff, 16, 1024), idesc_s, k > 0 ? 1u : 0u);
+                const uint32_t koff = ((k >> 2) * C::BOX_BYTES + (k & 3) * 32) / 16;
+                mma_ss(tmem + C::S_COL, kd0 + 16 * k, qd + koff, idesc_s, k > 0 ? 1u : 0u);
+                mma_ss(tmem + C::DP_COL, vd0 + 16 * k, dd + koff, idesc_s, k > 0 ? 1u : 0u);
             }
             mma_commit(bar);
         }
@@ -387,16 +392,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
         // ------------------------------------------------ dV += P^T dO, dK += dS^T Q
         if (threadIdx.x == 0) {
             tc_fence_after();
+            const uint64_t dd = sdesc_sw128(do_addr, C::BOX_BYTES, 1024);
+            const uint64_t qd = sdesc_sw128(q_addr, C::BOX_BYTES, 1024);
 #pragma unroll
             for (int jj = 0; jj < kQTile / 16; ++jj) {
                 const uint32_t acc = (first && jj == 0) ? 0u : 1u;
                 // dO and q as MN-major operands (N = head dim): 16 rows =
                 // 2048 bytes per K step, 8-row groups 1024 bytes apart,
                 // 64-value boxes BOX_BYTES apart along N
-                mma_ts(tmem + C::ACC0, tmem + C::S_COL + packed_step_col(jj),
-                       sdesc_sw128(do_addr + 2048 * jj, C::BOX_BYTES, 1024), idesc_acc, acc);
-                mma_ts(tmem + C::ACC1, tmem + C::DP_COL + packed_step_col(jj),
-                       sdesc_sw128(q_addr + 2048 * jj, C::BOX_BYTES, 1024), idesc_acc, acc);
+                mma_ts(tmem + C::ACC0, tmem + C::S_COL + packed_step_col(jj), dd + 128 * jj, idesc_acc,
+                       acc);
+                mma_ts(tmem + C::ACC1, tmem + C::DP_COL + packed_step_col(jj), qd + 128 * jj, idesc_acc,
+                       acc);
             }
             mma_commit(bar);
         }
@@ -587,6 +594,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
     const uint32_t idesc_s = idesc_bf16_f32(128, kKeyBlock, 0, 0);
     const uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
     const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
+    const uint64_t qd0 = sdesc_sw128(q_addr, 16, 1024);  // q, dO: K-major, swizzled
+    const uint64_t dd0 = sdesc_sw128(do_addr, 16, 1024);
     uint32_t phase = 0;
     bool ok = true;
     const int last_key = pos0 + rows - 1;  // the tile's last visible key
@@ -629,13 +638,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
         __syncthreads();
         if (threadIdx.x == 0) {
             tc_fence_after();
+            // descriptors by offset (16-byte units) from the step-0 ones
+            const uint64_t kd = sdesc_plain(kb_addr, 128, C::KGROUP_BYTES);
+            const uint64_t vd = sdesc_plain(vb_addr, 128, C::KGROUP_BYTES);
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
-                const uint32_t koff = (k >> 2) * C::BOX_BYTES + (k & 3) * 32;  // K-major, swizzled
-                mma_ss(tmem + C::S_COL, sdesc_sw128(q_addr + koff, 16, 1024),
-                       sdesc_plain(kb_addr + 256 * k, 128, C::KGROUP_BYTES), idesc_s, k > 0 ? 1u : 0u);
-                mma_ss(tmem + C::DP_COL, sdesc_sw128(do_addr + koff, 16, 1024),
-                       sdesc_plain(vb_addr + 256 * k, 128, C::KGROUP_BYTES), idesc_s, k > 0 ? 1u : 0u);
+                const uint32_t koff = ((k >> 2) * C::BOX_BYTES + (k & 3) * 32) / 16;  // K-major, swizzled
+                mma_ss(tmem + C::S_COL, qd0 + koff, kd + 16 * k, idesc_s, k > 0 ? 1u : 0u);
+                mma_ss(tmem + C::DP_COL, dd0 + koff, vd + 16 * k, idesc_s, k > 0 ? 1u : 0u);
             }
             mma_commit(bar);
         }
@@ -676,11 +686,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
         // ---------------------------------------------------- dQ += dS K
         if (threadIdx.x == 0) {
             tc_fence_after();
+            const uint64_t kd = sdesc_plain(kb_addr, C::KGROUP_BYTES, 128);
 #pragma unroll
             for (int jj = 0; jj < kKeyBlock / 16; ++jj)
                 mma_ts(tmem + C::ACC0, tmem + C::S_COL + packed_step_col(jj),
-                       sdesc_plain(kb_addr + jj * C::PAGE_BYTES, C::KGROUP_BYTES, 128), idesc_acc,
-                       (kb > 0 || jj > 0) ? 1u : 0u);
+                       kd + uint64_t(jj) * (C::PAGE_BYTES / 16), idesc_acc, (kb > 0 || jj > 0) ? 1u : 0u);
             mma_commit(bar);
         }
         ok = block_wait(bar, phase, ctl);
