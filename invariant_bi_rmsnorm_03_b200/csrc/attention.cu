@@ -1003,15 +1003,33 @@ __global__ void __launch_bounds__(1024) attn_order_kernel(const int32_t *__restr
     for (int b = tid; b < B; b += 1024) order[atomicAdd(&cnt[bucket(seq_lens[b])], 1)] = b;
 }
 
-// Continues the merge of a decode row past the first block's range, split by
-// split in ascending order; one warp per (sequence, query head).
-template <int D>
-__global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p)
+// Continues the merge of a decode row past the first block's range, record
+// by record in ascending order; one block per (sequence, query head).  The
+// row's records (the first block's state, then one per later split) lie
+// contiguously in the workspace; warps 1-3 copy them into shared memory,
+// CH records at a time and the next chunk while warp 0 merges the current
+// one, so the sequential merge reads shared memory instead of waiting on a
+// memory latency every few records.  Warp 0 does exactly the merges of the
+// one-warp form, in the same order, with the same functions, so CH (chosen
+// from the number of rows) never changes a bit.
+constexpr int kCombineThreads = 128;
+
+template <int D, int CH>
+constexpr size_t combine_smem_bytes()
+{
+    return size_t(2) * CH * Cfg<D>::REC * sizeof(float);
+}
+
+template <int D, int CH>
+__global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(const AttnParams p)
 {
     using C = Cfg<D>;
-    constexpr int PER = D / 32;  // columns per lane
-    const int64_t row = int64_t(blockIdx.x) * 4 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
+    constexpr int PER = D / 32;  // columns per lane of warp 0
+    static_assert(C::REC % 4 == 0, "records of whole 16-byte pieces");
+    extern __shared__ float4 s_rec4[];  // [2][CH * REC]
+    float *s_rec = reinterpret_cast<float *>(s_rec4);
+    const int64_t row = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (row >= int64_t(p.B) * p.Hq) return;
     const int b = static_cast<int>(row / p.Hq);
     const int L = p.seq_lens[b];
@@ -1021,52 +1039,61 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p)
     if (L <= 0 || n > p.max_splits) return;
     const int first_end = decode_chunk(p, n);  // splits merged by the first block
     if (n <= first_end) return;
-    const float *rec = base + int64_t(first_end - 1) * C::REC;
+    const int rec0 = first_end, count = n - first_end;  // records split by split
 #else
     // variant-off: one record per block of keys x R .. (x + 1) R - 1
     const int nblk = decode_blocks(p);
     if (L <= 0 || n > p.max_splits) return;
     const int R = variant_range(L, nblk);
     if (R >= L) return;  // one block: its output is written
-    const float *rec = base;
-#endif
-#if BI_INVARIANT
-    const int rec0 = first_end, count = n - first_end;  // records split by split
-#else
     const int rec0 = 1, count = (L + R - 1) / R - 1;    // records block by block
 #endif
-    float m = __ldg(rec), l = __ldg(rec + 1);
-    float O[PER];
+    // records rec0 - 1 (the state to continue from) .. rec0 + count - 1
+    const float4 *src = reinterpret_cast<const float4 *>(base + int64_t(rec0 - 1) * C::REC);
+    const int total = count + 1;
+    const int nchunk = (total + CH - 1) / CH;
+    auto copy_chunk = [&](int c, int t, int nt) {
+        const int n4 = min(CH, total - c * CH) * (C::REC / 4);
+        const float4 *g = src + int64_t(c) * CH * (C::REC / 4);
+        float4 *d = s_rec4 + (c & 1) * CH * (C::REC / 4);
+        for (int i = t; i < n4; i += nt) d[i] = __ldg(g + i);
+    };
+    copy_chunk(0, threadIdx.x, kCombineThreads);
+    __syncthreads();
+    float m = 0.0f, l = 0.0f, O[PER];
 #pragma unroll
-    for (int j = 0; j < PER; ++j) O[j] = __ldg(rec + 4 + lane * PER + j);
-    // The records are folded one after another in ascending order; their
-    // loads are issued AHEAD at a time, ahead of the merges that use them,
-    // so that a long sequence does not pay one memory latency per split.
-    constexpr int AHEAD = 16;
-    for (int i0 = 0; i0 < count; i0 += AHEAD) {
-        float rm[AHEAD], rl[AHEAD], ro[AHEAD][PER];
+    for (int j = 0; j < PER; ++j) O[j] = 0.0f;
+    for (int c = 0; c < nchunk; ++c) {
+        if (warp > 0) {
+            if (c + 1 < nchunk) copy_chunk(c + 1, threadIdx.x - 32, kCombineThreads - 32);
+        } else {
+            const float *buf = s_rec + (c & 1) * CH * C::REC;
+            const int nr = min(CH, total - c * CH);
+            int i = 0;
+            if (c == 0) {
+                m = buf[0];
+                l = buf[1];
 #pragma unroll
-        for (int i = 0; i < AHEAD; ++i) {
-            if (i0 + i < count) {
-                const float *r = base + int64_t(rec0 + i0 + i) * C::REC;
-                rm[i] = __ldg(r);
-                rl[i] = __ldg(r + 1);
-#pragma unroll
-                for (int j = 0; j < PER; ++j) ro[i][j] = __ldg(r + 4 + lane * PER + j);
+                for (int j = 0; j < PER; ++j) O[j] = buf[4 + lane * PER + j];
+                i = 1;
             }
-        }
+#pragma unroll 4
+            for (; i < nr; ++i) {
+                const float *r = buf + i * C::REC;
+                float ro[PER];
 #pragma unroll
-        for (int i = 0; i < AHEAD; ++i) {
-            if (i0 + i < count) {
+                for (int j = 0; j < PER; ++j) ro[j] = r[4 + lane * PER + j];
                 float mn, a, cc;
-                merge_scales(m, rm[i], mn, a, cc);
+                merge_scales(m, r[0], mn, a, cc);
 #pragma unroll
-                for (int j = 0; j < PER; ++j) O[j] = merge_val(O[j], a, ro[i][j], cc);
-                l = merge_val(l, a, rl[i], cc);
+                for (int j = 0; j < PER; ++j) O[j] = merge_val(O[j], a, ro[j], cc);
+                l = merge_val(l, a, r[1], cc);
                 m = mn;
             }
         }
+        __syncthreads();  // chunk c is merged and chunk c + 1 has landed
     }
+    if (warp != 0) return;
     __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.o) + row * D + lane * PER;
 #pragma unroll
     for (int j = 0; j < PER; j += 2)
@@ -1156,15 +1183,28 @@ cudaError_t launch_attn_order(const int32_t *seq_lens, int B, int32_t *order, cu
     return cudaGetLastError();
 }
 
+template <int D, int CH>
+static cudaError_t launch_combine(const AttnParams &p, unsigned blocks, cudaStream_t s)
+{
+    constexpr size_t smem = combine_smem_bytes<D, CH>();
+    const cudaError_t e = cudaFuncSetAttribute(attn_combine_kernel<D, CH>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    attn_combine_kernel<D, CH><<<blocks, kCombineThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_attn_combine(const AttnParams &p, int head_dim, cudaStream_t s)
 {
     const int64_t rows = int64_t(p.B) * p.Hq;
-    const unsigned blocks = static_cast<unsigned>((rows + 3) / 4);
+    if (rows > INT32_MAX) return cudaErrorInvalidValue;
+    const unsigned blocks = static_cast<unsigned>(rows);
+    // few rows: long chunks (fewer copy rounds per row); many rows: short
+    // ones (more blocks resident per SM); measured crossover ~500 rows
+    const bool few = rows <= 512;
     if (head_dim == 128)
-        attn_combine_kernel<128><<<blocks, 128, 0, s>>>(p);
-    else
-        attn_combine_kernel<64><<<blocks, 128, 0, s>>>(p);
-    return cudaGetLastError();
+        return few ? launch_combine<128, 64>(p, blocks, s) : launch_combine<128, 32>(p, blocks, s);
+    return few ? launch_combine<64, 64>(p, blocks, s) : launch_combine<64, 32>(p, blocks, s);
 }
 
 }  // namespace bi
