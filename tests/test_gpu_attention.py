@@ -360,3 +360,24 @@ def test_repeat_runs_are_identical(L):
     for _ in range(100):
         assert same_bytes(L.bi_attention_decode(dkv, q, sl, 5000), ref)
         assert same_bytes(L.bi_attention_prefill(pkv, qp, i32([0, S]), i32([0]), S), refp)
+
+
+def test_decode_long_sequence_merged_in_many_chunks(L):
+    """A 70 001-key request has 274 split records per row: the ordered merge
+    runs through several staged chunks, of 64 records when the batch has at
+    most 512 rows and of 32 beyond.  Against the oracle alone, and the same
+    bits alone and amid eleven other requests (768 rows)."""
+    g = rng(31)
+    lens = [70001] + [int(x) for x in g.integers(1, 6000, 11)]
+    kv = paged_kv(g, lens, 4, 128)
+    q = normal_bf16(g, (len(lens), 64, 128))
+    one = PagedKV(kv.k_cache, kv.v_cache, kv.block_table[:1], kv.seq_lens[:1], 4, 128)
+    alone, alone_l = decode_parity(L, one, q[:1])
+    o, lse = L.bi_attention_decode(dev_kv(kv), dev_bf16(q), i32(kv.seq_lens), 70001, want_lse=True)
+    assert same_bytes(o[0], alone[0])
+    assert same_bytes(lse[0], alone_l[0])
+    # and a work division that leaves every block one split
+    o1, l1 = L.bi_attention_decode(dev_kv(kv), dev_bf16(q), i32(kv.seq_lens), 70001, want_lse=True,
+                                   splits_per_cta=1)
+    assert same_bytes(o1, o) and same_bytes(l1, lse)
+    assert L.bi_device_status() == bi.Status.OK
