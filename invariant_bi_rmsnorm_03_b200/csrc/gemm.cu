@@ -350,6 +350,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
 
     if (threadIdx.x == 0) {
+        // the producer's first loads will need both descriptors
+        tma_prefetch_desc(&tma);
+        tma_prefetch_desc(&tmw);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
