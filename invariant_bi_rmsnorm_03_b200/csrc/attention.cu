@@ -863,9 +863,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const float m_s = sML[(b * 128 + row_id) * 2 + 0];
                 const float l_s = sML[(b * 128 + row_id) * 2 + 1];
                 if (active) {
-                    // 16-column TMEM loads (HW / 16 per split; one load's
-                    // registers at a time beside O, within the 96 a
-                    // thread of this block has)
+                    // 16-column TMEM loads (HW / 16 per split): one at a
+                    // time when a partial is written out, the next one in
+                    // flight while the current one merges
                     constexpr int NCH16 = HW / 16;
                     if (spill) {
                         // not the first block of this sequence: write the
@@ -894,11 +894,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                         const bool take = k0 <= t;  // the row sees at least key k0
                         float mn, a, cc;
                         merge_scales(m, m_s, mn, a, cc);
+                        // the next 16 columns load while these merge
+                        uint32_t r2[2][16];
+                        tmem_ld32x16(ob, r2[0]);
 #pragma unroll
                         for (int c = 0; c < NCH16; ++c) {
-                            uint32_t r[16];
-                            tmem_ld32x16(ob + 16 * c, r);
+                            uint32_t(&r)[16] = r2[c & 1];
                             tmem_wait_ld16(r);
+                            if (c + 1 < NCH16) tmem_ld32x16(ob + 16 * (c + 1), r2[(c + 1) & 1]);
                             if (c == NCH16 - 1) {  // O_s read: the buffer is free
                                 tc_fence_before();
                                 mbar_arrive(&barF[b]);
