@@ -1122,15 +1122,15 @@ size_t attn_ws_bytes(int B, int Hq, int head_dim, int max_splits, int max_chunks
 template <int D>
 cudaError_t check_register_split()
 {
-    static int verdict = 0;  // 0 not yet checked, 1 fits, -1 does not
-    if (verdict == 0) {
+    static int split_fits = 0;  // 0 not yet checked, 1 fits, -1 does not
+    if (split_fits == 0) {
         cudaFuncAttributes a;
         const cudaError_t e = cudaFuncGetAttributes(&a, attn_split_kernel<D>);
         if (e != cudaSuccess) return e;
         const long r = a.numRegs;
-        verdict = (128L * (kRegsCtl + 2 * r + 2 * kRegsFold) <= long(THREADS) * r) ? 1 : -1;
+        split_fits = (128L * (kRegsCtl + 2 * r + 2 * kRegsFold) <= long(THREADS) * r) ? 1 : -1;
     }
-    return verdict > 0 ? cudaSuccess : cudaErrorInvalidConfiguration;
+    return split_fits > 0 ? cudaSuccess : cudaErrorInvalidConfiguration;
 }
 
 cudaError_t launch_attention(const CUtensorMap &tq, const AttnParams &p_in, int head_dim,
